@@ -1,0 +1,61 @@
+"""Helpers shared by the tests: marshal a generated workload into the numpy
+arrays the oracle takes, and compare results.  No step arithmetic here."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from paged_kv_flight_b200.workloads import Workload
+
+
+def bits16(t: torch.Tensor) -> np.ndarray:
+    """bf16 tensor -> uint16 bit patterns (host copy)."""
+    return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16).copy()
+
+
+def bytes8(t: torch.Tensor) -> np.ndarray:
+    return t.detach().contiguous().cpu().numpy().view(np.uint8).copy()
+
+
+def pool_np(w: Workload, t: torch.Tensor) -> np.ndarray:
+    return bytes8(t) if w.kv_fp8 else bits16(t)
+
+
+def oracle_cfg(w: Workload) -> oracle.OracleConfig:
+    return oracle.OracleConfig(w.Hq, w.Hkv, w.d, w.P, w.kv_fp8, w.num_pages, w.rope_base)
+
+
+def host_inputs(w: Workload) -> dict:
+    """Fresh host copies of every input of the step, in oracle form."""
+    return dict(
+        q=bits16(w.q), k_new=bits16(w.k_new), v_new=bits16(w.v_new),
+        k_pool=pool_np(w, w.k_pool), v_pool=pool_np(w, w.v_pool),
+        k_scale=None if w.k_scale is None else w.k_scale.detach().cpu().numpy().copy(),
+        v_scale=None if w.v_scale is None else w.v_scale.detach().cpu().numpy().copy(),
+        block_tables=np.ascontiguousarray(w.block_tables, np.int32),
+        seq_lens=np.ascontiguousarray(w.seq_lens, np.int32),
+    )
+
+
+def oracle_step(w: Workload, h: dict | None = None):
+    """Run the oracle's append + attention on host copies; returns (h, out, st)."""
+    h = host_inputs(w) if h is None else h
+    cfg = oracle_cfg(w)
+    st1 = oracle.rope_append(cfg, h["q"], h["k_new"], h["v_new"], h["k_pool"], h["v_pool"],
+                             h["k_scale"], h["v_scale"], h["block_tables"], h["seq_lens"])
+    out, st2 = oracle.decode_attn(cfg, h["q"], h["k_pool"], h["v_pool"], h["k_scale"],
+                                  h["v_scale"], h["block_tables"], h["seq_lens"])
+    return h, out, max(st1, st2)
+
+
+def bf16_ordinal(bits: np.ndarray) -> np.ndarray:
+    """Monotone integer image of bf16 bit patterns (sign-magnitude -> ordinal),
+    so that |ordinal(a) - ordinal(b)| counts representable steps."""
+    b = bits.astype(np.int64)
+    mag = b & 0x7FFF
+    return np.where(b & 0x8000, -mag, mag)
+
+
+def f64_of_bf16_tensor(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)
