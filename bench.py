@@ -1,0 +1,515 @@
+#!/usr/bin/env python
+"""Benchmark: one in-flight-batched decode step over a paged KV cache
+(RoPE + append, then split-KV GQA decode attention), through the libpkv C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME|all]
+                    [--impl ours|reference]
+
+One step = pkv_rope_append + pkv_decode_attn over the whole batch of the
+workload.  Inputs are resident in HBM; L2 is flushed (memset of 2x the L2
+size) before every timed step, outside the CUDA-event window.  The value is
+whole-job HBM throughput: resident KV bytes attended plus q / out bytes, per
+step, summed over ranks, divided by the max-over-ranks step time.  Under
+torchrun every rank runs an independent replica of the workload (weak
+scaling; the step has no exchange between GPUs).
+
+``--impl reference`` times the CPU oracle (plain fp64 C, one thread) on a
+bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "paged-KV decode attn: HBM GB/s (% of B200 peak), request-tokens/s, step µs"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+DEFAULT_CONFIG = "llama8b"
+ATTN_SOURCES = ("paged_kv_flight_b200/csrc/decode_attn.cu", "paged_kv_flight_b200/csrc/pkv_device.cuh",
+                "paged_kv_flight_b200/csrc/pkv_internal.h")
+
+
+# ---------------------------------------------------------------- accounting
+
+def metric_bytes(seq_lens, Hq, Hkv, d, P, kv_fp8) -> int:
+    """Resident KV attended (the new token included) + q read + out written
+    (+ the two fp32 scales per attended page and kv head for E4M3 pools)."""
+    n = np.asarray(seq_lens, np.int64) + 1
+    s = 1 if kv_fp8 else 2
+    kv = int((2 * Hkv * n * d * s).sum())
+    qo = 2 * len(n) * Hq * d * 2
+    sc = int(2 * ((n + P - 1) // P).sum() * Hkv * 4) if kv_fp8 else 0
+    return kv + qo + sc
+
+
+def workload_bytes(w) -> int:
+    return metric_bytes(w.seq_lens, w.Hq, w.Hkv, w.d, w.P, w.kv_fp8)
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def attn_source_sha() -> str:
+    h = hashlib.sha256()
+    for rel in ATTN_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per attention launch from a committed ncu summary, if it was
+    taken on the current attention sources; otherwise None."""
+    sha = attn_source_sha()
+    pat = re.compile(r"traffic-per-launch:\s+(\S+)\s+(\d+)\s+src=([0-9a-f]+)")
+    pdir = os.path.join(ROOT, "profiles")
+    if not os.path.isdir(pdir):
+        return None
+    for fn in sorted(os.listdir(pdir)):
+        if not fn.endswith((".md", ".txt")):
+            continue
+        with open(os.path.join(pdir, fn)) as f:
+            for m in pat.finditer(f.read()):
+                if m.group(1) == workload and m.group(3) == sha:
+                    return int(m.group(2))
+    return None
+
+
+# ---------------------------------------------------------------- ranks
+
+def dist_info():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(x: float) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return x
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return x
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+# ---------------------------------------------------------------- clocks
+
+_REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+            0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+            0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    """Polls the SM clock and the clock-event (throttle) reasons of this
+    process's GPU through NVML while the timed region runs."""
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.period = period_s
+        self.samples, self.reason_bits = [], 0
+        self.err = None
+        self.h = None
+        try:
+            import pynvml
+            import torch
+            self.nv = pynvml
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            for cand in (uuid, "GPU-" + uuid):
+                try:
+                    self.h = pynvml.nvmlDeviceGetHandleByUUID(cand)
+                    break
+                except Exception:
+                    continue
+            if self.h is None:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report that, keep running
+            self.err = f"{type(e).__name__}: {e}"
+        self._stop = threading.Event()
+        self._t = None
+
+    def _reasons(self):
+        f = getattr(self.nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            self.nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        return int(f(self.h))
+
+    def sample(self):
+        if self.h is None:
+            return
+        try:
+            self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+            self.reason_bits |= self._reasons()
+        except Exception as e:
+            self.err = f"{type(e).__name__}: {e}"
+
+    def _run(self):
+        while not self._stop.is_set():
+            self.sample()
+            time.sleep(self.period)
+
+    def start(self):
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+
+    def stop(self) -> dict:
+        self._stop.set()
+        if self._t:
+            self._t.join()
+        out = {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+               "sm_max_mhz": getattr(self, "max_mhz", None),
+               "reasons": [n for b, n in _REASONS.items() if self.reason_bits & b and b != 0x1],
+               "samples": len(self.samples), "source": "nvml, polled every 10 ms during the timed steps"}
+        if self.err:
+            out["error"] = self.err
+        return out
+
+
+# ---------------------------------------------------------------- oracle leg
+
+def _request_pages(w, b, src):
+    """Host copies (oracle form) of request b's pages, block table renumbered."""
+    import torch
+    L = int(w.seq_lens[b])
+    npg = (L + 1 + w.P - 1) // w.P
+    idx = torch.from_numpy(w.block_tables[b, :npg].astype(np.int64)).to(src["k_pool"].device)
+
+    def b16(t):
+        return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16).copy()
+
+    def u8(t):
+        return t.contiguous().cpu().numpy().copy()
+
+    conv = u8 if w.kv_fp8 else b16
+    return dict(
+        npg=npg,
+        q=b16(src["q"][b:b + 1]), k_new=b16(src["k_new"][b:b + 1]), v_new=b16(src["v_new"][b:b + 1]),
+        k_pool=conv(src["k_pool"].index_select(0, idx)), v_pool=conv(src["v_pool"].index_select(0, idx)),
+        k_scale=None if src["k_scale"] is None else src["k_scale"].index_select(0, idx).cpu().numpy().copy(),
+        v_scale=None if src["v_scale"] is None else src["v_scale"].index_select(0, idx).cpu().numpy().copy(),
+        block_tables=np.arange(npg, dtype=np.int32)[None, :].copy(),
+        seq_lens=np.array([L], np.int32))
+
+
+def oracle_step_requests(w, views):
+    """The oracle's whole step (append + attention) for the given requests."""
+    import oracle
+    for v in views:
+        cfg = oracle.OracleConfig(w.Hq, w.Hkv, w.d, w.P, w.kv_fp8, v["npg"], w.rope_base)
+        q = v["q"].copy()
+        kp, vp = v["k_pool"].copy(), v["v_pool"].copy()
+        oracle.rope_append(cfg, q, v["k_new"], v["v_new"], kp, vp, v["k_scale"], v["v_scale"],
+                           v["block_tables"], v["seq_lens"])
+        oracle.decode_attn(cfg, q, kp, vp, v["k_scale"], v["v_scale"], v["block_tables"], v["seq_lens"])
+
+
+def sample_requests(w, token_head_budget: int):
+    """Prefix of the batch whose attended token-heads stay within the budget
+    (at least one request)."""
+    picks, acc = [], 0
+    for b, L in enumerate(w.seq_lens):
+        th = (int(L) + 1) * w.Hkv
+        if picks and acc + th > token_head_budget:
+            break
+        picks.append(b)
+        acc += th
+    return picks
+
+
+def cpu_baseline(w, src, time_budget_s: float = 20.0) -> dict:
+    """Times the oracle as it stands on this host (one thread), request by
+    request in batch order until the time budget is spent."""
+    views, t_sum, done = [], 0.0, []
+    for b in range(w.batch):
+        v = _request_pages(w, b, src)
+        t0 = time.perf_counter()
+        oracle_step_requests(w, [v])
+        t_sum += time.perf_counter() - t0
+        done.append(b)
+        if t_sum >= time_budget_s:
+            break
+    by = metric_bytes(w.seq_lens[done], w.Hq, w.Hkv, w.d, w.P, w.kv_fp8)
+    toks = int((w.seq_lens[done].astype(np.int64) + 1).sum())
+    return {"value": by / t_sum / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "seconds": t_sum,
+            "sample": f"requests 0..{len(done) - 1} of {w.batch} ({toks} attended tokens, "
+                      f"{100.0 * by / workload_bytes(w):.1f}% of the step's bytes); plain fp64 C oracle, "
+                      f"single thread, append + attention"}
+
+
+# ---------------------------------------------------------------- GPU leg
+
+def _device_inputs(w, device):
+    import torch
+    return dict(q=w.q.to(device).contiguous(), k_new=w.k_new.to(device).contiguous(),
+                v_new=w.v_new.to(device).contiguous(), k_pool=w.k_pool.to(device).contiguous(),
+                v_pool=w.v_pool.to(device).contiguous(),
+                k_scale=None if w.k_scale is None else w.k_scale.to(device).contiguous(),
+                v_scale=None if w.v_scale is None else w.v_scale.to(device).contiguous(),
+                block_tables=torch.from_numpy(w.block_tables).to(device).contiguous(),
+                seq_lens=torch.from_numpy(w.seq_lens).to(device).contiguous())
+
+
+def run_ours(args, name, rank, world, local_rank):
+    import torch
+    from paged_kv_flight_b200 import pkv, workloads
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = workloads.make(name, device=dev, offset=rank)
+    dv = _device_inputs(w, dev)
+    B = w.batch
+    cfg = pkv.make_config(w.Hq, w.Hkv, w.d, w.P, "fp8" if w.kv_fp8 else "bf16", w.rope_base, B,
+                          w.bt_stride, w.num_pages)
+    ctx = pkv.pkv_create(cfg)
+    out = torch.empty(B, w.Hq, w.d, dtype=torch.bfloat16, device=dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, dv, args.cpu_budget)
+
+    def step():
+        pkv.pkv_rope_append(ctx, dv["q"], dv["k_new"], dv["v_new"], dv["k_pool"], dv["v_pool"],
+                            dv["k_scale"], dv["v_scale"], dv["block_tables"], dv["seq_lens"])
+        pkv.pkv_decode_attn(ctx, dv["q"], dv["k_pool"], dv["v_pool"], dv["k_scale"], dv["v_scale"],
+                            dv["block_tables"], dv["seq_lens"], out)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    st, bits = pkv.pkv_check_device_error(ctx)
+    if st != pkv.PKV_OK:
+        raise RuntimeError(f"device error during warm-up: {pkv.pkv_status_str(st)} bits={bits}")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    clocks = ClockSampler(local_rank)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    for k in range(K):
+        flush.zero_()                       # outside the event window
+        ev[k][0].record()
+        pkv.pkv_rope_append(ctx, dv["q"], dv["k_new"], dv["v_new"], dv["k_pool"], dv["v_pool"],
+                            dv["k_scale"], dv["v_scale"], dv["block_tables"], dv["seq_lens"])
+        ev[k][1].record()
+        pkv.pkv_decode_attn(ctx, dv["q"], dv["k_pool"], dv["v_pool"], dv["k_scale"], dv["v_scale"],
+                            dv["block_tables"], dv["seq_lens"], out)
+        ev[k][2].record()
+    clocks.sample()
+    torch.cuda.synchronize()
+    clock_info = clocks.stop()
+    barrier()
+    step_ms = [a.elapsed_time(c) for a, _, c in ev]
+    rope_ms = [a.elapsed_time(b) for a, b, _ in ev]
+    attn_ms = [b.elapsed_time(c) for _, b, c in ev]
+    st, bits = pkv.pkv_check_device_error(ctx)
+    if st != pkv.PKV_OK:
+        raise RuntimeError(f"device error during timing: {pkv.pkv_status_str(st)} bits={bits}")
+
+    my_step = sum(step_ms) / K
+    my_attn = sum(attn_ms) / K
+    step_max = max_over_ranks(my_step)
+    attn_max = max_over_ranks(my_attn)
+    by = workload_bytes(w)
+    total_bytes = sum_over_ranks(float(by))
+    total_reqs = sum_over_ranks(float(B))
+
+    # unflushed ("hot L2") median, labelled as such
+    hot = []
+    for _ in range(min(K, 50)):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        step()
+        b.record()
+        hot.append((a, b))
+    torch.cuda.synchronize()
+    hot_ms = statistics.median(x.elapsed_time(y) for x, y in hot)
+
+    # end to end through the public API: pinned host inputs in, result out, every step
+    e2e = None
+    if not args.no_e2e:
+        host = {k: dv[k].cpu().pin_memory() for k in ("q", "k_new", "v_new", "block_tables", "seq_lens")}
+        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = out_h.numel() * out_h.element_size()
+        evs = []
+        for k in range(args.warmup + K):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            for key, t in host.items():
+                dv[key].copy_(t, non_blocking=True)
+            step()
+            out_h.copy_(out, non_blocking=True)
+            b.record()
+            if k >= args.warmup:
+                evs.append((a, b))
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / K)
+        e2e = {"value": total_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": e2e_ms,
+               "note": "pinned host q/k_new/v_new/block_tables/seq_lens copied in and out read back every "
+                       "step; the KV pools stay resident in HBM (the cache lives on the GPU)"}
+    pkv.pkv_destroy(ctx)
+
+    peak, peak_src = measured_peak()
+    value = total_bytes / (step_max * 1e-3) / 1e9
+    attn_gbs = by / (attn_max * 1e-3) / 1e9
+    traffic = recorded_traffic(name)
+    kernel = f"decode_attn_kernel<{w.d},{'e4m3' if w.kv_fp8 else 'bf16'}>"
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": step_max, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "e4m3-kv/bf16" if w.kv_fp8 else "bf16",
+        "data": "synthetic: seeded lengths, page permutation, block tables and N(0,1) q/k/v "
+                "(per-workload recipe in paged_kv_flight_b200/workloads.py)",
+        "config": {"workload": name, "description": workloads.DESCRIPTIONS[name], "batch": B,
+                   "tokens_attended": int((w.seq_lens.astype(np.int64) + 1).sum()),
+                   "metric_bytes_per_step": by, "l2": "flushed before every timed step (memset of 2x L2)",
+                   "replicas": world},
+        "request_tokens_per_s": total_reqs / (step_max * 1e-3),
+        "step_us": step_max * 1e3, "attn_us": attn_max * 1e3,
+        "rope_append_us": max_over_ranks(sum(rope_ms) / K) * 1e3,
+        "step_us_hot_l2": hot_ms * 1e3,
+        "pct_of_8TBs": 100.0 * value / world / NOMINAL_HBM_GBS,
+        "pct_of_measured_peak": 100.0 * value / world / peak,
+        "roofline": {"bound": "hbm", "achieved": attn_gbs, "peak": peak, "unit": "GB/s",
+                     "frac": attn_gbs / peak, "traffic": traffic, "kernel": kernel,
+                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
+                     else "fallback 6650 GB/s",
+                     "bytes_per_launch": by},
+        "e2e": e2e,
+        "gpu_launches": 2 * K,
+        "clocks": clock_info,
+        "when": datetime.datetime.utcnow().isoformat() + "Z",
+    }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    return line
+
+
+def run_reference(args, name):
+    """The CPU oracle as the reference arm, on a bounded sample per step."""
+    import torch
+    from paged_kv_flight_b200 import workloads
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    w = workloads.make(name, device=dev)
+    src = _device_inputs(w, dev)
+    picks = sample_requests(w, args.ref_budget)
+    views = [_request_pages(w, b, src) for b in picks]
+    by = metric_bytes(w.seq_lens[picks], w.Hq, w.Hkv, w.d, w.P, w.kv_fp8)
+    for _ in range(args.warmup):
+        oracle_step_requests(w, views)
+    ts = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle_step_requests(w, views)
+        ts.append(time.perf_counter() - t0)
+    sec = sum(ts) / len(ts)
+    value = by / sec / 1e9
+    toks = int((w.seq_lens[picks].astype(np.int64) + 1).sum())
+    sample = (f"requests 0..{len(picks) - 1} of {w.batch} ({toks} attended tokens, "
+              f"{100.0 * by / workload_bytes(w):.1f}% of the step's bytes) per step; plain fp64 C oracle, "
+              f"single thread, append + attention")
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic: same seeded workload as the GPU arm",
+        "config": {"workload": name, "description": workloads.DESCRIPTIONS[name], "batch": w.batch,
+                   "metric_bytes_per_step_sampled": by},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--config", default=DEFAULT_CONFIG)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--ref-budget", type=int, default=1_200_000,
+                    help="attended token-heads per reference step")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    from paged_kv_flight_b200 import workloads
+    names = list(workloads.CONFIG_NAMES) if args.config == "all" else [args.config]
+    rank, world, local_rank = dist_info()
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        for name in names:
+            print(json.dumps(run_reference(args, name)), flush=True)
+        return 0
+
+    import torch
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        for name in names:
+            line = run_ours(args, name, rank, world, local_rank)
+            if rank == 0:
+                print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

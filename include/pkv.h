@@ -1,0 +1,150 @@
+/*
+ * pkv.h -- libpkv, the C ABI of one in-flight-batched decode step over a
+ * paged KV cache on a B200 GPU (sm_100a).
+ *
+ * The step, for every request b of a batch of requests of different lengths
+ * ("Scaling TensorRT-LLM: Kernel Fusion and Inflight Batching in
+ * Production", section "Static vs. Dynamic vs. Inflight"):
+ *   1. rotary embedding of the new token's q (all query heads) and k at
+ *      position L_b = seq_lens[b] (same page, section "What Gets Fused",
+ *      RoPE bullet);
+ *   2. append of the rotated k and the raw v into slot L_b % P of physical
+ *      page block_tables[b][L_b / P] (same page, section "The Paged
+ *      KV-Cache"; "TensorRT-LLM Guide: High-Throughput GPU Inference
+ *      Engine", section "2. Paged KV Cache & Memory Virtualization");
+ *   3. grouped-query attention of the single new query over all n_b = L_b + 1
+ *      tokens of the request, each KV element read once for the G = Hq/Hkv
+ *      query heads that share it ("TensorRT-LLM Guide", section "3. Custom
+ *      Fused Attention Kernels: FMHA and XQA"), softmax kept on chip (first
+ *      page, section "What Gets Fused", Attention bullet).
+ * Optional E4M3 KV cache with one fp32 scale per (page, kv head)
+ * ("TensorRT-LLM Guide", section "4. Native FP8 Quantization on NVIDIA
+ * Hopper & Blackwell").
+ *
+ * Definitions used (the pages name the operations but give no formula):
+ *   RoPE: rotate-half pairs (i, i + d/2), theta_i = rope_base^(-2i/d),
+ *         x_i' = x_i cos(p theta_i) - x_{i+d/2} sin(p theta_i),
+ *         x_{i+d/2}' = x_{i+d/2} cos(p theta_i) + x_i sin(p theta_i);
+ *   attention: o_h = softmax(q_h K^T / sqrt(d)) V over the request's tokens
+ *         in logical order, K/V of kv head h / G (contiguous groups);
+ *   fp8 store: code = E4M3_RNE_satfinite(fl32(x / scale[page][kvh]));
+ *   fp8 load: value = code * scale[page][kvh].
+ *
+ * Layouts (all row-major, all caller-owned device memory):
+ *   q, out          [batch][Hq][d]        bf16
+ *   k_new, v_new    [batch][Hkv][d]       bf16
+ *   k_pool, v_pool  [num_pages][Hkv][P][d] bf16, or uint8 E4M3 codes
+ *   k_scale,v_scale [num_pages][Hkv]      fp32 (fp8 pools only; else NULL)
+ *   block_tables    [batch][bt_stride]    int32 physical page ids
+ *   seq_lens        [batch]               int32, L_b = tokens cached BEFORE
+ *                                         the step; the step attends L_b + 1
+ * Every pointer must be 16-byte aligned.
+ *
+ * Ownership and ordering: the library never allocates, frees or keeps caller
+ * tensors.  A context owns its workspace (split partials, per-(request, kv
+ * head) arrival counters, a device error word), allocated in pkv_create and
+ * freed in pkv_destroy; use one context from one stream at a time.  Calls are
+ * asynchronous and stream-ordered: they validate on the host, enqueue, and
+ * return.  pkv_rope_append writes q (in place) and exactly batch * Hkv slots
+ * of each pool; pkv_decode_attn writes only out.  The caller allocates the
+ * page the new token lands in before the step; block-table entries past
+ * ceil(n_b / P) are never read.
+ *
+ * Errors: host-side checks return PKV_ERR_INVALID_ARG / PKV_ERR_UNSUPPORTED
+ * and launch nothing.  A failed launch returns PKV_ERR_CUDA.  Range errors
+ * found on the device (a page id outside [0, num_pages), or L_b + 1 larger
+ * than bt_stride * P) skip the affected request or tile and set a sticky
+ * device error word, which pkv_check_device_error reads; no call traps.
+ * C++ exceptions never cross this ABI.
+ */
+#ifndef PKV_H
+#define PKV_H
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct pkv_ctx pkv_ctx;
+
+typedef enum {
+    PKV_OK = 0,
+    PKV_ERR_INVALID_ARG = 1,    /* NULL / misaligned pointer, bad size, bad config */
+    PKV_ERR_UNSUPPORTED = 2,    /* valid but not built: head_dim, page size, group size */
+    PKV_ERR_CUDA = 3,           /* a CUDA runtime call or launch failed */
+    PKV_ERR_OOM = 4,            /* workspace allocation failed */
+    PKV_ERR_DEVICE_BOUNDS = 5,  /* device saw a page id or length out of range */
+    PKV_ERR_DEVICE_TIMEOUT = 6  /* a bounded wait inside a kernel gave up */
+} pkv_status;
+
+typedef enum { PKV_KV_BF16 = 0, PKV_KV_FP8_E4M3 = 1 } pkv_kv_dtype;
+
+/* Shapes fixed at create time, like an engine built for one model and
+ * limits ("TensorRT-LLM", section "What the build step is for"). */
+typedef struct {
+    int num_q_heads;          /* Hq; a multiple of num_kv_heads */
+    int num_kv_heads;         /* Hkv; G = Hq / Hkv must be 1..8 */
+    int head_dim;             /* d: 64 or 128 */
+    int page_size;            /* P: 16, 32 or 64 tokens */
+    pkv_kv_dtype kv_dtype;    /* pool element type */
+    double rope_base;         /* > 1, e.g. 10000 or 500000 */
+    int max_batch;            /* largest batch a call may pass (<= 8192) */
+    int max_blocks_per_seq;   /* largest bt_stride a call may pass */
+    int num_pages;            /* physical pages in each pool */
+} pkv_config;
+
+/* Validates cfg, binds the context to the current CUDA device and allocates
+ * its workspace.  *out is set only on PKV_OK.  Validation happens before any
+ * CUDA call, so a bad cfg is reported without touching the device. */
+pkv_status pkv_create(const pkv_config* cfg, pkv_ctx** out);
+
+/* Step part 1 (RoPE + append).  Rotates q in place and k_new at position
+ * L_b, stores rotated k and raw v into slot L_b % P of page
+ * block_tables[b * bt_stride + L_b / P].  bf16 pools: k is rounded to bf16
+ * (nearest even) from the exact rotation, v copied bit for bit.  fp8 pools:
+ * the E4M3 store above with k_scale / v_scale of that page and kv head.
+ * batch == 0 is a no-op. */
+pkv_status pkv_rope_append(pkv_ctx* ctx, void* q, const void* k_new, const void* v_new,
+                           void* k_pool, void* v_pool,
+                           const float* k_scale, const float* v_scale,
+                           const int32_t* block_tables, int bt_stride,
+                           const int32_t* seq_lens, int batch, cudaStream_t stream);
+
+/* Step part 2 (decode attention).  q holds the rotated queries written by
+ * pkv_rope_append; seq_lens is the same L_b, and n_b = L_b + 1 tokens are
+ * attended (the new one included).  out[b][h][:] = bf16(o_h).  Work is split
+ * over all SMs by token ranges; partial results of a (request, kv head) cut
+ * between workers are merged by log-sum-exp in the same launch.
+ * batch == 0 is a no-op. */
+pkv_status pkv_decode_attn(pkv_ctx* ctx, const void* q, const void* k_pool, const void* v_pool,
+                           const float* k_scale, const float* v_scale,
+                           const int32_t* block_tables, int bt_stride,
+                           const int32_t* seq_lens, int batch, void* out,
+                           cudaStream_t stream);
+
+/* Frees the workspace.  NULL is accepted.  Synchronises the device. */
+pkv_status pkv_destroy(pkv_ctx* ctx);
+
+/* Static text for a status code. */
+const char* pkv_status_str(pkv_status s);
+
+/* Synchronises `stream`, reads and clears the context's device error word.
+ * Returns PKV_OK, PKV_ERR_DEVICE_BOUNDS or PKV_ERR_DEVICE_TIMEOUT; if
+ * `bits` is not NULL it receives the raw word (1: length out of range,
+ * 2: page id out of range, 4: wait timed out). */
+pkv_status pkv_check_device_error(pkv_ctx* ctx, cudaStream_t stream, int* bits);
+
+/* Caps the number of warp workers pkv_decode_attn splits the token ranges
+ * over (0 restores the automatic choice).  Results do not depend on it
+ * beyond rounding; tests use it to force 1, 2, 7, ... splits. */
+pkv_status pkv_set_workers(pkv_ctx* ctx, int workers);
+
+/* Bytes of device workspace the context holds. */
+size_t pkv_workspace_bytes(const pkv_ctx* ctx);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -1,0 +1,629 @@
+// decode_attn.cu -- step part 2: grouped-query decode attention of one new
+// query per request over its paged KV cache, split over all SMs.
+//
+// What it computes: o_h = softmax(q_h K^T / sqrt(d)) V over the request's
+// n_b = L_b + 1 tokens, K/V of kv head h / G.  Page lookup happens inside the
+// kernel ("Scaling TensorRT-LLM: Kernel Fusion and Inflight Batching in
+// Production", section "The Paged KV-Cache"); each KV element is read once
+// for all G query heads sharing it ("TensorRT-LLM Guide: High-Throughput GPU
+// Inference Engine", section "3. Custom Fused Attention Kernels: FMHA and
+// XQA"); scores and softmax never leave registers (first page, section "What
+// Gets Fused", Attention bullet).  E4M3 KV is dequantised in registers
+// ("TensorRT-LLM Guide", section "4. Native FP8 Quantization").
+//
+// Work decomposition (no host sync, one launch):
+//   * every CTA derives tiles-per-request (16 tokens per tile) from seq_lens
+//     and keeps their exclusive prefix in shared memory;
+//   * the flattened sequence of tiles, ordered (request, kv head, tile), is cut
+//     into W equal contiguous ranges, one per warp worker (W <= 8 warps x SMs),
+//     so every worker streams the same number of bytes whatever the length
+//     skew of the batch;
+//   * a (request, kv head) pair that lies inside one worker's range is
+//     finished by that worker; a pair cut between workers leaves one partial
+//     (unnormalised o, running max m, sum l) per worker, and the worker that
+//     arrives last at the pair's counter merges them by log-sum-exp.  Nobody
+//     ever waits for another worker.
+//
+// Per warp: a private ring of `stages` K+V tile buffers filled by 2-D TMA
+// tile loads (128-byte or 64-byte swizzle) that complete on one mbarrier per
+// stage; the warp's lane 0 issues the loads, the warp consumes: QK^T and P V
+// on warp-level mma.sync (query heads padded to 16 mma rows), online softmax
+// with quad shuffles, fp32 accumulators.  Every mbarrier wait is bounded in
+// time; a timeout marks the worker dead, sets a device error bit and lets
+// the control flow (and the combine protocol) run to the end without
+// touching data.
+#include <math.h>
+
+#include "pkv_internal.h"
+#include "pkv_device.cuh"
+
+namespace pkv {
+namespace {
+
+using namespace dev;
+
+constexpr uint64_t kWaitLimitNs = 500ull * 1000ull * 1000ull;  // 0.5 s per wait
+constexpr unsigned kFull = 0xFFFFFFFFu;
+
+template <int D, bool FP8>
+struct Geo {
+    static constexpr int ELEM = FP8 ? 1 : 2;
+    static constexpr int ROWB = D * ELEM;                  // bytes per token row
+    static constexpr int BOXB = ROWB > 128 ? 128 : ROWB;   // bytes per TMA box row
+    static constexpr int NBOX = ROWB / BOXB;               // boxes per tile per tensor
+    static constexpr int CPB = BOXB / 16;                  // 16-byte chunks per box row
+    static constexpr int BOX_BYTES = kTile * BOXB;
+    static constexpr int TILEB = kTile * ROWB;             // one K (or V) tile
+    static constexpr int STAGEB = 2 * TILEB;               // K + V
+};
+
+// Byte offset inside a tile of 16-byte chunk `ch` (counted along the token
+// row) of tile row `row`, as the TMA swizzle placed it.
+template <int D, bool FP8>
+__device__ __forceinline__ uint32_t tile_off(int row, int ch)
+{
+    using Gm = Geo<D, FP8>;
+    const int box = ch / Gm::CPB, cib = ch % Gm::CPB;
+    const int x = (Gm::BOXB == 128) ? (row & 7) : ((row >> 1) & 3);
+    return (uint32_t)(box * Gm::BOX_BYTES + row * Gm::BOXB + ((cib ^ x) << 4));
+}
+
+struct StageInfo {
+    float ks, vs;   // fp8 scales of the tile's page and kv head
+    int valid;      // 0: page id was out of range, tile skipped
+    int pad;
+};
+
+// Largest b with prefix[b] * Hkv <= x, for 0 <= x < prefix[B] * Hkv.
+__device__ __forceinline__ int seek_request(const int* prefix, int B, int Hkv, long long x)
+{
+    int lo = 0, hi = B;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if ((long long)prefix[mid] * Hkv <= x) lo = mid;
+        else hi = mid;
+    }
+    return lo;
+}
+
+template <int D, bool FP8>
+__global__ void __launch_bounds__(kAttnWarps * 32, 1)
+decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                   const AttnParams p)
+{
+    using Gm = Geo<D, FP8>;
+    constexpr int KSTEPS = D / 16;      // mma k-steps along d for QK^T
+    constexpr int NTD = D / 8;          // mma n-tiles along d for P V
+    constexpr int NT = kAttnWarps * 32;
+
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ int s_warp_tot[kAttnWarps];
+    __shared__ int s_bad;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int B = p.batch, Hkv = p.Hkv, P = p.P, S = p.stages;
+
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t stage_area = (raw + 1023u) & ~1023u;
+    uint8_t* const area_ptr = smem_raw + (stage_area - raw);
+    StageInfo* const info_all = reinterpret_cast<StageInfo*>(area_ptr + kAttnWarps * S * Gm::STAGEB);
+    uint8_t* const bar_ptr = reinterpret_cast<uint8_t*>(info_all + kAttnWarps * S);
+    int* const prefix = reinterpret_cast<int*>(bar_ptr + kAttnWarps * S * 8);
+
+    if (tid == 0) {
+        s_bad = 0;
+        prefetch_tensormap(&tmk);
+        prefetch_tensormap(&tmv);
+    }
+    __syncthreads();
+
+    // ---- 1. tiles per request and their exclusive prefix ----------------------
+    const long long cap = (long long)p.bt_stride * P;
+    const int per = (B + NT - 1) / NT;
+    const int lo = min(B, tid * per), hi = min(B, lo + per);
+    int local = 0;
+    for (int b = lo; b < hi; ++b) {
+        const int L = p.seq_lens[b];
+        const bool ok = L >= 0 && (long long)L < cap;
+        const int nt = ok ? (L + kTile) / kTile : 0;   // ceil((L + 1) / 16)
+        if (!ok) s_bad = 1;
+        prefix[b] = nt;
+        local += nt;
+    }
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) s_warp_tot[warp] = incl;
+    __syncthreads();
+    int run = incl - local;
+    for (int w2 = 0; w2 < warp; ++w2) run += s_warp_tot[w2];
+    for (int b = lo; b < hi; ++b) {
+        const int c = prefix[b];
+        prefix[b] = run;
+        run += c;
+    }
+    if (tid == NT - 1) prefix[B] = run;
+    __syncthreads();
+
+    if (s_bad && blockIdx.x == 0) {
+        // requests with an impossible length produce zeros and an error bit
+        if (tid == 0) atomicOr(p.err, kErrLength);
+        for (int b = warp; b < B; b += kAttnWarps) {
+            const int L = p.seq_lens[b];
+            if (L >= 0 && (long long)L < cap) continue;
+            uint32_t* o32 = reinterpret_cast<uint32_t*>(p.out + (size_t)b * p.Hq * D);
+            for (int i = lane; i < p.Hq * D / 2; i += 32) o32[i] = 0u;
+        }
+    }
+
+    // ---- 2. this warp's range of tiles --------------------------------------------
+    const long long T = (long long)prefix[B] * Hkv;
+    if (T == 0) return;
+    long long Wl = (long long)gridDim.x * kAttnWarps;
+    if (p.workers > 0) Wl = min(Wl, (long long)p.workers);
+    else Wl = min(Wl, (T + kMinTilesPerWorker - 1) / kMinTilesPerWorker);
+    Wl = max(1LL, min(Wl, T));
+    const int W = (int)Wl;
+    const int w = warp * gridDim.x + blockIdx.x;   // spread workers over SMs first
+    if (w >= W) return;
+    const long long t_begin = (long long)w * T / W;
+    const long long t_end = (long long)(w + 1) * T / W;
+    const int ntiles = (int)(t_end - t_begin);
+
+    const uint32_t my_stage0 = stage_area + (uint32_t)(warp * S * Gm::STAGEB);
+    StageInfo* const my_info = info_all + warp * S;
+    const uint32_t my_bar0 = smem_u32(bar_ptr) + (uint32_t)(warp * S * 8);
+    if (lane == 0) {
+        for (int s = 0; s < S; ++s) mbar_init(my_bar0 + 8u * s, 1u);
+        fence_mbar_init();
+    }
+    __syncwarp();
+
+    // ---- 3. producer: 32-tile lookahead of page ids and scales, TMA issue -------
+    long long la_base = t_begin - 64;
+    int la_valid = 0, la_row = 0;
+    float la_ks = 1.f, la_vs = 1.f;
+
+    auto la_fill = [&](long long x0) {
+        la_base = x0;
+        const long long y = x0 + lane;
+        la_valid = 0;
+        if (y < t_end) {
+            const int b = seek_request(prefix, B, Hkv, y);
+            const int ntb = prefix[b + 1] - prefix[b];
+            const long long r = y - (long long)prefix[b] * Hkv;
+            const int kvh = (int)(r / ntb), tt = (int)(r % ntb);
+            const int tok0 = tt * kTile;
+            const int lp = tok0 / P;
+            const int page = __ldg(&p.block_tables[(size_t)b * p.bt_stride + lp]);
+            if ((unsigned)page < (unsigned)p.num_pages) {
+                la_valid = 1;
+                la_row = (page * Hkv + kvh) * P + (tok0 - lp * P);
+                if (FP8) {
+                    la_ks = __ldg(&p.k_scale[(size_t)page * Hkv + kvh]);
+                    la_vs = __ldg(&p.v_scale[(size_t)page * Hkv + kvh]);
+                }
+            } else {
+                la_valid = 2;
+            }
+        }
+    };
+
+    auto issue = [&](long long x, int s) {
+        if (x >= la_base + 32) la_fill(x);
+        const int src = (int)(x - la_base);
+        const int v = __shfl_sync(kFull, la_valid, src);
+        const int row = __shfl_sync(kFull, la_row, src);
+        const float ks = __shfl_sync(kFull, la_ks, src);
+        const float vs = __shfl_sync(kFull, la_vs, src);
+        if (lane == 0) {
+            const uint32_t bar = my_bar0 + 8u * s;
+            StageInfo si;
+            si.ks = ks;
+            si.vs = vs;
+            si.valid = (v == 1);
+            si.pad = 0;
+            my_info[s] = si;
+            if (v == 1) {
+                mbar_arrive_expect_tx(bar, (uint32_t)Gm::STAGEB);
+                const uint32_t kdst = my_stage0 + (uint32_t)(s * Gm::STAGEB);
+                const uint32_t vdst = kdst + Gm::TILEB;
+#pragma unroll
+                for (int j = 0; j < Gm::NBOX; ++j) {
+                    tma_load_2d(kdst + j * Gm::BOX_BYTES, &tmk, j * (Gm::BOXB / Gm::ELEM), row, bar);
+                    tma_load_2d(vdst + j * Gm::BOX_BYTES, &tmv, j * (Gm::BOXB / Gm::ELEM), row, bar);
+                }
+            } else {
+                atomicOr(p.err, kErrPage);
+                mbar_arrive(bar);
+            }
+        }
+    };
+
+    const int pre = min(S, ntiles);
+    for (int k = 0; k < pre; ++k) issue(t_begin + k, k);
+    int issued = pre;
+
+    // ---- 4. consumer ----------------------------------------------------------------
+    int cb = seek_request(prefix, B, Hkv, t_begin);
+    int cnt = prefix[cb + 1] - prefix[cb];
+    int ckvh, ctt;
+    {
+        const long long r = t_begin - (long long)prefix[cb] * Hkv;
+        ckvh = (int)(r / cnt);
+        ctt = (int)(r % cnt);
+    }
+
+    const int g = lane >> 2;     // mma row = query head within the group
+    const int c4 = lane & 3;
+    const int G = p.G;
+    const int mi = lane >> 3, ri = lane & 7;        // ldmatrix: matrix index, row
+    const int tokK = ((mi >> 1) << 3) + ri;         // token row addressed for K
+    const int tokV = ((mi & 1) << 3) + ri;          // token row addressed for V (trans)
+
+    float o[NTD][2];
+    uint32_t qa[KSTEPS][2];
+    float m_run = -INFINITY, l_run = 0.f;
+    int n_cur = 0;
+    bool dead = false;
+    int k_dead = 0;
+
+    for (int k = 0; k < ntiles; ++k) {
+        const int s = k % S;
+        const uint32_t parity = (uint32_t)((k / S) & 1);
+
+        if (ctt == 0 || k == 0) {
+            // start of a (request, kv head) pair in this range: query fragments
+            n_cur = p.seq_lens[cb] + 1;
+            const __nv_bfloat16* qrow = p.q + ((size_t)cb * p.Hq + (size_t)ckvh * G + g) * D;
+#pragma unroll
+            for (int ks = 0; ks < KSTEPS; ++ks) {
+                if (g < G) {
+                    if (!FP8) {
+                        qa[ks][0] = *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * c4);
+                        qa[ks][1] = *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8 + 2 * c4);
+                    } else {
+                        // fp8 path: k-order inside a k-step follows the byte layout of
+                        // the E4M3 rows (4 consecutive d per quad lane), operands in f16
+                        const uint2 v = *reinterpret_cast<const uint2*>(qrow + 16 * ks + 4 * c4);
+                        qa[ks][0] = pack_f16(bf16_lo(v.x), bf16_hi(v.x));
+                        qa[ks][1] = pack_f16(bf16_lo(v.y), bf16_hi(v.y));
+                    }
+                } else {
+                    qa[ks][0] = qa[ks][1] = 0u;
+                }
+            }
+#pragma unroll
+            for (int nt = 0; nt < NTD; ++nt) o[nt][0] = o[nt][1] = 0.f;
+            m_run = -INFINITY;
+            l_run = 0.f;
+        }
+
+        if (!dead) {
+            const bool ok = __all_sync(kFull, mbar_wait_bounded(my_bar0 + 8u * s, parity, kWaitLimitNs));
+            if (!ok) {
+                dead = true;
+                k_dead = k;
+                if (lane == 0) atomicOr(p.err, kErrTimeout);
+            }
+        }
+
+        if (!dead && my_info[s].valid) {
+            const StageInfo si = my_info[s];
+            const uint32_t kb = my_stage0 + (uint32_t)(s * Gm::STAGEB);
+            const uint32_t vb = kb + Gm::TILEB;
+            const int tok0 = ctt * kTile;
+            const int rows_valid = min(kTile, n_cur - tok0);
+            if (rows_valid < kTile) {
+                // slots past the request's end may hold anything (NaN): zero them in V
+                constexpr int CPR = Gm::ROWB / 16;
+                const int nch = (kTile - rows_valid) * CPR;
+                for (int e = lane; e < nch; e += 32) {
+                    const int r = rows_valid + e / CPR, ch = e % CPR;
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(vb + tile_off<D, FP8>(r, ch)),
+                                 "r"(0u)
+                                 : "memory");
+                }
+                __syncwarp();
+            }
+
+            // S = Q K^T (two n-tiles of 8 tokens)
+            float sc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+            if (!FP8) {
+#pragma unroll
+                for (int ks = 0; ks < KSTEPS; ++ks) {
+                    uint32_t r0, r1, r2, r3;
+                    ldsm_x4(kb + tile_off<D, FP8>(tokK, 2 * ks + (mi & 1)), r0, r1, r2, r3);
+                    mma_bf16_r8(sc[0][0], sc[0][1], qa[ks][0], qa[ks][1], r0, r1);
+                    mma_bf16_r8(sc[1][0], sc[1][1], qa[ks][0], qa[ks][1], r2, r3);
+                }
+            } else {
+#pragma unroll
+                for (int s4 = 0; s4 < D / 32; ++s4) {
+                    uint32_t r0, r1, r2, r3;
+                    ldsm_x4(kb + tile_off<D, FP8>(tokK, 2 * s4 + (mi & 1)), r0, r1, r2, r3);
+                    mma_f16_r8(sc[0][0], sc[0][1], qa[2 * s4][0], qa[2 * s4][1], cvt_lo(r0), cvt_hi(r0));
+                    mma_f16_r8(sc[0][0], sc[0][1], qa[2 * s4 + 1][0], qa[2 * s4 + 1][1], cvt_lo(r1), cvt_hi(r1));
+                    mma_f16_r8(sc[1][0], sc[1][1], qa[2 * s4][0], qa[2 * s4][1], cvt_lo(r2), cvt_hi(r2));
+                    mma_f16_r8(sc[1][0], sc[1][1], qa[2 * s4 + 1][0], qa[2 * s4 + 1][1], cvt_lo(r3), cvt_hi(r3));
+                }
+            }
+
+            // online softmax in log2 units; masked tokens are -inf (never 0 * NaN)
+            const float slog2 = FP8 ? p.scale_log2 * si.ks : p.scale_log2;
+            float mx = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int tok = tok0 + 8 * j + 2 * c4 + e;
+                    sc[j][e] = (tok < n_cur) ? sc[j][e] * slog2 : -INFINITY;
+                    mx = fmaxf(mx, sc[j][e]);
+                }
+            mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+            const float m_new = fmaxf(m_run, mx);
+            const float m_ref = (m_new == -INFINITY) ? 0.f : m_new;
+            const float alpha = exp2f(m_run - m_ref);
+            const float p00 = exp2f(sc[0][0] - m_ref), p01 = exp2f(sc[0][1] - m_ref);
+            const float p10 = exp2f(sc[1][0] - m_ref), p11 = exp2f(sc[1][1] - m_ref);
+            uint32_t pa0, pa2;
+            float psum;
+            if (!FP8) {
+                pa0 = pack_bf16(p00, p01);
+                pa2 = pack_bf16(p10, p11);
+                psum = (bf16_lo(pa0) + bf16_hi(pa0)) + (bf16_lo(pa2) + bf16_hi(pa2));
+            } else {
+                pa0 = pack_f16(p00, p01);
+                pa2 = pack_f16(p10, p11);
+                const float2 f0 = f16x2_to_f32(pa0), f2 = f16x2_to_f32(pa2);
+                psum = (f0.x + f0.y) + (f2.x + f2.y);
+            }
+            l_run = l_run * alpha + psum;
+            m_run = m_new;
+#pragma unroll
+            for (int nt = 0; nt < NTD; ++nt) {
+                o[nt][0] *= alpha;
+                o[nt][1] *= alpha;
+            }
+
+            // O += P V
+            if (!FP8) {
+#pragma unroll
+                for (int dj = 0; dj < D / 16; ++dj) {
+                    uint32_t r0, r1, r2, r3;
+                    ldsm_x4_trans(vb + tile_off<D, FP8>(tokV, 2 * dj + (mi >> 1)), r0, r1, r2, r3);
+                    mma_bf16_r8(o[2 * dj][0], o[2 * dj][1], pa0, pa2, r0, r1);
+                    mma_bf16_r8(o[2 * dj + 1][0], o[2 * dj + 1][1], pa0, pa2, r2, r3);
+                }
+            } else {
+                // E4M3 V: lane (n = g, c4) loads d in [DV*n, DV*n + DV) of tokens
+                // 2c4, 2c4+1, 8+2c4, 9+2c4; byte permutes pair tokens per d, and the
+                // mma n-index j of n-tile nt stands for d = DV*j + nt.
+                constexpr int DV = D / 8;
+                constexpr int WORDS = DV / 4;
+                uint32_t wa[WORDS], wb[WORDS], wc[WORDS], wd[WORDS];
+                const int t0 = 2 * c4;
+                if constexpr (DV == 16) {
+                    const uint4 a = lds128(vb + tile_off<D, FP8>(t0, g));
+                    const uint4 b = lds128(vb + tile_off<D, FP8>(t0 + 1, g));
+                    const uint4 cc = lds128(vb + tile_off<D, FP8>(t0 + 8, g));
+                    const uint4 dd = lds128(vb + tile_off<D, FP8>(t0 + 9, g));
+                    wa[0] = a.x; wa[1] = a.y; wa[2] = a.z; wa[3] = a.w;
+                    wb[0] = b.x; wb[1] = b.y; wb[2] = b.z; wb[3] = b.w;
+                    wc[0] = cc.x; wc[1] = cc.y; wc[2] = cc.z; wc[3] = cc.w;
+                    wd[0] = dd.x; wd[1] = dd.y; wd[2] = dd.z; wd[3] = dd.w;
+                } else {
+                    const uint32_t off8 = (uint32_t)((g & 1) * 8);
+                    const uint2 a = lds64(vb + tile_off<D, FP8>(t0, g >> 1) + off8);
+                    const uint2 b = lds64(vb + tile_off<D, FP8>(t0 + 1, g >> 1) + off8);
+                    const uint2 cc = lds64(vb + tile_off<D, FP8>(t0 + 8, g >> 1) + off8);
+                    const uint2 dd = lds64(vb + tile_off<D, FP8>(t0 + 9, g >> 1) + off8);
+                    wa[0] = a.x; wa[1] = a.y;
+                    wb[0] = b.x; wb[1] = b.y;
+                    wc[0] = cc.x; wc[1] = cc.y;
+                    wd[0] = dd.x; wd[1] = dd.y;
+                }
+                const float vs = si.vs;
+#pragma unroll
+                for (int kw = 0; kw < WORDS; ++kw) {
+                    const uint32_t x0 = __byte_perm(wa[kw], wb[kw], 0x5140);
+                    const uint32_t x1 = __byte_perm(wa[kw], wb[kw], 0x7362);
+                    const uint32_t y0 = __byte_perm(wc[kw], wd[kw], 0x5140);
+                    const uint32_t y1 = __byte_perm(wc[kw], wd[kw], 0x7362);
+                    float t[4][2] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+                    mma_f16_r8(t[0][0], t[0][1], pa0, pa2, cvt_lo(x0), cvt_lo(y0));
+                    mma_f16_r8(t[1][0], t[1][1], pa0, pa2, cvt_hi(x0), cvt_hi(y0));
+                    mma_f16_r8(t[2][0], t[2][1], pa0, pa2, cvt_lo(x1), cvt_lo(y1));
+                    mma_f16_r8(t[3][0], t[3][1], pa0, pa2, cvt_hi(x1), cvt_hi(y1));
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        o[4 * kw + e][0] = fmaf(t[e][0], vs, o[4 * kw + e][0]);
+                        o[4 * kw + e][1] = fmaf(t[e][1], vs, o[4 * kw + e][1]);
+                    }
+                }
+            }
+        }
+        __syncwarp();
+
+        // refill this stage with the tile `S` ahead
+        if (!dead && issued < ntiles) {
+            if (lane == 0) fence_proxy_async_smem();
+            issue(t_begin + issued, s);
+            ++issued;
+        }
+
+        // ---- end of a pair (or of this range): write out or leave a partial -------
+        if (ctt == cnt - 1 || k == ntiles - 1) {
+            float lsum = l_run + __shfl_xor_sync(kFull, l_run, 1);
+            lsum += __shfl_xor_sync(kFull, lsum, 2);
+            const long long ts = (long long)prefix[cb] * Hkv + (long long)ckvh * cnt;
+            const long long te = ts + cnt;
+            const int wf = (int)(((ts + 1) * W - 1) / T);
+            const int wl = (int)((te * W - 1) / T);
+            const size_t orow = ((size_t)cb * p.Hq + (size_t)ckvh * G + g) * D;
+            if (wf == wl) {
+                if (g < G) {
+                    const float inv = 1.f / lsum;
+                    uint32_t* dst = reinterpret_cast<uint32_t*>(p.out + orow);
+                    if (!FP8) {
+#pragma unroll
+                        for (int nt = 0; nt < NTD; ++nt)
+                            dst[(8 * nt + 2 * c4) >> 1] = pack_bf16(o[nt][0] * inv, o[nt][1] * inv);
+                    } else {
+                        constexpr int DV = D / 8;
+#pragma unroll
+                        for (int e = 0; e < 2; ++e)
+#pragma unroll
+                            for (int u = 0; u < DV / 2; ++u)
+                                dst[(DV * (2 * c4 + e) + 2 * u) >> 1] =
+                                    pack_bf16(o[2 * u][e] * inv, o[2 * u + 1][e] * inv);
+                    }
+                }
+            } else {
+                const long long my_start = (long long)w * T / W;
+                const int slot = 2 * w + (my_start < ts ? 1 : 0);
+                const size_t prow = ((size_t)slot * kMaxGroup + g) * D;
+                if (g < G) {
+                    float* dst = p.part_o + prow;
+                    if (!FP8) {
+#pragma unroll
+                        for (int nt = 0; nt < NTD; ++nt)
+                            *reinterpret_cast<float2*>(dst + 8 * nt + 2 * c4) = make_float2(o[nt][0], o[nt][1]);
+                    } else {
+                        constexpr int DV = D / 8;
+#pragma unroll
+                        for (int e = 0; e < 2; ++e)
+#pragma unroll
+                            for (int u = 0; u < DV / 2; ++u)
+                                *reinterpret_cast<float2*>(dst + DV * (2 * c4 + e) + 2 * u) =
+                                    make_float2(o[2 * u][e], o[2 * u + 1][e]);
+                    }
+                    if (c4 == 0)
+                        *reinterpret_cast<float2*>(p.part_ml + ((size_t)slot * kMaxGroup + g) * 2) =
+                            make_float2(m_run, lsum);
+                }
+                __threadfence();
+                __syncwarp();
+                int old = 0;
+                if (lane == 0) old = atomicAdd(&p.counters[(size_t)cb * Hkv + ckvh], 1);
+                old = __shfl_sync(kFull, old, 0);
+                if (old == wl - wf) {
+                    // last arrival: merge the partials of this pair by log-sum-exp
+                    __threadfence();
+                    constexpr int DPL = D / 32;   // columns per lane
+                    for (int gg = 0; gg < G; ++gg) {
+                        float mstar = -INFINITY;
+                        for (int v = wf; v <= wl; ++v) {
+                            const int sl = 2 * v + (((long long)v * T / W) < ts ? 1 : 0);
+                            mstar = fmaxf(mstar, __ldcg(p.part_ml + ((size_t)sl * kMaxGroup + gg) * 2));
+                        }
+                        const float mref = (mstar == -INFINITY) ? 0.f : mstar;
+                        float lt = 0.f, acc[DPL];
+#pragma unroll
+                        for (int q = 0; q < DPL; ++q) acc[q] = 0.f;
+                        for (int v = wf; v <= wl; ++v) {
+                            const int sl = 2 * v + (((long long)v * T / W) < ts ? 1 : 0);
+                            const float2 ml = __ldcg(reinterpret_cast<const float2*>(
+                                p.part_ml + ((size_t)sl * kMaxGroup + gg) * 2));
+                            const float f = exp2f(ml.x - mref);
+                            lt += ml.y * f;
+                            const float* src = p.part_o + ((size_t)sl * kMaxGroup + gg) * D + lane * DPL;
+                            if constexpr (DPL == 4) {
+                                const float4 x = __ldcg(reinterpret_cast<const float4*>(src));
+                                acc[0] += f * x.x; acc[1] += f * x.y;
+                                acc[2] += f * x.z; acc[3] += f * x.w;
+                            } else {
+                                const float2 x = __ldcg(reinterpret_cast<const float2*>(src));
+                                acc[0] += f * x.x; acc[1] += f * x.y;
+                            }
+                        }
+                        const float inv = 1.f / lt;
+                        uint32_t* dst = reinterpret_cast<uint32_t*>(
+                            p.out + ((size_t)cb * p.Hq + (size_t)ckvh * G + gg) * D + lane * DPL);
+#pragma unroll
+                        for (int q = 0; q < DPL / 2; ++q) dst[q] = pack_bf16(acc[2 * q] * inv, acc[2 * q + 1] * inv);
+                    }
+                    if (lane == 0) atomicExch(&p.counters[(size_t)cb * Hkv + ckvh], 0);
+                }
+            }
+        }
+
+        // advance the consumer cursor
+        if (++ctt == cnt) {
+            ctt = 0;
+            if (++ckvh == Hkv) {
+                ckvh = 0;
+                do { ++cb; } while (cb < B && prefix[cb + 1] == prefix[cb]);
+            }
+            if (cb < B) cnt = prefix[cb + 1] - prefix[cb];
+        }
+    }
+
+    // a worker that timed out still owns the loads it issued for tiles
+    // k_dead .. issued-1 (one per stage): wait for them, bounded
+    if (dead && lane == 0) {
+        for (int k = k_dead; k < issued; ++k)
+            (void)mbar_wait_bounded(my_bar0 + 8u * (k % S), (uint32_t)((k / S) & 1), kWaitLimitNs / 8);
+    }
+}
+
+template <int D, bool FP8>
+size_t smem_bytes_for(int stages, int max_batch)
+{
+    using Gm = Geo<D, FP8>;
+    return 1024 + (size_t)kAttnWarps * stages * (Gm::STAGEB + sizeof(StageInfo) + 8) +
+           sizeof(int) * (size_t)(max_batch + 1);
+}
+
+template <int D, bool FP8>
+cudaError_t prepare_t(int num_sms, int max_batch, AttnLaunch* out)
+{
+    int dev = 0, optin = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e != cudaSuccess) return e;
+    const size_t budget = (size_t)optin - 256;   // static shared memory of the kernel
+    int stages = 8;
+    while (stages > 2 && smem_bytes_for<D, FP8>(stages, max_batch) > budget) --stages;
+    if (smem_bytes_for<D, FP8>(stages, max_batch) > budget) return cudaErrorInvalidConfiguration;
+    const size_t bytes = smem_bytes_for<D, FP8>(stages, max_batch);
+    e = cudaFuncSetAttribute(decode_attn_kernel<D, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)bytes);
+    if (e != cudaSuccess) return e;
+    out->ctas = num_sms;
+    out->stages = stages;
+    out->smem_bytes = bytes;
+    return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t attn_prepare(int head_dim, bool fp8, int num_sms, int max_batch, AttnLaunch* out)
+{
+    if (head_dim == 128) return fp8 ? prepare_t<128, true>(num_sms, max_batch, out)
+                                    : prepare_t<128, false>(num_sms, max_batch, out);
+    return fp8 ? prepare_t<64, true>(num_sms, max_batch, out) : prepare_t<64, false>(num_sms, max_batch, out);
+}
+
+cudaError_t launch_decode_attn(const AttnParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
+                               int head_dim, bool fp8, const AttnLaunch& L, cudaStream_t stream)
+{
+    const dim3 grid(L.ctas), block(kAttnWarps * 32);
+    AttnParams q = p;
+    q.stages = L.stages;
+    if (head_dim == 128) {
+        if (fp8) decode_attn_kernel<128, true><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
+        else decode_attn_kernel<128, false><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
+    } else {
+        if (fp8) decode_attn_kernel<64, true><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
+        else decode_attn_kernel<64, false><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace pkv

@@ -1,0 +1,284 @@
+// pkv_api.cu -- host side of the libpkv C ABI (include/pkv.h): validation,
+// workspace ownership, TMA descriptor encoding and kernel launches.  No C++
+// exception crosses the ABI (nothing here throws).
+//
+// Shapes are fixed when the context is created, like an engine built for one
+// model and its limits ("TensorRT-LLM", section "What the build step is
+// for"); errors come back per call as status codes.
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <cudaTypedefs.h>
+
+#include "pkv_internal.h"
+
+struct pkv_ctx {
+    pkv_config cfg;
+    int device;
+    int num_sms;
+    int G;
+    pkv::AttnLaunch attn;
+    int workers;
+    void* ws;             // one allocation, carved below
+    size_t ws_bytes;
+    int* d_err;
+    int* d_counters;
+    float* d_part_o;
+    float* d_part_ml;
+    const void* tm_k_ptr;
+    const void* tm_v_ptr;
+    CUtensorMap tmk, tmv;
+};
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+pkv_status validate_config(const pkv_config* c)
+{
+    if (!c) return PKV_ERR_INVALID_ARG;
+    if (c->num_q_heads <= 0 || c->num_kv_heads <= 0) return PKV_ERR_INVALID_ARG;
+    if (c->num_q_heads % c->num_kv_heads) return PKV_ERR_INVALID_ARG;
+    if (c->head_dim <= 0 || c->page_size <= 0) return PKV_ERR_INVALID_ARG;
+    if (c->kv_dtype != PKV_KV_BF16 && c->kv_dtype != PKV_KV_FP8_E4M3) return PKV_ERR_INVALID_ARG;
+    if (!(c->rope_base > 1.0) || !isfinite(c->rope_base)) return PKV_ERR_INVALID_ARG;
+    if (c->max_batch <= 0 || c->max_blocks_per_seq <= 0 || c->num_pages <= 0) return PKV_ERR_INVALID_ARG;
+    if ((long long)c->max_blocks_per_seq * c->page_size >= (1LL << 31)) return PKV_ERR_INVALID_ARG;
+    if (c->num_q_heads / c->num_kv_heads > pkv::kMaxGroup) return PKV_ERR_UNSUPPORTED;
+    if (c->head_dim != 64 && c->head_dim != 128) return PKV_ERR_UNSUPPORTED;
+    if (c->page_size != 16 && c->page_size != 32 && c->page_size != 64) return PKV_ERR_UNSUPPORTED;
+    if (c->max_batch > pkv::kMaxBatch) return PKV_ERR_UNSUPPORTED;
+    // TMA row coordinates are int32
+    if ((long long)c->num_pages * c->num_kv_heads * c->page_size >= (1LL << 31)) return PKV_ERR_UNSUPPORTED;
+    return PKV_OK;
+}
+
+pkv_status check_call(const pkv_ctx* ctx, int batch, int bt_stride, const void* k_pool,
+                      const void* v_pool, const float* k_scale, const float* v_scale,
+                      const int32_t* block_tables, const int32_t* seq_lens)
+{
+    if (!ctx) return PKV_ERR_INVALID_ARG;
+    if (batch < 0 || batch > ctx->cfg.max_batch) return PKV_ERR_INVALID_ARG;
+    if (batch == 0) return PKV_OK;
+    if (bt_stride <= 0 || bt_stride > ctx->cfg.max_blocks_per_seq) return PKV_ERR_INVALID_ARG;
+    if (!k_pool || !v_pool || !block_tables || !seq_lens) return PKV_ERR_INVALID_ARG;
+    if (!aligned16(k_pool) || !aligned16(v_pool) || !aligned16(block_tables) || !aligned16(seq_lens))
+        return PKV_ERR_INVALID_ARG;
+    if (ctx->cfg.kv_dtype == PKV_KV_FP8_E4M3) {
+        if (!k_scale || !v_scale || !aligned16(k_scale) || !aligned16(v_scale)) return PKV_ERR_INVALID_ARG;
+    }
+    return PKV_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// 2-D view of a pool: rows = num_pages * Hkv * P token rows of head_dim
+// elements; box = 16 rows x (128 or 64 bytes), swizzled to match the
+// kernel's shared-memory addressing.
+bool encode_pool(const pkv_ctx* ctx, const void* pool, CUtensorMap* map)
+{
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const bool fp8 = ctx->cfg.kv_dtype == PKV_KV_FP8_E4M3;
+    const int elem = fp8 ? 1 : 2;
+    const int rowb = ctx->cfg.head_dim * elem;
+    const int boxb = rowb > 128 ? 128 : rowb;
+    cuuint64_t dims[2] = {(cuuint64_t)ctx->cfg.head_dim,
+                          (cuuint64_t)ctx->cfg.num_pages * ctx->cfg.num_kv_heads * ctx->cfg.page_size};
+    cuuint64_t strides[1] = {(cuuint64_t)rowb};
+    cuuint32_t box[2] = {(cuuint32_t)(boxb / elem), (cuuint32_t)pkv::kTile};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                    const_cast<void*>(pool), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    boxb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+extern "C" {
+
+pkv_status pkv_create(const pkv_config* cfg, pkv_ctx** out)
+{
+    if (!out) return PKV_ERR_INVALID_ARG;
+    const pkv_status v = validate_config(cfg);
+    if (v != PKV_OK) return v;
+
+    pkv_ctx* ctx = static_cast<pkv_ctx*>(calloc(1, sizeof(pkv_ctx)));
+    if (!ctx) return PKV_ERR_OOM;
+    ctx->cfg = *cfg;
+    ctx->G = cfg->num_q_heads / cfg->num_kv_heads;
+    if (cudaGetDevice(&ctx->device) != cudaSuccess ||
+        cudaDeviceGetAttribute(&ctx->num_sms, cudaDevAttrMultiProcessorCount, ctx->device) != cudaSuccess) {
+        free(ctx);
+        return PKV_ERR_CUDA;
+    }
+    const bool fp8 = cfg->kv_dtype == PKV_KV_FP8_E4M3;
+    if (pkv::attn_prepare(cfg->head_dim, fp8, ctx->num_sms, cfg->max_batch, &ctx->attn) != cudaSuccess) {
+        free(ctx);
+        return PKV_ERR_CUDA;
+    }
+
+    const size_t max_workers = (size_t)ctx->attn.ctas * pkv::kAttnWarps;
+    const size_t b_err = 256;
+    const size_t b_cnt = ((size_t)cfg->max_batch * cfg->num_kv_heads * sizeof(int) + 255) & ~(size_t)255;
+    const size_t b_po = 2 * max_workers * pkv::kMaxGroup * cfg->head_dim * sizeof(float);
+    const size_t b_pml = 2 * max_workers * pkv::kMaxGroup * 2 * sizeof(float);
+    ctx->ws_bytes = b_err + b_cnt + b_po + b_pml;
+    if (cudaMalloc(&ctx->ws, ctx->ws_bytes) != cudaSuccess) {
+        cudaGetLastError();
+        free(ctx);
+        return PKV_ERR_OOM;
+    }
+    uint8_t* base = static_cast<uint8_t*>(ctx->ws);
+    ctx->d_err = reinterpret_cast<int*>(base);
+    ctx->d_counters = reinterpret_cast<int*>(base + b_err);
+    ctx->d_part_o = reinterpret_cast<float*>(base + b_err + b_cnt);
+    ctx->d_part_ml = reinterpret_cast<float*>(base + b_err + b_cnt + b_po);
+    if (cudaMemset(ctx->ws, 0, b_err + b_cnt) != cudaSuccess) {
+        cudaFree(ctx->ws);
+        free(ctx);
+        return PKV_ERR_CUDA;
+    }
+    *out = ctx;
+    return PKV_OK;
+}
+
+pkv_status pkv_rope_append(pkv_ctx* ctx, void* q, const void* k_new, const void* v_new, void* k_pool,
+                           void* v_pool, const float* k_scale, const float* v_scale,
+                           const int32_t* block_tables, int bt_stride, const int32_t* seq_lens, int batch,
+                           cudaStream_t stream)
+{
+    pkv_status st = check_call(ctx, batch, bt_stride, k_pool, v_pool, k_scale, v_scale, block_tables, seq_lens);
+    if (st != PKV_OK || batch == 0) return st;
+    if (!q || !k_new || !v_new || !aligned16(q) || !aligned16(k_new) || !aligned16(v_new))
+        return PKV_ERR_INVALID_ARG;
+
+    pkv::RopeParams p;
+    p.q = static_cast<__nv_bfloat16*>(q);
+    p.k_new = static_cast<const __nv_bfloat16*>(k_new);
+    p.v_new = static_cast<const __nv_bfloat16*>(v_new);
+    p.k_pool = k_pool;
+    p.v_pool = v_pool;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
+    p.block_tables = block_tables;
+    p.seq_lens = seq_lens;
+    p.err = ctx->d_err;
+    p.rope_base = ctx->cfg.rope_base;
+    p.batch = batch;
+    p.bt_stride = bt_stride;
+    p.Hq = ctx->cfg.num_q_heads;
+    p.Hkv = ctx->cfg.num_kv_heads;
+    p.D = ctx->cfg.head_dim;
+    p.P = ctx->cfg.page_size;
+    p.num_pages = ctx->cfg.num_pages;
+    p.fp8 = ctx->cfg.kv_dtype == PKV_KV_FP8_E4M3;
+    return pkv::launch_rope_append(p, stream) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+pkv_status pkv_decode_attn(pkv_ctx* ctx, const void* q, const void* k_pool, const void* v_pool,
+                           const float* k_scale, const float* v_scale, const int32_t* block_tables,
+                           int bt_stride, const int32_t* seq_lens, int batch, void* out,
+                           cudaStream_t stream)
+{
+    pkv_status st = check_call(ctx, batch, bt_stride, k_pool, v_pool, k_scale, v_scale, block_tables, seq_lens);
+    if (st != PKV_OK || batch == 0) return st;
+    if (!q || !out || !aligned16(q) || !aligned16(out)) return PKV_ERR_INVALID_ARG;
+
+    if (ctx->tm_k_ptr != k_pool) {
+        if (!encode_pool(ctx, k_pool, &ctx->tmk)) return PKV_ERR_CUDA;
+        ctx->tm_k_ptr = k_pool;
+    }
+    if (ctx->tm_v_ptr != v_pool) {
+        if (!encode_pool(ctx, v_pool, &ctx->tmv)) return PKV_ERR_CUDA;
+        ctx->tm_v_ptr = v_pool;
+    }
+
+    pkv::AttnParams p;
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
+    p.block_tables = block_tables;
+    p.seq_lens = seq_lens;
+    p.part_o = ctx->d_part_o;
+    p.part_ml = ctx->d_part_ml;
+    p.counters = ctx->d_counters;
+    p.err = ctx->d_err;
+    p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)ctx->cfg.head_dim));
+    p.batch = batch;
+    p.bt_stride = bt_stride;
+    p.Hq = ctx->cfg.num_q_heads;
+    p.Hkv = ctx->cfg.num_kv_heads;
+    p.G = ctx->G;
+    p.P = ctx->cfg.page_size;
+    p.num_pages = ctx->cfg.num_pages;
+    p.stages = ctx->attn.stages;
+    p.workers = ctx->workers;
+    const cudaError_t e = pkv::launch_decode_attn(p, ctx->tmk, ctx->tmv, ctx->cfg.head_dim,
+                                                  ctx->cfg.kv_dtype == PKV_KV_FP8_E4M3, ctx->attn, stream);
+    return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+pkv_status pkv_destroy(pkv_ctx* ctx)
+{
+    if (!ctx) return PKV_OK;
+    pkv_status st = PKV_OK;
+    if (cudaDeviceSynchronize() != cudaSuccess) st = PKV_ERR_CUDA;
+    if (ctx->ws && cudaFree(ctx->ws) != cudaSuccess) st = PKV_ERR_CUDA;
+    free(ctx);
+    return st;
+}
+
+const char* pkv_status_str(pkv_status s)
+{
+    switch (s) {
+    case PKV_OK: return "ok";
+    case PKV_ERR_INVALID_ARG: return "invalid argument";
+    case PKV_ERR_UNSUPPORTED: return "unsupported configuration";
+    case PKV_ERR_CUDA: return "CUDA error";
+    case PKV_ERR_OOM: return "out of device memory";
+    case PKV_ERR_DEVICE_BOUNDS: return "device saw a page id or length out of range";
+    case PKV_ERR_DEVICE_TIMEOUT: return "a bounded wait inside a kernel timed out";
+    }
+    return "unknown status";
+}
+
+pkv_status pkv_check_device_error(pkv_ctx* ctx, cudaStream_t stream, int* bits)
+{
+    if (!ctx) return PKV_ERR_INVALID_ARG;
+    int word = 0;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return PKV_ERR_CUDA;
+    if (cudaMemcpy(&word, ctx->d_err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return PKV_ERR_CUDA;
+    if (word && cudaMemset(ctx->d_err, 0, sizeof(int)) != cudaSuccess) return PKV_ERR_CUDA;
+    if (bits) *bits = word;
+    if (word & pkv::kErrTimeout) return PKV_ERR_DEVICE_TIMEOUT;
+    if (word & (pkv::kErrLength | pkv::kErrPage)) return PKV_ERR_DEVICE_BOUNDS;
+    return PKV_OK;
+}
+
+pkv_status pkv_set_workers(pkv_ctx* ctx, int workers)
+{
+    if (!ctx || workers < 0) return PKV_ERR_INVALID_ARG;
+    ctx->workers = workers;
+    return PKV_OK;
+}
+
+size_t pkv_workspace_bytes(const pkv_ctx* ctx) { return ctx ? ctx->ws_bytes : 0; }
+
+}  // extern "C"

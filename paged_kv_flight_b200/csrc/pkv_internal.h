@@ -1,0 +1,67 @@
+// pkv_internal.h -- structures shared by the host API (pkv_api.cu) and the
+// kernel launchers (rope_append.cu, decode_attn.cu).  Not part of the ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/pkv.h"
+
+namespace pkv {
+
+// Device error bits (sticky word in the context workspace).
+enum : int { kErrLength = 1, kErrPage = 2, kErrTimeout = 4 };
+
+constexpr int kTile = 16;          // tokens per attention tile (one TMA box height)
+constexpr int kMaxGroup = 8;       // query heads per kv head handled by one mma row block
+constexpr int kAttnWarps = 8;      // warps per attention CTA (one CTA per SM)
+constexpr int kMinTilesPerWorker = 8;
+constexpr int kMaxBatch = 8192;
+
+struct RopeParams {
+    __nv_bfloat16* q;
+    const __nv_bfloat16* k_new;
+    const __nv_bfloat16* v_new;
+    void* k_pool;
+    void* v_pool;
+    const float* k_scale;
+    const float* v_scale;
+    const int32_t* block_tables;
+    const int32_t* seq_lens;
+    int* err;
+    double rope_base;
+    int batch, bt_stride, Hq, Hkv, D, P, num_pages, fp8;
+};
+
+struct AttnParams {
+    const __nv_bfloat16* q;
+    __nv_bfloat16* out;
+    const float* k_scale;
+    const float* v_scale;
+    const int32_t* block_tables;
+    const int32_t* seq_lens;
+    float* part_o;        // [2 * max_workers][kMaxGroup][D] fp32, unnormalised
+    float* part_ml;       // [2 * max_workers][kMaxGroup][2] fp32 (m in log2 units, l)
+    int* counters;        // [max_batch * Hkv] arrivals per (request, kv head)
+    int* err;
+    float scale_log2;     // log2(e) / sqrt(d)
+    int batch, bt_stride, Hq, Hkv, G, P, num_pages;
+    int stages;           // pipeline depth per warp
+    int workers;          // 0: automatic
+};
+
+cudaError_t launch_rope_append(const RopeParams& p, cudaStream_t stream);
+
+// Host-side shape of the attention launch for a given head_dim / kv type.
+struct AttnLaunch {
+    int ctas;
+    int stages;
+    size_t smem_bytes;
+};
+cudaError_t attn_prepare(int head_dim, bool fp8, int num_sms, int max_batch, AttnLaunch* out);
+cudaError_t launch_decode_attn(const AttnParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
+                               int head_dim, bool fp8, const AttnLaunch& L, cudaStream_t stream);
+
+}  // namespace pkv

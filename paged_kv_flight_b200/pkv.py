@@ -1,0 +1,163 @@
+"""Thin ctypes binding of libpkv (``include/pkv.h``): the same function names,
+argument marshalling only.  Every step of the decode step runs in the CUDA
+kernels of ``libpkv.so``; this module never computes any of it.
+
+The library is loaded at import.  If it has not been built the import fails
+with an ImportError (build it with ``python -m paged_kv_flight_b200.build``);
+there is no fallback path.
+
+Tensors may be passed as torch tensors (their device pointer is used; they
+must be contiguous) or as raw integer device pointers.  ``stream`` may be a
+``torch.cuda.Stream``, a raw ``cudaStream_t`` integer, or None for torch's
+current stream.  Each call returns its ``pkv_status``; with ``check=True``
+(the default) a non-OK status raises :class:`PkvError` instead.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpkv.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(f"libpkv.so is not built ({_LIB_PATH}); run `python -m paged_kv_flight_b200.build`")
+lib = C.CDLL(_LIB_PATH)
+
+PKV_OK = 0
+PKV_ERR_INVALID_ARG = 1
+PKV_ERR_UNSUPPORTED = 2
+PKV_ERR_CUDA = 3
+PKV_ERR_OOM = 4
+PKV_ERR_DEVICE_BOUNDS = 5
+PKV_ERR_DEVICE_TIMEOUT = 6
+
+PKV_KV_BF16 = 0
+PKV_KV_FP8_E4M3 = 1
+
+# names of every symbol include/pkv.h declares
+EXPORTS = ("pkv_create", "pkv_rope_append", "pkv_decode_attn", "pkv_destroy", "pkv_status_str",
+           "pkv_check_device_error", "pkv_set_workers", "pkv_workspace_bytes")
+
+
+class pkv_config(C.Structure):
+    _fields_ = [("num_q_heads", C.c_int), ("num_kv_heads", C.c_int), ("head_dim", C.c_int),
+                ("page_size", C.c_int), ("kv_dtype", C.c_int), ("rope_base", C.c_double),
+                ("max_batch", C.c_int), ("max_blocks_per_seq", C.c_int), ("num_pages", C.c_int)]
+
+
+_V = C.c_void_p
+lib.pkv_create.argtypes = [C.POINTER(pkv_config), C.POINTER(_V)]
+lib.pkv_create.restype = C.c_int
+lib.pkv_rope_append.argtypes = [_V, _V, _V, _V, _V, _V, _V, _V, _V, C.c_int, _V, C.c_int, _V]
+lib.pkv_rope_append.restype = C.c_int
+lib.pkv_decode_attn.argtypes = [_V, _V, _V, _V, _V, _V, _V, C.c_int, _V, C.c_int, _V, _V]
+lib.pkv_decode_attn.restype = C.c_int
+lib.pkv_destroy.argtypes = [_V]
+lib.pkv_destroy.restype = C.c_int
+lib.pkv_status_str.argtypes = [C.c_int]
+lib.pkv_status_str.restype = C.c_char_p
+lib.pkv_check_device_error.argtypes = [_V, _V, C.POINTER(C.c_int)]
+lib.pkv_check_device_error.restype = C.c_int
+lib.pkv_set_workers.argtypes = [_V, C.c_int]
+lib.pkv_set_workers.restype = C.c_int
+lib.pkv_workspace_bytes.argtypes = [_V]
+lib.pkv_workspace_bytes.restype = C.c_size_t
+
+
+class PkvError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {pkv_status_str(status)} (status {status})")
+        self.status = status
+
+
+def pkv_status_str(status: int) -> str:
+    return lib.pkv_status_str(int(status)).decode()
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if isinstance(x, torch.Tensor):
+        if not x.is_contiguous():
+            raise ValueError("libpkv takes contiguous tensors")
+        return x.data_ptr()
+    raise TypeError(f"expected a tensor or a device pointer, got {type(x)}")
+
+
+def _stream(s):
+    if s is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(s, torch.cuda.Stream):
+        return s.cuda_stream
+    return int(s)
+
+
+def _done(status: int, where: str, check: bool) -> int:
+    if check and status != PKV_OK:
+        raise PkvError(status, where)
+    return status
+
+
+def make_config(num_q_heads, num_kv_heads, head_dim, page_size, kv_dtype, rope_base, max_batch,
+                max_blocks_per_seq, num_pages) -> pkv_config:
+    kv = kv_dtype if isinstance(kv_dtype, int) else (PKV_KV_FP8_E4M3 if kv_dtype in ("fp8", "e4m3") else PKV_KV_BF16)
+    return pkv_config(num_q_heads, num_kv_heads, head_dim, page_size, kv, float(rope_base), max_batch,
+                      max_blocks_per_seq, num_pages)
+
+
+def pkv_create(cfg: pkv_config, check: bool = True):
+    """Returns the context handle (an int), or (status, None) with check=False."""
+    h = _V()
+    st = lib.pkv_create(C.byref(cfg), C.byref(h))
+    if not check:
+        return st, (h.value if st == PKV_OK else None)
+    _done(st, "pkv_create", True)
+    return h.value
+
+
+def pkv_rope_append(ctx, q, k_new, v_new, k_pool, v_pool, k_scale, v_scale, block_tables, seq_lens,
+                    batch: int | None = None, bt_stride: int | None = None, stream=None,
+                    check: bool = True) -> int:
+    if batch is None:
+        batch = int(seq_lens.shape[0])
+    if bt_stride is None:
+        bt_stride = int(block_tables.shape[1])
+    st = lib.pkv_rope_append(ctx, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_pool), _ptr(v_pool),
+                             _ptr(k_scale), _ptr(v_scale), _ptr(block_tables), int(bt_stride),
+                             _ptr(seq_lens), int(batch), _stream(stream))
+    return _done(st, "pkv_rope_append", check)
+
+
+def pkv_decode_attn(ctx, q, k_pool, v_pool, k_scale, v_scale, block_tables, seq_lens, out,
+                    batch: int | None = None, bt_stride: int | None = None, stream=None,
+                    check: bool = True) -> int:
+    if batch is None:
+        batch = int(seq_lens.shape[0])
+    if bt_stride is None:
+        bt_stride = int(block_tables.shape[1])
+    st = lib.pkv_decode_attn(ctx, _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(k_scale), _ptr(v_scale),
+                             _ptr(block_tables), int(bt_stride), _ptr(seq_lens), int(batch), _ptr(out),
+                             _stream(stream))
+    return _done(st, "pkv_decode_attn", check)
+
+
+def pkv_destroy(ctx, check: bool = True) -> int:
+    return _done(lib.pkv_destroy(ctx), "pkv_destroy", check)
+
+
+def pkv_check_device_error(ctx, stream=None):
+    """(status, raw error bits); synchronises the stream."""
+    bits = C.c_int(0)
+    st = lib.pkv_check_device_error(ctx, _stream(stream), C.byref(bits))
+    return st, bits.value
+
+
+def pkv_set_workers(ctx, workers: int, check: bool = True) -> int:
+    return _done(lib.pkv_set_workers(ctx, int(workers)), "pkv_set_workers", check)
+
+
+def pkv_workspace_bytes(ctx) -> int:
+    return int(lib.pkv_workspace_bytes(ctx))

@@ -1,0 +1,83 @@
+"""Host-side logic of bench.py on CPU: byte accounting, request sampling, the
+reference (oracle) arm, and the max/sum-over-ranks reductions with two gloo
+ranks."""
+import json
+import os
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from paged_kv_flight_b200 import workloads  # noqa: E402
+
+
+def test_metric_bytes_by_hand():
+    # two requests, L = 0 and 15 -> n = 1 and 16 tokens; Hkv 2, d 64, bf16
+    kv = 2 * 2 * (1 + 16) * 64 * 2
+    qo = 2 * 2 * 8 * 64 * 2
+    assert bench.metric_bytes([0, 15], 8, 2, 64, 16, False) == kv + qo
+    # E4M3: one byte per element plus two fp32 scales per attended (page, kv head)
+    kv8 = 2 * 2 * (1 + 16) * 64 * 1
+    scales = 2 * (1 + 1) * 2 * 4
+    assert bench.metric_bytes([0, 15], 8, 2, 64, 16, True) == kv8 + qo + scales
+
+
+def test_llama8b_bytes_near_the_recipe_estimate():
+    w_lens = workloads.draw_lengths("llama8b", np.random.default_rng(workloads.config_seed("llama8b")))
+    by = bench.metric_bytes(w_lens, 32, 8, 128, 32, False)
+    assert 4.5e8 < by < 6.5e8
+
+
+def test_sample_requests_respects_budget():
+    w = workloads.make("tiny")
+    picks = bench.sample_requests(w, 100)
+    assert picks == [0]                      # at least one request
+    picks = bench.sample_requests(w, 10**9)
+    assert picks == list(range(w.batch))
+
+
+def test_reference_arm_prints_one_json_line_on_cpu():
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config",
+                        "tiny", "--steps", "3", "--warmup", "3"], capture_output=True, text=True, env=env,
+                       timeout=600, check=True)
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "GB/s" and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def _rank_main(rank, world, port, q):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        mx = bench.max_over_ranks(1.5 + rank)
+        sm = bench.sum_over_ranks(10.0 * (rank + 1))
+        bench.barrier()
+        q.put((rank, mx, sm))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_rank_reductions_with_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 29500 + (os.getpid() % 1000)
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(2))
+    assert [r[1] for r in res] == [2.5, 2.5]
+    assert [r[2] for r in res] == [30.0, 30.0]

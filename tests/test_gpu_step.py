@@ -1,0 +1,298 @@
+"""GPU parity: the CUDA path, called through the C ABI, against the CPU oracle.
+
+Small cases (several tiles, ragged tails, every page size / head_dim / group
+size / KV type) are compared element by element on the whole output and the
+whole pools.  The five named workloads run in the benchmark's launch
+configuration; at full size the oracle recomputes sampled requests one by one
+from the generator's original inputs.
+
+Bars: appended V bit-exact, appended K (and rotated q) within 1 bf16 ulp /
+1 E4M3 code step, every other pool byte untouched; attention max abs error
+<= 1e-2 and mean <= 1e-3 for bf16 KV, <= 6e-2 / 6e-3 for E4M3 KV."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from paged_kv_flight_b200 import workloads
+from tests import _gpu
+from tests._util import bf16_ordinal, bits16, bytes8, host_inputs, oracle_cfg, oracle_step
+
+pytestmark = pytest.mark.gpu
+
+SMALL = [
+    # name, Hq, Hkv, d, P, fp8, lengths
+    ("g4_d128_p32_bf16", 32, 8, 128, 32, False, [0, 1, 15, 16, 17, 31, 100, 257, 1000, 4095]),
+    ("g8_d128_p16_bf16", 64, 8, 128, 16, False, [5, 64, 200, 511, 2049]),
+    ("g4_d128_p64_bf16", 32, 8, 128, 64, False, [63, 64, 65, 3000]),
+    ("g1_d64_p16_bf16", 4, 4, 64, 16, False, [2, 77, 300]),
+    ("g2_d64_p32_bf16", 8, 4, 64, 32, False, [31, 32, 999]),
+    ("g4_d128_p32_fp8", 32, 8, 128, 32, True, [0, 16, 33, 700, 2500]),
+    ("g8_d128_p16_fp8", 64, 8, 128, 16, True, [7, 130, 1100]),
+    ("g4_d64_p16_fp8", 8, 2, 64, 16, True, [3, 40, 500]),
+    ("g2_d128_p64_fp8", 16, 8, 128, 64, True, [100, 1500]),
+]
+
+
+@pytest.fixture(scope="module")
+def pkv():
+    from paged_kv_flight_b200 import pkv as mod
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return mod
+
+
+def _small(case, seed=101):
+    name, Hq, Hkv, d, P, fp8, lengths = case
+    return workloads.build(name, Hq, Hkv, d, P, fp8, 5e5 if d == 128 else 1e4, lengths, seed, device="cpu")
+
+
+def _check_append(w, h_oracle, dv):
+    """GPU pools/q after the step against the oracle's, on host copies."""
+    gq = bits16(dv["q"])
+    assert np.abs(bf16_ordinal(gq) - bf16_ordinal(h_oracle["q"])).max() <= 1
+    conv = bytes8 if w.kv_fp8 else bits16
+    gk, gv = conv(dv["k_pool"]), conv(dv["v_pool"])
+    assert np.array_equal(gv, h_oracle["v_pool"]), "appended V must be bit-exact, nothing else touched"
+    diff = gk != h_oracle["k_pool"]
+    if diff.any():
+        rows = {tuple(r[:3]) for r in np.argwhere(diff)}
+        landing = {(int(w.block_tables[b, L // w.P]), kvh, int(L % w.P))
+                   for b, L in enumerate(w.seq_lens) for kvh in range(w.Hkv)}
+        assert rows <= landing, "K differs outside the landing slots"
+        if w.kv_fp8:
+            assert np.abs(gk[diff].astype(int) - h_oracle["k_pool"][diff].astype(int)).max() <= 1
+        else:
+            assert np.abs(bf16_ordinal(gk[diff]) - bf16_ordinal(h_oracle["k_pool"][diff])).max() <= 1
+
+
+@pytest.mark.parametrize("case", SMALL + [("tiny",)], ids=lambda c: c[0])
+def test_small_step_matches_oracle(pkv, case):
+    w = workloads.make("tiny") if case[0] == "tiny" else _small(case)
+    h, ref, st = oracle_step(w)
+    assert st == 0
+    dv = _gpu.to_device(w)
+    ctx = _gpu.make_ctx(pkv, w)
+    try:
+        out = _gpu.gpu_step(pkv, ctx, dv)
+        assert pkv.pkv_check_device_error(ctx)[0] == pkv.PKV_OK
+    finally:
+        pkv.pkv_destroy(ctx)
+    _check_append(w, h, dv)
+    mx, mean, finite = _gpu.errors(out, ref)
+    t = _gpu.tol(w)
+    assert finite, "non-finite output: a stray read of a NaN sentinel"
+    assert mx <= t["max"] and mean <= t["mean"], (mx, mean)
+
+
+def _sample(w, k=4, seed=0):
+    rng = np.random.default_rng(seed)
+    L = w.seq_lens
+    picks = {int(np.argmax(L)), int(np.argmin(L))}
+    picks |= set(int(x) for x in rng.choice(w.batch, size=min(k, w.batch), replace=False))
+    return sorted(picks)
+
+
+@pytest.mark.parametrize("name", ["llama8b", "hetero70b", "longctx", "fp8"])
+def test_full_size_sampled_requests_match_oracle(pkv, name):
+    w = workloads.make(name, device="cuda")
+    kvh_list = None if name != "longctx" else [0, 5]
+    picks = _sample(w, k=2 if name == "longctx" else 5)
+    views = {b: _gpu.request_view(w, b) for b in picks}          # original inputs, before the step
+    k_before = w.k_pool.clone()
+    dv = _gpu.to_device(w)
+    ctx = _gpu.make_ctx(pkv, w)
+    try:
+        out = _gpu.gpu_step(pkv, ctx, dv)
+        assert pkv.pkv_check_device_error(ctx)[0] == pkv.PKV_OK
+    finally:
+        pkv.pkv_destroy(ctx)
+    assert torch.isfinite(out.float()).all()
+    # exactly the landing rows of K changed
+    bitview = (lambda t: t) if w.kv_fp8 else (lambda t: t.view(torch.int16))   # NaN sentinels: compare bits
+    changed = (bitview(dv["k_pool"]) != bitview(k_before)).any(-1).nonzero().cpu().numpy()
+    landing = {(int(w.block_tables[b, L // w.P]), kvh, int(L % w.P))
+               for b, L in enumerate(w.seq_lens) for kvh in range(w.Hkv)}
+    assert {tuple(map(int, r)) for r in changed} <= landing
+    del k_before
+    t = _gpu.tol(w)
+    G = w.Hq // w.Hkv
+    for b in picks:
+        cfg, h = views[b]
+        oracle.rope_append(cfg, h["q"], h["k_new"], h["v_new"], h["k_pool"], h["v_pool"], h["k_scale"],
+                           h["v_scale"], h["block_tables"], h["seq_lens"])
+        ref = np.full((w.Hq, w.d), np.nan)
+        for kvh in (range(w.Hkv) if kvh_list is None else kvh_list):
+            o, st = oracle.decode_attn_group(cfg, h["q"], h["k_pool"], h["v_pool"], h["k_scale"],
+                                             h["v_scale"], h["block_tables"], h["seq_lens"], 0, kvh)
+            assert st == 0
+            ref[kvh * G:(kvh + 1) * G] = o
+        mx, mean, finite = _gpu.errors(out[b], ref)
+        assert finite and mx <= t["max"] and mean <= t["mean"], (b, mx, mean)
+        # the appended V row of this request is bit-exact with the oracle's
+        L = int(w.seq_lens[b])
+        page = int(w.block_tables[b, L // w.P])
+        conv = bytes8 if w.kv_fp8 else bits16
+        gv = conv(dv["v_pool"][page, :, L % w.P])
+        assert np.array_equal(gv, h["v_pool"][L // w.P, :, L % w.P])
+
+
+@pytest.mark.parametrize("case_name", ["g4_d128_p32_bf16", "g4_d128_p32_fp8", "llama8b"])
+def test_split_count_invariance(pkv, case_name):
+    if case_name == "llama8b":
+        w = workloads.make("llama8b", device="cuda")
+    else:
+        w = _small(next(c for c in SMALL if c[0] == case_name))
+    dv = _gpu.to_device(w)
+    ctx = _gpu.make_ctx(pkv, w)
+    outs = []
+    try:
+        pkv.pkv_rope_append(ctx, dv["q"], dv["k_new"], dv["v_new"], dv["k_pool"], dv["v_pool"],
+                            dv["k_scale"], dv["v_scale"], dv["block_tables"], dv["seq_lens"])
+        for workers in (1, 2, 7, 100, 0):
+            pkv.pkv_set_workers(ctx, workers)
+            out = torch.empty(w.batch, w.Hq, w.d, dtype=torch.bfloat16, device="cuda")
+            pkv.pkv_decode_attn(ctx, dv["q"], dv["k_pool"], dv["v_pool"], dv["k_scale"], dv["v_scale"],
+                                dv["block_tables"], dv["seq_lens"], out)
+            outs.append(out.float())
+        assert pkv.pkv_check_device_error(ctx)[0] == pkv.PKV_OK
+    finally:
+        pkv.pkv_destroy(ctx)
+    # a different split reorders fp32 sums (and the running max), which can move
+    # the bf16 output by an ulp or two: bound the mutual difference at 4 ulps
+    for o in outs[1:]:
+        bound = 2.0 ** -6 * torch.maximum(o.abs(), outs[0].abs()) + 1e-5
+        assert bool(((o - outs[0]).abs() <= bound).all())
+    if case_name != "llama8b":
+        _, ref, _ = oracle_step(w)
+        for o in outs:
+            mx, mean, _ = _gpu.errors(o, ref)
+            assert mx <= _gpu.tol(w)["max"] and mean <= _gpu.tol(w)["mean"]
+
+
+def test_one_token_context_returns_v_exactly(pkv):
+    w = workloads.build("one", 32, 8, 128, 32, False, 5e5, [0, 0, 0, 0], seed=3)
+    dv = _gpu.to_device(w)
+    ctx = _gpu.make_ctx(pkv, w)
+    try:
+        out = _gpu.gpu_step(pkv, ctx, dv)
+    finally:
+        pkv.pkv_destroy(ctx)
+    G = w.Hq // w.Hkv
+    want = w.v_new.to("cuda").repeat_interleave(G, dim=1)
+    assert torch.equal(out.view(torch.int16), want.view(torch.int16))
+
+
+def test_identical_keys_and_page_permutation(pkv):
+    w = _small(SMALL[0], seed=7)
+    dv = _gpu.to_device(w)
+    gen = torch.Generator(device="cuda").manual_seed(9)
+    key = torch.randn(w.Hkv, w.d, generator=gen, device="cuda").to(torch.bfloat16)
+    # test-written K (identical in every attended slot) and V (random) for every attended slot
+    for b, L in enumerate(w.seq_lens):
+        for t in range(int(L) + 1):
+            page = int(w.block_tables[b, t // w.P])
+            dv["k_pool"][page, :, t % w.P, :] = key
+            dv["v_pool"][page, :, t % w.P, :] = torch.randn(w.Hkv, w.d, generator=gen, device="cuda").to(torch.bfloat16)
+    ctx = _gpu.make_ctx(pkv, w)
+    try:
+        out = torch.empty(w.batch, w.Hq, w.d, dtype=torch.bfloat16, device="cuda")
+        pkv.pkv_decode_attn(ctx, dv["q"], dv["k_pool"], dv["v_pool"], None, None, dv["block_tables"],
+                            dv["seq_lens"], out)
+        # identical keys: the output is the mean of the values
+        G = w.Hq // w.Hkv
+        for b, L in enumerate(w.seq_lens):
+            n = int(L) + 1
+            idx = torch.arange(n)
+            pages = torch.from_numpy(w.block_tables[b][(idx // w.P).numpy()]).long().cuda()
+            V = dv["v_pool"][pages, :, (idx % w.P).cuda(), :].double()          # [n, Hkv, d]
+            mean = V.mean(0).repeat_interleave(G, dim=0)
+            assert (out[b].double() - mean).abs().max().item() <= 1e-2
+        # permuting physical pages (contents moved, table rewritten) changes nothing, bit for bit
+        perm = torch.randperm(w.num_pages, generator=torch.Generator().manual_seed(1)).cuda()
+        k2 = torch.empty_like(dv["k_pool"]); v2 = torch.empty_like(dv["v_pool"])
+        k2[perm] = dv["k_pool"]; v2[perm] = dv["v_pool"]
+        bt = dv["block_tables"].long()
+        bt2 = torch.where(bt >= 0, perm[bt.clamp(min=0)], bt).int().contiguous()
+        out2 = torch.empty_like(out)
+        pkv.pkv_decode_attn(ctx, dv["q"], k2, v2, None, None, bt2, dv["seq_lens"], out2)
+        assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
+    finally:
+        pkv.pkv_destroy(ctx)
+
+
+def test_repeated_attention_is_deterministic(pkv):
+    w = workloads.make("hetero70b", device="cuda")
+    dv = _gpu.to_device(w)
+    ctx = _gpu.make_ctx(pkv, w)
+    try:
+        out1 = _gpu.gpu_step(pkv, ctx, dv)
+        out2 = torch.empty_like(out1)
+        pkv.pkv_decode_attn(ctx, dv["q"], dv["k_pool"], dv["v_pool"], None, None, dv["block_tables"],
+                            dv["seq_lens"], out2)
+        assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+    finally:
+        pkv.pkv_destroy(ctx)
+
+
+# ---- errors: host-side rejections and device-side range checks (no trap) ------
+
+def test_host_side_rejections(pkv):
+    w = _small(SMALL[0])
+    dv = _gpu.to_device(w)
+    ctx = _gpu.make_ctx(pkv, w)
+    out = torch.empty(w.batch, w.Hq, w.d, dtype=torch.bfloat16, device="cuda")
+    try:
+        args = [dv["k_pool"], dv["v_pool"], None, None, dv["block_tables"], dv["seq_lens"]]
+        st = pkv.pkv_decode_attn(ctx, dv["q"].data_ptr() + 2, *args, out, check=False)
+        assert st == pkv.PKV_ERR_INVALID_ARG                      # misaligned q
+        st = pkv.pkv_decode_attn(ctx, dv["q"], *args, out, batch=w.batch + 1, check=False)
+        assert st == pkv.PKV_ERR_INVALID_ARG                      # batch > max_batch
+        st = pkv.pkv_decode_attn(ctx, dv["q"], *args, out, bt_stride=w.bt_stride + 1, check=False)
+        assert st == pkv.PKV_ERR_INVALID_ARG                      # bt_stride > max
+        st = pkv.pkv_decode_attn(ctx, dv["q"], *args, out, batch=0, check=False)
+        assert st == pkv.PKV_OK                                   # empty batch: no-op
+        st = pkv.pkv_rope_append(ctx, dv["q"], dv["k_new"], dv["v_new"], None, dv["v_pool"], None, None,
+                                 dv["block_tables"], dv["seq_lens"], check=False)
+        assert st == pkv.PKV_ERR_INVALID_ARG
+    finally:
+        pkv.pkv_destroy(ctx)
+    wf = _small(SMALL[5])
+    dvf = _gpu.to_device(wf)
+    ctx = _gpu.make_ctx(pkv, wf)
+    try:
+        st = pkv.pkv_rope_append(ctx, dvf["q"], dvf["k_new"], dvf["v_new"], dvf["k_pool"], dvf["v_pool"], None,
+                                 None, dvf["block_tables"], dvf["seq_lens"], check=False)
+        assert st == pkv.PKV_ERR_INVALID_ARG                      # fp8 pools need scales
+    finally:
+        pkv.pkv_destroy(ctx)
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_device_range_errors_are_reported_not_trapped(pkv, fp8):
+    case = SMALL[5] if fp8 else SMALL[0]
+    w = _small(case, seed=5)
+    h, ref, _ = oracle_step(w)
+    dv = _gpu.to_device(w)
+    bad_page_req, bad_len_req = w.batch - 1, 1     # longest request: page 0 is resident, not landing
+    # a resident page id out of range (not the landing page), and a length past the table
+    dv["block_tables"][bad_page_req, 0] = w.num_pages + 5
+    dv["seq_lens"][bad_len_req] = w.bt_stride * w.P
+    ctx = _gpu.make_ctx(pkv, w)
+    try:
+        out = _gpu.gpu_step(pkv, ctx, dv)
+        st, bits = pkv.pkv_check_device_error(ctx)
+        assert st == pkv.PKV_ERR_DEVICE_BOUNDS and bits & 1 and bits & 2
+        assert pkv.pkv_check_device_error(ctx) == (pkv.PKV_OK, 0)    # cleared after reading
+        assert torch.count_nonzero(out[bad_len_req].float()) == 0      # impossible length -> zeros
+        keep = [b for b in range(w.batch) if b not in (bad_page_req, bad_len_req)]
+        mx, mean, finite = _gpu.errors(out[keep], ref[keep])
+        t = _gpu.tol(w)
+        assert finite and mx <= t["max"] and mean <= t["mean"]
+        # the context still works afterwards
+        dv2 = _gpu.to_device(w)
+        out2 = _gpu.gpu_step(pkv, ctx, dv2)
+        assert pkv.pkv_check_device_error(ctx)[0] == pkv.PKV_OK
+        mx, mean, finite = _gpu.errors(out2, ref)
+        assert finite and mx <= t["max"]
+    finally:
+        pkv.pkv_destroy(ctx)
