@@ -15,7 +15,7 @@
 //   * every CTA derives tiles-per-request (16 tokens per tile) from seq_lens
 //     and keeps their exclusive prefix in shared memory;
 //   * the flattened sequence of tiles, ordered (request, kv head, tile), is cut
-//     into W equal contiguous ranges, one per warp worker (W <= 8 warps x SMs),
+//     into W equal contiguous ranges, one per warp worker (W <= warps x SMs),
 //     so every worker streams the same number of bytes whatever the length
 //     skew of the batch;
 //   * a (request, kv head) pair that lies inside one worker's range is
@@ -26,12 +26,14 @@
 //
 // Per warp: a private ring of `stages` K+V tile buffers filled by 2-D TMA
 // tile loads (128-byte or 64-byte swizzle) that complete on one mbarrier per
-// stage; the warp's lane 0 issues the loads, the warp consumes: QK^T and P V
+// stage; the warp's lane 0 issues the loads from a double-buffered 32-tile
+// lookahead of page ids (and E4M3 scales), the warp consumes: QK^T and P V
 // on warp-level mma.sync (query heads padded to 16 mma rows), online softmax
-// with quad shuffles, fp32 accumulators.  Every mbarrier wait is bounded in
-// time; a timeout marks the worker dead, sets a device error bit and lets
-// the control flow (and the combine protocol) run to the end without
-// touching data.
+// in log2 units with quad shuffles, fp32 accumulators rescaled only when the
+// running max moves.  The next pair's query fragments are fetched one tile
+// ahead.  Every mbarrier wait is bounded in time; a timeout marks the worker
+// dead, sets a device error bit and lets the control flow (and the combine
+// protocol) run to the end without touching data.
 #include <math.h>
 
 #include "pkv_internal.h"
@@ -86,18 +88,81 @@ __device__ __forceinline__ int seek_request(const int* prefix, int B, int Hkv, l
     return lo;
 }
 
+// Page ids (as TMA row coordinates) and scales of 32 consecutive tiles, one
+// per lane.
+struct Lookahead {
+    int valid;   // 0: past the range, 1: ok, 2: page id out of range
+    int row;
+    float ks, vs;
+};
+
+template <bool FP8>
+__device__ __forceinline__ Lookahead lookahead_fill(const AttnParams& p, const int* prefix, long long x0,
+                                                    long long t_end, int lane)
+{
+    Lookahead la{0, 0, 1.f, 1.f};
+    const long long y = x0 + lane;
+    if (y < t_end) {
+        const int b = seek_request(prefix, p.batch, p.Hkv, y);
+        const int ntb = prefix[b + 1] - prefix[b];
+        const long long r = y - (long long)prefix[b] * p.Hkv;
+        const int kvh = (int)(r / ntb), tt = (int)(r % ntb);
+        const int tok0 = tt * kTile;
+        const int lp = tok0 / p.P;
+        const int page = __ldg(&p.block_tables[(size_t)b * p.bt_stride + lp]);
+        if ((unsigned)page < (unsigned)p.num_pages) {
+            la.valid = 1;
+            la.row = (page * p.Hkv + kvh) * p.P + (tok0 - lp * p.P);
+            if (FP8) {
+                la.ks = __ldg(&p.k_scale[(size_t)page * p.Hkv + kvh]);
+                la.vs = __ldg(&p.v_scale[(size_t)page * p.Hkv + kvh]);
+            }
+        } else {
+            la.valid = 2;
+        }
+    }
+    return la;
+}
+
+// Query fragments of (request b, kv head kvh) for the mma A operand: row g =
+// query head kvh*G + g (zero for g >= G), k-step ks covers d in [16ks, 16ks+16).
+// bf16 path: a0 = d 16ks+2c..+1, a2 = d 16ks+8+2c..+1.  fp8 path (f16 operands):
+// the k order inside a k-step follows the byte layout of E4M3 rows, a0 = d
+// 16ks+4c..+1, a2 = d 16ks+4c+2..+3 (raw bf16 here, converted at pair start).
 template <int D, bool FP8>
-__global__ void __launch_bounds__(kAttnWarps * 32, 1)
+__device__ __forceinline__ void load_q(const AttnParams& p, int b, int kvh, int g, int c4,
+                                       uint32_t (&qa)[D / 16][2])
+{
+    const __nv_bfloat16* qrow = p.q + ((size_t)b * p.Hq + (size_t)kvh * p.G + g) * D;
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+        if (g < p.G) {
+            if constexpr (!FP8) {
+                qa[ks][0] = *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * c4);
+                qa[ks][1] = *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8 + 2 * c4);
+            } else {
+                const uint2 v = *reinterpret_cast<const uint2*>(qrow + 16 * ks + 4 * c4);
+                qa[ks][0] = v.x;
+                qa[ks][1] = v.y;
+            }
+        } else {
+            qa[ks][0] = qa[ks][1] = 0u;
+        }
+    }
+}
+
+template <int D, bool FP8, int WARPS>
+__global__ void __launch_bounds__(WARPS * 32, 1)
 decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                    const AttnParams p)
 {
     using Gm = Geo<D, FP8>;
     constexpr int KSTEPS = D / 16;      // mma k-steps along d for QK^T
     constexpr int NTD = D / 8;          // mma n-tiles along d for P V
-    constexpr int NT = kAttnWarps * 32;
+    constexpr int NT = WARPS * 32;
 
     extern __shared__ uint8_t smem_raw[];
-    __shared__ int s_warp_tot[kAttnWarps];
+    __shared__ int s_warp_tot[WARPS];
     __shared__ int s_bad;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -106,9 +171,9 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t stage_area = (raw + 1023u) & ~1023u;
     uint8_t* const area_ptr = smem_raw + (stage_area - raw);
-    StageInfo* const info_all = reinterpret_cast<StageInfo*>(area_ptr + kAttnWarps * S * Gm::STAGEB);
-    uint8_t* const bar_ptr = reinterpret_cast<uint8_t*>(info_all + kAttnWarps * S);
-    int* const prefix = reinterpret_cast<int*>(bar_ptr + kAttnWarps * S * 8);
+    StageInfo* const info_all = reinterpret_cast<StageInfo*>(area_ptr + WARPS * S * Gm::STAGEB);
+    uint8_t* const bar_ptr = reinterpret_cast<uint8_t*>(info_all + WARPS * S);
+    int* const prefix = reinterpret_cast<int*>(bar_ptr + WARPS * S * 8);
 
     if (tid == 0) {
         s_bad = 0;
@@ -151,7 +216,7 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
     if (s_bad && blockIdx.x == 0) {
         // requests with an impossible length produce zeros and an error bit
         if (tid == 0) atomicOr(p.err, kErrLength);
-        for (int b = warp; b < B; b += kAttnWarps) {
+        for (int b = warp; b < B; b += WARPS) {
             const int L = p.seq_lens[b];
             if (L >= 0 && (long long)L < cap) continue;
             uint32_t* o32 = reinterpret_cast<uint32_t*>(p.out + (size_t)b * p.Hq * D);
@@ -162,7 +227,7 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
     // ---- 2. this warp's range of tiles --------------------------------------------
     const long long T = (long long)prefix[B] * Hkv;
     if (T == 0) return;
-    long long Wl = (long long)gridDim.x * kAttnWarps;
+    long long Wl = (long long)gridDim.x * WARPS;
     if (p.workers > 0) Wl = min(Wl, (long long)p.workers);
     else Wl = min(Wl, (T + kMinTilesPerWorker - 1) / kMinTilesPerWorker);
     Wl = max(1LL, min(Wl, T));
@@ -182,43 +247,25 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
     }
     __syncwarp();
 
-    // ---- 3. producer: 32-tile lookahead of page ids and scales, TMA issue -------
-    long long la_base = t_begin - 64;
-    int la_valid = 0, la_row = 0;
-    float la_ks = 1.f, la_vs = 1.f;
-
-    auto la_fill = [&](long long x0) {
-        la_base = x0;
-        const long long y = x0 + lane;
-        la_valid = 0;
-        if (y < t_end) {
-            const int b = seek_request(prefix, B, Hkv, y);
-            const int ntb = prefix[b + 1] - prefix[b];
-            const long long r = y - (long long)prefix[b] * Hkv;
-            const int kvh = (int)(r / ntb), tt = (int)(r % ntb);
-            const int tok0 = tt * kTile;
-            const int lp = tok0 / P;
-            const int page = __ldg(&p.block_tables[(size_t)b * p.bt_stride + lp]);
-            if ((unsigned)page < (unsigned)p.num_pages) {
-                la_valid = 1;
-                la_row = (page * Hkv + kvh) * P + (tok0 - lp * P);
-                if (FP8) {
-                    la_ks = __ldg(&p.k_scale[(size_t)page * Hkv + kvh]);
-                    la_vs = __ldg(&p.v_scale[(size_t)page * Hkv + kvh]);
-                }
-            } else {
-                la_valid = 2;
-            }
-        }
-    };
+    // ---- 3. producer: double-buffered 32-tile lookahead, TMA issue ----------------
+    long long la_base = t_begin;
+    Lookahead la_cur = lookahead_fill<FP8>(p, prefix, t_begin, t_end, lane);
+    Lookahead la_nxt = lookahead_fill<FP8>(p, prefix, t_begin + 32, t_end, lane);
 
     auto issue = [&](long long x, int s) {
-        if (x >= la_base + 32) la_fill(x);
+        if (x >= la_base + 32) {
+            la_base += 32;
+            la_cur = la_nxt;
+            la_nxt = lookahead_fill<FP8>(p, prefix, la_base + 32, t_end, lane);
+        }
         const int src = (int)(x - la_base);
-        const int v = __shfl_sync(kFull, la_valid, src);
-        const int row = __shfl_sync(kFull, la_row, src);
-        const float ks = __shfl_sync(kFull, la_ks, src);
-        const float vs = __shfl_sync(kFull, la_vs, src);
+        const int v = __shfl_sync(kFull, la_cur.valid, src);
+        const int row = __shfl_sync(kFull, la_cur.row, src);
+        float ks = 1.f, vs = 1.f;
+        if (FP8) {
+            ks = __shfl_sync(kFull, la_cur.ks, src);
+            vs = __shfl_sync(kFull, la_cur.vs, src);
+        }
         if (lane == 0) {
             const uint32_t bar = my_bar0 + 8u * s;
             StageInfo si;
@@ -265,41 +312,45 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
     const int tokV = ((mi & 1) << 3) + ri;          // token row addressed for V (trans)
 
     float o[NTD][2];
-    uint32_t qa[KSTEPS][2];
+    uint32_t qa[KSTEPS][2], qn[KSTEPS][2];
     float m_run = -INFINITY, l_run = 0.f;
-    int n_cur = 0;
+    int n_cur = 0, n_next = 0;
     bool dead = false;
     int k_dead = 0;
+    int s = 0;
+    uint32_t parity = 0;
+
+    load_q<D, FP8>(p, cb, ckvh, g, c4, qn);
+    n_next = p.seq_lens[cb] + 1;
 
     for (int k = 0; k < ntiles; ++k) {
-        const int s = k % S;
-        const uint32_t parity = (uint32_t)((k / S) & 1);
-
         if (ctt == 0 || k == 0) {
-            // start of a (request, kv head) pair in this range: query fragments
-            n_cur = p.seq_lens[cb] + 1;
-            const __nv_bfloat16* qrow = p.q + ((size_t)cb * p.Hq + (size_t)ckvh * G + g) * D;
+            // start of a (request, kv head) pair: take the prefetched query
 #pragma unroll
             for (int ks = 0; ks < KSTEPS; ++ks) {
-                if (g < G) {
-                    if (!FP8) {
-                        qa[ks][0] = *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * c4);
-                        qa[ks][1] = *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8 + 2 * c4);
-                    } else {
-                        // fp8 path: k-order inside a k-step follows the byte layout of
-                        // the E4M3 rows (4 consecutive d per quad lane), operands in f16
-                        const uint2 v = *reinterpret_cast<const uint2*>(qrow + 16 * ks + 4 * c4);
-                        qa[ks][0] = pack_f16(bf16_lo(v.x), bf16_hi(v.x));
-                        qa[ks][1] = pack_f16(bf16_lo(v.y), bf16_hi(v.y));
-                    }
+                if constexpr (!FP8) {
+                    qa[ks][0] = qn[ks][0];
+                    qa[ks][1] = qn[ks][1];
                 } else {
-                    qa[ks][0] = qa[ks][1] = 0u;
+                    qa[ks][0] = pack_f16(bf16_lo(qn[ks][0]), bf16_hi(qn[ks][0]));
+                    qa[ks][1] = pack_f16(bf16_lo(qn[ks][1]), bf16_hi(qn[ks][1]));
                 }
             }
+            n_cur = n_next;
 #pragma unroll
             for (int nt = 0; nt < NTD; ++nt) o[nt][0] = o[nt][1] = 0.f;
             m_run = -INFINITY;
             l_run = 0.f;
+        }
+        if (ctt == cnt - 1 && k + 1 < ntiles) {
+            // this tile ends the pair: fetch the next pair's query now
+            int nb = cb, nkvh = ckvh + 1;
+            if (nkvh == Hkv) {
+                nkvh = 0;
+                do { ++nb; } while (nb < B - 1 && prefix[nb + 1] == prefix[nb]);
+            }
+            load_q<D, FP8>(p, nb, nkvh, g, c4, qn);
+            n_next = p.seq_lens[nb] + 1;
         }
 
         if (!dead) {
@@ -311,6 +362,7 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
             }
         }
 
+        bool zeroed = false;
         if (!dead && my_info[s].valid) {
             const StageInfo si = my_info[s];
             const uint32_t kb = my_stage0 + (uint32_t)(s * Gm::STAGEB);
@@ -327,52 +379,57 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
                                  "r"(0u)
                                  : "memory");
                 }
+                zeroed = true;
                 __syncwarp();
             }
 
-            // S = Q K^T (two n-tiles of 8 tokens)
-            float sc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
-            if (!FP8) {
+            // S = Q K^T (two n-tiles of 8 tokens), two accumulation chains
+            float sa[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, sb[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+            if constexpr (!FP8) {
 #pragma unroll
-                for (int ks = 0; ks < KSTEPS; ++ks) {
-                    uint32_t r0, r1, r2, r3;
+                for (int ks = 0; ks < KSTEPS; ks += 2) {
+                    uint32_t r0, r1, r2, r3, r4, r5, r6, r7;
                     ldsm_x4(kb + tile_off<D, FP8>(tokK, 2 * ks + (mi & 1)), r0, r1, r2, r3);
-                    mma_bf16_r8(sc[0][0], sc[0][1], qa[ks][0], qa[ks][1], r0, r1);
-                    mma_bf16_r8(sc[1][0], sc[1][1], qa[ks][0], qa[ks][1], r2, r3);
+                    ldsm_x4(kb + tile_off<D, FP8>(tokK, 2 * ks + 2 + (mi & 1)), r4, r5, r6, r7);
+                    mma_bf16_r8(sa[0][0], sa[0][1], qa[ks][0], qa[ks][1], r0, r1);
+                    mma_bf16_r8(sa[1][0], sa[1][1], qa[ks][0], qa[ks][1], r2, r3);
+                    mma_bf16_r8(sb[0][0], sb[0][1], qa[ks + 1][0], qa[ks + 1][1], r4, r5);
+                    mma_bf16_r8(sb[1][0], sb[1][1], qa[ks + 1][0], qa[ks + 1][1], r6, r7);
                 }
             } else {
 #pragma unroll
                 for (int s4 = 0; s4 < D / 32; ++s4) {
                     uint32_t r0, r1, r2, r3;
                     ldsm_x4(kb + tile_off<D, FP8>(tokK, 2 * s4 + (mi & 1)), r0, r1, r2, r3);
-                    mma_f16_r8(sc[0][0], sc[0][1], qa[2 * s4][0], qa[2 * s4][1], cvt_lo(r0), cvt_hi(r0));
-                    mma_f16_r8(sc[0][0], sc[0][1], qa[2 * s4 + 1][0], qa[2 * s4 + 1][1], cvt_lo(r1), cvt_hi(r1));
-                    mma_f16_r8(sc[1][0], sc[1][1], qa[2 * s4][0], qa[2 * s4][1], cvt_lo(r2), cvt_hi(r2));
-                    mma_f16_r8(sc[1][0], sc[1][1], qa[2 * s4 + 1][0], qa[2 * s4 + 1][1], cvt_lo(r3), cvt_hi(r3));
+                    mma_f16_r8(sa[0][0], sa[0][1], qa[2 * s4][0], qa[2 * s4][1], cvt_lo(r0), cvt_hi(r0));
+                    mma_f16_r8(sb[0][0], sb[0][1], qa[2 * s4 + 1][0], qa[2 * s4 + 1][1], cvt_lo(r1), cvt_hi(r1));
+                    mma_f16_r8(sa[1][0], sa[1][1], qa[2 * s4][0], qa[2 * s4][1], cvt_lo(r2), cvt_hi(r2));
+                    mma_f16_r8(sb[1][0], sb[1][1], qa[2 * s4 + 1][0], qa[2 * s4 + 1][1], cvt_lo(r3), cvt_hi(r3));
                 }
             }
 
             // online softmax in log2 units; masked tokens are -inf (never 0 * NaN)
             const float slog2 = FP8 ? p.scale_log2 * si.ks : p.scale_log2;
+            float sc[2][2];
             float mx = -INFINITY;
 #pragma unroll
             for (int j = 0; j < 2; ++j)
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     const int tok = tok0 + 8 * j + 2 * c4 + e;
-                    sc[j][e] = (tok < n_cur) ? sc[j][e] * slog2 : -INFINITY;
+                    sc[j][e] = (tok < n_cur) ? (sa[j][e] + sb[j][e]) * slog2 : -INFINITY;
                     mx = fmaxf(mx, sc[j][e]);
                 }
             mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
             mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
             const float m_new = fmaxf(m_run, mx);
             const float m_ref = (m_new == -INFINITY) ? 0.f : m_new;
-            const float alpha = exp2f(m_run - m_ref);
-            const float p00 = exp2f(sc[0][0] - m_ref), p01 = exp2f(sc[0][1] - m_ref);
-            const float p10 = exp2f(sc[1][0] - m_ref), p11 = exp2f(sc[1][1] - m_ref);
+            const float alpha = ex2(m_run - m_ref);
+            const float p00 = ex2(sc[0][0] - m_ref), p01 = ex2(sc[0][1] - m_ref);
+            const float p10 = ex2(sc[1][0] - m_ref), p11 = ex2(sc[1][1] - m_ref);
             uint32_t pa0, pa2;
             float psum;
-            if (!FP8) {
+            if constexpr (!FP8) {
                 pa0 = pack_bf16(p00, p01);
                 pa2 = pack_bf16(p10, p11);
                 psum = (bf16_lo(pa0) + bf16_hi(pa0)) + (bf16_lo(pa2) + bf16_hi(pa2));
@@ -384,14 +441,16 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
             }
             l_run = l_run * alpha + psum;
             m_run = m_new;
+            if (__any_sync(kFull, alpha != 1.f)) {
 #pragma unroll
-            for (int nt = 0; nt < NTD; ++nt) {
-                o[nt][0] *= alpha;
-                o[nt][1] *= alpha;
+                for (int nt = 0; nt < NTD; ++nt) {
+                    o[nt][0] *= alpha;
+                    o[nt][1] *= alpha;
+                }
             }
 
             // O += P V
-            if (!FP8) {
+            if constexpr (!FP8) {
 #pragma unroll
                 for (int dj = 0; dj < D / 16; ++dj) {
                     uint32_t r0, r1, r2, r3;
@@ -451,7 +510,9 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
 
         // refill this stage with the tile `S` ahead
         if (!dead && issued < ntiles) {
-            if (lane == 0) fence_proxy_async_smem();
+            // generic-proxy zero stores above must land before the async-proxy
+            // copy that overwrites the buffer
+            if (zeroed && lane == 0) fence_proxy_async_smem();
             issue(t_begin + issued, s);
             ++issued;
         }
@@ -469,7 +530,7 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
                 if (g < G) {
                     const float inv = 1.f / lsum;
                     uint32_t* dst = reinterpret_cast<uint32_t*>(p.out + orow);
-                    if (!FP8) {
+                    if constexpr (!FP8) {
 #pragma unroll
                         for (int nt = 0; nt < NTD; ++nt)
                             dst[(8 * nt + 2 * c4) >> 1] = pack_bf16(o[nt][0] * inv, o[nt][1] * inv);
@@ -489,7 +550,7 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
                 const size_t prow = ((size_t)slot * kMaxGroup + g) * D;
                 if (g < G) {
                     float* dst = p.part_o + prow;
-                    if (!FP8) {
+                    if constexpr (!FP8) {
 #pragma unroll
                         for (int nt = 0; nt < NTD; ++nt)
                             *reinterpret_cast<float2*>(dst + 8 * nt + 2 * c4) = make_float2(o[nt][0], o[nt][1]);
@@ -529,7 +590,7 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
                             const int sl = 2 * v + (((long long)v * T / W) < ts ? 1 : 0);
                             const float2 ml = __ldcg(reinterpret_cast<const float2*>(
                                 p.part_ml + ((size_t)sl * kMaxGroup + gg) * 2));
-                            const float f = exp2f(ml.x - mref);
+                            const float f = ex2(ml.x - mref);
                             lt += ml.y * f;
                             const float* src = p.part_o + ((size_t)sl * kMaxGroup + gg) * D + lane * DPL;
                             if constexpr (DPL == 4) {
@@ -552,7 +613,7 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
             }
         }
 
-        // advance the consumer cursor
+        // advance the consumer cursor and the ring position
         if (++ctt == cnt) {
             ctt = 0;
             if (++ckvh == Hkv) {
@@ -560,6 +621,10 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
                 do { ++cb; } while (cb < B && prefix[cb + 1] == prefix[cb]);
             }
             if (cb < B) cnt = prefix[cb + 1] - prefix[cb];
+        }
+        if (++s == S) {
+            s = 0;
+            parity ^= 1u;
         }
     }
 
@@ -588,11 +653,11 @@ cudaError_t prepare_t(int num_sms, int max_batch, AttnLaunch* out)
     e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     if (e != cudaSuccess) return e;
     const size_t budget = (size_t)optin - 256;   // static shared memory of the kernel
-    int stages = 8;
+    int stages = kAttnMaxStages;
     while (stages > 2 && smem_bytes_for<D, FP8>(stages, max_batch) > budget) --stages;
     if (smem_bytes_for<D, FP8>(stages, max_batch) > budget) return cudaErrorInvalidConfiguration;
     const size_t bytes = smem_bytes_for<D, FP8>(stages, max_batch);
-    e = cudaFuncSetAttribute(decode_attn_kernel<D, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(decode_attn_kernel<D, FP8, kAttnWarps>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)bytes);
     if (e != cudaSuccess) return e;
     out->ctas = num_sms;
@@ -617,11 +682,11 @@ cudaError_t launch_decode_attn(const AttnParams& p, const CUtensorMap& tmk, cons
     AttnParams q = p;
     q.stages = L.stages;
     if (head_dim == 128) {
-        if (fp8) decode_attn_kernel<128, true><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
-        else decode_attn_kernel<128, false><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
+        if (fp8) decode_attn_kernel<128, true, kAttnWarps><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
+        else decode_attn_kernel<128, false, kAttnWarps><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
     } else {
-        if (fp8) decode_attn_kernel<64, true><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
-        else decode_attn_kernel<64, false><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
+        if (fp8) decode_attn_kernel<64, true, kAttnWarps><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
+        else decode_attn_kernel<64, false, kAttnWarps><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
     }
     return cudaGetLastError();
 }

@@ -158,6 +158,14 @@ __device__ __forceinline__ void mma_f16_r8(float& d0, float& d1, uint32_t a0, ui
         : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "f"(0.f), "f"(0.f));
 }
 
+// 2^x on the SFU (ex2.approx, denormal results flushed to zero; 2^-inf = 0).
+__device__ __forceinline__ float ex2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // ---- conversions --------------------------------------------------------------
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)

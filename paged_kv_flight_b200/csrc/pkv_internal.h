@@ -14,9 +14,19 @@ namespace pkv {
 // Device error bits (sticky word in the context workspace).
 enum : int { kErrLength = 1, kErrPage = 2, kErrTimeout = 4 };
 
+// Warps per attention CTA (one CTA per SM) and the deepest per-warp TMA
+// ring; both can be overridden at build time for tuning sweeps.
+#ifndef PKV_ATTN_WARPS
+#define PKV_ATTN_WARPS 8
+#endif
+#ifndef PKV_ATTN_MAX_STAGES
+#define PKV_ATTN_MAX_STAGES 2
+#endif
+
 constexpr int kTile = 16;          // tokens per attention tile (one TMA box height)
 constexpr int kMaxGroup = 8;       // query heads per kv head handled by one mma row block
-constexpr int kAttnWarps = 8;      // warps per attention CTA (one CTA per SM)
+constexpr int kAttnWarps = PKV_ATTN_WARPS;
+constexpr int kAttnMaxStages = PKV_ATTN_MAX_STAGES;
 constexpr int kMinTilesPerWorker = 8;
 constexpr int kMaxBatch = 8192;
 

@@ -10,128 +10,145 @@
 // positions to physical blocks) and section "4. Native FP8 Quantization"
 // (E4M3 storage).
 //
-// One CTA per request.  The cos/sin table of the request's position is
-// computed once in fp64 (angle p * theta_i and sincos both in fp64, which
-// keeps the angle exact enough at positions past 10^5), then every q and k
-// row is rotated in fp64 and rounded once to the storage type.  Each thread
-// owns 8 rotation pairs of one row: two 16-byte loads, two 16-byte (bf16) or
-// 8-byte (E4M3) stores.
+// Grid (request, chunk): a request's Hq + Hkv rows are cut into work items of
+// 8 rotation pairs (two 16-byte loads, two 16-byte bf16 or 8-byte E4M3
+// stores), 128 items per CTA.  Each thread issues its row loads first; the
+// CTA meanwhile builds the cos/sin table of the request's position in fp64:
+// angle p * theta_i rounded once, reduced to [-pi, pi] with a two-part 2*pi
+// (Cody & Waite), then sincos.  Rotation is fp64 with separate roundings and
+// one final rounding to the storage type.
 #include "pkv_internal.h"
 #include "pkv_device.cuh"
 
 namespace pkv {
 namespace {
 
+constexpr int kRopeThreads = 128;
+
+// 2*pi = kTwoPiHi + kTwoPiLo; kTwoPiHi is the double nearest 2*pi.
+constexpr double kTwoPiHi = 6.283185307179586;
+constexpr double kTwoPiLo = 2.4492935982947064e-16;
+constexpr double kInvTwoPi = 0.15915494309189535;
+
+__device__ __forceinline__ void sincos_reduced(double phi, double* s, double* c)
+{
+    const double k = rint(phi * kInvTwoPi);
+    double r = fma(-k, kTwoPiHi, phi);
+    r = fma(-k, kTwoPiLo, r);
+    sincos(r, s, c);
+}
+
 template <int D, bool FP8>
-__global__ void __launch_bounds__(128) rope_append_kernel(const RopeParams p)
+__global__ void __launch_bounds__(kRopeThreads) rope_append_kernel(const RopeParams p)
 {
     constexpr int HALF = D / 2;
     constexpr int PIECES = HALF / 8;  // 8 pairs per work item
     __shared__ double s_cos[HALF], s_sin[HALF];
 
     const int b = blockIdx.x;
+    const int rows = p.Hq + p.Hkv;
+    const int it = blockIdx.y * kRopeThreads + threadIdx.x;
+    const bool active = it < rows * PIECES;
+    const int r = it / PIECES;
+    const int i0 = (it % PIECES) * 8;
+    const bool is_q = r < p.Hq;
+    const int kvh = r - p.Hq;
+
+    // loads that do not depend on the position go out first
+    uint4 xa = make_uint4(0, 0, 0, 0), xb = xa, va = xa, vb = xa;
+    if (active) {
+        const __nv_bfloat16* src = is_q ? p.q + ((size_t)b * p.Hq + r) * D
+                                        : p.k_new + ((size_t)b * p.Hkv + kvh) * D;
+        xa = *reinterpret_cast<const uint4*>(src + i0);          // x_i
+        xb = *reinterpret_cast<const uint4*>(src + i0 + HALF);   // x_{i+d/2}
+        if (!is_q) {
+            const __nv_bfloat16* vsrc = p.v_new + ((size_t)b * p.Hkv + kvh) * D;
+            va = *reinterpret_cast<const uint4*>(vsrc + i0);
+            vb = *reinterpret_cast<const uint4*>(vsrc + i0 + HALF);
+        }
+    }
+
     const int L = p.seq_lens[b];
-    if (L < 0 || (long long)L >= (long long)p.bt_stride * p.P) {
-        if (threadIdx.x == 0) atomicOr(p.err, kErrLength);
+    const bool len_ok = L >= 0 && (long long)L < (long long)p.bt_stride * p.P;
+    const int page = len_ok ? p.block_tables[(size_t)b * p.bt_stride + L / p.P] : -1;
+    if (!len_ok) {
+        if (threadIdx.x == 0 && blockIdx.y == 0) atomicOr(p.err, kErrLength);
         return;
     }
-    const int page = p.block_tables[(size_t)b * p.bt_stride + L / p.P];
     if (page < 0 || page >= p.num_pages) {
-        if (threadIdx.x == 0) atomicOr(p.err, kErrPage);
+        if (threadIdx.x == 0 && blockIdx.y == 0) atomicOr(p.err, kErrPage);
         return;
     }
     const int slot = L % p.P;
 
     for (int i = threadIdx.x; i < HALF; i += blockDim.x) {
         const double theta = pow(p.rope_base, (-2.0 * i) / D);
-        const double phi = (double)L * theta;
         double s, c;
-        sincos(phi, &s, &c);
+        sincos_reduced((double)L * theta, &s, &c);
         s_cos[i] = c;
         s_sin[i] = s;
     }
     __syncthreads();
+    if (!active) return;
 
-    const int rows = p.Hq + p.Hkv;
-    for (int it = threadIdx.x; it < rows * PIECES; it += blockDim.x) {
-        const int r = it / PIECES;
-        const int i0 = (it % PIECES) * 8;
-        const bool is_q = r < p.Hq;
-        const int kvh = r - p.Hq;
-        const __nv_bfloat16* src = is_q ? p.q + ((size_t)b * p.Hq + r) * D
-                                        : p.k_new + ((size_t)b * p.Hkv + kvh) * D;
-        const uint4 xa = *reinterpret_cast<const uint4*>(src + i0);          // x_i
-        const uint4 xb = *reinterpret_cast<const uint4*>(src + i0 + HALF);   // x_{i+d/2}
-        const uint32_t wa[4] = {xa.x, xa.y, xa.z, xa.w};
-        const uint32_t wb[4] = {xb.x, xb.y, xb.z, xb.w};
-        double ya[8], yb[8];
+    const uint32_t wa[4] = {xa.x, xa.y, xa.z, xa.w};
+    const uint32_t wb[4] = {xb.x, xb.y, xb.z, xb.w};
+    double ya[8], yb[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const double a = (double)((k & 1) ? dev::bf16_hi(wa[k >> 1]) : dev::bf16_lo(wa[k >> 1]));
+        const double bb = (double)((k & 1) ? dev::bf16_hi(wb[k >> 1]) : dev::bf16_lo(wb[k >> 1]));
+        const double c = s_cos[i0 + k], s = s_sin[i0 + k];
+        // separate roundings, no fused multiply-add
+        ya[k] = __dsub_rn(__dmul_rn(a, c), __dmul_rn(bb, s));
+        yb[k] = __dadd_rn(__dmul_rn(bb, c), __dmul_rn(a, s));
+    }
+
+    const size_t prow = ((size_t)page * p.Hkv + kvh) * p.P + slot;   // pool row (k rows only)
+    if (is_q || !FP8) {
+        uint32_t oa[4], ob[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            oa[k] = (uint32_t)__bfloat16_as_ushort(dev::bf16_from_f64(ya[2 * k])) |
+                    ((uint32_t)__bfloat16_as_ushort(dev::bf16_from_f64(ya[2 * k + 1])) << 16);
+            ob[k] = (uint32_t)__bfloat16_as_ushort(dev::bf16_from_f64(yb[2 * k])) |
+                    ((uint32_t)__bfloat16_as_ushort(dev::bf16_from_f64(yb[2 * k + 1])) << 16);
+        }
+        __nv_bfloat16* dst = is_q ? p.q + ((size_t)b * p.Hq + r) * D
+                                  : reinterpret_cast<__nv_bfloat16*>(p.k_pool) + prow * D;
+        *reinterpret_cast<uint4*>(dst + i0) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
+        *reinterpret_cast<uint4*>(dst + i0 + HALF) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+    }
+    if (is_q) return;
+
+    if (!FP8) {
+        __nv_bfloat16* vdst = reinterpret_cast<__nv_bfloat16*>(p.v_pool) + prow * D;
+        *reinterpret_cast<uint4*>(vdst + i0) = va;
+        *reinterpret_cast<uint4*>(vdst + i0 + HALF) = vb;
+    } else {
+        const size_t si = (size_t)page * p.Hkv + kvh;
+        const double sk = (double)p.k_scale[si];
+        const float sv = p.v_scale[si];
+        const uint32_t vwa[4] = {va.x, va.y, va.z, va.w};
+        const uint32_t vwb[4] = {vb.x, vb.y, vb.z, vb.w};
+        uint8_t ka[8], kb[8], qa8[8], qb8[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-            const double a = (double)((k & 1) ? dev::bf16_hi(wa[k >> 1]) : dev::bf16_lo(wa[k >> 1]));
-            const double bb = (double)((k & 1) ? dev::bf16_hi(wb[k >> 1]) : dev::bf16_lo(wb[k >> 1]));
-            const double c = s_cos[i0 + k], s = s_sin[i0 + k];
-            // separate roundings, no fused multiply-add
-            ya[k] = __dsub_rn(__dmul_rn(a, c), __dmul_rn(bb, s));
-            yb[k] = __dadd_rn(__dmul_rn(bb, c), __dmul_rn(a, s));
+            // k: fp64 quotient rounded once to fp32, then E4M3 RNE satfinite
+            ka[k] = dev::e4m3_satfinite(__double2float_rn(__ddiv_rn(ya[k], sk)));
+            kb[k] = dev::e4m3_satfinite(__double2float_rn(__ddiv_rn(yb[k], sk)));
+            // v: exact bf16 value, IEEE fp32 quotient
+            const float a = (k & 1) ? dev::bf16_hi(vwa[k >> 1]) : dev::bf16_lo(vwa[k >> 1]);
+            const float bb = (k & 1) ? dev::bf16_hi(vwb[k >> 1]) : dev::bf16_lo(vwb[k >> 1]);
+            qa8[k] = dev::e4m3_satfinite(__fdiv_rn(a, sv));
+            qb8[k] = dev::e4m3_satfinite(__fdiv_rn(bb, sv));
         }
-
-        if (is_q || !FP8) {
-            uint32_t oa[4], ob[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const __nv_bfloat16 a0 = dev::bf16_from_f64(ya[2 * k]);
-                const __nv_bfloat16 a1 = dev::bf16_from_f64(ya[2 * k + 1]);
-                const __nv_bfloat16 b0 = dev::bf16_from_f64(yb[2 * k]);
-                const __nv_bfloat16 b1 = dev::bf16_from_f64(yb[2 * k + 1]);
-                oa[k] = (uint32_t)__bfloat16_as_ushort(a0) | ((uint32_t)__bfloat16_as_ushort(a1) << 16);
-                ob[k] = (uint32_t)__bfloat16_as_ushort(b0) | ((uint32_t)__bfloat16_as_ushort(b1) << 16);
-            }
-            __nv_bfloat16* dst;
-            if (is_q) {
-                dst = p.q + ((size_t)b * p.Hq + r) * D;
-            } else {
-                const size_t row = ((size_t)page * p.Hkv + kvh) * p.P + slot;
-                dst = reinterpret_cast<__nv_bfloat16*>(p.k_pool) + row * D;
-            }
-            *reinterpret_cast<uint4*>(dst + i0) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
-            *reinterpret_cast<uint4*>(dst + i0 + HALF) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
-        }
-
-        if (!is_q) {
-            const size_t row = ((size_t)page * p.Hkv + kvh) * p.P + slot;
-            const __nv_bfloat16* vsrc = p.v_new + ((size_t)b * p.Hkv + kvh) * D;
-            const uint4 va = *reinterpret_cast<const uint4*>(vsrc + i0);
-            const uint4 vb = *reinterpret_cast<const uint4*>(vsrc + i0 + HALF);
-            if (!FP8) {
-                __nv_bfloat16* vdst = reinterpret_cast<__nv_bfloat16*>(p.v_pool) + row * D;
-                *reinterpret_cast<uint4*>(vdst + i0) = va;
-                *reinterpret_cast<uint4*>(vdst + i0 + HALF) = vb;
-            } else {
-                const size_t si = (size_t)page * p.Hkv + kvh;
-                const double sk = (double)p.k_scale[si];
-                const float sv = p.v_scale[si];
-                const uint32_t vwa[4] = {va.x, va.y, va.z, va.w};
-                const uint32_t vwb[4] = {vb.x, vb.y, vb.z, vb.w};
-                uint8_t ka[8], kb[8], qa8[8], qb8[8];
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    // k: fp64 quotient rounded once to fp32, then E4M3 RNE satfinite
-                    ka[k] = dev::e4m3_satfinite(__double2float_rn(__ddiv_rn(ya[k], sk)));
-                    kb[k] = dev::e4m3_satfinite(__double2float_rn(__ddiv_rn(yb[k], sk)));
-                    // v: exact bf16 value, IEEE fp32 quotient
-                    const float a = (k & 1) ? dev::bf16_hi(vwa[k >> 1]) : dev::bf16_lo(vwa[k >> 1]);
-                    const float bb = (k & 1) ? dev::bf16_hi(vwb[k >> 1]) : dev::bf16_lo(vwb[k >> 1]);
-                    qa8[k] = dev::e4m3_satfinite(__fdiv_rn(a, sv));
-                    qb8[k] = dev::e4m3_satfinite(__fdiv_rn(bb, sv));
-                }
-                uint8_t* kdst = reinterpret_cast<uint8_t*>(p.k_pool) + row * D;
-                uint8_t* vdst = reinterpret_cast<uint8_t*>(p.v_pool) + row * D;
-                *reinterpret_cast<uint2*>(kdst + i0) = *reinterpret_cast<const uint2*>(ka);
-                *reinterpret_cast<uint2*>(kdst + i0 + HALF) = *reinterpret_cast<const uint2*>(kb);
-                *reinterpret_cast<uint2*>(vdst + i0) = *reinterpret_cast<const uint2*>(qa8);
-                *reinterpret_cast<uint2*>(vdst + i0 + HALF) = *reinterpret_cast<const uint2*>(qb8);
-            }
-        }
+        uint8_t* kdst = reinterpret_cast<uint8_t*>(p.k_pool) + prow * D;
+        uint8_t* vdst = reinterpret_cast<uint8_t*>(p.v_pool) + prow * D;
+        *reinterpret_cast<uint2*>(kdst + i0) = *reinterpret_cast<const uint2*>(ka);
+        *reinterpret_cast<uint2*>(kdst + i0 + HALF) = *reinterpret_cast<const uint2*>(kb);
+        *reinterpret_cast<uint2*>(vdst + i0) = *reinterpret_cast<const uint2*>(qa8);
+        *reinterpret_cast<uint2*>(vdst + i0 + HALF) = *reinterpret_cast<const uint2*>(qb8);
     }
 }
 
@@ -139,7 +156,8 @@ __global__ void __launch_bounds__(128) rope_append_kernel(const RopeParams p)
 
 cudaError_t launch_rope_append(const RopeParams& p, cudaStream_t stream)
 {
-    const dim3 grid(p.batch), block(128);
+    const int items = (p.Hq + p.Hkv) * (p.D / 16);
+    const dim3 grid(p.batch, (items + kRopeThreads - 1) / kRopeThreads), block(kRopeThreads);
     if (p.D == 128) {
         if (p.fp8) rope_append_kernel<128, true><<<grid, block, 0, stream>>>(p);
         else rope_append_kernel<128, false><<<grid, block, 0, stream>>>(p);

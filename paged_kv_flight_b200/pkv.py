@@ -19,7 +19,10 @@ import os
 
 import torch
 
-_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpkv.so")
+# PKV_LIBRARY may point at another build of the same library (e.g. a tuning
+# variant); by default the in-tree build is loaded.
+_LIB_PATH = os.environ.get("PKV_LIBRARY") or os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                                                           "libpkv.so")
 if not os.path.exists(_LIB_PATH):
     raise ImportError(f"libpkv.so is not built ({_LIB_PATH}); run `python -m paged_kv_flight_b200.build`")
 lib = C.CDLL(_LIB_PATH)

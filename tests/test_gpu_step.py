@@ -157,11 +157,13 @@ def test_split_count_invariance(pkv, case_name):
         assert pkv.pkv_check_device_error(ctx)[0] == pkv.PKV_OK
     finally:
         pkv.pkv_destroy(ctx)
-    # a different split reorders fp32 sums (and the running max), which can move
-    # the bf16 output by an ulp or two: bound the mutual difference at 4 ulps
+    # a different split reorders fp32 sums and moves the running max, so the
+    # bf16-rounded probabilities differ: bound the mutual difference at 4 bf16
+    # ulps of the largest output of the same (request, head) row
     for o in outs[1:]:
-        bound = 2.0 ** -6 * torch.maximum(o.abs(), outs[0].abs()) + 1e-5
-        assert bool(((o - outs[0]).abs() <= bound).all())
+        scale = torch.maximum(o.abs().amax(-1, keepdim=True), outs[0].abs().amax(-1, keepdim=True))
+        diff = (o - outs[0]).abs()
+        assert bool((diff <= 2.0 ** -6 * scale + 1e-6).all()), float((diff / scale).max())
     if case_name != "llama8b":
         _, ref, _ = oracle_step(w)
         for o in outs:
