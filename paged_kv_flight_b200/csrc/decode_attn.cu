@@ -151,6 +151,71 @@ __device__ __forceinline__ void load_q(const AttnParams& p, int b, int kvh, int 
     }
 }
 
+// Log-sum-exp merge of the partials that workers wf..wl left for pair (b, kvh)
+// whose first tile is ts (worker v's range starts at v*T/W; its slot for the
+// pair is 2v + 1 if that start lies before ts, else 2v).  One query head at a
+// time: lanes own workers (lane, lane + 32, ...) for the maximum and the
+// weights, and D/32 output columns for the weighted rows, whose loads are
+// issued eight contributors at a time.  Writes the bf16 output rows.
+template <int D>
+__device__ __forceinline__ void merge_partials(const AttnParams& p, int b, int kvh, long long ts, int wf, int wl,
+                                               long long T, int W, int lane)
+{
+    constexpr unsigned kFullMask = 0xFFFFFFFFu;
+    constexpr int DPL = D / 32;
+    const int k = wl - wf + 1;
+    for (int gg = 0; gg < p.G; ++gg) {
+        float m = -INFINITY;
+        for (int i0 = 0; i0 < k; i0 += 32) {
+            const int v = wf + i0 + lane;
+            if (v <= wl) {
+                const int sl = 2 * v + (((long long)v * T / W) < ts ? 1 : 0);
+                m = fmaxf(m, __ldcg(p.part_ml + ((size_t)sl * kMaxGroup + gg) * 2));
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFullMask, m, o));
+        if (m == -INFINITY) m = 0.f;
+        float lt = 0.f, acc[DPL];
+#pragma unroll
+        for (int q = 0; q < DPL; ++q) acc[q] = 0.f;
+        for (int i0 = 0; i0 < k; i0 += 32) {
+            const int v = wf + i0 + lane;
+            int my_sl = 0;
+            float fw = 0.f;
+            if (v <= wl) {
+                my_sl = 2 * v + (((long long)v * T / W) < ts ? 1 : 0);
+                const float2 ml =
+                    __ldcg(reinterpret_cast<const float2*>(p.part_ml + ((size_t)my_sl * kMaxGroup + gg) * 2));
+                fw = ex2(ml.x - m);
+                lt += ml.y * fw;
+            }
+            const int here = min(32, k - i0);
+#pragma unroll 8
+            for (int vv = 0; vv < here; ++vv) {
+                const int sl = __shfl_sync(kFullMask, my_sl, vv);
+                const float f = __shfl_sync(kFullMask, fw, vv);
+                const float* row = p.part_o + ((size_t)sl * kMaxGroup + gg) * D + lane * DPL;
+                if constexpr (DPL == 4) {
+                    const float4 x = __ldcg(reinterpret_cast<const float4*>(row));
+                    acc[0] += f * x.x; acc[1] += f * x.y;
+                    acc[2] += f * x.z; acc[3] += f * x.w;
+                } else {
+                    const float2 x = __ldcg(reinterpret_cast<const float2*>(row));
+                    acc[0] += f * x.x; acc[1] += f * x.y;
+                }
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) lt += __shfl_xor_sync(kFullMask, lt, o);
+        const float inv = 1.f / lt;
+        uint32_t* dst =
+            reinterpret_cast<uint32_t*>(p.out + ((size_t)b * p.Hq + (size_t)kvh * p.G + gg) * D + lane * DPL);
+#pragma unroll
+        for (int q = 0; q < DPL / 2; ++q) dst[q] = pack_bf16(acc[2 * q] * inv, acc[2 * q + 1] * inv);
+    }
+}
+
 template <int D, bool FP8, int WARPS>
 __global__ void __launch_bounds__(WARPS * 32, 1)
 decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
@@ -575,39 +640,7 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
                 if (old == wl - wf) {
                     // last arrival: merge the partials of this pair by log-sum-exp
                     __threadfence();
-                    constexpr int DPL = D / 32;   // columns per lane
-                    for (int gg = 0; gg < G; ++gg) {
-                        float mstar = -INFINITY;
-                        for (int v = wf; v <= wl; ++v) {
-                            const int sl = 2 * v + (((long long)v * T / W) < ts ? 1 : 0);
-                            mstar = fmaxf(mstar, __ldcg(p.part_ml + ((size_t)sl * kMaxGroup + gg) * 2));
-                        }
-                        const float mref = (mstar == -INFINITY) ? 0.f : mstar;
-                        float lt = 0.f, acc[DPL];
-#pragma unroll
-                        for (int q = 0; q < DPL; ++q) acc[q] = 0.f;
-                        for (int v = wf; v <= wl; ++v) {
-                            const int sl = 2 * v + (((long long)v * T / W) < ts ? 1 : 0);
-                            const float2 ml = __ldcg(reinterpret_cast<const float2*>(
-                                p.part_ml + ((size_t)sl * kMaxGroup + gg) * 2));
-                            const float f = ex2(ml.x - mref);
-                            lt += ml.y * f;
-                            const float* src = p.part_o + ((size_t)sl * kMaxGroup + gg) * D + lane * DPL;
-                            if constexpr (DPL == 4) {
-                                const float4 x = __ldcg(reinterpret_cast<const float4*>(src));
-                                acc[0] += f * x.x; acc[1] += f * x.y;
-                                acc[2] += f * x.z; acc[3] += f * x.w;
-                            } else {
-                                const float2 x = __ldcg(reinterpret_cast<const float2*>(src));
-                                acc[0] += f * x.x; acc[1] += f * x.y;
-                            }
-                        }
-                        const float inv = 1.f / lt;
-                        uint32_t* dst = reinterpret_cast<uint32_t*>(
-                            p.out + ((size_t)cb * p.Hq + (size_t)ckvh * G + gg) * D + lane * DPL);
-#pragma unroll
-                        for (int q = 0; q < DPL / 2; ++q) dst[q] = pack_bf16(acc[2 * q] * inv, acc[2 * q + 1] * inv);
-                    }
+                    merge_partials<D>(p, cb, ckvh, ts, wf, wl, T, W, lane);
                     if (lane == 0) atomicExch(&p.counters[(size_t)cb * Hkv + ckvh], 0);
                 }
             }
