@@ -144,6 +144,34 @@ pkv_status pkv_set_workers(pkv_ctx* ctx, int workers);
 /* Bytes of device workspace the context holds. */
 size_t pkv_workspace_bytes(const pkv_ctx* ctx);
 
+/* pkv_decode_attn for callers that cannot allocate device memory.  The pages
+ * describe no such entry point; it exists for callers such as a serving
+ * runtime that reserved all device memory for its own pool at start-up, a
+ * plug-in that may only use memory its host framework hands it, or a
+ * latency-critical path that must not pay for an allocation and the device
+ * synchronisation that can come with it.  pkv_create allocates a workspace;
+ * this call allocates nothing (no cudaMalloc, cudaFree or allocating library
+ * routine) and takes the shapes from cfg instead of a context.  Arguments,
+ * layouts and results are those of pkv_decode_attn.
+ *
+ * Its scratch is one fixed device array of 16 MiB inside the library, which
+ * every GPU that loads the library holds until the process exits.  A call
+ * whose scratch would not fit (error word + batch * Hkv counters + split
+ * partials for 8 warps per SM) returns PKV_ERR_UNSUPPORTED without launching.
+ * The first call on a device, made with that device current, looks up the
+ * array's device address and caches it; make that first call before any
+ * stream capture.  Every call shares the array and the previous call's
+ * contents stay in it: each call clears the part that must start at zero with
+ * cudaMemsetAsync on `stream`, so calls ordered on one stream are
+ * independent, but calls that overlap on the GPU race.  Device-side range
+ * errors are handled as in pkv_decode_attn but cannot be read back (there is
+ * no context). */
+pkv_status pkv_decode_attn_noalloc(const pkv_config* cfg, const void* q, const void* k_pool,
+                                   const void* v_pool, const float* k_scale, const float* v_scale,
+                                   const int32_t* block_tables, int bt_stride,
+                                   const int32_t* seq_lens, int batch, void* out,
+                                   cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -40,7 +40,7 @@ PKV_KV_FP8_E4M3 = 1
 
 # names of every symbol include/pkv.h declares
 EXPORTS = ("pkv_create", "pkv_rope_append", "pkv_decode_attn", "pkv_destroy", "pkv_status_str",
-           "pkv_check_device_error", "pkv_set_workers", "pkv_workspace_bytes")
+           "pkv_check_device_error", "pkv_set_workers", "pkv_workspace_bytes", "pkv_decode_attn_noalloc")
 
 
 class pkv_config(C.Structure):
@@ -66,6 +66,9 @@ lib.pkv_set_workers.argtypes = [_V, C.c_int]
 lib.pkv_set_workers.restype = C.c_int
 lib.pkv_workspace_bytes.argtypes = [_V]
 lib.pkv_workspace_bytes.restype = C.c_size_t
+lib.pkv_decode_attn_noalloc.argtypes = [C.POINTER(pkv_config), _V, _V, _V, _V, _V, _V, C.c_int, _V, C.c_int,
+                                        _V, _V]
+lib.pkv_decode_attn_noalloc.restype = C.c_int
 
 
 class PkvError(RuntimeError):
@@ -164,3 +167,19 @@ def pkv_set_workers(ctx, workers: int, check: bool = True) -> int:
 
 def pkv_workspace_bytes(ctx) -> int:
     return int(lib.pkv_workspace_bytes(ctx))
+
+
+def pkv_decode_attn_noalloc(cfg: pkv_config, q, k_pool, v_pool, k_scale, v_scale, block_tables, seq_lens, out,
+                            batch: int | None = None, bt_stride: int | None = None, stream=None,
+                            check: bool = True) -> int:
+    """pkv_decode_attn without a context, for callers that may not allocate
+    device memory: its scratch is a fixed 16 MiB array inside the library,
+    shared by every call (calls that overlap on the GPU race)."""
+    if batch is None:
+        batch = int(seq_lens.shape[0])
+    if bt_stride is None:
+        bt_stride = int(block_tables.shape[1])
+    st = lib.pkv_decode_attn_noalloc(C.byref(cfg), _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(k_scale),
+                                     _ptr(v_scale), _ptr(block_tables), int(bt_stride), _ptr(seq_lens),
+                                     int(batch), _ptr(out), _stream(stream))
+    return _done(st, "pkv_decode_attn_noalloc", check)
