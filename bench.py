@@ -382,22 +382,42 @@ def run_ours(args, name, rank, world, local_rank):
     torch.cuda.synchronize()
     hot_ms = statistics.median(x.elapsed_time(y) for x, y in hot)
 
-    # end to end through the public API: pinned host inputs in, result out, every step
+    # end to end through the public API: pinned host inputs in, result out, every
+    # step.  The step's inputs are packed into one pinned buffer (16-byte aligned
+    # segments) and copied in with one copy; the library is called on views of
+    # the device copy; the output is read back with one copy.
     e2e = None
     if not args.no_e2e:
-        host = {k: dv[k].cpu().pin_memory() for k in ("q", "k_new", "v_new", "block_tables", "seq_lens")}
+        keys = ("q", "k_new", "v_new", "block_tables", "seq_lens")
+        sizes = [dv[k].numel() * dv[k].element_size() for k in keys]
+        offs, off = [], 0
+        for sz in sizes:
+            offs.append(off)
+            off += (sz + 255) // 256 * 256
+        host_buf = torch.empty(off, dtype=torch.uint8).pin_memory()
+        dev_buf = torch.empty(off, dtype=torch.uint8, device=dev)
+        views = {}
+        for k, o, sz in zip(keys, offs, sizes):
+            host_buf[o:o + sz].copy_(dv[k].contiguous().view(torch.uint8).reshape(-1).cpu())
+            views[k] = dev_buf[o:o + sz].view(dv[k].dtype).view(dv[k].shape)
         out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        h2d = sum(sizes)
         d2h = out_h.numel() * out_h.element_size()
+
+        def e2e_step():
+            dev_buf.copy_(host_buf, non_blocking=True)
+            pkv.pkv_rope_append(ctx, views["q"], views["k_new"], views["v_new"], dv["k_pool"], dv["v_pool"],
+                                dv["k_scale"], dv["v_scale"], views["block_tables"], views["seq_lens"])
+            pkv.pkv_decode_attn(ctx, views["q"], dv["k_pool"], dv["v_pool"], dv["k_scale"], dv["v_scale"],
+                                views["block_tables"], views["seq_lens"], out)
+            out_h.copy_(out, non_blocking=True)
+
         evs = []
         for k in range(args.warmup + K):
             flush.zero_()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record()
-            for key, t in host.items():
-                dv[key].copy_(t, non_blocking=True)
-            step()
-            out_h.copy_(out, non_blocking=True)
+            e2e_step()
             b.record()
             if k >= args.warmup:
                 evs.append((a, b))
@@ -406,8 +426,9 @@ def run_ours(args, name, rank, world, local_rank):
         e2e = {"value": total_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": e2e_ms,
-               "note": "pinned host q/k_new/v_new/block_tables/seq_lens copied in and out read back every "
-                       "step; the KV pools stay resident in HBM (the cache lives on the GPU)"}
+               "note": "every step: q, k_new, v_new, block_tables and seq_lens copied in from one pinned host "
+                       "buffer (one copy), the step run through the C ABI, out read back (one copy); the KV "
+                       "pools stay resident in HBM (the cache lives on the GPU)"}
     pkv.pkv_destroy(ctx)
 
     peak, peak_src = measured_peak()

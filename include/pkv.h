@@ -41,8 +41,8 @@
  * Every pointer must be 16-byte aligned.
  *
  * Ownership and ordering: the library never allocates, frees or keeps caller
- * tensors.  A context owns its workspace (split partials, per-(request, kv
- * head) arrival counters, a device error word), allocated in pkv_create and
+ * tensors.  A context owns its workspace (split partials, the split geometry
+ * passed from the attention kernel to its combine, a device error word), allocated in pkv_create and
  * freed in pkv_destroy; use one context from one stream at a time.  Calls are
  * asynchronous and stream-ordered: they validate on the host, enqueue, and
  * return.  pkv_rope_append writes q (in place) and exactly batch * Hkv slots
@@ -116,7 +116,8 @@ pkv_status pkv_rope_append(pkv_ctx* ctx, void* q, const void* k_new, const void*
  * pkv_rope_append; seq_lens is the same L_b, and n_b = L_b + 1 tokens are
  * attended (the new one included).  out[b][h][:] = bf16(o_h).  Work is split
  * over all SMs by token ranges; partial results of a (request, kv head) cut
- * between workers are merged by log-sum-exp in the same launch.
+ * between workers are merged by log-sum-exp in a second, small kernel
+ * enqueued right after on the same stream.
  * batch == 0 is a no-op. */
 pkv_status pkv_decode_attn(pkv_ctx* ctx, const void* q, const void* k_pool, const void* v_pool,
                            const float* k_scale, const float* v_scale,
@@ -156,8 +157,9 @@ size_t pkv_workspace_bytes(const pkv_ctx* ctx);
  *
  * Its scratch is one fixed device array of 16 MiB inside the library, which
  * every GPU that loads the library holds until the process exits.  A call
- * whose scratch would not fit (error word + batch * Hkv counters + split
- * partials for 8 warps per SM) returns PKV_ERR_UNSUPPORTED without launching.
+ * whose scratch would not fit (error word + batch + 8 ints of split geometry
+ * + split partials for 8 warps per SM: 9.9 MB on a 148-SM B200 at d = 128)
+ * returns PKV_ERR_UNSUPPORTED without launching.
  * The first call on a device, made with that device current, looks up the
  * array's device address and caches it; make that first call before any
  * stream capture.  Every call shares the array and the previous call's

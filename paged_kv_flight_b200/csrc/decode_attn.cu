@@ -20,9 +20,9 @@
 //     skew of the batch;
 //   * a (request, kv head) pair that lies inside one worker's range is
 //     finished by that worker; a pair cut between workers leaves one partial
-//     (unnormalised o, running max m, sum l) per worker, and the worker that
-//     arrives last at the pair's counter merges them by log-sum-exp.  Nobody
-//     ever waits for another worker.
+//     (unnormalised o, running max m, sum l) per worker, stored without any
+//     fence or counter; a small combine kernel launched right after merges
+//     them by log-sum-exp (one CTA per pair).  No worker waits for another.
 //
 // Per warp: a private ring of `stages` K+V tile buffers filled by 2-D TMA
 // tile loads (128-byte or 64-byte swizzle) that complete on one mbarrier per
@@ -151,71 +151,6 @@ __device__ __forceinline__ void load_q(const AttnParams& p, int b, int kvh, int 
     }
 }
 
-// Log-sum-exp merge of the partials that workers wf..wl left for pair (b, kvh)
-// whose first tile is ts (worker v's range starts at v*T/W; its slot for the
-// pair is 2v + 1 if that start lies before ts, else 2v).  One query head at a
-// time: lanes own workers (lane, lane + 32, ...) for the maximum and the
-// weights, and D/32 output columns for the weighted rows, whose loads are
-// issued eight contributors at a time.  Writes the bf16 output rows.
-template <int D>
-__device__ __forceinline__ void merge_partials(const AttnParams& p, int b, int kvh, long long ts, int wf, int wl,
-                                               long long T, int W, int lane)
-{
-    constexpr unsigned kFullMask = 0xFFFFFFFFu;
-    constexpr int DPL = D / 32;
-    const int k = wl - wf + 1;
-    for (int gg = 0; gg < p.G; ++gg) {
-        float m = -INFINITY;
-        for (int i0 = 0; i0 < k; i0 += 32) {
-            const int v = wf + i0 + lane;
-            if (v <= wl) {
-                const int sl = 2 * v + (((long long)v * T / W) < ts ? 1 : 0);
-                m = fmaxf(m, __ldcg(p.part_ml + ((size_t)sl * kMaxGroup + gg) * 2));
-            }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFullMask, m, o));
-        if (m == -INFINITY) m = 0.f;
-        float lt = 0.f, acc[DPL];
-#pragma unroll
-        for (int q = 0; q < DPL; ++q) acc[q] = 0.f;
-        for (int i0 = 0; i0 < k; i0 += 32) {
-            const int v = wf + i0 + lane;
-            int my_sl = 0;
-            float fw = 0.f;
-            if (v <= wl) {
-                my_sl = 2 * v + (((long long)v * T / W) < ts ? 1 : 0);
-                const float2 ml =
-                    __ldcg(reinterpret_cast<const float2*>(p.part_ml + ((size_t)my_sl * kMaxGroup + gg) * 2));
-                fw = ex2(ml.x - m);
-                lt += ml.y * fw;
-            }
-            const int here = min(32, k - i0);
-#pragma unroll 8
-            for (int vv = 0; vv < here; ++vv) {
-                const int sl = __shfl_sync(kFullMask, my_sl, vv);
-                const float f = __shfl_sync(kFullMask, fw, vv);
-                const float* row = p.part_o + ((size_t)sl * kMaxGroup + gg) * D + lane * DPL;
-                if constexpr (DPL == 4) {
-                    const float4 x = __ldcg(reinterpret_cast<const float4*>(row));
-                    acc[0] += f * x.x; acc[1] += f * x.y;
-                    acc[2] += f * x.z; acc[3] += f * x.w;
-                } else {
-                    const float2 x = __ldcg(reinterpret_cast<const float2*>(row));
-                    acc[0] += f * x.x; acc[1] += f * x.y;
-                }
-            }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) lt += __shfl_xor_sync(kFullMask, lt, o);
-        const float inv = 1.f / lt;
-        uint32_t* dst =
-            reinterpret_cast<uint32_t*>(p.out + ((size_t)b * p.Hq + (size_t)kvh * p.G + gg) * D + lane * DPL);
-#pragma unroll
-        for (int q = 0; q < DPL / 2; ++q) dst[q] = pack_bf16(acc[2 * q] * inv, acc[2 * q + 1] * inv);
-    }
-}
-
 template <int D, bool FP8, int WARPS>
 __global__ void __launch_bounds__(WARPS * 32, 1)
 decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
@@ -291,12 +226,21 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
 
     // ---- 2. this warp's range of tiles --------------------------------------------
     const long long T = (long long)prefix[B] * Hkv;
-    if (T == 0) return;
     long long Wl = (long long)gridDim.x * WARPS;
     if (p.workers > 0) Wl = min(Wl, (long long)p.workers);
     else Wl = min(Wl, (T + kMinTilesPerWorker - 1) / kMinTilesPerWorker);
-    Wl = max(1LL, min(Wl, T));
+    Wl = max(1LL, min(Wl, max(T, 1LL)));
     const int W = (int)Wl;
+    if (blockIdx.x == 0) {
+        // the combine kernel that follows needs the same split geometry
+        if (tid == 0) {
+            p.meta[0] = W;
+            p.meta[1] = (int)(T & 0xFFFFFFFFll);
+            p.meta[2] = (int)(T >> 32);
+        }
+        for (int b = tid; b <= B; b += NT) p.meta[4 + b] = prefix[b];
+    }
+    if (T == 0) return;
     const int w = warp * gridDim.x + blockIdx.x;   // spread workers over SMs first
     if (w >= W) return;
     const long long t_begin = (long long)w * T / W;
@@ -632,17 +576,6 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
                         *reinterpret_cast<float2*>(p.part_ml + ((size_t)slot * kMaxGroup + g) * 2) =
                             make_float2(m_run, lsum);
                 }
-                __threadfence();
-                __syncwarp();
-                int old = 0;
-                if (lane == 0) old = atomicAdd(&p.counters[(size_t)cb * Hkv + ckvh], 1);
-                old = __shfl_sync(kFull, old, 0);
-                if (old == wl - wf) {
-                    // last arrival: merge the partials of this pair by log-sum-exp
-                    __threadfence();
-                    merge_partials<D>(p, cb, ckvh, ts, wf, wl, T, W, lane);
-                    if (lane == 0) atomicExch(&p.counters[(size_t)cb * Hkv + ckvh], 0);
-                }
             }
         }
 
@@ -669,6 +602,105 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
     }
 }
 
+// Split combine: one CTA per (request, kv head) pair.  A pair whose tiles lay
+// in more than one warp's range left one partial per range (unnormalised o,
+// running max m in log2 units, sum l); here they are merged by log-sum-exp,
+//   m* = max m_v,  l* = sum l_v 2^(m_v - m*),  o = sum o_v 2^(m_v - m*) / l*,
+// and written as bf16.  Pairs finished inside one range, and requests with an
+// impossible length, are skipped.  Runs after the attention kernel on the
+// same stream, which orders every partial before it is read.
+constexpr int kCombineThreads = 256;   // 8 warps: one per query head of the group when reducing
+
+// Dynamic shared memory of the combine: slot, m and l of every (contributor,
+// head), for up to max_workers contributors.
+inline size_t combine_smem_bytes(int max_workers, int G)
+{
+    return (size_t)max_workers * (sizeof(int) + 2 * sizeof(float) * G);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kCombineThreads, 1) combine_kernel(const AttnParams p)
+{
+    constexpr unsigned kFullMask = 0xFFFFFFFFu;
+    constexpr int NV = (kMaxGroup * D + kCombineThreads - 1) / kCombineThreads;   // outputs per thread
+    extern __shared__ float s_dyn[];
+    __shared__ float s_m[kMaxGroup], s_l[kMaxGroup];
+
+    const int pair = blockIdx.x;
+    const int b = pair / p.Hkv, kvh = pair - b * p.Hkv;
+    const int W = __ldg(&p.meta[0]);
+    const long long T = (long long)(unsigned)__ldg(&p.meta[1]) | ((long long)__ldg(&p.meta[2]) << 32);
+    if (T == 0 || b >= p.batch) return;
+    const int* prefix = p.meta + 4;
+    const int nt = __ldg(&prefix[b + 1]) - __ldg(&prefix[b]);
+    if (nt == 0) return;
+    const long long ts = (long long)__ldg(&prefix[b]) * p.Hkv + (long long)kvh * nt;
+    const long long te = ts + nt;
+    const int wf = (int)(((ts + 1) * W - 1) / T);
+    const int wl = (int)((te * W - 1) / T);
+    if (wf == wl) return;
+    const int k = wl - wf + 1, G = p.G;   // k <= W <= max_workers: the dynamic shared memory fits
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    float* const s_mv = s_dyn;                                   // [k * G] m, later the weight
+    float* const s_lv = s_dyn + (size_t)k * G;                   // [k * G] l
+    int* const s_slot = reinterpret_cast<int*>(s_dyn + 2 * (size_t)k * G);   // [k]
+
+    for (int i = tid; i < k; i += kCombineThreads) {
+        const int v = wf + i;
+        s_slot[i] = 2 * v + (((long long)v * T / W) < ts ? 1 : 0);
+    }
+    __syncthreads();
+    for (int e = tid; e < k * G; e += kCombineThreads) {
+        const int i = e / G, gg = e - i * G;
+        const float2 ml = __ldg(reinterpret_cast<const float2*>(p.part_ml + ((size_t)s_slot[i] * kMaxGroup + gg) * 2));
+        s_mv[e] = ml.x;
+        s_lv[e] = ml.y;
+    }
+    __syncthreads();
+    if (warp < G) {
+        float m = -INFINITY;
+        for (int i = lane; i < k; i += 32) m = fmaxf(m, s_mv[i * G + warp]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFullMask, m, o));
+        if (m == -INFINITY) m = 0.f;
+        float l = 0.f;
+        for (int i = lane; i < k; i += 32) l += s_lv[i * G + warp] * ex2(s_mv[i * G + warp] - m);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(kFullMask, l, o);
+        if (lane == 0) {
+            s_m[warp] = m;
+            s_l[warp] = l;
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < k * G; e += kCombineThreads) {
+        const int gg = e % G;
+        s_mv[e] = ex2(s_mv[e] - s_m[gg]) / s_l[gg];   // now the weight
+    }
+    __syncthreads();
+
+    // every thread accumulates its NV outputs together: NV independent loads per contributor
+    float acc[NV];
+    int gv[NV], cv[NV];
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+        acc[j] = 0.f;
+        const int e = tid + j * kCombineThreads;
+        gv[j] = e / D;
+        cv[j] = e - gv[j] * D;
+    }
+#pragma unroll 4
+    for (int i = 0; i < k; ++i) {
+        const size_t base = (size_t)s_slot[i] * kMaxGroup * D;
+#pragma unroll
+        for (int j = 0; j < NV; ++j)
+            if (gv[j] < G) acc[j] += s_mv[i * G + gv[j]] * __ldg(p.part_o + base + (size_t)gv[j] * D + cv[j]);
+    }
+#pragma unroll
+    for (int j = 0; j < NV; ++j)
+        if (gv[j] < G) p.out[((size_t)b * p.Hq + (size_t)kvh * G + gv[j]) * D + cv[j]] = __float2bfloat16_rn(acc[j]);
+}
+
 template <int D, bool FP8>
 size_t smem_bytes_for(int stages, int max_batch)
 {
@@ -693,6 +725,9 @@ cudaError_t prepare_t(int num_sms, int max_batch, AttnLaunch* out)
     e = cudaFuncSetAttribute(decode_attn_kernel<D, FP8, kAttnWarps>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)bytes);
     if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(combine_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)combine_smem_bytes(num_sms * kAttnWarps, kMaxGroup));
+    if (e != cudaSuccess) return e;
     out->ctas = num_sms;
     out->stages = stages;
     out->smem_bytes = bytes;
@@ -714,12 +749,16 @@ cudaError_t launch_decode_attn(const AttnParams& p, const CUtensorMap& tmk, cons
     const dim3 grid(L.ctas), block(kAttnWarps * 32);
     AttnParams q = p;
     q.stages = L.stages;
+    const dim3 cgrid((unsigned)(p.batch * p.Hkv)), cblock(kCombineThreads);
+    const size_t csmem = combine_smem_bytes(L.ctas * kAttnWarps, p.G);
     if (head_dim == 128) {
         if (fp8) decode_attn_kernel<128, true, kAttnWarps><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
         else decode_attn_kernel<128, false, kAttnWarps><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
+        combine_kernel<128><<<cgrid, cblock, csmem, stream>>>(q);
     } else {
         if (fp8) decode_attn_kernel<64, true, kAttnWarps><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
         else decode_attn_kernel<64, false, kAttnWarps><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
+        combine_kernel<64><<<cgrid, cblock, csmem, stream>>>(q);
     }
     return cudaGetLastError();
 }

@@ -23,7 +23,7 @@ struct pkv_ctx {
     void* ws;             // one allocation, carved below
     size_t ws_bytes;
     int* d_err;
-    int* d_counters;
+    int* d_meta;
     float* d_part_o;
     float* d_part_ml;
     const void* tm_k_ptr;
@@ -135,7 +135,7 @@ pkv_status pkv_create(const pkv_config* cfg, pkv_ctx** out)
 
     const size_t max_workers = (size_t)ctx->attn.ctas * pkv::kAttnWarps;
     const size_t b_err = 256;
-    const size_t b_cnt = ((size_t)cfg->max_batch * cfg->num_kv_heads * sizeof(int) + 255) & ~(size_t)255;
+    const size_t b_cnt = ((size_t)(cfg->max_batch + 8) * sizeof(int) + 255) & ~(size_t)255;
     const size_t b_po = 2 * max_workers * pkv::kMaxGroup * cfg->head_dim * sizeof(float);
     const size_t b_pml = 2 * max_workers * pkv::kMaxGroup * 2 * sizeof(float);
     ctx->ws_bytes = b_err + b_cnt + b_po + b_pml;
@@ -146,7 +146,7 @@ pkv_status pkv_create(const pkv_config* cfg, pkv_ctx** out)
     }
     uint8_t* base = static_cast<uint8_t*>(ctx->ws);
     ctx->d_err = reinterpret_cast<int*>(base);
-    ctx->d_counters = reinterpret_cast<int*>(base + b_err);
+    ctx->d_meta = reinterpret_cast<int*>(base + b_err);
     ctx->d_part_o = reinterpret_cast<float*>(base + b_err + b_cnt);
     ctx->d_part_ml = reinterpret_cast<float*>(base + b_err + b_cnt + b_po);
     if (cudaMemset(ctx->ws, 0, b_err + b_cnt) != cudaSuccess) {
@@ -218,7 +218,7 @@ pkv_status pkv_decode_attn(pkv_ctx* ctx, const void* q, const void* k_pool, cons
     p.seq_lens = seq_lens;
     p.part_o = ctx->d_part_o;
     p.part_ml = ctx->d_part_ml;
-    p.counters = ctx->d_counters;
+    p.meta = ctx->d_meta;
     p.err = ctx->d_err;
     p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)ctx->cfg.head_dim));
     p.batch = batch;

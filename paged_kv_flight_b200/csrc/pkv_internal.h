@@ -54,7 +54,7 @@ struct AttnParams {
     const int32_t* seq_lens;
     float* part_o;        // [2 * max_workers][kMaxGroup][D] fp32, unnormalised
     float* part_ml;       // [2 * max_workers][kMaxGroup][2] fp32 (m in log2 units, l)
-    int* counters;        // [max_batch * Hkv] arrivals per (request, kv head)
+    int* meta;            // [4 + max_batch + 1]: W, T (lo, hi), -, tile prefix; written by the attention kernel for the combine
     int* err;
     float scale_log2;     // log2(e) / sqrt(d)
     int batch, bt_stride, Hq, Hkv, G, P, num_pages;

@@ -7,8 +7,9 @@
 // its host framework, or a latency-critical path that must not pay for an
 // allocation and the device synchronisation that can come with it.  Creating a
 // context (pkv_create) allocates the attention workspace; this entry point
-// allocates nothing.  Its scratch (split partials, per-(request, kv head)
-// arrival counters, the device error word) lives in one file-scope device
+// allocates nothing.  Its scratch (split partials, the split geometry the
+// attention kernel hands to the combine kernel, the device error word) lives
+// in one file-scope device
 // array of kScratchBytes that every GPU that loads this library holds until
 // the process exits.
 //
@@ -16,8 +17,9 @@
 // current: the device address of the array is looked up with
 // cudaGetSymbolAddress and cached.  That first call should therefore come
 // before any stream capture.  Every call shares the one array, which keeps
-// the previous call's contents: the counters and the error word are cleared
-// with cudaMemsetAsync on the caller's stream at each call, so calls ordered
+// the previous call's contents: the error word is cleared with
+// cudaMemsetAsync on the caller's stream at each call, and everything else is
+// written before it is read within the call, so calls ordered
 // on one stream are independent, but calls that overlap on the GPU (different
 // streams, or different host threads without ordering) race on the array.
 // Device-side range errors (page id or length out of range) are handled as in
@@ -129,10 +131,10 @@ extern "C" pkv_status pkv_decode_attn_noalloc(const pkv_config* cfg, const void*
         cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return PKV_ERR_CUDA;
 
-    // scratch layout: [error word | counters | partial rows | partial (m, l)]
+    // scratch layout: [error word | split geometry | partial rows | partial (m, l)]
     const size_t workers = (size_t)num_sms * pkv::kAttnWarps;
     const size_t b_err = 256;
-    const size_t b_cnt = ((size_t)batch * cfg->num_kv_heads * sizeof(int) + 255) & ~(size_t)255;
+    const size_t b_cnt = ((size_t)(batch + 8) * sizeof(int) + 255) & ~(size_t)255;
     const size_t b_po = 2 * workers * pkv::kMaxGroup * cfg->head_dim * sizeof(float);
     const size_t b_pml = 2 * workers * pkv::kMaxGroup * 2 * sizeof(float);
     if (b_err + b_cnt + b_po + b_pml > kScratchBytes) return PKV_ERR_UNSUPPORTED;   // beyond the fixed scratch
@@ -147,7 +149,7 @@ extern "C" pkv_status pkv_decode_attn_noalloc(const pkv_config* cfg, const void*
     if (!encode_pool(cfg, k_pool, &tmk) || !encode_pool(cfg, v_pool, &tmv)) return PKV_ERR_CUDA;
 
     // the previous call may have left anything here: clear what must start at zero
-    if (cudaMemsetAsync(base, 0, b_err + b_cnt, stream) != cudaSuccess) return PKV_ERR_CUDA;
+    if (cudaMemsetAsync(base, 0, b_err, stream) != cudaSuccess) return PKV_ERR_CUDA;
 
     pkv::AttnParams p;
     p.q = static_cast<const __nv_bfloat16*>(q);
@@ -157,7 +159,7 @@ extern "C" pkv_status pkv_decode_attn_noalloc(const pkv_config* cfg, const void*
     p.block_tables = block_tables;
     p.seq_lens = seq_lens;
     p.err = reinterpret_cast<int*>(base);
-    p.counters = reinterpret_cast<int*>(base + b_err);
+    p.meta = reinterpret_cast<int*>(base + b_err);
     p.part_o = reinterpret_cast<float*>(base + b_err + b_cnt);
     p.part_ml = reinterpret_cast<float*>(base + b_err + b_cnt + b_po);
     p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)cfg->head_dim));

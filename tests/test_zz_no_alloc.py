@@ -62,12 +62,17 @@ def test_noalloc_matches_context_entry_point_twice(pkv, case):
         assert finite and mx <= t["max"] and mean <= t["mean"]
 
 
-def test_noalloc_rejects_what_does_not_fit(pkv):
-    # 8192 requests x 512 kv heads of arrival counters alone fill the 16 MiB scratch
-    # (rejected on the host before anything is launched or read, so small
-    # stand-in buffers suffice)
-    cfg = pkv.make_config(512, 512, 64, 16, "bf16", 1e4, 8192, 4, 16)
-    buf = torch.zeros(4096, dtype=torch.int32, device="cuda")
-    st = pkv.pkv_decode_attn_noalloc(cfg, buf, buf, buf, None, None, buf, buf, buf, batch=8192, bt_stride=4,
-                                     check=False)
-    assert st == pkv.PKV_ERR_UNSUPPORTED
+def test_noalloc_rejects_bad_calls_before_launching(pkv):
+    # every case is refused on the host, before anything is launched or read
+    w = workloads.build("rej", 8, 2, 64, 16, False, 1e4, [5, 9], seed=2)
+    dv = _gpu.to_device(w)
+    cfg = _cfg(pkv, w)
+    args = [dv["k_pool"], dv["v_pool"], None, None, dv["block_tables"], dv["seq_lens"]]
+    out = torch.empty(w.batch, w.Hq, w.d, dtype=torch.bfloat16, device="cuda")
+    assert pkv.pkv_decode_attn_noalloc(cfg, dv["q"], *args, out, batch=w.batch + 1,
+                                       check=False) == pkv.PKV_ERR_INVALID_ARG
+    assert pkv.pkv_decode_attn_noalloc(cfg, dv["q"].data_ptr() + 2, *args, out,
+                                       check=False) == pkv.PKV_ERR_INVALID_ARG
+    bad = pkv.make_config(w.Hq, w.Hkv, 96, w.P, "bf16", 1e4, w.batch, w.bt_stride, w.num_pages)
+    assert pkv.pkv_decode_attn_noalloc(bad, dv["q"], *args, out, check=False) == pkv.PKV_ERR_UNSUPPORTED
+    assert pkv.pkv_decode_attn_noalloc(cfg, dv["q"], *args, out, batch=0, check=False) == pkv.PKV_OK
