@@ -382,10 +382,14 @@ def run_ours(args, name, rank, world, local_rank):
     torch.cuda.synchronize()
     hot_ms = statistics.median(x.elapsed_time(y) for x, y in hot)
 
-    # end to end through the public API: pinned host inputs in, result out, every
-    # step.  The step's inputs are packed into one pinned buffer (16-byte aligned
-    # segments) and copied in with one copy; the library is called on views of
-    # the device copy; the output is read back with one copy.
+    # end to end through the public API: every step copies its inputs (q, k_new,
+    # v_new, block_tables, seq_lens, packed in one pinned host buffer) to the
+    # device, runs the step through the C ABI and reads `out` back to pinned
+    # host memory.  Copy-in, compute and copy-out run on three streams with
+    # double-buffered device staging, so step k+1's upload and step k-1's
+    # download overlap step k's kernels, as a serving loop would pipeline them.
+    # The KV pools stay resident (the cache lives on the GPU); they are 4-20x
+    # the L2, so this leg relies on "inputs larger than L2" instead of a flush.
     e2e = None
     if not args.no_e2e:
         keys = ("q", "k_new", "v_new", "block_tables", "seq_lens")
@@ -395,40 +399,60 @@ def run_ours(args, name, rank, world, local_rank):
             offs.append(off)
             off += (sz + 255) // 256 * 256
         host_buf = torch.empty(off, dtype=torch.uint8).pin_memory()
-        dev_buf = torch.empty(off, dtype=torch.uint8, device=dev)
-        views = {}
         for k, o, sz in zip(keys, offs, sizes):
             host_buf[o:o + sz].copy_(dv[k].contiguous().view(torch.uint8).reshape(-1).cpu())
-            views[k] = dev_buf[o:o + sz].view(dv[k].dtype).view(dv[k].shape)
-        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        dev_bufs = [torch.empty(off, dtype=torch.uint8, device=dev) for _ in range(2)]
+        views = [{k: buf[o:o + sz].view(dv[k].dtype).view(dv[k].shape) for k, o, sz in zip(keys, offs, sizes)}
+                 for buf in dev_bufs]
+        outs = [torch.empty_like(out) for _ in range(2)]
+        outs_h = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
         h2d = sum(sizes)
-        d2h = out_h.numel() * out_h.element_size()
+        d2h = outs_h[0].numel() * outs_h[0].element_size()
+        s_in, s_comp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_comp = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
 
-        def e2e_step():
-            dev_buf.copy_(host_buf, non_blocking=True)
-            pkv.pkv_rope_append(ctx, views["q"], views["k_new"], views["v_new"], dv["k_pool"], dv["v_pool"],
-                                dv["k_scale"], dv["v_scale"], views["block_tables"], views["seq_lens"])
-            pkv.pkv_decode_attn(ctx, views["q"], dv["k_pool"], dv["v_pool"], dv["k_scale"], dv["v_scale"],
-                                views["block_tables"], views["seq_lens"], out)
-            out_h.copy_(out, non_blocking=True)
+        def e2e_run(n):
+            for i in range(n):
+                sl = i % 2
+                v = views[sl]
+                if i >= 2:
+                    s_in.wait_event(ev_comp[sl])          # staging slot free again
+                with torch.cuda.stream(s_in):
+                    dev_bufs[sl].copy_(host_buf, non_blocking=True)
+                    ev_in[sl].record(s_in)
+                s_comp.wait_event(ev_in[sl])
+                if i >= 2:
+                    s_comp.wait_event(ev_out[sl])         # output slot read back
+                pkv.pkv_rope_append(ctx, v["q"], v["k_new"], v["v_new"], dv["k_pool"], dv["v_pool"],
+                                    dv["k_scale"], dv["v_scale"], v["block_tables"], v["seq_lens"], stream=s_comp)
+                pkv.pkv_decode_attn(ctx, v["q"], dv["k_pool"], dv["v_pool"], dv["k_scale"], dv["v_scale"],
+                                    v["block_tables"], v["seq_lens"], outs[sl], stream=s_comp)
+                ev_comp[sl].record(s_comp)
+                s_out.wait_event(ev_comp[sl])
+                with torch.cuda.stream(s_out):
+                    outs_h[sl].copy_(outs[sl], non_blocking=True)
+                    ev_out[sl].record(s_out)
 
-        evs = []
-        for k in range(args.warmup + K):
-            flush.zero_()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record()
-            e2e_step()
-            b.record()
-            if k >= args.warmup:
-                evs.append((a, b))
+        e2e_run(args.warmup)
         torch.cuda.synchronize()
-        e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / K)
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(s_in)
+        e2e_run(K)
+        s_in.wait_event(ev_out[(K - 1) % 2])
+        s_in.wait_event(ev_out[K % 2])
+        b.record(s_in)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(a.elapsed_time(b) / K)
         e2e = {"value": total_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": e2e_ms,
-               "note": "every step: q, k_new, v_new, block_tables and seq_lens copied in from one pinned host "
-                       "buffer (one copy), the step run through the C ABI, out read back (one copy); the KV "
-                       "pools stay resident in HBM (the cache lives on the GPU)"}
+               "note": "every step: q, k_new, v_new, block_tables, seq_lens copied in from one pinned host buffer, "
+                       "the step run through the C ABI, out read back to pinned memory; copy-in, compute and "
+                       "copy-out pipelined on three streams (double-buffered); KV pools resident and larger "
+                       "than L2 (no flush in this leg)"}
     pkv.pkv_destroy(ctx)
 
     peak, peak_src = measured_peak()
