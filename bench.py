@@ -371,6 +371,31 @@ def run_ours(args, name, rank, world, local_rank):
     total_bytes = sum_over_ranks(float(by))
     total_reqs = sum_over_ranks(float(B))
 
+    # the same step captured once in a CUDA graph and replayed (L2 flushed
+    # between replays, outside the event window): launch cost of the three
+    # kernels taken out
+    graph_us = None
+    if not args.no_graph:
+        side = torch.cuda.Stream(dev)
+        with torch.cuda.stream(side):
+            step()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            step()
+        gev = []
+        for _ in range(args.warmup + min(K, 200)):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            graph.replay()
+            b.record()
+            gev.append((a, b))
+        torch.cuda.synchronize()
+        gev = gev[args.warmup:]
+        graph_us = max_over_ranks(sum(a.elapsed_time(b) for a, b in gev) / len(gev)) * 1e3
+        del graph
+
     # unflushed ("hot L2") median, labelled as such
     hot = []
     for _ in range(min(K, 50)):
@@ -474,6 +499,7 @@ def run_ours(args, name, rank, world, local_rank):
         "step_us": step_max * 1e3, "attn_us": attn_max * 1e3,
         "rope_append_us": max_over_ranks(sum(rope_ms) / K) * 1e3,
         "step_us_hot_l2": hot_ms * 1e3,
+        "step_us_cuda_graph": graph_us,
         "pct_of_8TBs": 100.0 * value / world / NOMINAL_HBM_GBS,
         "pct_of_measured_peak": 100.0 * value / world / peak,
         "roofline": {"bound": "hbm", "achieved": attn_gbs, "peak": peak, "unit": "GB/s",
@@ -535,6 +561,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay timing")
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--ref-budget", type=int, default=1_200_000,
                     help="attended token-heads per reference step")
