@@ -301,6 +301,8 @@ def run_ours(args, name, rank, world, local_rank):
     cfg = pkv.make_config(w.Hq, w.Hkv, w.d, w.P, "fp8" if w.kv_fp8 else "bf16", w.rope_base, B,
                           w.bt_stride, w.num_pages)
     ctx = pkv.pkv_create(cfg)
+    if args.tail_chunks is not None:
+        pkv.pkv_set_tail_chunks(ctx, args.tail_chunks)
     out = torch.empty(B, w.Hq, w.d, dtype=torch.bfloat16, device=dev)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush_w = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
@@ -562,6 +564,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay timing")
+    ap.add_argument("--tail-chunks", type=int, default=None,
+                    help="cap on dynamic tail chunks per warp range (library default if omitted; 0: static split)")
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--ref-budget", type=int, default=1_200_000,
                     help="attended token-heads per reference step")

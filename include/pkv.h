@@ -115,9 +115,12 @@ pkv_status pkv_rope_append(pkv_ctx* ctx, void* q, const void* k_new, const void*
 /* Step part 2 (decode attention).  q holds the rotated queries written by
  * pkv_rope_append; seq_lens is the same L_b, and n_b = L_b + 1 tokens are
  * attended (the new one included).  out[b][h][:] = bf16(o_h).  Work is split
- * over all SMs by token ranges; partial results of a (request, kv head) cut
- * between workers are merged by log-sum-exp in a second, small kernel
- * enqueued right after on the same stream.
+ * over all SMs by token ranges (optionally with a dynamic tail, see
+ * pkv_set_tail_chunks); partial results of a (request, kv head) cut between
+ * ranges or chunks are merged by log-sum-exp in a second, small kernel
+ * enqueued right after on the same stream.  That kernel also resets the
+ * context's chunk counter; if this call returns PKV_ERR_CUDA the context
+ * should be destroyed, not reused.
  * batch == 0 is a no-op. */
 pkv_status pkv_decode_attn(pkv_ctx* ctx, const void* q, const void* k_pool, const void* v_pool,
                            const float* k_scale, const float* v_scale,
@@ -141,6 +144,14 @@ pkv_status pkv_check_device_error(pkv_ctx* ctx, cudaStream_t stream, int* bits);
  * over (0 restores the automatic choice).  Results do not depend on it
  * beyond rounding; tests use it to force 1, 2, 7, ... splits. */
 pkv_status pkv_set_workers(pkv_ctx* ctx, int workers);
+
+/* Caps the number of dynamic chunks each warp range's tail is cut into
+ * (0 .. 8; 0, the default, gives a static split).  With a cap above 0 the
+ * last quarter of every range (at most 48 tiles of 16 tokens) is cut into
+ * chunks of at least 4 tiles that warps which finish their own share early
+ * claim; ranges under 32 tiles get no tail.  Results do not depend on it
+ * beyond rounding. */
+pkv_status pkv_set_tail_chunks(pkv_ctx* ctx, int max_chunks);
 
 /* Bytes of device workspace the context holds. */
 size_t pkv_workspace_bytes(const pkv_ctx* ctx);

@@ -18,11 +18,18 @@
 //     into W equal contiguous ranges, one per warp worker (W <= warps x SMs),
 //     so every worker streams the same number of bytes whatever the length
 //     skew of the batch;
-//   * a (request, kv head) pair that lies inside one worker's range is
-//     finished by that worker; a pair cut between workers leaves one partial
-//     (unnormalised o, running max m, sum l) per worker, stored without any
-//     fence or counter; a small combine kernel launched right after merges
-//     them by log-sum-exp (one CTA per pair).  No worker waits for another.
+//   * optionally each range is cut into units: a static head that its own
+//     warp streams, and (for ranges of 32 tiles or more) a tail of its last
+//     quarter (at most 48 tiles) cut into K chunks of at least 4 tiles.  A
+//     warp that has finished its head claims tail chunks of any range from
+//     one atomic counter, so warps that the memory system served faster take
+//     over the work of slower ones and all finish within about one chunk of
+//     each other;
+//   * a (request, kv head) pair that lies inside one unit is finished there; a
+//     pair cut between units leaves one partial (unnormalised o, running max
+//     m, sum l) per unit, stored without any fence; a small combine kernel
+//     launched right after merges them by log-sum-exp (one CTA per pair) and
+//     resets the chunk counter.  No worker waits for another.
 //
 // Per warp: a private ring of `stages` K+V tile buffers filled by 2-D TMA
 // tile loads (128-byte or 64-byte swizzle) that complete on one mbarrier per
@@ -76,6 +83,66 @@ struct StageInfo {
     int pad;
 };
 
+// Units of the split.  Warp range v is [r(v), r(v+1)), r(v) = v T / W.  With
+// K = 0 a range is one unit.  With K > 0 unit v (K+1) is the head
+// [r(v), s(v)) and units v (K+1) + 1 + j, j < K, cut the tail [s(v), r(v+1))
+// of tl = min(range / kTailDen, kTailMaxTiles) tiles at s(v) + j tl / K.
+// Units are numbered in the order of the tiles they hold, none is empty, and
+// together they cover [0, T) once.  W < 2^16, so r(v) needs one 32-bit
+// division (T = qT W + rT), and tl is small.
+struct Split {
+    long long T, qT;
+    int W, K, rT;
+
+    __device__ __forceinline__ long long r(int v) const
+    {
+        return (long long)v * qT + (long long)(((unsigned)v * (unsigned)rT) / (unsigned)W);
+    }
+    __device__ __forceinline__ static int tail_of(long long range)
+    {
+        return (int)min(range / kTailDen, (long long)kTailMaxTiles);
+    }
+    // first tile of unit U (U = W (K+1) gives T)
+    __device__ __forceinline__ long long ustart(int U) const
+    {
+        if (K == 0) return r(U);
+        const int v = U / (K + 1), j = U - v * (K + 1);
+        const long long rv = r(v);
+        if (j == 0) return rv;
+        const long long range = r(v + 1) - rv;
+        const int tl = tail_of(range);
+        return rv + range - tl + (j - 1) * tl / K;
+    }
+    // index of the unit holding tile x, 0 <= x < T
+    __device__ __forceinline__ int unit_of(long long x) const
+    {
+        const int v = (int)(((x + 1) * W - 1) / T);
+        if (K == 0) return v;
+        const long long rv = r(v), range = r(v + 1) - rv;
+        const int tl = tail_of(range);
+        const long long sv = rv + range - tl;
+        if (x < sv) return v * (K + 1);
+        const int y = (int)(x - sv);
+        return v * (K + 1) + 1 + ((y + 1) * K - 1) / tl;
+    }
+};
+
+// K for T tiles over W warps, at most `max_chunks`: chunks of at least
+// kTailChunkTiles tiles, none when the shortest range is under kTailMinTiles
+// tiles (its tail then holds at least 8 tiles, and the head at least 24).
+__device__ __forceinline__ Split make_split(long long T, int W, int max_chunks)
+{
+    Split sp;
+    sp.T = T;
+    sp.W = W;
+    sp.qT = T / W;
+    sp.rT = (int)(T - sp.qT * W);
+    sp.K = 0;
+    if (max_chunks > 0 && sp.qT >= kTailMinTiles)
+        sp.K = min(max_chunks, max(1, Split::tail_of(sp.qT) / kTailChunkTiles));
+    return sp;
+}
+
 // Largest b with prefix[b] * Hkv <= x, for 0 <= x < prefix[B] * Hkv.
 __device__ __forceinline__ int seek_request(const int* prefix, int B, int Hkv, long long x)
 {
@@ -86,6 +153,22 @@ __device__ __forceinline__ int seek_request(const int* prefix, int B, int Hkv, l
         else hi = mid;
     }
     return lo;
+}
+
+// (request, kv head, tile within the pair) of flattened tile x
+__device__ __forceinline__ void locate(const int* prefix, int B, int Hkv, long long x, int& b, int& kvh,
+                                       int& tt, int& cnt)
+{
+    b = seek_request(prefix, B, Hkv, x);
+    cnt = prefix[b + 1] - prefix[b];
+    const long long r = x - (long long)prefix[b] * Hkv;
+    if (r <= 0x7fffffffll) {   // the usual case: 32-bit division
+        kvh = (int)r / cnt;
+        tt = (int)r - kvh * cnt;
+    } else {
+        kvh = (int)(r / cnt);
+        tt = (int)(r % cnt);
+    }
 }
 
 // Page ids (as TMA row coordinates) and scales of 32 consecutive tiles, one
@@ -224,28 +307,28 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
         }
     }
 
-    // ---- 2. this warp's range of tiles --------------------------------------------
+    // ---- 2. split geometry and this warp's head unit ------------------------------
     const long long T = (long long)prefix[B] * Hkv;
     long long Wl = (long long)gridDim.x * WARPS;
     if (p.workers > 0) Wl = min(Wl, (long long)p.workers);
     else Wl = min(Wl, (T + kMinTilesPerWorker - 1) / kMinTilesPerWorker);
     Wl = max(1LL, min(Wl, max(T, 1LL)));
     const int W = (int)Wl;
+    const Split sp = make_split(max(T, 1LL), W, p.tail_chunks);
     if (blockIdx.x == 0) {
         // the combine kernel that follows needs the same split geometry
         if (tid == 0) {
             p.meta[0] = W;
             p.meta[1] = (int)(T & 0xFFFFFFFFll);
             p.meta[2] = (int)(T >> 32);
+            p.meta[3] = sp.K;
         }
         for (int b = tid; b <= B; b += NT) p.meta[4 + b] = prefix[b];
     }
     if (T == 0) return;
     const int w = warp * gridDim.x + blockIdx.x;   // spread workers over SMs first
     if (w >= W) return;
-    const long long t_begin = (long long)w * T / W;
-    const long long t_end = (long long)(w + 1) * T / W;
-    const int ntiles = (int)(t_end - t_begin);
+    const long long n_chunks = (long long)W * sp.K;
 
     const uint32_t my_stage0 = stage_area + (uint32_t)(warp * S * Gm::STAGEB);
     StageInfo* const my_info = info_all + warp * S;
@@ -256,18 +339,51 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
     }
     __syncwarp();
 
-    // ---- 3. producer: double-buffered 32-tile lookahead, TMA issue ----------------
-    long long la_base = t_begin;
-    Lookahead la_cur = lookahead_fill<FP8>(p, prefix, t_begin, t_end, lane);
-    Lookahead la_nxt = lookahead_fill<FP8>(p, prefix, t_begin + 32, t_end, lane);
+    // ---- 3. producer: units in issue order, 32-tile lookahead, TMA issue ------------
+    // The producer issues the tiles of its current unit [pu0, pu0 + p_left
+    // ...) from two 32-tile lookahead windows (la_cur from index la_i, la_nxt;
+    // la_fill is the first tile of the window after them).  When kClaimAhead
+    // tiles of the unit are left to issue it claims the next tail chunk
+    // (atomic on the chunk counter) and, once the unit is fully issued, reads
+    // the claim and loads the first window of the next unit (nU, la_new).
+    constexpr int kNone = -1, kPending = -2;
+    constexpr int kClaimAhead = 2;
+    int pU = w * (sp.K + 1);
+    long long pu0 = sp.ustart(pU), pu1 = sp.ustart(pU + 1);
+    int p_left = (int)(pu1 - pu0);   // a head holds at most T / W + 1 tiles
+    int la_i = 0;
+    long long la_fill = pu0 + 64;
+    Lookahead la_cur = lookahead_fill<FP8>(p, prefix, pu0, pu1, lane);
+    Lookahead la_nxt = lookahead_fill<FP8>(p, prefix, pu0 + 32, pu1, lane);
+    int nU = sp.K > 0 ? kPending : kNone;
+    long long nu0 = 0, nu1 = 0;
+    Lookahead la_new{0, 0, 1.f, 1.f};
+    int claim = 0;
+    bool claim_sent = false;
 
-    auto issue = [&](long long x, int s) {
-        if (x >= la_base + 32) {
-            la_base += 32;
-            la_cur = la_nxt;
-            la_nxt = lookahead_fill<FP8>(p, prefix, la_base + 32, t_end, lane);
+    // issues the next tile of this warp's sequence into stage s; false when
+    // there is none left
+    auto issue_next = [&](int s) -> bool {
+        if (p_left == 0) {
+            if (nU < 0) return false;
+            pU = nU;
+            pu0 = nu0;
+            pu1 = nu1;
+            p_left = (int)(nu1 - nu0);
+            la_i = 0;
+            la_cur = la_new;
+            la_nxt = lookahead_fill<FP8>(p, prefix, nu0 + 32, nu1, lane);
+            la_fill = nu0 + 64;
+            nU = kPending;
         }
-        const int src = (int)(x - la_base);
+        if (la_i == 32) {
+            la_i = 0;
+            la_cur = la_nxt;
+            la_nxt = lookahead_fill<FP8>(p, prefix, la_fill, pu1, lane);
+            la_fill += 32;
+        }
+        const int src = la_i++;
+        --p_left;
         const int v = __shfl_sync(kFull, la_cur.valid, src);
         const int row = __shfl_sync(kFull, la_cur.row, src);
         float ks = 1.f, vs = 1.f;
@@ -297,22 +413,32 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
                 mbar_arrive(bar);
             }
         }
+        if (nU == kPending) {
+            if (!claim_sent && p_left <= kClaimAhead) {
+                if (lane == 0) claim = atomicAdd(p.claim, 1);
+                claim_sent = true;
+            }
+            if (p_left == 0) {
+                const int c = __shfl_sync(kFull, claim, 0);
+                claim_sent = false;
+                if (c >= n_chunks) {
+                    nU = kNone;
+                } else {
+                    const int v2 = c % W;
+                    nU = v2 * (sp.K + 1) + 1 + (c - v2) / W;
+                    nu0 = sp.ustart(nU);
+                    nu1 = sp.ustart(nU + 1);
+                    la_new = lookahead_fill<FP8>(p, prefix, nu0, nu1, lane);
+                }
+            }
+        }
+        return true;
     };
 
-    const int pre = min(S, ntiles);
-    for (int k = 0; k < pre; ++k) issue(t_begin + k, k);
-    int issued = pre;
+    int issued = 0;
+    while (issued < S && issue_next(issued)) ++issued;
 
     // ---- 4. consumer ----------------------------------------------------------------
-    int cb = seek_request(prefix, B, Hkv, t_begin);
-    int cnt = prefix[cb + 1] - prefix[cb];
-    int ckvh, ctt;
-    {
-        const long long r = t_begin - (long long)prefix[cb] * Hkv;
-        ckvh = (int)(r / cnt);
-        ctt = (int)(r % cnt);
-    }
-
     const int g = lane >> 2;     // mma row = query head within the group
     const int c4 = lane & 3;
     const int G = p.G;
@@ -329,12 +455,43 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
     int s = 0;
     uint32_t parity = 0;
 
+    // consumer: unit [cu0, cu1) with index cU and c_left tiles still to
+    // consume; cursor = pair (cb, ckvh) of cnt tiles, tile ctt of it.  A unit
+    // is longer than the producer's lead (at most S tiles), so when the
+    // consumer reaches the end of a unit the producer is already inside the
+    // next one, whose bounds it still holds.
+    int cU = pU;
+    long long cu0 = pu0, cu1 = pu1;
+    int c_left = (int)(pu1 - pu0);
+    bool unit_first = true;
+    int cb, ckvh, ctt, cnt;
+    locate(prefix, B, Hkv, cu0, cb, ckvh, ctt, cnt);
     load_q<D, FP8>(p, cb, ckvh, g, c4, qn);
     n_next = p.seq_lens[cb] + 1;
 
-    for (int k = 0; k < ntiles; ++k) {
-        if (ctt == 0 || k == 0) {
-            // start of a (request, kv head) pair: take the prefetched query
+    for (int k = 0; k < issued; ++k) {
+        if (!dead) {
+            const bool ok = __all_sync(kFull, mbar_wait_bounded(my_bar0 + 8u * s, parity, kWaitLimitNs));
+            if (!ok) {
+                dead = true;
+                k_dead = k;
+                if (lane == 0) atomicOr(p.err, kErrTimeout);
+            }
+        }
+        if (dead) {
+            // control flow only: no data, no writes
+            if (++s == S) {
+                s = 0;
+                parity ^= 1u;
+            }
+            continue;
+        }
+        const StageInfo si = my_info[s];
+        const bool unit_end = c_left == 1;
+        const bool pair_end = ctt == cnt - 1 || unit_end;
+
+        if (ctt == 0 || unit_first) {
+            // start of a (request, kv head) pair or of a unit: take the prefetched query
 #pragma unroll
             for (int ks = 0; ks < KSTEPS; ++ks) {
                 if constexpr (!FP8) {
@@ -350,11 +507,15 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
             for (int nt = 0; nt < NTD; ++nt) o[nt][0] = o[nt][1] = 0.f;
             m_run = -INFINITY;
             l_run = 0.f;
+            unit_first = false;
         }
-        if (ctt == cnt - 1 && k + 1 < ntiles) {
-            // this tile ends the pair: fetch the next pair's query now
+        if (pair_end && k + 1 < issued) {
+            // the next tile starts another pair: fetch its query now
             int nb = cb, nkvh = ckvh + 1;
-            if (nkvh == Hkv) {
+            if (unit_end) {
+                int ntt, ncnt;
+                locate(prefix, B, Hkv, pu0, nb, nkvh, ntt, ncnt);   // the producer's unit is the next one
+            } else if (nkvh == Hkv) {
                 nkvh = 0;
                 do { ++nb; } while (nb < B - 1 && prefix[nb + 1] == prefix[nb]);
             }
@@ -362,18 +523,8 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
             n_next = p.seq_lens[nb] + 1;
         }
 
-        if (!dead) {
-            const bool ok = __all_sync(kFull, mbar_wait_bounded(my_bar0 + 8u * s, parity, kWaitLimitNs));
-            if (!ok) {
-                dead = true;
-                k_dead = k;
-                if (lane == 0) atomicOr(p.err, kErrTimeout);
-            }
-        }
-
         bool zeroed = false;
-        if (!dead && my_info[s].valid) {
-            const StageInfo si = my_info[s];
+        if (si.valid) {
             const uint32_t kb = my_stage0 + (uint32_t)(s * Gm::STAGEB);
             const uint32_t vb = kb + Gm::TILEB;
             const int tok0 = ctt * kTile;
@@ -391,7 +542,6 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
                 zeroed = true;
                 __syncwarp();
             }
-
             // S = Q K^T (two n-tiles of 8 tokens), two accumulation chains
             float sa[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, sb[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
             if constexpr (!FP8) {
@@ -517,25 +667,19 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
         }
         __syncwarp();
 
-        // refill this stage with the tile `S` ahead
-        if (!dead && issued < ntiles) {
-            // generic-proxy zero stores above must land before the async-proxy
-            // copy that overwrites the buffer
-            if (zeroed && lane == 0) fence_proxy_async_smem();
-            issue(t_begin + issued, s);
-            ++issued;
-        }
+        // refill this stage with the tile `S` ahead; generic-proxy zero stores
+        // above must land before the async-proxy copy that overwrites the buffer
+        if (zeroed && lane == 0) fence_proxy_async_smem();
+        if (issue_next(s)) ++issued;
 
-        // ---- end of a pair (or of this range): write out or leave a partial -------
-        if (ctt == cnt - 1 || k == ntiles - 1) {
+        // ---- end of a pair (or of a unit): write out or leave a partial -----------
+        if (pair_end) {
             float lsum = l_run + __shfl_xor_sync(kFull, l_run, 1);
             lsum += __shfl_xor_sync(kFull, lsum, 2);
             const long long ts = (long long)prefix[cb] * Hkv + (long long)ckvh * cnt;
             const long long te = ts + cnt;
-            const int wf = (int)(((ts + 1) * W - 1) / T);
-            const int wl = (int)((te * W - 1) / T);
             const size_t orow = ((size_t)cb * p.Hq + (size_t)ckvh * G + g) * D;
-            if (wf == wl) {
+            if (cu0 <= ts && te <= cu1) {
                 if (g < G) {
                     const float inv = 1.f / lsum;
                     uint32_t* dst = reinterpret_cast<uint32_t*>(p.out + orow);
@@ -554,9 +698,9 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
                     }
                 }
             } else {
-                const long long my_start = (long long)w * T / W;
-                const int slot = 2 * w + (my_start < ts ? 1 : 0);
-                const size_t prow = ((size_t)slot * kMaxGroup + g) * D;
+                // slot 2U for the pair the unit starts in, 2U + 1 for one that starts inside it
+                const int slot = 2 * cU + (cu0 < ts ? 1 : 0);
+                const size_t prow = ((size_t)slot * G + g) * D;
                 if (g < G) {
                     float* dst = p.part_o + prow;
                     if constexpr (!FP8) {
@@ -573,20 +717,32 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
                                     make_float2(o[2 * u][e], o[2 * u + 1][e]);
                     }
                     if (c4 == 0)
-                        *reinterpret_cast<float2*>(p.part_ml + ((size_t)slot * kMaxGroup + g) * 2) =
+                        *reinterpret_cast<float2*>(p.part_ml + ((size_t)slot * G + g) * 2) =
                             make_float2(m_run, lsum);
                 }
             }
         }
 
         // advance the consumer cursor and the ring position
-        if (++ctt == cnt) {
-            ctt = 0;
-            if (++ckvh == Hkv) {
-                ckvh = 0;
-                do { ++cb; } while (cb < B && prefix[cb + 1] == prefix[cb]);
+        if (unit_end) {
+            if (k + 1 < issued) {
+                cU = pU;
+                cu0 = pu0;
+                cu1 = pu1;
+                c_left = (int)(pu1 - pu0);
+                unit_first = true;
+                locate(prefix, B, Hkv, cu0, cb, ckvh, ctt, cnt);
             }
-            if (cb < B) cnt = prefix[cb + 1] - prefix[cb];
+        } else {
+            --c_left;
+            if (++ctt == cnt) {
+                ctt = 0;
+                if (++ckvh == Hkv) {
+                    ckvh = 0;
+                    do { ++cb; } while (cb < B && prefix[cb + 1] == prefix[cb]);
+                }
+                if (cb < B) cnt = prefix[cb + 1] - prefix[cb];
+            }
         }
         if (++s == S) {
             s = 0;
@@ -603,29 +759,46 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
 }
 
 // Split combine: one CTA per (request, kv head) pair.  A pair whose tiles lay
-// in more than one warp's range left one partial per range (unnormalised o,
-// running max m in log2 units, sum l); here they are merged by log-sum-exp,
+// in more than one unit left one partial per unit (unnormalised o, running max
+// m in log2 units, sum l); here they are merged by log-sum-exp,
 //   m* = max m_v,  l* = sum l_v 2^(m_v - m*),  o = sum o_v 2^(m_v - m*) / l*,
-// and written as bf16.  Pairs finished inside one range, and requests with an
+// and written as bf16.  Pairs finished inside one unit, and requests with an
 // impossible length, are skipped.  Runs after the attention kernel on the
-// same stream, which orders every partial before it is read.
-constexpr int kCombineThreads = 256;   // 8 warps: one per query head of the group when reducing
+// same stream, which orders every partial before it is read; it also resets
+// the chunk counter of the attention's dynamic tail for the next launch.
+// Contributors are staged in shared memory kCombineBlock at a time: one pass
+// for m* and l* (one warp per head), one for the weighted sum (in reverse
+// block order, so a pair with at most kCombineBlock contributors is staged
+// once) in which warp j sums contributors j, j + 8, ... over all G x D
+// values with 16-byte loads, and the eight warp sums are added in a fixed
+// order.
+constexpr int kCombineThreads = 256;
+constexpr int kCombineWarps = kCombineThreads / 32;
+constexpr int kCombineBlock = 256;
 
-// Dynamic shared memory of the combine: slot, m and l of every (contributor,
-// head), for up to max_workers contributors.
-inline size_t combine_smem_bytes(int max_workers, int G)
+// floats of the staging area (slots, m, l of kb contributors), rounded up to 16 bytes
+inline __host__ __device__ size_t combine_stage_floats(int kb, int G)
 {
-    return (size_t)max_workers * (sizeof(int) + 2 * sizeof(float) * G);
+    return (((size_t)kb * (2 * G + 1)) + 3) & ~(size_t)3;
+}
+
+// Dynamic shared memory of the combine for at most `contributors` per pair.
+inline size_t combine_smem_bytes(int contributors, int G, int D)
+{
+    const int kb = contributors < kCombineBlock ? contributors : kCombineBlock;
+    return sizeof(float) * (combine_stage_floats(kb, G) + (size_t)kCombineWarps * G * D);
 }
 
 template <int D>
-__global__ void __launch_bounds__(kCombineThreads, 1) combine_kernel(const AttnParams p)
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const AttnParams p)
 {
     constexpr unsigned kFullMask = 0xFFFFFFFFu;
-    constexpr int NV = (kMaxGroup * D + kCombineThreads - 1) / kCombineThreads;   // outputs per thread
-    extern __shared__ float s_dyn[];
+    constexpr int F4 = kMaxGroup * D / 4 / 32;   // 16-byte chunks per lane per contributor, at most
+    extern __shared__ float4 s_dyn4[];
+    float* const s_dyn = reinterpret_cast<float*>(s_dyn4);
     __shared__ float s_m[kMaxGroup], s_l[kMaxGroup];
 
+    if (blockIdx.x == 0 && threadIdx.x == 0) *p.claim = 0;   // the attention launch has ended
     const int pair = blockIdx.x;
     const int b = pair / p.Hkv, kvh = pair - b * p.Hkv;
     const int W = __ldg(&p.meta[0]);
@@ -634,71 +807,116 @@ __global__ void __launch_bounds__(kCombineThreads, 1) combine_kernel(const AttnP
     const int* prefix = p.meta + 4;
     const int nt = __ldg(&prefix[b + 1]) - __ldg(&prefix[b]);
     if (nt == 0) return;
+    Split sp = make_split(T, W, 0);
+    sp.K = __ldg(&p.meta[3]);   // as the attention launch chose it
     const long long ts = (long long)__ldg(&prefix[b]) * p.Hkv + (long long)kvh * nt;
-    const long long te = ts + nt;
-    const int wf = (int)(((ts + 1) * W - 1) / T);
-    const int wl = (int)((te * W - 1) / T);
-    if (wf == wl) return;
-    const int k = wl - wf + 1, G = p.G;   // k <= W <= max_workers: the dynamic shared memory fits
+    const int U0 = sp.unit_of(ts), U1 = sp.unit_of(ts + nt - 1);
+    if (U0 == U1) return;
+    const int k = U1 - U0 + 1, G = p.G, GD4 = G * D / 4;
+    const int side0 = sp.ustart(U0) < ts ? 1 : 0;   // slot side of the first unit
+    const int kb = min(k, kCombineBlock);              // the dynamic shared memory holds kb contributors
+    const int nblk = (k + kCombineBlock - 1) / kCombineBlock;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    float* const s_mv = s_dyn;                                   // [k * G] m, later the weight
-    float* const s_lv = s_dyn + (size_t)k * G;                   // [k * G] l
-    int* const s_slot = reinterpret_cast<int*>(s_dyn + 2 * (size_t)k * G);   // [k]
+    float* const s_mv = s_dyn;                                                  // [kb * G] m, later the weight
+    float* const s_lv = s_dyn + (size_t)kb * G;                                 // [kb * G] l
+    int* const s_slot = reinterpret_cast<int*>(s_dyn + 2 * (size_t)kb * G);    // [kb]
+    float4* const s_red = s_dyn4 + combine_stage_floats(kb, G) / 4;            // [warps][G * D / 4]
 
-    for (int i = tid; i < k; i += kCombineThreads) {
-        const int v = wf + i;
-        s_slot[i] = 2 * v + (((long long)v * T / W) < ts ? 1 : 0);
-    }
-    __syncthreads();
-    for (int e = tid; e < k * G; e += kCombineThreads) {
-        const int i = e / G, gg = e - i * G;
-        const float2 ml = __ldg(reinterpret_cast<const float2*>(p.part_ml + ((size_t)s_slot[i] * kMaxGroup + gg) * 2));
-        s_mv[e] = ml.x;
-        s_lv[e] = ml.y;
-    }
-    __syncthreads();
-    if (warp < G) {
-        float m = -INFINITY;
-        for (int i = lane; i < k; i += 32) m = fmaxf(m, s_mv[i * G + warp]);
+    // slots, m and l of the contributors of block blk; returns how many
+    auto stage = [&](int blk) -> int {
+        const int i0 = blk * kCombineBlock, n = min(kCombineBlock, k - i0);
+        for (int i = tid; i < n; i += kCombineThreads)
+            s_slot[i] = 2 * (U0 + i0 + i) + (i0 + i == 0 ? side0 : 0);
+        __syncthreads();
+        for (int e = tid; e < n * G; e += kCombineThreads) {
+            const int i = e / G, gg = e - i * G;
+            const float2 ml = __ldg(reinterpret_cast<const float2*>(p.part_ml + ((size_t)s_slot[i] * G + gg) * 2));
+            s_mv[e] = ml.x;
+            s_lv[e] = ml.y;
+        }
+        __syncthreads();
+        return n;
+    };
+
+    // pass 1: m* and l* per head (warp g), merged over blocks
+    float Mg = -INFINITY, Lg = 0.f;
+    int n_last = 0;
+    for (int blk = 0; blk < nblk; ++blk) {
+        if (blk > 0) __syncthreads();
+        const int n = stage(blk);
+        n_last = n;
+        if (warp < G) {
+            float m = -INFINITY;
+            for (int i = lane; i < n; i += 32) m = fmaxf(m, s_mv[i * G + warp]);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFullMask, m, o));
-        if (m == -INFINITY) m = 0.f;
-        float l = 0.f;
-        for (int i = lane; i < k; i += 32) l += s_lv[i * G + warp] * ex2(s_mv[i * G + warp] - m);
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFullMask, m, o));
+            const float m_new = fmaxf(Mg, m);
+            const float m_ref = (m_new == -INFINITY) ? 0.f : m_new;
+            float l = 0.f;
+            for (int i = lane; i < n; i += 32) l += s_lv[i * G + warp] * ex2(s_mv[i * G + warp] - m_ref);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(kFullMask, l, o);
-        if (lane == 0) {
-            s_m[warp] = m;
-            s_l[warp] = l;
+            for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(kFullMask, l, o);
+            Lg = Lg * ex2(Mg - m_ref) + l;
+            Mg = m_new;
         }
     }
-    __syncthreads();
-    for (int e = tid; e < k * G; e += kCombineThreads) {
-        const int gg = e % G;
-        s_mv[e] = ex2(s_mv[e] - s_m[gg]) / s_l[gg];   // now the weight
+    if (warp < G && lane == 0) {
+        s_m[warp] = (Mg == -INFINITY) ? 0.f : Mg;
+        s_l[warp] = Lg;
     }
     __syncthreads();
 
-    // every thread accumulates its NV outputs together: NV independent loads per contributor
-    float acc[NV];
-    int gv[NV], cv[NV];
+    // pass 2: warp j sums contributors j, j + 8, ... (all G x D values)
+    float4 acc[F4];
 #pragma unroll
-    for (int j = 0; j < NV; ++j) {
-        acc[j] = 0.f;
-        const int e = tid + j * kCombineThreads;
-        gv[j] = e / D;
-        cv[j] = e - gv[j] * D;
+    for (int t = 0; t < F4; ++t) acc[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int blk = nblk - 1; blk >= 0; --blk) {
+        int n = n_last;
+        if (blk != nblk - 1) {
+            __syncthreads();
+            n = stage(blk);
+        }
+        for (int e = tid; e < n * G; e += kCombineThreads) {
+            const int gg = e % G;
+            s_mv[e] = ex2(s_mv[e] - s_m[gg]) / s_l[gg];   // now the weight
+        }
+        __syncthreads();
+#pragma unroll 2
+        for (int i = warp; i < n; i += kCombineWarps) {
+            const float4* src = reinterpret_cast<const float4*>(p.part_o + (size_t)s_slot[i] * G * D);
+#pragma unroll
+            for (int t = 0; t < F4; ++t) {
+                const int f = lane + 32 * t;
+                if (f < GD4) {
+                    const float wgt = s_mv[i * G + (4 * f) / D];
+                    const float4 v = __ldg(src + f);
+                    acc[t].x += wgt * v.x;
+                    acc[t].y += wgt * v.y;
+                    acc[t].z += wgt * v.z;
+                    acc[t].w += wgt * v.w;
+                }
+            }
+        }
     }
-#pragma unroll 4
-    for (int i = 0; i < k; ++i) {
-        const size_t base = (size_t)s_slot[i] * kMaxGroup * D;
 #pragma unroll
-        for (int j = 0; j < NV; ++j)
-            if (gv[j] < G) acc[j] += s_mv[i * G + gv[j]] * __ldg(p.part_o + base + (size_t)gv[j] * D + cv[j]);
+    for (int t = 0; t < F4; ++t) {
+        const int f = lane + 32 * t;
+        if (f < GD4) s_red[warp * GD4 + f] = acc[t];
     }
+    __syncthreads();
+    uint2* const dst = reinterpret_cast<uint2*>(p.out + ((size_t)b * p.Hq + (size_t)kvh * G) * D);
+    for (int f = tid; f < GD4; f += kCombineThreads) {
+        float4 sum = s_red[f];
 #pragma unroll
-    for (int j = 0; j < NV; ++j)
-        if (gv[j] < G) p.out[((size_t)b * p.Hq + (size_t)kvh * G + gv[j]) * D + cv[j]] = __float2bfloat16_rn(acc[j]);
+        for (int j = 1; j < kCombineWarps; ++j) {
+            const float4 v = s_red[j * GD4 + f];
+            sum.x += v.x;
+            sum.y += v.y;
+            sum.z += v.z;
+            sum.w += v.w;
+        }
+        dst[f] = make_uint2(pack_bf16(sum.x, sum.y), pack_bf16(sum.z, sum.w));
+    }
 }
 
 template <int D, bool FP8>
@@ -726,7 +944,7 @@ cudaError_t prepare_t(int num_sms, int max_batch, AttnLaunch* out)
                              (int)bytes);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(combine_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)combine_smem_bytes(num_sms * kAttnWarps, kMaxGroup));
+                             (int)combine_smem_bytes(kCombineBlock, kMaxGroup, D));
     if (e != cudaSuccess) return e;
     out->ctas = num_sms;
     out->stages = stages;
@@ -750,7 +968,7 @@ cudaError_t launch_decode_attn(const AttnParams& p, const CUtensorMap& tmk, cons
     AttnParams q = p;
     q.stages = L.stages;
     const dim3 cgrid((unsigned)(p.batch * p.Hkv)), cblock(kCombineThreads);
-    const size_t csmem = combine_smem_bytes(L.ctas * kAttnWarps, p.G);
+    const size_t csmem = combine_smem_bytes((int)max_units(L.ctas * kAttnWarps, p.tail_chunks), p.G, head_dim);
     if (head_dim == 128) {
         if (fp8) decode_attn_kernel<128, true, kAttnWarps><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
         else decode_attn_kernel<128, false, kAttnWarps><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);

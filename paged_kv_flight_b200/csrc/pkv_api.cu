@@ -20,9 +20,11 @@ struct pkv_ctx {
     int G;
     pkv::AttnLaunch attn;
     int workers;
+    int tail_chunks;      // largest number of dynamic tail chunks per warp range
     void* ws;             // one allocation, carved below
     size_t ws_bytes;
     int* d_err;
+    int* d_claim;         // chunk counter of the attention's dynamic tail
     int* d_meta;
     float* d_part_o;
     float* d_part_ml;
@@ -133,11 +135,13 @@ pkv_status pkv_create(const pkv_config* cfg, pkv_ctx** out)
         return PKV_ERR_CUDA;
     }
 
-    const size_t max_workers = (size_t)ctx->attn.ctas * pkv::kAttnWarps;
+    // [error word, chunk counter | split geometry | partial rows | partial (m, l)];
+    // two partial slots per unit of the split, G rows each
+    const size_t units = pkv::max_units(ctx->attn.ctas * pkv::kAttnWarps, pkv::kMaxTailChunks);
     const size_t b_err = 256;
     const size_t b_cnt = ((size_t)(cfg->max_batch + 8) * sizeof(int) + 255) & ~(size_t)255;
-    const size_t b_po = 2 * max_workers * pkv::kMaxGroup * cfg->head_dim * sizeof(float);
-    const size_t b_pml = 2 * max_workers * pkv::kMaxGroup * 2 * sizeof(float);
+    const size_t b_po = 2 * units * ctx->G * cfg->head_dim * sizeof(float);
+    const size_t b_pml = 2 * units * ctx->G * 2 * sizeof(float);
     ctx->ws_bytes = b_err + b_cnt + b_po + b_pml;
     if (cudaMalloc(&ctx->ws, ctx->ws_bytes) != cudaSuccess) {
         cudaGetLastError();
@@ -146,6 +150,8 @@ pkv_status pkv_create(const pkv_config* cfg, pkv_ctx** out)
     }
     uint8_t* base = static_cast<uint8_t*>(ctx->ws);
     ctx->d_err = reinterpret_cast<int*>(base);
+    ctx->d_claim = reinterpret_cast<int*>(base + 128);
+    ctx->tail_chunks = pkv::kDefaultTailChunks;
     ctx->d_meta = reinterpret_cast<int*>(base + b_err);
     ctx->d_part_o = reinterpret_cast<float*>(base + b_err + b_cnt);
     ctx->d_part_ml = reinterpret_cast<float*>(base + b_err + b_cnt + b_po);
@@ -220,6 +226,7 @@ pkv_status pkv_decode_attn(pkv_ctx* ctx, const void* q, const void* k_pool, cons
     p.part_ml = ctx->d_part_ml;
     p.meta = ctx->d_meta;
     p.err = ctx->d_err;
+    p.claim = ctx->d_claim;
     p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)ctx->cfg.head_dim));
     p.batch = batch;
     p.bt_stride = bt_stride;
@@ -230,6 +237,7 @@ pkv_status pkv_decode_attn(pkv_ctx* ctx, const void* q, const void* k_pool, cons
     p.num_pages = ctx->cfg.num_pages;
     p.stages = ctx->attn.stages;
     p.workers = ctx->workers;
+    p.tail_chunks = ctx->tail_chunks;
     const cudaError_t e = pkv::launch_decode_attn(p, ctx->tmk, ctx->tmv, ctx->cfg.head_dim,
                                                   ctx->cfg.kv_dtype == PKV_KV_FP8_E4M3, ctx->attn, stream);
     return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
@@ -276,6 +284,13 @@ pkv_status pkv_set_workers(pkv_ctx* ctx, int workers)
 {
     if (!ctx || workers < 0) return PKV_ERR_INVALID_ARG;
     ctx->workers = workers;
+    return PKV_OK;
+}
+
+pkv_status pkv_set_tail_chunks(pkv_ctx* ctx, int max_chunks)
+{
+    if (!ctx || max_chunks < 0 || max_chunks > pkv::kMaxTailChunks) return PKV_ERR_INVALID_ARG;
+    ctx->tail_chunks = max_chunks;
     return PKV_OK;
 }
 

@@ -30,6 +30,26 @@ constexpr int kAttnMaxStages = PKV_ATTN_MAX_STAGES;
 constexpr int kMinTilesPerWorker = 8;
 constexpr int kMaxBatch = 8192;
 
+// Dynamic tail of the attention split: the last 1/kTailDen of every warp's
+// range (at most kTailMaxTiles tiles) is cut into at most kMaxTailChunks
+// chunks of at least kTailChunkTiles tiles that any warp may claim once its
+// own static part is done.  Only applies when every warp range holds at
+// least kTailMinTiles tiles.
+constexpr int kTailDen = 4;
+constexpr int kTailMaxTiles = 48;
+constexpr int kTailChunkTiles = 4;
+constexpr int kTailMinTiles = 32;
+constexpr int kMaxTailChunks = 8;
+// a chunk must outlast the producer's lead over the consumer (see decode_attn.cu)
+static_assert(kTailChunkTiles > PKV_ATTN_MAX_STAGES, "tail chunks must be longer than the TMA ring");
+constexpr int kDefaultTailChunks = 0;
+
+// Units the split may cut the tiles into (two partial slots each).
+inline size_t max_units(int max_workers, int tail_chunks)
+{
+    return (size_t)max_workers * (size_t)(tail_chunks + 1);
+}
+
 struct RopeParams {
     __nv_bfloat16* q;
     const __nv_bfloat16* k_new;
@@ -52,14 +72,16 @@ struct AttnParams {
     const float* v_scale;
     const int32_t* block_tables;
     const int32_t* seq_lens;
-    float* part_o;        // [2 * max_workers][kMaxGroup][D] fp32, unnormalised
-    float* part_ml;       // [2 * max_workers][kMaxGroup][2] fp32 (m in log2 units, l)
-    int* meta;            // [4 + max_batch + 1]: W, T (lo, hi), -, tile prefix; written by the attention kernel for the combine
+    float* part_o;        // [2 * units][G][D] fp32, unnormalised
+    float* part_ml;       // [2 * units][G][2] fp32 (m in log2 units, l)
+    int* meta;            // [4 + max_batch + 1]: W, T (lo, hi), K, tile prefix; written by the attention kernel for the combine
     int* err;
+    int* claim;           // chunk counter of the dynamic tail; zero when a launch starts, reset by the combine
     float scale_log2;     // log2(e) / sqrt(d)
     int batch, bt_stride, Hq, Hkv, G, P, num_pages;
     int stages;           // pipeline depth per warp
     int workers;          // 0: automatic
+    int tail_chunks;      // largest K (chunks per warp tail); 0: static split only
 };
 
 cudaError_t launch_rope_append(const RopeParams& p, cudaStream_t stream);

@@ -131,7 +131,8 @@ extern "C" pkv_status pkv_decode_attn_noalloc(const pkv_config* cfg, const void*
         cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return PKV_ERR_CUDA;
 
-    // scratch layout: [error word | split geometry | partial rows | partial (m, l)]
+    // scratch layout: [error word, chunk counter | split geometry | partial rows | partial (m, l)];
+    // a static split (no dynamic tail): two partial slots per warp
     const size_t workers = (size_t)num_sms * pkv::kAttnWarps;
     const size_t b_err = 256;
     const size_t b_cnt = ((size_t)(batch + 8) * sizeof(int) + 255) & ~(size_t)255;
@@ -159,6 +160,7 @@ extern "C" pkv_status pkv_decode_attn_noalloc(const pkv_config* cfg, const void*
     p.block_tables = block_tables;
     p.seq_lens = seq_lens;
     p.err = reinterpret_cast<int*>(base);
+    p.claim = reinterpret_cast<int*>(base + 128);
     p.meta = reinterpret_cast<int*>(base + b_err);
     p.part_o = reinterpret_cast<float*>(base + b_err + b_cnt);
     p.part_ml = reinterpret_cast<float*>(base + b_err + b_cnt + b_po);
@@ -172,6 +174,7 @@ extern "C" pkv_status pkv_decode_attn_noalloc(const pkv_config* cfg, const void*
     p.num_pages = cfg->num_pages;
     p.stages = L.stages;
     p.workers = 0;
+    p.tail_chunks = 0;
     return pkv::launch_decode_attn(p, tmk, tmv, cfg->head_dim, fp8, L, stream) == cudaSuccess ? PKV_OK
                                                                                               : PKV_ERR_CUDA;
 }

@@ -40,7 +40,8 @@ PKV_KV_FP8_E4M3 = 1
 
 # names of every symbol include/pkv.h declares
 EXPORTS = ("pkv_create", "pkv_rope_append", "pkv_decode_attn", "pkv_destroy", "pkv_status_str",
-           "pkv_check_device_error", "pkv_set_workers", "pkv_workspace_bytes", "pkv_decode_attn_noalloc")
+           "pkv_check_device_error", "pkv_set_workers", "pkv_workspace_bytes", "pkv_decode_attn_noalloc",
+           "pkv_set_tail_chunks")
 
 
 class pkv_config(C.Structure):
@@ -64,6 +65,8 @@ lib.pkv_check_device_error.argtypes = [_V, _V, C.POINTER(C.c_int)]
 lib.pkv_check_device_error.restype = C.c_int
 lib.pkv_set_workers.argtypes = [_V, C.c_int]
 lib.pkv_set_workers.restype = C.c_int
+lib.pkv_set_tail_chunks.argtypes = [_V, C.c_int]
+lib.pkv_set_tail_chunks.restype = C.c_int
 lib.pkv_workspace_bytes.argtypes = [_V]
 lib.pkv_workspace_bytes.restype = C.c_size_t
 lib.pkv_decode_attn_noalloc.argtypes = [C.POINTER(pkv_config), _V, _V, _V, _V, _V, _V, C.c_int, _V, C.c_int,
@@ -163,6 +166,10 @@ def pkv_check_device_error(ctx, stream=None):
 
 def pkv_set_workers(ctx, workers: int, check: bool = True) -> int:
     return _done(lib.pkv_set_workers(ctx, int(workers)), "pkv_set_workers", check)
+
+
+def pkv_set_tail_chunks(ctx, max_chunks: int, check: bool = True) -> int:
+    return _done(lib.pkv_set_tail_chunks(ctx, int(max_chunks)), "pkv_set_tail_chunks", check)
 
 
 def pkv_workspace_bytes(ctx) -> int:

@@ -74,6 +74,7 @@ def test_null_context_and_status_strings(pkv):
     assert pkv.lib.pkv_rope_append(None, None, None, None, None, None, None, None, None, 1, None, 1, None) == 1
     assert pkv.lib.pkv_decode_attn(None, None, None, None, None, None, None, 1, None, 1, None, None) == 1
     assert pkv.lib.pkv_set_workers(None, 3) == 1
+    assert pkv.lib.pkv_set_tail_chunks(None, 3) == 1
     assert pkv.lib.pkv_destroy(None) == 0
     assert pkv.lib.pkv_workspace_bytes(None) == 0
     for s in range(7):

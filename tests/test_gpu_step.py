@@ -148,7 +148,10 @@ def test_split_count_invariance(pkv, case_name):
     try:
         pkv.pkv_rope_append(ctx, dv["q"], dv["k_new"], dv["v_new"], dv["k_pool"], dv["v_pool"],
                             dv["k_scale"], dv["v_scale"], dv["block_tables"], dv["seq_lens"])
-        for workers in (1, 2, 7, 100, 0):
+        # static splits, then splits whose range tails are claimed dynamically
+        for tail, workers in [(0, 1), (0, 2), (0, 7), (0, 100), (0, 0), (1, 2), (8, 1), (8, 2), (8, 7),
+                              (8, 100), (8, 0)]:
+            pkv.pkv_set_tail_chunks(ctx, tail)
             pkv.pkv_set_workers(ctx, workers)
             out = torch.empty(w.batch, w.Hq, w.d, dtype=torch.bfloat16, device="cuda")
             pkv.pkv_decode_attn(ctx, dv["q"], dv["k_pool"], dv["v_pool"], dv["k_scale"], dv["v_scale"],
@@ -169,6 +172,26 @@ def test_split_count_invariance(pkv, case_name):
         for o in outs:
             mx, mean, _ = _gpu.errors(o, ref)
             assert mx <= _gpu.tol(w)["max"] and mean <= _gpu.tol(w)["mean"]
+
+
+def test_combine_merges_more_contributors_than_one_staging_block(pkv):
+    # one (request, kv head) pair of 270,001 tokens over 128 warps: 16,876
+    # tiles, 131 per warp range, a tail of 8 chunks per range -> 1,152 units
+    # all cut from the same pair, several times what the combine stages at
+    # once (256)
+    w = workloads.build("one_long_pair", 8, 1, 128, 64, False, 5e5, [270000], seed=11)
+    dv = _gpu.to_device(w)
+    ctx = _gpu.make_ctx(pkv, w)
+    try:
+        pkv.pkv_set_workers(ctx, 128)
+        pkv.pkv_set_tail_chunks(ctx, 8)
+        out = _gpu.gpu_step(pkv, ctx, dv)
+        assert pkv.pkv_check_device_error(ctx)[0] == pkv.PKV_OK
+    finally:
+        pkv.pkv_destroy(ctx)
+    _, ref = _gpu.oracle_request(w, 0)
+    mx, mean, _ = _gpu.errors(out[0:1].float(), ref[None])
+    assert mx <= _gpu.TOL_BF16["max"] and mean <= _gpu.TOL_BF16["mean"], (mx, mean)
 
 
 def test_one_token_context_returns_v_exactly(pkv):
