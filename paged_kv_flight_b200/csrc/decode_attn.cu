@@ -919,6 +919,126 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const AttnPara
     }
 }
 
+// The same merge with one warp per pair, for batches with many pairs: all
+// pairs then fit in about one wave and no shared memory or CTA barrier is
+// needed.  Lanes take contributors 32 at a time for m* and l* (online, then a
+// butterfly over the lanes) and for the weights; the weighted sum walks the
+// contributors with every lane on its own 16-byte pieces of the G x D
+// values, a piece of D = 128 belonging to head t for the t-th piece of the
+// lane and a piece of D = 64 to head 2t or 2t + 1 by lane half.
+constexpr int kCombineWarpThreads = 256;
+
+template <int D>
+__global__ void __launch_bounds__(kCombineWarpThreads, 2) combine_warp_kernel(const AttnParams p)
+{
+    constexpr unsigned kFullMask = 0xFFFFFFFFu;
+    constexpr int F4 = kMaxGroup * D / 4 / 32;   // 16-byte pieces per lane, at most
+    static_assert(D == 128 || D == 64, "head_dim");
+
+    if (blockIdx.x == 0 && threadIdx.x == 0) *p.claim = 0;   // the attention launch has ended
+    const int lane = threadIdx.x & 31;
+    const int pair = blockIdx.x * (kCombineWarpThreads / 32) + (threadIdx.x >> 5);
+    if (pair >= p.batch * p.Hkv) return;
+    const int b = pair / p.Hkv, kvh = pair - b * p.Hkv;
+    const int W = __ldg(&p.meta[0]);
+    const long long T = (long long)(unsigned)__ldg(&p.meta[1]) | ((long long)__ldg(&p.meta[2]) << 32);
+    const int* prefix = p.meta + 4;
+    const int pb = __ldg(&prefix[b]);
+    const int nt = __ldg(&prefix[b + 1]) - pb;
+    if (T == 0 || nt == 0) return;
+    Split sp = make_split(T, W, 0);
+    sp.K = __ldg(&p.meta[3]);   // as the attention launch chose it
+    const long long ts = (long long)pb * p.Hkv + (long long)kvh * nt;
+    const int U0 = sp.unit_of(ts), U1 = sp.unit_of(ts + nt - 1);
+    if (U0 == U1) return;
+    const int k = U1 - U0 + 1, G = p.G, GD4 = G * D / 4;
+    const int side0 = sp.ustart(U0) < ts ? 1 : 0;
+
+    // pass 1: m* and l* per head
+    float M[kMaxGroup], L[kMaxGroup];
+#pragma unroll
+    for (int g = 0; g < kMaxGroup; ++g) {
+        M[g] = -INFINITY;
+        L[g] = 0.f;
+    }
+    for (int i = lane; i < k; i += 32) {
+        const int slot = 2 * (U0 + i) + (i == 0 ? side0 : 0);
+#pragma unroll
+        for (int g = 0; g < kMaxGroup; ++g) {
+            if (g < G) {
+                const float2 ml = __ldg(reinterpret_cast<const float2*>(p.part_ml + ((size_t)slot * G + g) * 2));
+                const float m_new = fmaxf(M[g], ml.x);
+                const float ref = (m_new == -INFINITY) ? 0.f : m_new;
+                L[g] = L[g] * ex2(M[g] - ref) + ml.y * ex2(ml.x - ref);
+                M[g] = m_new;
+            }
+        }
+    }
+#pragma unroll
+    for (int g = 0; g < kMaxGroup; ++g) {
+        if (g < G) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const float m2 = __shfl_xor_sync(kFullMask, M[g], o), l2 = __shfl_xor_sync(kFullMask, L[g], o);
+                const float m_new = fmaxf(M[g], m2);
+                const float ref = (m_new == -INFINITY) ? 0.f : m_new;
+                L[g] = L[g] * ex2(M[g] - ref) + l2 * ex2(m2 - ref);
+                M[g] = m_new;
+            }
+            if (M[g] == -INFINITY) M[g] = 0.f;
+        }
+    }
+
+    // pass 2: weighted sum, contributors in batches of 32 (lane j holds the
+    // slot and the weights of contributor i0 + j)
+    float4 acc[F4];
+#pragma unroll
+    for (int t = 0; t < F4; ++t) acc[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i0 = 0; i0 < k; i0 += 32) {
+        const int i = i0 + lane;
+        int slot_l = 0;
+        float wl[kMaxGroup];
+#pragma unroll
+        for (int g = 0; g < kMaxGroup; ++g) wl[g] = 0.f;
+        if (i < k) {
+            slot_l = 2 * (U0 + i) + (i == 0 ? side0 : 0);
+#pragma unroll
+            for (int g = 0; g < kMaxGroup; ++g)
+                if (g < G) wl[g] = ex2(__ldg(p.part_ml + ((size_t)slot_l * G + g) * 2) - M[g]) / L[g];
+        }
+        const int n = min(32, k - i0);
+        for (int j = 0; j < n; ++j) {
+            const int slot = __shfl_sync(kFullMask, slot_l, j);
+            const float4* src = reinterpret_cast<const float4*>(p.part_o + (size_t)slot * G * D);
+#pragma unroll
+            for (int t = 0; t < F4; ++t) {
+                float w;
+                if constexpr (D == 128) {
+                    w = __shfl_sync(kFullMask, wl[t], j);
+                } else {
+                    const float wa = __shfl_sync(kFullMask, wl[2 * t], j);
+                    const float wb = __shfl_sync(kFullMask, wl[2 * t + 1], j);
+                    w = lane < 16 ? wa : wb;
+                }
+                const int f = lane + 32 * t;
+                if (f < GD4) {
+                    const float4 v = __ldg(src + f);
+                    acc[t].x += w * v.x;
+                    acc[t].y += w * v.y;
+                    acc[t].z += w * v.z;
+                    acc[t].w += w * v.w;
+                }
+            }
+        }
+    }
+    uint2* const dst = reinterpret_cast<uint2*>(p.out + ((size_t)b * p.Hq + (size_t)kvh * G) * D);
+#pragma unroll
+    for (int t = 0; t < F4; ++t) {
+        const int f = lane + 32 * t;
+        if (f < GD4) dst[f] = make_uint2(pack_bf16(acc[t].x, acc[t].y), pack_bf16(acc[t].z, acc[t].w));
+    }
+}
+
 template <int D, bool FP8>
 size_t smem_bytes_for(int stages, int max_batch)
 {
@@ -967,16 +1087,25 @@ cudaError_t launch_decode_attn(const AttnParams& p, const CUtensorMap& tmk, cons
     const dim3 grid(L.ctas), block(kAttnWarps * 32);
     AttnParams q = p;
     q.stages = L.stages;
-    const dim3 cgrid((unsigned)(p.batch * p.Hkv)), cblock(kCombineThreads);
+    // the combine: a warp per pair when there are at least two pairs per
+    // attention warp slot of a wave (many pairs, each with few
+    // contributors), else a CTA per pair
+    const int pairs = p.batch * p.Hkv;
+    const bool warp_mode = pairs >= 2 * L.ctas;
+    const dim3 cgrid((unsigned)pairs), cblock(kCombineThreads);
     const size_t csmem = combine_smem_bytes((int)max_units(L.ctas * kAttnWarps, p.tail_chunks), p.G, head_dim);
+    const int wpc = kCombineWarpThreads / 32;
+    const dim3 wgrid((unsigned)((pairs + wpc - 1) / wpc)), wblock(kCombineWarpThreads);
     if (head_dim == 128) {
         if (fp8) decode_attn_kernel<128, true, kAttnWarps><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
         else decode_attn_kernel<128, false, kAttnWarps><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
-        combine_kernel<128><<<cgrid, cblock, csmem, stream>>>(q);
+        if (warp_mode) combine_warp_kernel<128><<<wgrid, wblock, 0, stream>>>(q);
+        else combine_kernel<128><<<cgrid, cblock, csmem, stream>>>(q);
     } else {
         if (fp8) decode_attn_kernel<64, true, kAttnWarps><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
         else decode_attn_kernel<64, false, kAttnWarps><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
-        combine_kernel<64><<<cgrid, cblock, csmem, stream>>>(q);
+        if (warp_mode) combine_warp_kernel<64><<<wgrid, wblock, 0, stream>>>(q);
+        else combine_kernel<64><<<cgrid, cblock, csmem, stream>>>(q);
     }
     return cudaGetLastError();
 }

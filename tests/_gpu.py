@@ -20,12 +20,13 @@ def tol(w: Workload):
 
 
 def to_device(w: Workload, device="cuda"):
-    """Device copies of every step input (the generator may draw on the CPU)."""
-    d = dict(q=w.q.to(device).contiguous(), k_new=w.k_new.to(device).contiguous(),
-             v_new=w.v_new.to(device).contiguous(), k_pool=w.k_pool.to(device).contiguous(),
-             v_pool=w.v_pool.to(device).contiguous(),
-             k_scale=None if w.k_scale is None else w.k_scale.to(device).contiguous(),
-             v_scale=None if w.v_scale is None else w.v_scale.to(device).contiguous(),
+    """Device copies of every step input (the generator may draw on the CPU).
+    Always copies, also when the workload already lives on the device, so the
+    step never writes into the generator's original tensors."""
+    def cp(t):
+        return None if t is None else t.to(device, copy=True).contiguous()
+    d = dict(q=cp(w.q), k_new=cp(w.k_new), v_new=cp(w.v_new), k_pool=cp(w.k_pool), v_pool=cp(w.v_pool),
+             k_scale=cp(w.k_scale), v_scale=cp(w.v_scale),
              block_tables=torch.from_numpy(w.block_tables).to(device).contiguous(),
              seq_lens=torch.from_numpy(w.seq_lens).to(device).contiguous())
     return d

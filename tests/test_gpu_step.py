@@ -194,6 +194,38 @@ def test_combine_merges_more_contributors_than_one_staging_block(pkv):
     assert mx <= _gpu.TOL_BF16["max"] and mean <= _gpu.TOL_BF16["mean"], (mx, mean)
 
 
+def test_warp_combine_merges_more_than_32_contributors(pkv):
+    # 40 requests x 8 kv heads = 320 pairs (the combine then runs one warp per
+    # pair) of about 1,000 tiles each; 1,184 warp ranges of about 270 tiles
+    # with a tail of 8 chunks -> 9 units per range, about 35 per pair, more
+    # than the 32 contributors one pass of the warp handles
+    lengths = [16000 + 37 * i for i in range(40)]
+    w = workloads.build("warp_combine", 32, 8, 128, 32, False, 5e5, lengths, seed=13, device="cuda")
+    picks = (0, 17, 39)
+    views = {b: _gpu.request_view(w, b) for b in picks}   # original inputs: the step rotates q in place
+    dv = _gpu.to_device(w)
+    ctx = _gpu.make_ctx(pkv, w)
+    try:
+        pkv.pkv_set_tail_chunks(ctx, 8)
+        out = _gpu.gpu_step(pkv, ctx, dv)
+        assert pkv.pkv_check_device_error(ctx)[0] == pkv.PKV_OK
+    finally:
+        pkv.pkv_destroy(ctx)
+    for b in picks:
+        cfg, h = views[b]
+        assert oracle.rope_append(cfg, h["q"], h["k_new"], h["v_new"], h["k_pool"], h["v_pool"], None, None,
+                                  h["block_tables"], h["seq_lens"]) == 0
+        ref = np.full((w.Hq, w.d), np.nan)
+        G = w.Hq // w.Hkv
+        for kvh in range(w.Hkv):
+            o, st = oracle.decode_attn_group(cfg, h["q"], h["k_pool"], h["v_pool"], None, None,
+                                             h["block_tables"], h["seq_lens"], 0, kvh)
+            assert st == 0
+            ref[kvh * G:(kvh + 1) * G] = o
+        mx, mean, _ = _gpu.errors(out[b], ref)
+        assert mx <= _gpu.TOL_BF16["max"] and mean <= _gpu.TOL_BF16["mean"], (b, mx, mean)
+
+
 def test_one_token_context_returns_v_exactly(pkv):
     w = workloads.build("one", 32, 8, 128, 32, False, 5e5, [0, 0, 0, 0], seed=3)
     dv = _gpu.to_device(w)
