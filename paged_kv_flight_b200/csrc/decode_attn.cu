@@ -954,12 +954,14 @@ __global__ void __launch_bounds__(kCombineWarpThreads, 2) combine_warp_kernel(co
     const int k = U1 - U0 + 1, G = p.G, GD4 = G * D / 4;
     const int side0 = sp.ustart(U0) < ts ? 1 : 0;
 
-    // pass 1: m* and l* per head
-    float M[kMaxGroup], L[kMaxGroup];
+    // pass 1: m* and l* per head; lane j keeps the m of its first contributor
+    // (j) so that the weights of the first 32 need no second load
+    float M[kMaxGroup], L[kMaxGroup], m_own[kMaxGroup];
 #pragma unroll
     for (int g = 0; g < kMaxGroup; ++g) {
         M[g] = -INFINITY;
         L[g] = 0.f;
+        m_own[g] = -INFINITY;
     }
     for (int i = lane; i < k; i += 32) {
         const int slot = 2 * (U0 + i) + (i == 0 ? side0 : 0);
@@ -967,6 +969,7 @@ __global__ void __launch_bounds__(kCombineWarpThreads, 2) combine_warp_kernel(co
         for (int g = 0; g < kMaxGroup; ++g) {
             if (g < G) {
                 const float2 ml = __ldg(reinterpret_cast<const float2*>(p.part_ml + ((size_t)slot * G + g) * 2));
+                if (i == lane) m_own[g] = ml.x;
                 const float m_new = fmaxf(M[g], ml.x);
                 const float ref = (m_new == -INFINITY) ? 0.f : m_new;
                 L[g] = L[g] * ex2(M[g] - ref) + ml.y * ex2(ml.x - ref);
@@ -1003,8 +1006,12 @@ __global__ void __launch_bounds__(kCombineWarpThreads, 2) combine_warp_kernel(co
         if (i < k) {
             slot_l = 2 * (U0 + i) + (i == 0 ? side0 : 0);
 #pragma unroll
-            for (int g = 0; g < kMaxGroup; ++g)
-                if (g < G) wl[g] = ex2(__ldg(p.part_ml + ((size_t)slot_l * G + g) * 2) - M[g]) / L[g];
+            for (int g = 0; g < kMaxGroup; ++g) {
+                if (g < G) {
+                    const float m = (i0 == 0) ? m_own[g] : __ldg(p.part_ml + ((size_t)slot_l * G + g) * 2);
+                    wl[g] = ex2(m - M[g]) / L[g];
+                }
+            }
         }
         const int n = min(32, k - i0);
         for (int j = 0; j < n; ++j) {
