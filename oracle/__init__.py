@@ -56,6 +56,15 @@ def _load():
         lib.orc_decode_attn.argtypes = [C.POINTER(_Cfg), P, P, P, P, P, P, C.c_int,
                                         P, C.c_int, P]
         lib.orc_decode_attn.restype = C.c_int
+        lib.orc_rope_append_tokens.argtypes = [C.POINTER(_Cfg), P, P, P, P, P, P, P, P,
+                                               C.c_int, P, C.c_int, C.c_int]
+        lib.orc_rope_append_tokens.restype = C.c_int
+        lib.orc_decode_attn_tokens_group.argtypes = [C.POINTER(_Cfg), P, P, P, P, P, P, C.c_int, P,
+                                                     C.c_int, C.c_int, C.c_int, C.c_int, P]
+        lib.orc_decode_attn_tokens_group.restype = C.c_int
+        lib.orc_decode_attn_tokens.argtypes = [C.POINTER(_Cfg), P, P, P, P, P, P, C.c_int, P,
+                                               C.c_int, C.c_int, P]
+        lib.orc_decode_attn_tokens.restype = C.c_int
         _lib = lib
     return _lib
 
@@ -179,4 +188,53 @@ def decode_attn(cfg: OracleConfig, q, k_pool, v_pool, k_scale, v_scale, block_ta
     st = _load().orc_decode_attn(C.byref(c), _ptr(q), _ptr(k_pool), _ptr(v_pool),
                                  _ptr(k_scale), _ptr(v_scale), _ptr(block_tables),
                                  block_tables.shape[1], _ptr(seq_lens), B, _ptr(out))
+    return out, st
+
+
+# ---- several new tokens per request (speculative-decode verification) ------
+
+def rope_append_tokens(cfg: OracleConfig, q, k_new, v_new, k_pool, v_pool, k_scale, v_scale,
+                       block_tables, seq_lens) -> int:
+    """In place, for q [batch, q_len, Hq, d] and k_new / v_new [batch, q_len,
+    Hkv, d]: new token t of request b is rotated at position L_b + t and its
+    k / v stored in that position's page slot.  Returns the oracle status."""
+    _need(q, np.uint16, "q"); _need(k_new, np.uint16, "k_new"); _need(v_new, np.uint16, "v_new")
+    _need(k_pool, _pool_dtype(cfg), "k_pool"); _need(v_pool, _pool_dtype(cfg), "v_pool")
+    _need(block_tables, np.int32, "block_tables"); _need(seq_lens, np.int32, "seq_lens")
+    if cfg.kv_fp8:
+        _need(k_scale, np.float32, "k_scale"); _need(v_scale, np.float32, "v_scale")
+    B, Q = q.shape[0], q.shape[1]
+    c = cfg._c()
+    return _load().orc_rope_append_tokens(C.byref(c), _ptr(q), _ptr(k_new), _ptr(v_new),
+                                          _ptr(k_pool), _ptr(v_pool), _ptr(k_scale), _ptr(v_scale),
+                                          _ptr(block_tables), block_tables.shape[1],
+                                          _ptr(seq_lens), B, Q)
+
+
+def decode_attn_tokens_group(cfg: OracleConfig, q, k_pool, v_pool, k_scale, v_scale,
+                             block_tables, seq_lens, b: int, t: int, kvh: int):
+    """fp64 output [G, d] of new token t of request b, kv head kvh (it attends
+    tokens 0 .. L_b + t); (out, status).  q is [batch, q_len, Hq, d]."""
+    G = cfg.num_q_heads // cfg.num_kv_heads
+    out = np.zeros((G, cfg.head_dim), np.float64)
+    c = cfg._c()
+    st = _load().orc_decode_attn_tokens_group(C.byref(c), _ptr(q), _ptr(k_pool), _ptr(v_pool),
+                                              _ptr(k_scale), _ptr(v_scale), _ptr(block_tables),
+                                              block_tables.shape[1], _ptr(seq_lens), q.shape[1],
+                                              int(b), int(t), int(kvh), _ptr(out))
+    return out, st
+
+
+def decode_attn_tokens(cfg: OracleConfig, q, k_pool, v_pool, k_scale, v_scale, block_tables,
+                       seq_lens):
+    """fp64 output [batch, q_len, Hq, d]; (out, status)."""
+    _need(q, np.uint16, "q")
+    _need(k_pool, _pool_dtype(cfg), "k_pool"); _need(v_pool, _pool_dtype(cfg), "v_pool")
+    _need(block_tables, np.int32, "block_tables"); _need(seq_lens, np.int32, "seq_lens")
+    B, Q = q.shape[0], q.shape[1]
+    out = np.zeros((B, Q, cfg.num_q_heads, cfg.head_dim), np.float64)
+    c = cfg._c()
+    st = _load().orc_decode_attn_tokens(C.byref(c), _ptr(q), _ptr(k_pool), _ptr(v_pool),
+                                        _ptr(k_scale), _ptr(v_scale), _ptr(block_tables),
+                                        block_tables.shape[1], _ptr(seq_lens), B, Q, _ptr(out))
     return out, st

@@ -255,24 +255,15 @@ static double kv_value(const orc_cfg* cfg, const void* pool, const float* scale,
            (double)scale[(size_t)page * cfg->num_kv_heads + kvh];
 }
 
-int orc_decode_attn_group(const orc_cfg* cfg, const uint16_t* q,
-                          const void* k_pool, const void* v_pool,
-                          const float* k_scale, const float* v_scale,
-                          const int32_t* block_tables, int bt_stride,
-                          const int32_t* seq_lens, int b, int kvh, double* out)
+/* The definition for G query rows (bf16 bits, G x d, the heads kvh*G ..
+ * kvh*G + G-1) over the first n tokens of one request's block-table row bt:
+ * explicit gather of the tokens in logical order, then per row
+ * o = softmax(q K^T / sqrt(d)) V with the maximum subtracted, in fp64. */
+static int attend_rows(const orc_cfg* cfg, const uint16_t* qrows, const void* k_pool,
+                       const void* v_pool, const float* k_scale, const float* v_scale,
+                       const int32_t* bt, int n, int kvh, double* out)
 {
-    if (!cfg_ok(cfg) || !q || !k_pool || !v_pool || !block_tables || !seq_lens || !out)
-        return ORC_ERR_ARG;
-    if (cfg->kv_fp8 && (!k_scale || !v_scale)) return ORC_ERR_ARG;
-    if (kvh < 0 || kvh >= cfg->num_kv_heads || b < 0 || bt_stride <= 0) return ORC_ERR_ARG;
-
-    const int Hq = cfg->num_q_heads, Hkv = cfg->num_kv_heads, d = cfg->head_dim;
-    const int P = cfg->page_size, G = Hq / Hkv;
-    const int L = seq_lens[b];
-    if (L < 0 || (long long)L >= (long long)bt_stride * P) return ORC_ERR_RANGE;
-    const int n = L + 1;
-
-    /* explicit gather of this request's tokens, in logical order */
+    const int d = cfg->head_dim, P = cfg->page_size, G = cfg->num_q_heads / cfg->num_kv_heads;
     double* K = (double*)malloc(sizeof(double) * (size_t)n * d);
     double* V = (double*)malloc(sizeof(double) * (size_t)n * d);
     double* w = (double*)malloc(sizeof(double) * (size_t)n);
@@ -280,7 +271,7 @@ int orc_decode_attn_group(const orc_cfg* cfg, const uint16_t* q,
     if (!K || !V || !w || !qh) { free(K); free(V); free(w); free(qh); return ORC_ERR_ARG; }
     int status = ORC_OK;
     for (int t = 0; t < n && status == ORC_OK; ++t) {
-        const int page = block_tables[(size_t)b * bt_stride + t / P];
+        const int page = bt[t / P];
         if (page < 0 || page >= cfg->num_pages) { status = ORC_ERR_RANGE; break; }
         for (int j = 0; j < d; ++j) {
             K[(size_t)t * d + j] = kv_value(cfg, k_pool, k_scale, page, kvh, t % P, j);
@@ -291,8 +282,7 @@ int orc_decode_attn_group(const orc_cfg* cfg, const uint16_t* q,
     if (status == ORC_OK) {
         const double inv_sqrt_d = 1.0 / sqrt((double)d);
         for (int g = 0; g < G; ++g) {
-            const int h = kvh * G + g;
-            for (int j = 0; j < d; ++j) qh[j] = orc_bf16_decode(q[((size_t)b * Hq + h) * d + j]);
+            for (int j = 0; j < d; ++j) qh[j] = orc_bf16_decode(qrows[(size_t)g * d + j]);
             double m = -INFINITY;
             for (int t = 0; t < n; ++t) {
                 double s = 0.0;
@@ -319,6 +309,25 @@ int orc_decode_attn_group(const orc_cfg* cfg, const uint16_t* q,
     return status;
 }
 
+int orc_decode_attn_group(const orc_cfg* cfg, const uint16_t* q,
+                          const void* k_pool, const void* v_pool,
+                          const float* k_scale, const float* v_scale,
+                          const int32_t* block_tables, int bt_stride,
+                          const int32_t* seq_lens, int b, int kvh, double* out)
+{
+    if (!cfg_ok(cfg) || !q || !k_pool || !v_pool || !block_tables || !seq_lens || !out)
+        return ORC_ERR_ARG;
+    if (cfg->kv_fp8 && (!k_scale || !v_scale)) return ORC_ERR_ARG;
+    if (kvh < 0 || kvh >= cfg->num_kv_heads || b < 0 || bt_stride <= 0) return ORC_ERR_ARG;
+
+    const int Hq = cfg->num_q_heads, Hkv = cfg->num_kv_heads, d = cfg->head_dim;
+    const int P = cfg->page_size, G = Hq / Hkv;
+    const int L = seq_lens[b];
+    if (L < 0 || (long long)L >= (long long)bt_stride * P) return ORC_ERR_RANGE;
+    return attend_rows(cfg, q + ((size_t)b * Hq + (size_t)kvh * G) * d, k_pool, v_pool, k_scale, v_scale,
+                       block_tables + (size_t)b * bt_stride, L + 1, kvh, out);
+}
+
 int orc_decode_attn(const orc_cfg* cfg, const uint16_t* q,
                     const void* k_pool, const void* v_pool,
                     const float* k_scale, const float* v_scale,
@@ -337,6 +346,131 @@ int orc_decode_attn(const orc_cfg* cfg, const uint16_t* q,
             if (s != ORC_OK) {
                 for (size_t i = 0; i < (size_t)G * d; ++i) dst[i] = NAN;
                 if (status == ORC_OK) status = s;
+            }
+        }
+    }
+    return status;
+}
+
+/* ------------------------------------------------------------------ */
+/* Several new tokens per request: a draft proposes tokens and the      */
+/* target checks all of them in one pass ("Scaling TensorRT-LLM",       */
+/* section "3. Speculative Decoding for Tail Latency"; "TensorRT-LLM    */
+/* Guide", section "2. Pipelined Speculative Decoding").  New token t   */
+/* (0 <= t < q_len) of request b sits at position L_b + t; q is         */
+/* [batch][q_len][Hq][d], k_new / v_new [batch][q_len][Hkv][d].         */
+/* ------------------------------------------------------------------ */
+
+int orc_rope_append_tokens(const orc_cfg* cfg,
+                           uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,
+                           void* k_pool, void* v_pool,
+                           const float* k_scale, const float* v_scale,
+                           const int32_t* block_tables, int bt_stride,
+                           const int32_t* seq_lens, int batch, int q_len)
+{
+    if (!cfg_ok(cfg) || batch < 0 || bt_stride <= 0 || q_len <= 0) return ORC_ERR_ARG;
+    if (batch == 0) return ORC_OK;
+    if (!q || !k_new || !v_new || !k_pool || !v_pool || !block_tables || !seq_lens)
+        return ORC_ERR_ARG;
+    if (cfg->kv_fp8 && (!k_scale || !v_scale)) return ORC_ERR_ARG;
+
+    const int Hq = cfg->num_q_heads, Hkv = cfg->num_kv_heads, d = cfg->head_dim;
+    const int P = cfg->page_size;
+    double* x = (double*)malloc(sizeof(double) * d);
+    double* y = (double*)malloc(sizeof(double) * d);
+    if (!x || !y) { free(x); free(y); return ORC_ERR_ARG; }
+    int status = ORC_OK;
+
+    for (int b = 0; b < batch; ++b) {
+        for (int t = 0; t < q_len; ++t) {
+            const long long pos = (long long)seq_lens[b] + t;   /* position of new token t */
+            if (seq_lens[b] < 0 || pos >= (long long)bt_stride * P) { status = ORC_ERR_RANGE; continue; }
+            const int page = block_tables[(size_t)b * bt_stride + pos / P];
+            if (page < 0 || page >= cfg->num_pages) { status = ORC_ERR_RANGE; continue; }
+            const int slot = (int)(pos % P);
+            const size_t bt_row = (size_t)b * q_len + t;   /* row of (b, t) in q, k_new, v_new */
+
+            for (int h = 0; h < Hq; ++h) {
+                uint16_t* row = q + (bt_row * Hq + h) * d;
+                for (int j = 0; j < d; ++j) x[j] = orc_bf16_decode(row[j]);
+                orc_rope_f64(x, y, d, (double)pos, cfg->rope_base);
+                for (int j = 0; j < d; ++j) row[j] = orc_bf16_encode_rne(y[j]);
+            }
+            for (int kvh = 0; kvh < Hkv; ++kvh) {
+                const uint16_t* krow = k_new + (bt_row * Hkv + kvh) * d;
+                const uint16_t* vrow = v_new + (bt_row * Hkv + kvh) * d;
+                for (int j = 0; j < d; ++j) x[j] = orc_bf16_decode(krow[j]);
+                orc_rope_f64(x, y, d, (double)pos, cfg->rope_base);
+                const size_t dst = pool_row(cfg, page, kvh, slot) * (size_t)d;
+                if (!cfg->kv_fp8) {
+                    uint16_t* kp = (uint16_t*)k_pool;
+                    uint16_t* vp = (uint16_t*)v_pool;
+                    for (int j = 0; j < d; ++j) {
+                        kp[dst + j] = orc_bf16_encode_rne(y[j]);
+                        vp[dst + j] = vrow[j];
+                    }
+                } else {
+                    uint8_t* kp = (uint8_t*)k_pool;
+                    uint8_t* vp = (uint8_t*)v_pool;
+                    const double sk = k_scale[(size_t)page * Hkv + kvh];
+                    const double sv = v_scale[(size_t)page * Hkv + kvh];
+                    for (int j = 0; j < d; ++j) {
+                        kp[dst + j] = orc_e4m3_encode_satfinite(orc_f32_round(y[j] / sk));
+                        vp[dst + j] = orc_e4m3_encode_satfinite(
+                            orc_f32_round(orc_bf16_decode(vrow[j]) / sv));
+                    }
+                }
+            }
+        }
+    }
+    free(x);
+    free(y);
+    return status;
+}
+
+/* New token t attends tokens 0 .. L_b + t: everything cached, the new
+ * tokens before it and itself, none after it (each candidate is checked as
+ * if the ones before it had been accepted). */
+int orc_decode_attn_tokens_group(const orc_cfg* cfg, const uint16_t* q,
+                                 const void* k_pool, const void* v_pool,
+                                 const float* k_scale, const float* v_scale,
+                                 const int32_t* block_tables, int bt_stride,
+                                 const int32_t* seq_lens, int q_len, int b, int t, int kvh,
+                                 double* out)
+{
+    if (!cfg_ok(cfg) || !q || !k_pool || !v_pool || !block_tables || !seq_lens || !out)
+        return ORC_ERR_ARG;
+    if (cfg->kv_fp8 && (!k_scale || !v_scale)) return ORC_ERR_ARG;
+    if (q_len <= 0 || t < 0 || t >= q_len || kvh < 0 || kvh >= cfg->num_kv_heads || b < 0 || bt_stride <= 0)
+        return ORC_ERR_ARG;
+    const int Hq = cfg->num_q_heads, G = Hq / cfg->num_kv_heads, d = cfg->head_dim;
+    const long long n = (long long)seq_lens[b] + t + 1;
+    if (seq_lens[b] < 0 || n > (long long)bt_stride * cfg->page_size) return ORC_ERR_RANGE;
+    const size_t bt_row = (size_t)b * q_len + t;
+    return attend_rows(cfg, q + (bt_row * Hq + (size_t)kvh * G) * d, k_pool, v_pool, k_scale, v_scale,
+                       block_tables + (size_t)b * bt_stride, (int)n, kvh, out);
+}
+
+int orc_decode_attn_tokens(const orc_cfg* cfg, const uint16_t* q,
+                           const void* k_pool, const void* v_pool,
+                           const float* k_scale, const float* v_scale,
+                           const int32_t* block_tables, int bt_stride,
+                           const int32_t* seq_lens, int batch, int q_len, double* out)
+{
+    if (!cfg_ok(cfg) || batch < 0 || q_len <= 0 || !out) return ORC_ERR_ARG;
+    const int Hq = cfg->num_q_heads, Hkv = cfg->num_kv_heads, d = cfg->head_dim;
+    const int G = Hq / Hkv;
+    int status = ORC_OK;
+    for (int b = 0; b < batch; ++b) {
+        for (int t = 0; t < q_len; ++t) {
+            for (int kvh = 0; kvh < Hkv; ++kvh) {
+                double* dst = out + (((size_t)b * q_len + t) * Hq + (size_t)kvh * G) * d;
+                int s = orc_decode_attn_tokens_group(cfg, q, k_pool, v_pool, k_scale, v_scale, block_tables,
+                                                     bt_stride, seq_lens, q_len, b, t, kvh, dst);
+                if (s != ORC_OK) {
+                    for (size_t i = 0; i < (size_t)G * d; ++i) dst[i] = NAN;
+                    if (status == ORC_OK) status = s;
+                }
             }
         }
     }

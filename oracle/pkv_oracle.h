@@ -103,6 +103,34 @@ int orc_decode_attn(const orc_cfg* cfg, const uint16_t* q,
                     const int32_t* block_tables, int bt_stride,
                     const int32_t* seq_lens, int batch, double* out);
 
+/* ---- several new tokens per request ---------------------------------- */
+/* Speculative-decode verification: new token t (0 <= t < q_len) of request
+ * b sits at position L_b + t.  q is [batch][q_len][Hq][d] (rotated in
+ * place), k_new / v_new [batch][q_len][Hkv][d]; each token is rotated and
+ * stored exactly as orc_rope_append stores the single new token. */
+int orc_rope_append_tokens(const orc_cfg* cfg,
+                           uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,
+                           void* k_pool, void* v_pool,
+                           const float* k_scale, const float* v_scale,
+                           const int32_t* block_tables, int bt_stride,
+                           const int32_t* seq_lens, int batch, int q_len);
+
+/* New token t attends tokens 0 .. L_b + t (causal among the new tokens):
+ * out[g*d + j] for the G query heads of kv head kvh. */
+int orc_decode_attn_tokens_group(const orc_cfg* cfg, const uint16_t* q,
+                                 const void* k_pool, const void* v_pool,
+                                 const float* k_scale, const float* v_scale,
+                                 const int32_t* block_tables, int bt_stride,
+                                 const int32_t* seq_lens, int q_len, int b, int t, int kvh,
+                                 double* out);
+
+/* All groups: out is [batch][q_len][Hq][d] fp64. */
+int orc_decode_attn_tokens(const orc_cfg* cfg, const uint16_t* q,
+                           const void* k_pool, const void* v_pool,
+                           const float* k_scale, const float* v_scale,
+                           const int32_t* block_tables, int bt_stride,
+                           const int32_t* seq_lens, int batch, int q_len, double* out);
+
 #ifdef __cplusplus
 }
 #endif

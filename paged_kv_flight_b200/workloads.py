@@ -15,8 +15,10 @@ Virtualization").
 Recipe (all seeded):
   * lengths L_b (tokens cached before the step) per configuration, drawn
     with numpy ``default_rng(seed)``;
-  * each request owns ceil((L_b + 1) / P) pages, the last one holding the
-    slot the new token lands in; physical page ids are the first
+  * each request owns ceil((L_b + q_len) / P) pages, the last ones holding
+    the slots the q_len new tokens land in (q_len = 1 for the five decode
+    configurations, 4 for the speculative-verification one); physical page
+    ids are the first
     sum(pages) entries of a seeded permutation of the pool, handed out in
     logical order; the pool has 10% free pages (64 pages for ``tiny``);
   * block-table entries past a request's pages are -1;
@@ -52,8 +54,12 @@ _SHAPES = {
     "hetero70b": dict(index=2, Hq=64, Hkv=8, d=128, P=16, kv_fp8=False, base=5e5),
     "longctx":   dict(index=3, Hq=32, Hkv=8, d=128, P=64, kv_fp8=False, base=5e5),
     "fp8":       dict(index=4, Hq=32, Hkv=8, d=128, P=32, kv_fp8=True,  base=5e5),
+    # several new tokens per request (speculative-decode verification)
+    "spec4":     dict(index=5, Hq=32, Hkv=8, d=128, P=32, kv_fp8=False, base=5e5, q_len=4),
 }
-CONFIG_NAMES = tuple(_SHAPES)
+# the five single-token decode configurations, and the multi-token one
+CONFIG_NAMES = ("tiny", "llama8b", "hetero70b", "longctx", "fp8")
+TOKEN_CONFIG_NAMES = ("spec4",)
 
 DESCRIPTIONS = {
     "tiny": "4 requests, cached lengths {17,64,100,255}, Hq 8 / Hkv 2, d 64, page 16, "
@@ -66,6 +72,9 @@ DESCRIPTIONS = {
                "d 128, page 64, bf16 KV N(0,1), RoPE base 5e5",
     "fp8": "fp8 KV: batch 128, lengths log-normal(median 1024, sigma 1) clipped [16,16384], "
            "Hq 32 / Hkv 8, d 128, page 32, E4M3 KV with per-(page, kv head) scale amax/448",
+    "spec4": "speculative-decode verification on the Llama-3-8B-shaped layer: batch 64, cached "
+             "lengths U[128,4096], 4 new tokens per request (positions L..L+3, causal among "
+             "them), Hq 32 / Hkv 8, d 128, page 32, bf16 KV N(0,1), RoPE base 5e5, pool +10%",
 }
 
 
@@ -77,7 +86,7 @@ def draw_lengths(name: str, rng: np.random.Generator) -> np.ndarray:
     """Cached lengths L_b (before the step) for a named configuration."""
     if name == "tiny":
         return np.array([17, 64, 100, 255], np.int64)
-    if name == "llama8b":
+    if name in ("llama8b", "spec4"):
         return rng.integers(128, 4096, size=64, endpoint=True)
     if name == "hetero70b":
         B = 256
@@ -107,14 +116,15 @@ class Workload:
     seq_lens: np.ndarray          # [B] int32, L_b before the step
     block_tables: np.ndarray      # [B, bt_stride] int32, -1 past the used pages
     num_pages: int
-    q: torch.Tensor               # [B, Hq, d] bf16
-    k_new: torch.Tensor           # [B, Hkv, d] bf16
-    v_new: torch.Tensor           # [B, Hkv, d] bf16
+    q: torch.Tensor               # [B, Hq, d] bf16; [B, q_len, Hq, d] when q_len > 1
+    k_new: torch.Tensor           # [B, Hkv, d] bf16; [B, q_len, Hkv, d] when q_len > 1
+    v_new: torch.Tensor           # as k_new
     k_pool: torch.Tensor          # [num_pages, Hkv, P, d] bf16 or uint8 (E4M3 codes)
     v_pool: torch.Tensor
     k_scale: Optional[torch.Tensor] = None   # [num_pages, Hkv] fp32 (fp8 only)
     v_scale: Optional[torch.Tensor] = None
     seed: int = 0
+    q_len: int = 1                # new tokens per request (positions L_b .. L_b + q_len - 1)
     extra: dict = field(default_factory=dict)
 
     @property
@@ -131,8 +141,8 @@ class Workload:
 
 
 def _assign_pages(lengths: np.ndarray, P: int, num_pages: Optional[int],
-                  rng: np.random.Generator):
-    pages_needed = (lengths + 1 + P - 1) // P          # includes the landing page
+                  rng: np.random.Generator, q_len: int = 1):
+    pages_needed = (lengths + q_len + P - 1) // P      # includes the landing page(s)
     total = int(pages_needed.sum())
     if num_pages is None:
         num_pages = int(math.ceil(1.1 * total))
@@ -152,7 +162,7 @@ def _resident_mask(lengths: np.ndarray, bt: np.ndarray, num_pages: int, P: int) 
     """[num_pages, P] bool: True where a slot holds a resident (pre-step) token."""
     mask = np.zeros((num_pages, P), bool)
     for b, L in enumerate(lengths):
-        for lp in range(int((L + 1 + P - 1) // P)):
+        for lp in range(int((L + P - 1) // P)):
             page = bt[b, lp]
             lo = lp * P
             n_here = int(min(P, max(0, L - lo)))
@@ -162,11 +172,12 @@ def _resident_mask(lengths: np.ndarray, bt: np.ndarray, num_pages: int, P: int) 
 
 def build(name: str, Hq: int, Hkv: int, d: int, P: int, kv_fp8: bool, rope_base: float,
           lengths, seed: int, device="cpu", num_pages: Optional[int] = None,
-          bt_stride: Optional[int] = None) -> Workload:
-    """Draw one workload with the given shapes and cached lengths."""
+          bt_stride: Optional[int] = None, q_len: int = 1) -> Workload:
+    """Draw one workload with the given shapes and cached lengths; q_len new
+    tokens per request (q_len > 1 gives q, k_new, v_new a token axis)."""
     lengths = np.asarray(lengths, np.int64)
     rng = np.random.default_rng(seed + 7)   # page permutation stream
-    bt, num_pages = _assign_pages(lengths, P, num_pages, rng)
+    bt, num_pages = _assign_pages(lengths, P, num_pages, rng, q_len)
     if bt_stride is not None and bt_stride > bt.shape[1]:
         bt = np.concatenate([bt, np.full((bt.shape[0], bt_stride - bt.shape[1]), -1, np.int32)], 1)
     B = lengths.shape[0]
@@ -206,13 +217,15 @@ def build(name: str, Hq: int, Hkv: int, d: int, P: int, kv_fp8: bool, rope_base:
         k_pool, v_pool = pools
         k_scale, v_scale = scales
 
-    q = randn(B, Hq, d).to(torch.bfloat16)
-    k_new = randn(B, Hkv, d).to(torch.bfloat16)
-    v_new = randn(B, Hkv, d).to(torch.bfloat16)
+    tok = () if q_len == 1 else (q_len,)
+    q = randn(B, *tok, Hq, d).to(torch.bfloat16)
+    k_new = randn(B, *tok, Hkv, d).to(torch.bfloat16)
+    v_new = randn(B, *tok, Hkv, d).to(torch.bfloat16)
     return Workload(name=name, Hq=Hq, Hkv=Hkv, d=d, P=P, kv_fp8=kv_fp8, rope_base=rope_base,
                     seq_lens=lengths.astype(np.int32), block_tables=bt, num_pages=num_pages,
                     q=q, k_new=k_new, v_new=v_new, k_pool=k_pool.contiguous(),
-                    v_pool=v_pool.contiguous(), k_scale=k_scale, v_scale=v_scale, seed=seed)
+                    v_pool=v_pool.contiguous(), k_scale=k_scale, v_scale=v_scale, seed=seed,
+                    q_len=q_len)
 
 
 def make(name: str, device="cpu", offset: int = 0) -> Workload:
@@ -221,7 +234,7 @@ def make(name: str, device="cpu", offset: int = 0) -> Workload:
     seed = config_seed(name, offset)
     lengths = draw_lengths(name, np.random.default_rng(seed))
     return build(name, s["Hq"], s["Hkv"], s["d"], s["P"], s["kv_fp8"], s["base"], lengths,
-                 seed, device=device, num_pages=64 if name == "tiny" else None)
+                 seed, device=device, num_pages=64 if name == "tiny" else None, q_len=s.get("q_len", 1))
 
 
 def shape_of(name: str) -> dict:
