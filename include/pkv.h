@@ -128,6 +128,43 @@ pkv_status pkv_decode_attn(pkv_ctx* ctx, const void* q, const void* k_pool, cons
                            const int32_t* seq_lens, int batch, void* out,
                            cudaStream_t stream);
 
+/* Several new tokens per request: the verification pass of speculative
+ * decoding, where a draft proposes tokens and the target model checks all of
+ * them in one forward pass ("Scaling TensorRT-LLM: Kernel Fusion and
+ * Inflight Batching in Production", section "3. Speculative Decoding for
+ * Tail Latency"; "TensorRT-LLM Guide: High-Throughput GPU Inference Engine",
+ * section "2. Pipelined Speculative Decoding").  q_len >= 1 new tokens per
+ * request, the same for every request of the call; new token t of request b
+ * sits at position L_b + t (L_b = seq_lens[b], tokens cached before the
+ * call).  Layouts: q and out [batch][q_len][Hq][d], k_new and v_new
+ * [batch][q_len][Hkv][d], the rest as above.
+ *
+ * Step part 1 for several new tokens: each token is rotated at its position
+ * and its k / v stored in slot (L_b + t) % P of page
+ * block_tables[b][(L_b + t) / P], exactly as pkv_rope_append stores one new
+ * token (bf16 or fp8 pools).  Positions past bt_stride * P are range errors
+ * (device error word, the token is skipped). */
+pkv_status pkv_rope_append_tokens(pkv_ctx* ctx, void* q, const void* k_new, const void* v_new,
+                                  void* k_pool, void* v_pool,
+                                  const float* k_scale, const float* v_scale,
+                                  const int32_t* block_tables, int bt_stride,
+                                  const int32_t* seq_lens, int batch, int q_len,
+                                  cudaStream_t stream);
+
+/* Step part 2 for several new tokens: new token t attends tokens
+ * 0 .. L_b + t (the cache, the new tokens before it and itself; causal among
+ * the new tokens), out[b][t][h][:] = bf16(o).  The G x q_len query rows of a
+ * (request, kv head) share each K/V tile, so the cache is read once per
+ * call whatever q_len is.  Needs G * q_len <= 16 and bf16 pools
+ * (PKV_ERR_UNSUPPORTED otherwise); requests whose L_b + q_len exceeds
+ * bt_stride * P get zeros and set the device error word.  The split merge
+ * runs in a second kernel, as for pkv_decode_attn. */
+pkv_status pkv_decode_attn_tokens(pkv_ctx* ctx, const void* q, const void* k_pool, const void* v_pool,
+                                  const float* k_scale, const float* v_scale,
+                                  const int32_t* block_tables, int bt_stride,
+                                  const int32_t* seq_lens, int batch, int q_len, void* out,
+                                  cudaStream_t stream);
+
 /* Frees the workspace.  NULL is accepted.  Synchronises the device. */
 pkv_status pkv_destroy(pkv_ctx* ctx);
 

@@ -43,169 +43,13 @@
 // protocol) run to the end without touching data.
 #include <math.h>
 
-#include "pkv_internal.h"
-#include "pkv_device.cuh"
+#include "attn_common.cuh"
 
 namespace pkv {
 namespace {
 
 using namespace dev;
-
-constexpr uint64_t kWaitLimitNs = 500ull * 1000ull * 1000ull;  // 0.5 s per wait
-constexpr unsigned kFull = 0xFFFFFFFFu;
-
-template <int D, bool FP8>
-struct Geo {
-    static constexpr int ELEM = FP8 ? 1 : 2;
-    static constexpr int ROWB = D * ELEM;                  // bytes per token row
-    static constexpr int BOXB = ROWB > 128 ? 128 : ROWB;   // bytes per TMA box row
-    static constexpr int NBOX = ROWB / BOXB;               // boxes per tile per tensor
-    static constexpr int CPB = BOXB / 16;                  // 16-byte chunks per box row
-    static constexpr int BOX_BYTES = kTile * BOXB;
-    static constexpr int TILEB = kTile * ROWB;             // one K (or V) tile
-    static constexpr int STAGEB = 2 * TILEB;               // K + V
-};
-
-// Byte offset inside a tile of 16-byte chunk `ch` (counted along the token
-// row) of tile row `row`, as the TMA swizzle placed it.
-template <int D, bool FP8>
-__device__ __forceinline__ uint32_t tile_off(int row, int ch)
-{
-    using Gm = Geo<D, FP8>;
-    const int box = ch / Gm::CPB, cib = ch % Gm::CPB;
-    const int x = (Gm::BOXB == 128) ? (row & 7) : ((row >> 1) & 3);
-    return (uint32_t)(box * Gm::BOX_BYTES + row * Gm::BOXB + ((cib ^ x) << 4));
-}
-
-struct StageInfo {
-    float ks, vs;   // fp8 scales of the tile's page and kv head
-    int valid;      // 0: page id was out of range, tile skipped
-    int pad;
-};
-
-// Units of the split.  Warp range v is [r(v), r(v+1)), r(v) = v T / W.  With
-// K = 0 a range is one unit.  With K > 0 unit v (K+1) is the head
-// [r(v), s(v)) and units v (K+1) + 1 + j, j < K, cut the tail [s(v), r(v+1))
-// of tl = min(range / kTailDen, kTailMaxTiles) tiles at s(v) + j tl / K.
-// Units are numbered in the order of the tiles they hold, none is empty, and
-// together they cover [0, T) once.  W < 2^16, so r(v) needs one 32-bit
-// division (T = qT W + rT), and tl is small.
-struct Split {
-    long long T, qT;
-    int W, K, rT;
-
-    __device__ __forceinline__ long long r(int v) const
-    {
-        return (long long)v * qT + (long long)(((unsigned)v * (unsigned)rT) / (unsigned)W);
-    }
-    __device__ __forceinline__ static int tail_of(long long range)
-    {
-        return (int)min(range / kTailDen, (long long)kTailMaxTiles);
-    }
-    // first tile of unit U (U = W (K+1) gives T)
-    __device__ __forceinline__ long long ustart(int U) const
-    {
-        if (K == 0) return r(U);
-        const int v = U / (K + 1), j = U - v * (K + 1);
-        const long long rv = r(v);
-        if (j == 0) return rv;
-        const long long range = r(v + 1) - rv;
-        const int tl = tail_of(range);
-        return rv + range - tl + (j - 1) * tl / K;
-    }
-    // index of the unit holding tile x, 0 <= x < T
-    __device__ __forceinline__ int unit_of(long long x) const
-    {
-        const int v = (int)(((x + 1) * W - 1) / T);
-        if (K == 0) return v;
-        const long long rv = r(v), range = r(v + 1) - rv;
-        const int tl = tail_of(range);
-        const long long sv = rv + range - tl;
-        if (x < sv) return v * (K + 1);
-        const int y = (int)(x - sv);
-        return v * (K + 1) + 1 + ((y + 1) * K - 1) / tl;
-    }
-};
-
-// K for T tiles over W warps, at most `max_chunks`: chunks of at least
-// kTailChunkTiles tiles, none when the shortest range is under kTailMinTiles
-// tiles (its tail then holds at least 8 tiles, and the head at least 24).
-__device__ __forceinline__ Split make_split(long long T, int W, int max_chunks)
-{
-    Split sp;
-    sp.T = T;
-    sp.W = W;
-    sp.qT = T / W;
-    sp.rT = (int)(T - sp.qT * W);
-    sp.K = 0;
-    if (max_chunks > 0 && sp.qT >= kTailMinTiles)
-        sp.K = min(max_chunks, max(1, Split::tail_of(sp.qT) / kTailChunkTiles));
-    return sp;
-}
-
-// Largest b with prefix[b] * Hkv <= x, for 0 <= x < prefix[B] * Hkv.
-__device__ __forceinline__ int seek_request(const int* prefix, int B, int Hkv, long long x)
-{
-    int lo = 0, hi = B;
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if ((long long)prefix[mid] * Hkv <= x) lo = mid;
-        else hi = mid;
-    }
-    return lo;
-}
-
-// (request, kv head, tile within the pair) of flattened tile x
-__device__ __forceinline__ void locate(const int* prefix, int B, int Hkv, long long x, int& b, int& kvh,
-                                       int& tt, int& cnt)
-{
-    b = seek_request(prefix, B, Hkv, x);
-    cnt = prefix[b + 1] - prefix[b];
-    const long long r = x - (long long)prefix[b] * Hkv;
-    if (r <= 0x7fffffffll) {   // the usual case: 32-bit division
-        kvh = (int)r / cnt;
-        tt = (int)r - kvh * cnt;
-    } else {
-        kvh = (int)(r / cnt);
-        tt = (int)(r % cnt);
-    }
-}
-
-// Page ids (as TMA row coordinates) and scales of 32 consecutive tiles, one
-// per lane.
-struct Lookahead {
-    int valid;   // 0: past the range, 1: ok, 2: page id out of range
-    int row;
-    float ks, vs;
-};
-
-template <bool FP8>
-__device__ __forceinline__ Lookahead lookahead_fill(const AttnParams& p, const int* prefix, long long x0,
-                                                    long long t_end, int lane)
-{
-    Lookahead la{0, 0, 1.f, 1.f};
-    const long long y = x0 + lane;
-    if (y < t_end) {
-        const int b = seek_request(prefix, p.batch, p.Hkv, y);
-        const int ntb = prefix[b + 1] - prefix[b];
-        const long long r = y - (long long)prefix[b] * p.Hkv;
-        const int kvh = (int)(r / ntb), tt = (int)(r % ntb);
-        const int tok0 = tt * kTile;
-        const int lp = tok0 / p.P;
-        const int page = __ldg(&p.block_tables[(size_t)b * p.bt_stride + lp]);
-        if ((unsigned)page < (unsigned)p.num_pages) {
-            la.valid = 1;
-            la.row = (page * p.Hkv + kvh) * p.P + (tok0 - lp * p.P);
-            if (FP8) {
-                la.ks = __ldg(&p.k_scale[(size_t)page * p.Hkv + kvh]);
-                la.vs = __ldg(&p.v_scale[(size_t)page * p.Hkv + kvh]);
-            }
-        } else {
-            la.valid = 2;
-        }
-    }
-    return la;
-}
+using namespace attn;
 
 // Query fragments of (request b, kv head kvh) for the mma A operand: row g =
 // query head kvh*G + g (zero for g >= G), k-step ks covers d in [16ks, 16ks+16).
@@ -758,294 +602,6 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
     }
 }
 
-// Split combine: one CTA per (request, kv head) pair.  A pair whose tiles lay
-// in more than one unit left one partial per unit (unnormalised o, running max
-// m in log2 units, sum l); here they are merged by log-sum-exp,
-//   m* = max m_v,  l* = sum l_v 2^(m_v - m*),  o = sum o_v 2^(m_v - m*) / l*,
-// and written as bf16.  Pairs finished inside one unit, and requests with an
-// impossible length, are skipped.  Runs after the attention kernel on the
-// same stream, which orders every partial before it is read; it also resets
-// the chunk counter of the attention's dynamic tail for the next launch.
-// Contributors are staged in shared memory kCombineBlock at a time: one pass
-// for m* and l* (one warp per head), one for the weighted sum (in reverse
-// block order, so a pair with at most kCombineBlock contributors is staged
-// once) in which warp j sums contributors j, j + 8, ... over all G x D
-// values with 16-byte loads, and the eight warp sums are added in a fixed
-// order.
-constexpr int kCombineThreads = 256;
-constexpr int kCombineWarps = kCombineThreads / 32;
-constexpr int kCombineBlock = 256;
-
-// floats of the staging area (slots, m, l of kb contributors), rounded up to 16 bytes
-inline __host__ __device__ size_t combine_stage_floats(int kb, int G)
-{
-    return (((size_t)kb * (2 * G + 1)) + 3) & ~(size_t)3;
-}
-
-// Dynamic shared memory of the combine for at most `contributors` per pair.
-inline size_t combine_smem_bytes(int contributors, int G, int D)
-{
-    const int kb = contributors < kCombineBlock ? contributors : kCombineBlock;
-    return sizeof(float) * (combine_stage_floats(kb, G) + (size_t)kCombineWarps * G * D);
-}
-
-template <int D>
-__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const AttnParams p)
-{
-    constexpr unsigned kFullMask = 0xFFFFFFFFu;
-    constexpr int F4 = kMaxGroup * D / 4 / 32;   // 16-byte chunks per lane per contributor, at most
-    extern __shared__ float4 s_dyn4[];
-    float* const s_dyn = reinterpret_cast<float*>(s_dyn4);
-    __shared__ float s_m[kMaxGroup], s_l[kMaxGroup];
-
-    if (blockIdx.x == 0 && threadIdx.x == 0) *p.claim = 0;   // the attention launch has ended
-    const int pair = blockIdx.x;
-    const int b = pair / p.Hkv, kvh = pair - b * p.Hkv;
-    const int W = __ldg(&p.meta[0]);
-    const long long T = (long long)(unsigned)__ldg(&p.meta[1]) | ((long long)__ldg(&p.meta[2]) << 32);
-    if (T == 0 || b >= p.batch) return;
-    const int* prefix = p.meta + 4;
-    const int nt = __ldg(&prefix[b + 1]) - __ldg(&prefix[b]);
-    if (nt == 0) return;
-    Split sp = make_split(T, W, 0);
-    sp.K = __ldg(&p.meta[3]);   // as the attention launch chose it
-    const long long ts = (long long)__ldg(&prefix[b]) * p.Hkv + (long long)kvh * nt;
-    const int U0 = sp.unit_of(ts), U1 = sp.unit_of(ts + nt - 1);
-    if (U0 == U1) return;
-    const int k = U1 - U0 + 1, G = p.G, GD4 = G * D / 4;
-    const int side0 = sp.ustart(U0) < ts ? 1 : 0;   // slot side of the first unit
-    const int kb = min(k, kCombineBlock);              // the dynamic shared memory holds kb contributors
-    const int nblk = (k + kCombineBlock - 1) / kCombineBlock;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    float* const s_mv = s_dyn;                                                  // [kb * G] m, later the weight
-    float* const s_lv = s_dyn + (size_t)kb * G;                                 // [kb * G] l
-    int* const s_slot = reinterpret_cast<int*>(s_dyn + 2 * (size_t)kb * G);    // [kb]
-    float4* const s_red = s_dyn4 + combine_stage_floats(kb, G) / 4;            // [warps][G * D / 4]
-
-    // slots, m and l of the contributors of block blk; returns how many
-    auto stage = [&](int blk) -> int {
-        const int i0 = blk * kCombineBlock, n = min(kCombineBlock, k - i0);
-        for (int i = tid; i < n; i += kCombineThreads)
-            s_slot[i] = 2 * (U0 + i0 + i) + (i0 + i == 0 ? side0 : 0);
-        __syncthreads();
-        for (int e = tid; e < n * G; e += kCombineThreads) {
-            const int i = e / G, gg = e - i * G;
-            const float2 ml = __ldg(reinterpret_cast<const float2*>(p.part_ml + ((size_t)s_slot[i] * G + gg) * 2));
-            s_mv[e] = ml.x;
-            s_lv[e] = ml.y;
-        }
-        __syncthreads();
-        return n;
-    };
-
-    // pass 1: m* and l* per head (warp g), merged over blocks
-    float Mg = -INFINITY, Lg = 0.f;
-    int n_last = 0;
-    for (int blk = 0; blk < nblk; ++blk) {
-        if (blk > 0) __syncthreads();
-        const int n = stage(blk);
-        n_last = n;
-        if (warp < G) {
-            float m = -INFINITY;
-            for (int i = lane; i < n; i += 32) m = fmaxf(m, s_mv[i * G + warp]);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFullMask, m, o));
-            const float m_new = fmaxf(Mg, m);
-            const float m_ref = (m_new == -INFINITY) ? 0.f : m_new;
-            float l = 0.f;
-            for (int i = lane; i < n; i += 32) l += s_lv[i * G + warp] * ex2(s_mv[i * G + warp] - m_ref);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(kFullMask, l, o);
-            Lg = Lg * ex2(Mg - m_ref) + l;
-            Mg = m_new;
-        }
-    }
-    if (warp < G && lane == 0) {
-        s_m[warp] = (Mg == -INFINITY) ? 0.f : Mg;
-        s_l[warp] = Lg;
-    }
-    __syncthreads();
-
-    // pass 2: warp j sums contributors j, j + 8, ... (all G x D values)
-    float4 acc[F4];
-#pragma unroll
-    for (int t = 0; t < F4; ++t) acc[t] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int blk = nblk - 1; blk >= 0; --blk) {
-        int n = n_last;
-        if (blk != nblk - 1) {
-            __syncthreads();
-            n = stage(blk);
-        }
-        for (int e = tid; e < n * G; e += kCombineThreads) {
-            const int gg = e % G;
-            s_mv[e] = ex2(s_mv[e] - s_m[gg]) / s_l[gg];   // now the weight
-        }
-        __syncthreads();
-#pragma unroll 2
-        for (int i = warp; i < n; i += kCombineWarps) {
-            const float4* src = reinterpret_cast<const float4*>(p.part_o + (size_t)s_slot[i] * G * D);
-#pragma unroll
-            for (int t = 0; t < F4; ++t) {
-                const int f = lane + 32 * t;
-                if (f < GD4) {
-                    const float wgt = s_mv[i * G + (4 * f) / D];
-                    const float4 v = __ldg(src + f);
-                    acc[t].x += wgt * v.x;
-                    acc[t].y += wgt * v.y;
-                    acc[t].z += wgt * v.z;
-                    acc[t].w += wgt * v.w;
-                }
-            }
-        }
-    }
-#pragma unroll
-    for (int t = 0; t < F4; ++t) {
-        const int f = lane + 32 * t;
-        if (f < GD4) s_red[warp * GD4 + f] = acc[t];
-    }
-    __syncthreads();
-    uint2* const dst = reinterpret_cast<uint2*>(p.out + ((size_t)b * p.Hq + (size_t)kvh * G) * D);
-    for (int f = tid; f < GD4; f += kCombineThreads) {
-        float4 sum = s_red[f];
-#pragma unroll
-        for (int j = 1; j < kCombineWarps; ++j) {
-            const float4 v = s_red[j * GD4 + f];
-            sum.x += v.x;
-            sum.y += v.y;
-            sum.z += v.z;
-            sum.w += v.w;
-        }
-        dst[f] = make_uint2(pack_bf16(sum.x, sum.y), pack_bf16(sum.z, sum.w));
-    }
-}
-
-// The same merge with one warp per pair, for batches with many pairs: all
-// pairs then fit in about one wave and no shared memory or CTA barrier is
-// needed.  Lanes take contributors 32 at a time for m* and l* (online, then a
-// butterfly over the lanes) and for the weights; the weighted sum walks the
-// contributors with every lane on its own 16-byte pieces of the G x D
-// values, a piece of D = 128 belonging to head t for the t-th piece of the
-// lane and a piece of D = 64 to head 2t or 2t + 1 by lane half.
-constexpr int kCombineWarpThreads = 256;
-
-template <int D>
-__global__ void __launch_bounds__(kCombineWarpThreads, 2) combine_warp_kernel(const AttnParams p)
-{
-    constexpr unsigned kFullMask = 0xFFFFFFFFu;
-    constexpr int F4 = kMaxGroup * D / 4 / 32;   // 16-byte pieces per lane, at most
-    static_assert(D == 128 || D == 64, "head_dim");
-
-    if (blockIdx.x == 0 && threadIdx.x == 0) *p.claim = 0;   // the attention launch has ended
-    const int lane = threadIdx.x & 31;
-    const int pair = blockIdx.x * (kCombineWarpThreads / 32) + (threadIdx.x >> 5);
-    if (pair >= p.batch * p.Hkv) return;
-    const int b = pair / p.Hkv, kvh = pair - b * p.Hkv;
-    const int W = __ldg(&p.meta[0]);
-    const long long T = (long long)(unsigned)__ldg(&p.meta[1]) | ((long long)__ldg(&p.meta[2]) << 32);
-    const int* prefix = p.meta + 4;
-    const int pb = __ldg(&prefix[b]);
-    const int nt = __ldg(&prefix[b + 1]) - pb;
-    if (T == 0 || nt == 0) return;
-    Split sp = make_split(T, W, 0);
-    sp.K = __ldg(&p.meta[3]);   // as the attention launch chose it
-    const long long ts = (long long)pb * p.Hkv + (long long)kvh * nt;
-    const int U0 = sp.unit_of(ts), U1 = sp.unit_of(ts + nt - 1);
-    if (U0 == U1) return;
-    const int k = U1 - U0 + 1, G = p.G, GD4 = G * D / 4;
-    const int side0 = sp.ustart(U0) < ts ? 1 : 0;
-
-    // pass 1: m* and l* per head; lane j keeps the m of its first contributor
-    // (j) so that the weights of the first 32 need no second load
-    float M[kMaxGroup], L[kMaxGroup], m_own[kMaxGroup];
-#pragma unroll
-    for (int g = 0; g < kMaxGroup; ++g) {
-        M[g] = -INFINITY;
-        L[g] = 0.f;
-        m_own[g] = -INFINITY;
-    }
-    for (int i = lane; i < k; i += 32) {
-        const int slot = 2 * (U0 + i) + (i == 0 ? side0 : 0);
-#pragma unroll
-        for (int g = 0; g < kMaxGroup; ++g) {
-            if (g < G) {
-                const float2 ml = __ldg(reinterpret_cast<const float2*>(p.part_ml + ((size_t)slot * G + g) * 2));
-                if (i == lane) m_own[g] = ml.x;
-                const float m_new = fmaxf(M[g], ml.x);
-                const float ref = (m_new == -INFINITY) ? 0.f : m_new;
-                L[g] = L[g] * ex2(M[g] - ref) + ml.y * ex2(ml.x - ref);
-                M[g] = m_new;
-            }
-        }
-    }
-#pragma unroll
-    for (int g = 0; g < kMaxGroup; ++g) {
-        if (g < G) {
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const float m2 = __shfl_xor_sync(kFullMask, M[g], o), l2 = __shfl_xor_sync(kFullMask, L[g], o);
-                const float m_new = fmaxf(M[g], m2);
-                const float ref = (m_new == -INFINITY) ? 0.f : m_new;
-                L[g] = L[g] * ex2(M[g] - ref) + l2 * ex2(m2 - ref);
-                M[g] = m_new;
-            }
-            if (M[g] == -INFINITY) M[g] = 0.f;
-        }
-    }
-
-    // pass 2: weighted sum, contributors in batches of 32 (lane j holds the
-    // slot and the weights of contributor i0 + j)
-    float4 acc[F4];
-#pragma unroll
-    for (int t = 0; t < F4; ++t) acc[t] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int i0 = 0; i0 < k; i0 += 32) {
-        const int i = i0 + lane;
-        int slot_l = 0;
-        float wl[kMaxGroup];
-#pragma unroll
-        for (int g = 0; g < kMaxGroup; ++g) wl[g] = 0.f;
-        if (i < k) {
-            slot_l = 2 * (U0 + i) + (i == 0 ? side0 : 0);
-#pragma unroll
-            for (int g = 0; g < kMaxGroup; ++g) {
-                if (g < G) {
-                    const float m = (i0 == 0) ? m_own[g] : __ldg(p.part_ml + ((size_t)slot_l * G + g) * 2);
-                    wl[g] = ex2(m - M[g]) / L[g];
-                }
-            }
-        }
-        const int n = min(32, k - i0);
-        for (int j = 0; j < n; ++j) {
-            const int slot = __shfl_sync(kFullMask, slot_l, j);
-            const float4* src = reinterpret_cast<const float4*>(p.part_o + (size_t)slot * G * D);
-#pragma unroll
-            for (int t = 0; t < F4; ++t) {
-                float w;
-                if constexpr (D == 128) {
-                    w = __shfl_sync(kFullMask, wl[t], j);
-                } else {
-                    const float wa = __shfl_sync(kFullMask, wl[2 * t], j);
-                    const float wb = __shfl_sync(kFullMask, wl[2 * t + 1], j);
-                    w = lane < 16 ? wa : wb;
-                }
-                const int f = lane + 32 * t;
-                if (f < GD4) {
-                    const float4 v = __ldg(src + f);
-                    acc[t].x += w * v.x;
-                    acc[t].y += w * v.y;
-                    acc[t].z += w * v.z;
-                    acc[t].w += w * v.w;
-                }
-            }
-        }
-    }
-    uint2* const dst = reinterpret_cast<uint2*>(p.out + ((size_t)b * p.Hq + (size_t)kvh * G) * D);
-#pragma unroll
-    for (int t = 0; t < F4; ++t) {
-        const int f = lane + 32 * t;
-        if (f < GD4) dst[f] = make_uint2(pack_bf16(acc[t].x, acc[t].y), pack_bf16(acc[t].z, acc[t].w));
-    }
-}
-
 template <int D, bool FP8>
 size_t smem_bytes_for(int stages, int max_batch)
 {
@@ -1070,8 +626,7 @@ cudaError_t prepare_t(int num_sms, int max_batch, AttnLaunch* out)
     e = cudaFuncSetAttribute(decode_attn_kernel<D, FP8, kAttnWarps>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)bytes);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(combine_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)combine_smem_bytes(kCombineBlock, kMaxGroup, D));
+    e = combine_prepare(D);
     if (e != cudaSuccess) return e;
     out->ctas = num_sms;
     out->stages = stages;
@@ -1094,27 +649,16 @@ cudaError_t launch_decode_attn(const AttnParams& p, const CUtensorMap& tmk, cons
     const dim3 grid(L.ctas), block(kAttnWarps * 32);
     AttnParams q = p;
     q.stages = L.stages;
-    // the combine: a warp per pair when there are at least two pairs per
-    // attention warp slot of a wave (many pairs, each with few
-    // contributors), else a CTA per pair
-    const int pairs = p.batch * p.Hkv;
-    const bool warp_mode = pairs >= 2 * L.ctas;
-    const dim3 cgrid((unsigned)pairs), cblock(kCombineThreads);
-    const size_t csmem = combine_smem_bytes((int)max_units(L.ctas * kAttnWarps, p.tail_chunks), p.G, head_dim);
-    const int wpc = kCombineWarpThreads / 32;
-    const dim3 wgrid((unsigned)((pairs + wpc - 1) / wpc)), wblock(kCombineWarpThreads);
     if (head_dim == 128) {
         if (fp8) decode_attn_kernel<128, true, kAttnWarps><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
         else decode_attn_kernel<128, false, kAttnWarps><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
-        if (warp_mode) combine_warp_kernel<128><<<wgrid, wblock, 0, stream>>>(q);
-        else combine_kernel<128><<<cgrid, cblock, csmem, stream>>>(q);
     } else {
         if (fp8) decode_attn_kernel<64, true, kAttnWarps><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
         else decode_attn_kernel<64, false, kAttnWarps><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
-        if (warp_mode) combine_warp_kernel<64><<<wgrid, wblock, 0, stream>>>(q);
-        else combine_kernel<64><<<cgrid, cblock, csmem, stream>>>(q);
     }
-    return cudaGetLastError();
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return launch_combine(q, head_dim, (int)max_units(L.ctas * kAttnWarps, p.tail_chunks), L.ctas, stream);
 }
 
 }  // namespace pkv

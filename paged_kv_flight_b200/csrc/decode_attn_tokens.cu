@@ -1,0 +1,463 @@
+// decode_attn_tokens.cu -- attention of several new tokens per request over
+// the paged KV cache: the verification pass of speculative decoding, where a
+// draft proposes tokens and the target model checks all of them in one
+// forward pass ("Scaling TensorRT-LLM: Kernel Fusion and Inflight Batching in
+// Production", section "3. Speculative Decoding for Tail Latency";
+// "TensorRT-LLM Guide: High-Throughput GPU Inference Engine", section
+// "2. Pipelined Speculative Decoding").
+//
+// What it computes: new token t (0 <= t < q_len) of request b sits at
+// position L_b + t and attends tokens 0 .. L_b + t (the cache, the new tokens
+// before it and itself), o = softmax(q K^T / sqrt(d)) V, K/V of kv head h / G.
+// All q_len x G query rows of a (request, kv head) pair share each K/V tile:
+// they are the R = G q_len <= 16 rows of one m16n8k16 mma (row t G + h), so
+// the cache is read once per pair whatever q_len is.  Each row has its own
+// causal limit (tokens below L_b + t + 1).
+//
+// The rest is the single-token kernel's design (decode_attn.cu): tiles of 16
+// tokens ((request, kv head, tile) flattened and cut into equal contiguous
+// warp ranges, a static split), a per-warp ring of TMA tile loads on
+// mbarriers fed by a 32-tile page-id lookahead, online softmax in log2 units,
+// partial (m, l, o) rows for pairs cut between ranges, merged afterwards by
+// the combine kernel (combine.cu).  bf16 pools only.
+#include "attn_common.cuh"
+
+namespace pkv {
+namespace {
+
+using namespace dev;
+using namespace attn;
+
+// Query rows of (request b, kv head kvh) as mma A fragments: rows g (a0, a2)
+// and g + 8 (a1, a3) of the 16; row r = t G + h is head kvh G + h of new
+// token t, rows r >= R are zero.
+template <int D>
+__device__ __forceinline__ void load_q_rows(const AttnParams& p, int b, int kvh, int g, int c4, int R,
+                                            uint32_t (&qa)[D / 16][4])
+{
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        const int r = g + 8 * half;
+        const bool ok = r < R;
+        const int t = ok ? r / p.G : 0, h = ok ? r - t * p.G : 0;
+        const __nv_bfloat16* qrow = p.q + (((size_t)b * p.q_len + t) * p.Hq + (size_t)kvh * p.G + h) * D;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+            qa[ks][half] = ok ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * c4) : 0u;
+            qa[ks][2 + half] = ok ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8 + 2 * c4) : 0u;
+        }
+    }
+}
+
+template <int D, int WARPS>
+__global__ void __launch_bounds__(WARPS * 32, 1)
+decode_attn_tokens_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                          const AttnParams p)
+{
+    using Gm = Geo<D, false>;
+    constexpr int KSTEPS = D / 16;      // mma k-steps along d for QK^T
+    constexpr int NTD = D / 8;          // mma n-tiles along d for P V
+    constexpr int NT = WARPS * 32;
+
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ int s_warp_tot[WARPS];
+    __shared__ int s_bad;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int B = p.batch, Hkv = p.Hkv, S = p.stages, QL = p.q_len;
+    const int G = p.G, R = G * QL;
+
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t stage_area = (raw + 1023u) & ~1023u;
+    uint8_t* const area_ptr = smem_raw + (stage_area - raw);
+    StageInfo* const info_all = reinterpret_cast<StageInfo*>(area_ptr + WARPS * S * Gm::STAGEB);
+    uint8_t* const bar_ptr = reinterpret_cast<uint8_t*>(info_all + WARPS * S);
+    int* const prefix = reinterpret_cast<int*>(bar_ptr + WARPS * S * 8);
+
+    if (tid == 0) {
+        s_bad = 0;
+        prefetch_tensormap(&tmk);
+        prefetch_tensormap(&tmv);
+    }
+    __syncthreads();
+
+    // ---- 1. tiles per request (they cover the last new token's L_b + q_len
+    //         tokens) and their exclusive prefix ---------------------------------
+    const long long cap = (long long)p.bt_stride * p.P;
+    const int per = (B + NT - 1) / NT;
+    const int lo = min(B, tid * per), hi = min(B, lo + per);
+    int local = 0;
+    for (int b = lo; b < hi; ++b) {
+        const int L = p.seq_lens[b];
+        const bool ok = L >= 0 && (long long)L + QL <= cap;
+        const int nt = ok ? (L + QL + kTile - 1) / kTile : 0;
+        if (!ok) s_bad = 1;
+        prefix[b] = nt;
+        local += nt;
+    }
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) s_warp_tot[warp] = incl;
+    __syncthreads();
+    int run = incl - local;
+    for (int w2 = 0; w2 < warp; ++w2) run += s_warp_tot[w2];
+    for (int b = lo; b < hi; ++b) {
+        const int c = prefix[b];
+        prefix[b] = run;
+        run += c;
+    }
+    if (tid == NT - 1) prefix[B] = run;
+    __syncthreads();
+
+    if (s_bad && blockIdx.x == 0) {
+        // requests with an impossible length produce zeros and an error bit
+        if (tid == 0) atomicOr(p.err, kErrLength);
+        for (int b = warp; b < B; b += WARPS) {
+            const int L = p.seq_lens[b];
+            if (L >= 0 && (long long)L + QL <= cap) continue;
+            uint32_t* o32 = reinterpret_cast<uint32_t*>(p.out + (size_t)b * QL * p.Hq * D);
+            for (int i = lane; i < QL * p.Hq * D / 2; i += 32) o32[i] = 0u;
+        }
+    }
+
+    // ---- 2. static split: this warp's range --------------------------------------
+    const long long T = (long long)prefix[B] * Hkv;
+    long long Wl = (long long)gridDim.x * WARPS;
+    if (p.workers > 0) Wl = min(Wl, (long long)p.workers);
+    else Wl = min(Wl, (T + kMinTilesPerWorker - 1) / kMinTilesPerWorker);
+    Wl = max(1LL, min(Wl, max(T, 1LL)));
+    const int W = (int)Wl;
+    const Split sp = make_split(max(T, 1LL), W, 0);
+    if (blockIdx.x == 0) {
+        // the combine kernel that follows needs the same split geometry
+        if (tid == 0) {
+            p.meta[0] = W;
+            p.meta[1] = (int)(T & 0xFFFFFFFFll);
+            p.meta[2] = (int)(T >> 32);
+            p.meta[3] = 0;
+        }
+        for (int b = tid; b <= B; b += NT) p.meta[4 + b] = prefix[b];
+    }
+    if (T == 0) return;
+    const int w = warp * gridDim.x + blockIdx.x;   // spread workers over SMs first
+    if (w >= W) return;
+    const long long u0 = sp.ustart(w), u1 = sp.ustart(w + 1);
+    const int ntiles = (int)(u1 - u0);
+
+    const uint32_t my_stage0 = stage_area + (uint32_t)(warp * S * Gm::STAGEB);
+    StageInfo* const my_info = info_all + warp * S;
+    const uint32_t my_bar0 = smem_u32(bar_ptr) + (uint32_t)(warp * S * 8);
+    if (lane == 0) {
+        for (int s = 0; s < S; ++s) mbar_init(my_bar0 + 8u * s, 1u);
+        fence_mbar_init();
+    }
+    __syncwarp();
+
+    // ---- 3. producer: double-buffered 32-tile lookahead, TMA issue -----------------
+    int la_i = 0;
+    long long la_fill = u0 + 64;
+    Lookahead la_cur = lookahead_fill<false>(p, prefix, u0, u1, lane);
+    Lookahead la_nxt = lookahead_fill<false>(p, prefix, u0 + 32, u1, lane);
+
+    auto issue = [&](int s) {
+        if (la_i == 32) {
+            la_i = 0;
+            la_cur = la_nxt;
+            la_nxt = lookahead_fill<false>(p, prefix, la_fill, u1, lane);
+            la_fill += 32;
+        }
+        const int src = la_i++;
+        const int v = __shfl_sync(kFull, la_cur.valid, src);
+        const int row = __shfl_sync(kFull, la_cur.row, src);
+        if (lane == 0) {
+            const uint32_t bar = my_bar0 + 8u * s;
+            StageInfo si;
+            si.ks = 1.f;
+            si.vs = 1.f;
+            si.valid = (v == 1);
+            si.pad = 0;
+            my_info[s] = si;
+            if (v == 1) {
+                mbar_arrive_expect_tx(bar, (uint32_t)Gm::STAGEB);
+                const uint32_t kdst = my_stage0 + (uint32_t)(s * Gm::STAGEB);
+                const uint32_t vdst = kdst + Gm::TILEB;
+#pragma unroll
+                for (int j = 0; j < Gm::NBOX; ++j) {
+                    tma_load_2d(kdst + j * Gm::BOX_BYTES, &tmk, j * (Gm::BOXB / Gm::ELEM), row, bar);
+                    tma_load_2d(vdst + j * Gm::BOX_BYTES, &tmv, j * (Gm::BOXB / Gm::ELEM), row, bar);
+                }
+            } else {
+                atomicOr(p.err, kErrPage);
+                mbar_arrive(bar);
+            }
+        }
+    };
+
+    const int pre = min(S, ntiles);
+    for (int k = 0; k < pre; ++k) issue(k);
+    int issued = pre;
+
+    // ---- 4. consumer ----------------------------------------------------------------
+    const int g = lane >> 2;     // mma rows g and g + 8
+    const int c4 = lane & 3;
+    const int mi = lane >> 3, ri = lane & 7;        // ldmatrix: matrix index, row
+    const int tokK = ((mi >> 1) << 3) + ri;         // token row addressed for K
+    const int tokV = ((mi & 1) << 3) + ri;          // token row addressed for V (trans)
+    // new token of rows g and g + 8 (rows >= R see no token)
+    const int trow0 = g < R ? g / G : -1;
+    const int trow1 = g + 8 < R ? (g + 8) / G : -1;
+
+    float o[NTD][4];
+    uint32_t qa[KSTEPS][4];
+    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+    int lim[2] = {0, 0};          // tokens visible to rows g and g + 8
+    int n_max = 0;                // tokens of the pair's last new token
+    bool dead = false;
+    int k_dead = 0;
+    int s = 0;
+    uint32_t parity = 0;
+
+    int cb, ckvh, ctt, cnt;
+    locate(prefix, B, Hkv, u0, cb, ckvh, ctt, cnt);
+
+    for (int k = 0; k < ntiles; ++k) {
+        if (!dead) {
+            const bool ok = __all_sync(kFull, mbar_wait_bounded(my_bar0 + 8u * s, parity, kWaitLimitNs));
+            if (!ok) {
+                dead = true;
+                k_dead = k;
+                if (lane == 0) atomicOr(p.err, kErrTimeout);
+            }
+        }
+        if (dead) {
+            if (++s == S) {
+                s = 0;
+                parity ^= 1u;
+            }
+            continue;
+        }
+        if (ctt == 0 || k == 0) {
+            // start of a (request, kv head) pair or of this range
+            load_q_rows<D>(p, cb, ckvh, g, c4, R, qa);
+            const int n0 = p.seq_lens[cb] + 1;   // tokens visible to new token 0
+            lim[0] = trow0 >= 0 ? n0 + trow0 : 0;
+            lim[1] = trow1 >= 0 ? n0 + trow1 : 0;
+            n_max = n0 + QL - 1;
+#pragma unroll
+            for (int nt = 0; nt < NTD; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+            m_run[0] = m_run[1] = -INFINITY;
+            l_run[0] = l_run[1] = 0.f;
+        }
+        const bool pair_end = ctt == cnt - 1 || k == ntiles - 1;
+
+        const StageInfo si = my_info[s];
+        bool zeroed = false;
+        if (si.valid) {
+            const uint32_t kb = my_stage0 + (uint32_t)(s * Gm::STAGEB);
+            const uint32_t vb = kb + Gm::TILEB;
+            const int tok0 = ctt * kTile;
+            const int rows_valid = min(kTile, n_max - tok0);
+            if (rows_valid < kTile) {
+                // slots past the last new token may hold anything (NaN): zero them in V
+                constexpr int CPR = Gm::ROWB / 16;
+                const int nch = (kTile - rows_valid) * CPR;
+                for (int e = lane; e < nch; e += 32) {
+                    const int r = rows_valid + e / CPR, ch = e % CPR;
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(vb + tile_off<D, false>(r, ch)),
+                                 "r"(0u)
+                                 : "memory");
+                }
+                zeroed = true;
+                __syncwarp();
+            }
+
+            // S = Q K^T: two n-tiles of 8 tokens, rows g (e 0, 1) and g + 8 (e 2, 3), two chains
+            float sa[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            float sb[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+            for (int ks = 0; ks < KSTEPS; ks += 2) {
+                uint32_t r0, r1, r2, r3, r4, r5, r6, r7;
+                ldsm_x4(kb + tile_off<D, false>(tokK, 2 * ks + (mi & 1)), r0, r1, r2, r3);
+                ldsm_x4(kb + tile_off<D, false>(tokK, 2 * ks + 2 + (mi & 1)), r4, r5, r6, r7);
+                mma_bf16_16(sa[0], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], r0, r1);
+                mma_bf16_16(sa[1], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], r2, r3);
+                mma_bf16_16(sb[0], qa[ks + 1][0], qa[ks + 1][1], qa[ks + 1][2], qa[ks + 1][3], r4, r5);
+                mma_bf16_16(sb[1], qa[ks + 1][0], qa[ks + 1][1], qa[ks + 1][2], qa[ks + 1][3], r6, r7);
+            }
+
+            // online softmax per row in log2 units; tokens at or past a row's
+            // limit are -inf (never 0 * NaN)
+            float sc[2][4];
+            float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int tok = tok0 + 8 * j + 2 * c4 + (e & 1);
+                    sc[j][e] = (tok < lim[e >> 1]) ? (sa[j][e] + sb[j][e]) * p.scale_log2 : -INFINITY;
+                    mx[e >> 1] = fmaxf(mx[e >> 1], sc[j][e]);
+                }
+            float alpha[2], m_ref[2];
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                mx[hf] = fmaxf(mx[hf], __shfl_xor_sync(kFull, mx[hf], 1));
+                mx[hf] = fmaxf(mx[hf], __shfl_xor_sync(kFull, mx[hf], 2));
+                const float m_new = fmaxf(m_run[hf], mx[hf]);
+                m_ref[hf] = (m_new == -INFINITY) ? 0.f : m_new;
+                alpha[hf] = ex2(m_run[hf] - m_ref[hf]);
+                m_run[hf] = m_new;
+            }
+            // P as the A operand: a0 row g tokens 2c4.., a1 row g+8, a2/a3 tokens 8+2c4..
+            const uint32_t pa0 = pack_bf16(ex2(sc[0][0] - m_ref[0]), ex2(sc[0][1] - m_ref[0]));
+            const uint32_t pa1 = pack_bf16(ex2(sc[0][2] - m_ref[1]), ex2(sc[0][3] - m_ref[1]));
+            const uint32_t pa2 = pack_bf16(ex2(sc[1][0] - m_ref[0]), ex2(sc[1][1] - m_ref[0]));
+            const uint32_t pa3 = pack_bf16(ex2(sc[1][2] - m_ref[1]), ex2(sc[1][3] - m_ref[1]));
+            l_run[0] = l_run[0] * alpha[0] + ((bf16_lo(pa0) + bf16_hi(pa0)) + (bf16_lo(pa2) + bf16_hi(pa2)));
+            l_run[1] = l_run[1] * alpha[1] + ((bf16_lo(pa1) + bf16_hi(pa1)) + (bf16_lo(pa3) + bf16_hi(pa3)));
+            if (__any_sync(kFull, alpha[0] != 1.f || alpha[1] != 1.f)) {
+#pragma unroll
+                for (int nt = 0; nt < NTD; ++nt) {
+                    o[nt][0] *= alpha[0];
+                    o[nt][1] *= alpha[0];
+                    o[nt][2] *= alpha[1];
+                    o[nt][3] *= alpha[1];
+                }
+            }
+
+            // O += P V
+#pragma unroll
+            for (int dj = 0; dj < D / 16; ++dj) {
+                uint32_t r0, r1, r2, r3;
+                ldsm_x4_trans(vb + tile_off<D, false>(tokV, 2 * dj + (mi >> 1)), r0, r1, r2, r3);
+                mma_bf16_16(o[2 * dj], pa0, pa1, pa2, pa3, r0, r1);
+                mma_bf16_16(o[2 * dj + 1], pa0, pa1, pa2, pa3, r2, r3);
+            }
+        }
+        __syncwarp();
+
+        // refill this stage with the tile `S` ahead; generic-proxy zero stores
+        // above must land before the async-proxy copy that overwrites the buffer
+        if (issued < ntiles) {
+            if (zeroed && lane == 0) fence_proxy_async_smem();
+            issue(s);
+            ++issued;
+        }
+
+        // ---- end of a pair (or of this range): write out or leave a partial -------
+        if (pair_end) {
+            float lsum[2];
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                lsum[hf] = l_run[hf] + __shfl_xor_sync(kFull, l_run[hf], 1);
+                lsum[hf] += __shfl_xor_sync(kFull, lsum[hf], 2);
+            }
+            const long long ts = (long long)prefix[cb] * Hkv + (long long)ckvh * cnt;
+            const long long te = ts + cnt;
+            const bool whole = u0 <= ts && te <= u1;
+            const int slot = 2 * w + (u0 < ts ? 1 : 0);
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                const int r = g + 8 * hf;
+                if (r >= R) continue;
+                if (whole) {
+                    const int t = r / G, h = r - t * G;
+                    const float inv = 1.f / lsum[hf];
+                    uint32_t* dst = reinterpret_cast<uint32_t*>(
+                        p.out + (((size_t)cb * QL + t) * p.Hq + (size_t)ckvh * G + h) * D);
+#pragma unroll
+                    for (int nt = 0; nt < NTD; ++nt)
+                        dst[(8 * nt + 2 * c4) >> 1] = pack_bf16(o[nt][2 * hf] * inv, o[nt][2 * hf + 1] * inv);
+                } else {
+                    float* dst = p.part_o + ((size_t)slot * R + r) * D;
+#pragma unroll
+                    for (int nt = 0; nt < NTD; ++nt)
+                        *reinterpret_cast<float2*>(dst + 8 * nt + 2 * c4) = make_float2(o[nt][2 * hf], o[nt][2 * hf + 1]);
+                    if (c4 == 0)
+                        *reinterpret_cast<float2*>(p.part_ml + ((size_t)slot * R + r) * 2) =
+                            make_float2(m_run[hf], lsum[hf]);
+                }
+            }
+        }
+
+        // advance the consumer cursor and the ring position
+        if (++ctt == cnt) {
+            ctt = 0;
+            if (++ckvh == Hkv) {
+                ckvh = 0;
+                do { ++cb; } while (cb < B && prefix[cb + 1] == prefix[cb]);
+            }
+            if (cb < B) cnt = prefix[cb + 1] - prefix[cb];
+        }
+        if (++s == S) {
+            s = 0;
+            parity ^= 1u;
+        }
+    }
+
+    // a worker that timed out still owns the loads it issued for tiles
+    // k_dead .. issued-1 (one per stage): wait for them, bounded
+    if (dead && lane == 0) {
+        for (int k = k_dead; k < issued; ++k)
+            (void)mbar_wait_bounded(my_bar0 + 8u * (k % S), (uint32_t)((k / S) & 1), kWaitLimitNs / 8);
+    }
+}
+
+template <int D>
+size_t tokens_smem_bytes(int stages, int max_batch)
+{
+    using Gm = Geo<D, false>;
+    return 1024 + (size_t)kAttnWarps * stages * (Gm::STAGEB + sizeof(StageInfo) + 8) +
+           sizeof(int) * (size_t)(max_batch + 1);
+}
+
+template <int D>
+cudaError_t prepare_tokens_t(int num_sms, int max_batch, AttnLaunch* out)
+{
+    int dev = 0, optin = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e != cudaSuccess) return e;
+    const int stages = kAttnMaxStages;
+    const size_t bytes = tokens_smem_bytes<D>(stages, max_batch);
+    if (bytes > (size_t)optin - 256) return cudaErrorInvalidConfiguration;
+    e = cudaFuncSetAttribute(decode_attn_tokens_kernel<D, kAttnWarps>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)bytes);
+    if (e != cudaSuccess) return e;
+    e = combine_prepare(D);
+    if (e != cudaSuccess) return e;
+    out->ctas = num_sms;
+    out->stages = stages;
+    out->smem_bytes = bytes;
+    return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t attn_tokens_prepare(int head_dim, int num_sms, int max_batch, AttnLaunch* out)
+{
+    return head_dim == 128 ? prepare_tokens_t<128>(num_sms, max_batch, out)
+                           : prepare_tokens_t<64>(num_sms, max_batch, out);
+}
+
+cudaError_t launch_decode_attn_tokens(const AttnParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
+                                      int head_dim, const AttnLaunch& L, cudaStream_t stream)
+{
+    const dim3 grid(L.ctas), block(kAttnWarps * 32);
+    AttnParams q = p;
+    q.stages = L.stages;
+    q.tail_chunks = 0;
+    if (head_dim == 128)
+        decode_attn_tokens_kernel<128, kAttnWarps><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
+    else
+        decode_attn_tokens_kernel<64, kAttnWarps><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return launch_combine(q, head_dim, L.ctas * kAttnWarps, L.ctas, stream);
+}
+
+}  // namespace pkv

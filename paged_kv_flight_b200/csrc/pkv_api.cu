@@ -9,6 +9,8 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <algorithm>
+
 #include <cudaTypedefs.h>
 
 #include "pkv_internal.h"
@@ -19,6 +21,7 @@ struct pkv_ctx {
     int num_sms;
     int G;
     pkv::AttnLaunch attn;
+    pkv::AttnLaunch attn_tok;     // several new tokens per request (bf16 pools)
     int workers;
     int tail_chunks;      // largest number of dynamic tail chunks per warp range
     void* ws;             // one allocation, carved below
@@ -134,14 +137,21 @@ pkv_status pkv_create(const pkv_config* cfg, pkv_ctx** out)
         free(ctx);
         return PKV_ERR_CUDA;
     }
+    if (!fp8 && pkv::attn_tokens_prepare(cfg->head_dim, ctx->num_sms, cfg->max_batch, &ctx->attn_tok) != cudaSuccess) {
+        free(ctx);
+        return PKV_ERR_CUDA;
+    }
 
     // [error word, chunk counter | split geometry | partial rows | partial (m, l)];
-    // two partial slots per unit of the split, G rows each
+    // two partial slots per unit of the split: G rows each for one new token
+    // per request (up to kMaxTailChunks + 1 units per warp), up to
+    // kMaxTokenRows rows for several (one unit per warp)
     const size_t units = pkv::max_units(ctx->attn.ctas * pkv::kAttnWarps, pkv::kMaxTailChunks);
+    const size_t rows_units = std::max(units * ctx->G, (size_t)ctx->attn.ctas * pkv::kAttnWarps * pkv::kMaxTokenRows);
     const size_t b_err = 256;
     const size_t b_cnt = ((size_t)(cfg->max_batch + 8) * sizeof(int) + 255) & ~(size_t)255;
-    const size_t b_po = 2 * units * ctx->G * cfg->head_dim * sizeof(float);
-    const size_t b_pml = 2 * units * ctx->G * 2 * sizeof(float);
+    const size_t b_po = 2 * rows_units * cfg->head_dim * sizeof(float);
+    const size_t b_pml = 2 * rows_units * 2 * sizeof(float);
     ctx->ws_bytes = b_err + b_cnt + b_po + b_pml;
     if (cudaMalloc(&ctx->ws, ctx->ws_bytes) != cudaSuccess) {
         cudaGetLastError();
@@ -194,6 +204,7 @@ pkv_status pkv_rope_append(pkv_ctx* ctx, void* q, const void* k_new, const void*
     p.P = ctx->cfg.page_size;
     p.num_pages = ctx->cfg.num_pages;
     p.fp8 = ctx->cfg.kv_dtype == PKV_KV_FP8_E4M3;
+    p.q_len = 1;
     return pkv::launch_rope_append(p, stream) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
@@ -238,8 +249,94 @@ pkv_status pkv_decode_attn(pkv_ctx* ctx, const void* q, const void* k_pool, cons
     p.stages = ctx->attn.stages;
     p.workers = ctx->workers;
     p.tail_chunks = ctx->tail_chunks;
+    p.q_len = 1;
     const cudaError_t e = pkv::launch_decode_attn(p, ctx->tmk, ctx->tmv, ctx->cfg.head_dim,
                                                   ctx->cfg.kv_dtype == PKV_KV_FP8_E4M3, ctx->attn, stream);
+    return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+pkv_status pkv_rope_append_tokens(pkv_ctx* ctx, void* q, const void* k_new, const void* v_new, void* k_pool,
+                                  void* v_pool, const float* k_scale, const float* v_scale,
+                                  const int32_t* block_tables, int bt_stride, const int32_t* seq_lens, int batch,
+                                  int q_len, cudaStream_t stream)
+{
+    pkv_status st = check_call(ctx, batch, bt_stride, k_pool, v_pool, k_scale, v_scale, block_tables, seq_lens);
+    if (st != PKV_OK || batch == 0) return st;
+    if (q_len < 1 || (long long)batch * q_len > (1LL << 31) - 1) return PKV_ERR_INVALID_ARG;
+    if (!q || !k_new || !v_new || !aligned16(q) || !aligned16(k_new) || !aligned16(v_new))
+        return PKV_ERR_INVALID_ARG;
+
+    pkv::RopeParams p;
+    p.q = static_cast<__nv_bfloat16*>(q);
+    p.k_new = static_cast<const __nv_bfloat16*>(k_new);
+    p.v_new = static_cast<const __nv_bfloat16*>(v_new);
+    p.k_pool = k_pool;
+    p.v_pool = v_pool;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
+    p.block_tables = block_tables;
+    p.seq_lens = seq_lens;
+    p.err = ctx->d_err;
+    p.rope_base = ctx->cfg.rope_base;
+    p.batch = batch;
+    p.bt_stride = bt_stride;
+    p.Hq = ctx->cfg.num_q_heads;
+    p.Hkv = ctx->cfg.num_kv_heads;
+    p.D = ctx->cfg.head_dim;
+    p.P = ctx->cfg.page_size;
+    p.num_pages = ctx->cfg.num_pages;
+    p.fp8 = ctx->cfg.kv_dtype == PKV_KV_FP8_E4M3;
+    p.q_len = q_len;
+    return pkv::launch_rope_append(p, stream) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+pkv_status pkv_decode_attn_tokens(pkv_ctx* ctx, const void* q, const void* k_pool, const void* v_pool,
+                                  const float* k_scale, const float* v_scale, const int32_t* block_tables,
+                                  int bt_stride, const int32_t* seq_lens, int batch, int q_len, void* out,
+                                  cudaStream_t stream)
+{
+    pkv_status st = check_call(ctx, batch, bt_stride, k_pool, v_pool, k_scale, v_scale, block_tables, seq_lens);
+    if (st != PKV_OK || batch == 0) return st;
+    if (q_len < 1) return PKV_ERR_INVALID_ARG;
+    if (ctx->cfg.kv_dtype != PKV_KV_BF16) return PKV_ERR_UNSUPPORTED;
+    if ((long long)ctx->G * q_len > pkv::kMaxTokenRows) return PKV_ERR_UNSUPPORTED;
+    if (!q || !out || !aligned16(q) || !aligned16(out)) return PKV_ERR_INVALID_ARG;
+
+    if (ctx->tm_k_ptr != k_pool) {
+        if (!encode_pool(ctx, k_pool, &ctx->tmk)) return PKV_ERR_CUDA;
+        ctx->tm_k_ptr = k_pool;
+    }
+    if (ctx->tm_v_ptr != v_pool) {
+        if (!encode_pool(ctx, v_pool, &ctx->tmv)) return PKV_ERR_CUDA;
+        ctx->tm_v_ptr = v_pool;
+    }
+
+    pkv::AttnParams p;
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.k_scale = nullptr;
+    p.v_scale = nullptr;
+    p.block_tables = block_tables;
+    p.seq_lens = seq_lens;
+    p.part_o = ctx->d_part_o;
+    p.part_ml = ctx->d_part_ml;
+    p.meta = ctx->d_meta;
+    p.err = ctx->d_err;
+    p.claim = ctx->d_claim;
+    p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)ctx->cfg.head_dim));
+    p.batch = batch;
+    p.bt_stride = bt_stride;
+    p.Hq = ctx->cfg.num_q_heads;
+    p.Hkv = ctx->cfg.num_kv_heads;
+    p.G = ctx->G;
+    p.P = ctx->cfg.page_size;
+    p.num_pages = ctx->cfg.num_pages;
+    p.stages = ctx->attn_tok.stages;
+    p.workers = ctx->workers;
+    p.tail_chunks = 0;
+    p.q_len = q_len;
+    const cudaError_t e = pkv::launch_decode_attn_tokens(p, ctx->tmk, ctx->tmv, ctx->cfg.head_dim, ctx->attn_tok,
+                                                         stream);
     return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 

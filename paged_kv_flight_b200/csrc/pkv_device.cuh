@@ -147,6 +147,19 @@ __device__ __forceinline__ void mma_bf16_r8(float& d0, float& d1, uint32_t a0, u
         : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "f"(0.f), "f"(0.f));
 }
 
+// D = A * B + D for one full m16n8k16 tile: d[0], d[1] row lane/4, d[2], d[3]
+// row lane/4 + 8 (columns 2 (lane%4) and +1); a0/a2 rows lane/4, a1/a3 rows
+// lane/4 + 8 (k 2 (lane%4).. and 8 + 2 (lane%4)..).
+__device__ __forceinline__ void mma_bf16_16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                            uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 __device__ __forceinline__ void mma_f16_r8(float& d0, float& d1, uint32_t a0, uint32_t a2,
                                            uint32_t b0, uint32_t b1)
 {

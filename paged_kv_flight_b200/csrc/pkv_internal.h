@@ -25,6 +25,7 @@ enum : int { kErrLength = 1, kErrPage = 2, kErrTimeout = 4 };
 
 constexpr int kTile = 16;          // tokens per attention tile (one TMA box height)
 constexpr int kMaxGroup = 8;       // query heads per kv head handled by one mma row block
+constexpr int kMaxTokenRows = 16;  // G x q_len rows of the several-new-tokens attention
 constexpr int kAttnWarps = PKV_ATTN_WARPS;
 constexpr int kAttnMaxStages = PKV_ATTN_MAX_STAGES;
 constexpr int kMinTilesPerWorker = 8;
@@ -63,6 +64,7 @@ struct RopeParams {
     int* err;
     double rope_base;
     int batch, bt_stride, Hq, Hkv, D, P, num_pages, fp8;
+    int q_len;            // new tokens per request, at positions L_b .. L_b + q_len - 1
 };
 
 struct AttnParams {
@@ -82,6 +84,7 @@ struct AttnParams {
     int stages;           // pipeline depth per warp
     int workers;          // 0: automatic
     int tail_chunks;      // largest K (chunks per warp tail); 0: static split only
+    int q_len;            // new tokens per request (1: one new token); partial rows = G x q_len
 };
 
 cudaError_t launch_rope_append(const RopeParams& p, cudaStream_t stream);
@@ -95,5 +98,18 @@ struct AttnLaunch {
 cudaError_t attn_prepare(int head_dim, bool fp8, int num_sms, int max_batch, AttnLaunch* out);
 cudaError_t launch_decode_attn(const AttnParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
                                int head_dim, bool fp8, const AttnLaunch& L, cudaStream_t stream);
+
+// Attention of several new tokens per request (decode_attn_tokens.cu, bf16
+// pools, G x q_len <= 16): shape of its launch and the launch itself
+// (attention, then the combine).
+cudaError_t attn_tokens_prepare(int head_dim, int num_sms, int max_batch, AttnLaunch* out);
+cudaError_t launch_decode_attn_tokens(const AttnParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
+                                      int head_dim, const AttnLaunch& L, cudaStream_t stream);
+
+// The split combine (combine.cu), run after either attention kernel: sets its
+// shared-memory limits once per head_dim, and launches it for p (max_units_n:
+// units the split may use; ctas: attention CTAs, for the choice of mode).
+cudaError_t combine_prepare(int head_dim);
+cudaError_t launch_combine(const AttnParams& p, int head_dim, int max_units_n, int ctas, cudaStream_t stream);
 
 }  // namespace pkv

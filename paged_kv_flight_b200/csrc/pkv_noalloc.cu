@@ -175,6 +175,7 @@ extern "C" pkv_status pkv_decode_attn_noalloc(const pkv_config* cfg, const void*
     p.stages = L.stages;
     p.workers = 0;
     p.tail_chunks = 0;
+    p.q_len = 1;
     return pkv::launch_decode_attn(p, tmk, tmv, cfg->head_dim, fp8, L, stream) == cudaSuccess ? PKV_OK
                                                                                               : PKV_ERR_CUDA;
 }

@@ -10,7 +10,12 @@
 // positions to physical blocks) and section "4. Native FP8 Quantization"
 // (E4M3 storage).
 //
-// Grid (request, chunk): a request's Hq + Hkv rows are cut into work items of
+// Several new tokens per request (speculative-decode verification: "Scaling
+// TensorRT-LLM", section "3. Speculative Decoding for Tail Latency") are the
+// same operation at positions L_b + t: the grid's first axis runs over
+// (request, new token) and q / k_new / v_new carry a token axis.
+//
+// Grid (request x new token, chunk): a token's Hq + Hkv rows are cut into work items of
 // 8 rotation pairs (two 16-byte loads, two 16-byte bf16 or 8-byte E4M3
 // stores), 128 items per CTA.  Each thread issues its row loads first; the
 // CTA meanwhile builds the cos/sin table of the request's position in fp64:
@@ -45,7 +50,8 @@ __global__ void __launch_bounds__(kRopeThreads) rope_append_kernel(const RopePar
     constexpr int PIECES = HALF / 8;  // 8 pairs per work item
     __shared__ double s_cos[HALF], s_sin[HALF];
 
-    const int b = blockIdx.x;
+    const int bt = blockIdx.x;               // (request, new token) row of q, k_new, v_new
+    const int b = bt / p.q_len, t = bt - b * p.q_len;
     const int rows = p.Hq + p.Hkv;
     const int it = blockIdx.y * kRopeThreads + threadIdx.x;
     const bool active = it < rows * PIECES;
@@ -57,19 +63,21 @@ __global__ void __launch_bounds__(kRopeThreads) rope_append_kernel(const RopePar
     // loads that do not depend on the position go out first
     uint4 xa = make_uint4(0, 0, 0, 0), xb = xa, va = xa, vb = xa;
     if (active) {
-        const __nv_bfloat16* src = is_q ? p.q + ((size_t)b * p.Hq + r) * D
-                                        : p.k_new + ((size_t)b * p.Hkv + kvh) * D;
+        const __nv_bfloat16* src = is_q ? p.q + ((size_t)bt * p.Hq + r) * D
+                                        : p.k_new + ((size_t)bt * p.Hkv + kvh) * D;
         xa = *reinterpret_cast<const uint4*>(src + i0);          // x_i
         xb = *reinterpret_cast<const uint4*>(src + i0 + HALF);   // x_{i+d/2}
         if (!is_q) {
-            const __nv_bfloat16* vsrc = p.v_new + ((size_t)b * p.Hkv + kvh) * D;
+            const __nv_bfloat16* vsrc = p.v_new + ((size_t)bt * p.Hkv + kvh) * D;
             va = *reinterpret_cast<const uint4*>(vsrc + i0);
             vb = *reinterpret_cast<const uint4*>(vsrc + i0 + HALF);
         }
     }
 
-    const int L = p.seq_lens[b];
-    const bool len_ok = L >= 0 && (long long)L < (long long)p.bt_stride * p.P;
+    const int L0 = p.seq_lens[b];
+    const long long Lt = (long long)L0 + t;  // position of this new token
+    const bool len_ok = L0 >= 0 && Lt < (long long)p.bt_stride * p.P;
+    const int L = (int)Lt;
     const int page = len_ok ? p.block_tables[(size_t)b * p.bt_stride + L / p.P] : -1;
     if (!len_ok) {
         if (threadIdx.x == 0 && blockIdx.y == 0) atomicOr(p.err, kErrLength);
@@ -114,7 +122,7 @@ __global__ void __launch_bounds__(kRopeThreads) rope_append_kernel(const RopePar
             ob[k] = (uint32_t)__bfloat16_as_ushort(dev::bf16_from_f64(yb[2 * k])) |
                     ((uint32_t)__bfloat16_as_ushort(dev::bf16_from_f64(yb[2 * k + 1])) << 16);
         }
-        __nv_bfloat16* dst = is_q ? p.q + ((size_t)b * p.Hq + r) * D
+        __nv_bfloat16* dst = is_q ? p.q + ((size_t)bt * p.Hq + r) * D
                                   : reinterpret_cast<__nv_bfloat16*>(p.k_pool) + prow * D;
         *reinterpret_cast<uint4*>(dst + i0) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
         *reinterpret_cast<uint4*>(dst + i0 + HALF) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
@@ -157,7 +165,7 @@ __global__ void __launch_bounds__(kRopeThreads) rope_append_kernel(const RopePar
 cudaError_t launch_rope_append(const RopeParams& p, cudaStream_t stream)
 {
     const int items = (p.Hq + p.Hkv) * (p.D / 16);
-    const dim3 grid(p.batch, (items + kRopeThreads - 1) / kRopeThreads), block(kRopeThreads);
+    const dim3 grid(p.batch * p.q_len, (items + kRopeThreads - 1) / kRopeThreads), block(kRopeThreads);
     if (p.D == 128) {
         if (p.fp8) rope_append_kernel<128, true><<<grid, block, 0, stream>>>(p);
         else rope_append_kernel<128, false><<<grid, block, 0, stream>>>(p);

@@ -41,7 +41,7 @@ PKV_KV_FP8_E4M3 = 1
 # names of every symbol include/pkv.h declares
 EXPORTS = ("pkv_create", "pkv_rope_append", "pkv_decode_attn", "pkv_destroy", "pkv_status_str",
            "pkv_check_device_error", "pkv_set_workers", "pkv_workspace_bytes", "pkv_decode_attn_noalloc",
-           "pkv_set_tail_chunks")
+           "pkv_set_tail_chunks", "pkv_rope_append_tokens", "pkv_decode_attn_tokens")
 
 
 class pkv_config(C.Structure):
@@ -65,6 +65,10 @@ lib.pkv_check_device_error.argtypes = [_V, _V, C.POINTER(C.c_int)]
 lib.pkv_check_device_error.restype = C.c_int
 lib.pkv_set_workers.argtypes = [_V, C.c_int]
 lib.pkv_set_workers.restype = C.c_int
+lib.pkv_rope_append_tokens.argtypes = [_V, _V, _V, _V, _V, _V, _V, _V, _V, C.c_int, _V, C.c_int, C.c_int, _V]
+lib.pkv_rope_append_tokens.restype = C.c_int
+lib.pkv_decode_attn_tokens.argtypes = [_V, _V, _V, _V, _V, _V, _V, C.c_int, _V, C.c_int, C.c_int, _V, _V]
+lib.pkv_decode_attn_tokens.restype = C.c_int
 lib.pkv_set_tail_chunks.argtypes = [_V, C.c_int]
 lib.pkv_set_tail_chunks.restype = C.c_int
 lib.pkv_workspace_bytes.argtypes = [_V]
@@ -190,3 +194,35 @@ def pkv_decode_attn_noalloc(cfg: pkv_config, q, k_pool, v_pool, k_scale, v_scale
                                      _ptr(v_scale), _ptr(block_tables), int(bt_stride), _ptr(seq_lens),
                                      int(batch), _ptr(out), _stream(stream))
     return _done(st, "pkv_decode_attn_noalloc", check)
+
+
+def pkv_rope_append_tokens(ctx, q, k_new, v_new, k_pool, v_pool, k_scale, v_scale, block_tables, seq_lens,
+                           batch: int | None = None, q_len: int | None = None, bt_stride: int | None = None,
+                           stream=None, check: bool = True) -> int:
+    """q [batch, q_len, Hq, d], k_new / v_new [batch, q_len, Hkv, d]."""
+    if batch is None:
+        batch = int(seq_lens.shape[0])
+    if q_len is None:
+        q_len = int(q.shape[1])
+    if bt_stride is None:
+        bt_stride = int(block_tables.shape[1])
+    st = lib.pkv_rope_append_tokens(ctx, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_pool), _ptr(v_pool),
+                                    _ptr(k_scale), _ptr(v_scale), _ptr(block_tables), int(bt_stride),
+                                    _ptr(seq_lens), int(batch), int(q_len), _stream(stream))
+    return _done(st, "pkv_rope_append_tokens", check)
+
+
+def pkv_decode_attn_tokens(ctx, q, k_pool, v_pool, k_scale, v_scale, block_tables, seq_lens, out,
+                           batch: int | None = None, q_len: int | None = None, bt_stride: int | None = None,
+                           stream=None, check: bool = True) -> int:
+    """q and out [batch, q_len, Hq, d]."""
+    if batch is None:
+        batch = int(seq_lens.shape[0])
+    if q_len is None:
+        q_len = int(q.shape[1])
+    if bt_stride is None:
+        bt_stride = int(block_tables.shape[1])
+    st = lib.pkv_decode_attn_tokens(ctx, _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(k_scale), _ptr(v_scale),
+                                    _ptr(block_tables), int(bt_stride), _ptr(seq_lens), int(batch), int(q_len),
+                                    _ptr(out), _stream(stream))
+    return _done(st, "pkv_decode_attn_tokens", check)

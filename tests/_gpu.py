@@ -54,7 +54,7 @@ def request_view(w: Workload, b: int, dev_orig: dict | None = None):
     """Oracle inputs for request b alone: its pages copied out of the original
     pools into a private pool, block table renumbered 0..n-1."""
     L = int(w.seq_lens[b])
-    npg = (L + 1 + w.P - 1) // w.P
+    npg = (L + w.q_len + w.P - 1) // w.P          # pages up to the last new token
     pages = w.block_tables[b, :npg].astype(np.int64)
     src = dev_orig if dev_orig is not None else dict(k_pool=w.k_pool, v_pool=w.v_pool, k_scale=w.k_scale,
                                                      v_scale=w.v_scale, q=w.q, k_new=w.k_new, v_new=w.v_new)
