@@ -40,25 +40,27 @@ METRIC = "paged-KV decode attn: HBM GB/s (% of B200 peak), request-tokens/s, ste
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 DEFAULT_CONFIG = "llama8b"
-ATTN_SOURCES = ("paged_kv_flight_b200/csrc/decode_attn.cu", "paged_kv_flight_b200/csrc/pkv_device.cuh",
-                "paged_kv_flight_b200/csrc/pkv_internal.h")
+ATTN_SOURCES = ("paged_kv_flight_b200/csrc/decode_attn.cu", "paged_kv_flight_b200/csrc/decode_attn_tokens.cu",
+                "paged_kv_flight_b200/csrc/attn_common.cuh", "paged_kv_flight_b200/csrc/combine.cu",
+                "paged_kv_flight_b200/csrc/pkv_device.cuh", "paged_kv_flight_b200/csrc/pkv_internal.h")
 
 
 # ---------------------------------------------------------------- accounting
 
-def metric_bytes(seq_lens, Hq, Hkv, d, P, kv_fp8) -> int:
-    """Resident KV attended (the new token included) + q read + out written
-    (+ the two fp32 scales per attended page and kv head for E4M3 pools)."""
-    n = np.asarray(seq_lens, np.int64) + 1
+def metric_bytes(seq_lens, Hq, Hkv, d, P, kv_fp8, q_len=1) -> int:
+    """Resident KV attended (the new tokens included, read once per request
+    and kv head) + q read + out written (+ the two fp32 scales per attended
+    page and kv head for E4M3 pools)."""
+    n = np.asarray(seq_lens, np.int64) + q_len
     s = 1 if kv_fp8 else 2
     kv = int((2 * Hkv * n * d * s).sum())
-    qo = 2 * len(n) * Hq * d * 2
+    qo = 2 * len(n) * q_len * Hq * d * 2
     sc = int(2 * ((n + P - 1) // P).sum() * Hkv * 4) if kv_fp8 else 0
     return kv + qo + sc
 
 
 def workload_bytes(w) -> int:
-    return metric_bytes(w.seq_lens, w.Hq, w.Hkv, w.d, w.P, w.kv_fp8)
+    return metric_bytes(w.seq_lens, w.Hq, w.Hkv, w.d, w.P, w.kv_fp8, w.q_len)
 
 
 def measured_peak():
@@ -210,7 +212,7 @@ def _request_pages(w, b, src):
     """Host copies (oracle form) of request b's pages, block table renumbered."""
     import torch
     L = int(w.seq_lens[b])
-    npg = (L + 1 + w.P - 1) // w.P
+    npg = (L + w.q_len + w.P - 1) // w.P
     idx = torch.from_numpy(w.block_tables[b, :npg].astype(np.int64)).to(src["k_pool"].device)
 
     def b16(t):
@@ -237,9 +239,15 @@ def oracle_step_requests(w, views):
         cfg = oracle.OracleConfig(w.Hq, w.Hkv, w.d, w.P, w.kv_fp8, v["npg"], w.rope_base)
         q = v["q"].copy()
         kp, vp = v["k_pool"].copy(), v["v_pool"].copy()
-        oracle.rope_append(cfg, q, v["k_new"], v["v_new"], kp, vp, v["k_scale"], v["v_scale"],
-                           v["block_tables"], v["seq_lens"])
-        oracle.decode_attn(cfg, q, kp, vp, v["k_scale"], v["v_scale"], v["block_tables"], v["seq_lens"])
+        if w.q_len > 1:
+            oracle.rope_append_tokens(cfg, q, v["k_new"], v["v_new"], kp, vp, v["k_scale"], v["v_scale"],
+                                      v["block_tables"], v["seq_lens"])
+            oracle.decode_attn_tokens(cfg, q, kp, vp, v["k_scale"], v["v_scale"], v["block_tables"],
+                                      v["seq_lens"])
+        else:
+            oracle.rope_append(cfg, q, v["k_new"], v["v_new"], kp, vp, v["k_scale"], v["v_scale"],
+                               v["block_tables"], v["seq_lens"])
+            oracle.decode_attn(cfg, q, kp, vp, v["k_scale"], v["v_scale"], v["block_tables"], v["seq_lens"])
 
 
 def sample_requests(w, token_head_budget: int):
@@ -247,7 +255,7 @@ def sample_requests(w, token_head_budget: int):
     (at least one request)."""
     picks, acc = [], 0
     for b, L in enumerate(w.seq_lens):
-        th = (int(L) + 1) * w.Hkv
+        th = (int(L) + w.q_len) * w.Hkv
         if picks and acc + th > token_head_budget:
             break
         picks.append(b)
@@ -267,8 +275,8 @@ def cpu_baseline(w, src, time_budget_s: float = 20.0) -> dict:
         done.append(b)
         if t_sum >= time_budget_s:
             break
-    by = metric_bytes(w.seq_lens[done], w.Hq, w.Hkv, w.d, w.P, w.kv_fp8)
-    toks = int((w.seq_lens[done].astype(np.int64) + 1).sum())
+    by = metric_bytes(w.seq_lens[done], w.Hq, w.Hkv, w.d, w.P, w.kv_fp8, w.q_len)
+    toks = int((w.seq_lens[done].astype(np.int64) + w.q_len).sum())
     return {"value": by / t_sum / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
             "seconds": t_sum,
             "sample": f"requests 0..{len(done) - 1} of {w.batch} ({toks} attended tokens, "
@@ -303,8 +311,19 @@ def run_ours(args, name, rank, world, local_rank):
     ctx = pkv.pkv_create(cfg)
     if args.tail_chunks is not None:
         pkv.pkv_set_tail_chunks(ctx, args.tail_chunks)
-    out = torch.empty(B, w.Hq, w.d, dtype=torch.bfloat16, device=dev)
+    tok = w.q_len > 1          # several new tokens per request: the *_tokens entry points
+    out = torch.empty(B, *((w.q_len,) if tok else ()), w.Hq, w.d, dtype=torch.bfloat16, device=dev)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+
+    def rope_call(x, stream=None):
+        fn = pkv.pkv_rope_append_tokens if tok else pkv.pkv_rope_append
+        fn(ctx, x["q"], x["k_new"], x["v_new"], dv["k_pool"], dv["v_pool"], dv["k_scale"], dv["v_scale"],
+           x["block_tables"], x["seq_lens"], stream=stream)
+
+    def attn_call(x, o, stream=None):
+        fn = pkv.pkv_decode_attn_tokens if tok else pkv.pkv_decode_attn
+        fn(ctx, x["q"], dv["k_pool"], dv["v_pool"], dv["k_scale"], dv["v_scale"], x["block_tables"],
+           x["seq_lens"], o, stream=stream)
     flush_w = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
     flush_r = torch.ones(2 * l2 // 8, dtype=torch.int64, device=dev)
     flush_sink = torch.empty((), dtype=torch.int64, device=dev)
@@ -326,10 +345,8 @@ def run_ours(args, name, rank, world, local_rank):
         cpu = cpu_baseline(w, dv, args.cpu_budget)
 
     def step():
-        pkv.pkv_rope_append(ctx, dv["q"], dv["k_new"], dv["v_new"], dv["k_pool"], dv["v_pool"],
-                            dv["k_scale"], dv["v_scale"], dv["block_tables"], dv["seq_lens"])
-        pkv.pkv_decode_attn(ctx, dv["q"], dv["k_pool"], dv["v_pool"], dv["k_scale"], dv["v_scale"],
-                            dv["block_tables"], dv["seq_lens"], out)
+        rope_call(dv)
+        attn_call(dv, out)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -366,11 +383,9 @@ def run_ours(args, name, rank, world, local_rank):
     for k in range(K):
         flush.zero_()                       # outside the event window
         ev[k][0].record()
-        pkv.pkv_rope_append(ctx, dv["q"], dv["k_new"], dv["v_new"], dv["k_pool"], dv["v_pool"],
-                            dv["k_scale"], dv["v_scale"], dv["block_tables"], dv["seq_lens"])
+        rope_call(dv)
         ev[k][1].record()
-        pkv.pkv_decode_attn(ctx, dv["q"], dv["k_pool"], dv["v_pool"], dv["k_scale"], dv["v_scale"],
-                            dv["block_tables"], dv["seq_lens"], out)
+        attn_call(dv, out)
         ev[k][2].record()
     clocks.sample()
     torch.cuda.synchronize()
@@ -461,10 +476,8 @@ def run_ours(args, name, rank, world, local_rank):
                 s_comp.wait_event(ev_in[sl])
                 if i >= 2:
                     s_comp.wait_event(ev_out[sl])         # output slot read back
-                pkv.pkv_rope_append(ctx, v["q"], v["k_new"], v["v_new"], dv["k_pool"], dv["v_pool"],
-                                    dv["k_scale"], dv["v_scale"], v["block_tables"], v["seq_lens"], stream=s_comp)
-                pkv.pkv_decode_attn(ctx, v["q"], dv["k_pool"], dv["v_pool"], dv["k_scale"], dv["v_scale"],
-                                    v["block_tables"], v["seq_lens"], outs[sl], stream=s_comp)
+                rope_call(v, stream=s_comp)
+                attn_call(v, outs[sl], stream=s_comp)
                 ev_comp[sl].record(s_comp)
                 s_out.wait_event(ev_comp[sl])
                 with torch.cuda.stream(s_out):
@@ -495,7 +508,8 @@ def run_ours(args, name, rank, world, local_rank):
     value = total_bytes / (step_max * 1e-3) / 1e9
     attn_gbs = by / (attn_max * 1e-3) / 1e9
     traffic = recorded_traffic(name)
-    kernel = f"decode_attn_kernel<{w.d},{'e4m3' if w.kv_fp8 else 'bf16'}>"
+    kernel = (f"decode_attn_tokens_kernel<{w.d},bf16>" if tok
+              else f"decode_attn_kernel<{w.d},{'e4m3' if w.kv_fp8 else 'bf16'}>")
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": step_max, "higher_is_better": True, "scaling": "weak",
@@ -503,7 +517,8 @@ def run_ours(args, name, rank, world, local_rank):
         "data": "synthetic: seeded lengths, page permutation, block tables and N(0,1) q/k/v "
                 "(per-workload recipe in paged_kv_flight_b200/workloads.py)",
         "config": {"workload": name, "description": workloads.DESCRIPTIONS[name], "batch": B,
-                   "tokens_attended": int((w.seq_lens.astype(np.int64) + 1).sum()),
+                   "tokens_attended": int((w.seq_lens.astype(np.int64) + w.q_len).sum()),
+                   "new_tokens_per_request": w.q_len,
                    "metric_bytes_per_step": by, "l2": "flushed before every timed step, outside the event window: write 2x L2, then read 2x L2",
                    "timing": ("each step replayed from one CUDA-graph capture of pkv_rope_append + pkv_decode_attn "
                               "(3 kernels); per-kernel times from the same steps launched eagerly"
@@ -539,7 +554,7 @@ def run_reference(args, name):
     src = _device_inputs(w, dev)
     picks = sample_requests(w, args.ref_budget)
     views = [_request_pages(w, b, src) for b in picks]
-    by = metric_bytes(w.seq_lens[picks], w.Hq, w.Hkv, w.d, w.P, w.kv_fp8)
+    by = metric_bytes(w.seq_lens[picks], w.Hq, w.Hkv, w.d, w.P, w.kv_fp8, w.q_len)
     for _ in range(args.warmup):
         oracle_step_requests(w, views)
     ts = []
@@ -549,7 +564,7 @@ def run_reference(args, name):
         ts.append(time.perf_counter() - t0)
     sec = sum(ts) / len(ts)
     value = by / sec / 1e9
-    toks = int((w.seq_lens[picks].astype(np.int64) + 1).sum())
+    toks = int((w.seq_lens[picks].astype(np.int64) + w.q_len).sum())
     sample = (f"requests 0..{len(picks) - 1} of {w.batch} ({toks} attended tokens, "
               f"{100.0 * by / workload_bytes(w):.1f}% of the step's bytes) per step; plain fp64 C oracle, "
               f"single thread, append + attention")
@@ -585,7 +600,7 @@ def main(argv=None):
         ap.error("--warmup must be >= 3")
 
     from paged_kv_flight_b200 import workloads
-    names = list(workloads.CONFIG_NAMES) if args.config == "all" else [args.config]
+    names = list(workloads.CONFIG_NAMES) + list(workloads.TOKEN_CONFIG_NAMES) if args.config == "all" else [args.config]
     rank, world, local_rank = dist_info()
 
     if args.impl == "reference":

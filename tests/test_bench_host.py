@@ -28,6 +28,14 @@ def test_metric_bytes_by_hand():
     assert bench.metric_bytes([0, 15], 8, 2, 64, 16, True) == kv8 + qo + scales
 
 
+def test_metric_bytes_with_several_new_tokens_by_hand():
+    # L = 0 and 15 with 3 new tokens each -> 3 and 18 tokens read once per
+    # (request, kv head); q and out for 3 tokens per request
+    kv = 2 * 2 * (3 + 18) * 64 * 2
+    qo = 2 * 2 * 3 * 8 * 64 * 2
+    assert bench.metric_bytes([0, 15], 8, 2, 64, 16, False, q_len=3) == kv + qo
+
+
 def test_llama8b_bytes_near_the_recipe_estimate():
     w_lens = workloads.draw_lengths("llama8b", np.random.default_rng(workloads.config_seed("llama8b")))
     by = bench.metric_bytes(w_lens, 32, 8, 128, 32, False)
