@@ -21,7 +21,7 @@ NVCC_FLAGS = [
 
 
 def sources():
-    return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+    return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cpp")))
 
 
 def needs_build() -> bool:
@@ -29,7 +29,7 @@ def needs_build() -> bool:
         return True
     t = os.path.getmtime(LIB)
     deps = sources() + glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh")) + \
-        [os.path.join(ROOT, "include", "pkv.h")]
+        [os.path.join(ROOT, "include", "pkv.h"), os.path.join(ROOT, "include", "pkv_pages.h")]
     return any(os.path.getmtime(d) > t for d in deps)
 
 

@@ -41,7 +41,10 @@ PKV_KV_FP8_E4M3 = 1
 # names of every symbol include/pkv.h declares
 EXPORTS = ("pkv_create", "pkv_rope_append", "pkv_decode_attn", "pkv_destroy", "pkv_status_str",
            "pkv_check_device_error", "pkv_set_workers", "pkv_workspace_bytes", "pkv_decode_attn_noalloc",
-           "pkv_set_tail_chunks", "pkv_rope_append_tokens", "pkv_decode_attn_tokens")
+           "pkv_set_tail_chunks", "pkv_rope_append_tokens", "pkv_decode_attn_tokens",
+           "pkv_pages_create", "pkv_pages_destroy", "pkv_pages_admit", "pkv_pages_reserve", "pkv_pages_advance",
+           "pkv_pages_release", "pkv_pages_block_table", "pkv_pages_seq_lens", "pkv_pages_active",
+           "pkv_pages_refcount", "pkv_pages_free_count", "pkv_pages_take_changes")
 
 
 class pkv_config(C.Structure):
@@ -69,6 +72,22 @@ lib.pkv_rope_append_tokens.argtypes = [_V, _V, _V, _V, _V, _V, _V, _V, _V, C.c_i
 lib.pkv_rope_append_tokens.restype = C.c_int
 lib.pkv_decode_attn_tokens.argtypes = [_V, _V, _V, _V, _V, _V, _V, C.c_int, _V, C.c_int, C.c_int, _V, _V]
 lib.pkv_decode_attn_tokens.restype = C.c_int
+lib.pkv_pages_create.argtypes = [C.c_int, C.c_int, C.c_int, C.c_int, C.POINTER(_V)]
+lib.pkv_pages_create.restype = C.c_int
+lib.pkv_pages_destroy.argtypes = [_V]
+lib.pkv_pages_destroy.restype = C.c_int
+lib.pkv_pages_admit.argtypes = [_V, C.c_int, C.c_int, C.c_int, C.c_int]
+lib.pkv_pages_admit.restype = C.c_int
+for _f in (lib.pkv_pages_reserve, lib.pkv_pages_advance, lib.pkv_pages_release):
+    _f.argtypes = [_V, C.c_int]
+    _f.restype = C.c_int
+for _f in (lib.pkv_pages_block_table, lib.pkv_pages_seq_lens, lib.pkv_pages_active, lib.pkv_pages_refcount):
+    _f.argtypes = [_V]
+    _f.restype = C.POINTER(C.c_int32)
+lib.pkv_pages_free_count.argtypes = [_V]
+lib.pkv_pages_free_count.restype = C.c_int
+lib.pkv_pages_take_changes.argtypes = [_V, _V, C.c_int]
+lib.pkv_pages_take_changes.restype = C.c_int
 lib.pkv_set_tail_chunks.argtypes = [_V, C.c_int]
 lib.pkv_set_tail_chunks.restype = C.c_int
 lib.pkv_workspace_bytes.argtypes = [_V]
@@ -226,3 +245,58 @@ def pkv_decode_attn_tokens(ctx, q, k_pool, v_pool, k_scale, v_scale, block_table
                                     _ptr(block_tables), int(bt_stride), _ptr(seq_lens), int(batch), int(q_len),
                                     _ptr(out), _stream(stream))
     return _done(st, "pkv_decode_attn_tokens", check)
+
+
+class Pages:
+    """The host page allocator (include/pkv_pages.h): marshalling only.  The
+    views (block_table, seq_lens, active, refcount) are numpy arrays over the
+    library's own memory, valid while the object lives."""
+
+    def __init__(self, num_pages: int, page_size: int, max_batch: int, max_blocks_per_seq: int):
+        h = _V()
+        _done(lib.pkv_pages_create(num_pages, page_size, max_batch, max_blocks_per_seq, C.byref(h)),
+              "pkv_pages_create", True)
+        self.h = h.value
+        self.num_pages, self.P, self.max_batch, self.max_blocks = num_pages, page_size, max_batch, max_blocks_per_seq
+        import numpy as np
+        self.block_table = np.ctypeslib.as_array(lib.pkv_pages_block_table(self.h),
+                                                 shape=(max_batch, max_blocks_per_seq))
+        self.seq_lens = np.ctypeslib.as_array(lib.pkv_pages_seq_lens(self.h), shape=(max_batch,))
+        self.active = np.ctypeslib.as_array(lib.pkv_pages_active(self.h), shape=(max_batch,))
+        self.refcount = np.ctypeslib.as_array(lib.pkv_pages_refcount(self.h), shape=(num_pages,))
+
+    def admit(self, slot: int, length: int, share_slot: int = -1, share_tokens: int = 0, check: bool = True) -> int:
+        return _done(lib.pkv_pages_admit(self.h, slot, length, share_slot, share_tokens), "pkv_pages_admit", check)
+
+    def reserve(self, q_len: int = 1, check: bool = True) -> int:
+        return _done(lib.pkv_pages_reserve(self.h, q_len), "pkv_pages_reserve", check)
+
+    def advance(self, q_len: int = 1, check: bool = True) -> int:
+        return _done(lib.pkv_pages_advance(self.h, q_len), "pkv_pages_advance", check)
+
+    def release(self, slot: int, check: bool = True) -> int:
+        return _done(lib.pkv_pages_release(self.h, slot), "pkv_pages_release", check)
+
+    @property
+    def free_count(self) -> int:
+        return lib.pkv_pages_free_count(self.h)
+
+    def take_changes(self, out) -> int:
+        """Block-table writes since the last call into `out` (int32, at least
+        3 * max entries, a numpy array or a host pointer): their count, or -1
+        when a full copy of the table is due."""
+        import numpy as np
+        if isinstance(out, np.ndarray):
+            return lib.pkv_pages_take_changes(self.h, out.ctypes.data, out.size // 3)
+        return lib.pkv_pages_take_changes(self.h, _ptr(out), int(out.numel()) // 3)
+
+    def close(self):
+        if self.h:
+            lib.pkv_pages_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,4 +1,4 @@
-"""The C-ABI library loads, exports every symbol include/pkv.h declares, and
+"""The C-ABI library loads, exports every symbol include/*.h declares, and
 rejects bad arguments on the host before any CUDA call (runs without a GPU)."""
 import ctypes as C
 import os
@@ -8,7 +8,7 @@ import subprocess
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "pkv.h")
+HEADERS = [os.path.join(ROOT, "include", h) for h in ("pkv.h", "pkv_pages.h")]
 
 
 @pytest.fixture(scope="module")
@@ -20,7 +20,7 @@ def pkv():
 
 
 def _declared():
-    text = open(HEADER).read()
+    text = "".join(open(h).read() for h in HEADERS)
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(pkv_[a-z_]+)\s*\(", text)))
 
