@@ -65,6 +65,8 @@ def _load():
         lib.orc_decode_attn_tokens.argtypes = [C.POINTER(_Cfg), P, P, P, P, P, P, C.c_int, P,
                                                C.c_int, C.c_int, P]
         lib.orc_decode_attn_tokens.restype = C.c_int
+        lib.orc_project_bf16.argtypes = [P, P, C.c_int, C.c_int, C.c_int, P]
+        lib.orc_project_bf16.restype = C.c_int
         _lib = lib
     return _lib
 
@@ -238,3 +240,18 @@ def decode_attn_tokens(cfg: OracleConfig, q, k_pool, v_pool, k_scale, v_scale, b
                                         _ptr(k_scale), _ptr(v_scale), _ptr(block_tables),
                                         block_tables.shape[1], _ptr(seq_lens), B, Q, _ptr(out))
     return out, st
+
+
+# ---- the QKV projection -------------------------------------------------------
+
+def project_bf16(x, w):
+    """bf16 bits: x [T, hidden], w [N, hidden] -> out [T, N] = bf16_RNE(x w^T),
+    the dot products in fp64."""
+    _need(x, np.uint16, "x"); _need(w, np.uint16, "w")
+    T, H = x.shape
+    N = w.shape[0]
+    assert w.shape[1] == H
+    out = np.zeros((T, N), np.uint16)
+    st = _load().orc_project_bf16(_ptr(x), _ptr(w), T, N, H, _ptr(out))
+    assert st == ORC_OK
+    return out

@@ -476,3 +476,26 @@ int orc_decode_attn_tokens(const orc_cfg* cfg, const uint16_t* q,
     }
     return status;
 }
+
+/* ------------------------------------------------------------------ */
+/* The QKV projection that produces q, k_new and v_new from the layer   */
+/* input, fused with RoPE and the append on the GPU ("Scaling           */
+/* TensorRT-LLM", section "What Gets Fused": the attention block's      */
+/* projections with their epilogues).  Definition: out[t][n] =          */
+/* bf16_RNE( sum_j x[t][j] * w[n][j] ) with the sum in fp64; w is        */
+/* [N][hidden] (one row per output feature).                            */
+/* ------------------------------------------------------------------ */
+
+int orc_project_bf16(const uint16_t* x, const uint16_t* w, int T, int N, int hidden, uint16_t* out)
+{
+    if (!x || !w || !out || T < 0 || N <= 0 || hidden <= 0) return ORC_ERR_ARG;
+    for (int t = 0; t < T; ++t) {
+        for (int n = 0; n < N; ++n) {
+            double s = 0.0;
+            for (int j = 0; j < hidden; ++j)
+                s += orc_bf16_decode(x[(size_t)t * hidden + j]) * orc_bf16_decode(w[(size_t)n * hidden + j]);
+            out[(size_t)t * N + n] = orc_bf16_encode_rne(s);
+        }
+    }
+    return ORC_OK;
+}

@@ -131,6 +131,11 @@ int orc_decode_attn_tokens(const orc_cfg* cfg, const uint16_t* q,
                            const int32_t* block_tables, int bt_stride,
                            const int32_t* seq_lens, int batch, int q_len, double* out);
 
+/* ---- the QKV projection ------------------------------------------------ */
+/* out[t][n] = bf16_RNE(sum_j x[t][j] w[n][j]), the sum in fp64; x is
+ * [T][hidden], w [N][hidden], out [T][N], all bf16 bits. */
+int orc_project_bf16(const uint16_t* x, const uint16_t* w, int T, int N, int hidden, uint16_t* out);
+
 #ifdef __cplusplus
 }
 #endif
