@@ -165,6 +165,25 @@ pkv_status pkv_decode_attn_tokens(pkv_ctx* ctx, const void* q, const void* k_poo
                                   const int32_t* seq_lens, int batch, int q_len, void* out,
                                   cudaStream_t stream);
 
+/* Step part 1 from the layer input: the QKV projection of the new tokens
+ * fused with RoPE and the append ("Scaling TensorRT-LLM: Kernel Fusion and
+ * Inflight Batching in Production", section "What Gets Fused").  x is the
+ * new tokens' input [batch][hidden] bf16 (one new token per request), w_qkv
+ * the projection [(Hq + 2 Hkv) d][hidden] bf16 (one row per output feature:
+ * the Hq q heads, then the Hkv k heads, then the Hkv v heads; row h d + i is
+ * dimension i of head h).  With y = bf16_RNE(x w_qkv^T) (fp32 accumulation on
+ * the tensor cores), it does what pkv_rope_append does with q = y's q part,
+ * k_new = y's k part, v_new = y's v part: q_out [batch][Hq][d] receives the
+ * rotated q, rotated k and raw v go into slot L_b % P of page
+ * block_tables[b][L_b / P] (bf16 or E4M3 pools).  hidden must be a multiple
+ * of 64 (PKV_ERR_UNSUPPORTED otherwise); x, w_qkv and q_out 16-byte aligned.
+ * Range errors as for pkv_rope_append. */
+pkv_status pkv_qkv_rope_append(pkv_ctx* ctx, const void* x, const void* w_qkv, int hidden, void* q_out,
+                               void* k_pool, void* v_pool,
+                               const float* k_scale, const float* v_scale,
+                               const int32_t* block_tables, int bt_stride,
+                               const int32_t* seq_lens, int batch, cudaStream_t stream);
+
 /* Frees the workspace.  NULL is accepted.  Synchronises the device. */
 pkv_status pkv_destroy(pkv_ctx* ctx);
 

@@ -34,6 +34,11 @@ struct pkv_ctx {
     const void* tm_k_ptr;
     const void* tm_v_ptr;
     CUtensorMap tmk, tmv;
+    const void* tm_w_ptr;        // QKV weight and input maps of pkv_qkv_rope_append
+    int tm_w_hidden;
+    const void* tm_x_ptr;
+    int tm_x_hidden, tm_x_rows;
+    CUtensorMap tmw, tmx;
 };
 
 namespace {
@@ -113,6 +118,22 @@ bool encode_pool(const pkv_ctx* ctx, const void* pool, CUtensorMap* map)
     return r == CUDA_SUCCESS;
 }
 
+// 2-D view of a row-major bf16 matrix [rows][cols] for the projection's TMA
+// loads: box = box_rows x 64 elements (one 128-byte row), 128-byte swizzle,
+// rows past the end read as zero.
+bool encode_rows(const void* base, int rows, int cols, int box_rows, CUtensorMap* map)
+{
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 extern "C" {
@@ -138,6 +159,10 @@ pkv_status pkv_create(const pkv_config* cfg, pkv_ctx** out)
         return PKV_ERR_CUDA;
     }
     if (!fp8 && pkv::attn_tokens_prepare(cfg->head_dim, ctx->num_sms, cfg->max_batch, &ctx->attn_tok) != cudaSuccess) {
+        free(ctx);
+        return PKV_ERR_CUDA;
+    }
+    if (pkv::qkv_prepare() != cudaSuccess) {
         free(ctx);
         return PKV_ERR_CUDA;
     }
@@ -338,6 +363,50 @@ pkv_status pkv_decode_attn_tokens(pkv_ctx* ctx, const void* q, const void* k_poo
     const cudaError_t e = pkv::launch_decode_attn_tokens(p, ctx->tmk, ctx->tmv, ctx->cfg.head_dim, ctx->attn_tok,
                                                          stream);
     return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+pkv_status pkv_qkv_rope_append(pkv_ctx* ctx, const void* x, const void* w_qkv, int hidden, void* q_out,
+                               void* k_pool, void* v_pool, const float* k_scale, const float* v_scale,
+                               const int32_t* block_tables, int bt_stride, const int32_t* seq_lens, int batch,
+                               cudaStream_t stream)
+{
+    pkv_status st = check_call(ctx, batch, bt_stride, k_pool, v_pool, k_scale, v_scale, block_tables, seq_lens);
+    if (st != PKV_OK || batch == 0) return st;
+    if (hidden < 64 || hidden % 64 != 0) return PKV_ERR_UNSUPPORTED;
+    if (!x || !w_qkv || !q_out || !aligned16(x) || !aligned16(w_qkv) || !aligned16(q_out))
+        return PKV_ERR_INVALID_ARG;
+    const int N = (ctx->cfg.num_q_heads + 2 * ctx->cfg.num_kv_heads) * ctx->cfg.head_dim;
+    if (ctx->tm_w_ptr != w_qkv || ctx->tm_w_hidden != hidden) {
+        if (!encode_rows(w_qkv, N, hidden, 16, &ctx->tmw)) return PKV_ERR_CUDA;
+        ctx->tm_w_ptr = w_qkv;
+        ctx->tm_w_hidden = hidden;
+    }
+    if (ctx->tm_x_ptr != x || ctx->tm_x_hidden != hidden || ctx->tm_x_rows != batch) {
+        if (!encode_rows(x, batch, hidden, 128, &ctx->tmx)) return PKV_ERR_CUDA;
+        ctx->tm_x_ptr = x;
+        ctx->tm_x_hidden = hidden;
+        ctx->tm_x_rows = batch;
+    }
+    pkv::QkvParams p;
+    p.seq_lens = seq_lens;
+    p.block_tables = block_tables;
+    p.q_out = static_cast<__nv_bfloat16*>(q_out);
+    p.k_pool = k_pool;
+    p.v_pool = v_pool;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
+    p.err = ctx->d_err;
+    p.rope_base = ctx->cfg.rope_base;
+    p.batch = batch;
+    p.hidden = hidden;
+    p.bt_stride = bt_stride;
+    p.Hq = ctx->cfg.num_q_heads;
+    p.Hkv = ctx->cfg.num_kv_heads;
+    p.D = ctx->cfg.head_dim;
+    p.P = ctx->cfg.page_size;
+    p.num_pages = ctx->cfg.num_pages;
+    p.fp8 = ctx->cfg.kv_dtype == PKV_KV_FP8_E4M3;
+    return pkv::launch_qkv_rope_append(p, ctx->tmx, ctx->tmw, stream) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
 pkv_status pkv_destroy(pkv_ctx* ctx)

@@ -106,6 +106,25 @@ cudaError_t attn_tokens_prepare(int head_dim, int num_sms, int max_batch, AttnLa
 cudaError_t launch_decode_attn_tokens(const AttnParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
                                       int head_dim, const AttnLaunch& L, cudaStream_t stream);
 
+// QKV projection of the new tokens on tcgen05, fused with RoPE and the append
+// (qkv_rope_append.cu).
+struct QkvParams {
+    const int32_t* seq_lens;
+    const int32_t* block_tables;
+    __nv_bfloat16* q_out;     // [batch][Hq][D], rotated
+    void* k_pool;
+    void* v_pool;
+    const float* k_scale;
+    const float* v_scale;
+    int* err;
+    double rope_base;
+    int batch, hidden, bt_stride, Hq, Hkv, D, P, num_pages, fp8;
+};
+size_t qkv_smem_bytes();
+cudaError_t qkv_prepare();
+cudaError_t launch_qkv_rope_append(const QkvParams& p, const CUtensorMap& tmx, const CUtensorMap& tmw,
+                                   cudaStream_t stream);
+
 // The split combine (combine.cu), run after either attention kernel: sets its
 // shared-memory limits once per head_dim, and launches it for p (max_units_n:
 // units the split may use; ctas: attention CTAs, for the choice of mode).

@@ -44,7 +44,7 @@ EXPORTS = ("pkv_create", "pkv_rope_append", "pkv_decode_attn", "pkv_destroy", "p
            "pkv_set_tail_chunks", "pkv_rope_append_tokens", "pkv_decode_attn_tokens",
            "pkv_pages_create", "pkv_pages_destroy", "pkv_pages_admit", "pkv_pages_reserve", "pkv_pages_advance",
            "pkv_pages_release", "pkv_pages_block_table", "pkv_pages_seq_lens", "pkv_pages_active",
-           "pkv_pages_refcount", "pkv_pages_free_count", "pkv_pages_take_changes")
+           "pkv_pages_refcount", "pkv_pages_free_count", "pkv_pages_take_changes", "pkv_qkv_rope_append")
 
 
 class pkv_config(C.Structure):
@@ -88,6 +88,8 @@ lib.pkv_pages_free_count.argtypes = [_V]
 lib.pkv_pages_free_count.restype = C.c_int
 lib.pkv_pages_take_changes.argtypes = [_V, _V, C.c_int]
 lib.pkv_pages_take_changes.restype = C.c_int
+lib.pkv_qkv_rope_append.argtypes = [_V, _V, _V, C.c_int, _V, _V, _V, _V, _V, _V, C.c_int, _V, C.c_int, _V]
+lib.pkv_qkv_rope_append.restype = C.c_int
 lib.pkv_set_tail_chunks.argtypes = [_V, C.c_int]
 lib.pkv_set_tail_chunks.restype = C.c_int
 lib.pkv_workspace_bytes.argtypes = [_V]
@@ -300,3 +302,18 @@ class Pages:
             self.close()
         except Exception:
             pass
+
+
+def pkv_qkv_rope_append(ctx, x, w_qkv, q_out, k_pool, v_pool, k_scale, v_scale, block_tables, seq_lens,
+                        batch: int | None = None, bt_stride: int | None = None, stream=None,
+                        check: bool = True) -> int:
+    """x [batch, hidden], w_qkv [(Hq + 2 Hkv) d, hidden], q_out [batch, Hq, d]."""
+    if batch is None:
+        batch = int(seq_lens.shape[0])
+    if bt_stride is None:
+        bt_stride = int(block_tables.shape[1])
+    hidden = int(x.shape[-1])
+    st = lib.pkv_qkv_rope_append(ctx, _ptr(x), _ptr(w_qkv), hidden, _ptr(q_out), _ptr(k_pool), _ptr(v_pool),
+                                 _ptr(k_scale), _ptr(v_scale), _ptr(block_tables), int(bt_stride), _ptr(seq_lens),
+                                 int(batch), _stream(stream))
+    return _done(st, "pkv_qkv_rope_append", check)

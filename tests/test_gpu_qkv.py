@@ -1,0 +1,113 @@
+"""GPU parity of the fused QKV projection + RoPE + append
+(pkv_qkv_rope_append, tcgen05 tensor cores) against the oracle: the fp64
+projection rounded to bf16 (orc_project_bf16), split into q / k_new / v_new,
+then the oracle's own RoPE + append (orc_rope_append).
+
+The kernel sums the hidden-size products in fp32 on the tensor cores (each
+bf16 x bf16 product is exact in fp32; the order and rounding of the sum are
+the hardware's), so a projection output differs from the fp64 sum by at most
+K 2^-23 S (K = hidden, S = sum_j |x_j w_j|, the worst case for fp32
+accumulation in any order, truncating or rounding), which can move it to
+another bf16 value; the rotation mixes the two members of a pair.  The bar:
+every element within 3 bf16 ulps of the larger magnitude of its rotation
+pair plus K 2^-23 S of the pair's features; at least 97% of the elements
+bit-identical; E4M3 codes within one step; every pool byte outside the
+landing slots untouched."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from paged_kv_flight_b200 import workloads
+from tests import _gpu
+from tests._util import bf16_ordinal, bits16, bytes8, host_inputs, oracle_cfg
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    # name, Hq, Hkv, d, P, hidden, lengths, fp8
+    ("small_d128", 8, 2, 128, 16, 256, [0, 5, 17, 40, 100], False),
+    ("llama8b_like", 32, 8, 128, 32, 4096, list(range(100, 100 + 64 * 37, 37)), False),
+    ("two_m_tiles_d64", 16, 4, 64, 16, 512, [3 * i for i in range(130)], False),
+    ("fp8_pools", 8, 2, 128, 32, 512, [1, 31, 32, 77, 300, 600, 1000], True),
+]
+
+
+@pytest.fixture(scope="module")
+def pkv():
+    from paged_kv_flight_b200 import pkv as mod
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return mod
+
+
+def _f(bits):
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: c[0])
+def test_fused_projection_matches_oracle(pkv, case):
+    name, Hq, Hkv, d, P, hidden, lengths, fp8 = case
+    w = workloads.build(name, Hq, Hkv, d, P, fp8, 5e5 if d == 128 else 1e4, lengths, 17, device="cpu")
+    B, N = w.batch, (Hq + 2 * Hkv) * d
+    gen = torch.Generator().manual_seed(5)
+    x = torch.randn(B, hidden, generator=gen).to(torch.bfloat16)
+    wq = (torch.randn(N, hidden, generator=gen) / hidden ** 0.5).to(torch.bfloat16)
+
+    dv = _gpu.to_device(w)
+    xd, wd = x.cuda(), wq.cuda()
+    q_out = torch.empty(B, Hq, d, dtype=torch.bfloat16, device="cuda")
+    ctx = _gpu.make_ctx(pkv, w)
+    try:
+        pkv.pkv_qkv_rope_append(ctx, xd, wd, q_out, dv["k_pool"], dv["v_pool"], dv["k_scale"], dv["v_scale"],
+                                dv["block_tables"], dv["seq_lens"])
+        assert pkv.pkv_check_device_error(ctx)[0] == pkv.PKV_OK
+    finally:
+        pkv.pkv_destroy(ctx)
+
+    # oracle: fp64 projection -> bf16, then the oracle's RoPE + append
+    y = oracle.project_bf16(bits16(x), bits16(wq))
+    # fp32 accumulation bound per (token, feature): K 2^-23 sum_j |x_j w_j|
+    acc = hidden * 2.0 ** -23 * (np.abs(x.double().numpy()) @ np.abs(wq.double().numpy()).T)
+    h = host_inputs(w)
+    h["q"] = np.ascontiguousarray(y[:, :Hq * d].reshape(B, Hq, d))
+    h["k_new"] = np.ascontiguousarray(y[:, Hq * d:(Hq + Hkv) * d].reshape(B, Hkv, d))
+    h["v_new"] = np.ascontiguousarray(y[:, (Hq + Hkv) * d:].reshape(B, Hkv, d))
+    assert oracle.rope_append(oracle_cfg(w), h["q"], h["k_new"], h["v_new"], h["k_pool"], h["v_pool"],
+                              h["k_scale"], h["v_scale"], h["block_tables"], h["seq_lens"]) == 0
+
+    def pair_max(a):
+        half = d // 2
+        m = np.maximum(a[..., :half], a[..., half:])
+        return np.concatenate([m, m], axis=-1)
+
+    def close_pairs(got_bits, ref_bits, acc_err, ulps=3):
+        """|got - ref| <= ulps 2^-8 max(|ref_i|, |ref_{i+d/2}|) + the pair's accumulation bound."""
+        g, r = _f(got_bits), _f(ref_bits)
+        tol = ulps * 2.0 ** -8 * np.maximum(pair_max(np.abs(r)), 2.0 ** -20) + pair_max(acc_err)
+        return bool((np.abs(g - r) <= tol).all())
+
+    acc_q = acc[:, :Hq * d].reshape(B, Hq, d)
+    acc_k = acc[:, Hq * d:(Hq + Hkv) * d].reshape(B, Hkv, d)
+    acc_v = acc[:, (Hq + Hkv) * d:].reshape(B, Hkv, d)
+    gq = bits16(q_out)
+    assert close_pairs(gq, h["q"], acc_q)
+    same = [np.mean(gq == h["q"])]
+    landing = {(int(w.block_tables[b, L // P]), kvh, int(L % P)) for b, L in enumerate(w.seq_lens)
+               for kvh in range(Hkv)}
+    conv = bytes8 if fp8 else bits16
+    for key in ("k_pool", "v_pool"):
+        got, ref = conv(dv[key]), h[key]
+        diff = got != ref
+        rows = {tuple(map(int, r[:3])) for r in np.argwhere(diff)}
+        assert rows <= landing, f"{key}: bytes changed outside the landing slots"
+        order = sorted((int(w.block_tables[b, L // P]), kvh, int(L % P), b) for b, L in enumerate(w.seq_lens)
+                       for kvh in range(Hkv))
+        gl = np.stack([got[pg, kvh, sl] for pg, kvh, sl, _ in order])
+        rl = np.stack([ref[pg, kvh, sl] for pg, kvh, sl, _ in order])
+        ae = np.stack([(acc_k if key == "k_pool" else acc_v)[b, kvh] for _, kvh, _, b in order])
+        if fp8:
+            assert np.abs(gl.astype(int) - rl.astype(int)).max() <= 1      # one E4M3 code step
+        else:
+            assert close_pairs(gl, rl, ae, ulps=3 if key == "k_pool" else 1)
+        same.append(np.mean(gl == rl))
+    assert min(same) >= 0.97, same
