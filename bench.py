@@ -42,7 +42,8 @@ FALLBACK_HBM_GBS = 6650.0
 DEFAULT_CONFIG = "llama8b"
 ATTN_SOURCES = ("paged_kv_flight_b200/csrc/decode_attn.cu", "paged_kv_flight_b200/csrc/decode_attn_tokens.cu",
                 "paged_kv_flight_b200/csrc/attn_common.cuh", "paged_kv_flight_b200/csrc/combine.cu",
-                "paged_kv_flight_b200/csrc/pkv_device.cuh", "paged_kv_flight_b200/csrc/pkv_internal.h")
+                "paged_kv_flight_b200/csrc/pkv_device.cuh", "paged_kv_flight_b200/csrc/pkv_internal.h",
+                "paged_kv_flight_b200/csrc/qkv_rope_append.cu")
 
 
 # ---------------------------------------------------------------- accounting
@@ -580,6 +581,120 @@ def run_reference(args, name):
     }
 
 
+def run_qkv(args, rank, world, local_rank):
+    """The attention step from the layer input on the llama8b batch: the QKV
+    projection on tcgen05 fused with RoPE and the append
+    (pkv_qkv_rope_append: x [64, 4096] bf16, W [6144, 4096] bf16, N(0,1) and
+    N(0, 1/4096)), then pkv_decode_attn.  L2 flushed before every step; the
+    projection timed alone with events, the whole step replayed from a CUDA
+    graph."""
+    import torch
+    from paged_kv_flight_b200 import pkv, workloads
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = workloads.make("llama8b", device=dev, offset=rank)
+    dv = _device_inputs(w, dev)
+    hidden = 4096
+    N = (w.Hq + 2 * w.Hkv) * w.d
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(workloads.config_seed("llama8b", rank) + 17)
+    x = torch.randn(w.batch, hidden, generator=gen, device=dev).to(torch.bfloat16)
+    W = (torch.randn(N, hidden, generator=gen, device=dev) / hidden ** 0.5).to(torch.bfloat16)
+    q = torch.empty(w.batch, w.Hq, w.d, dtype=torch.bfloat16, device=dev)
+    out = torch.empty_like(q)
+    cfg = pkv.make_config(w.Hq, w.Hkv, w.d, w.P, "bf16", w.rope_base, w.batch, w.bt_stride, w.num_pages)
+    ctx = pkv.pkv_create(cfg)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush_w = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+    flush_r = torch.ones(2 * l2 // 8, dtype=torch.int64, device=dev)
+    sink = torch.empty((), dtype=torch.int64, device=dev)
+
+    def flush():
+        flush_w.zero_()
+        torch.sum(flush_r, dim=0, out=sink)
+
+    def proj():
+        pkv.pkv_qkv_rope_append(ctx, x, W, q, dv["k_pool"], dv["v_pool"], None, None, dv["block_tables"],
+                                dv["seq_lens"])
+
+    def step():
+        proj()
+        pkv.pkv_decode_attn(ctx, q, dv["k_pool"], dv["v_pool"], None, None, dv["block_tables"], dv["seq_lens"], out)
+
+    for _ in range(args.warmup):
+        flush()
+        step()
+    torch.cuda.synchronize()
+    K = args.steps
+    side = torch.cuda.Stream(dev)
+    with torch.cuda.stream(side):
+        step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        step()
+    for _ in range(args.warmup):
+        flush()
+        graph.replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for k in range(K):
+        flush()
+        ev[k][0].record()
+        proj()
+        ev[k][1].record()
+    clocks.sample()
+    gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for k in range(K):
+        flush()
+        gev[k][0].record()
+        graph.replay()
+        gev[k][1].record()
+    clocks.sample()
+    torch.cuda.synchronize()
+    barrier()
+    clock_info = clocks.stop()
+    st, bits = pkv.pkv_check_device_error(ctx)
+    if st != pkv.PKV_OK:
+        raise RuntimeError(f"device error: {pkv.pkv_status_str(st)} bits={bits}")
+    del graph
+    pkv.pkv_destroy(ctx)
+    proj_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev) / K)
+    step_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in gev) / K)
+    # the projection's algorithmic bytes: weights and x read once, q written,
+    # k and v rows written; its flops: 2 x tokens x features x hidden
+    proj_bytes = N * hidden * 2 + w.batch * hidden * 2 + w.batch * N * 2
+    proj_flop = 2.0 * w.batch * N * hidden
+    attn_bytes = workload_bytes(w)
+    by = sum_over_ranks(float(proj_bytes + attn_bytes))
+    peak, peak_src = measured_peak()
+    gbs = proj_bytes / (proj_ms * 1e-3) / 1e9
+    tflops_peak = None
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            tflops_peak = float(json.load(f)["bf16_tflops"])
+    except Exception:
+        tflops_peak = 1590.0
+    return {"metric": METRIC, "value": by / (step_ms * 1e-3) / 1e9, "unit": "GB/s", "n_gpus": world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "qkv8b", "description": "llama8b batch (64 tokens) from the layer input: "
+                       "QKV projection 4096 -> 6144 on tcgen05 fused with RoPE + append, then decode attention",
+                       "l2": "flushed before every step, outside the event window",
+                       "timing": "projection alone: eager events; step: CUDA-graph replay of projection + attention"},
+            "step_us": step_ms * 1e3, "projection_us": proj_ms * 1e3,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                         "traffic": recorded_traffic("qkv8b"), "kernel": "qkv_rope_append_kernel<128>",
+                         "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)", "bytes_per_launch": proj_bytes},
+            "projection_tflops": proj_flop / (proj_ms * 1e-3) / 1e12,
+            "projection_tflops_frac_of_bf16_peak": proj_flop / (proj_ms * 1e-3) / 1e12 / tflops_peak,
+            "gpu_launches": 4 * K, "clocks": clock_info}
+
+
 def run_loop(args, rank, world, local_rank):
     """The continuous-batching loop (serve_loop.py) on a 70B-shaped layer:
     256 slots, prompts {64,128,512,2048} (+ a 512-token system prompt shared
@@ -654,6 +769,8 @@ def main(argv=None):
         for name in names:
             if name == "loop70b":
                 line = run_loop(args, rank, world, local_rank)
+            elif name == "qkv8b":
+                line = run_qkv(args, rank, world, local_rank)
             else:
                 line = run_ours(args, name, rank, world, local_rank)
             if rank == 0:

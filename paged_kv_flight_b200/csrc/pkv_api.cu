@@ -381,8 +381,9 @@ pkv_status pkv_qkv_rope_append(pkv_ctx* ctx, const void* x, const void* w_qkv, i
         ctx->tm_w_ptr = w_qkv;
         ctx->tm_w_hidden = hidden;
     }
+    const int x_rows = batch >= 128 ? 128 : (batch + 15) / 16 * 16;
     if (ctx->tm_x_ptr != x || ctx->tm_x_hidden != hidden || ctx->tm_x_rows != batch) {
-        if (!encode_rows(x, batch, hidden, 128, &ctx->tmx)) return PKV_ERR_CUDA;
+        if (!encode_rows(x, batch, hidden, x_rows, &ctx->tmx)) return PKV_ERR_CUDA;
         ctx->tm_x_ptr = x;
         ctx->tm_x_hidden = hidden;
         ctx->tm_x_rows = batch;
@@ -406,6 +407,7 @@ pkv_status pkv_qkv_rope_append(pkv_ctx* ctx, const void* x, const void* w_qkv, i
     p.P = ctx->cfg.page_size;
     p.num_pages = ctx->cfg.num_pages;
     p.fp8 = ctx->cfg.kv_dtype == PKV_KV_FP8_E4M3;
+    p.x_rows = x_rows;
     return pkv::launch_qkv_rope_append(p, ctx->tmx, ctx->tmw, stream) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 

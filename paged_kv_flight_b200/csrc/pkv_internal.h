@@ -119,6 +119,7 @@ struct QkvParams {
     int* err;
     double rope_base;
     int batch, hidden, bt_stride, Hq, Hkv, D, P, num_pages, fp8;
+    int x_rows;               // token rows per x TMA box: min(128, batch rounded up to 16)
 };
 size_t qkv_smem_bytes();
 cudaError_t qkv_prepare();

@@ -40,7 +40,7 @@ constexpr int kQkvThreads = 128;
 constexpr int kQkvM = 128;                 // tokens per tile (TMEM lanes, rows of A)
 constexpr int kQkvN = 32;                  // features per CTA: 16 pairs x 2 halves
 constexpr int kQkvBK = 64;                 // hidden elements per stage: one 128-byte row
-constexpr int kQkvStages = 6;
+constexpr int kQkvStages = 5;                // 5 x 20 KB: two CTAs per SM
 constexpr int kQkvAB = kQkvM * kQkvBK * 2; // 16 KB
 constexpr int kQkvBB = kQkvN * kQkvBK * 2; // 4 KB
 constexpr int kQkvStageB = kQkvAB + kQkvBB;
@@ -119,7 +119,7 @@ __device__ __forceinline__ void sincos_reduced(double phi, double* s, double* c)
 }
 
 template <int D>
-__global__ void __launch_bounds__(kQkvThreads, 1)
+__global__ void __launch_bounds__(kQkvThreads, 2)
 qkv_rope_append_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmw,
                        const QkvParams p)
 {
@@ -174,7 +174,10 @@ qkv_rope_append_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_con
                     break;
                 }
                 const uint32_t a = stage0 + (uint32_t)(s * kQkvStageB), b = a + kQkvAB;
-                mbar_arrive_expect_tx(full0 + 8u * s, (uint32_t)kQkvStageB);
+                // x_rows (<= 128) token rows; the MMA reads all 128 rows of the
+                // stage's A area, rows past x_rows only feed accumulator rows
+                // of no token
+                mbar_arrive_expect_tx(full0 + 8u * s, (uint32_t)(p.x_rows * kQkvBK * 2 + kQkvBB));
                 tma_load_2d(a, &tmx, kb * kQkvBK, m0, full0 + 8u * s);
                 tma_load_2d(b, &tmw, kb * kQkvBK, row_lo, full0 + 8u * s);
                 tma_load_2d(b + kQkvBB / 2, &tmw, kb * kQkvBK, row_hi, full0 + 8u * s);
@@ -201,11 +204,13 @@ qkv_rope_append_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_con
             umma_commit(done);   // arrives once every MMA issued above has completed
         }
     }
+    // the other lanes of warps 0 and 1 wait here, not in a spin beside the
+    // issuing lane, which keeps its warp's issue slots
+    __syncwarp();
 
     // ---- epilogue: every warp reads its 32 token rows out of tensor memory
     const bool ok = mbar_wait_bounded(done, 0u, kQkvWaitNs);
     if (!ok && tid == 0) atomicOr(p.err, kErrTimeout);
-    __syncwarp();                            // the warp's lanes converge before the aligned TMEM load
     tmem_fence_after();
     float acc[32];
     tmem_ld32(tmem + ((uint32_t)(32 * warp) << 16), acc);
