@@ -40,10 +40,15 @@ METRIC = "paged-KV decode attn: HBM GB/s (% of B200 peak), request-tokens/s, ste
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 DEFAULT_CONFIG = "llama8b"
-ATTN_SOURCES = ("paged_kv_flight_b200/csrc/decode_attn.cu", "paged_kv_flight_b200/csrc/decode_attn_tokens.cu",
-                "paged_kv_flight_b200/csrc/attn_common.cuh", "paged_kv_flight_b200/csrc/combine.cu",
-                "paged_kv_flight_b200/csrc/pkv_device.cuh", "paged_kv_flight_b200/csrc/pkv_internal.h",
-                "paged_kv_flight_b200/csrc/qkv_rope_append.cu")
+# sources of the kernel whose DRAM traffic a profile line records: the
+# attention kernels for the attention workloads, the fused projection for qkv8b
+KERNEL_SOURCES = {
+    "attn": ("paged_kv_flight_b200/csrc/decode_attn.cu", "paged_kv_flight_b200/csrc/decode_attn_tokens.cu",
+             "paged_kv_flight_b200/csrc/attn_common.cuh", "paged_kv_flight_b200/csrc/combine.cu",
+             "paged_kv_flight_b200/csrc/pkv_device.cuh", "paged_kv_flight_b200/csrc/pkv_internal.h"),
+    "qkv": ("paged_kv_flight_b200/csrc/qkv_rope_append.cu", "paged_kv_flight_b200/csrc/pkv_device.cuh",
+            "paged_kv_flight_b200/csrc/pkv_internal.h"),
+}
 
 
 # ---------------------------------------------------------------- accounting
@@ -74,18 +79,19 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def attn_source_sha() -> str:
+def source_sha(kernel: str = "attn") -> str:
     h = hashlib.sha256()
-    for rel in ATTN_SOURCES:
+    for rel in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(workload: str):
-    """DRAM bytes per attention launch from a committed ncu summary, if it was
-    taken on the current attention sources; otherwise None."""
-    sha = attn_source_sha()
+    """DRAM bytes per launch of the workload's dominant kernel from a
+    committed ncu summary, if it was taken on that kernel's current sources;
+    otherwise None."""
+    sha = source_sha("qkv" if workload == "qkv8b" else "attn")
     pat = re.compile(r"traffic-per-launch:\s+(\S+)\s+(\d+)\s+src=([0-9a-f]+)")
     pdir = os.path.join(ROOT, "profiles")
     if not os.path.isdir(pdir):
@@ -613,9 +619,14 @@ def run_qkv(args, rank, world, local_rank):
         flush_w.zero_()
         torch.sum(flush_r, dim=0, out=sink)
 
-    def proj():
-        pkv.pkv_qkv_rope_append(ctx, x, W, q, dv["k_pool"], dv["v_pool"], None, None, dv["block_tables"],
-                                dv["seq_lens"])
+    # the weight is static: packed once into the tiled layout at load time
+    Wt = torch.empty_like(W)
+    pkv.pkv_qkv_pack_weight(ctx, W, Wt)
+    shape = pkv.pkv_qkv_launch_shape(ctx, w.batch, hidden)
+
+    def proj(layout=pkv.PKV_W_TILED):
+        pkv.pkv_qkv_rope_append(ctx, x, Wt if layout == pkv.PKV_W_TILED else W, q, dv["k_pool"], dv["v_pool"],
+                                None, None, dv["block_tables"], dv["seq_lens"], w_layout=layout)
 
     def step():
         proj()
@@ -648,6 +659,12 @@ def run_qkv(args, rank, world, local_rank):
         proj()
         ev[k][1].record()
     clocks.sample()
+    rev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for k in range(K):
+        flush()
+        rev[k][0].record()
+        proj(pkv.PKV_W_ROWS)
+        rev[k][1].record()
     gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     for k in range(K):
         flush()
@@ -664,6 +681,7 @@ def run_qkv(args, rank, world, local_rank):
     del graph
     pkv.pkv_destroy(ctx)
     proj_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev) / K)
+    rows_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in rev) / K)
     step_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in gev) / K)
     # the projection's algorithmic bytes: weights and x read once, q written,
     # k and v rows written; its flops: 2 x tokens x features x hidden
@@ -685,14 +703,17 @@ def run_qkv(args, rank, world, local_rank):
             "config": {"workload": "qkv8b", "description": "llama8b batch (64 tokens) from the layer input: "
                        "QKV projection 4096 -> 6144 on tcgen05 fused with RoPE + append, then decode attention",
                        "l2": "flushed before every step, outside the event window",
-                       "timing": "projection alone: eager events; step: CUDA-graph replay of projection + attention"},
+                       "timing": "projection alone: eager events; step: CUDA-graph replay of projection + attention",
+                       "weights": "packed once into the tiled layout (pkv_qkv_pack_weight) before timing"},
             "step_us": step_ms * 1e3, "projection_us": proj_ms * 1e3,
+            "projection_rows_layout_us": rows_ms * 1e3,
+            "projection_launch": dict(shape, clusters=w.Hq + 2 * w.Hkv),
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
                          "traffic": recorded_traffic("qkv8b"), "kernel": "qkv_rope_append_kernel<128>",
                          "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)", "bytes_per_launch": proj_bytes},
             "projection_tflops": proj_flop / (proj_ms * 1e-3) / 1e12,
             "projection_tflops_frac_of_bf16_peak": proj_flop / (proj_ms * 1e-3) / 1e12 / tflops_peak,
-            "gpu_launches": 4 * K, "clocks": clock_info}
+            "gpu_launches": 5 * K, "clocks": clock_info}
 
 
 def run_loop(args, rank, world, local_rank):

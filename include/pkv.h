@@ -177,12 +177,32 @@ pkv_status pkv_decode_attn_tokens(pkv_ctx* ctx, const void* q, const void* k_poo
  * rotated q, rotated k and raw v go into slot L_b % P of page
  * block_tables[b][L_b / P] (bf16 or E4M3 pools).  hidden must be a multiple
  * of 64 (PKV_ERR_UNSUPPORTED otherwise); x, w_qkv and q_out 16-byte aligned.
- * Range errors as for pkv_rope_append. */
-pkv_status pkv_qkv_rope_append(pkv_ctx* ctx, const void* x, const void* w_qkv, int hidden, void* q_out,
-                               void* k_pool, void* v_pool,
+ * Range errors as for pkv_rope_append.
+ *
+ * w_layout says how w_qkv is stored: PKV_W_ROWS, the row-major
+ * [(Hq + 2 Hkv) d][hidden] above, or PKV_W_TILED, the same values in the
+ * layout pkv_qkv_pack_weight writes, which the kernel reads as one
+ * contiguous 16 KB (d = 128) run per head and 64-element slice of hidden.
+ * Results are bit-identical between the two; the tiled layout is the fast
+ * one (the row-major one reads 128-byte pieces 2 hidden bytes apart). */
+pkv_status pkv_qkv_rope_append(pkv_ctx* ctx, const void* x, const void* w_qkv, int hidden, int w_layout,
+                               void* q_out, void* k_pool, void* v_pool,
                                const float* k_scale, const float* v_scale,
                                const int32_t* block_tables, int bt_stride,
                                const int32_t* seq_lens, int batch, cudaStream_t stream);
+
+/* Layouts of the QKV weight for pkv_qkv_rope_append. */
+enum { PKV_W_ROWS = 0, PKV_W_TILED = 1 };
+
+/* Writes w_qkv [(Hq + 2 Hkv) d][hidden] bf16 (row-major, as for
+ * pkv_qkv_rope_append) into w_tiled in the tiled layout
+ * [Hq + 2 Hkv][hidden / 64][d][64]: element (h, kb, i, j) is row h d + i,
+ * column 64 kb + j of w_qkv.  A load-time step for a static weight; the
+ * output has the input's size, must not overlap it, and both are 16-byte
+ * aligned.  hidden a multiple of 64 (PKV_ERR_UNSUPPORTED otherwise).
+ * Asynchronous on `stream`. */
+pkv_status pkv_qkv_pack_weight(pkv_ctx* ctx, const void* w_qkv, int hidden, void* w_tiled,
+                               cudaStream_t stream);
 
 /* Frees the workspace.  NULL is accepted.  Synchronises the device. */
 pkv_status pkv_destroy(pkv_ctx* ctx);
@@ -208,6 +228,20 @@ pkv_status pkv_set_workers(pkv_ctx* ctx, int workers);
  * claim; ranges under 32 tiles get no tail.  Results do not depend on it
  * beyond rounding. */
 pkv_status pkv_set_tail_chunks(pkv_ctx* ctx, int max_chunks);
+
+/* Sets how many CTAs (one thread-block cluster) share each head's hidden
+ * dimension in pkv_qkv_rope_append: 1 .. 4, or 0 (the default) for the
+ * automatic choice (as many as the SMs hold in one wave).  At most one
+ * 64-element block of hidden per CTA.  Results do not depend on it beyond
+ * the order of the fp32 sums; tests use it to cover every split. */
+pkv_status pkv_set_qkv_split(pkv_ctx* ctx, int split);
+
+/* The launch shape pkv_qkv_rope_append uses for (batch, hidden) under the
+ * current split setting: shape[0] = CTAs per cluster (the split), shape[1] =
+ * TMA ring stages, shape[2] = dynamic shared memory bytes per CTA, shape[3]
+ * = clusters of that shape the GPU holds at once (0 if unknown; the grid has
+ * (Hq + 2 Hkv) x ceil(batch / 128) clusters).  Host-only query. */
+pkv_status pkv_qkv_launch_shape(pkv_ctx* ctx, int batch, int hidden, int* shape);
 
 /* Bytes of device workspace the context holds. */
 size_t pkv_workspace_bytes(const pkv_ctx* ctx);

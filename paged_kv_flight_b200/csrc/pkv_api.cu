@@ -35,7 +35,10 @@ struct pkv_ctx {
     const void* tm_v_ptr;
     CUtensorMap tmk, tmv;
     const void* tm_w_ptr;        // QKV weight and input maps of pkv_qkv_rope_append
-    int tm_w_hidden;
+    int tm_w_hidden, tm_w_layout;
+    int qkv_split;               // 0: automatic
+    int plan_key[6];             // (x_rows, D, heads, tiles, hidden, forced split) of the cached plan
+    pkv::QkvPlan plan;
     const void* tm_x_ptr;
     int tm_x_hidden, tm_x_rows;
     CUtensorMap tmw, tmx;
@@ -132,6 +135,20 @@ bool encode_rows(const void* base, int rows, int cols, int box_rows, CUtensorMap
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The cached projection plan for (batch, hidden) under the context's shapes.
+bool qkv_plan_for(pkv_ctx* ctx, int batch, int hidden)
+{
+    const int x_rows = batch >= 128 ? 128 : (batch + 15) / 16 * 16;
+    const int heads = ctx->cfg.num_q_heads + 2 * ctx->cfg.num_kv_heads, tiles = (batch + 127) / 128;
+    const int key[6] = {x_rows, ctx->cfg.head_dim, heads, tiles, hidden, ctx->qkv_split};
+    if (memcmp(key, ctx->plan_key, sizeof(key)) == 0) return true;
+    if (pkv::qkv_plan(x_rows, ctx->cfg.head_dim, heads, tiles, hidden, ctx->num_sms, ctx->qkv_split,
+                      &ctx->plan) != cudaSuccess)
+        return false;
+    memcpy(ctx->plan_key, key, sizeof(key));
+    return true;
 }
 
 }  // namespace
@@ -365,21 +382,42 @@ pkv_status pkv_decode_attn_tokens(pkv_ctx* ctx, const void* q, const void* k_poo
     return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
-pkv_status pkv_qkv_rope_append(pkv_ctx* ctx, const void* x, const void* w_qkv, int hidden, void* q_out,
-                               void* k_pool, void* v_pool, const float* k_scale, const float* v_scale,
+pkv_status pkv_qkv_pack_weight(pkv_ctx* ctx, const void* w_qkv, int hidden, void* w_tiled, cudaStream_t stream)
+{
+    if (!ctx || !w_qkv || !w_tiled || !aligned16(w_qkv) || !aligned16(w_tiled)) return PKV_ERR_INVALID_ARG;
+    if (hidden < 64 || hidden % 64 != 0) return PKV_ERR_UNSUPPORTED;
+    const int N = (ctx->cfg.num_q_heads + 2 * ctx->cfg.num_kv_heads) * ctx->cfg.head_dim;
+    const size_t bytes = (size_t)N * hidden * 2;
+    const uintptr_t a = reinterpret_cast<uintptr_t>(w_qkv), b = reinterpret_cast<uintptr_t>(w_tiled);
+    if (a < b + bytes && b < a + bytes) return PKV_ERR_INVALID_ARG;
+    return pkv::launch_qkv_pack_weight(static_cast<const __nv_bfloat16*>(w_qkv), static_cast<__nv_bfloat16*>(w_tiled),
+                                       N, hidden, ctx->cfg.head_dim, stream) == cudaSuccess
+               ? PKV_OK
+               : PKV_ERR_CUDA;
+}
+
+pkv_status pkv_qkv_rope_append(pkv_ctx* ctx, const void* x, const void* w_qkv, int hidden, int w_layout,
+                               void* q_out, void* k_pool, void* v_pool, const float* k_scale, const float* v_scale,
                                const int32_t* block_tables, int bt_stride, const int32_t* seq_lens, int batch,
                                cudaStream_t stream)
 {
     pkv_status st = check_call(ctx, batch, bt_stride, k_pool, v_pool, k_scale, v_scale, block_tables, seq_lens);
     if (st != PKV_OK || batch == 0) return st;
+    if (w_layout != PKV_W_ROWS && w_layout != PKV_W_TILED) return PKV_ERR_INVALID_ARG;
     if (hidden < 64 || hidden % 64 != 0) return PKV_ERR_UNSUPPORTED;
     if (!x || !w_qkv || !q_out || !aligned16(x) || !aligned16(w_qkv) || !aligned16(q_out))
         return PKV_ERR_INVALID_ARG;
     const int N = (ctx->cfg.num_q_heads + 2 * ctx->cfg.num_kv_heads) * ctx->cfg.head_dim;
-    if (ctx->tm_w_ptr != w_qkv || ctx->tm_w_hidden != hidden) {
-        if (!encode_rows(w_qkv, N, hidden, 16, &ctx->tmw)) return PKV_ERR_CUDA;
+    if (ctx->tm_w_ptr != w_qkv || ctx->tm_w_hidden != hidden || ctx->tm_w_layout != w_layout) {
+        // tiled: a 2-D view of 64-element rows, one box = the d rows of one
+        // (head, 64-slice) run
+        const bool ok = w_layout == PKV_W_TILED
+                            ? encode_rows(w_qkv, N * (hidden / 64), 64, ctx->cfg.head_dim, &ctx->tmw)
+                            : encode_rows(w_qkv, N, hidden, ctx->cfg.head_dim, &ctx->tmw);
+        if (!ok) return PKV_ERR_CUDA;
         ctx->tm_w_ptr = w_qkv;
         ctx->tm_w_hidden = hidden;
+        ctx->tm_w_layout = w_layout;
     }
     const int x_rows = batch >= 128 ? 128 : (batch + 15) / 16 * 16;
     if (ctx->tm_x_ptr != x || ctx->tm_x_hidden != hidden || ctx->tm_x_rows != batch) {
@@ -408,7 +446,10 @@ pkv_status pkv_qkv_rope_append(pkv_ctx* ctx, const void* x, const void* w_qkv, i
     p.num_pages = ctx->cfg.num_pages;
     p.fp8 = ctx->cfg.kv_dtype == PKV_KV_FP8_E4M3;
     p.x_rows = x_rows;
-    return pkv::launch_qkv_rope_append(p, ctx->tmx, ctx->tmw, stream) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+    p.w_tiled = w_layout == PKV_W_TILED;
+    if (!qkv_plan_for(ctx, batch, hidden)) return PKV_ERR_CUDA;
+    return pkv::launch_qkv_rope_append(p, ctx->plan, ctx->tmx, ctx->tmw, stream) == cudaSuccess ? PKV_OK
+                                                                                                : PKV_ERR_CUDA;
 }
 
 pkv_status pkv_destroy(pkv_ctx* ctx)
@@ -452,6 +493,25 @@ pkv_status pkv_set_workers(pkv_ctx* ctx, int workers)
 {
     if (!ctx || workers < 0) return PKV_ERR_INVALID_ARG;
     ctx->workers = workers;
+    return PKV_OK;
+}
+
+pkv_status pkv_qkv_launch_shape(pkv_ctx* ctx, int batch, int hidden, int* shape)
+{
+    if (!ctx || !shape || batch <= 0 || batch > ctx->cfg.max_batch) return PKV_ERR_INVALID_ARG;
+    if (hidden < 64 || hidden % 64 != 0) return PKV_ERR_UNSUPPORTED;
+    if (!qkv_plan_for(ctx, batch, hidden)) return PKV_ERR_CUDA;
+    shape[0] = ctx->plan.split;
+    shape[1] = ctx->plan.stages;
+    shape[2] = (int)ctx->plan.smem;
+    shape[3] = ctx->plan.max_clusters;
+    return PKV_OK;
+}
+
+pkv_status pkv_set_qkv_split(pkv_ctx* ctx, int split)
+{
+    if (!ctx || split < 0 || split > pkv::kQkvMaxSplit) return PKV_ERR_INVALID_ARG;
+    ctx->qkv_split = split;
     return PKV_OK;
 }
 

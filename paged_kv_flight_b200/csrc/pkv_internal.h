@@ -108,6 +108,8 @@ cudaError_t launch_decode_attn_tokens(const AttnParams& p, const CUtensorMap& tm
 
 // QKV projection of the new tokens on tcgen05, fused with RoPE and the append
 // (qkv_rope_append.cu).
+constexpr int kQkvMaxSplit = 4;   // CTAs (one cluster) that share a head's hidden dimension
+
 struct QkvParams {
     const int32_t* seq_lens;
     const int32_t* block_tables;
@@ -120,10 +122,26 @@ struct QkvParams {
     double rope_base;
     int batch, hidden, bt_stride, Hq, Hkv, D, P, num_pages, fp8;
     int x_rows;               // token rows per x TMA box: min(128, batch rounded up to 16)
+    int w_tiled;              // 1: weights in the tiled layout of pkv_qkv_pack_weight
+    int split;                // hidden-dimension split = cluster size (set from the plan)
+    int stages;               // ring depth (set from the plan)
+    int ring_bytes;           // ring area; the rotation table follows it (set from the plan)
 };
-size_t qkv_smem_bytes();
+
+// Launch shape of the projection for one (x_rows, D, heads, token tiles,
+// hidden): the split, the ring and the shared memory.
+struct QkvPlan {
+    int split, stages, ring_bytes;
+    size_t smem;
+    int max_clusters;         // clusters of this shape the GPU holds at once (0: unknown)
+};
 cudaError_t qkv_prepare();
-cudaError_t launch_qkv_rope_append(const QkvParams& p, const CUtensorMap& tmx, const CUtensorMap& tmw,
+cudaError_t qkv_plan(int x_rows, int D, int heads, int tiles, int hidden, int num_sms, int forced_split,
+                     QkvPlan* out);
+cudaError_t launch_qkv_rope_append(const QkvParams& p, const QkvPlan& plan, const CUtensorMap& tmx,
+                                   const CUtensorMap& tmw, cudaStream_t stream);
+// Copies w [N][hidden] into the tiled layout [N / D][hidden / 64][D][64].
+cudaError_t launch_qkv_pack_weight(const __nv_bfloat16* w, __nv_bfloat16* out, int N, int hidden, int D,
                                    cudaStream_t stream);
 
 // The split combine (combine.cu), run after either attention kernel: sets its

@@ -44,7 +44,8 @@ EXPORTS = ("pkv_create", "pkv_rope_append", "pkv_decode_attn", "pkv_destroy", "p
            "pkv_set_tail_chunks", "pkv_rope_append_tokens", "pkv_decode_attn_tokens",
            "pkv_pages_create", "pkv_pages_destroy", "pkv_pages_admit", "pkv_pages_reserve", "pkv_pages_advance",
            "pkv_pages_release", "pkv_pages_block_table", "pkv_pages_seq_lens", "pkv_pages_active",
-           "pkv_pages_refcount", "pkv_pages_free_count", "pkv_pages_take_changes", "pkv_qkv_rope_append")
+           "pkv_pages_refcount", "pkv_pages_free_count", "pkv_pages_take_changes", "pkv_qkv_rope_append",
+           "pkv_qkv_pack_weight", "pkv_set_qkv_split", "pkv_qkv_launch_shape")
 
 
 class pkv_config(C.Structure):
@@ -88,8 +89,15 @@ lib.pkv_pages_free_count.argtypes = [_V]
 lib.pkv_pages_free_count.restype = C.c_int
 lib.pkv_pages_take_changes.argtypes = [_V, _V, C.c_int]
 lib.pkv_pages_take_changes.restype = C.c_int
-lib.pkv_qkv_rope_append.argtypes = [_V, _V, _V, C.c_int, _V, _V, _V, _V, _V, _V, C.c_int, _V, C.c_int, _V]
+lib.pkv_qkv_rope_append.argtypes = [_V, _V, _V, C.c_int, C.c_int, _V, _V, _V, _V, _V, _V, C.c_int, _V, C.c_int,
+                                    _V]
 lib.pkv_qkv_rope_append.restype = C.c_int
+lib.pkv_qkv_pack_weight.argtypes = [_V, _V, C.c_int, _V, _V]
+lib.pkv_qkv_pack_weight.restype = C.c_int
+lib.pkv_set_qkv_split.argtypes = [_V, C.c_int]
+lib.pkv_set_qkv_split.restype = C.c_int
+lib.pkv_qkv_launch_shape.argtypes = [_V, C.c_int, C.c_int, _V]
+lib.pkv_qkv_launch_shape.restype = C.c_int
 lib.pkv_set_tail_chunks.argtypes = [_V, C.c_int]
 lib.pkv_set_tail_chunks.restype = C.c_int
 lib.pkv_workspace_bytes.argtypes = [_V]
@@ -304,16 +312,40 @@ class Pages:
             pass
 
 
+PKV_W_ROWS, PKV_W_TILED = 0, 1
+
+
+def pkv_set_qkv_split(ctx, split: int, check: bool = True) -> int:
+    """CTAs (a cluster) per head over the hidden dimension: 1 .. 4, 0 = automatic."""
+    return _done(lib.pkv_set_qkv_split(ctx, int(split)), "pkv_set_qkv_split", check)
+
+
+def pkv_qkv_launch_shape(ctx, batch: int, hidden: int) -> dict:
+    """The projection's launch shape: split (CTAs per cluster), ring stages,
+    shared memory bytes per CTA, clusters the GPU holds at once."""
+    out = (C.c_int * 4)()
+    _done(lib.pkv_qkv_launch_shape(ctx, int(batch), int(hidden), out), "pkv_qkv_launch_shape", True)
+    return {"split": out[0], "stages": out[1], "smem_bytes": out[2], "max_clusters": out[3]}
+
+
+def pkv_qkv_pack_weight(ctx, w_qkv, w_tiled, stream=None, check: bool = True) -> int:
+    """w_qkv [(Hq + 2 Hkv) d, hidden] -> w_tiled (same size) in the tiled layout."""
+    st = lib.pkv_qkv_pack_weight(ctx, _ptr(w_qkv), int(w_qkv.shape[-1]), _ptr(w_tiled), _stream(stream))
+    return _done(st, "pkv_qkv_pack_weight", check)
+
+
 def pkv_qkv_rope_append(ctx, x, w_qkv, q_out, k_pool, v_pool, k_scale, v_scale, block_tables, seq_lens,
                         batch: int | None = None, bt_stride: int | None = None, stream=None,
-                        check: bool = True) -> int:
-    """x [batch, hidden], w_qkv [(Hq + 2 Hkv) d, hidden], q_out [batch, Hq, d]."""
+                        check: bool = True, w_layout: int = PKV_W_ROWS) -> int:
+    """x [batch, hidden], w_qkv [(Hq + 2 Hkv) d, hidden] (PKV_W_ROWS) or as
+    pkv_qkv_pack_weight wrote it (PKV_W_TILED), q_out [batch, Hq, d]."""
     if batch is None:
         batch = int(seq_lens.shape[0])
     if bt_stride is None:
         bt_stride = int(block_tables.shape[1])
     hidden = int(x.shape[-1])
-    st = lib.pkv_qkv_rope_append(ctx, _ptr(x), _ptr(w_qkv), hidden, _ptr(q_out), _ptr(k_pool), _ptr(v_pool),
+    st = lib.pkv_qkv_rope_append(ctx, _ptr(x), _ptr(w_qkv), hidden, int(w_layout), _ptr(q_out), _ptr(k_pool),
+                                 _ptr(v_pool),
                                  _ptr(k_scale), _ptr(v_scale), _ptr(block_tables), int(bt_stride), _ptr(seq_lens),
                                  int(batch), _stream(stream))
     return _done(st, "pkv_qkv_rope_append", check)

@@ -12,7 +12,10 @@ another bf16 value; the rotation mixes the two members of a pair.  The bar:
 every element within 3 bf16 ulps of the larger magnitude of its rotation
 pair plus K 2^-23 S of the pair's features; at least 97% of the elements
 bit-identical; E4M3 codes within one step; every pool byte outside the
-landing slots untouched."""
+landing slots untouched.  The same projection from the tiled weight layout
+(pkv_qkv_pack_weight) must give the same bytes as from the row-major one, and
+every split of the hidden dimension over a cluster (1 .. 4 CTAs, reduced
+through distributed shared memory) must meet the same bar."""
 import numpy as np
 import pytest
 import torch
@@ -53,16 +56,31 @@ def test_fused_projection_matches_oracle(pkv, case):
     x = torch.randn(B, hidden, generator=gen).to(torch.bfloat16)
     wq = (torch.randn(N, hidden, generator=gen) / hidden ** 0.5).to(torch.bfloat16)
 
-    dv = _gpu.to_device(w)
     xd, wd = x.cuda(), wq.cuda()
-    q_out = torch.empty(B, Hq, d, dtype=torch.bfloat16, device="cuda")
+    wt = torch.empty_like(wd)
+    # (split, layout) runs: automatic split from both layouts, then every split
+    runs = [(0, pkv.PKV_W_ROWS), (0, pkv.PKV_W_TILED)] + [(sp, pkv.PKV_W_TILED) for sp in (1, 2, 3, 4)]
+    results = []
     ctx = _gpu.make_ctx(pkv, w)
     try:
-        pkv.pkv_qkv_rope_append(ctx, xd, wd, q_out, dv["k_pool"], dv["v_pool"], dv["k_scale"], dv["v_scale"],
-                                dv["block_tables"], dv["seq_lens"])
-        assert pkv.pkv_check_device_error(ctx)[0] == pkv.PKV_OK
+        pkv.pkv_qkv_pack_weight(ctx, wd, wt)
+        for sp, layout in runs:
+            dv = _gpu.to_device(w)
+            q_out = torch.empty(B, Hq, d, dtype=torch.bfloat16, device="cuda")
+            pkv.pkv_set_qkv_split(ctx, sp)
+            pkv.pkv_qkv_rope_append(ctx, xd, wt if layout == pkv.PKV_W_TILED else wd, q_out, dv["k_pool"],
+                                    dv["v_pool"], dv["k_scale"], dv["v_scale"], dv["block_tables"], dv["seq_lens"],
+                                    w_layout=layout)
+            assert pkv.pkv_check_device_error(ctx)[0] == pkv.PKV_OK
+            results.append((sp, layout, q_out.cpu(), dv["k_pool"].cpu(), dv["v_pool"].cpu()))
     finally:
         pkv.pkv_destroy(ctx)
+    # the tiled layout holds the same values in another order (a permutation,
+    # checked byte for byte), and the kernel's sums run in the same order
+    perm = wq.view(Hq + 2 * Hkv, d, hidden // 64, 64).permute(0, 2, 1, 3).contiguous()
+    assert torch.equal(wt.cpu().view(torch.int16), perm.reshape(N, hidden).view(torch.int16))
+    for a, b in zip(results[0][2:], results[1][2:]):
+        assert torch.equal(a.view(torch.uint8), b.view(torch.uint8))
 
     # oracle: fp64 projection -> bf16, then the oracle's RoPE + append
     y = oracle.project_bf16(bits16(x), bits16(wq))
@@ -89,25 +107,26 @@ def test_fused_projection_matches_oracle(pkv, case):
     acc_q = acc[:, :Hq * d].reshape(B, Hq, d)
     acc_k = acc[:, Hq * d:(Hq + Hkv) * d].reshape(B, Hkv, d)
     acc_v = acc[:, (Hq + Hkv) * d:].reshape(B, Hkv, d)
-    gq = bits16(q_out)
-    assert close_pairs(gq, h["q"], acc_q)
-    same = [np.mean(gq == h["q"])]
     landing = {(int(w.block_tables[b, L // P]), kvh, int(L % P)) for b, L in enumerate(w.seq_lens)
                for kvh in range(Hkv)}
+    order = sorted((int(w.block_tables[b, L // P]), kvh, int(L % P), b) for b, L in enumerate(w.seq_lens)
+                   for kvh in range(Hkv))
     conv = bytes8 if fp8 else bits16
-    for key in ("k_pool", "v_pool"):
-        got, ref = conv(dv[key]), h[key]
-        diff = got != ref
-        rows = {tuple(map(int, r[:3])) for r in np.argwhere(diff)}
-        assert rows <= landing, f"{key}: bytes changed outside the landing slots"
-        order = sorted((int(w.block_tables[b, L // P]), kvh, int(L % P), b) for b, L in enumerate(w.seq_lens)
-                       for kvh in range(Hkv))
-        gl = np.stack([got[pg, kvh, sl] for pg, kvh, sl, _ in order])
-        rl = np.stack([ref[pg, kvh, sl] for pg, kvh, sl, _ in order])
-        ae = np.stack([(acc_k if key == "k_pool" else acc_v)[b, kvh] for _, kvh, _, b in order])
-        if fp8:
-            assert np.abs(gl.astype(int) - rl.astype(int)).max() <= 1      # one E4M3 code step
-        else:
-            assert close_pairs(gl, rl, ae, ulps=3 if key == "k_pool" else 1)
-        same.append(np.mean(gl == rl))
-    assert min(same) >= 0.97, same
+    for sp, layout, q_out, k_pool, v_pool in results:
+        gq = bits16(q_out)
+        assert close_pairs(gq, h["q"], acc_q), (sp, layout)
+        same = [np.mean(gq == h["q"])]
+        for key, pool in (("k_pool", k_pool), ("v_pool", v_pool)):
+            got, ref = conv(pool), h[key]
+            diff = got != ref
+            rows = {tuple(map(int, r[:3])) for r in np.argwhere(diff)}
+            assert rows <= landing, f"{key}: bytes changed outside the landing slots (split {sp})"
+            gl = np.stack([got[pg, kvh, sl] for pg, kvh, sl, _ in order])
+            rl = np.stack([ref[pg, kvh, sl] for pg, kvh, sl, _ in order])
+            ae = np.stack([(acc_k if key == "k_pool" else acc_v)[b, kvh] for _, kvh, _, b in order])
+            if fp8:
+                assert np.abs(gl.astype(int) - rl.astype(int)).max() <= 1      # one E4M3 code step
+            else:
+                assert close_pairs(gl, rl, ae, ulps=3 if key == "k_pool" else 1), (sp, key)
+            same.append(np.mean(gl == rl))
+        assert min(same) >= 0.97, (sp, layout, same)
