@@ -47,14 +47,32 @@ def _f(bits):
     return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
+def pair_max(a):
+    half = a.shape[-1] // 2
+    m = np.maximum(a[..., :half], a[..., half:])
+    return np.concatenate([m, m], axis=-1)
+
+
+def close_pairs(got_bits, ref_bits, acc_err, ulps=3):
+    """|got - ref| <= ulps 2^-8 max(|ref_i|, |ref_{i+d/2}|) + the pair's accumulation bound."""
+    g, r = _f(got_bits), _f(ref_bits)
+    tol = ulps * 2.0 ** -8 * np.maximum(pair_max(np.abs(r)), 2.0 ** -20) + pair_max(acc_err)
+    return bool((np.abs(g - r) <= tol).all())
+
+
+def _inputs(B, N, hidden, seed=5):
+    gen = torch.Generator().manual_seed(seed)
+    x = torch.randn(B, hidden, generator=gen).to(torch.bfloat16)
+    wq = (torch.randn(N, hidden, generator=gen) / hidden ** 0.5).to(torch.bfloat16)
+    return x, wq
+
+
 @pytest.mark.parametrize("case", CASES, ids=lambda c: c[0])
 def test_fused_projection_matches_oracle(pkv, case):
     name, Hq, Hkv, d, P, hidden, lengths, fp8 = case
     w = workloads.build(name, Hq, Hkv, d, P, fp8, 5e5 if d == 128 else 1e4, lengths, 17, device="cpu")
     B, N = w.batch, (Hq + 2 * Hkv) * d
-    gen = torch.Generator().manual_seed(5)
-    x = torch.randn(B, hidden, generator=gen).to(torch.bfloat16)
-    wq = (torch.randn(N, hidden, generator=gen) / hidden ** 0.5).to(torch.bfloat16)
+    x, wq = _inputs(B, N, hidden)
 
     xd, wd = x.cuda(), wq.cuda()
     wt = torch.empty_like(wd)
@@ -93,17 +111,6 @@ def test_fused_projection_matches_oracle(pkv, case):
     assert oracle.rope_append(oracle_cfg(w), h["q"], h["k_new"], h["v_new"], h["k_pool"], h["v_pool"],
                               h["k_scale"], h["v_scale"], h["block_tables"], h["seq_lens"]) == 0
 
-    def pair_max(a):
-        half = d // 2
-        m = np.maximum(a[..., :half], a[..., half:])
-        return np.concatenate([m, m], axis=-1)
-
-    def close_pairs(got_bits, ref_bits, acc_err, ulps=3):
-        """|got - ref| <= ulps 2^-8 max(|ref_i|, |ref_{i+d/2}|) + the pair's accumulation bound."""
-        g, r = _f(got_bits), _f(ref_bits)
-        tol = ulps * 2.0 ** -8 * np.maximum(pair_max(np.abs(r)), 2.0 ** -20) + pair_max(acc_err)
-        return bool((np.abs(g - r) <= tol).all())
-
     acc_q = acc[:, :Hq * d].reshape(B, Hq, d)
     acc_k = acc[:, Hq * d:(Hq + Hkv) * d].reshape(B, Hkv, d)
     acc_v = acc[:, (Hq + Hkv) * d:].reshape(B, Hkv, d)
@@ -130,3 +137,93 @@ def test_fused_projection_matches_oracle(pkv, case):
                 assert close_pairs(gl, rl, ae, ulps=3 if key == "k_pool" else 1), (sp, key)
             same.append(np.mean(gl == rl))
         assert min(same) >= 0.97, (sp, layout, same)
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_device_range_errors_skip_the_token(pkv, fp8):
+    """A length past the block table (error bit 1) and an out-of-range landing
+    page id (bit 2) are the kernel's own checks: the token with the bad length
+    stores nothing, the one with the bad page stores its q but no k / v, every
+    other token is stored as the oracle says, and the context keeps working."""
+    Hq, Hkv, d, P, hidden = 8, 2, 128, 16, 512
+    lengths = [0, 5, 17, 40, 100, 63]
+    w = workloads.build("qkv_err", Hq, Hkv, d, P, fp8, 5e5, lengths, 23, device="cpu")
+    B, N = w.batch, (Hq + 2 * Hkv) * d
+    x, wq = _inputs(B, N, hidden, seed=9)
+    bad_len, bad_page = 1, 3
+    lp = lengths[bad_page] // P
+    y = oracle.project_bf16(bits16(x), bits16(wq))
+    acc = hidden * 2.0 ** -23 * (np.abs(x.double().numpy()) @ np.abs(wq.double().numpy()).T)
+    h = host_inputs(w)
+    pool0 = {key: h[key].copy() for key in ("k_pool", "v_pool")}
+    h["q"] = np.ascontiguousarray(y[:, :Hq * d].reshape(B, Hq, d))
+    h["k_new"] = np.ascontiguousarray(y[:, Hq * d:(Hq + Hkv) * d].reshape(B, Hkv, d))
+    h["v_new"] = np.ascontiguousarray(y[:, (Hq + Hkv) * d:].reshape(B, Hkv, d))
+    assert oracle.rope_append(oracle_cfg(w), h["q"], h["k_new"], h["v_new"], h["k_pool"], h["v_pool"],
+                              h["k_scale"], h["v_scale"], h["block_tables"], h["seq_lens"]) == 0
+    good = [b for b in range(B) if b not in (bad_len, bad_page)]
+    conv = bytes8 if fp8 else bits16
+    sentinel = torch.full((B, Hq, d), 7.0, dtype=torch.bfloat16)
+    ctx = _gpu.make_ctx(pkv, w)
+    try:
+        for sp in (0, 1, 3):
+            dv = _gpu.to_device(w)
+            dv["seq_lens"][bad_len] = w.bt_stride * P
+            dv["block_tables"][bad_page, lp] = w.num_pages + 5
+            q_out = sentinel.cuda()
+            pkv.pkv_set_qkv_split(ctx, sp)
+            pkv.pkv_qkv_rope_append(ctx, x.cuda(), wq.cuda(), q_out, dv["k_pool"], dv["v_pool"], dv["k_scale"],
+                                    dv["v_scale"], dv["block_tables"], dv["seq_lens"])
+            st, bits = pkv.pkv_check_device_error(ctx)
+            assert st == pkv.PKV_ERR_DEVICE_BOUNDS and bits & 1 and bits & 2, (sp, st, bits)
+            gq = bits16(q_out)
+            assert (gq[bad_len] == bits16(sentinel)[bad_len]).all(), sp        # nothing stored
+            ok_q = [b for b in range(B) if b != bad_len]
+            assert close_pairs(gq[ok_q], h["q"][ok_q], acc[ok_q, :Hq * d].reshape(len(ok_q), Hq, d)), sp
+            for key in ("k_pool", "v_pool"):
+                got, ref, base = conv(dv[key].cpu()), h[key], pool0[key]
+                slots = {(int(w.block_tables[b, lengths[b] // P]), kvh, lengths[b] % P) for b in good
+                         for kvh in range(Hkv)}
+                for idx in map(tuple, np.argwhere((got != base).any(axis=-1))):
+                    assert idx in slots, (sp, key, idx)                      # only good tokens' slots
+                for b in good:
+                    pg = int(w.block_tables[b, lengths[b] // P])
+                    off = Hq * d if key == "k_pool" else (Hq + Hkv) * d
+                    for kvh in range(Hkv):
+                        g_, r_ = got[pg, kvh, lengths[b] % P], ref[pg, kvh, lengths[b] % P]
+                        if fp8:
+                            assert np.abs(g_.astype(int) - r_.astype(int)).max() <= 1
+                        else:
+                            a_ = acc[b, off + kvh * d: off + (kvh + 1) * d]
+                            assert close_pairs(g_[None], r_[None], a_[None]), (sp, key, b)
+        # the context still works afterwards
+        dv = _gpu.to_device(w)
+        pkv.pkv_set_qkv_split(ctx, 0)
+        q_out = torch.empty(B, Hq, d, dtype=torch.bfloat16, device="cuda")
+        pkv.pkv_qkv_rope_append(ctx, x.cuda(), wq.cuda(), q_out, dv["k_pool"], dv["v_pool"], dv["k_scale"],
+                                dv["v_scale"], dv["block_tables"], dv["seq_lens"])
+        assert pkv.pkv_check_device_error(ctx)[0] == pkv.PKV_OK
+        assert close_pairs(bits16(q_out), h["q"], acc[:, :Hq * d].reshape(B, Hq, d))
+    finally:
+        pkv.pkv_destroy(ctx)
+
+
+def test_host_side_rejections(pkv):
+    w = workloads.build("qkv_rej", 8, 2, 128, 16, False, 5e5, [3, 9], 3, device="cpu")
+    dv = _gpu.to_device(w)
+    x = torch.zeros(w.batch, 256, dtype=torch.bfloat16, device="cuda")
+    wq = torch.zeros(12 * 128, 256, dtype=torch.bfloat16, device="cuda")
+    q_out = torch.empty(w.batch, 8, 128, dtype=torch.bfloat16, device="cuda")
+    ctx = _gpu.make_ctx(pkv, w)
+    try:
+        args = (dv["k_pool"], dv["v_pool"], None, None, dv["block_tables"], dv["seq_lens"])
+        x96 = torch.zeros(w.batch, 96, dtype=torch.bfloat16, device="cuda")   # hidden not a multiple of 64
+        assert pkv.pkv_qkv_rope_append(ctx, x96, wq, q_out, *args, check=False) == pkv.PKV_ERR_UNSUPPORTED
+        assert pkv.pkv_qkv_rope_append(ctx, x, wq, q_out, *args, check=False, w_layout=2) == pkv.PKV_ERR_INVALID_ARG
+        assert pkv.pkv_set_qkv_split(ctx, 5, check=False) == pkv.PKV_ERR_INVALID_ARG
+        assert pkv.pkv_qkv_pack_weight(ctx, wq, wq, check=False) == pkv.PKV_ERR_INVALID_ARG      # overlap
+        shape = pkv.pkv_qkv_launch_shape(ctx, w.batch, 256)
+        assert 1 <= shape["split"] <= 4 and shape["stages"] >= 2 and shape["smem_bytes"] > 0
+    finally:
+        pkv.pkv_destroy(ctx)
+
