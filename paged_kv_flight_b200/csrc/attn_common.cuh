@@ -15,24 +15,26 @@ using namespace dev;
 constexpr uint64_t kWaitLimitNs = 500ull * 1000ull * 1000ull;  // 0.5 s per wait
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
-template <int D, bool FP8>
+// Tile geometry: TT tokens per tile (16, or 32 for E4M3 pools with pages of
+// at least 32 tokens), one TMA box of TT rows per 128 (or 64) bytes of row.
+template <int D, bool FP8, int TT = kTile>
 struct Geo {
     static constexpr int ELEM = FP8 ? 1 : 2;
     static constexpr int ROWB = D * ELEM;                  // bytes per token row
     static constexpr int BOXB = ROWB > 128 ? 128 : ROWB;   // bytes per TMA box row
     static constexpr int NBOX = ROWB / BOXB;               // boxes per tile per tensor
     static constexpr int CPB = BOXB / 16;                  // 16-byte chunks per box row
-    static constexpr int BOX_BYTES = kTile * BOXB;
-    static constexpr int TILEB = kTile * ROWB;             // one K (or V) tile
+    static constexpr int BOX_BYTES = TT * BOXB;
+    static constexpr int TILEB = TT * ROWB;                // one K (or V) tile
     static constexpr int STAGEB = 2 * TILEB;               // K + V
 };
 
 // Byte offset inside a tile of 16-byte chunk `ch` (counted along the token
 // row) of tile row `row`, as the TMA swizzle placed it.
-template <int D, bool FP8>
+template <int D, bool FP8, int TT = kTile>
 __device__ __forceinline__ uint32_t tile_off(int row, int ch)
 {
-    using Gm = Geo<D, FP8>;
+    using Gm = Geo<D, FP8, TT>;
     const int box = ch / Gm::CPB, cib = ch % Gm::CPB;
     const int x = (Gm::BOXB == 128) ? (row & 7) : ((row >> 1) & 3);
     return (uint32_t)(box * Gm::BOX_BYTES + row * Gm::BOXB + ((cib ^ x) << 4));
@@ -132,15 +134,15 @@ __device__ __forceinline__ void locate(const int* prefix, int B, int Hkv, long l
     }
 }
 
-// Page ids (as TMA row coordinates) and scales of 32 consecutive tiles, one
-// per lane.
+// Page ids (as TMA row coordinates) and scales of 32 consecutive tiles of
+// TT tokens (TT <= P, so a tile never crosses a page), one per lane.
 struct Lookahead {
     int valid;   // 0: past the range, 1: ok, 2: page id out of range
     int row;
     float ks, vs;
 };
 
-template <bool FP8>
+template <bool FP8, int TT = kTile>
 __device__ __forceinline__ Lookahead lookahead_fill(const AttnParams& p, const int* prefix, long long x0,
                                                     long long t_end, int lane)
 {
@@ -151,7 +153,7 @@ __device__ __forceinline__ Lookahead lookahead_fill(const AttnParams& p, const i
         const int ntb = prefix[b + 1] - prefix[b];
         const long long r = y - (long long)prefix[b] * p.Hkv;
         const int kvh = (int)(r / ntb), tt = (int)(r % ntb);
-        const int tok0 = tt * kTile;
+        const int tok0 = tt * TT;
         const int lp = tok0 / p.P;
         const int page = __ldg(&p.block_tables[(size_t)b * p.bt_stride + lp]);
         if ((unsigned)page < (unsigned)p.num_pages) {

@@ -78,12 +78,12 @@ __device__ __forceinline__ void load_q(const AttnParams& p, int b, int kvh, int 
     }
 }
 
-template <int D, bool FP8, int WARPS>
+template <int D, bool FP8, int WARPS, int TT>
 __global__ void __launch_bounds__(WARPS * 32, 1)
 decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                    const AttnParams p)
 {
-    using Gm = Geo<D, FP8>;
+    using Gm = Geo<D, FP8, TT>;
     constexpr int KSTEPS = D / 16;      // mma k-steps along d for QK^T
     constexpr int NTD = D / 8;          // mma n-tiles along d for P V
     constexpr int NT = WARPS * 32;
@@ -117,7 +117,7 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
     for (int b = lo; b < hi; ++b) {
         const int L = p.seq_lens[b];
         const bool ok = L >= 0 && (long long)L < cap;
-        const int nt = ok ? (L + kTile) / kTile : 0;   // ceil((L + 1) / 16)
+        const int nt = ok ? (L + TT) / TT : 0;   // ceil((L + 1) / TT)
         if (!ok) s_bad = 1;
         prefix[b] = nt;
         local += nt;
@@ -197,8 +197,8 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
     int p_left = (int)(pu1 - pu0);   // a head holds at most T / W + 1 tiles
     int la_i = 0;
     long long la_fill = pu0 + 64;
-    Lookahead la_cur = lookahead_fill<FP8>(p, prefix, pu0, pu1, lane);
-    Lookahead la_nxt = lookahead_fill<FP8>(p, prefix, pu0 + 32, pu1, lane);
+    Lookahead la_cur = lookahead_fill<FP8, TT>(p, prefix, pu0, pu1, lane);
+    Lookahead la_nxt = lookahead_fill<FP8, TT>(p, prefix, pu0 + 32, pu1, lane);
     int nU = sp.K > 0 ? kPending : kNone;
     long long nu0 = 0, nu1 = 0;
     Lookahead la_new{0, 0, 1.f, 1.f};
@@ -216,14 +216,14 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
             p_left = (int)(nu1 - nu0);
             la_i = 0;
             la_cur = la_new;
-            la_nxt = lookahead_fill<FP8>(p, prefix, nu0 + 32, nu1, lane);
+            la_nxt = lookahead_fill<FP8, TT>(p, prefix, nu0 + 32, nu1, lane);
             la_fill = nu0 + 64;
             nU = kPending;
         }
         if (la_i == 32) {
             la_i = 0;
             la_cur = la_nxt;
-            la_nxt = lookahead_fill<FP8>(p, prefix, la_fill, pu1, lane);
+            la_nxt = lookahead_fill<FP8, TT>(p, prefix, la_fill, pu1, lane);
             la_fill += 32;
         }
         const int src = la_i++;
@@ -272,7 +272,7 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
                     nU = v2 * (sp.K + 1) + 1 + (c - v2) / W;
                     nu0 = sp.ustart(nU);
                     nu1 = sp.ustart(nU + 1);
-                    la_new = lookahead_fill<FP8>(p, prefix, nu0, nu1, lane);
+                    la_new = lookahead_fill<FP8, TT>(p, prefix, nu0, nu1, lane);
                 }
             }
         }
@@ -371,29 +371,32 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
         if (si.valid) {
             const uint32_t kb = my_stage0 + (uint32_t)(s * Gm::STAGEB);
             const uint32_t vb = kb + Gm::TILEB;
-            const int tok0 = ctt * kTile;
-            const int rows_valid = min(kTile, n_cur - tok0);
-            if (rows_valid < kTile) {
+            const int tok0 = ctt * TT;
+            const int rows_valid = min(TT, n_cur - tok0);
+            if (rows_valid < TT) {
                 // slots past the request's end may hold anything (NaN): zero them in V
                 constexpr int CPR = Gm::ROWB / 16;
-                const int nch = (kTile - rows_valid) * CPR;
+                const int nch = (TT - rows_valid) * CPR;
                 for (int e = lane; e < nch; e += 32) {
                     const int r = rows_valid + e / CPR, ch = e % CPR;
-                    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(vb + tile_off<D, FP8>(r, ch)),
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(vb + tile_off<D, FP8, TT>(r, ch)),
                                  "r"(0u)
                                  : "memory");
                 }
                 zeroed = true;
                 __syncwarp();
             }
-            // S = Q K^T (two n-tiles of 8 tokens), two accumulation chains
-            float sa[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, sb[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+            // S = Q K^T (NJ n-tiles of 8 tokens), two accumulation chains
+            constexpr int NJ = TT / 8;
+            float sa[NJ][2], sb[NJ][2];
+#pragma unroll
+            for (int j = 0; j < NJ; ++j) sa[j][0] = sa[j][1] = sb[j][0] = sb[j][1] = 0.f;
             if constexpr (!FP8) {
 #pragma unroll
                 for (int ks = 0; ks < KSTEPS; ks += 2) {
                     uint32_t r0, r1, r2, r3, r4, r5, r6, r7;
-                    ldsm_x4(kb + tile_off<D, FP8>(tokK, 2 * ks + (mi & 1)), r0, r1, r2, r3);
-                    ldsm_x4(kb + tile_off<D, FP8>(tokK, 2 * ks + 2 + (mi & 1)), r4, r5, r6, r7);
+                    ldsm_x4(kb + tile_off<D, FP8, TT>(tokK, 2 * ks + (mi & 1)), r0, r1, r2, r3);
+                    ldsm_x4(kb + tile_off<D, FP8, TT>(tokK, 2 * ks + 2 + (mi & 1)), r4, r5, r6, r7);
                     mma_bf16_r8(sa[0][0], sa[0][1], qa[ks][0], qa[ks][1], r0, r1);
                     mma_bf16_r8(sa[1][0], sa[1][1], qa[ks][0], qa[ks][1], r2, r3);
                     mma_bf16_r8(sb[0][0], sb[0][1], qa[ks + 1][0], qa[ks + 1][1], r4, r5);
@@ -401,22 +404,31 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
                 }
             } else {
 #pragma unroll
-                for (int s4 = 0; s4 < D / 32; ++s4) {
-                    uint32_t r0, r1, r2, r3;
-                    ldsm_x4(kb + tile_off<D, FP8>(tokK, 2 * s4 + (mi & 1)), r0, r1, r2, r3);
-                    mma_f16_r8(sa[0][0], sa[0][1], qa[2 * s4][0], qa[2 * s4][1], cvt_lo(r0), cvt_hi(r0));
-                    mma_f16_r8(sb[0][0], sb[0][1], qa[2 * s4 + 1][0], qa[2 * s4 + 1][1], cvt_lo(r1), cvt_hi(r1));
-                    mma_f16_r8(sa[1][0], sa[1][1], qa[2 * s4][0], qa[2 * s4][1], cvt_lo(r2), cvt_hi(r2));
-                    mma_f16_r8(sb[1][0], sb[1][1], qa[2 * s4 + 1][0], qa[2 * s4 + 1][1], cvt_lo(r3), cvt_hi(r3));
-                }
+                for (int s4 = 0; s4 < D / 32; ++s4)
+#pragma unroll
+                    for (int h16 = 0; h16 < TT / 16; ++h16) {   // tokens 16 h16 .. 16 h16 + 15
+                        uint32_t r0, r1, r2, r3;
+                        ldsm_x4(kb + tile_off<D, FP8, TT>(16 * h16 + tokK, 2 * s4 + (mi & 1)), r0, r1, r2, r3);
+                        // two n-tiles: even and odd k-steps on separate chains; four
+                        // n-tiles already make four independent chains (fewer registers)
+                        float(&odd)[NJ][2] = NJ == 2 ? sb : sa;
+                        mma_f16_r8(sa[2 * h16][0], sa[2 * h16][1], qa[2 * s4][0], qa[2 * s4][1], cvt_lo(r0),
+                                   cvt_hi(r0));
+                        mma_f16_r8(odd[2 * h16][0], odd[2 * h16][1], qa[2 * s4 + 1][0], qa[2 * s4 + 1][1],
+                                   cvt_lo(r1), cvt_hi(r1));
+                        mma_f16_r8(sa[2 * h16 + 1][0], sa[2 * h16 + 1][1], qa[2 * s4][0], qa[2 * s4][1], cvt_lo(r2),
+                                   cvt_hi(r2));
+                        mma_f16_r8(odd[2 * h16 + 1][0], odd[2 * h16 + 1][1], qa[2 * s4 + 1][0], qa[2 * s4 + 1][1],
+                                   cvt_lo(r3), cvt_hi(r3));
+                    }
             }
 
             // online softmax in log2 units; masked tokens are -inf (never 0 * NaN)
             const float slog2 = FP8 ? p.scale_log2 * si.ks : p.scale_log2;
-            float sc[2][2];
+            float sc[NJ][2];
             float mx = -INFINITY;
 #pragma unroll
-            for (int j = 0; j < 2; ++j)
+            for (int j = 0; j < NJ; ++j)
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     const int tok = tok0 + 8 * j + 2 * c4 + e;
@@ -428,19 +440,24 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
             const float m_new = fmaxf(m_run, mx);
             const float m_ref = (m_new == -INFINITY) ? 0.f : m_new;
             const float alpha = ex2(m_run - m_ref);
-            const float p00 = ex2(sc[0][0] - m_ref), p01 = ex2(sc[0][1] - m_ref);
-            const float p10 = ex2(sc[1][0] - m_ref), p11 = ex2(sc[1][1] - m_ref);
-            uint32_t pa0, pa2;
-            float psum;
-            if constexpr (!FP8) {
-                pa0 = pack_bf16(p00, p01);
-                pa2 = pack_bf16(p10, p11);
-                psum = (bf16_lo(pa0) + bf16_hi(pa0)) + (bf16_lo(pa2) + bf16_hi(pa2));
-            } else {
-                pa0 = pack_f16(p00, p01);
-                pa2 = pack_f16(p10, p11);
-                const float2 f0 = f16x2_to_f32(pa0), f2 = f16x2_to_f32(pa2);
-                psum = (f0.x + f0.y) + (f2.x + f2.y);
+            // P as the A operand of the P V mma, one k-step of 16 tokens per h16:
+            // a0 = tokens 16 h16 + 2c4, +1; a2 = tokens 16 h16 + 8 + 2c4, +1
+            uint32_t pa0[TT / 16], pa2[TT / 16];
+            float psum = 0.f;
+#pragma unroll
+            for (int h16 = 0; h16 < TT / 16; ++h16) {
+                const float p00 = ex2(sc[2 * h16][0] - m_ref), p01 = ex2(sc[2 * h16][1] - m_ref);
+                const float p10 = ex2(sc[2 * h16 + 1][0] - m_ref), p11 = ex2(sc[2 * h16 + 1][1] - m_ref);
+                if constexpr (!FP8) {
+                    pa0[h16] = pack_bf16(p00, p01);
+                    pa2[h16] = pack_bf16(p10, p11);
+                    psum += (bf16_lo(pa0[h16]) + bf16_hi(pa0[h16])) + (bf16_lo(pa2[h16]) + bf16_hi(pa2[h16]));
+                } else {
+                    pa0[h16] = pack_f16(p00, p01);
+                    pa2[h16] = pack_f16(p10, p11);
+                    const float2 f0 = f16x2_to_f32(pa0[h16]), f2 = f16x2_to_f32(pa2[h16]);
+                    psum += (f0.x + f0.y) + (f2.x + f2.y);
+                }
             }
             l_run = l_run * alpha + psum;
             m_run = m_new;
@@ -457,54 +474,62 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
 #pragma unroll
                 for (int dj = 0; dj < D / 16; ++dj) {
                     uint32_t r0, r1, r2, r3;
-                    ldsm_x4_trans(vb + tile_off<D, FP8>(tokV, 2 * dj + (mi >> 1)), r0, r1, r2, r3);
-                    mma_bf16_r8(o[2 * dj][0], o[2 * dj][1], pa0, pa2, r0, r1);
-                    mma_bf16_r8(o[2 * dj + 1][0], o[2 * dj + 1][1], pa0, pa2, r2, r3);
+                    ldsm_x4_trans(vb + tile_off<D, FP8, TT>(tokV, 2 * dj + (mi >> 1)), r0, r1, r2, r3);
+                    mma_bf16_r8(o[2 * dj][0], o[2 * dj][1], pa0[0], pa2[0], r0, r1);
+                    mma_bf16_r8(o[2 * dj + 1][0], o[2 * dj + 1][1], pa0[0], pa2[0], r2, r3);
                 }
             } else {
                 // E4M3 V: lane (n = g, c4) loads d in [DV*n, DV*n + DV) of tokens
-                // 2c4, 2c4+1, 8+2c4, 9+2c4; byte permutes pair tokens per d, and the
-                // mma n-index j of n-tile nt stands for d = DV*j + nt.
+                // 2c4, 2c4+1, 8+2c4, 9+2c4 (+16 h16); byte permutes pair tokens per
+                // d, and the mma n-index j of n-tile nt stands for d = DV*j + nt.
                 constexpr int DV = D / 8;
                 constexpr int WORDS = DV / 4;
-                uint32_t wa[WORDS], wb[WORDS], wc[WORDS], wd[WORDS];
-                const int t0 = 2 * c4;
-                if constexpr (DV == 16) {
-                    const uint4 a = lds128(vb + tile_off<D, FP8>(t0, g));
-                    const uint4 b = lds128(vb + tile_off<D, FP8>(t0 + 1, g));
-                    const uint4 cc = lds128(vb + tile_off<D, FP8>(t0 + 8, g));
-                    const uint4 dd = lds128(vb + tile_off<D, FP8>(t0 + 9, g));
-                    wa[0] = a.x; wa[1] = a.y; wa[2] = a.z; wa[3] = a.w;
-                    wb[0] = b.x; wb[1] = b.y; wb[2] = b.z; wb[3] = b.w;
-                    wc[0] = cc.x; wc[1] = cc.y; wc[2] = cc.z; wc[3] = cc.w;
-                    wd[0] = dd.x; wd[1] = dd.y; wd[2] = dd.z; wd[3] = dd.w;
-                } else {
-                    const uint32_t off8 = (uint32_t)((g & 1) * 8);
-                    const uint2 a = lds64(vb + tile_off<D, FP8>(t0, g >> 1) + off8);
-                    const uint2 b = lds64(vb + tile_off<D, FP8>(t0 + 1, g >> 1) + off8);
-                    const uint2 cc = lds64(vb + tile_off<D, FP8>(t0 + 8, g >> 1) + off8);
-                    const uint2 dd = lds64(vb + tile_off<D, FP8>(t0 + 9, g >> 1) + off8);
-                    wa[0] = a.x; wa[1] = a.y;
-                    wb[0] = b.x; wb[1] = b.y;
-                    wc[0] = cc.x; wc[1] = cc.y;
-                    wd[0] = dd.x; wd[1] = dd.y;
-                }
                 const float vs = si.vs;
+                // one 16-token half at a time (not unrolled: the second half's
+                // loads are not hoisted over the first's mma, which keeps the
+                // 32-token tile within the register file)
+#pragma unroll 1
+                for (int h16 = 0; h16 < TT / 16; ++h16) {
+                    const uint32_t pl = (TT == 16 || h16 == 0) ? pa0[0] : pa0[TT / 16 - 1];
+                    const uint32_t ph = (TT == 16 || h16 == 0) ? pa2[0] : pa2[TT / 16 - 1];
+                    uint32_t wa[WORDS], wb[WORDS], wc[WORDS], wd[WORDS];
+                    const int t0 = 16 * h16 + 2 * c4;
+                    if constexpr (DV == 16) {
+                        const uint4 a = lds128(vb + tile_off<D, FP8, TT>(t0, g));
+                        const uint4 b = lds128(vb + tile_off<D, FP8, TT>(t0 + 1, g));
+                        const uint4 cc = lds128(vb + tile_off<D, FP8, TT>(t0 + 8, g));
+                        const uint4 dd = lds128(vb + tile_off<D, FP8, TT>(t0 + 9, g));
+                        wa[0] = a.x; wa[1] = a.y; wa[2] = a.z; wa[3] = a.w;
+                        wb[0] = b.x; wb[1] = b.y; wb[2] = b.z; wb[3] = b.w;
+                        wc[0] = cc.x; wc[1] = cc.y; wc[2] = cc.z; wc[3] = cc.w;
+                        wd[0] = dd.x; wd[1] = dd.y; wd[2] = dd.z; wd[3] = dd.w;
+                    } else {
+                        const uint32_t off8 = (uint32_t)((g & 1) * 8);
+                        const uint2 a = lds64(vb + tile_off<D, FP8, TT>(t0, g >> 1) + off8);
+                        const uint2 b = lds64(vb + tile_off<D, FP8, TT>(t0 + 1, g >> 1) + off8);
+                        const uint2 cc = lds64(vb + tile_off<D, FP8, TT>(t0 + 8, g >> 1) + off8);
+                        const uint2 dd = lds64(vb + tile_off<D, FP8, TT>(t0 + 9, g >> 1) + off8);
+                        wa[0] = a.x; wa[1] = a.y;
+                        wb[0] = b.x; wb[1] = b.y;
+                        wc[0] = cc.x; wc[1] = cc.y;
+                        wd[0] = dd.x; wd[1] = dd.y;
+                    }
 #pragma unroll
-                for (int kw = 0; kw < WORDS; ++kw) {
-                    const uint32_t x0 = __byte_perm(wa[kw], wb[kw], 0x5140);
-                    const uint32_t x1 = __byte_perm(wa[kw], wb[kw], 0x7362);
-                    const uint32_t y0 = __byte_perm(wc[kw], wd[kw], 0x5140);
-                    const uint32_t y1 = __byte_perm(wc[kw], wd[kw], 0x7362);
-                    float t[4][2] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
-                    mma_f16_r8(t[0][0], t[0][1], pa0, pa2, cvt_lo(x0), cvt_lo(y0));
-                    mma_f16_r8(t[1][0], t[1][1], pa0, pa2, cvt_hi(x0), cvt_hi(y0));
-                    mma_f16_r8(t[2][0], t[2][1], pa0, pa2, cvt_lo(x1), cvt_lo(y1));
-                    mma_f16_r8(t[3][0], t[3][1], pa0, pa2, cvt_hi(x1), cvt_hi(y1));
+                    for (int kw = 0; kw < WORDS; ++kw) {
+                        const uint32_t x0 = __byte_perm(wa[kw], wb[kw], 0x5140);
+                        const uint32_t x1 = __byte_perm(wa[kw], wb[kw], 0x7362);
+                        const uint32_t y0 = __byte_perm(wc[kw], wd[kw], 0x5140);
+                        const uint32_t y1 = __byte_perm(wc[kw], wd[kw], 0x7362);
+                        float t[4][2] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+                        mma_f16_r8(t[0][0], t[0][1], pl, ph, cvt_lo(x0), cvt_lo(y0));
+                        mma_f16_r8(t[1][0], t[1][1], pl, ph, cvt_hi(x0), cvt_hi(y0));
+                        mma_f16_r8(t[2][0], t[2][1], pl, ph, cvt_lo(x1), cvt_lo(y1));
+                        mma_f16_r8(t[3][0], t[3][1], pl, ph, cvt_hi(x1), cvt_hi(y1));
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        o[4 * kw + e][0] = fmaf(t[e][0], vs, o[4 * kw + e][0]);
-                        o[4 * kw + e][1] = fmaf(t[e][1], vs, o[4 * kw + e][1]);
+                        for (int e = 0; e < 4; ++e) {
+                            o[4 * kw + e][0] = fmaf(t[e][0], vs, o[4 * kw + e][0]);
+                            o[4 * kw + e][1] = fmaf(t[e][1], vs, o[4 * kw + e][1]);
+                        }
                     }
                 }
             }
@@ -602,15 +627,15 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
     }
 }
 
-template <int D, bool FP8>
+template <int D, bool FP8, int TT>
 size_t smem_bytes_for(int stages, int max_batch)
 {
-    using Gm = Geo<D, FP8>;
+    using Gm = Geo<D, FP8, TT>;
     return 1024 + (size_t)kAttnWarps * stages * (Gm::STAGEB + sizeof(StageInfo) + 8) +
            sizeof(int) * (size_t)(max_batch + 1);
 }
 
-template <int D, bool FP8>
+template <int D, bool FP8, int TT>
 cudaError_t prepare_t(int num_sms, int max_batch, AttnLaunch* out)
 {
     int dev = 0, optin = 0;
@@ -620,10 +645,10 @@ cudaError_t prepare_t(int num_sms, int max_batch, AttnLaunch* out)
     if (e != cudaSuccess) return e;
     const size_t budget = (size_t)optin - 256;   // static shared memory of the kernel
     int stages = kAttnMaxStages;
-    while (stages > 2 && smem_bytes_for<D, FP8>(stages, max_batch) > budget) --stages;
-    if (smem_bytes_for<D, FP8>(stages, max_batch) > budget) return cudaErrorInvalidConfiguration;
-    const size_t bytes = smem_bytes_for<D, FP8>(stages, max_batch);
-    e = cudaFuncSetAttribute(decode_attn_kernel<D, FP8, kAttnWarps>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    while (stages > 2 && smem_bytes_for<D, FP8, TT>(stages, max_batch) > budget) --stages;
+    if (smem_bytes_for<D, FP8, TT>(stages, max_batch) > budget) return cudaErrorInvalidConfiguration;
+    const size_t bytes = smem_bytes_for<D, FP8, TT>(stages, max_batch);
+    e = cudaFuncSetAttribute(decode_attn_kernel<D, FP8, kAttnWarps, TT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)bytes);
     if (e != cudaSuccess) return e;
     e = combine_prepare(D);
@@ -631,16 +656,23 @@ cudaError_t prepare_t(int num_sms, int max_batch, AttnLaunch* out)
     out->ctas = num_sms;
     out->stages = stages;
     out->smem_bytes = bytes;
+    out->tile = TT;
     return cudaSuccess;
 }
 
 }  // namespace
 
-cudaError_t attn_prepare(int head_dim, bool fp8, int num_sms, int max_batch, AttnLaunch* out)
+cudaError_t attn_prepare(int head_dim, bool fp8, int page_size, int num_sms, int max_batch, AttnLaunch* out)
 {
-    if (head_dim == 128) return fp8 ? prepare_t<128, true>(num_sms, max_batch, out)
-                                    : prepare_t<128, false>(num_sms, max_batch, out);
-    return fp8 ? prepare_t<64, true>(num_sms, max_batch, out) : prepare_t<64, false>(num_sms, max_batch, out);
+    const bool wide = attn_tile(fp8, page_size) == kTileWide;
+    if (head_dim == 128) {
+        if (!fp8) return prepare_t<128, false, kTile>(num_sms, max_batch, out);
+        return wide ? prepare_t<128, true, kTileWide>(num_sms, max_batch, out)
+                    : prepare_t<128, true, kTile>(num_sms, max_batch, out);
+    }
+    if (!fp8) return prepare_t<64, false, kTile>(num_sms, max_batch, out);
+    return wide ? prepare_t<64, true, kTileWide>(num_sms, max_batch, out)
+                : prepare_t<64, true, kTile>(num_sms, max_batch, out);
 }
 
 cudaError_t launch_decode_attn(const AttnParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
@@ -649,12 +681,17 @@ cudaError_t launch_decode_attn(const AttnParams& p, const CUtensorMap& tmk, cons
     const dim3 grid(L.ctas), block(kAttnWarps * 32);
     AttnParams q = p;
     q.stages = L.stages;
+    const bool wide = L.tile == kTileWide;
     if (head_dim == 128) {
-        if (fp8) decode_attn_kernel<128, true, kAttnWarps><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
-        else decode_attn_kernel<128, false, kAttnWarps><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
+        if (!fp8) decode_attn_kernel<128, false, kAttnWarps, kTile><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
+        else if (wide)
+            decode_attn_kernel<128, true, kAttnWarps, kTileWide><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
+        else decode_attn_kernel<128, true, kAttnWarps, kTile><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
     } else {
-        if (fp8) decode_attn_kernel<64, true, kAttnWarps><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
-        else decode_attn_kernel<64, false, kAttnWarps><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
+        if (!fp8) decode_attn_kernel<64, false, kAttnWarps, kTile><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
+        else if (wide)
+            decode_attn_kernel<64, true, kAttnWarps, kTileWide><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
+        else decode_attn_kernel<64, true, kAttnWarps, kTile><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
     }
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;

@@ -99,7 +99,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
 }
 
 // 2-D view of a pool: rows = num_pages * Hkv * P token rows of head_dim
-// elements; box = 16 rows x (128 or 64 bytes), swizzled to match the
+// elements; box = one attention tile of rows (16, or 32 for E4M3 pools with
+// pages of at least 32 tokens) x (128 or 64 bytes), swizzled to match the
 // kernel's shared-memory addressing.
 bool encode_pool(const pkv_ctx* ctx, const void* pool, CUtensorMap* map)
 {
@@ -112,7 +113,7 @@ bool encode_pool(const pkv_ctx* ctx, const void* pool, CUtensorMap* map)
     cuuint64_t dims[2] = {(cuuint64_t)ctx->cfg.head_dim,
                           (cuuint64_t)ctx->cfg.num_pages * ctx->cfg.num_kv_heads * ctx->cfg.page_size};
     cuuint64_t strides[1] = {(cuuint64_t)rowb};
-    cuuint32_t box[2] = {(cuuint32_t)(boxb / elem), (cuuint32_t)pkv::kTile};
+    cuuint32_t box[2] = {(cuuint32_t)(boxb / elem), (cuuint32_t)pkv::attn_tile(fp8, ctx->cfg.page_size)};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
                     const_cast<void*>(pool), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -171,7 +172,8 @@ pkv_status pkv_create(const pkv_config* cfg, pkv_ctx** out)
         return PKV_ERR_CUDA;
     }
     const bool fp8 = cfg->kv_dtype == PKV_KV_FP8_E4M3;
-    if (pkv::attn_prepare(cfg->head_dim, fp8, ctx->num_sms, cfg->max_batch, &ctx->attn) != cudaSuccess) {
+    if (pkv::attn_prepare(cfg->head_dim, fp8, cfg->page_size, ctx->num_sms, cfg->max_batch, &ctx->attn) !=
+        cudaSuccess) {
         free(ctx);
         return PKV_ERR_CUDA;
     }

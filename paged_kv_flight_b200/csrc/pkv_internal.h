@@ -24,6 +24,12 @@ enum : int { kErrLength = 1, kErrPage = 2, kErrTimeout = 4 };
 #endif
 
 constexpr int kTile = 16;          // tokens per attention tile (one TMA box height)
+constexpr int kTileWide = 32;      // E4M3 tiles when pages hold at least 32 tokens
+
+// Tokens per tile of the one-new-token attention: 32 for E4M3 pools whose
+// pages hold a whole 32-token tile (the same bytes as a 16-token bf16 tile,
+// half the per-tile work per token), else 16.
+inline int attn_tile(bool fp8, int page_size) { return (fp8 && page_size >= kTileWide) ? kTileWide : kTile; }
 constexpr int kMaxGroup = 8;       // query heads per kv head handled by one mma row block
 constexpr int kMaxTokenRows = 16;  // G x q_len rows of the several-new-tokens attention
 constexpr int kAttnWarps = PKV_ATTN_WARPS;
@@ -94,8 +100,9 @@ struct AttnLaunch {
     int ctas;
     int stages;
     size_t smem_bytes;
+    int tile;             // tokens per tile (attn_tile)
 };
-cudaError_t attn_prepare(int head_dim, bool fp8, int num_sms, int max_batch, AttnLaunch* out);
+cudaError_t attn_prepare(int head_dim, bool fp8, int page_size, int num_sms, int max_batch, AttnLaunch* out);
 cudaError_t launch_decode_attn(const AttnParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
                                int head_dim, bool fp8, const AttnLaunch& L, cudaStream_t stream);
 

@@ -96,7 +96,7 @@ bool encode_pool(const pkv_config* c, const void* pool, CUtensorMap* map)
     const int boxb = rowb > 128 ? 128 : rowb;
     cuuint64_t dims[2] = {(cuuint64_t)c->head_dim, (cuuint64_t)c->num_pages * c->num_kv_heads * c->page_size};
     cuuint64_t strides[1] = {(cuuint64_t)rowb};
-    cuuint32_t box[2] = {(cuuint32_t)(boxb / elem), (cuuint32_t)pkv::kTile};
+    cuuint32_t box[2] = {(cuuint32_t)(boxb / elem), (cuuint32_t)pkv::attn_tile(fp8, c->page_size)};
     cuuint32_t estr[2] = {1, 1};
     return fn(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
               const_cast<void*>(pool), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -144,7 +144,8 @@ extern "C" pkv_status pkv_decode_attn_noalloc(const pkv_config* cfg, const void*
     // the largest batch the shared memory is sized for, so that this call never
     // lowers the kernel's shared-memory limit below what a context set
     pkv::AttnLaunch L;
-    if (pkv::attn_prepare(cfg->head_dim, fp8, num_sms, pkv::kMaxBatch, &L) != cudaSuccess) return PKV_ERR_CUDA;
+    if (pkv::attn_prepare(cfg->head_dim, fp8, cfg->page_size, num_sms, pkv::kMaxBatch, &L) != cudaSuccess)
+        return PKV_ERR_CUDA;
 
     CUtensorMap tmk, tmv;
     if (!encode_pool(cfg, k_pool, &tmk) || !encode_pool(cfg, v_pool, &tmv)) return PKV_ERR_CUDA;

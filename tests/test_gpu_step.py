@@ -31,6 +31,7 @@ SMALL = [
     ("g8_d128_p16_fp8", 64, 8, 128, 16, True, [7, 130, 1100]),
     ("g4_d64_p16_fp8", 8, 2, 64, 16, True, [3, 40, 500]),
     ("g2_d128_p64_fp8", 16, 8, 128, 64, True, [100, 1500]),
+    ("g4_d64_p32_fp8", 8, 2, 64, 32, True, [0, 31, 32, 33, 63, 64, 999]),
 ]
 
 
