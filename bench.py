@@ -742,12 +742,13 @@ def run_loop(args, rank, world, local_rank):
                        "description": "continuous batching over 256 slots, Hq 64 / Hkv 8, d 128, page 16: "
                                       "host page allocator between steps, requests finish and are replaced, "
                                       "30% share a 512-token system prompt's pages",
-                       "timing": "device events around all iterations; host allocator calls, the H2D copy "
-                                 "of the batch's block table and lengths and the stand-in prefill of new "
-                                 "requests' pages included; L2 not flushed (the pools are far larger)"},
+                       "timing": "device events around all iterations; host allocator calls, the one H2D "
+                                 "copy per step of the table changes, slots and lengths, the device table "
+                                 "sync (pkv_table_sync) and the stand-in prefill of new requests' pages "
+                                 "included; L2 not flushed (the pools are far larger)"},
             "decode_tokens_per_s": toks, "us_per_iteration": r["us_per_iteration"],
             "host_allocator_us_per_iteration": r["host_allocator_us_per_iteration"],
-            "loop_stats": r["stats"], "gpu_launches": 3 * args.steps, "clocks": clock_info}
+            "loop_stats": r["stats"], "gpu_launches": int(r["stats"].get("pkv_launches", 0)), "clocks": clock_info}
 
 
 def main(argv=None):

@@ -191,6 +191,26 @@ pkv_status pkv_qkv_rope_append(pkv_ctx* ctx, const void* x, const void* w_qkv, i
                                const int32_t* block_tables, int bt_stride,
                                const int32_t* seq_lens, int batch, cudaStream_t stream);
 
+/* Device side of the host page allocator (pkv_pages.h) for a decode loop,
+ * in two small kernels on `stream`: applies the allocator's change log to a
+ * device copy of the block table, then gathers the rows and lengths of the
+ * step's batch into the block_tables / seq_lens arguments of the step
+ * (page_size is checked to be positive; the rows are copied whole).
+ *   upload    device int32 [3 n_changes + 2 batch]: the (slot, index, value)
+ *             triples of pkv_pages_take_changes (each entry at most once),
+ *             then the batch's slots, then their lengths L (tokens cached
+ *             before the step) -- one host-to-device copy per step;
+ *   table     device int32 [max_batch][max_blocks], updated in place;
+ *   bt_out    device int32 [batch][max_blocks]: row b receives row slot_b
+ *             of the updated table (-1 everywhere for a slot outside it);
+ *   lens_out  device int32 [batch]: the lengths.
+ * Triples outside the table are skipped.  All pointers 4-byte
+ * aligned and caller-owned.  Asynchronous; PKV_ERR_INVALID_ARG for bad sizes
+ * or pointers, PKV_ERR_CUDA on a launch failure. */
+pkv_status pkv_table_sync(const int32_t* upload, int n_changes, int batch, int max_batch, int max_blocks,
+                          int page_size, int32_t* table, int32_t* bt_out, int32_t* lens_out,
+                          cudaStream_t stream);
+
 /* Layouts of the QKV weight for pkv_qkv_rope_append. */
 enum { PKV_W_ROWS = 0, PKV_W_TILED = 1 };
 

@@ -86,13 +86,16 @@ const int32_t* pkv_pages_refcount(const pkv_pages* pp);
 int pkv_pages_free_count(const pkv_pages* pp);
 
 /* The block-table writes since the previous call (admissions, pages added by
- * pkv_pages_reserve, rows cleared by pkv_pages_release), in order, as
- * (slot, index, value) int32 triples written to out: a caller that keeps a
- * copy of the table (on the device, say) replays them instead of copying the
- * whole table each step.  Returns the number of triples, or -1 when there
- * were more than max_changes (or more than the log holds, about num_pages),
- * in which case nothing is written and the caller should copy the whole
- * table.  Either way the log starts empty again. */
+ * pkv_pages_reserve, rows cleared by pkv_pages_release) as (slot, index,
+ * value) int32 triples written to out: an entry written more than once
+ * appears once, with its last value (so the triples can be applied in any
+ * order, in parallel), in the order of those last writes.  A caller that
+ * keeps a copy of the table (on the device, say: pkv_table_sync) applies
+ * them instead of copying the whole table each step.  Returns the number of
+ * triples, or -1 when there were more than max_changes (or more writes than
+ * the log holds, about num_pages), in which case the contents of out are
+ * unspecified and the caller should copy the whole table.  Either way the
+ * log starts empty again. */
 int pkv_pages_take_changes(pkv_pages* pp, int32_t* out, int max_changes);
 
 #ifdef __cplusplus

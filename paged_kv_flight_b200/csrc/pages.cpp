@@ -11,6 +11,7 @@
 #include <string.h>
 
 #include <new>
+#include <utility>
 #include <vector>
 
 #include "../../include/pkv_pages.h"
@@ -26,6 +27,7 @@ struct pkv_pages {
     int free_top = 0;                // entries of free_stack in use
     std::vector<int32_t> log;        // (slot, index, value) of every table write since the last take
     bool log_full = false;           // more writes than the log holds: the caller must copy the table
+    std::vector<uint8_t> seen;       // [max_batch][max_blocks] scratch of pkv_pages_take_changes, all 0 between calls
 };
 
 namespace {
@@ -82,6 +84,7 @@ pkv_status pkv_pages_create(int num_pages, int page_size, int max_batch, int max
         pp->ref.assign(num_pages, 0);
         pp->free_stack.resize(num_pages);
         pp->log.reserve(3 * (size_t)num_pages + 3 * 1024);
+        pp->seen.assign((size_t)max_batch * max_blocks_per_seq, 0);
     } catch (...) {
         delete pp;
         return PKV_ERR_OOM;
@@ -181,12 +184,32 @@ int pkv_pages_take_changes(pkv_pages* pp, int32_t* out, int max_changes)
 {
     if (!pp || max_changes < 0 || (!out && max_changes > 0)) return -1;
     const int n = (int)(pp->log.size() / 3);
-    int ret;
-    if (pp->log_full || n > max_changes) {
-        ret = -1;
-    } else {
-        if (n) memcpy(out, pp->log.data(), sizeof(int32_t) * 3 * (size_t)n);
-        ret = n;
+    int ret = -1;
+    if (!pp->log_full) {
+        // the last write of each entry, once, in the order of those writes:
+        // walk the log backwards keeping first sightings, then reverse them
+        const int32_t* lg = pp->log.data();
+        int m = 0;
+        bool fits = true;
+        for (int k = n - 1; k >= 0; --k) {
+            const size_t key = (size_t)lg[3 * k] * pp->max_blocks + lg[3 * k + 1];
+            if (pp->seen[key]) continue;
+            pp->seen[key] = 1;
+            if (m >= max_changes) {
+                fits = false;
+                continue;   // keep marking, so the clean-up below finds every entry
+            }
+            out[3 * m] = lg[3 * k];
+            out[3 * m + 1] = lg[3 * k + 1];
+            out[3 * m + 2] = lg[3 * k + 2];
+            ++m;
+        }
+        for (int k = 0; k < n; ++k) pp->seen[(size_t)lg[3 * k] * pp->max_blocks + lg[3 * k + 1]] = 0;
+        if (fits) {
+            for (int a = 0, b = m - 1; a < b; ++a, --b)
+                for (int c = 0; c < 3; ++c) std::swap(out[3 * a + c], out[3 * b + c]);
+            ret = m;
+        }
     }
     pp->log.clear();
     pp->log_full = false;

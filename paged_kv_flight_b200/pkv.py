@@ -45,7 +45,8 @@ EXPORTS = ("pkv_create", "pkv_rope_append", "pkv_decode_attn", "pkv_destroy", "p
            "pkv_pages_create", "pkv_pages_destroy", "pkv_pages_admit", "pkv_pages_reserve", "pkv_pages_advance",
            "pkv_pages_release", "pkv_pages_block_table", "pkv_pages_seq_lens", "pkv_pages_active",
            "pkv_pages_refcount", "pkv_pages_free_count", "pkv_pages_take_changes", "pkv_qkv_rope_append",
-           "pkv_qkv_pack_weight", "pkv_set_qkv_split", "pkv_qkv_launch_shape")
+           "pkv_qkv_pack_weight", "pkv_set_qkv_split", "pkv_qkv_launch_shape",
+           "pkv_table_sync")
 
 
 class pkv_config(C.Structure):
@@ -98,6 +99,8 @@ lib.pkv_set_qkv_split.argtypes = [_V, C.c_int]
 lib.pkv_set_qkv_split.restype = C.c_int
 lib.pkv_qkv_launch_shape.argtypes = [_V, C.c_int, C.c_int, _V]
 lib.pkv_qkv_launch_shape.restype = C.c_int
+lib.pkv_table_sync.argtypes = [_V, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, _V, _V, _V, _V]
+lib.pkv_table_sync.restype = C.c_int
 lib.pkv_set_tail_chunks.argtypes = [_V, C.c_int]
 lib.pkv_set_tail_chunks.restype = C.c_int
 lib.pkv_workspace_bytes.argtypes = [_V]
@@ -318,6 +321,16 @@ PKV_W_ROWS, PKV_W_TILED = 0, 1
 def pkv_set_qkv_split(ctx, split: int, check: bool = True) -> int:
     """CTAs (a cluster) per head over the hidden dimension: 1 .. 4, 0 = automatic."""
     return _done(lib.pkv_set_qkv_split(ctx, int(split)), "pkv_set_qkv_split", check)
+
+
+def pkv_table_sync(upload, n_changes: int, batch: int, table, bt_out, lens_out, page_size: int, stream=None,
+                   check: bool = True) -> int:
+    """upload: device int32 [3 n_changes + 2 batch] (changes, slots, lengths);
+    table [max_batch, max_blocks] updated in place; bt_out [>= batch,
+    max_blocks] and lens_out [>= batch] receive the batch's rows and lengths."""
+    st = lib.pkv_table_sync(_ptr(upload), int(n_changes), int(batch), int(table.shape[0]), int(table.shape[1]),
+                            int(page_size), _ptr(table), _ptr(bt_out), _ptr(lens_out), _stream(stream))
+    return _done(st, "pkv_table_sync", check)
 
 
 def pkv_qkv_launch_shape(ctx, batch: int, hidden: int) -> dict:

@@ -11,10 +11,11 @@ Production", section "What the Scheduler Actually Does"):
      new page (pages are allocated on demand as tokens are generated); if the
      pool is short, preempt the most recently admitted request (its pages go
      back, it is re-queued to be recomputed later) and retry;
-  2. bring the device copy of the block table up to date by replaying the
+  2. bring the device copy of the block table up to date by applying the
      allocator's change log (a few entries per step instead of the whole
      table), and gather the active slots' rows and lengths into a contiguous
-     batch on the device;
+     batch on the device: one pinned upload (changes, slots, lengths) and one
+     pkv_table_sync call, two small kernels;
   3. run the step: pkv_rope_append + pkv_decode_attn over that batch;
   4. advance every active request by one token; requests that reached their
      output budget finish, their pages return to the pool at once, and
@@ -64,10 +65,8 @@ class _Staging:
 
     def __init__(self, max_changes, max_batch, max_blocks):
         pin = lambda n: torch.empty(n, dtype=torch.int32).pin_memory()
-        self.changes = pin(3 * max_changes)
-        self.slots = pin(max_batch)
-        self.lens = pin(max_batch)
-        self.pages = pin(max_blocks)
+        self.upload = pin(3 * max_changes + 2 * max_batch)    # changes, then slots, then lengths
+        self.pages = torch.empty(max_blocks, dtype=torch.int64).pin_memory()
         self.done = None
 
     def wait(self):
@@ -100,8 +99,8 @@ class DecodeLoop:
         self.ring = [_Staging(self.max_changes, c.max_batch, c.max_blocks) for _ in range(16)]
         self.ring_i = 0
         self.table_dev = torch.full((c.max_batch, c.max_blocks), -1, dtype=torch.int32, device=self.dev)
-        self.chg_dev = torch.empty(3 * self.max_changes, dtype=torch.int32, device=self.dev)
-        self.slots_dev = torch.empty(c.max_batch, dtype=torch.int64, device=self.dev)
+        self.upload_dev = torch.empty(3 * self.max_changes + 2 * c.max_batch, dtype=torch.int32, device=self.dev)
+        self.bt_dev = torch.full((c.max_batch, c.max_blocks), -1, dtype=torch.int32, device=self.dev)
         self.len_dev = torch.empty(c.max_batch, dtype=torch.int32, device=self.dev)
         self.slots = np.zeros(0, np.int64)
         # slot 0: the system prompt, decoding for the whole run
@@ -134,12 +133,13 @@ class DecodeLoop:
             st_buf = self._staging()
             host = st_buf.pages[:npg - own]
             host.numpy()[:] = self.pages.block_table[slot, own:npg]
-            pages = host.to(self.dev, non_blocking=True).long()
+            pages = host.to(self.dev, non_blocking=True)
             st_buf.done = torch.cuda.Event()
             st_buf.done.record()
-            shape = (len(pages), c.Hkv, c.P, c.d)
-            self.k_pool[pages] = torch.randn(shape, generator=self.gen, device=self.dev).to(torch.bfloat16)
-            self.v_pool[pages] = torch.randn(shape, generator=self.gen, device=self.dev).to(torch.bfloat16)
+            kv = torch.randn((2, len(pages), c.Hkv, c.P, c.d), generator=self.gen, device=self.dev,
+                             dtype=torch.bfloat16)
+            self.k_pool.index_copy_(0, pages, kv[0])
+            self.v_pool.index_copy_(0, pages, kv[1])
         self.stats["admitted"] += 1
         self.stats["shared"] += int(share_tokens > 0)
         return True
@@ -169,45 +169,43 @@ class DecodeLoop:
             if not self._preempt_one():
                 raise RuntimeError("page pool too small for one request")
         st = self._staging()
-        n = self.pages.take_changes(st.changes.numpy())
+        up = st.upload.numpy()
+        # the last write of each table entry, once (the allocator merges repeats)
+        n = self.pages.take_changes(up[:3 * self.max_changes])
         if n < 0:      # too many writes for the log: copy the whole table
             self.table_dev.copy_(torch.from_numpy(self.pages.block_table.copy()))
-        elif n > 0:
-            # an entry written twice (a slot released and refilled) keeps its last value
-            log = st.changes.numpy()[:3 * n].reshape(n, 3)
-            key = log[:, 0].astype(np.int64) * self.cfg.max_blocks + log[:, 1]
-            _, last = np.unique(key[::-1], return_index=True)
-            uniq = log[::-1][last]
-            m = len(uniq)
-            st.changes.numpy()[:3 * m] = uniq.reshape(-1)
-            chg = self.chg_dev[:3 * m]
-            chg.copy_(st.changes[:3 * m], non_blocking=True)
-            t = chg.view(m, 3).long()
-            self.table_dev[t[:, 0], t[:, 1]] = t[:, 2].int()
+            n = 0
         slots = np.flatnonzero(self.pages.active)
         B = len(slots)
-        st.slots[:B].numpy()[:] = slots
-        st.lens[:B].numpy()[:] = self.pages.seq_lens[slots]
-        self.slots_dev[:B].copy_(st.slots[:B], non_blocking=True)
-        self.len_dev[:B].copy_(st.lens[:B], non_blocking=True)
+        up[3 * n:3 * n + B] = slots
+        up[3 * n + B:3 * n + 2 * B] = self.pages.seq_lens[slots]
+        k = 3 * n + 2 * B
+        self.upload_dev[:k].copy_(st.upload[:k], non_blocking=True)
         st.done = torch.cuda.Event()
         st.done.record()
+        pkv.pkv_table_sync(self.upload_dev, n, B, self.table_dev, self.bt_dev, self.len_dev, self.cfg.P)
+        self.stats["pkv_launches"] += (n > 0) + (B > 0)          # apply changes, gather rows
         self.slots = slots
         return slots
 
     def inputs(self, B):
+        """q, k_new, v_new of the step: N(0, 1) bf16, one draw cut in three."""
         c = self.cfg
-        r = lambda *s: torch.randn(*s, generator=self.gen, device=self.dev).to(torch.bfloat16)
-        return r(B, c.Hq, c.d), r(B, c.Hkv, c.d), r(B, c.Hkv, c.d)
+        nq, nk = B * c.Hq * c.d, B * c.Hkv * c.d
+        flat = torch.randn(nq + 2 * nk, generator=self.gen, device=self.dev, dtype=torch.bfloat16)
+        return (flat[:nq].view(B, c.Hq, c.d), flat[nq:nq + nk].view(B, c.Hkv, c.d),
+                flat[nq + nk:].view(B, c.Hkv, c.d))
 
     def batch_tables(self, B):
-        """The batch's block-table rows (gathered on the device) and lengths."""
-        return self.table_dev.index_select(0, self.slots_dev[:B]), self.len_dev[:B]
+        """The batch's block-table rows (gathered on the device by
+        pkv_table_sync in schedule) and lengths."""
+        return self.bt_dev[:B], self.len_dev[:B]
 
     def device_step(self, slots, q, k_new, v_new, out):
         bt, ln = self.batch_tables(len(slots))
         pkv.pkv_rope_append(self.ctx, q, k_new, v_new, self.k_pool, self.v_pool, None, None, bt, ln)
         pkv.pkv_decode_attn(self.ctx, q, self.k_pool, self.v_pool, None, None, bt, ln, out)
+        self.stats["pkv_launches"] += 3                          # rope + append, attention, combine
         return bt, ln
 
     def finish(self, slots):
@@ -215,10 +213,10 @@ class DecodeLoop:
         waiting ones in."""
         self.pages.advance(1)
         self.budget[slots] -= 1
-        done = [int(s) for s in slots if s != 0 and self.budget[s] <= 0]
+        done = slots[(slots != 0) & (self.budget[slots] <= 0)]
         for s in done:
-            self.pages.release(s)
-            self.stats["finished"] += 1
+            self.pages.release(int(s))
+        self.stats["finished"] += len(done)
         self.iteration += 1
         for s in np.flatnonzero(self.pages.active == 0):
             if s == 0:

@@ -95,3 +95,32 @@ def test_loop_survives_a_tight_pool_by_preempting():
         assert (names == np.asarray(loop.pages.refcount)).all()
     finally:
         loop.close()
+
+
+def test_table_sync_applies_changes_and_gathers_rows():
+    """pkv_table_sync against numpy: every in-range triple applied, triples
+    outside the table skipped, each batch row = the updated table's row of its
+    slot (a slot outside the table gives -1), lengths passed through."""
+    from paged_kv_flight_b200 import pkv
+    rng = np.random.default_rng(3)
+    max_batch, max_blocks = 12, 20
+    table = rng.integers(-1, 100, size=(max_batch, max_blocks)).astype(np.int32)
+    keys = rng.choice(max_batch * max_blocks, size=40, replace=False)
+    chg = np.stack([keys // max_blocks, keys % max_blocks, rng.integers(0, 100, 40)], 1).astype(np.int32)
+    chg = np.concatenate([chg, np.array([[max_batch + 3, 0, 7], [0, max_blocks, 7], [-1, 2, 7]], np.int32)])
+    slots = np.array([5, 0, 11, 3, 40], np.int32)
+    lens = np.array([10, 0, 300, 17, 5], np.int32)
+    up = torch.from_numpy(np.concatenate([chg.ravel(), slots, lens]).astype(np.int32)).cuda()
+    t_dev = torch.from_numpy(table.copy()).cuda()
+    bt = torch.zeros(len(slots), max_blocks, dtype=torch.int32, device="cuda")
+    ln = torch.zeros(len(slots), dtype=torch.int32, device="cuda")
+    pkv.pkv_table_sync(up, len(chg), len(slots), t_dev, bt, ln, 16)
+    ref = table.copy()
+    for s, i, v in chg[:40]:
+        ref[s, i] = v
+    assert np.array_equal(t_dev.cpu().numpy(), ref)
+    want = np.stack([ref[s] if 0 <= s < max_batch else np.full(max_blocks, -1, np.int32) for s in slots])
+    assert np.array_equal(bt.cpu().numpy(), want)
+    assert np.array_equal(ln.cpu().numpy(), lens)
+    assert pkv.pkv_table_sync(up, -1, 1, t_dev, bt, ln, 16, check=False) == pkv.PKV_ERR_INVALID_ARG
+    assert pkv.pkv_table_sync(up, 0, 13, t_dev, bt, ln, 16, check=False) == pkv.PKV_ERR_INVALID_ARG

@@ -143,6 +143,8 @@ def test_random_operations_match_the_model(seed):
             _agree(pp, m)
             n = pp.take_changes(buf)
             assert n >= 0
+            keys = {(int(slot), int(i)) for slot, i, _ in buf[:3 * n].reshape(n, 3)}
+            assert len(keys) == n                      # each entry at most once: order-free
             for slot, i, v in buf[:3 * n].reshape(n, 3):
                 replica[slot, i] = v
             assert np.array_equal(replica, pp.block_table)
