@@ -12,7 +12,8 @@
 // ("TensorRT-LLM Guide", section "4. Native FP8 Quantization").
 //
 // Work decomposition (no host sync, one launch):
-//   * every CTA derives tiles-per-request (16 tokens per tile) from seq_lens
+//   * every CTA derives tiles-per-request (16 tokens per tile; 32 for E4M3
+//     pools whose pages hold 32 tokens or more) from seq_lens
 //     and keeps their exclusive prefix in shared memory;
 //   * the flattened sequence of tiles, ordered (request, kv head, tile), is cut
 //     into W equal contiguous ranges, one per warp worker (W <= warps x SMs),

@@ -132,8 +132,18 @@ def _ptr(x):
     raise TypeError(f"expected a tensor or a device pointer, got {type(x)}")
 
 
+# The current CUDA stream of the current device as a raw cudaStream_t: the
+# query PyTorch's own generated code uses (no Stream object is built, which
+# is most of the host cost of torch.cuda.current_stream()), else the public
+# API.
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+_cur_device = getattr(torch._C, "_cuda_getDevice", None)
+
+
 def _stream(s):
     if s is None:
+        if _raw_stream is not None and _cur_device is not None:
+            return _raw_stream(_cur_device())
         return torch.cuda.current_stream().cuda_stream
     if isinstance(s, torch.cuda.Stream):
         return s.cuda_stream
