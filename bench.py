@@ -716,6 +716,121 @@ def run_qkv(args, rank, world, local_rank):
             "gpu_launches": 5 * K, "clocks": clock_info}
 
 
+def run_mixed(args, rank, world, local_rank):
+    """Chunked prefill mixed with decode (pkv_rope_append_varlen +
+    pkv_decode_attn_varlen) on the llama8b batch: 8 seeded requests take a
+    64-token chunk, the other 56 one new token.  L2 flushed before every step;
+    the step replayed from a CUDA graph, attention alone timed eagerly."""
+    import torch
+    from paged_kv_flight_b200 import pkv, workloads
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w, q_lens = workloads.make_mixed(device=dev, offset=rank)
+    B = w.batch
+    cu = np.zeros(B + 1, np.int32)
+    cu[1:] = np.cumsum(q_lens)
+    n_tok = int(cu[-1])
+    keep = torch.from_numpy(np.concatenate([b * w.q_len + np.arange(q) for b, q in enumerate(q_lens)])).to(dev)
+    pack = lambda t: t.reshape(B * w.q_len, *t.shape[2:]).index_select(0, keep).contiguous()   # noqa: E731
+    q0, k_new, v_new = pack(w.q), pack(w.k_new), pack(w.v_new)
+    q = q0.clone()
+    out = torch.empty_like(q)
+    k_pool, v_pool = w.k_pool.to(dev).contiguous(), w.v_pool.to(dev).contiguous()
+    bt = torch.from_numpy(w.block_tables).to(dev)
+    sl = torch.from_numpy(w.seq_lens).to(dev)
+    cu_d = torch.from_numpy(cu).to(dev)
+    cfg = pkv.make_config(w.Hq, w.Hkv, w.d, w.P, "bf16", w.rope_base, B, w.bt_stride, w.num_pages)
+    ctx = pkv.pkv_create(cfg)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush_w = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+    flush_r = torch.ones(2 * l2 // 8, dtype=torch.int64, device=dev)
+    sink = torch.empty((), dtype=torch.int64, device=dev)
+
+    def flush():
+        flush_w.zero_()
+        torch.sum(flush_r, dim=0, out=sink)
+
+    def attn():
+        pkv.pkv_decode_attn_varlen(ctx, q, k_pool, v_pool, bt, sl, cu_d, out)
+
+    def step():
+        q.copy_(q0)    # the step rotates q in place: every step starts from the same q
+        pkv.pkv_rope_append_varlen(ctx, q, k_new, v_new, k_pool, v_pool, None, None, bt, sl, cu_d)
+        attn()
+
+    for _ in range(args.warmup):
+        flush()
+        step()
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream(dev)
+    with torch.cuda.stream(side):
+        step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        step()
+    for _ in range(args.warmup):
+        flush()
+        graph.replay()
+    torch.cuda.synchronize()
+    K = args.steps
+    clocks = ClockSampler(local_rank)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for k in range(K):
+        flush()
+        gev[k][0].record()
+        graph.replay()
+        gev[k][1].record()
+    clocks.sample()
+    aev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for k in range(K):
+        flush()
+        aev[k][0].record()
+        attn()
+        aev[k][1].record()
+    clocks.sample()
+    torch.cuda.synchronize()
+    barrier()
+    clock_info = clocks.stop()
+    st, bits = pkv.pkv_check_device_error(ctx)
+    if st != pkv.PKV_OK:
+        raise RuntimeError(f"device error: {pkv.pkv_status_str(st)} bits={bits}")
+    del graph
+    pkv.pkv_destroy(ctx)
+    step_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in gev) / K)
+    attn_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in aev) / K)
+    L = w.seq_lens.astype(np.int64)
+    row = 2 * w.Hkv * w.d * 2                      # K + V bytes of one token
+    # metric bytes: each request's cache (its new tokens included) once, q and out of every new token
+    by = int((row * (L + q_lens)).sum()) + 2 * n_tok * w.Hq * w.d * 2
+    # streamed: every block of 16 / G new tokens reads its own prefix
+    blk = 16 // (w.Hq // w.Hkv)
+    streamed = sum(row * (int(Lb) + min(j + blk, int(qb)))
+                   for Lb, qb in zip(L, q_lens) for j in range(0, int(qb), blk)) + 2 * n_tok * w.Hq * w.d * 2
+    peak, peak_src = measured_peak()
+    gbs = by / (attn_ms * 1e-3) / 1e9
+    return {"metric": METRIC, "value": sum_over_ranks(float(by)) / (step_ms * 1e-3) / 1e9, "unit": "GB/s",
+            "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "mixed",
+                       "description": "llama8b batch, 56 requests decode one token, 8 prefill a 64-token "
+                                      "chunk (568 new tokens): varlen RoPE + append, then varlen attention",
+                       "l2": "flushed before every step, outside the event window",
+                       "timing": "step: CUDA-graph replay; attention alone: eager events"},
+            "step_us": step_ms * 1e3, "attn_us": attn_ms * 1e3, "new_tokens": n_tok,
+            "new_tokens_per_s": sum_over_ranks(float(n_tok)) / (step_ms * 1e-3),
+            "streamed_bytes_per_launch": streamed,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                         "traffic": None, "kernel": "decode_attn_tokens_kernel<128> (varlen)",
+                         "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)", "bytes_per_launch": by,
+                         "note": "bytes = each request's cache once (the metric); a prefill chunk's blocks "
+                                 "re-read their prefix, see streamed_bytes_per_launch"},
+            "gpu_launches": 7 * K, "clocks": clock_info}   # step: rope, plan, attention, combine; alone: 3
+
+
 def run_loop(args, rank, world, local_rank):
     """The continuous-batching loop (serve_loop.py) on a 70B-shaped layer:
     256 slots, prompts {64,128,512,2048} (+ a 512-token system prompt shared
@@ -793,6 +908,8 @@ def main(argv=None):
                 line = run_loop(args, rank, world, local_rank)
             elif name == "qkv8b":
                 line = run_qkv(args, rank, world, local_rank)
+            elif name == "mixed":
+                line = run_mixed(args, rank, world, local_rank)
             else:
                 line = run_ours(args, name, rank, world, local_rank)
             if rank == 0:

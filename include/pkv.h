@@ -165,6 +165,41 @@ pkv_status pkv_decode_attn_tokens(pkv_ctx* ctx, const void* q, const void* k_poo
                                   const int32_t* seq_lens, int batch, int q_len, void* out,
                                   cudaStream_t stream);
 
+/* Several new tokens per request, a different number for each ("varlen"):
+ * chunked prefill mixed with decode in one batch ("Scaling TensorRT-LLM:
+ * Kernel Fusion and Inflight Batching in Production", section "What the
+ * Scheduler Actually Does"; "TensorRT-LLM Guide: High-Throughput GPU
+ * Inference Engine", section "1. In-Flight Batching: Continuous Iteration
+ * Scheduling").  The new tokens of all requests are packed: cu_q [batch + 1]
+ * int32 on the device, cu_q[0] = 0, non-decreasing, cu_q[batch] = n_tokens;
+ * token i of request b (cu_q[b] <= i < cu_q[b + 1]; a request may have none)
+ * sits at position L_b + i - cu_q[b].  q [n_tokens][Hq][d], k_new / v_new
+ * [n_tokens][Hkv][d], out [n_tokens][Hq][d], all bf16.
+ *
+ * pkv_rope_append_varlen: pkv_rope_append_tokens for packed tokens (bf16 or
+ * E4M3 pools): rotates q in place, appends every new token's k / v. */
+pkv_status pkv_rope_append_varlen(pkv_ctx* ctx, void* q, const void* k_new, const void* v_new,
+                                  void* k_pool, void* v_pool,
+                                  const float* k_scale, const float* v_scale,
+                                  const int32_t* block_tables, int bt_stride,
+                                  const int32_t* seq_lens, const int32_t* cu_q, int batch, int n_tokens,
+                                  cudaStream_t stream);
+
+/* pkv_decode_attn_varlen: token i of request b attends tokens 0 .. L_b + i -
+ * cu_q[b] of its cache (after pkv_rope_append_varlen: the cache, the earlier
+ * new tokens and itself), bf16 pools (PKV_ERR_UNSUPPORTED for E4M3).  A plan
+ * kernel cuts each request's new tokens into blocks of 16 / G tokens (the G x
+ * 16/G query rows of a block and kv head are one 16-row mma), each block
+ * streams its prefix of the cache once for its tokens.  The context holds
+ * room for 4 x max_batch blocks (at most 8192): a call with batch +
+ * ceil(n_tokens / (16 / G)) above that returns PKV_ERR_UNSUPPORTED without
+ * launching; lengths past the block table zero the affected tokens' output
+ * and set the error word, as for pkv_decode_attn. */
+pkv_status pkv_decode_attn_varlen(pkv_ctx* ctx, const void* q, const void* k_pool, const void* v_pool,
+                                  const int32_t* block_tables, int bt_stride, const int32_t* seq_lens,
+                                  const int32_t* cu_q, int batch, int n_tokens, void* out,
+                                  cudaStream_t stream);
+
 /* Step part 1 from the layer input: the QKV projection of the new tokens
  * fused with RoPE and the append ("Scaling TensorRT-LLM: Kernel Fusion and
  * Inflight Batching in Production", section "What Gets Fused").  x is the

@@ -242,6 +242,51 @@ def decode_attn_tokens(cfg: OracleConfig, q, k_pool, v_pool, k_scale, v_scale, b
     return out, st
 
 
+# ---- several new tokens, a different number per request (varlen) ---------------
+#
+# Packed new tokens: cu_q [batch + 1], request b's tokens are rows
+# cu_q[b] .. cu_q[b+1] - 1, token i at position L_b + i - cu_q[b].  By
+# definition this is, request by request, the several-new-tokens case with
+# that request's own count, so the oracle is that composition ("Scaling
+# TensorRT-LLM: Kernel Fusion and Inflight Batching in Production", section
+# "What the Scheduler Actually Does": prefill chunks and decode tokens in one
+# batch).
+
+def rope_append_varlen(cfg: OracleConfig, q, k_new, v_new, k_pool, v_pool, k_scale, v_scale,
+                       block_tables, seq_lens, cu_q) -> int:
+    """In place, for q [n_tokens, Hq, d] and k_new / v_new [n_tokens, Hkv, d];
+    returns the OR of the per-request statuses."""
+    st = 0
+    for b in range(len(seq_lens)):
+        a, e = int(cu_q[b]), int(cu_q[b + 1])
+        if e <= a:
+            continue
+        qb = np.ascontiguousarray(q[a:e][None])
+        st |= rope_append_tokens(cfg, qb, np.ascontiguousarray(k_new[a:e][None]),
+                                 np.ascontiguousarray(v_new[a:e][None]), k_pool, v_pool, k_scale, v_scale,
+                                 np.ascontiguousarray(block_tables[b:b + 1]),
+                                 np.ascontiguousarray(seq_lens[b:b + 1]))
+        q[a:e] = qb[0]
+    return st
+
+
+def decode_attn_varlen(cfg: OracleConfig, q, k_pool, v_pool, k_scale, v_scale, block_tables, seq_lens,
+                       cu_q):
+    """fp64 output [n_tokens, Hq, d]; (out, OR of the per-request statuses)."""
+    out = np.zeros((q.shape[0], cfg.num_q_heads, cfg.head_dim), np.float64)
+    st = 0
+    for b in range(len(seq_lens)):
+        a, e = int(cu_q[b]), int(cu_q[b + 1])
+        if e <= a:
+            continue
+        o, s = decode_attn_tokens(cfg, np.ascontiguousarray(q[a:e][None]), k_pool, v_pool, k_scale, v_scale,
+                                  np.ascontiguousarray(block_tables[b:b + 1]),
+                                  np.ascontiguousarray(seq_lens[b:b + 1]))
+        out[a:e] = o[0]
+        st |= s
+    return out, st
+
+
 # ---- the QKV projection -------------------------------------------------------
 
 def project_bf16(x, w):

@@ -155,7 +155,8 @@ __device__ __forceinline__ Lookahead lookahead_fill(const AttnParams& p, const i
         const int kvh = (int)(r / ntb), tt = (int)(r % ntb);
         const int tok0 = tt * TT;
         const int lp = tok0 / p.P;
-        const int page = __ldg(&p.block_tables[(size_t)b * p.bt_stride + lp]);
+        const int brow = p.vmap ? __ldg(&p.vmap[b].x) : b;   // a virtual request reads its request's row
+        const int page = __ldg(&p.block_tables[(size_t)brow * p.bt_stride + lp]);
         if ((unsigned)page < (unsigned)p.num_pages) {
             la.valid = 1;
             la.row = (page * p.Hkv + kvh) * p.P + (tok0 - lp * p.P);

@@ -60,7 +60,8 @@ __global__ void __launch_bounds__(kCombineThreads, 2) combine_kernel(const AttnP
     const int b = pair / p.Hkv, kvh = pair - b * p.Hkv;
     const int W = __ldg(&p.meta[0]);
     const long long T = (long long)(unsigned)__ldg(&p.meta[1]) | ((long long)__ldg(&p.meta[2]) << 32);
-    if (T == 0 || b >= p.batch) return;
+    const int B = p.vmap ? min(__ldg(p.vcount), p.batch) : p.batch;   // requests, or virtual requests
+    if (T == 0 || b >= B) return;
     const int* prefix = p.meta + 4;
     const int nt = __ldg(&prefix[b + 1]) - __ldg(&prefix[b]);
     if (nt == 0) return;
@@ -185,11 +186,19 @@ __global__ void __launch_bounds__(kCombineThreads, 2) combine_kernel(const AttnP
             sum.z += v.z;
             sum.w += v.w;
         }
-        // row r = t G + h -> out[b][t][kvh G + h] (token-major output)
+        // row r = t G + h -> out[q0 + t][kvh G + h] (token-major output; q0 =
+        // the first q row of the request, or of the virtual request, whose
+        // tokens past its count are not stored)
         const int r = (4 * f) / D, col = 4 * f - r * D;
         const int t = r / G, h = r - t * G;
+        int q0 = b * p.q_len;
+        if (p.vmap) {
+            const int4 e = p.vmap[b];
+            if (t >= e.z) continue;
+            q0 = e.y;
+        }
         uint2* const dst = reinterpret_cast<uint2*>(
-            p.out + (((size_t)b * p.q_len + t) * p.Hq + (size_t)kvh * G + h) * D + col);
+            p.out + (((size_t)q0 + t) * p.Hq + (size_t)kvh * G + h) * D + col);
         *dst = make_uint2(pack_bf16(sum.x, sum.y), pack_bf16(sum.z, sum.w));
     }
 }

@@ -20,6 +20,16 @@
 // mbarriers fed by a 32-tile page-id lookahead, online softmax in log2 units,
 // partial (m, l, o) rows for pairs cut between ranges, merged afterwards by
 // the combine kernel (combine.cu).  bf16 pools only.
+//
+// Varlen calls (a different number of new tokens per request: chunked
+// prefill mixed with decode in one batch, "Scaling TensorRT-LLM: Kernel
+// Fusion and Inflight Batching in Production", section "What the Scheduler
+// Actually Does"; "TensorRT-LLM Guide", section "1. In-Flight Batching")
+// run the same kernel over virtual requests: a plan kernel cuts request b's
+// new tokens into blocks of q_len = 16 / G (the last may be shorter), and
+// block j becomes a request with L = L_b + j q_len cached tokens (the
+// earlier new tokens are already in the pages), its own q / out rows and the
+// block table row of b (AttnParams::vmap).
 #include "attn_common.cuh"
 
 namespace pkv {
@@ -28,11 +38,12 @@ namespace {
 using namespace dev;
 using namespace attn;
 
-// Query rows of (request b, kv head kvh) as mma A fragments: rows g (a0, a2)
-// and g + 8 (a1, a3) of the 16; row r = t G + h is head kvh G + h of new
-// token t, rows r >= R are zero.
+// Query rows of a (request, kv head kvh) pair whose new tokens are q rows
+// qrow0, qrow0 + 1, ... as mma A fragments: rows g (a0, a2) and g + 8 (a1,
+// a3) of the 16; row r = t G + h is head kvh G + h of new token t, rows
+// r >= R are zero.
 template <int D>
-__device__ __forceinline__ void load_q_rows(const AttnParams& p, int b, int kvh, int g, int c4, int R,
+__device__ __forceinline__ void load_q_rows(const AttnParams& p, int qrow0, int kvh, int g, int c4, int R,
                                             uint32_t (&qa)[D / 16][4])
 {
 #pragma unroll
@@ -40,7 +51,7 @@ __device__ __forceinline__ void load_q_rows(const AttnParams& p, int b, int kvh,
         const int r = g + 8 * half;
         const bool ok = r < R;
         const int t = ok ? r / p.G : 0, h = ok ? r - t * p.G : 0;
-        const __nv_bfloat16* qrow = p.q + (((size_t)b * p.q_len + t) * p.Hq + (size_t)kvh * p.G + h) * D;
+        const __nv_bfloat16* qrow = p.q + (((size_t)qrow0 + t) * p.Hq + (size_t)kvh * p.G + h) * D;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
             qa[ks][half] = ok ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * c4) : 0u;
@@ -64,8 +75,23 @@ decode_attn_tokens_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_
     __shared__ int s_bad;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int B = p.batch, Hkv = p.Hkv, S = p.stages, QL = p.q_len;
-    const int G = p.G, R = G * QL;
+    const int B = p.vmap ? min(__ldg(p.vcount), p.batch) : p.batch;   // requests, or virtual requests
+    const int Hkv = p.Hkv, S = p.stages, QL = p.q_len;
+    const int G = p.G, R = G * QL;                   // partial rows per pair
+    // (cached tokens before the first new token, new tokens, their first q /
+    // out row) of request (or virtual request) v
+    auto vinfo = [&](int v, int& L, int& nq, int& qrow0) {
+        if (p.vmap) {
+            const int4 e = p.vmap[v];
+            L = e.w;
+            nq = e.z;
+            qrow0 = e.y;
+        } else {
+            L = p.seq_lens[v];
+            nq = QL;
+            qrow0 = v * QL;
+        }
+    };
 
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t stage_area = (raw + 1023u) & ~1023u;
@@ -88,9 +114,10 @@ decode_attn_tokens_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_
     const int lo = min(B, tid * per), hi = min(B, lo + per);
     int local = 0;
     for (int b = lo; b < hi; ++b) {
-        const int L = p.seq_lens[b];
-        const bool ok = L >= 0 && (long long)L + QL <= cap;
-        const int nt = ok ? (L + QL + kTile - 1) / kTile : 0;
+        int L, nq, q0;
+        vinfo(b, L, nq, q0);
+        const bool ok = L >= 0 && (long long)L + nq <= cap;
+        const int nt = ok ? (L + nq + kTile - 1) / kTile : 0;
         if (!ok) s_bad = 1;
         prefix[b] = nt;
         local += nt;
@@ -112,15 +139,24 @@ decode_attn_tokens_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_
     }
     if (tid == NT - 1) prefix[B] = run;
     __syncthreads();
+    if (B < p.batch) {
+        // varlen: the page lookahead searches the prefix over p.batch entries
+        // (the plan's capacity); past the last virtual request they hold the
+        // total, which no search for a tile below it selects
+        const int tot = prefix[B];
+        for (int b = B + 1 + tid; b <= p.batch; b += NT) prefix[b] = tot;
+        __syncthreads();
+    }
 
     if (s_bad && blockIdx.x == 0) {
         // requests with an impossible length produce zeros and an error bit
         if (tid == 0) atomicOr(p.err, kErrLength);
         for (int b = warp; b < B; b += WARPS) {
-            const int L = p.seq_lens[b];
-            if (L >= 0 && (long long)L + QL <= cap) continue;
-            uint32_t* o32 = reinterpret_cast<uint32_t*>(p.out + (size_t)b * QL * p.Hq * D);
-            for (int i = lane; i < QL * p.Hq * D / 2; i += 32) o32[i] = 0u;
+            int L, nq, q0;
+            vinfo(b, L, nq, q0);
+            if (L >= 0 && (long long)L + nq <= cap) continue;
+            uint32_t* o32 = reinterpret_cast<uint32_t*>(p.out + (size_t)q0 * p.Hq * D);
+            for (int i = lane; i < nq * p.Hq * D / 2; i += 32) o32[i] = 0u;
         }
     }
 
@@ -207,9 +243,8 @@ decode_attn_tokens_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_
     const int mi = lane >> 3, ri = lane & 7;        // ldmatrix: matrix index, row
     const int tokK = ((mi >> 1) << 3) + ri;         // token row addressed for K
     const int tokV = ((mi & 1) << 3) + ri;          // token row addressed for V (trans)
-    // new token of rows g and g + 8 (rows >= R see no token)
-    const int trow0 = g < R ? g / G : -1;
-    const int trow1 = g + 8 < R ? (g + 8) / G : -1;
+    // the current pair: its first q / out row, its rows (G x its new tokens)
+    int cur_q0 = 0, Rv = R;
 
     float o[NTD][4];
     uint32_t qa[KSTEPS][4];
@@ -242,11 +277,15 @@ decode_attn_tokens_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_
         }
         if (ctt == 0 || k == 0) {
             // start of a (request, kv head) pair or of this range
-            load_q_rows<D>(p, cb, ckvh, g, c4, R, qa);
-            const int n0 = p.seq_lens[cb] + 1;   // tokens visible to new token 0
-            lim[0] = trow0 >= 0 ? n0 + trow0 : 0;
-            lim[1] = trow1 >= 0 ? n0 + trow1 : 0;
-            n_max = n0 + QL - 1;
+            int L, nq;
+            vinfo(cb, L, nq, cur_q0);
+            Rv = G * nq;
+            load_q_rows<D>(p, cur_q0, ckvh, g, c4, Rv, qa);
+            const int n0 = L + 1;                // tokens visible to new token 0
+            // new token of rows g and g + 8 (rows >= Rv see no token)
+            lim[0] = g < Rv ? n0 + g / G : 0;
+            lim[1] = g + 8 < Rv ? n0 + (g + 8) / G : 0;
+            n_max = n0 + nq - 1;
 #pragma unroll
             for (int nt = 0; nt < NTD; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
             m_run[0] = m_run[1] = -INFINITY;
@@ -362,12 +401,12 @@ decode_attn_tokens_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
                 const int r = g + 8 * hf;
-                if (r >= R) continue;
+                if (r >= Rv) continue;
                 if (whole) {
                     const int t = r / G, h = r - t * G;
                     const float inv = 1.f / lsum[hf];
                     uint32_t* dst = reinterpret_cast<uint32_t*>(
-                        p.out + (((size_t)cb * QL + t) * p.Hq + (size_t)ckvh * G + h) * D);
+                        p.out + (((size_t)cur_q0 + t) * p.Hq + (size_t)ckvh * G + h) * D);
 #pragma unroll
                     for (int nt = 0; nt < NTD; ++nt)
                         dst[(8 * nt + 2 * c4) >> 1] = pack_bf16(o[nt][2 * hf] * inv, o[nt][2 * hf + 1] * inv);
@@ -437,6 +476,72 @@ cudaError_t prepare_tokens_t(int num_sms, int max_batch, AttnLaunch* out)
 }
 
 }  // namespace
+
+namespace {
+
+// One CTA: request b's new tokens (cu_q[b + 1] - cu_q[b] of them) cut into
+// blocks of `block`; vmap[v] = {b, first q row, tokens, L_b + offset of the
+// block}, v counted in request order (an exclusive scan of the blocks per
+// request).  More than vmax blocks, or a negative token count, set kErrLength
+// (the surplus is dropped).
+__global__ void __launch_bounds__(1024) varlen_plan_kernel(const int32_t* __restrict__ cu_q,
+                                                           const int32_t* __restrict__ seq_lens, int batch,
+                                                           int block, int vmax, int4* __restrict__ vmap,
+                                                           int* __restrict__ vcount, int* __restrict__ err)
+{
+    __shared__ int s_warp[32];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+    const int per = (batch + (int)blockDim.x - 1) / (int)blockDim.x;
+    const int lo = min(batch, tid * per), hi = min(batch, lo + per);
+    int local = 0;
+    for (int b = lo; b < hi; ++b) {
+        const int q = cu_q[b + 1] - cu_q[b];
+        local += q > 0 ? (q + block - 1) / block : 0;
+    }
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    int run = incl - local;
+    for (int w2 = 0; w2 < warp; ++w2) run += s_warp[w2];
+    for (int b = lo; b < hi; ++b) {
+        const int a = cu_q[b], q = cu_q[b + 1] - a;
+        if (q < 0) {
+            atomicOr(err, kErrLength);
+            continue;
+        }
+        const long long L = seq_lens[b];
+        for (int j = 0; (long long)j * block < q; ++j) {
+            const long long pos = L + (long long)j * block;
+            if (run < vmax)
+                vmap[run] = make_int4(b, a + j * block, min(block, q - j * block),
+                                      (L < 0 || pos > 0x7fffffffll) ? -1 : (int)pos);
+            ++run;
+        }
+    }
+    if (tid == 0) {
+        int total = 0;
+        for (int w2 = 0; w2 < nwarps; ++w2) total += s_warp[w2];
+        if (total > vmax) {
+            atomicOr(err, kErrLength);
+            total = vmax;
+        }
+        *vcount = total;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_varlen_plan(const int32_t* cu_q, const int32_t* seq_lens, int batch, int block, int vmax,
+                               int4* vmap, int* vcount, int* err, cudaStream_t stream)
+{
+    varlen_plan_kernel<<<1, 1024, 0, stream>>>(cu_q, seq_lens, batch, block, vmax, vmap, vcount, err);
+    return cudaGetLastError();
+}
 
 cudaError_t attn_tokens_prepare(int head_dim, int num_sms, int max_batch, AttnLaunch* out)
 {

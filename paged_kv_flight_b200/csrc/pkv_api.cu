@@ -29,6 +29,9 @@ struct pkv_ctx {
     int* d_err;
     int* d_claim;         // chunk counter of the attention's dynamic tail
     int* d_meta;
+    int vmax;             // virtual requests a varlen attention call may have (bf16 pools)
+    int4* d_vmap;         // [vmax] the varlen plan
+    int* d_vcount;
     float* d_part_o;
     float* d_part_ml;
     const void* tm_k_ptr;
@@ -177,7 +180,10 @@ pkv_status pkv_create(const pkv_config* cfg, pkv_ctx** out)
         free(ctx);
         return PKV_ERR_CUDA;
     }
-    if (!fp8 && pkv::attn_tokens_prepare(cfg->head_dim, ctx->num_sms, cfg->max_batch, &ctx->attn_tok) != cudaSuccess) {
+    // varlen calls cut requests into virtual ones: room for 4 per request
+    ctx->vmax = fp8 ? 0 : std::min(4 * cfg->max_batch, pkv::kMaxBatch);
+    if (!fp8 && pkv::attn_tokens_prepare(cfg->head_dim, ctx->num_sms, std::max(cfg->max_batch, ctx->vmax),
+                                         &ctx->attn_tok) != cudaSuccess) {
         free(ctx);
         return PKV_ERR_CUDA;
     }
@@ -193,10 +199,11 @@ pkv_status pkv_create(const pkv_config* cfg, pkv_ctx** out)
     const size_t units = pkv::max_units(ctx->attn.ctas * pkv::kAttnWarps, pkv::kMaxTailChunks);
     const size_t rows_units = std::max(units * ctx->G, (size_t)ctx->attn.ctas * pkv::kAttnWarps * pkv::kMaxTokenRows);
     const size_t b_err = 256;
-    const size_t b_cnt = ((size_t)(cfg->max_batch + 8) * sizeof(int) + 255) & ~(size_t)255;
+    const size_t b_cnt = ((size_t)(std::max(cfg->max_batch, ctx->vmax) + 8) * sizeof(int) + 255) & ~(size_t)255;
     const size_t b_po = 2 * rows_units * cfg->head_dim * sizeof(float);
     const size_t b_pml = 2 * rows_units * 2 * sizeof(float);
-    ctx->ws_bytes = b_err + b_cnt + b_po + b_pml;
+    const size_t b_vm = (size_t)ctx->vmax * sizeof(int4) + 256;   // varlen plan + its count
+    ctx->ws_bytes = b_err + b_cnt + b_po + b_pml + b_vm;
     if (cudaMalloc(&ctx->ws, ctx->ws_bytes) != cudaSuccess) {
         cudaGetLastError();
         free(ctx);
@@ -209,6 +216,8 @@ pkv_status pkv_create(const pkv_config* cfg, pkv_ctx** out)
     ctx->d_meta = reinterpret_cast<int*>(base + b_err);
     ctx->d_part_o = reinterpret_cast<float*>(base + b_err + b_cnt);
     ctx->d_part_ml = reinterpret_cast<float*>(base + b_err + b_cnt + b_po);
+    ctx->d_vcount = reinterpret_cast<int*>(base + b_err + b_cnt + b_po + b_pml);
+    ctx->d_vmap = reinterpret_cast<int4*>(base + b_err + b_cnt + b_po + b_pml + 256);
     if (cudaMemset(ctx->ws, 0, b_err + b_cnt) != cudaSuccess) {
         cudaFree(ctx->ws);
         free(ctx);
@@ -334,18 +343,17 @@ pkv_status pkv_rope_append_tokens(pkv_ctx* ctx, void* q, const void* k_new, cons
     return pkv::launch_rope_append(p, stream) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
-pkv_status pkv_decode_attn_tokens(pkv_ctx* ctx, const void* q, const void* k_pool, const void* v_pool,
-                                  const float* k_scale, const float* v_scale, const int32_t* block_tables,
-                                  int bt_stride, const int32_t* seq_lens, int batch, int q_len, void* out,
-                                  cudaStream_t stream)
-{
-    pkv_status st = check_call(ctx, batch, bt_stride, k_pool, v_pool, k_scale, v_scale, block_tables, seq_lens);
-    if (st != PKV_OK || batch == 0) return st;
-    if (q_len < 1) return PKV_ERR_INVALID_ARG;
-    if (ctx->cfg.kv_dtype != PKV_KV_BF16) return PKV_ERR_UNSUPPORTED;
-    if ((long long)ctx->G * q_len > pkv::kMaxTokenRows) return PKV_ERR_UNSUPPORTED;
-    if (!q || !out || !aligned16(q) || !aligned16(out)) return PKV_ERR_INVALID_ARG;
+}  // extern "C"
 
+namespace {
+
+// The several-new-tokens attention launch, for the uniform calls (vmap null:
+// `batch` requests of q_len tokens) and the varlen ones (batch = the plan's
+// capacity, q_len = the block length).
+pkv_status attn_tokens_launch(pkv_ctx* ctx, const void* q, const void* k_pool, const void* v_pool,
+                              const int32_t* block_tables, int bt_stride, const int32_t* seq_lens, int batch,
+                              int q_len, const int4* vmap, const int* vcount, void* out, cudaStream_t stream)
+{
     if (ctx->tm_k_ptr != k_pool) {
         if (!encode_pool(ctx, k_pool, &ctx->tmk)) return PKV_ERR_CUDA;
         ctx->tm_k_ptr = k_pool;
@@ -379,9 +387,89 @@ pkv_status pkv_decode_attn_tokens(pkv_ctx* ctx, const void* q, const void* k_poo
     p.workers = ctx->workers;
     p.tail_chunks = 0;
     p.q_len = q_len;
+    p.vmap = vmap;
+    p.vcount = vcount;
     const cudaError_t e = pkv::launch_decode_attn_tokens(p, ctx->tmk, ctx->tmv, ctx->cfg.head_dim, ctx->attn_tok,
                                                          stream);
     return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+pkv_status pkv_decode_attn_tokens(pkv_ctx* ctx, const void* q, const void* k_pool, const void* v_pool,
+                                  const float* k_scale, const float* v_scale, const int32_t* block_tables,
+                                  int bt_stride, const int32_t* seq_lens, int batch, int q_len, void* out,
+                                  cudaStream_t stream)
+{
+    pkv_status st = check_call(ctx, batch, bt_stride, k_pool, v_pool, k_scale, v_scale, block_tables, seq_lens);
+    if (st != PKV_OK || batch == 0) return st;
+    if (q_len < 1) return PKV_ERR_INVALID_ARG;
+    if (ctx->cfg.kv_dtype != PKV_KV_BF16) return PKV_ERR_UNSUPPORTED;
+    if ((long long)ctx->G * q_len > pkv::kMaxTokenRows) return PKV_ERR_UNSUPPORTED;
+    if (!q || !out || !aligned16(q) || !aligned16(out)) return PKV_ERR_INVALID_ARG;
+    return attn_tokens_launch(ctx, q, k_pool, v_pool, block_tables, bt_stride, seq_lens, batch, q_len, nullptr,
+                              nullptr, out, stream);
+}
+
+pkv_status pkv_rope_append_varlen(pkv_ctx* ctx, void* q, const void* k_new, const void* v_new, void* k_pool,
+                                  void* v_pool, const float* k_scale, const float* v_scale,
+                                  const int32_t* block_tables, int bt_stride, const int32_t* seq_lens,
+                                  const int32_t* cu_q, int batch, int n_tokens, cudaStream_t stream)
+{
+    pkv_status st = check_call(ctx, batch, bt_stride, k_pool, v_pool, k_scale, v_scale, block_tables, seq_lens);
+    if (st != PKV_OK) return st;
+    if (n_tokens < 0) return PKV_ERR_INVALID_ARG;
+    if (batch == 0 || n_tokens == 0) return PKV_OK;
+    if (!cu_q || !aligned16(cu_q)) return PKV_ERR_INVALID_ARG;
+    if (!q || !k_new || !v_new || !aligned16(q) || !aligned16(k_new) || !aligned16(v_new))
+        return PKV_ERR_INVALID_ARG;
+
+    pkv::RopeParams p;
+    p.q = static_cast<__nv_bfloat16*>(q);
+    p.k_new = static_cast<const __nv_bfloat16*>(k_new);
+    p.v_new = static_cast<const __nv_bfloat16*>(v_new);
+    p.k_pool = k_pool;
+    p.v_pool = v_pool;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
+    p.block_tables = block_tables;
+    p.seq_lens = seq_lens;
+    p.err = ctx->d_err;
+    p.rope_base = ctx->cfg.rope_base;
+    p.batch = batch;
+    p.bt_stride = bt_stride;
+    p.Hq = ctx->cfg.num_q_heads;
+    p.Hkv = ctx->cfg.num_kv_heads;
+    p.D = ctx->cfg.head_dim;
+    p.P = ctx->cfg.page_size;
+    p.num_pages = ctx->cfg.num_pages;
+    p.fp8 = ctx->cfg.kv_dtype == PKV_KV_FP8_E4M3;
+    p.q_len = 1;
+    p.cu_q = cu_q;
+    p.n_tokens = n_tokens;
+    return pkv::launch_rope_append(p, stream) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+pkv_status pkv_decode_attn_varlen(pkv_ctx* ctx, const void* q, const void* k_pool, const void* v_pool,
+                                  const int32_t* block_tables, int bt_stride, const int32_t* seq_lens,
+                                  const int32_t* cu_q, int batch, int n_tokens, void* out, cudaStream_t stream)
+{
+    if (ctx && ctx->cfg.kv_dtype != PKV_KV_BF16) return PKV_ERR_UNSUPPORTED;   // bf16 pools only
+    pkv_status st = check_call(ctx, batch, bt_stride, k_pool, v_pool, nullptr, nullptr, block_tables, seq_lens);
+    if (st != PKV_OK) return st;
+    if (n_tokens < 0) return PKV_ERR_INVALID_ARG;
+    if (batch == 0 || n_tokens == 0) return PKV_OK;
+    if (!cu_q || !aligned16(cu_q) || !q || !out || !aligned16(q) || !aligned16(out)) return PKV_ERR_INVALID_ARG;
+    // blocks of `block` new tokens: G x block <= 16 query rows per (block, kv head)
+    const int block = pkv::kMaxTokenRows / ctx->G;
+    if ((long long)batch + (n_tokens + block - 1) / block > ctx->vmax) return PKV_ERR_UNSUPPORTED;
+    if (pkv::launch_varlen_plan(cu_q, seq_lens, batch, block, ctx->vmax, ctx->d_vmap, ctx->d_vcount, ctx->d_err,
+                                stream) != cudaSuccess)
+        return PKV_ERR_CUDA;
+    return attn_tokens_launch(ctx, q, k_pool, v_pool, block_tables, bt_stride, seq_lens, ctx->vmax, block,
+                              ctx->d_vmap, ctx->d_vcount, out, stream);
 }
 
 pkv_status pkv_qkv_pack_weight(pkv_ctx* ctx, const void* w_qkv, int hidden, void* w_tiled, cudaStream_t stream)

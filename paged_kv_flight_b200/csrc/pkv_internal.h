@@ -71,6 +71,10 @@ struct RopeParams {
     double rope_base;
     int batch, bt_stride, Hq, Hkv, D, P, num_pages, fp8;
     int q_len;            // new tokens per request, at positions L_b .. L_b + q_len - 1
+    // varlen: token i of request b (cu_q[b] <= i < cu_q[b + 1]) sits at
+    // position L_b + i - cu_q[b]; the grid covers n_tokens rows; q_len unused
+    const int32_t* cu_q = nullptr;
+    int n_tokens = 0;
 };
 
 struct AttnParams {
@@ -91,6 +95,13 @@ struct AttnParams {
     int workers;          // 0: automatic
     int tail_chunks;      // largest K (chunks per warp tail); 0: static split only
     int q_len;            // new tokens per request (1: one new token); partial rows = G x q_len
+    // varlen (several new tokens, a different count per request): the kernel
+    // works on virtual requests, blocks of at most q_len new tokens of one
+    // request; vmap[v] = {request, first token row, tokens, position of the
+    // first}, *vcount of them (at most batch), both written on the device by
+    // the varlen plan; null for the other calls
+    const int4* vmap = nullptr;
+    const int* vcount = nullptr;
 };
 
 cudaError_t launch_rope_append(const RopeParams& p, cudaStream_t stream);
@@ -110,6 +121,11 @@ cudaError_t launch_decode_attn(const AttnParams& p, const CUtensorMap& tmk, cons
 // pools, G x q_len <= 16): shape of its launch and the launch itself
 // (attention, then the combine).
 cudaError_t attn_tokens_prepare(int head_dim, int num_sms, int max_batch, AttnLaunch* out);
+// The virtual requests of a varlen call: blocks of `block` new tokens (the
+// last of a request may be shorter) of requests with cu_q[b + 1] > cu_q[b];
+// writes vmap and the count (capped at vmax; more sets kErrLength).
+cudaError_t launch_varlen_plan(const int32_t* cu_q, const int32_t* seq_lens, int batch, int block, int vmax,
+                               int4* vmap, int* vcount, int* err, cudaStream_t stream);
 cudaError_t launch_decode_attn_tokens(const AttnParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
                                       int head_dim, const AttnLaunch& L, cudaStream_t stream);
 

@@ -51,7 +51,22 @@ __global__ void __launch_bounds__(kRopeThreads) rope_append_kernel(const RopePar
     __shared__ double s_cos[HALF], s_sin[HALF];
 
     const int bt = blockIdx.x;               // (request, new token) row of q, k_new, v_new
-    const int b = bt / p.q_len, t = bt - b * p.q_len;
+    int b, t;
+    if (p.cu_q) {
+        // varlen: the request whose rows [cu_q[b], cu_q[b + 1]) hold row bt
+        // (the last b with cu_q[b] <= bt: requests with no new token are skipped)
+        int lo = 0, hi = p.batch;
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (p.cu_q[mid] <= bt) lo = mid;
+            else hi = mid;
+        }
+        b = lo;
+        t = bt - p.cu_q[b];
+    } else {
+        b = bt / p.q_len;
+        t = bt - b * p.q_len;
+    }
     const int rows = p.Hq + p.Hkv;
     const int it = blockIdx.y * kRopeThreads + threadIdx.x;
     const bool active = it < rows * PIECES;
@@ -76,7 +91,7 @@ __global__ void __launch_bounds__(kRopeThreads) rope_append_kernel(const RopePar
 
     const int L0 = p.seq_lens[b];
     const long long Lt = (long long)L0 + t;  // position of this new token
-    const bool len_ok = L0 >= 0 && Lt < (long long)p.bt_stride * p.P;
+    const bool len_ok = L0 >= 0 && Lt >= 0 && Lt < (long long)p.bt_stride * p.P;   // (t < 0: bad cu_q)
     const int L = (int)Lt;
     const int page = len_ok ? p.block_tables[(size_t)b * p.bt_stride + L / p.P] : -1;
     if (!len_ok) {
@@ -165,7 +180,8 @@ __global__ void __launch_bounds__(kRopeThreads) rope_append_kernel(const RopePar
 cudaError_t launch_rope_append(const RopeParams& p, cudaStream_t stream)
 {
     const int items = (p.Hq + p.Hkv) * (p.D / 16);
-    const dim3 grid(p.batch * p.q_len, (items + kRopeThreads - 1) / kRopeThreads), block(kRopeThreads);
+    const int rows = p.cu_q ? p.n_tokens : p.batch * p.q_len;
+    const dim3 grid(rows, (items + kRopeThreads - 1) / kRopeThreads), block(kRopeThreads);
     if (p.D == 128) {
         if (p.fp8) rope_append_kernel<128, true><<<grid, block, 0, stream>>>(p);
         else rope_append_kernel<128, false><<<grid, block, 0, stream>>>(p);

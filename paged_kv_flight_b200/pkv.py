@@ -46,7 +46,7 @@ EXPORTS = ("pkv_create", "pkv_rope_append", "pkv_decode_attn", "pkv_destroy", "p
            "pkv_pages_release", "pkv_pages_block_table", "pkv_pages_seq_lens", "pkv_pages_active",
            "pkv_pages_refcount", "pkv_pages_free_count", "pkv_pages_take_changes", "pkv_qkv_rope_append",
            "pkv_qkv_pack_weight", "pkv_set_qkv_split", "pkv_qkv_launch_shape",
-           "pkv_table_sync")
+           "pkv_table_sync", "pkv_rope_append_varlen", "pkv_decode_attn_varlen")
 
 
 class pkv_config(C.Structure):
@@ -101,6 +101,10 @@ lib.pkv_qkv_launch_shape.argtypes = [_V, C.c_int, C.c_int, _V]
 lib.pkv_qkv_launch_shape.restype = C.c_int
 lib.pkv_table_sync.argtypes = [_V, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, _V, _V, _V, _V]
 lib.pkv_table_sync.restype = C.c_int
+lib.pkv_rope_append_varlen.argtypes = [_V, _V, _V, _V, _V, _V, _V, _V, _V, C.c_int, _V, _V, C.c_int, C.c_int, _V]
+lib.pkv_rope_append_varlen.restype = C.c_int
+lib.pkv_decode_attn_varlen.argtypes = [_V, _V, _V, _V, _V, C.c_int, _V, _V, C.c_int, C.c_int, _V, _V]
+lib.pkv_decode_attn_varlen.restype = C.c_int
 lib.pkv_set_tail_chunks.argtypes = [_V, C.c_int]
 lib.pkv_set_tail_chunks.restype = C.c_int
 lib.pkv_workspace_bytes.argtypes = [_V]
@@ -331,6 +335,36 @@ PKV_W_ROWS, PKV_W_TILED = 0, 1
 def pkv_set_qkv_split(ctx, split: int, check: bool = True) -> int:
     """CTAs (a cluster) per head over the hidden dimension: 1 .. 4, 0 = automatic."""
     return _done(lib.pkv_set_qkv_split(ctx, int(split)), "pkv_set_qkv_split", check)
+
+
+def pkv_rope_append_varlen(ctx, q, k_new, v_new, k_pool, v_pool, k_scale, v_scale, block_tables, seq_lens,
+                           cu_q, batch: int | None = None, bt_stride: int | None = None, stream=None,
+                           check: bool = True) -> int:
+    """q [n_tokens, Hq, d] (rotated in place), k_new / v_new [n_tokens, Hkv, d];
+    cu_q [batch + 1] int32: request b's new tokens are rows cu_q[b] .. cu_q[b+1]-1."""
+    if batch is None:
+        batch = int(seq_lens.shape[0])
+    if bt_stride is None:
+        bt_stride = int(block_tables.shape[1])
+    st = lib.pkv_rope_append_varlen(ctx, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_pool), _ptr(v_pool),
+                                    _ptr(k_scale), _ptr(v_scale), _ptr(block_tables), int(bt_stride),
+                                    _ptr(seq_lens), _ptr(cu_q), int(batch), int(q.shape[0]), _stream(stream))
+    return _done(st, "pkv_rope_append_varlen", check)
+
+
+def pkv_decode_attn_varlen(ctx, q, k_pool, v_pool, block_tables, seq_lens, cu_q, out,
+                           batch: int | None = None, bt_stride: int | None = None, stream=None,
+                           check: bool = True) -> int:
+    """q / out [n_tokens, Hq, d]; token i of request b attends its cache up to
+    position L_b + i - cu_q[b]."""
+    if batch is None:
+        batch = int(seq_lens.shape[0])
+    if bt_stride is None:
+        bt_stride = int(block_tables.shape[1])
+    st = lib.pkv_decode_attn_varlen(ctx, _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(block_tables), int(bt_stride),
+                                    _ptr(seq_lens), _ptr(cu_q), int(batch), int(q.shape[0]), _ptr(out),
+                                    _stream(stream))
+    return _done(st, "pkv_decode_attn_varlen", check)
 
 
 def pkv_table_sync(upload, n_changes: int, batch: int, table, bt_out, lens_out, page_size: int, stream=None,

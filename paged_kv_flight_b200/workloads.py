@@ -237,5 +237,22 @@ def make(name: str, device="cpu", offset: int = 0) -> Workload:
                  seed, device=device, num_pages=64 if name == "tiny" else None, q_len=s.get("q_len", 1))
 
 
+def make_mixed(device="cpu", offset: int = 0, chunk: int = 64, prefills: int = 8):
+    """Chunked prefill mixed with decode on the llama8b batch: the llama8b
+    lengths and shapes, `prefills` seeded requests take a chunk of `chunk` new
+    tokens, the others one.  Returns (workload with a token axis of `chunk`,
+    new tokens per request); the varlen step uses the first q_lens[b] tokens
+    of request b."""
+    s = _SHAPES["llama8b"]
+    seed = config_seed("llama8b", offset) + 31
+    rng = np.random.default_rng(seed)
+    lengths = draw_lengths("llama8b", np.random.default_rng(config_seed("llama8b", offset)))
+    q_lens = np.ones(len(lengths), np.int64)
+    q_lens[rng.choice(len(lengths), size=prefills, replace=False)] = chunk
+    w = build("mixed", s["Hq"], s["Hkv"], s["d"], s["P"], s["kv_fp8"], s["base"], lengths, seed, device=device,
+              q_len=chunk)
+    return w, q_lens
+
+
 def shape_of(name: str) -> dict:
     return dict(_SHAPES[name])

@@ -59,3 +59,18 @@ def bf16_ordinal(bits: np.ndarray) -> np.ndarray:
 
 def f64_of_bf16_tensor(t: torch.Tensor) -> np.ndarray:
     return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def varlen_host(w: Workload, q_lens) -> dict:
+    """Host inputs of a varlen step from a several-new-tokens workload (token
+    axis of at least max(q_lens), pages for them): request b keeps its first
+    q_lens[b] new tokens, packed in request order, and cu_q [batch + 1]."""
+    h = host_inputs(w)
+    q_lens = np.asarray(q_lens, np.int64)
+    assert len(q_lens) == w.batch and (q_lens <= w.q_len).all()
+    cu = np.zeros(w.batch + 1, np.int32)
+    cu[1:] = np.cumsum(q_lens)
+    for key in ("q", "k_new", "v_new"):
+        h[key] = np.ascontiguousarray(np.concatenate([h[key][b, :int(q)] for b, q in enumerate(q_lens)]))
+    h["cu_q"] = cu
+    return h

@@ -80,3 +80,17 @@ def test_null_context_and_status_strings(pkv):
     for s in range(7):
         assert pkv.pkv_status_str(s) and pkv.pkv_status_str(s) != "unknown status"
     assert pkv.pkv_status_str(99) == "unknown status"
+
+
+def test_table_sync_rejects_bad_sizes_without_touching_the_device():
+    """Argument checks of pkv_table_sync run on the host before any launch."""
+    import torch
+    from paged_kv_flight_b200 import pkv
+    t = torch.zeros(4, 8, dtype=torch.int32)
+    up = torch.zeros(64, dtype=torch.int32)
+    bt, ln = torch.zeros(4, 8, dtype=torch.int32), torch.zeros(4, dtype=torch.int32)
+    call = lambda n, b, P: pkv.pkv_table_sync(up, n, b, t, bt, ln, P, stream=0, check=False)   # noqa: E731
+    assert call(-1, 1, 16) == pkv.PKV_ERR_INVALID_ARG
+    assert call(0, 5, 16) == pkv.PKV_ERR_INVALID_ARG      # batch above the table's rows
+    assert call(0, 1, 0) == pkv.PKV_ERR_INVALID_ARG       # page size
+    assert call(0, 0, 16) == pkv.PKV_OK                    # nothing to do

@@ -1,0 +1,145 @@
+"""GPU parity of the varlen step (pkv_rope_append_varlen +
+pkv_decode_attn_varlen): a different number of new tokens per request,
+packed, as in chunked prefill mixed with decode ("Scaling TensorRT-LLM:
+Kernel Fusion and Inflight Batching in Production", section "What the
+Scheduler Actually Does").  Against the oracle on the same inputs: appended V
+bit-exact and K / q within 1 bf16 ulp at every landing slot, every other pool
+byte untouched, attention within the bf16 tolerances; the split does not
+matter beyond rounding; host rejections and device range errors."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from paged_kv_flight_b200 import workloads
+from tests import _gpu
+from tests._util import bf16_ordinal, bits16, oracle_cfg, varlen_host
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    # name, Hq, Hkv, d, P, lengths, new tokens per request
+    ("g4_d128_p32", 32, 8, 128, 32, [100, 0, 517, 1200, 33, 64, 2000, 15], [1, 20, 1, 64, 0, 3, 1, 37]),
+    ("g8_d128_p16", 64, 8, 128, 16, [5, 300, 1000], [7, 1, 33]),
+    ("g2_d64_p64", 8, 4, 64, 64, [0, 63, 64, 200], [16, 1, 9, 65]),
+    ("g1_d64_p16", 4, 4, 64, 16, [10, 40, 0], [50, 1, 1]),
+]
+
+
+@pytest.fixture(scope="module")
+def pkv():
+    from paged_kv_flight_b200 import pkv as mod
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return mod
+
+
+def _dev_bits(a):
+    return torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16).contiguous()
+
+
+def _setup(case, seed=41):
+    name, Hq, Hkv, d, P, lengths, q_lens = case
+    w = workloads.build(name, Hq, Hkv, d, P, False, 5e5 if d == 128 else 1e4, lengths, seed, device="cpu",
+                        q_len=max(q_lens))
+    h = varlen_host(w, q_lens)
+    return w, h, q_lens
+
+
+def _device(h):
+    return dict(q=_dev_bits(h["q"]), k_new=_dev_bits(h["k_new"]), v_new=_dev_bits(h["v_new"]),
+                k_pool=_dev_bits(h["k_pool"]), v_pool=_dev_bits(h["v_pool"]),
+                block_tables=torch.from_numpy(h["block_tables"]).cuda(),
+                seq_lens=torch.from_numpy(h["seq_lens"]).cuda(), cu_q=torch.from_numpy(h["cu_q"]).cuda())
+
+
+def _oracle(w, h):
+    ho = {k: (v.copy() if isinstance(v, np.ndarray) else v) for k, v in h.items()}
+    cfg = oracle_cfg(w)
+    assert oracle.rope_append_varlen(cfg, ho["q"], ho["k_new"], ho["v_new"], ho["k_pool"], ho["v_pool"], None,
+                                     None, ho["block_tables"], ho["seq_lens"], ho["cu_q"]) == 0
+    out, st = oracle.decode_attn_varlen(cfg, ho["q"], ho["k_pool"], ho["v_pool"], None, None, ho["block_tables"],
+                                        ho["seq_lens"], ho["cu_q"])
+    assert st == 0
+    return ho, out
+
+
+def _step(pkv, ctx, dv):
+    out = torch.full_like(dv["q"], float("nan"))
+    pkv.pkv_rope_append_varlen(ctx, dv["q"], dv["k_new"], dv["v_new"], dv["k_pool"], dv["v_pool"], None, None,
+                               dv["block_tables"], dv["seq_lens"], dv["cu_q"])
+    pkv.pkv_decode_attn_varlen(ctx, dv["q"], dv["k_pool"], dv["v_pool"], dv["block_tables"], dv["seq_lens"],
+                               dv["cu_q"], out)
+    return out
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: c[0])
+def test_varlen_step_matches_oracle(pkv, case):
+    w, h, q_lens = _setup(case)
+    ho, ref = _oracle(w, h)
+    dv = _device(h)
+    ctx = _gpu.make_ctx(pkv, w, max_batch=64)
+    try:
+        out = _step(pkv, ctx, dv)
+        assert pkv.pkv_check_device_error(ctx)[0] == pkv.PKV_OK
+    finally:
+        pkv.pkv_destroy(ctx)
+    # q rotated in place: within 1 ulp; pools: V bit-exact, K within 1 ulp, nothing else changed
+    assert np.abs(bf16_ordinal(bits16(dv["q"])) - bf16_ordinal(ho["q"])).max() <= 1
+    assert np.array_equal(bits16(dv["v_pool"]), ho["v_pool"])
+    assert np.abs(bf16_ordinal(bits16(dv["k_pool"])) - bf16_ordinal(ho["k_pool"])).max() <= 1
+    mx, mean, finite = _gpu.errors(out, ref)
+    assert finite and mx <= _gpu.TOL_BF16["max"] and mean <= _gpu.TOL_BF16["mean"], (mx, mean)
+
+
+def test_varlen_split_invariance(pkv):
+    w, h, _ = _setup(CASES[0], seed=43)
+    _, ref = _oracle(w, h)
+    outs = []
+    ctx = _gpu.make_ctx(pkv, w, max_batch=64)
+    try:
+        for workers in (1, 7, 0):
+            pkv.pkv_set_workers(ctx, workers)
+            outs.append(_step(pkv, ctx, _device(h)))
+            assert pkv.pkv_check_device_error(ctx)[0] == pkv.PKV_OK
+    finally:
+        pkv.pkv_destroy(ctx)
+    for o in outs:
+        mx, mean, finite = _gpu.errors(o, ref)
+        assert finite and mx <= _gpu.TOL_BF16["max"] and mean <= _gpu.TOL_BF16["mean"]
+
+
+def test_varlen_rejections_and_range_errors(pkv):
+    w, h, q_lens = _setup(CASES[1], seed=45)
+    dv = _device(h)
+    out = torch.empty_like(dv["q"])
+    ctx = _gpu.make_ctx(pkv, w, max_batch=4)          # room for 16 blocks of 2 tokens
+    try:
+        # 41 new tokens in blocks of 2 (G = 8): 3 + 21 blocks > 16
+        st = pkv.pkv_decode_attn_varlen(ctx, dv["q"], dv["k_pool"], dv["v_pool"], dv["block_tables"],
+                                        dv["seq_lens"], dv["cu_q"], out, check=False)
+        assert st == pkv.PKV_ERR_UNSUPPORTED
+    finally:
+        pkv.pkv_destroy(ctx)
+    ctx = _gpu.make_ctx(pkv, w, max_batch=64)
+    try:
+        bad = dv["seq_lens"].clone()
+        bad[1] = w.bt_stride * w.P                    # request 1's one token lies past its table
+        out = torch.full_like(dv["q"], 1.0)
+        pkv.pkv_decode_attn_varlen(ctx, dv["q"], dv["k_pool"], dv["v_pool"], dv["block_tables"], bad, dv["cu_q"],
+                                   out)
+        st, bits = pkv.pkv_check_device_error(ctx)
+        assert st == pkv.PKV_ERR_DEVICE_BOUNDS and bits & 1
+        i = int(h["cu_q"][1])
+        assert torch.count_nonzero(out[i].float()) == 0   # its token's output is zeros
+    finally:
+        pkv.pkv_destroy(ctx)
+    wf = workloads.build("vf", 8, 2, 64, 16, True, 1e4, [3, 9], 3, device="cpu")
+    ctx = _gpu.make_ctx(pkv, wf, max_batch=8)
+    try:
+        dvf = _gpu.to_device(wf)
+        cu = torch.tensor([0, 1, 2], dtype=torch.int32, device="cuda")
+        st = pkv.pkv_decode_attn_varlen(ctx, dvf["q"], dvf["k_pool"], dvf["v_pool"], dvf["block_tables"],
+                                        dvf["seq_lens"], cu, torch.empty_like(dvf["q"]), check=False)
+        assert st == pkv.PKV_ERR_UNSUPPORTED            # E4M3 pools: one-token or multi-token calls only
+    finally:
+        pkv.pkv_destroy(ctx)
