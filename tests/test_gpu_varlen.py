@@ -143,3 +143,30 @@ def test_varlen_rejections_and_range_errors(pkv):
         assert st == pkv.PKV_ERR_UNSUPPORTED            # E4M3 pools: one-token or multi-token calls only
     finally:
         pkv.pkv_destroy(ctx)
+
+
+def test_varlen_append_into_e4m3_pools(pkv):
+    """pkv_rope_append_varlen with E4M3 pools: V codes bit-exact, K codes
+    within one step, q within 1 ulp, nothing else changed."""
+    q_lens = [3, 0, 1, 9]
+    w = workloads.build("vl8", 8, 2, 128, 32, True, 5e5, [10, 4, 63, 100], 47, device="cpu", q_len=max(q_lens))
+    h = varlen_host(w, q_lens)
+    ho = {k: (v.copy() if isinstance(v, np.ndarray) else v) for k, v in h.items()}
+    assert oracle.rope_append_varlen(oracle_cfg(w), ho["q"], ho["k_new"], ho["v_new"], ho["k_pool"], ho["v_pool"],
+                                     ho["k_scale"], ho["v_scale"], ho["block_tables"], ho["seq_lens"],
+                                     ho["cu_q"]) == 0
+    dq, dk, dv_ = _dev_bits(h["q"]), _dev_bits(h["k_new"]), _dev_bits(h["v_new"])
+    kp = torch.from_numpy(h["k_pool"]).cuda()
+    vp = torch.from_numpy(h["v_pool"]).cuda()
+    ks = torch.from_numpy(h["k_scale"]).cuda()
+    vs = torch.from_numpy(h["v_scale"]).cuda()
+    ctx = _gpu.make_ctx(pkv, w, max_batch=8)
+    try:
+        pkv.pkv_rope_append_varlen(ctx, dq, dk, dv_, kp, vp, ks, vs, torch.from_numpy(h["block_tables"]).cuda(),
+                                   torch.from_numpy(h["seq_lens"]).cuda(), torch.from_numpy(h["cu_q"]).cuda())
+        assert pkv.pkv_check_device_error(ctx)[0] == pkv.PKV_OK
+    finally:
+        pkv.pkv_destroy(ctx)
+    assert np.array_equal(vp.cpu().numpy(), ho["v_pool"])
+    assert np.abs(kp.cpu().numpy().astype(int) - ho["k_pool"].astype(int)).max() <= 1
+    assert np.abs(bf16_ordinal(bits16(dq)) - bf16_ordinal(ho["q"])).max() <= 1

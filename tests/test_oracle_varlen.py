@@ -105,3 +105,17 @@ def test_a_request_without_new_tokens_changes_nothing():
     a0, a2 = slice(0, 2), slice(6, 9)
     assert np.array_equal(out1[0:2], _run(w, varlen_host(w, [2, 4, 3]))[0][a0])
     assert np.array_equal(out1[2:5], _run(w, varlen_host(w, [2, 4, 3]))[0][a2])
+
+
+def test_e4m3_append_one_token_each_is_the_single_token_append():
+    w1 = workloads.build("onef", 8, 2, 64, 16, True, 1e4, [3, 17, 40, 0], 6, device="cpu")
+    h1 = host_inputs(w1)
+    hv = {k: (v.copy() if isinstance(v, np.ndarray) else v) for k, v in h1.items()}
+    cfg = oracle_cfg(w1)
+    assert oracle.rope_append(cfg, h1["q"], h1["k_new"], h1["v_new"], h1["k_pool"], h1["v_pool"], h1["k_scale"],
+                              h1["v_scale"], h1["block_tables"], h1["seq_lens"]) == 0
+    assert oracle.rope_append_varlen(cfg, hv["q"], hv["k_new"], hv["v_new"], hv["k_pool"], hv["v_pool"],
+                                     hv["k_scale"], hv["v_scale"], hv["block_tables"], hv["seq_lens"],
+                                     np.arange(w1.batch + 1, dtype=np.int32)) == 0
+    assert np.array_equal(h1["k_pool"], hv["k_pool"]) and np.array_equal(h1["v_pool"], hv["v_pool"])
+    assert np.array_equal(h1["q"], hv["q"])
