@@ -824,7 +824,7 @@ def run_mixed(args, rank, world, local_rank):
             "new_tokens_per_s": sum_over_ranks(float(n_tok)) / (step_ms * 1e-3),
             "streamed_bytes_per_launch": streamed,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
-                         "traffic": None, "kernel": "decode_attn_tokens_kernel<128> (varlen)",
+                         "traffic": recorded_traffic("mixed"), "kernel": "decode_attn_tokens_kernel<128> (varlen)",
                          "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)", "bytes_per_launch": by,
                          "note": "bytes = each request's cache once (the metric); a prefill chunk's blocks "
                                  "re-read their prefix, see streamed_bytes_per_launch"},
