@@ -50,6 +50,20 @@
  * page the new token lands in before the step; block-table entries past
  * ceil(n_b / P) are never read.
  *
+ * Beyond the step (each declared below with its own contract):
+ *   pkv_rope_append_tokens / pkv_decode_attn_tokens  several new tokens per
+ *       request, the same count for all (speculative verification);
+ *   pkv_rope_append_varlen / pkv_decode_attn_varlen  a count per request,
+ *       packed (chunked prefill mixed with decode);
+ *   pkv_qkv_rope_append, pkv_qkv_pack_weight         the QKV projection of
+ *       the new tokens on the tensor cores fused with RoPE and the append;
+ *   pkv_table_sync                                   the device side of the
+ *       host page allocator of pkv_pages.h;
+ *   pkv_decode_attn_noalloc                          the attention without a
+ *       context (no allocation);
+ *   pkv_set_workers, pkv_set_tail_chunks, pkv_set_qkv_split,
+ *   pkv_qkv_launch_shape, pkv_workspace_bytes        tuning and inspection.
+ *
  * Errors: host-side checks return PKV_ERR_INVALID_ARG / PKV_ERR_UNSUPPORTED
  * and launch nothing.  A failed launch returns PKV_ERR_CUDA.  Range errors
  * found on the device (a page id outside [0, num_pages), or L_b + 1 larger
