@@ -751,7 +751,7 @@ def run_mixed(args, rank, world, local_rank):
         torch.sum(flush_r, dim=0, out=sink)
 
     def attn():
-        pkv.pkv_decode_attn_varlen(ctx, q, k_pool, v_pool, bt, sl, cu_d, out)
+        pkv.pkv_decode_attn_varlen(ctx, q, k_pool, v_pool, None, None, bt, sl, cu_d, out)
 
     def step():
         q.copy_(q0)    # the step rotates q in place: every step starts from the same q

@@ -169,8 +169,9 @@ pkv_status pkv_rope_append_tokens(pkv_ctx* ctx, void* q, const void* k_new, cons
  * 0 .. L_b + t (the cache, the new tokens before it and itself; causal among
  * the new tokens), out[b][t][h][:] = bf16(o).  The G x q_len query rows of a
  * (request, kv head) share each K/V tile, so the cache is read once per
- * call whatever q_len is.  Needs G * q_len <= 16 and bf16 pools
- * (PKV_ERR_UNSUPPORTED otherwise); requests whose L_b + q_len exceeds
+ * call whatever q_len is.  Needs G * q_len <= 16 (PKV_ERR_UNSUPPORTED
+ * otherwise); bf16 or E4M3 pools (scales as for pkv_decode_attn, E4M3 read
+ * in 16-token tiles here); requests whose L_b + q_len exceeds
  * bt_stride * P get zeros and set the device error word.  The split merge
  * runs in a second kernel, as for pkv_decode_attn. */
 pkv_status pkv_decode_attn_tokens(pkv_ctx* ctx, const void* q, const void* k_pool, const void* v_pool,
@@ -201,7 +202,8 @@ pkv_status pkv_rope_append_varlen(pkv_ctx* ctx, void* q, const void* k_new, cons
 
 /* pkv_decode_attn_varlen: token i of request b attends tokens 0 .. L_b + i -
  * cu_q[b] of its cache (after pkv_rope_append_varlen: the cache, the earlier
- * new tokens and itself), bf16 pools (PKV_ERR_UNSUPPORTED for E4M3).  A plan
+ * new tokens and itself), bf16 or E4M3 pools (scales as for
+ * pkv_decode_attn).  A plan
  * kernel cuts each request's new tokens into blocks of 16 / G tokens (the G x
  * 16/G query rows of a block and kv head are one 16-row mma), each block
  * streams its prefix of the cache once for its tokens.  The context holds
@@ -210,6 +212,7 @@ pkv_status pkv_rope_append_varlen(pkv_ctx* ctx, void* q, const void* k_new, cons
  * launching; lengths past the block table zero the affected tokens' output
  * and set the error word, as for pkv_decode_attn. */
 pkv_status pkv_decode_attn_varlen(pkv_ctx* ctx, const void* q, const void* k_pool, const void* v_pool,
+                                  const float* k_scale, const float* v_scale,
                                   const int32_t* block_tables, int bt_stride, const int32_t* seq_lens,
                                   const int32_t* cu_q, int batch, int n_tokens, void* out,
                                   cudaStream_t stream);

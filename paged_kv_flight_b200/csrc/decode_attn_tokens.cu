@@ -19,7 +19,11 @@
 // warp ranges, a static split), a per-warp ring of TMA tile loads on
 // mbarriers fed by a 32-tile page-id lookahead, online softmax in log2 units,
 // partial (m, l, o) rows for pairs cut between ranges, merged afterwards by
-// the combine kernel (combine.cu).  bf16 pools only.
+// the combine kernel (combine.cu).  E4M3 pools as in the single-token kernel:
+// codes converted to f16 in registers (K in the byte order of its rows, q
+// loaded in the same order; V pairs of tokens permuted per d), the per-(page,
+// kv head) scales folded into the scores and into each tile's P V, the mma
+// in f16.
 //
 // Varlen calls (a different number of new tokens per request: chunked
 // prefill mixed with decode in one batch, "Scaling TensorRT-LLM: Kernel
@@ -41,8 +45,10 @@ using namespace attn;
 // Query rows of a (request, kv head kvh) pair whose new tokens are q rows
 // qrow0, qrow0 + 1, ... as mma A fragments: rows g (a0, a2) and g + 8 (a1,
 // a3) of the 16; row r = t G + h is head kvh G + h of new token t, rows
-// r >= R are zero.
-template <int D>
+// r >= R are zero.  bf16: a0 = d 16ks+2c..+1, a2 = d 16ks+8+2c..+1.  E4M3
+// (f16 operands): the k order inside a k-step follows the byte layout of the
+// E4M3 rows, a0 = d 16ks+4c..+1, a2 = d 16ks+4c+2..+3, converted to f16.
+template <int D, bool FP8>
 __device__ __forceinline__ void load_q_rows(const AttnParams& p, int qrow0, int kvh, int g, int c4, int R,
                                             uint32_t (&qa)[D / 16][4])
 {
@@ -54,18 +60,35 @@ __device__ __forceinline__ void load_q_rows(const AttnParams& p, int qrow0, int 
         const __nv_bfloat16* qrow = p.q + (((size_t)qrow0 + t) * p.Hq + (size_t)kvh * p.G + h) * D;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-            qa[ks][half] = ok ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * c4) : 0u;
-            qa[ks][2 + half] = ok ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8 + 2 * c4) : 0u;
+            if constexpr (!FP8) {
+                qa[ks][half] = ok ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * c4) : 0u;
+                qa[ks][2 + half] = ok ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8 + 2 * c4) : 0u;
+            } else {
+                const uint2 v = ok ? *reinterpret_cast<const uint2*>(qrow + 16 * ks + 4 * c4) : make_uint2(0u, 0u);
+                qa[ks][half] = pack_f16(bf16_lo(v.x), bf16_hi(v.x));
+                qa[ks][2 + half] = pack_f16(bf16_lo(v.y), bf16_hi(v.y));
+            }
         }
     }
 }
 
-template <int D, int WARPS>
+// m16n8k16 with f16 A and B (all 16 rows), fp32 accumulation.
+__device__ __forceinline__ void mma_f16_16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                           uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+template <int D, bool FP8, int WARPS>
 __global__ void __launch_bounds__(WARPS * 32, 1)
 decode_attn_tokens_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                           const AttnParams p)
 {
-    using Gm = Geo<D, false>;
+    using Gm = Geo<D, FP8>;
     constexpr int KSTEPS = D / 16;      // mma k-steps along d for QK^T
     constexpr int NTD = D / 8;          // mma n-tiles along d for P V
     constexpr int NT = WARPS * 32;
@@ -196,24 +219,29 @@ decode_attn_tokens_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_
     // ---- 3. producer: double-buffered 32-tile lookahead, TMA issue -----------------
     int la_i = 0;
     long long la_fill = u0 + 64;
-    Lookahead la_cur = lookahead_fill<false>(p, prefix, u0, u1, lane);
-    Lookahead la_nxt = lookahead_fill<false>(p, prefix, u0 + 32, u1, lane);
+    Lookahead la_cur = lookahead_fill<FP8>(p, prefix, u0, u1, lane);
+    Lookahead la_nxt = lookahead_fill<FP8>(p, prefix, u0 + 32, u1, lane);
 
     auto issue = [&](int s) {
         if (la_i == 32) {
             la_i = 0;
             la_cur = la_nxt;
-            la_nxt = lookahead_fill<false>(p, prefix, la_fill, u1, lane);
+            la_nxt = lookahead_fill<FP8>(p, prefix, la_fill, u1, lane);
             la_fill += 32;
         }
         const int src = la_i++;
         const int v = __shfl_sync(kFull, la_cur.valid, src);
         const int row = __shfl_sync(kFull, la_cur.row, src);
+        float ks = 1.f, vs = 1.f;
+        if (FP8) {
+            ks = __shfl_sync(kFull, la_cur.ks, src);
+            vs = __shfl_sync(kFull, la_cur.vs, src);
+        }
         if (lane == 0) {
             const uint32_t bar = my_bar0 + 8u * s;
             StageInfo si;
-            si.ks = 1.f;
-            si.vs = 1.f;
+            si.ks = ks;
+            si.vs = vs;
             si.valid = (v == 1);
             si.pad = 0;
             my_info[s] = si;
@@ -280,7 +308,7 @@ decode_attn_tokens_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_
             int L, nq;
             vinfo(cb, L, nq, cur_q0);
             Rv = G * nq;
-            load_q_rows<D>(p, cur_q0, ckvh, g, c4, Rv, qa);
+            load_q_rows<D, FP8>(p, cur_q0, ckvh, g, c4, Rv, qa);
             const int n0 = L + 1;                // tokens visible to new token 0
             // new token of rows g and g + 8 (rows >= Rv see no token)
             lim[0] = g < Rv ? n0 + g / G : 0;
@@ -306,7 +334,7 @@ decode_attn_tokens_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_
                 const int nch = (kTile - rows_valid) * CPR;
                 for (int e = lane; e < nch; e += 32) {
                     const int r = rows_valid + e / CPR, ch = e % CPR;
-                    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(vb + tile_off<D, false>(r, ch)),
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(vb + tile_off<D, FP8>(r, ch)),
                                  "r"(0u)
                                  : "memory");
                 }
@@ -317,19 +345,38 @@ decode_attn_tokens_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_
             // S = Q K^T: two n-tiles of 8 tokens, rows g (e 0, 1) and g + 8 (e 2, 3), two chains
             float sa[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
             float sb[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            if constexpr (!FP8) {
 #pragma unroll
-            for (int ks = 0; ks < KSTEPS; ks += 2) {
-                uint32_t r0, r1, r2, r3, r4, r5, r6, r7;
-                ldsm_x4(kb + tile_off<D, false>(tokK, 2 * ks + (mi & 1)), r0, r1, r2, r3);
-                ldsm_x4(kb + tile_off<D, false>(tokK, 2 * ks + 2 + (mi & 1)), r4, r5, r6, r7);
-                mma_bf16_16(sa[0], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], r0, r1);
-                mma_bf16_16(sa[1], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], r2, r3);
-                mma_bf16_16(sb[0], qa[ks + 1][0], qa[ks + 1][1], qa[ks + 1][2], qa[ks + 1][3], r4, r5);
-                mma_bf16_16(sb[1], qa[ks + 1][0], qa[ks + 1][1], qa[ks + 1][2], qa[ks + 1][3], r6, r7);
+                for (int ks = 0; ks < KSTEPS; ks += 2) {
+                    uint32_t r0, r1, r2, r3, r4, r5, r6, r7;
+                    ldsm_x4(kb + tile_off<D, FP8>(tokK, 2 * ks + (mi & 1)), r0, r1, r2, r3);
+                    ldsm_x4(kb + tile_off<D, FP8>(tokK, 2 * ks + 2 + (mi & 1)), r4, r5, r6, r7);
+                    mma_bf16_16(sa[0], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], r0, r1);
+                    mma_bf16_16(sa[1], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], r2, r3);
+                    mma_bf16_16(sb[0], qa[ks + 1][0], qa[ks + 1][1], qa[ks + 1][2], qa[ks + 1][3], r4, r5);
+                    mma_bf16_16(sb[1], qa[ks + 1][0], qa[ks + 1][1], qa[ks + 1][2], qa[ks + 1][3], r6, r7);
+                }
+            } else {
+                // one 16-byte chunk of an E4M3 row = one k-step: r0 / r1 tokens 0-7,
+                // chunks 2s4 / 2s4+1; r2 / r3 tokens 8-15
+#pragma unroll
+                for (int s4 = 0; s4 < D / 32; ++s4) {
+                    uint32_t r0, r1, r2, r3;
+                    ldsm_x4(kb + tile_off<D, FP8>(tokK, 2 * s4 + (mi & 1)), r0, r1, r2, r3);
+                    mma_f16_16(sa[0], qa[2 * s4][0], qa[2 * s4][1], qa[2 * s4][2], qa[2 * s4][3], cvt_lo(r0),
+                               cvt_hi(r0));
+                    mma_f16_16(sb[0], qa[2 * s4 + 1][0], qa[2 * s4 + 1][1], qa[2 * s4 + 1][2], qa[2 * s4 + 1][3],
+                               cvt_lo(r1), cvt_hi(r1));
+                    mma_f16_16(sa[1], qa[2 * s4][0], qa[2 * s4][1], qa[2 * s4][2], qa[2 * s4][3], cvt_lo(r2),
+                               cvt_hi(r2));
+                    mma_f16_16(sb[1], qa[2 * s4 + 1][0], qa[2 * s4 + 1][1], qa[2 * s4 + 1][2], qa[2 * s4 + 1][3],
+                               cvt_lo(r3), cvt_hi(r3));
+                }
             }
 
             // online softmax per row in log2 units; tokens at or past a row's
             // limit are -inf (never 0 * NaN)
+            const float slog2 = FP8 ? p.scale_log2 * si.ks : p.scale_log2;
             float sc[2][4];
             float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
@@ -337,7 +384,7 @@ decode_attn_tokens_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int tok = tok0 + 8 * j + 2 * c4 + (e & 1);
-                    sc[j][e] = (tok < lim[e >> 1]) ? (sa[j][e] + sb[j][e]) * p.scale_log2 : -INFINITY;
+                    sc[j][e] = (tok < lim[e >> 1]) ? (sa[j][e] + sb[j][e]) * slog2 : -INFINITY;
                     mx[e >> 1] = fmaxf(mx[e >> 1], sc[j][e]);
                 }
             float alpha[2], m_ref[2];
@@ -351,12 +398,25 @@ decode_attn_tokens_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_
                 m_run[hf] = m_new;
             }
             // P as the A operand: a0 row g tokens 2c4.., a1 row g+8, a2/a3 tokens 8+2c4..
-            const uint32_t pa0 = pack_bf16(ex2(sc[0][0] - m_ref[0]), ex2(sc[0][1] - m_ref[0]));
-            const uint32_t pa1 = pack_bf16(ex2(sc[0][2] - m_ref[1]), ex2(sc[0][3] - m_ref[1]));
-            const uint32_t pa2 = pack_bf16(ex2(sc[1][0] - m_ref[0]), ex2(sc[1][1] - m_ref[0]));
-            const uint32_t pa3 = pack_bf16(ex2(sc[1][2] - m_ref[1]), ex2(sc[1][3] - m_ref[1]));
-            l_run[0] = l_run[0] * alpha[0] + ((bf16_lo(pa0) + bf16_hi(pa0)) + (bf16_lo(pa2) + bf16_hi(pa2)));
-            l_run[1] = l_run[1] * alpha[1] + ((bf16_lo(pa1) + bf16_hi(pa1)) + (bf16_lo(pa3) + bf16_hi(pa3)));
+            // (bf16, or f16 for E4M3 pools), l summed from the rounded values
+            uint32_t pa0, pa1, pa2, pa3;
+            if constexpr (!FP8) {
+                pa0 = pack_bf16(ex2(sc[0][0] - m_ref[0]), ex2(sc[0][1] - m_ref[0]));
+                pa1 = pack_bf16(ex2(sc[0][2] - m_ref[1]), ex2(sc[0][3] - m_ref[1]));
+                pa2 = pack_bf16(ex2(sc[1][0] - m_ref[0]), ex2(sc[1][1] - m_ref[0]));
+                pa3 = pack_bf16(ex2(sc[1][2] - m_ref[1]), ex2(sc[1][3] - m_ref[1]));
+                l_run[0] = l_run[0] * alpha[0] + ((bf16_lo(pa0) + bf16_hi(pa0)) + (bf16_lo(pa2) + bf16_hi(pa2)));
+                l_run[1] = l_run[1] * alpha[1] + ((bf16_lo(pa1) + bf16_hi(pa1)) + (bf16_lo(pa3) + bf16_hi(pa3)));
+            } else {
+                pa0 = pack_f16(ex2(sc[0][0] - m_ref[0]), ex2(sc[0][1] - m_ref[0]));
+                pa1 = pack_f16(ex2(sc[0][2] - m_ref[1]), ex2(sc[0][3] - m_ref[1]));
+                pa2 = pack_f16(ex2(sc[1][0] - m_ref[0]), ex2(sc[1][1] - m_ref[0]));
+                pa3 = pack_f16(ex2(sc[1][2] - m_ref[1]), ex2(sc[1][3] - m_ref[1]));
+                const float2 f0 = f16x2_to_f32(pa0), f1 = f16x2_to_f32(pa1), f2 = f16x2_to_f32(pa2),
+                             f3 = f16x2_to_f32(pa3);
+                l_run[0] = l_run[0] * alpha[0] + ((f0.x + f0.y) + (f2.x + f2.y));
+                l_run[1] = l_run[1] * alpha[1] + ((f1.x + f1.y) + (f3.x + f3.y));
+            }
             if (__any_sync(kFull, alpha[0] != 1.f || alpha[1] != 1.f)) {
 #pragma unroll
                 for (int nt = 0; nt < NTD; ++nt) {
@@ -368,12 +428,60 @@ decode_attn_tokens_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_
             }
 
             // O += P V
+            if constexpr (!FP8) {
 #pragma unroll
-            for (int dj = 0; dj < D / 16; ++dj) {
-                uint32_t r0, r1, r2, r3;
-                ldsm_x4_trans(vb + tile_off<D, false>(tokV, 2 * dj + (mi >> 1)), r0, r1, r2, r3);
-                mma_bf16_16(o[2 * dj], pa0, pa1, pa2, pa3, r0, r1);
-                mma_bf16_16(o[2 * dj + 1], pa0, pa1, pa2, pa3, r2, r3);
+                for (int dj = 0; dj < D / 16; ++dj) {
+                    uint32_t r0, r1, r2, r3;
+                    ldsm_x4_trans(vb + tile_off<D, FP8>(tokV, 2 * dj + (mi >> 1)), r0, r1, r2, r3);
+                    mma_bf16_16(o[2 * dj], pa0, pa1, pa2, pa3, r0, r1);
+                    mma_bf16_16(o[2 * dj + 1], pa0, pa1, pa2, pa3, r2, r3);
+                }
+            } else {
+                // E4M3 V: lane (n = g, c4) loads d in [DV*n, DV*n + DV) of tokens
+                // 2c4, 2c4+1, 8+2c4, 9+2c4; byte permutes pair tokens per d, and the
+                // mma n-index j of n-tile nt stands for d = DV*j + nt
+                constexpr int DV = D / 8;
+                constexpr int WORDS = DV / 4;
+                uint32_t wa[WORDS], wb[WORDS], wc[WORDS], wd[WORDS];
+                const int t0 = 2 * c4;
+                if constexpr (DV == 16) {
+                    const uint4 a = lds128(vb + tile_off<D, FP8>(t0, g));
+                    const uint4 b = lds128(vb + tile_off<D, FP8>(t0 + 1, g));
+                    const uint4 cc = lds128(vb + tile_off<D, FP8>(t0 + 8, g));
+                    const uint4 dd = lds128(vb + tile_off<D, FP8>(t0 + 9, g));
+                    wa[0] = a.x; wa[1] = a.y; wa[2] = a.z; wa[3] = a.w;
+                    wb[0] = b.x; wb[1] = b.y; wb[2] = b.z; wb[3] = b.w;
+                    wc[0] = cc.x; wc[1] = cc.y; wc[2] = cc.z; wc[3] = cc.w;
+                    wd[0] = dd.x; wd[1] = dd.y; wd[2] = dd.z; wd[3] = dd.w;
+                } else {
+                    const uint32_t off8 = (uint32_t)((g & 1) * 8);
+                    const uint2 a = lds64(vb + tile_off<D, FP8>(t0, g >> 1) + off8);
+                    const uint2 b = lds64(vb + tile_off<D, FP8>(t0 + 1, g >> 1) + off8);
+                    const uint2 cc = lds64(vb + tile_off<D, FP8>(t0 + 8, g >> 1) + off8);
+                    const uint2 dd = lds64(vb + tile_off<D, FP8>(t0 + 9, g >> 1) + off8);
+                    wa[0] = a.x; wa[1] = a.y;
+                    wb[0] = b.x; wb[1] = b.y;
+                    wc[0] = cc.x; wc[1] = cc.y;
+                    wd[0] = dd.x; wd[1] = dd.y;
+                }
+                const float vs = si.vs;
+#pragma unroll
+                for (int kw = 0; kw < WORDS; ++kw) {
+                    const uint32_t x0 = __byte_perm(wa[kw], wb[kw], 0x5140);
+                    const uint32_t x1 = __byte_perm(wa[kw], wb[kw], 0x7362);
+                    const uint32_t y0 = __byte_perm(wc[kw], wd[kw], 0x5140);
+                    const uint32_t y1 = __byte_perm(wc[kw], wd[kw], 0x7362);
+                    float t[4][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f},
+                                     {0.f, 0.f, 0.f, 0.f}};
+                    mma_f16_16(t[0], pa0, pa1, pa2, pa3, cvt_lo(x0), cvt_lo(y0));
+                    mma_f16_16(t[1], pa0, pa1, pa2, pa3, cvt_hi(x0), cvt_hi(y0));
+                    mma_f16_16(t[2], pa0, pa1, pa2, pa3, cvt_lo(x1), cvt_lo(y1));
+                    mma_f16_16(t[3], pa0, pa1, pa2, pa3, cvt_hi(x1), cvt_hi(y1));
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) o[4 * kw + e][u] = fmaf(t[e][u], vs, o[4 * kw + e][u]);
+                }
             }
         }
         __syncwarp();
@@ -407,14 +515,36 @@ decode_attn_tokens_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_
                     const float inv = 1.f / lsum[hf];
                     uint32_t* dst = reinterpret_cast<uint32_t*>(
                         p.out + (((size_t)cur_q0 + t) * p.Hq + (size_t)ckvh * G + h) * D);
+                    if constexpr (!FP8) {
 #pragma unroll
-                    for (int nt = 0; nt < NTD; ++nt)
-                        dst[(8 * nt + 2 * c4) >> 1] = pack_bf16(o[nt][2 * hf] * inv, o[nt][2 * hf + 1] * inv);
+                        for (int nt = 0; nt < NTD; ++nt)
+                            dst[(8 * nt + 2 * c4) >> 1] = pack_bf16(o[nt][2 * hf] * inv, o[nt][2 * hf + 1] * inv);
+                    } else {
+                        // n-tile nt, column j = 2c4 + e holds d = DV j + nt
+                        constexpr int DV = D / 8;
+#pragma unroll
+                        for (int e = 0; e < 2; ++e)
+#pragma unroll
+                            for (int u = 0; u < DV / 2; ++u)
+                                dst[(DV * (2 * c4 + e) + 2 * u) >> 1] =
+                                    pack_bf16(o[2 * u][2 * hf + e] * inv, o[2 * u + 1][2 * hf + e] * inv);
+                    }
                 } else {
                     float* dst = p.part_o + ((size_t)slot * R + r) * D;
+                    if constexpr (!FP8) {
 #pragma unroll
-                    for (int nt = 0; nt < NTD; ++nt)
-                        *reinterpret_cast<float2*>(dst + 8 * nt + 2 * c4) = make_float2(o[nt][2 * hf], o[nt][2 * hf + 1]);
+                        for (int nt = 0; nt < NTD; ++nt)
+                            *reinterpret_cast<float2*>(dst + 8 * nt + 2 * c4) =
+                                make_float2(o[nt][2 * hf], o[nt][2 * hf + 1]);
+                    } else {
+                        constexpr int DV = D / 8;
+#pragma unroll
+                        for (int e = 0; e < 2; ++e)
+#pragma unroll
+                            for (int u = 0; u < DV / 2; ++u)
+                                *reinterpret_cast<float2*>(dst + DV * (2 * c4 + e) + 2 * u) =
+                                    make_float2(o[2 * u][2 * hf + e], o[2 * u + 1][2 * hf + e]);
+                    }
                     if (c4 == 0)
                         *reinterpret_cast<float2*>(p.part_ml + ((size_t)slot * R + r) * 2) =
                             make_float2(m_run[hf], lsum[hf]);
@@ -445,15 +575,15 @@ decode_attn_tokens_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_
     }
 }
 
-template <int D>
+template <int D, bool FP8>
 size_t tokens_smem_bytes(int stages, int max_batch)
 {
-    using Gm = Geo<D, false>;
+    using Gm = Geo<D, FP8>;
     return 1024 + (size_t)kAttnWarps * stages * (Gm::STAGEB + sizeof(StageInfo) + 8) +
            sizeof(int) * (size_t)(max_batch + 1);
 }
 
-template <int D>
+template <int D, bool FP8>
 cudaError_t prepare_tokens_t(int num_sms, int max_batch, AttnLaunch* out)
 {
     int dev = 0, optin = 0;
@@ -462,16 +592,17 @@ cudaError_t prepare_tokens_t(int num_sms, int max_batch, AttnLaunch* out)
     e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     if (e != cudaSuccess) return e;
     const int stages = kAttnMaxStages;
-    const size_t bytes = tokens_smem_bytes<D>(stages, max_batch);
+    const size_t bytes = tokens_smem_bytes<D, FP8>(stages, max_batch);
     if (bytes > (size_t)optin - 256) return cudaErrorInvalidConfiguration;
-    e = cudaFuncSetAttribute(decode_attn_tokens_kernel<D, kAttnWarps>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)bytes);
+    e = cudaFuncSetAttribute(decode_attn_tokens_kernel<D, FP8, kAttnWarps>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess) return e;
     e = combine_prepare(D);
     if (e != cudaSuccess) return e;
     out->ctas = num_sms;
     out->stages = stages;
     out->smem_bytes = bytes;
+    out->tile = kTile;
     return cudaSuccess;
 }
 
@@ -543,23 +674,28 @@ cudaError_t launch_varlen_plan(const int32_t* cu_q, const int32_t* seq_lens, int
     return cudaGetLastError();
 }
 
-cudaError_t attn_tokens_prepare(int head_dim, int num_sms, int max_batch, AttnLaunch* out)
+cudaError_t attn_tokens_prepare(int head_dim, bool fp8, int num_sms, int max_batch, AttnLaunch* out)
 {
-    return head_dim == 128 ? prepare_tokens_t<128>(num_sms, max_batch, out)
-                           : prepare_tokens_t<64>(num_sms, max_batch, out);
+    if (head_dim == 128)
+        return fp8 ? prepare_tokens_t<128, true>(num_sms, max_batch, out)
+                   : prepare_tokens_t<128, false>(num_sms, max_batch, out);
+    return fp8 ? prepare_tokens_t<64, true>(num_sms, max_batch, out) : prepare_tokens_t<64, false>(num_sms, max_batch, out);
 }
 
 cudaError_t launch_decode_attn_tokens(const AttnParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
-                                      int head_dim, const AttnLaunch& L, cudaStream_t stream)
+                                      int head_dim, bool fp8, const AttnLaunch& L, cudaStream_t stream)
 {
     const dim3 grid(L.ctas), block(kAttnWarps * 32);
     AttnParams q = p;
     q.stages = L.stages;
     q.tail_chunks = 0;
-    if (head_dim == 128)
-        decode_attn_tokens_kernel<128, kAttnWarps><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
-    else
-        decode_attn_tokens_kernel<64, kAttnWarps><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
+    if (head_dim == 128) {
+        if (fp8) decode_attn_tokens_kernel<128, true, kAttnWarps><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
+        else decode_attn_tokens_kernel<128, false, kAttnWarps><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
+    } else {
+        if (fp8) decode_attn_tokens_kernel<64, true, kAttnWarps><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
+        else decode_attn_tokens_kernel<64, false, kAttnWarps><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
+    }
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     return launch_combine(q, head_dim, L.ctas * kAttnWarps, L.ctas, stream);

@@ -21,7 +21,7 @@ struct pkv_ctx {
     int num_sms;
     int G;
     pkv::AttnLaunch attn;
-    pkv::AttnLaunch attn_tok;     // several new tokens per request (bf16 pools)
+    pkv::AttnLaunch attn_tok;     // several new tokens per request
     int workers;
     int tail_chunks;      // largest number of dynamic tail chunks per warp range
     void* ws;             // one allocation, carved below
@@ -37,6 +37,11 @@ struct pkv_ctx {
     const void* tm_k_ptr;
     const void* tm_v_ptr;
     CUtensorMap tmk, tmv;
+    // 16-row boxes for the several-new-tokens path where the one-token maps
+    // use 32-row ones (E4M3 pools with pages of 32 tokens or more)
+    const void* t16_k_ptr;
+    const void* t16_v_ptr;
+    CUtensorMap t16k, t16v;
     const void* tm_w_ptr;        // QKV weight and input maps of pkv_qkv_rope_append
     int tm_w_hidden, tm_w_layout;
     int qkv_split;               // 0: automatic
@@ -105,7 +110,15 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
 // elements; box = one attention tile of rows (16, or 32 for E4M3 pools with
 // pages of at least 32 tokens) x (128 or 64 bytes), swizzled to match the
 // kernel's shared-memory addressing.
+bool encode_pool_rows(const pkv_ctx* ctx, const void* pool, int box_rows, CUtensorMap* map);
+
 bool encode_pool(const pkv_ctx* ctx, const void* pool, CUtensorMap* map)
+{
+    const bool fp8 = ctx->cfg.kv_dtype == PKV_KV_FP8_E4M3;
+    return encode_pool_rows(ctx, pool, pkv::attn_tile(fp8, ctx->cfg.page_size), map);
+}
+
+bool encode_pool_rows(const pkv_ctx* ctx, const void* pool, int box_rows, CUtensorMap* map)
 {
     auto fn = encode_fn();
     if (!fn) return false;
@@ -116,7 +129,7 @@ bool encode_pool(const pkv_ctx* ctx, const void* pool, CUtensorMap* map)
     cuuint64_t dims[2] = {(cuuint64_t)ctx->cfg.head_dim,
                           (cuuint64_t)ctx->cfg.num_pages * ctx->cfg.num_kv_heads * ctx->cfg.page_size};
     cuuint64_t strides[1] = {(cuuint64_t)rowb};
-    cuuint32_t box[2] = {(cuuint32_t)(boxb / elem), (cuuint32_t)pkv::attn_tile(fp8, ctx->cfg.page_size)};
+    cuuint32_t box[2] = {(cuuint32_t)(boxb / elem), (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
                     const_cast<void*>(pool), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -181,9 +194,9 @@ pkv_status pkv_create(const pkv_config* cfg, pkv_ctx** out)
         return PKV_ERR_CUDA;
     }
     // varlen calls cut requests into virtual ones: room for 4 per request
-    ctx->vmax = fp8 ? 0 : std::min(4 * cfg->max_batch, pkv::kMaxBatch);
-    if (!fp8 && pkv::attn_tokens_prepare(cfg->head_dim, ctx->num_sms, std::max(cfg->max_batch, ctx->vmax),
-                                         &ctx->attn_tok) != cudaSuccess) {
+    ctx->vmax = std::min(4 * cfg->max_batch, pkv::kMaxBatch);
+    if (pkv::attn_tokens_prepare(cfg->head_dim, fp8, ctx->num_sms, std::max(cfg->max_batch, ctx->vmax),
+                                 &ctx->attn_tok) != cudaSuccess) {
         free(ctx);
         return PKV_ERR_CUDA;
     }
@@ -351,23 +364,41 @@ namespace {
 // `batch` requests of q_len tokens) and the varlen ones (batch = the plan's
 // capacity, q_len = the block length).
 pkv_status attn_tokens_launch(pkv_ctx* ctx, const void* q, const void* k_pool, const void* v_pool,
-                              const int32_t* block_tables, int bt_stride, const int32_t* seq_lens, int batch,
-                              int q_len, const int4* vmap, const int* vcount, void* out, cudaStream_t stream)
+                              const float* k_scale, const float* v_scale, const int32_t* block_tables,
+                              int bt_stride, const int32_t* seq_lens, int batch, int q_len, const int4* vmap,
+                              const int* vcount, void* out, cudaStream_t stream)
 {
-    if (ctx->tm_k_ptr != k_pool) {
-        if (!encode_pool(ctx, k_pool, &ctx->tmk)) return PKV_ERR_CUDA;
-        ctx->tm_k_ptr = k_pool;
-    }
-    if (ctx->tm_v_ptr != v_pool) {
-        if (!encode_pool(ctx, v_pool, &ctx->tmv)) return PKV_ERR_CUDA;
-        ctx->tm_v_ptr = v_pool;
+    const bool fp8 = ctx->cfg.kv_dtype == PKV_KV_FP8_E4M3;
+    const CUtensorMap* mk = &ctx->tmk;
+    const CUtensorMap* mv = &ctx->tmv;
+    if (pkv::attn_tile(fp8, ctx->cfg.page_size) == pkv::kTile) {
+        // the one-token maps already have 16-row boxes
+        if (ctx->tm_k_ptr != k_pool) {
+            if (!encode_pool(ctx, k_pool, &ctx->tmk)) return PKV_ERR_CUDA;
+            ctx->tm_k_ptr = k_pool;
+        }
+        if (ctx->tm_v_ptr != v_pool) {
+            if (!encode_pool(ctx, v_pool, &ctx->tmv)) return PKV_ERR_CUDA;
+            ctx->tm_v_ptr = v_pool;
+        }
+    } else {
+        if (ctx->t16_k_ptr != k_pool) {
+            if (!encode_pool_rows(ctx, k_pool, pkv::kTile, &ctx->t16k)) return PKV_ERR_CUDA;
+            ctx->t16_k_ptr = k_pool;
+        }
+        if (ctx->t16_v_ptr != v_pool) {
+            if (!encode_pool_rows(ctx, v_pool, pkv::kTile, &ctx->t16v)) return PKV_ERR_CUDA;
+            ctx->t16_v_ptr = v_pool;
+        }
+        mk = &ctx->t16k;
+        mv = &ctx->t16v;
     }
 
     pkv::AttnParams p;
     p.q = static_cast<const __nv_bfloat16*>(q);
     p.out = static_cast<__nv_bfloat16*>(out);
-    p.k_scale = nullptr;
-    p.v_scale = nullptr;
+    p.k_scale = fp8 ? k_scale : nullptr;
+    p.v_scale = fp8 ? v_scale : nullptr;
     p.block_tables = block_tables;
     p.seq_lens = seq_lens;
     p.part_o = ctx->d_part_o;
@@ -389,8 +420,7 @@ pkv_status attn_tokens_launch(pkv_ctx* ctx, const void* q, const void* k_pool, c
     p.q_len = q_len;
     p.vmap = vmap;
     p.vcount = vcount;
-    const cudaError_t e = pkv::launch_decode_attn_tokens(p, ctx->tmk, ctx->tmv, ctx->cfg.head_dim, ctx->attn_tok,
-                                                         stream);
+    const cudaError_t e = pkv::launch_decode_attn_tokens(p, *mk, *mv, ctx->cfg.head_dim, fp8, ctx->attn_tok, stream);
     return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
@@ -406,11 +436,10 @@ pkv_status pkv_decode_attn_tokens(pkv_ctx* ctx, const void* q, const void* k_poo
     pkv_status st = check_call(ctx, batch, bt_stride, k_pool, v_pool, k_scale, v_scale, block_tables, seq_lens);
     if (st != PKV_OK || batch == 0) return st;
     if (q_len < 1) return PKV_ERR_INVALID_ARG;
-    if (ctx->cfg.kv_dtype != PKV_KV_BF16) return PKV_ERR_UNSUPPORTED;
     if ((long long)ctx->G * q_len > pkv::kMaxTokenRows) return PKV_ERR_UNSUPPORTED;
     if (!q || !out || !aligned16(q) || !aligned16(out)) return PKV_ERR_INVALID_ARG;
-    return attn_tokens_launch(ctx, q, k_pool, v_pool, block_tables, bt_stride, seq_lens, batch, q_len, nullptr,
-                              nullptr, out, stream);
+    return attn_tokens_launch(ctx, q, k_pool, v_pool, k_scale, v_scale, block_tables, bt_stride, seq_lens, batch,
+                              q_len, nullptr, nullptr, out, stream);
 }
 
 pkv_status pkv_rope_append_varlen(pkv_ctx* ctx, void* q, const void* k_new, const void* v_new, void* k_pool,
@@ -453,11 +482,11 @@ pkv_status pkv_rope_append_varlen(pkv_ctx* ctx, void* q, const void* k_new, cons
 }
 
 pkv_status pkv_decode_attn_varlen(pkv_ctx* ctx, const void* q, const void* k_pool, const void* v_pool,
-                                  const int32_t* block_tables, int bt_stride, const int32_t* seq_lens,
-                                  const int32_t* cu_q, int batch, int n_tokens, void* out, cudaStream_t stream)
+                                  const float* k_scale, const float* v_scale, const int32_t* block_tables,
+                                  int bt_stride, const int32_t* seq_lens, const int32_t* cu_q, int batch,
+                                  int n_tokens, void* out, cudaStream_t stream)
 {
-    if (ctx && ctx->cfg.kv_dtype != PKV_KV_BF16) return PKV_ERR_UNSUPPORTED;   // bf16 pools only
-    pkv_status st = check_call(ctx, batch, bt_stride, k_pool, v_pool, nullptr, nullptr, block_tables, seq_lens);
+    pkv_status st = check_call(ctx, batch, bt_stride, k_pool, v_pool, k_scale, v_scale, block_tables, seq_lens);
     if (st != PKV_OK) return st;
     if (n_tokens < 0) return PKV_ERR_INVALID_ARG;
     if (batch == 0 || n_tokens == 0) return PKV_OK;
@@ -468,8 +497,8 @@ pkv_status pkv_decode_attn_varlen(pkv_ctx* ctx, const void* q, const void* k_poo
     if (pkv::launch_varlen_plan(cu_q, seq_lens, batch, block, ctx->vmax, ctx->d_vmap, ctx->d_vcount, ctx->d_err,
                                 stream) != cudaSuccess)
         return PKV_ERR_CUDA;
-    return attn_tokens_launch(ctx, q, k_pool, v_pool, block_tables, bt_stride, seq_lens, ctx->vmax, block,
-                              ctx->d_vmap, ctx->d_vcount, out, stream);
+    return attn_tokens_launch(ctx, q, k_pool, v_pool, k_scale, v_scale, block_tables, bt_stride, seq_lens,
+                              ctx->vmax, block, ctx->d_vmap, ctx->d_vcount, out, stream);
 }
 
 pkv_status pkv_qkv_pack_weight(pkv_ctx* ctx, const void* w_qkv, int hidden, void* w_tiled, cudaStream_t stream)

@@ -118,16 +118,16 @@ cudaError_t launch_decode_attn(const AttnParams& p, const CUtensorMap& tmk, cons
                                int head_dim, bool fp8, const AttnLaunch& L, cudaStream_t stream);
 
 // Attention of several new tokens per request (decode_attn_tokens.cu, bf16
-// pools, G x q_len <= 16): shape of its launch and the launch itself
-// (attention, then the combine).
-cudaError_t attn_tokens_prepare(int head_dim, int num_sms, int max_batch, AttnLaunch* out);
+// or E4M3 pools with 16-token tiles, G x q_len <= 16): shape of its launch
+// and the launch itself (attention, then the combine).
+cudaError_t attn_tokens_prepare(int head_dim, bool fp8, int num_sms, int max_batch, AttnLaunch* out);
 // The virtual requests of a varlen call: blocks of `block` new tokens (the
 // last of a request may be shorter) of requests with cu_q[b + 1] > cu_q[b];
 // writes vmap and the count (capped at vmax; more sets kErrLength).
 cudaError_t launch_varlen_plan(const int32_t* cu_q, const int32_t* seq_lens, int batch, int block, int vmax,
                                int4* vmap, int* vcount, int* err, cudaStream_t stream);
 cudaError_t launch_decode_attn_tokens(const AttnParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
-                                      int head_dim, const AttnLaunch& L, cudaStream_t stream);
+                                      int head_dim, bool fp8, const AttnLaunch& L, cudaStream_t stream);
 
 // QKV projection of the new tokens on tcgen05, fused with RoPE and the append
 // (qkv_rope_append.cu).

@@ -103,7 +103,7 @@ lib.pkv_table_sync.argtypes = [_V, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, 
 lib.pkv_table_sync.restype = C.c_int
 lib.pkv_rope_append_varlen.argtypes = [_V, _V, _V, _V, _V, _V, _V, _V, _V, C.c_int, _V, _V, C.c_int, C.c_int, _V]
 lib.pkv_rope_append_varlen.restype = C.c_int
-lib.pkv_decode_attn_varlen.argtypes = [_V, _V, _V, _V, _V, C.c_int, _V, _V, C.c_int, C.c_int, _V, _V]
+lib.pkv_decode_attn_varlen.argtypes = [_V, _V, _V, _V, _V, _V, _V, C.c_int, _V, _V, C.c_int, C.c_int, _V, _V]
 lib.pkv_decode_attn_varlen.restype = C.c_int
 lib.pkv_set_tail_chunks.argtypes = [_V, C.c_int]
 lib.pkv_set_tail_chunks.restype = C.c_int
@@ -352,16 +352,17 @@ def pkv_rope_append_varlen(ctx, q, k_new, v_new, k_pool, v_pool, k_scale, v_scal
     return _done(st, "pkv_rope_append_varlen", check)
 
 
-def pkv_decode_attn_varlen(ctx, q, k_pool, v_pool, block_tables, seq_lens, cu_q, out,
+def pkv_decode_attn_varlen(ctx, q, k_pool, v_pool, k_scale, v_scale, block_tables, seq_lens, cu_q, out,
                            batch: int | None = None, bt_stride: int | None = None, stream=None,
                            check: bool = True) -> int:
     """q / out [n_tokens, Hq, d]; token i of request b attends its cache up to
-    position L_b + i - cu_q[b]."""
+    position L_b + i - cu_q[b] (E4M3 pools take their scales, else None)."""
     if batch is None:
         batch = int(seq_lens.shape[0])
     if bt_stride is None:
         bt_stride = int(block_tables.shape[1])
-    st = lib.pkv_decode_attn_varlen(ctx, _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(block_tables), int(bt_stride),
+    st = lib.pkv_decode_attn_varlen(ctx, _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(k_scale), _ptr(v_scale),
+                                    _ptr(block_tables), int(bt_stride),
                                     _ptr(seq_lens), _ptr(cu_q), int(batch), int(q.shape[0]), _ptr(out),
                                     _stream(stream))
     return _done(st, "pkv_decode_attn_varlen", check)

@@ -171,8 +171,50 @@ def test_tokens_host_side_rejections(pkv):
     ctx = _gpu.make_ctx(pkv, wf)
     try:
         outf = torch.empty(2, 2, 32, 128, dtype=torch.bfloat16, device="cuda")
-        st = pkv.pkv_decode_attn_tokens(ctx, dvf["q"], dvf["k_pool"], dvf["v_pool"], dvf["k_scale"],
-                                        dvf["v_scale"], dvf["block_tables"], dvf["seq_lens"], outf, check=False)
-        assert st == pkv.PKV_ERR_UNSUPPORTED
+        st = pkv.pkv_decode_attn_tokens(ctx, dvf["q"], dvf["k_pool"], dvf["v_pool"], None, None,
+                                        dvf["block_tables"], dvf["seq_lens"], outf, q_len=2, check=False)
+        assert st == pkv.PKV_ERR_INVALID_ARG                 # E4M3 pools need their scales
     finally:
         pkv.pkv_destroy(ctx)
+
+
+E4M3_CASES = [
+    # name, Hq, Hkv, d, P, q_len, lengths (P >= 32: the 16-row maps of this path)
+    ("f8_g4_q4_d128_p32", 32, 8, 128, 32, 4, [0, 15, 16, 31, 100, 900]),
+    ("f8_g8_q2_d128_p16", 64, 8, 128, 16, 2, [3, 14, 300]),
+    ("f8_g2_q8_d64_p64", 8, 4, 64, 64, 8, [0, 63, 64, 500]),
+]
+
+
+@pytest.mark.parametrize("case", E4M3_CASES, ids=lambda c: c[0])
+def test_e4m3_tokens_step_matches_oracle(pkv, case):
+    """Several new tokens with E4M3 pools: V codes bit-exact, K codes within
+    one step, q within 1 ulp, attention within the E4M3 tolerances against
+    the oracle fed the same codes and scales."""
+    name, Hq, Hkv, d, P, q_len, lengths = case
+    w = workloads.build(name, Hq, Hkv, d, P, True, 5e5 if d == 128 else 1e4, lengths, 33, device="cpu",
+                        q_len=q_len)
+    dv = _gpu.to_device(w)
+    ctx = _gpu.make_ctx(pkv, w)
+    try:
+        out = torch.empty(w.batch, q_len, Hq, d, dtype=torch.bfloat16, device="cuda")
+        q, kn, vn = (dv[k].contiguous() for k in ("q", "k_new", "v_new"))
+        pkv.pkv_rope_append_tokens(ctx, q, kn, vn, dv["k_pool"], dv["v_pool"], dv["k_scale"], dv["v_scale"],
+                                   dv["block_tables"], dv["seq_lens"], q_len=q_len)
+        pkv.pkv_decode_attn_tokens(ctx, q, dv["k_pool"], dv["v_pool"], dv["k_scale"], dv["v_scale"],
+                                   dv["block_tables"], dv["seq_lens"], out, q_len=q_len)
+        assert pkv.pkv_check_device_error(ctx)[0] == pkv.PKV_OK
+    finally:
+        pkv.pkv_destroy(ctx)
+    h = host_inputs(w)
+    cfg = oracle_cfg(w)
+    assert oracle.rope_append_tokens(cfg, h["q"], h["k_new"], h["v_new"], h["k_pool"], h["v_pool"], h["k_scale"],
+                                     h["v_scale"], h["block_tables"], h["seq_lens"]) == 0
+    ref, st = oracle.decode_attn_tokens(cfg, h["q"], h["k_pool"], h["v_pool"], h["k_scale"], h["v_scale"],
+                                        h["block_tables"], h["seq_lens"])
+    assert st == 0
+    assert np.abs(bf16_ordinal(bits16(q)) - bf16_ordinal(h["q"])).max() <= 1
+    assert np.array_equal(dv["v_pool"].cpu().numpy(), h["v_pool"])
+    assert np.abs(dv["k_pool"].cpu().numpy().astype(int) - h["k_pool"].astype(int)).max() <= 1
+    mx, mean, finite = _gpu.errors(out, ref)
+    assert finite and mx <= _gpu.TOL_FP8["max"] and mean <= _gpu.TOL_FP8["mean"], (mx, mean)

@@ -67,7 +67,7 @@ def _step(pkv, ctx, dv):
     out = torch.full_like(dv["q"], float("nan"))
     pkv.pkv_rope_append_varlen(ctx, dv["q"], dv["k_new"], dv["v_new"], dv["k_pool"], dv["v_pool"], None, None,
                                dv["block_tables"], dv["seq_lens"], dv["cu_q"])
-    pkv.pkv_decode_attn_varlen(ctx, dv["q"], dv["k_pool"], dv["v_pool"], dv["block_tables"], dv["seq_lens"],
+    pkv.pkv_decode_attn_varlen(ctx, dv["q"], dv["k_pool"], dv["v_pool"], None, None, dv["block_tables"], dv["seq_lens"],
                                dv["cu_q"], out)
     return out
 
@@ -115,7 +115,7 @@ def test_varlen_rejections_and_range_errors(pkv):
     ctx = _gpu.make_ctx(pkv, w, max_batch=4)          # room for 16 blocks of 2 tokens
     try:
         # 41 new tokens in blocks of 2 (G = 8): 3 + 21 blocks > 16
-        st = pkv.pkv_decode_attn_varlen(ctx, dv["q"], dv["k_pool"], dv["v_pool"], dv["block_tables"],
+        st = pkv.pkv_decode_attn_varlen(ctx, dv["q"], dv["k_pool"], dv["v_pool"], None, None, dv["block_tables"],
                                         dv["seq_lens"], dv["cu_q"], out, check=False)
         assert st == pkv.PKV_ERR_UNSUPPORTED
     finally:
@@ -125,7 +125,7 @@ def test_varlen_rejections_and_range_errors(pkv):
         bad = dv["seq_lens"].clone()
         bad[1] = w.bt_stride * w.P                    # request 1's one token lies past its table
         out = torch.full_like(dv["q"], 1.0)
-        pkv.pkv_decode_attn_varlen(ctx, dv["q"], dv["k_pool"], dv["v_pool"], dv["block_tables"], bad, dv["cu_q"],
+        pkv.pkv_decode_attn_varlen(ctx, dv["q"], dv["k_pool"], dv["v_pool"], None, None, dv["block_tables"], bad, dv["cu_q"],
                                    out)
         st, bits = pkv.pkv_check_device_error(ctx)
         assert st == pkv.PKV_ERR_DEVICE_BOUNDS and bits & 1
@@ -133,16 +133,43 @@ def test_varlen_rejections_and_range_errors(pkv):
         assert torch.count_nonzero(out[i].float()) == 0   # its token's output is zeros
     finally:
         pkv.pkv_destroy(ctx)
-    wf = workloads.build("vf", 8, 2, 64, 16, True, 1e4, [3, 9], 3, device="cpu")
-    ctx = _gpu.make_ctx(pkv, wf, max_batch=8)
+
+
+
+@pytest.mark.parametrize("P", [16, 32])
+def test_varlen_step_with_e4m3_pools(pkv, P):
+    """The varlen step with E4M3 pools (P = 32: the 16-row maps of the
+    several-new-tokens path): V codes bit-exact, K codes within one step,
+    attention within the E4M3 tolerances."""
+    q_lens = [1, 9, 0, 4, 17]
+    w = workloads.build("vf8", 32, 8, 128, P, True, 5e5, [40, 0, 7, 300, 63], 49, device="cpu",
+                        q_len=max(q_lens))
+    h = varlen_host(w, q_lens)
+    ho = {k: (v.copy() if isinstance(v, np.ndarray) else v) for k, v in h.items()}
+    cfg = oracle_cfg(w)
+    assert oracle.rope_append_varlen(cfg, ho["q"], ho["k_new"], ho["v_new"], ho["k_pool"], ho["v_pool"],
+                                     ho["k_scale"], ho["v_scale"], ho["block_tables"], ho["seq_lens"],
+                                     ho["cu_q"]) == 0
+    ref, st = oracle.decode_attn_varlen(cfg, ho["q"], ho["k_pool"], ho["v_pool"], ho["k_scale"], ho["v_scale"],
+                                        ho["block_tables"], ho["seq_lens"], ho["cu_q"])
+    assert st == 0
+    q = _dev_bits(h["q"])
+    kp, vp = torch.from_numpy(h["k_pool"]).cuda(), torch.from_numpy(h["v_pool"]).cuda()
+    ks, vs = torch.from_numpy(h["k_scale"]).cuda(), torch.from_numpy(h["v_scale"]).cuda()
+    bt, sl = torch.from_numpy(h["block_tables"]).cuda(), torch.from_numpy(h["seq_lens"]).cuda()
+    cu = torch.from_numpy(h["cu_q"]).cuda()
+    out = torch.full_like(q, float("nan"))
+    ctx = _gpu.make_ctx(pkv, w, max_batch=16)
     try:
-        dvf = _gpu.to_device(wf)
-        cu = torch.tensor([0, 1, 2], dtype=torch.int32, device="cuda")
-        st = pkv.pkv_decode_attn_varlen(ctx, dvf["q"], dvf["k_pool"], dvf["v_pool"], dvf["block_tables"],
-                                        dvf["seq_lens"], cu, torch.empty_like(dvf["q"]), check=False)
-        assert st == pkv.PKV_ERR_UNSUPPORTED            # E4M3 pools: one-token or multi-token calls only
+        pkv.pkv_rope_append_varlen(ctx, q, _dev_bits(h["k_new"]), _dev_bits(h["v_new"]), kp, vp, ks, vs, bt, sl, cu)
+        pkv.pkv_decode_attn_varlen(ctx, q, kp, vp, ks, vs, bt, sl, cu, out)
+        assert pkv.pkv_check_device_error(ctx)[0] == pkv.PKV_OK
     finally:
         pkv.pkv_destroy(ctx)
+    assert np.array_equal(vp.cpu().numpy(), ho["v_pool"])
+    assert np.abs(kp.cpu().numpy().astype(int) - ho["k_pool"].astype(int)).max() <= 1
+    mx, mean, finite = _gpu.errors(out, ref)
+    assert finite and mx <= _gpu.TOL_FP8["max"] and mean <= _gpu.TOL_FP8["mean"], (mx, mean)
 
 
 def test_varlen_append_into_e4m3_pools(pkv):
