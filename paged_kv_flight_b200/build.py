@@ -1,6 +1,6 @@
 """Build libpkv.so (the C-ABI CUDA library) in-tree for sm_100a with nvcc.
 
-    python -m paged_kv_flight_b200.build [--force] [--debug-bounds]
+    python -m paged_kv_flight_b200.build [--force] [--ptxas-v]
 """
 import glob
 import os
