@@ -69,6 +69,37 @@ def workload_bytes(w) -> int:
     return metric_bytes(w.seq_lens, w.Hq, w.Hkv, w.d, w.P, w.kv_fp8, w.q_len)
 
 
+def full_step_bytes(seq_lens, Hq, Hkv, d, P, kv_fp8, q_len=1) -> int:
+    """The step's whole algorithmic traffic: the metric bytes plus what the
+    RoPE + append kernel moves (q read and written back, k_new / v_new read,
+    the new k / v rows written, the landing pages' scales for E4M3 pools) and
+    the index reads of both kernels (block-table entries of the attended
+    pages, seq_lens, the landing pages' entries).  The split partials are left
+    out: how many there are is planned on the device each step."""
+    n = np.asarray(seq_lens, np.int64) + q_len
+    B = len(n)
+    s = 1 if kv_fp8 else 2
+    rope = B * q_len * (2 * Hq * d * 2 + 2 * Hkv * d * 2 + 2 * Hkv * d * s + 4)
+    if kv_fp8:
+        rope += B * q_len * 2 * Hkv * 4
+    index = int(((n + P - 1) // P).sum()) * 4 + 2 * B * 4
+    return metric_bytes(seq_lens, Hq, Hkv, d, P, kv_fp8, q_len) + rope + index
+
+
+def host_cpu() -> dict:
+    """The host's CPU model and hardware thread count, for the CPU baselines."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"cpu_model": model, "host_threads": os.cpu_count()}
+
+
 def measured_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -285,7 +316,7 @@ def cpu_baseline(w, src, time_budget_s: float = 20.0) -> dict:
     by = metric_bytes(w.seq_lens[done], w.Hq, w.Hkv, w.d, w.P, w.kv_fp8, w.q_len)
     toks = int((w.seq_lens[done].astype(np.int64) + w.q_len).sum())
     return {"value": by / t_sum / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "seconds": t_sum,
+            "seconds": t_sum, **host_cpu(),
             "sample": f"requests 0..{len(done) - 1} of {w.batch} ({toks} attended tokens, "
                       f"{100.0 * by / workload_bytes(w):.1f}% of the step's bytes); plain fp64 C oracle, "
                       f"single thread, append + attention"}
@@ -526,7 +557,9 @@ def run_ours(args, name, rank, world, local_rank):
         "config": {"workload": name, "description": workloads.DESCRIPTIONS[name], "batch": B,
                    "tokens_attended": int((w.seq_lens.astype(np.int64) + w.q_len).sum()),
                    "new_tokens_per_request": w.q_len,
-                   "metric_bytes_per_step": by, "l2": "flushed before every timed step, outside the event window: write 2x L2, then read 2x L2",
+                   "metric_bytes_per_step": by,
+                   "full_step_bytes": full_step_bytes(w.seq_lens, w.Hq, w.Hkv, w.d, w.P, w.kv_fp8, w.q_len),
+                   "l2": "flushed before every timed step, outside the event window: write 2x L2, then read 2x L2",
                    "timing": ("each step replayed from one CUDA-graph capture of pkv_rope_append + pkv_decode_attn "
                               "(3 kernels); per-kernel times from the same steps launched eagerly"
                               if graph_ms is not None else "eager launches through the C ABI"),
@@ -582,7 +615,8 @@ def run_reference(args, name):
         "data": "synthetic: same seeded workload as the GPU arm",
         "config": {"workload": name, "description": workloads.DESCRIPTIONS[name], "batch": w.batch,
                    "metric_bytes_per_step_sampled": by},
-        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample,
+                         **host_cpu()},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 

@@ -36,6 +36,39 @@ def test_metric_bytes_with_several_new_tokens_by_hand():
     assert bench.metric_bytes([0, 15], 8, 2, 64, 16, False, q_len=3) == kv + qo
 
 
+def test_full_step_bytes_by_hand():
+    # L = 0 and 15 -> 1 and 16 attended tokens over 1 and 1 pages (P 16); Hq 8, Hkv 2, d 64
+    metric = bench.metric_bytes([0, 15], 8, 2, 64, 16, False)
+    rope = 2 * (2 * 8 * 64 * 2          # q read and written back
+                + 2 * 2 * 64 * 2        # k_new, v_new read
+                + 2 * 2 * 64 * 2        # k, v rows written (bf16)
+                + 4)                    # the landing page's block-table entry
+    index = (1 + 1) * 4 + 2 * 2 * 4     # attended pages' entries; seq_lens read by both kernels
+    assert bench.full_step_bytes([0, 15], 8, 2, 64, 16, False) == metric + rope + index
+    # E4M3: one byte per stored element, plus the landing page's two scales per kv head
+    metric8 = bench.metric_bytes([0, 15], 8, 2, 64, 16, True)
+    rope8 = 2 * (2 * 8 * 64 * 2 + 2 * 2 * 64 * 2 + 2 * 2 * 64 * 1 + 4 + 2 * 2 * 4)
+    assert bench.full_step_bytes([0, 15], 8, 2, 64, 16, True) == metric8 + rope8 + index
+    # several new tokens: L = 15 with 3 new -> 18 tokens over 2 pages
+    m3 = bench.metric_bytes([15], 8, 2, 64, 16, False, q_len=3)
+    r3 = 3 * (2 * 8 * 64 * 2 + 2 * 2 * 64 * 2 + 2 * 2 * 64 * 2 + 4)
+    assert bench.full_step_bytes([15], 8, 2, 64, 16, False, q_len=3) == m3 + r3 + 2 * 4 + 2 * 4
+
+
+def test_full_step_bytes_stay_near_the_metric_on_every_workload():
+    for name in workloads.CONFIG_NAMES:
+        w = workloads.make(name)
+        by, full = bench.workload_bytes(w), bench.full_step_bytes(w.seq_lens, w.Hq, w.Hkv, w.d, w.P, w.kv_fp8,
+                                                                  w.q_len)
+        assert by < full < 1.1 * by + 64 * 1024, name
+
+
+def test_host_cpu_reports_a_model_and_thread_count():
+    info = bench.host_cpu()
+    assert isinstance(info["cpu_model"], str) and info["cpu_model"]
+    assert info["host_threads"] >= 1
+
+
 def test_llama8b_bytes_near_the_recipe_estimate():
     w_lens = workloads.draw_lengths("llama8b", np.random.default_rng(workloads.config_seed("llama8b")))
     by = bench.metric_bytes(w_lens, 32, 8, 128, 32, False)
@@ -60,6 +93,7 @@ def test_reference_arm_prints_one_json_line_on_cpu():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["unit"] == "GB/s" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 1
+    assert d["cpu_baseline"]["host_threads"] >= 1 and d["cpu_baseline"]["cpu_model"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0
 
 

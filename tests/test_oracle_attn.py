@@ -4,7 +4,8 @@ Each test checks the oracle against something outside it: the closed-form
 slot placement, independent numpy RoPE, a library SDPA in fp64 on a numpy
 gather, an explicit brute-force loop, and the closed-form special cases the
 method has (one-token context returns v exactly; identical keys or a zero
-query give the mean of the values; permuting physical pages changes
+query give the mean of the values; adding one vector to every key, which adds
+one constant to every score, changes nothing; permuting physical pages changes
 nothing)."""
 import math
 
@@ -224,6 +225,47 @@ def test_zero_query_gives_mean_of_values():
         for hh in range(w.Hq):
             V = _gather(h, w, b, hh // G, int(L) + 1, "v_pool", None)
             assert np.allclose(out[b, hh], V.mean(0), rtol=0, atol=1e-13)
+
+
+def _encode_exact(vals, kv_fp8):
+    """Pool codes of values that both formats hold exactly (multiples of 1/4
+    within +-1.5)."""
+    t = torch.from_numpy(np.ascontiguousarray(vals, np.float32))
+    if kv_fp8:
+        return t.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    return bits16(t.to(torch.bfloat16))
+
+
+@pytest.mark.parametrize("kv_fp8", [False, True])
+def test_common_key_offset_shifts_scores_and_changes_nothing(kv_fp8):
+    """softmax(s + c) = softmax(s): keys K_t and K_t + u (the same u for every
+    token of a kv head) give scores that differ by the constant q.u / sqrt(d),
+    so the output must not move beyond fp64 rounding."""
+    w = _small(kv_fp8=kv_fp8, lengths=(5, 40, 70))
+    h = host_inputs(w)
+    cfg = oracle_cfg(w)
+    oracle.rope_append(cfg, h["q"], h["k_new"], h["v_new"], h["k_pool"], h["v_pool"],
+                       h["k_scale"], h["v_scale"], h["block_tables"], h["seq_lens"])
+    rng = np.random.default_rng(9)
+    if kv_fp8:                                    # unit scales: codes are the values themselves
+        h["k_scale"][:] = 1.0
+    base = rng.integers(-2, 3, size=h["k_pool"].shape) / 4.0           # K'  in {-0.5 .. 0.5}
+    u = rng.integers(-4, 5, size=(w.Hkv, w.d)) / 4.0                   # u   in {-1 .. 1}
+    shifted = base + u[None, :, None, :]                                # |K' + u| <= 1.5, exact
+    h["k_pool"][:] = _encode_exact(base, kv_fp8)
+    out0, st0 = oracle.decode_attn(cfg, h["q"], h["k_pool"], h["v_pool"], h["k_scale"], h["v_scale"],
+                                   h["block_tables"], h["seq_lens"])
+    h["k_pool"][:] = _encode_exact(shifted, kv_fp8)
+    out1, st1 = oracle.decode_attn(cfg, h["q"], h["k_pool"], h["v_pool"], h["k_scale"], h["v_scale"],
+                                   h["block_tables"], h["seq_lens"])
+    assert st0 == 0 and st1 == 0
+    # the offset really moves the scores (by q.u / sqrt(d), a few units here)
+    qf = (h["q"].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    G = w.Hq // w.Hkv
+    shift = np.einsum("bhd,hd->bh", qf, np.repeat(u, G, axis=0)) / math.sqrt(w.d)
+    assert np.abs(shift).max() > 1.0
+    assert np.allclose(out0, out1, rtol=0, atol=1e-12)
+    assert np.abs(out0).max() > 0.1
 
 
 @pytest.mark.parametrize("kv_fp8", [False, True])
