@@ -6,8 +6,11 @@ The library is loaded at import.  If it has not been built the import fails
 with an ImportError (build it with ``python -m paged_kv_flight_b200.build``);
 there is no fallback path.
 
-Tensors may be passed as torch tensors (their device pointer is used; they
-must be contiguous) or as raw integer device pointers.  ``stream`` may be a
+Tensors may be passed as torch tensors or as raw integer device pointers.
+A tensor must be a contiguous CUDA tensor of the element type the call reads
+it as: bf16 activations and weights, bf16 or uint8 / float8_e4m3fn pools,
+float32 scales, int32 block tables, lengths and offsets.  Anything else
+raises before the library is called; raw pointers pass through unchecked.  ``stream`` may be a
 ``torch.cuda.Stream``, a raw ``cudaStream_t`` integer, or None for torch's
 current stream.  Each call returns its ``pkv_status``; with ``check=True``
 (the default) a non-OK status raises :class:`PkvError` instead.
@@ -124,16 +127,50 @@ def pkv_status_str(status: int) -> str:
     return lib.pkv_status_str(int(status)).decode()
 
 
-def _ptr(x):
+# element types the library reads each kind of device argument as
+_ACT = (torch.bfloat16,)                                      # q, k_new, v_new, out, x, weights
+_POOL = (torch.bfloat16, torch.uint8, torch.float8_e4m3fn)    # KV pools: bf16, or E4M3 codes
+_F32 = (torch.float32,)                                       # E4M3 scales
+_I32 = (torch.int32,)                                         # block tables, lengths, offsets
+
+
+def _ptr(x, kinds=None, name="argument"):
+    """Device pointer of a device-memory argument: None; a raw integer device
+    pointer (passed through unchecked); or a contiguous CUDA tensor whose
+    dtype is one of `kinds`.  A host tensor or another element type would
+    make the kernels read or write memory the caller did not mean, so it
+    raises here, before the library is called."""
     if x is None:
         return None
     if isinstance(x, int):
         return x
     if isinstance(x, torch.Tensor):
+        if not x.is_cuda:
+            raise ValueError(f"{name}: libpkv takes device tensors, got one on {x.device}")
+        if kinds is not None and x.dtype not in kinds:
+            raise TypeError(f"{name}: expected {' or '.join(str(k) for k in kinds)}, got {x.dtype}")
         if not x.is_contiguous():
-            raise ValueError("libpkv takes contiguous tensors")
+            raise ValueError(f"{name}: libpkv takes contiguous tensors")
         return x.data_ptr()
-    raise TypeError(f"expected a tensor or a device pointer, got {type(x)}")
+    raise TypeError(f"{name}: expected a tensor or a device pointer, got {type(x)}")
+
+
+def _kv(k_pool, v_pool, k_scale, v_scale):
+    """The pools and their scales, in the order every call takes them."""
+    return (_ptr(k_pool, _POOL, "k_pool"), _ptr(v_pool, _POOL, "v_pool"),
+            _ptr(k_scale, _F32, "k_scale"), _ptr(v_scale, _F32, "v_scale"))
+
+
+def _hptr(x, name="argument"):
+    """Host pointer of an int32 host buffer: a contiguous CPU tensor or a raw
+    integer host pointer."""
+    if isinstance(x, int):
+        return x
+    if isinstance(x, torch.Tensor):
+        if x.is_cuda or x.dtype != torch.int32 or not x.is_contiguous():
+            raise ValueError(f"{name}: expected a contiguous int32 host tensor")
+        return x.data_ptr()
+    raise TypeError(f"{name}: expected a tensor or a host pointer, got {type(x)}")
 
 
 # The current CUDA stream of the current device as a raw cudaStream_t: the
@@ -184,9 +221,10 @@ def pkv_rope_append(ctx, q, k_new, v_new, k_pool, v_pool, k_scale, v_scale, bloc
         batch = int(seq_lens.shape[0])
     if bt_stride is None:
         bt_stride = int(block_tables.shape[1])
-    st = lib.pkv_rope_append(ctx, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_pool), _ptr(v_pool),
-                             _ptr(k_scale), _ptr(v_scale), _ptr(block_tables), int(bt_stride),
-                             _ptr(seq_lens), int(batch), _stream(stream))
+    st = lib.pkv_rope_append(ctx, _ptr(q, _ACT, "q"), _ptr(k_new, _ACT, "k_new"), _ptr(v_new, _ACT, "v_new"),
+                             *_kv(k_pool, v_pool, k_scale, v_scale),
+                             _ptr(block_tables, _I32, "block_tables"), int(bt_stride),
+                             _ptr(seq_lens, _I32, "seq_lens"), int(batch), _stream(stream))
     return _done(st, "pkv_rope_append", check)
 
 
@@ -197,8 +235,9 @@ def pkv_decode_attn(ctx, q, k_pool, v_pool, k_scale, v_scale, block_tables, seq_
         batch = int(seq_lens.shape[0])
     if bt_stride is None:
         bt_stride = int(block_tables.shape[1])
-    st = lib.pkv_decode_attn(ctx, _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(k_scale), _ptr(v_scale),
-                             _ptr(block_tables), int(bt_stride), _ptr(seq_lens), int(batch), _ptr(out),
+    st = lib.pkv_decode_attn(ctx, _ptr(q, _ACT, "q"), *_kv(k_pool, v_pool, k_scale, v_scale),
+                             _ptr(block_tables, _I32, "block_tables"), int(bt_stride),
+                             _ptr(seq_lens, _I32, "seq_lens"), int(batch), _ptr(out, _ACT, "out"),
                              _stream(stream))
     return _done(st, "pkv_decode_attn", check)
 
@@ -236,9 +275,10 @@ def pkv_decode_attn_noalloc(cfg: pkv_config, q, k_pool, v_pool, k_scale, v_scale
         batch = int(seq_lens.shape[0])
     if bt_stride is None:
         bt_stride = int(block_tables.shape[1])
-    st = lib.pkv_decode_attn_noalloc(C.byref(cfg), _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(k_scale),
-                                     _ptr(v_scale), _ptr(block_tables), int(bt_stride), _ptr(seq_lens),
-                                     int(batch), _ptr(out), _stream(stream))
+    st = lib.pkv_decode_attn_noalloc(C.byref(cfg), _ptr(q, _ACT, "q"), *_kv(k_pool, v_pool, k_scale, v_scale),
+                                     _ptr(block_tables, _I32, "block_tables"), int(bt_stride),
+                                     _ptr(seq_lens, _I32, "seq_lens"), int(batch), _ptr(out, _ACT, "out"),
+                                     _stream(stream))
     return _done(st, "pkv_decode_attn_noalloc", check)
 
 
@@ -252,9 +292,10 @@ def pkv_rope_append_tokens(ctx, q, k_new, v_new, k_pool, v_pool, k_scale, v_scal
         q_len = int(q.shape[1])
     if bt_stride is None:
         bt_stride = int(block_tables.shape[1])
-    st = lib.pkv_rope_append_tokens(ctx, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_pool), _ptr(v_pool),
-                                    _ptr(k_scale), _ptr(v_scale), _ptr(block_tables), int(bt_stride),
-                                    _ptr(seq_lens), int(batch), int(q_len), _stream(stream))
+    st = lib.pkv_rope_append_tokens(ctx, _ptr(q, _ACT, "q"), _ptr(k_new, _ACT, "k_new"), _ptr(v_new, _ACT, "v_new"),
+                                    *_kv(k_pool, v_pool, k_scale, v_scale),
+                                    _ptr(block_tables, _I32, "block_tables"), int(bt_stride),
+                                    _ptr(seq_lens, _I32, "seq_lens"), int(batch), int(q_len), _stream(stream))
     return _done(st, "pkv_rope_append_tokens", check)
 
 
@@ -268,9 +309,10 @@ def pkv_decode_attn_tokens(ctx, q, k_pool, v_pool, k_scale, v_scale, block_table
         q_len = int(q.shape[1])
     if bt_stride is None:
         bt_stride = int(block_tables.shape[1])
-    st = lib.pkv_decode_attn_tokens(ctx, _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(k_scale), _ptr(v_scale),
-                                    _ptr(block_tables), int(bt_stride), _ptr(seq_lens), int(batch), int(q_len),
-                                    _ptr(out), _stream(stream))
+    st = lib.pkv_decode_attn_tokens(ctx, _ptr(q, _ACT, "q"), *_kv(k_pool, v_pool, k_scale, v_scale),
+                                    _ptr(block_tables, _I32, "block_tables"), int(bt_stride),
+                                    _ptr(seq_lens, _I32, "seq_lens"), int(batch), int(q_len),
+                                    _ptr(out, _ACT, "out"), _stream(stream))
     return _done(st, "pkv_decode_attn_tokens", check)
 
 
@@ -315,7 +357,7 @@ class Pages:
         import numpy as np
         if isinstance(out, np.ndarray):
             return lib.pkv_pages_take_changes(self.h, out.ctypes.data, out.size // 3)
-        return lib.pkv_pages_take_changes(self.h, _ptr(out), int(out.numel()) // 3)
+        return lib.pkv_pages_take_changes(self.h, _hptr(out, "out"), int(out.numel()) // 3)
 
     def close(self):
         if self.h:
@@ -346,9 +388,11 @@ def pkv_rope_append_varlen(ctx, q, k_new, v_new, k_pool, v_pool, k_scale, v_scal
         batch = int(seq_lens.shape[0])
     if bt_stride is None:
         bt_stride = int(block_tables.shape[1])
-    st = lib.pkv_rope_append_varlen(ctx, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_pool), _ptr(v_pool),
-                                    _ptr(k_scale), _ptr(v_scale), _ptr(block_tables), int(bt_stride),
-                                    _ptr(seq_lens), _ptr(cu_q), int(batch), int(q.shape[0]), _stream(stream))
+    st = lib.pkv_rope_append_varlen(ctx, _ptr(q, _ACT, "q"), _ptr(k_new, _ACT, "k_new"), _ptr(v_new, _ACT, "v_new"),
+                                    *_kv(k_pool, v_pool, k_scale, v_scale),
+                                    _ptr(block_tables, _I32, "block_tables"), int(bt_stride),
+                                    _ptr(seq_lens, _I32, "seq_lens"), _ptr(cu_q, _I32, "cu_q"), int(batch),
+                                    int(q.shape[0]), _stream(stream))
     return _done(st, "pkv_rope_append_varlen", check)
 
 
@@ -361,9 +405,10 @@ def pkv_decode_attn_varlen(ctx, q, k_pool, v_pool, k_scale, v_scale, block_table
         batch = int(seq_lens.shape[0])
     if bt_stride is None:
         bt_stride = int(block_tables.shape[1])
-    st = lib.pkv_decode_attn_varlen(ctx, _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(k_scale), _ptr(v_scale),
-                                    _ptr(block_tables), int(bt_stride),
-                                    _ptr(seq_lens), _ptr(cu_q), int(batch), int(q.shape[0]), _ptr(out),
+    st = lib.pkv_decode_attn_varlen(ctx, _ptr(q, _ACT, "q"), *_kv(k_pool, v_pool, k_scale, v_scale),
+                                    _ptr(block_tables, _I32, "block_tables"), int(bt_stride),
+                                    _ptr(seq_lens, _I32, "seq_lens"), _ptr(cu_q, _I32, "cu_q"), int(batch),
+                                    int(q.shape[0]), _ptr(out, _ACT, "out"),
                                     _stream(stream))
     return _done(st, "pkv_decode_attn_varlen", check)
 
@@ -373,8 +418,9 @@ def pkv_table_sync(upload, n_changes: int, batch: int, table, bt_out, lens_out, 
     """upload: device int32 [3 n_changes + 2 batch] (changes, slots, lengths);
     table [max_batch, max_blocks] updated in place; bt_out [>= batch,
     max_blocks] and lens_out [>= batch] receive the batch's rows and lengths."""
-    st = lib.pkv_table_sync(_ptr(upload), int(n_changes), int(batch), int(table.shape[0]), int(table.shape[1]),
-                            int(page_size), _ptr(table), _ptr(bt_out), _ptr(lens_out), _stream(stream))
+    st = lib.pkv_table_sync(_ptr(upload, _I32, "upload"), int(n_changes), int(batch), int(table.shape[0]),
+                            int(table.shape[1]), int(page_size), _ptr(table, _I32, "table"),
+                            _ptr(bt_out, _I32, "bt_out"), _ptr(lens_out, _I32, "lens_out"), _stream(stream))
     return _done(st, "pkv_table_sync", check)
 
 
@@ -388,7 +434,8 @@ def pkv_qkv_launch_shape(ctx, batch: int, hidden: int) -> dict:
 
 def pkv_qkv_pack_weight(ctx, w_qkv, w_tiled, stream=None, check: bool = True) -> int:
     """w_qkv [(Hq + 2 Hkv) d, hidden] -> w_tiled (same size) in the tiled layout."""
-    st = lib.pkv_qkv_pack_weight(ctx, _ptr(w_qkv), int(w_qkv.shape[-1]), _ptr(w_tiled), _stream(stream))
+    st = lib.pkv_qkv_pack_weight(ctx, _ptr(w_qkv, _ACT, "w_qkv"), int(w_qkv.shape[-1]),
+                                 _ptr(w_tiled, _ACT, "w_tiled"), _stream(stream))
     return _done(st, "pkv_qkv_pack_weight", check)
 
 
@@ -402,8 +449,8 @@ def pkv_qkv_rope_append(ctx, x, w_qkv, q_out, k_pool, v_pool, k_scale, v_scale, 
     if bt_stride is None:
         bt_stride = int(block_tables.shape[1])
     hidden = int(x.shape[-1])
-    st = lib.pkv_qkv_rope_append(ctx, _ptr(x), _ptr(w_qkv), hidden, int(w_layout), _ptr(q_out), _ptr(k_pool),
-                                 _ptr(v_pool),
-                                 _ptr(k_scale), _ptr(v_scale), _ptr(block_tables), int(bt_stride), _ptr(seq_lens),
-                                 int(batch), _stream(stream))
+    st = lib.pkv_qkv_rope_append(ctx, _ptr(x, _ACT, "x"), _ptr(w_qkv, _ACT, "w_qkv"), hidden, int(w_layout),
+                                 _ptr(q_out, _ACT, "q_out"), *_kv(k_pool, v_pool, k_scale, v_scale),
+                                 _ptr(block_tables, _I32, "block_tables"), int(bt_stride),
+                                 _ptr(seq_lens, _I32, "seq_lens"), int(batch), _stream(stream))
     return _done(st, "pkv_qkv_rope_append", check)

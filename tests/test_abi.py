@@ -86,11 +86,61 @@ def test_table_sync_rejects_bad_sizes_without_touching_the_device():
     """Argument checks of pkv_table_sync run on the host before any launch."""
     import torch
     from paged_kv_flight_b200 import pkv
+    # host buffers through the raw C entry point: every case below returns
+    # before a pointer is dereferenced or a kernel launched
     t = torch.zeros(4, 8, dtype=torch.int32)
     up = torch.zeros(64, dtype=torch.int32)
     bt, ln = torch.zeros(4, 8, dtype=torch.int32), torch.zeros(4, dtype=torch.int32)
-    call = lambda n, b, P: pkv.pkv_table_sync(up, n, b, t, bt, ln, P, stream=0, check=False)   # noqa: E731
+    call = lambda n, b, P: pkv.lib.pkv_table_sync(up.data_ptr(), n, b, 4, 8, P, t.data_ptr(),   # noqa: E731
+                                                  bt.data_ptr(), ln.data_ptr(), None)
     assert call(-1, 1, 16) == pkv.PKV_ERR_INVALID_ARG
     assert call(0, 5, 16) == pkv.PKV_ERR_INVALID_ARG      # batch above the table's rows
     assert call(0, 1, 0) == pkv.PKV_ERR_INVALID_ARG       # page size
     assert call(0, 0, 16) == pkv.PKV_OK                    # nothing to do
+
+
+def test_binding_rejects_host_tensors_and_wrong_element_types():
+    """The Python binding checks each tensor argument before the library is
+    called: device memory, the element type the kernels read it as, and
+    contiguity.  A host tensor or a narrower element type would have the
+    kernels touch memory the caller did not mean."""
+    import pytest
+    import torch
+    from paged_kv_flight_b200 import pkv
+    q = torch.zeros(2, 8, 64, dtype=torch.bfloat16)          # on the host
+    lens = torch.zeros(2, dtype=torch.int32)
+    bt = torch.zeros(2, 4, dtype=torch.int32)
+    with pytest.raises(ValueError, match="device tensors"):
+        pkv.pkv_decode_attn(None, q, 0x1000, 0x1000, None, None, bt, lens, q)
+    with pytest.raises(ValueError, match="device tensors"):
+        pkv.pkv_table_sync(lens, 0, 0, bt, bt, lens, 16, stream=0)
+    # raw integer pointers pass through unchecked (the C-level checks still run)
+    assert pkv._ptr(0x1000, pkv._ACT, "q") == 0x1000 and pkv._ptr(None, pkv._ACT, "q") is None
+    # the element-type and layout checks, on host tensors that report
+    # themselves as device tensors (no CUDA context is needed)
+    class _OnDevice(torch.Tensor):
+        @property
+        def is_cuda(self):
+            return True
+
+    class _Fake:
+        pass
+
+    dev = lambda dt, n=4: torch.zeros(n, dtype=dt).as_subclass(_OnDevice)   # noqa: E731
+    for dt, kinds in ((torch.float32, pkv._ACT), (torch.float16, pkv._ACT), (torch.int64, pkv._I32),
+                      (torch.int16, pkv._POOL), (torch.float64, pkv._F32)):
+        with pytest.raises(TypeError, match="expected"):
+            pkv._ptr(dev(dt), kinds, "arg")
+    for dt, kinds in ((torch.bfloat16, pkv._ACT), (torch.uint8, pkv._POOL), (torch.float8_e4m3fn, pkv._POOL),
+                      (torch.bfloat16, pkv._POOL), (torch.int32, pkv._I32), (torch.float32, pkv._F32)):
+        t = dev(dt)
+        assert pkv._ptr(t, kinds, "arg") == t.data_ptr()
+    strided = torch.zeros(4, 4, dtype=torch.bfloat16).as_subclass(_OnDevice).t()
+    with pytest.raises(ValueError, match="contiguous"):
+        pkv._ptr(strided, pkv._ACT, "q")
+    with pytest.raises(TypeError):
+        pkv._ptr(_Fake(), pkv._ACT, "q")
+    # the page allocator's change log is a host int32 buffer
+    with pytest.raises(ValueError):
+        pkv._hptr(torch.zeros(6, dtype=torch.int64), "out")
+    assert pkv._hptr(lens, "out") == lens.data_ptr()
