@@ -17,7 +17,7 @@
  * formats' closed forms and a library cast, RoPE identities and a complex-
  * number formulation, brute-force attention loops, a library SDPA in fp64,
  * and the closed-form special cases (one-token context, identical keys,
- * zero query, permuted physical pages).
+ * zero query, one offset added to every key, permuted physical pages).
  */
 #include "pkv_oracle.h"
 
