@@ -14,8 +14,6 @@ import sys
 ROOT = os.path.dirname(os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
 sys.path.insert(0, ROOT)
 
-import numpy as np  # noqa: E402
-
 from tests._util import oracle_step  # noqa: E402
 from paged_kv_flight_b200 import workloads  # noqa: E402
 

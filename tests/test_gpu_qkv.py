@@ -23,7 +23,7 @@ import torch
 import oracle
 from paged_kv_flight_b200 import workloads
 from tests import _gpu
-from tests._util import bf16_ordinal, bits16, bytes8, host_inputs, oracle_cfg
+from tests._util import bits16, bytes8, host_inputs, oracle_cfg
 
 pytestmark = pytest.mark.gpu
 

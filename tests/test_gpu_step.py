@@ -16,7 +16,7 @@ import torch
 import oracle
 from paged_kv_flight_b200 import workloads
 from tests import _gpu
-from tests._util import bf16_ordinal, bits16, bytes8, host_inputs, oracle_cfg, oracle_step
+from tests._util import bf16_ordinal, bits16, bytes8, oracle_step
 
 pytestmark = pytest.mark.gpu
 
