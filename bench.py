@@ -585,8 +585,10 @@ def run_ours(args, name, rank, world, local_rank):
     return line
 
 
-def run_reference(args, name):
-    """The CPU oracle as the reference arm, on a bounded sample per step."""
+def run_reference(args, name, world=1):
+    """The CPU oracle as the reference arm, on a bounded sample per step.
+    Under a multi-rank launch only rank 0 runs it; n_gpus mirrors the
+    launch."""
     import torch
     from paged_kv_flight_b200 import workloads
     dev = "cuda" if torch.cuda.is_available() else "cpu"
@@ -609,7 +611,7 @@ def run_reference(args, name):
               f"{100.0 * by / workload_bytes(w):.1f}% of the step's bytes) per step; plain fp64 C oracle, "
               f"single thread, append + attention")
     return {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": 1,
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic: same seeded workload as the GPU arm",
@@ -927,7 +929,7 @@ def main(argv=None):
         if rank != 0:
             return 0
         for name in names:
-            print(json.dumps(run_reference(args, name)), flush=True)
+            print(json.dumps(run_reference(args, name, world)), flush=True)
         return 0
 
     import torch

@@ -122,3 +122,19 @@ def test_rank_reductions_with_two_gloo_ranks():
     res = sorted(q.get(timeout=10) for _ in range(2))
     assert [r[1] for r in res] == [2.5, 2.5]
     assert [r[2] for r in res] == [30.0, 30.0]
+
+
+def test_reference_arm_under_torchrun_prints_once_from_rank_zero():
+    """Launched like the multi-GPU runs (torchrun, two ranks), the reference
+    arm runs on rank 0 alone: one JSON line, every rank exits 0."""
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    port = 29700 + (os.getpid() % 200)
+    r = subprocess.run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+                        "--master-addr", "127.0.0.1", "--master-port", str(port),
+                        os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config", "tiny",
+                        "--gpus", "2", "--steps", "3", "--warmup", "3"],
+                       capture_output=True, text=True, env=env, timeout=600, check=True)
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
