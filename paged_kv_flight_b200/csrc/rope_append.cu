@@ -13,7 +13,12 @@
 // Several new tokens per request (speculative-decode verification: "Scaling
 // TensorRT-LLM", section "3. Speculative Decoding for Tail Latency") are the
 // same operation at positions L_b + t: the grid's first axis runs over
-// (request, new token) and q / k_new / v_new carry a token axis.
+// (request, new token) and q / k_new / v_new carry a token axis.  With a
+// count of new tokens per request (chunked prefill mixed with decodes:
+// "Scaling TensorRT-LLM", section "What the Scheduler Actually Does") the
+// rows are packed, cu_q[b] .. cu_q[b + 1] - 1 being request b's, and the
+// grid's first axis runs over the packed rows; each finds its request by a
+// binary search of cu_q.
 //
 // Grid (request x new token, chunk): a token's Hq + Hkv rows are cut into work items of
 // 8 rotation pairs (two 16-byte loads, two 16-byte bf16 or 8-byte E4M3
