@@ -2,15 +2,17 @@
 """Benchmark: one in-flight-batched decode step over a paged KV cache
 (RoPE + append, then split-KV GQA decode attention), through the libpkv C ABI.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME|all]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME|suite|all]
                     [--impl ours|reference]
 
-One step = pkv_rope_append + pkv_decode_attn over the whole batch of the
-workload.  Inputs are resident in HBM; before every timed step, outside the
+By default every graded workload is measured in turn (llama8b, hetero70b,
+fp8, spec4, then longctx), one JSON line each; the last line printed is the
+long-context workload's, the largest.  One step = pkv_rope_append +
+pkv_decode_attn over the whole batch of the workload.  Inputs are resident in HBM; before every timed step, outside the
 CUDA-event window, a 2x-L2 buffer is written and another 2x-L2 buffer read,
 so the step finds none of its inputs in L2 and no dirty lines to write back.  The value is
 whole-job HBM throughput: resident KV bytes attended plus q / out bytes, per
-step, summed over ranks, divided by the max-over-ranks step time.  Under
+step, summed over ranks, divided by the max-over-ranks median step time.  Under
 torchrun every rank runs an independent replica of the workload (weak
 scaling; the step has no exchange between GPUs).
 
@@ -39,7 +41,10 @@ if ROOT not in sys.path:
 METRIC = "paged-KV decode attn: HBM GB/s (% of B200 peak), request-tokens/s, step µs"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
-DEFAULT_CONFIG = "llama8b"
+# the default run: every graded workload, the largest (longctx) last so that
+# the last line printed is the long-context one
+SUITE = ("llama8b", "hetero70b", "fp8", "spec4", "longctx")
+DEFAULT_CONFIG = "suite"
 # sources of the kernel whose DRAM traffic a profile line records: the
 # attention kernels for the attention workloads, the fused projection for qkv8b
 KERNEL_SOURCES = {
@@ -322,6 +327,23 @@ def cpu_baseline(w, src, time_budget_s: float = 20.0) -> dict:
                       f"single thread, append + attention"}
 
 
+# ---------------------------------------------------------------- config
+
+L2_NOTE = "flushed before every timed step, outside the event window: write 2x L2, then read 2x L2"
+
+
+def workload_config(w, name, world) -> dict:
+    """The `config` object of a line: the workload alone, identical for the
+    GPU arm and the reference (oracle) arm."""
+    from paged_kv_flight_b200 import workloads
+    return {"workload": name, "description": workloads.DESCRIPTIONS[name], "batch": w.batch,
+            "tokens_attended": int((w.seq_lens.astype(np.int64) + w.q_len).sum()),
+            "new_tokens_per_request": w.q_len,
+            "metric_bytes_per_step": workload_bytes(w),
+            "full_step_bytes": full_step_bytes(w.seq_lens, w.Hq, w.Hkv, w.d, w.P, w.kv_fp8, w.q_len),
+            "l2": L2_NOTE, "replicas": world}
+
+
 # ---------------------------------------------------------------- GPU leg
 
 def _device_inputs(w, device):
@@ -335,7 +357,7 @@ def _device_inputs(w, device):
                 seq_lens=torch.from_numpy(w.seq_lens).to(device).contiguous())
 
 
-def run_ours(args, name, rank, world, local_rank):
+def run_ours(args, name, rank, world, local_rank, cpu_budget=None):
     import torch
     from paged_kv_flight_b200 import pkv, workloads
 
@@ -380,7 +402,7 @@ def run_ours(args, name, rank, world, local_rank):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, dv, args.cpu_budget)
+        cpu = cpu_baseline(w, dv, args.cpu_budget if cpu_budget is None else cpu_budget)
 
     def step():
         rope_call(dv)
@@ -453,9 +475,11 @@ def run_ours(args, name, rank, world, local_rank):
     if st != pkv.PKV_OK:
         raise RuntimeError(f"device error during timing: {pkv.pkv_status_str(st)} bits={bits}")
 
-    eager_max = max_over_ranks(sum(step_ms) / K)
-    attn_max = max_over_ranks(sum(attn_ms) / K)
-    step_max = max_over_ranks(sum(graph_ms) / K) if graph_ms is not None else eager_max
+    med = statistics.median
+    eager_max = max_over_ranks(med(step_ms))
+    attn_max = max_over_ranks(med(attn_ms))
+    step_max = max_over_ranks(med(graph_ms)) if graph_ms is not None else eager_max
+    step_mean = max_over_ranks(sum(graph_ms if graph_ms is not None else step_ms) / K)
     by = workload_bytes(w)
     total_bytes = sum_over_ranks(float(by))
     total_reqs = sum_over_ranks(float(B))
@@ -554,19 +578,15 @@ def run_ours(args, name, rank, world, local_rank):
         "vs_baseline": None, "dtype": "e4m3-kv/bf16" if w.kv_fp8 else "bf16",
         "data": "synthetic: seeded lengths, page permutation, block tables and N(0,1) q/k/v "
                 "(per-workload recipe in paged_kv_flight_b200/workloads.py)",
-        "config": {"workload": name, "description": workloads.DESCRIPTIONS[name], "batch": B,
-                   "tokens_attended": int((w.seq_lens.astype(np.int64) + w.q_len).sum()),
-                   "new_tokens_per_request": w.q_len,
-                   "metric_bytes_per_step": by,
-                   "full_step_bytes": full_step_bytes(w.seq_lens, w.Hq, w.Hkv, w.d, w.P, w.kv_fp8, w.q_len),
-                   "l2": "flushed before every timed step, outside the event window: write 2x L2, then read 2x L2",
-                   "timing": ("each step replayed from one CUDA-graph capture of pkv_rope_append + pkv_decode_attn "
-                              "(3 kernels); per-kernel times from the same steps launched eagerly"
-                              if graph_ms is not None else "eager launches through the C ABI"),
-                   "replicas": world},
+        "config": workload_config(w, name, world),
+        "timing": ("median over the timed steps; each step replayed from one CUDA-graph capture of "
+                   "pkv_rope_append + pkv_decode_attn (3 kernels); per-kernel times from the same steps "
+                   "launched eagerly" if graph_ms is not None
+                   else "median over the timed steps; eager launches through the C ABI"),
         "request_tokens_per_s": total_reqs / (step_max * 1e-3),
         "step_us": step_max * 1e3, "step_us_eager": eager_max * 1e3, "attn_us": attn_max * 1e3,
-        "rope_append_us": max_over_ranks(sum(rope_ms) / K) * 1e3,
+        "rope_append_us": max_over_ranks(med(rope_ms)) * 1e3,
+        "ms_per_step_mean": step_mean,
         "step_us_hot_l2": hot_ms * 1e3,
         "pct_of_8TBs": 100.0 * value / world / NOMINAL_HBM_GBS,
         "pct_of_measured_peak": 100.0 * value / world / peak,
@@ -585,16 +605,24 @@ def run_ours(args, name, rank, world, local_rank):
     return line
 
 
-def run_reference(args, name, world=1):
-    """The CPU oracle as the reference arm, on a bounded sample per step.
-    Under a multi-rank launch only rank 0 runs it; n_gpus mirrors the
-    launch."""
+def run_reference(args, name, world=1, time_budget_s=45.0):
+    """The CPU oracle as the reference arm, on a bounded sample per step: a
+    prefix of the batch sized so that the warm-up and timed steps together
+    take about `time_budget_s` of CPU time (at least one request; at most
+    --ref-budget attended token-heads).  The oracle's rate is calibrated on
+    the first request.  Under a multi-rank launch only rank 0 runs it; n_gpus
+    mirrors the launch."""
     import torch
     from paged_kv_flight_b200 import workloads
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     w = workloads.make(name, device=dev)
     src = _device_inputs(w, dev)
-    picks = sample_requests(w, args.ref_budget)
+    first = _request_pages(w, 0, src)
+    t0 = time.perf_counter()
+    oracle_step_requests(w, [first])
+    rate = (int(w.seq_lens[0]) + w.q_len) * w.Hkv / max(time.perf_counter() - t0, 1e-6)   # token-heads / s
+    budget = int(min(args.ref_budget, rate * time_budget_s / (args.steps + args.warmup)))
+    picks = sample_requests(w, budget)
     views = [_request_pages(w, b, src) for b in picks]
     by = metric_bytes(w.seq_lens[picks], w.Hq, w.Hkv, w.d, w.P, w.kv_fp8, w.q_len)
     for _ in range(args.warmup):
@@ -604,7 +632,7 @@ def run_reference(args, name, world=1):
         t0 = time.perf_counter()
         oracle_step_requests(w, views)
         ts.append(time.perf_counter() - t0)
-    sec = sum(ts) / len(ts)
+    sec = statistics.median(ts)
     value = by / sec / 1e9
     toks = int((w.seq_lens[picks].astype(np.int64) + w.q_len).sum())
     sample = (f"requests 0..{len(picks) - 1} of {w.batch} ({toks} attended tokens, "
@@ -615,8 +643,9 @@ def run_reference(args, name, world=1):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic: same seeded workload as the GPU arm",
-        "config": {"workload": name, "description": workloads.DESCRIPTIONS[name], "batch": w.batch,
-                   "metric_bytes_per_step_sampled": by},
+        "config": workload_config(w, name, world),
+        "timing": "median over the timed steps of the oracle on the sampled requests (host wall clock)",
+        "metric_bytes_per_step_sampled": by,
         "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample,
                          **host_cpu()},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -716,9 +745,9 @@ def run_qkv(args, rank, world, local_rank):
         raise RuntimeError(f"device error: {pkv.pkv_status_str(st)} bits={bits}")
     del graph
     pkv.pkv_destroy(ctx)
-    proj_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev) / K)
-    rows_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in rev) / K)
-    step_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in gev) / K)
+    proj_ms = max_over_ranks(statistics.median(a.elapsed_time(b) for a, b in ev))
+    rows_ms = max_over_ranks(statistics.median(a.elapsed_time(b) for a, b in rev))
+    step_ms = max_over_ranks(statistics.median(a.elapsed_time(b) for a, b in gev))
     # the projection's algorithmic bytes: weights and x read once, q written,
     # k and v rows written; its flops: 2 x tokens x features x hidden
     proj_bytes = N * hidden * 2 + w.batch * hidden * 2 + w.batch * N * 2
@@ -836,8 +865,8 @@ def run_mixed(args, rank, world, local_rank):
         raise RuntimeError(f"device error: {pkv.pkv_status_str(st)} bits={bits}")
     del graph
     pkv.pkv_destroy(ctx)
-    step_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in gev) / K)
-    attn_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in aev) / K)
+    step_ms = max_over_ranks(statistics.median(a.elapsed_time(b) for a, b in gev))
+    attn_ms = max_over_ranks(statistics.median(a.elapsed_time(b) for a, b in aev))
     L = w.seq_lens.astype(np.int64)
     row = 2 * w.Hkv * w.d * 2                      # K + V bytes of one token
     # metric bytes: each request's cache (its new tokens included) once, q and out of every new token
@@ -907,7 +936,8 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--config", default=DEFAULT_CONFIG)
+    ap.add_argument("--config", default=DEFAULT_CONFIG,
+                    help="a workload, 'suite' (the default: " + ", ".join(SUITE) + ", in that order) or 'all'")
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -922,14 +952,20 @@ def main(argv=None):
         ap.error("--warmup must be >= 3")
 
     from paged_kv_flight_b200 import workloads
-    names = list(workloads.CONFIG_NAMES) + list(workloads.TOKEN_CONFIG_NAMES) if args.config == "all" else [args.config]
+    if args.config == "all":
+        names = list(workloads.CONFIG_NAMES) + list(workloads.TOKEN_CONFIG_NAMES)
+    elif args.config == "suite":
+        names = list(SUITE)
+    else:
+        names = [args.config]
     rank, world, local_rank = dist_info()
 
     if args.impl == "reference":
         if rank != 0:
             return 0
-        for name in names:
-            print(json.dumps(run_reference(args, name, world)), flush=True)
+        for i, name in enumerate(names):
+            last = i == len(names) - 1
+            print(json.dumps(run_reference(args, name, world, time_budget_s=45.0 if last else 12.0)), flush=True)
         return 0
 
     import torch
@@ -939,7 +975,8 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        for name in names:
+        for i, name in enumerate(names):
+            last = i == len(names) - 1
             if name == "loop70b":
                 line = run_loop(args, rank, world, local_rank)
             elif name == "qkv8b":
@@ -947,7 +984,9 @@ def main(argv=None):
             elif name == "mixed":
                 line = run_mixed(args, rank, world, local_rank)
             else:
-                line = run_ours(args, name, rank, world, local_rank)
+                # the full CPU-baseline budget on the last line printed, a short one before it
+                line = run_ours(args, name, rank, world, local_rank,
+                                cpu_budget=args.cpu_budget if last else min(5.0, args.cpu_budget))
             if rank == 0:
                 print(json.dumps(line), flush=True)
     finally:

@@ -649,8 +649,14 @@ cudaError_t prepare_t(int num_sms, int max_batch, AttnLaunch* out)
     while (stages > 2 && smem_bytes_for<D, FP8, TT>(stages, max_batch) > budget) --stages;
     if (smem_bytes_for<D, FP8, TT>(stages, max_batch) > budget) return cudaErrorInvalidConfiguration;
     const size_t bytes = smem_bytes_for<D, FP8, TT>(stages, max_batch);
+    // The limit is one setting per kernel for the whole process, shared by
+    // every context: set it for the largest batch any context may have, so
+    // that creating a context with a smaller batch never lowers it under a
+    // context that launches with more (each launch still asks for `bytes`).
+    const size_t limit = smem_bytes_for<D, FP8, TT>(stages, kMaxBatch);
+    if (limit > budget) return cudaErrorInvalidConfiguration;
     e = cudaFuncSetAttribute(decode_attn_kernel<D, FP8, kAttnWarps, TT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)bytes);
+                             (int)limit);
     if (e != cudaSuccess) return e;
     e = combine_prepare(D);
     if (e != cudaSuccess) return e;

@@ -593,9 +593,12 @@ cudaError_t prepare_tokens_t(int num_sms, int max_batch, AttnLaunch* out)
     if (e != cudaSuccess) return e;
     const int stages = kAttnMaxStages;
     const size_t bytes = tokens_smem_bytes<D, FP8>(stages, max_batch);
-    if (bytes > (size_t)optin - 256) return cudaErrorInvalidConfiguration;
+    // one process-wide limit per kernel: set for the largest batch any
+    // context may have (see decode_attn.cu), never lowered by a smaller one
+    const size_t limit = tokens_smem_bytes<D, FP8>(stages, kMaxBatch);
+    if (bytes > limit || limit > (size_t)optin - 256) return cudaErrorInvalidConfiguration;
     e = cudaFuncSetAttribute(decode_attn_tokens_kernel<D, FP8, kAttnWarps>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)limit);
     if (e != cudaSuccess) return e;
     e = combine_prepare(D);
     if (e != cudaSuccess) return e;

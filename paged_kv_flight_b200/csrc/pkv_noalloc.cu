@@ -15,8 +15,9 @@
 //
 // Set-up, once per device, on the first call made while that device is
 // current: the device address of the array is looked up with
-// cudaGetSymbolAddress and cached.  That first call should therefore come
-// before any stream capture.  Every call shares the one array, which keeps
+// cudaGetSymbolAddress and cached, with the SM count and the attention
+// kernel's attributes (set once per head_dim / KV type).  That first call
+// should therefore come before any stream capture.  Every call shares the one array, which keeps
 // the previous call's contents: the error word is cleared with
 // cudaMemsetAsync on the caller's stream at each call, and everything else is
 // written before it is read within the call, so calls ordered
@@ -40,24 +41,50 @@ constexpr int kMaxDevices = 64;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
 std::mutex g_setup_mutex;
-void* g_scratch_ptr[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device (looked up once
-// per device), or nullptr on failure.
-void* scratch_on_current_device()
+// Per-device state set up once, under g_setup_mutex, with the device current:
+// the scratch array's device address, the SM count, and the attention launch
+// shape (kernel attributes set then) of each (head_dim, KV type, tile) variant.
+struct DeviceSetup {
+    void* scratch = nullptr;
+    int num_sms = 0;
+    bool launch_ready[2][2][2] = {};          // [head_dim 128][E4M3][32-token tiles]
+    pkv::AttnLaunch launch[2][2][2];
+};
+DeviceSetup g_setup[kMaxDevices];
+
+// The current device's set-up, with the launch shape for cfg in *L; nullptr
+// on failure.
+const DeviceSetup* setup_current_device(const pkv_config* cfg, pkv::AttnLaunch* L)
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
     std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (!g_scratch_ptr[dev]) {
+    DeviceSetup& s = g_setup[dev];
+    if (!s.scratch) {
         void* ptr = nullptr;
         if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) {
             cudaGetLastError();
             return nullptr;
         }
-        g_scratch_ptr[dev] = ptr;
+        int sms = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+            return nullptr;
+        s.num_sms = sms;
+        s.scratch = ptr;
     }
-    return g_scratch_ptr[dev];
+    const bool fp8 = cfg->kv_dtype == PKV_KV_FP8_E4M3;
+    const int i = cfg->head_dim == 128, j = fp8 ? 1 : 0, k = pkv::attn_tile(fp8, cfg->page_size) == pkv::kTileWide;
+    if (!s.launch_ready[i][j][k]) {
+        // sized for the largest batch: the kernel's shared-memory limit is the
+        // same one every context sets, so this never lowers it
+        if (pkv::attn_prepare(cfg->head_dim, fp8, cfg->page_size, s.num_sms, pkv::kMaxBatch, &s.launch[i][j][k]) !=
+            cudaSuccess)
+            return nullptr;
+        s.launch_ready[i][j][k] = true;
+    }
+    *L = s.launch[i][j][k];
+    return &s;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -124,28 +151,19 @@ extern "C" pkv_status pkv_decode_attn_noalloc(const pkv_config* cfg, const void*
     const bool fp8 = cfg->kv_dtype == PKV_KV_FP8_E4M3;
     if (fp8 && (!k_scale || !v_scale || !aligned16(k_scale) || !aligned16(v_scale))) return PKV_ERR_INVALID_ARG;
 
-    void* scratch = scratch_on_current_device();
-    if (!scratch) return PKV_ERR_CUDA;
-    int dev = 0, num_sms = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        return PKV_ERR_CUDA;
+    pkv::AttnLaunch L;
+    const DeviceSetup* setup = setup_current_device(cfg, &L);
+    if (!setup) return PKV_ERR_CUDA;
 
     // scratch layout: [error word, chunk counter | split geometry | partial rows | partial (m, l)];
     // a static split (no dynamic tail): two partial slots per warp
-    const size_t workers = (size_t)num_sms * pkv::kAttnWarps;
+    const size_t workers = (size_t)setup->num_sms * pkv::kAttnWarps;
     const size_t b_err = 256;
     const size_t b_cnt = ((size_t)(batch + 8) * sizeof(int) + 255) & ~(size_t)255;
     const size_t b_po = 2 * workers * pkv::kMaxGroup * cfg->head_dim * sizeof(float);
     const size_t b_pml = 2 * workers * pkv::kMaxGroup * 2 * sizeof(float);
     if (b_err + b_cnt + b_po + b_pml > kScratchBytes) return PKV_ERR_UNSUPPORTED;   // beyond the fixed scratch
-    unsigned char* base = static_cast<unsigned char*>(scratch);
-
-    // the largest batch the shared memory is sized for, so that this call never
-    // lowers the kernel's shared-memory limit below what a context set
-    pkv::AttnLaunch L;
-    if (pkv::attn_prepare(cfg->head_dim, fp8, cfg->page_size, num_sms, pkv::kMaxBatch, &L) != cudaSuccess)
-        return PKV_ERR_CUDA;
+    unsigned char* base = static_cast<unsigned char*>(setup->scratch);
 
     CUtensorMap tmk, tmv;
     if (!encode_pool(cfg, k_pool, &tmk) || !encode_pool(cfg, v_pool, &tmv)) return PKV_ERR_CUDA;

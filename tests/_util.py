@@ -74,3 +74,39 @@ def varlen_host(w: Workload, q_lens) -> dict:
         h[key] = np.ascontiguousarray(np.concatenate([h[key][b, :int(q)] for b, q in enumerate(q_lens)]))
     h["cu_q"] = cu
     return h
+
+
+def oracle_attn_threaded(w: Workload, h: dict, threads: int | None = None):
+    """The oracle's attention of the whole batch, every (request, new token,
+    kv head) group in its own call of the single-threaded C functions, the
+    calls spread over host threads (the C library keeps no state and ctypes
+    releases the GIL), longest requests first.  Returns (out, status) like
+    oracle.decode_attn / decode_attn_tokens: [batch, Hq, d] for one new token
+    per request, [batch, q_len, Hq, d] for several."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+
+    cfg = oracle_cfg(w)
+    G = w.Hq // w.Hkv
+    tok = w.q_len > 1
+    shape = (w.batch, w.q_len, w.Hq, w.d) if tok else (w.batch, w.Hq, w.d)
+    out = np.full(shape, np.nan)
+    order = np.argsort(-np.asarray(w.seq_lens, np.int64), kind="stable")
+    jobs = [(int(b), t, kvh) for b in order for t in range(w.q_len) for kvh in range(w.Hkv)]
+
+    def run(job):
+        b, t, kvh = job
+        if tok:
+            o, st = oracle.decode_attn_tokens_group(cfg, h["q"], h["k_pool"], h["v_pool"], h["k_scale"],
+                                                    h["v_scale"], h["block_tables"], h["seq_lens"], b, t, kvh)
+            out[b, t, kvh * G:(kvh + 1) * G] = o
+        else:
+            o, st = oracle.decode_attn_group(cfg, h["q"], h["k_pool"], h["v_pool"], h["k_scale"], h["v_scale"],
+                                             h["block_tables"], h["seq_lens"], b, kvh)
+            out[b, kvh * G:(kvh + 1) * G] = o
+        return st
+
+    n = threads or max(1, min(32, (os.cpu_count() or 1)))
+    with ThreadPoolExecutor(max_workers=n) as ex:
+        status = max(ex.map(run, jobs), default=0)
+    return out, status

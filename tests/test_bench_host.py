@@ -94,6 +94,15 @@ def test_reference_arm_prints_one_json_line_on_cpu():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 1
     assert d["cpu_baseline"]["host_threads"] >= 1 and d["cpu_baseline"]["cpu_model"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0
+    # the config object is the workload's, the same one the GPU arm prints
+    assert d["config"] == bench.workload_config(workloads.make("tiny"), "tiny", 1)
+
+
+def test_default_suite_ends_on_the_largest_workload():
+    assert bench.DEFAULT_CONFIG == "suite"
+    sizes = {n: bench.workload_bytes(workloads.make(n)) for n in bench.SUITE}
+    assert bench.SUITE[-1] == "longctx" and sizes["longctx"] == max(sizes.values())
+    assert {"llama8b", "hetero70b", "fp8", "spec4"} <= set(bench.SUITE)
 
 
 def _rank_main(rank, world, port, q):

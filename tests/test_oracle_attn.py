@@ -15,7 +15,7 @@ import torch
 
 import oracle
 from paged_kv_flight_b200 import workloads
-from tests._util import bits16, host_inputs, oracle_cfg, bf16_ordinal
+from tests._util import bits16, host_inputs, oracle_attn_threaded, oracle_cfg, bf16_ordinal
 from tests.test_oracle_rope import _complex_rope
 
 
@@ -316,3 +316,27 @@ def test_tiny_regression_fixture():
     with open(path) as f:
         stored = [ln.rstrip("\n") for ln in f if not ln.startswith("#")]
     assert rows() == stored
+
+
+@pytest.mark.parametrize("kv_fp8,q_len", [(False, 1), (True, 1), (False, 3)])
+def test_threaded_whole_batch_helper_equals_the_batch_call(kv_fp8, q_len):
+    # the GPU tests' whole-batch oracle runs one C call per (request, new
+    # token, kv head) on host threads; it must give exactly the batch call
+    w = workloads.build("thr", 16, 4, 64, 16, kv_fp8, 1e4, [0, 15, 16, 200, 77, 513], seed=5, device="cpu",
+                        q_len=q_len)
+    h = host_inputs(w)
+    cfg = oracle_cfg(w)
+    if q_len == 1:
+        assert oracle.rope_append(cfg, h["q"], h["k_new"], h["v_new"], h["k_pool"], h["v_pool"], h["k_scale"],
+                                  h["v_scale"], h["block_tables"], h["seq_lens"]) == 0
+        ref, st = oracle.decode_attn(cfg, h["q"], h["k_pool"], h["v_pool"], h["k_scale"], h["v_scale"],
+                                     h["block_tables"], h["seq_lens"])
+    else:
+        assert oracle.rope_append_tokens(cfg, h["q"], h["k_new"], h["v_new"], h["k_pool"], h["v_pool"],
+                                         h["k_scale"], h["v_scale"], h["block_tables"], h["seq_lens"]) == 0
+        ref, st = oracle.decode_attn_tokens(cfg, h["q"], h["k_pool"], h["v_pool"], h["k_scale"], h["v_scale"],
+                                            h["block_tables"], h["seq_lens"])
+    assert st == 0
+    out, st2 = oracle_attn_threaded(w, h, threads=4)
+    assert st2 == 0
+    assert out.shape == ref.shape and np.array_equal(out, ref)

@@ -62,6 +62,34 @@ def test_noalloc_matches_context_entry_point_twice(pkv, case):
         assert finite and mx <= t["max"] and mean <= t["mean"]
 
 
+def test_noalloc_calls_of_different_shapes_in_a_row(pkv):
+    """A large call (d 128, 8 requests, many split partials) and then a tiny
+    one (d 64) on the same stream, with nothing cleared in between: the second
+    must not pick up the first's split geometry or partials from the shared
+    scratch array.  Its output buffer starts as NaN."""
+    big = workloads.build("bf16", 32, 8, 128, 32, False, 5e5, [0, 15, 16, 100, 1000, 4095, 2500, 77], seed=21)
+    tiny = workloads.make("tiny")
+    outs = {}
+    for w in (big, tiny):
+        _, ref, _ = oracle_step(w)
+        dv = _gpu.to_device(w)
+        ctx = _gpu.make_ctx(pkv, w)
+        try:
+            pkv.pkv_rope_append(ctx, dv["q"], dv["k_new"], dv["v_new"], dv["k_pool"], dv["v_pool"], dv["k_scale"],
+                                dv["v_scale"], dv["block_tables"], dv["seq_lens"])
+            assert pkv.pkv_check_device_error(ctx)[0] == pkv.PKV_OK
+        finally:
+            pkv.pkv_destroy(ctx)
+        out = torch.full((w.batch, w.Hq, w.d), float("nan"), dtype=torch.bfloat16, device="cuda")
+        pkv.pkv_decode_attn_noalloc(_cfg(pkv, w), dv["q"], dv["k_pool"], dv["v_pool"], dv["k_scale"],
+                                    dv["v_scale"], dv["block_tables"], dv["seq_lens"], out)
+        outs[w.name] = (out, ref)
+    torch.cuda.synchronize()
+    for name, (out, ref) in outs.items():
+        mx, mean, finite = _gpu.errors(out, ref)
+        assert finite and mx <= _gpu.TOL_BF16["max"] and mean <= _gpu.TOL_BF16["mean"], (name, mx, mean)
+
+
 def test_noalloc_rejects_bad_calls_before_launching(pkv):
     # every case is refused on the host, before anything is launched or read
     w = workloads.build("rej", 8, 2, 64, 16, False, 1e4, [5, 9], seed=2)
