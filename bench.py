@@ -7,8 +7,9 @@
 
 By default every graded workload is measured in turn (llama8b, hetero70b,
 fp8, spec4, then longctx), one JSON line each; the last line printed is the
-long-context workload's, the largest.  One step = pkv_rope_append +
-pkv_decode_attn over the whole batch of the workload.  Inputs are resident in HBM; before every timed step, outside the
+long-context workload's, the largest.  One step = pkv_decode_step (RoPE +
+append, then the attention as a programmatic dependent of the append kernel,
+then the split combine) over the whole batch of the workload.  Inputs are resident in HBM; before every timed step, outside the
 CUDA-event window, a 2x-L2 buffer is written and another 2x-L2 buffer read,
 so the step finds none of its inputs in L2 and no dirty lines to write back.  The value is
 whole-job HBM throughput: resident KV bytes attended plus q / out bytes, per
@@ -404,9 +405,15 @@ def run_ours(args, name, rank, world, local_rank, cpu_budget=None):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, dv, args.cpu_budget if cpu_budget is None else cpu_budget)
 
-    def step():
-        rope_call(dv)
-        attn_call(dv, out)
+    def step(x=dv, o=out, stream=None):
+        """One step: pkv_decode_step (the attention a programmatic dependent
+        of the append kernel), or with --two-calls the two calls."""
+        if args.two_calls:
+            rope_call(x, stream=stream)
+            attn_call(x, o, stream=stream)
+        else:
+            pkv.pkv_decode_step(ctx, x["q"], x["k_new"], x["v_new"], dv["k_pool"], dv["v_pool"], dv["k_scale"],
+                                dv["v_scale"], x["block_tables"], x["seq_lens"], o, q_len=w.q_len, stream=stream)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -467,6 +474,19 @@ def run_ours(args, name, rank, world, local_rank, cpu_budget=None):
         barrier()
         graph_ms = [a.elapsed_time(b) for a, b in gev]
         del graph
+
+    # timed region 3: the same K steps launched eagerly as one call each
+    sev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    torch.cuda.synchronize()
+    for k in range(K):
+        flush.zero_()
+        sev[k][0].record()
+        step()
+        sev[k][1].record()
+    clocks.sample()
+    torch.cuda.synchronize()
+    barrier()
+    step_call_ms = [a.elapsed_time(b) for a, b in sev]
     clock_info = clocks.stop()
     step_ms = [a.elapsed_time(c) for a, _, c in ev]
     rope_ms = [a.elapsed_time(b) for a, b, _ in ev]
@@ -538,8 +558,7 @@ def run_ours(args, name, rank, world, local_rank, cpu_budget=None):
                 s_comp.wait_event(ev_in[sl])
                 if i >= 2:
                     s_comp.wait_event(ev_out[sl])         # output slot read back
-                rope_call(v, stream=s_comp)
-                attn_call(v, outs[sl], stream=s_comp)
+                step(v, outs[sl], stream=s_comp)
                 ev_comp[sl].record(s_comp)
                 s_out.wait_event(ev_comp[sl])
                 with torch.cuda.stream(s_out):
@@ -580,11 +599,13 @@ def run_ours(args, name, rank, world, local_rank, cpu_budget=None):
                 "(per-workload recipe in paged_kv_flight_b200/workloads.py)",
         "config": workload_config(w, name, world),
         "timing": ("median over the timed steps; each step replayed from one CUDA-graph capture of "
-                   "pkv_rope_append + pkv_decode_attn (3 kernels); per-kernel times from the same steps "
-                   "launched eagerly" if graph_ms is not None
+                   + ("pkv_rope_append + pkv_decode_attn" if args.two_calls else "pkv_decode_step")
+                   + " (3 kernels); per-kernel times (rope_append_us, attn_us, step_us_eager) from the same "
+                   "steps launched eagerly as two calls with events between them" if graph_ms is not None
                    else "median over the timed steps; eager launches through the C ABI"),
         "request_tokens_per_s": total_reqs / (step_max * 1e-3),
-        "step_us": step_max * 1e3, "step_us_eager": eager_max * 1e3, "attn_us": attn_max * 1e3,
+        "step_us": step_max * 1e3, "step_us_eager_one_call": max_over_ranks(med(step_call_ms)) * 1e3,
+        "step_us_eager": eager_max * 1e3, "attn_us": attn_max * 1e3,
         "rope_append_us": max_over_ranks(med(rope_ms)) * 1e3,
         "ms_per_step_mean": step_mean,
         "step_us_hot_l2": hot_ms * 1e3,
@@ -942,6 +963,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay timing")
+    ap.add_argument("--two-calls", action="store_true",
+                    help="time the step as pkv_rope_append + pkv_decode_attn instead of pkv_decode_step")
     ap.add_argument("--tail-chunks", type=int, default=None,
                     help="cap on dynamic tail chunks per warp range (library default if omitted; 0: static split)")
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")

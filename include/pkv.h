@@ -51,6 +51,8 @@
  * ceil(n_b / P) are never read.
  *
  * Beyond the step (each declared below with its own contract):
+ *   pkv_decode_step                                  both parts of the step in
+ *       one call, the attention overlapping the end of the append;
  *   pkv_rope_append_tokens / pkv_decode_attn_tokens  several new tokens per
  *       request, the same count for all (speculative verification);
  *   pkv_rope_append_varlen / pkv_decode_attn_varlen  a count per request,
@@ -179,6 +181,23 @@ pkv_status pkv_decode_attn_tokens(pkv_ctx* ctx, const void* q, const void* k_poo
                                   const int32_t* block_tables, int bt_stride,
                                   const int32_t* seq_lens, int batch, int q_len, void* out,
                                   cudaStream_t stream);
+
+/* The whole step in one call: pkv_rope_append then pkv_decode_attn (q_len =
+ * 1), or pkv_rope_append_tokens then pkv_decode_attn_tokens (q_len > 1,
+ * G * q_len <= 16), with the same arguments, layouts, results and errors as
+ * that pair of calls (q rotated in place, the new tokens appended, out
+ * written).  The pages fuse the attention-side work of a decode step into as
+ * few passes as possible ("Scaling TensorRT-LLM: Kernel Fusion and Inflight
+ * Batching in Production", section "What Gets Fused"); here the attention is
+ * launched as a programmatic dependent of the RoPE + append kernel, so its
+ * start (the split over the SMs, the first page-table lookups) runs while
+ * that kernel finishes; it reads q and issues its first tile load only once
+ * the append is complete.  On a host-side error nothing is launched; if the
+ * append launches and the attention does not, PKV_ERR_CUDA is returned. */
+pkv_status pkv_decode_step(pkv_ctx* ctx, void* q, const void* k_new, const void* v_new,
+                           void* k_pool, void* v_pool, const float* k_scale, const float* v_scale,
+                           const int32_t* block_tables, int bt_stride, const int32_t* seq_lens,
+                           int batch, int q_len, void* out, cudaStream_t stream);
 
 /* Several new tokens per request, a different number for each ("varlen"):
  * chunked prefill mixed with decode in one batch ("Scaling TensorRT-LLM:

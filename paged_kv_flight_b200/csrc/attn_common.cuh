@@ -171,5 +171,27 @@ __device__ __forceinline__ Lookahead lookahead_fill(const AttnParams& p, const i
     return la;
 }
 
+// Launches an attention kernel (K / V tensor maps, parameters); with `pdl`
+// as a programmatic dependent of the kernel before it on the stream, which
+// lets its prologue (split, page lookahead) run while that kernel finishes.
+// The kernel waits for it (grid_dependency_wait) before it reads q or issues
+// a tile load.
+template <typename... Args>
+cudaError_t launch_attn_kernel(void (*kern)(Args...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                               bool pdl, const CUtensorMap& tmk, const CUtensorMap& tmv, const AttnParams& p)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, tmk, tmv, p);
+}
+
 }  // namespace attn
 }  // namespace pkv

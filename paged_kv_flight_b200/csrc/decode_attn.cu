@@ -189,10 +189,12 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
     // ...) from two 32-tile lookahead windows (la_cur from index la_i, la_nxt;
     // la_fill is the first tile of the window after them).  When kClaimAhead
     // tiles of the unit are left to issue it claims the next tail chunk
-    // (atomic on the chunk counter) and, once the unit is fully issued, reads
-    // the claim and loads the first window of the next unit (nU, la_new).
+    // (atomic on the chunk counter); when kResolveAhead are left it reads the
+    // claim and starts the page-id (and scale) loads of the next unit's first
+    // window (nU, la_new), so that neither latency stalls the first issue of
+    // the next unit.
     constexpr int kNone = -1, kPending = -2;
-    constexpr int kClaimAhead = 2;
+    constexpr int kClaimAhead = 4, kResolveAhead = 2;
     int pU = w * (sp.K + 1);
     long long pu0 = sp.ustart(pU), pu1 = sp.ustart(pU + 1);
     int p_left = (int)(pu1 - pu0);   // a head holds at most T / W + 1 tiles
@@ -263,7 +265,7 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
                 if (lane == 0) claim = atomicAdd(p.claim, 1);
                 claim_sent = true;
             }
-            if (p_left == 0) {
+            if (claim_sent && p_left <= kResolveAhead) {
                 const int c = __shfl_sync(kFull, claim, 0);
                 claim_sent = false;
                 if (c >= n_chunks) {
@@ -280,6 +282,10 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
         return true;
     };
 
+    // everything above reads only seq_lens and block_tables; q and the slots
+    // the RoPE + append kernel writes are read after it has finished (a
+    // no-op unless launched as its programmatic dependent)
+    grid_dependency_wait();
     int issued = 0;
     while (issued < S && issue_next(issued)) ++issued;
 
@@ -683,24 +689,24 @@ cudaError_t attn_prepare(int head_dim, bool fp8, int page_size, int num_sms, int
 }
 
 cudaError_t launch_decode_attn(const AttnParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
-                               int head_dim, bool fp8, const AttnLaunch& L, cudaStream_t stream)
+                               int head_dim, bool fp8, const AttnLaunch& L, cudaStream_t stream, bool pdl)
 {
     const dim3 grid(L.ctas), block(kAttnWarps * 32);
     AttnParams q = p;
     q.stages = L.stages;
     const bool wide = L.tile == kTileWide;
+    cudaError_t e;
     if (head_dim == 128) {
-        if (!fp8) decode_attn_kernel<128, false, kAttnWarps, kTile><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
+        if (!fp8) e = launch_attn_kernel(decode_attn_kernel<128, false, kAttnWarps, kTile>, grid, block, L.smem_bytes, stream, pdl, tmk, tmv, q);
         else if (wide)
-            decode_attn_kernel<128, true, kAttnWarps, kTileWide><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
-        else decode_attn_kernel<128, true, kAttnWarps, kTile><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
+            e = launch_attn_kernel(decode_attn_kernel<128, true, kAttnWarps, kTileWide>, grid, block, L.smem_bytes, stream, pdl, tmk, tmv, q);
+        else e = launch_attn_kernel(decode_attn_kernel<128, true, kAttnWarps, kTile>, grid, block, L.smem_bytes, stream, pdl, tmk, tmv, q);
     } else {
-        if (!fp8) decode_attn_kernel<64, false, kAttnWarps, kTile><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
+        if (!fp8) e = launch_attn_kernel(decode_attn_kernel<64, false, kAttnWarps, kTile>, grid, block, L.smem_bytes, stream, pdl, tmk, tmv, q);
         else if (wide)
-            decode_attn_kernel<64, true, kAttnWarps, kTileWide><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
-        else decode_attn_kernel<64, true, kAttnWarps, kTile><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
+            e = launch_attn_kernel(decode_attn_kernel<64, true, kAttnWarps, kTileWide>, grid, block, L.smem_bytes, stream, pdl, tmk, tmv, q);
+        else e = launch_attn_kernel(decode_attn_kernel<64, true, kAttnWarps, kTile>, grid, block, L.smem_bytes, stream, pdl, tmk, tmv, q);
     }
-    const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     return launch_combine(q, head_dim, (int)max_units(L.ctas * kAttnWarps, p.tail_chunks), L.ctas, stream);
 }

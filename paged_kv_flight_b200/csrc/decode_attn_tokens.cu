@@ -261,6 +261,9 @@ decode_attn_tokens_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_
         }
     };
 
+    // q and the slots the RoPE + append kernel writes are read only after it
+    // has finished (a no-op unless launched as its programmatic dependent)
+    grid_dependency_wait();
     const int pre = min(S, ntiles);
     for (int k = 0; k < pre; ++k) issue(k);
     int issued = pre;
@@ -686,20 +689,20 @@ cudaError_t attn_tokens_prepare(int head_dim, bool fp8, int num_sms, int max_bat
 }
 
 cudaError_t launch_decode_attn_tokens(const AttnParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
-                                      int head_dim, bool fp8, const AttnLaunch& L, cudaStream_t stream)
+                                      int head_dim, bool fp8, const AttnLaunch& L, cudaStream_t stream, bool pdl)
 {
     const dim3 grid(L.ctas), block(kAttnWarps * 32);
     AttnParams q = p;
     q.stages = L.stages;
     q.tail_chunks = 0;
+    cudaError_t e;
     if (head_dim == 128) {
-        if (fp8) decode_attn_tokens_kernel<128, true, kAttnWarps><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
-        else decode_attn_tokens_kernel<128, false, kAttnWarps><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
+        if (fp8) e = launch_attn_kernel(decode_attn_tokens_kernel<128, true, kAttnWarps>, grid, block, L.smem_bytes, stream, pdl, tmk, tmv, q);
+        else e = launch_attn_kernel(decode_attn_tokens_kernel<128, false, kAttnWarps>, grid, block, L.smem_bytes, stream, pdl, tmk, tmv, q);
     } else {
-        if (fp8) decode_attn_tokens_kernel<64, true, kAttnWarps><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
-        else decode_attn_tokens_kernel<64, false, kAttnWarps><<<grid, block, L.smem_bytes, stream>>>(tmk, tmv, q);
+        if (fp8) e = launch_attn_kernel(decode_attn_tokens_kernel<64, true, kAttnWarps>, grid, block, L.smem_bytes, stream, pdl, tmk, tmv, q);
+        else e = launch_attn_kernel(decode_attn_tokens_kernel<64, false, kAttnWarps>, grid, block, L.smem_bytes, stream, pdl, tmk, tmv, q);
     }
-    const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     return launch_combine(q, head_dim, L.ctas * kAttnWarps, L.ctas, stream);
 }

@@ -274,14 +274,17 @@ pkv_status pkv_rope_append(pkv_ctx* ctx, void* q, const void* k_new, const void*
     return pkv::launch_rope_append(p, stream) == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
-pkv_status pkv_decode_attn(pkv_ctx* ctx, const void* q, const void* k_pool, const void* v_pool,
-                           const float* k_scale, const float* v_scale, const int32_t* block_tables,
-                           int bt_stride, const int32_t* seq_lens, int batch, void* out,
-                           cudaStream_t stream)
+}  // extern "C"
+
+namespace {
+
+// pkv_decode_attn after its checks; pdl: as a programmatic dependent of the
+// RoPE + append kernel just launched on the stream (pkv_decode_step only).
+pkv_status decode_attn_launch(pkv_ctx* ctx, const void* q, const void* k_pool, const void* v_pool,
+                              const float* k_scale, const float* v_scale, const int32_t* block_tables,
+                              int bt_stride, const int32_t* seq_lens, int batch, void* out,
+                              cudaStream_t stream, bool pdl)
 {
-    pkv_status st = check_call(ctx, batch, bt_stride, k_pool, v_pool, k_scale, v_scale, block_tables, seq_lens);
-    if (st != PKV_OK || batch == 0) return st;
-    if (!q || !out || !aligned16(q) || !aligned16(out)) return PKV_ERR_INVALID_ARG;
 
     if (ctx->tm_k_ptr != k_pool) {
         if (!encode_pool(ctx, k_pool, &ctx->tmk)) return PKV_ERR_CUDA;
@@ -317,8 +320,24 @@ pkv_status pkv_decode_attn(pkv_ctx* ctx, const void* q, const void* k_pool, cons
     p.tail_chunks = ctx->tail_chunks;
     p.q_len = 1;
     const cudaError_t e = pkv::launch_decode_attn(p, ctx->tmk, ctx->tmv, ctx->cfg.head_dim,
-                                                  ctx->cfg.kv_dtype == PKV_KV_FP8_E4M3, ctx->attn, stream);
+                                                  ctx->cfg.kv_dtype == PKV_KV_FP8_E4M3, ctx->attn, stream, pdl);
     return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+pkv_status pkv_decode_attn(pkv_ctx* ctx, const void* q, const void* k_pool, const void* v_pool,
+                           const float* k_scale, const float* v_scale, const int32_t* block_tables,
+                           int bt_stride, const int32_t* seq_lens, int batch, void* out,
+                           cudaStream_t stream)
+{
+    pkv_status st = check_call(ctx, batch, bt_stride, k_pool, v_pool, k_scale, v_scale, block_tables, seq_lens);
+    if (st != PKV_OK || batch == 0) return st;
+    if (!q || !out || !aligned16(q) || !aligned16(out)) return PKV_ERR_INVALID_ARG;
+    return decode_attn_launch(ctx, q, k_pool, v_pool, k_scale, v_scale, block_tables, bt_stride, seq_lens, batch,
+                              out, stream, false);
 }
 
 pkv_status pkv_rope_append_tokens(pkv_ctx* ctx, void* q, const void* k_new, const void* v_new, void* k_pool,
@@ -366,7 +385,7 @@ namespace {
 pkv_status attn_tokens_launch(pkv_ctx* ctx, const void* q, const void* k_pool, const void* v_pool,
                               const float* k_scale, const float* v_scale, const int32_t* block_tables,
                               int bt_stride, const int32_t* seq_lens, int batch, int q_len, const int4* vmap,
-                              const int* vcount, void* out, cudaStream_t stream)
+                              const int* vcount, void* out, cudaStream_t stream, bool pdl = false)
 {
     const bool fp8 = ctx->cfg.kv_dtype == PKV_KV_FP8_E4M3;
     const CUtensorMap* mk = &ctx->tmk;
@@ -420,7 +439,8 @@ pkv_status attn_tokens_launch(pkv_ctx* ctx, const void* q, const void* k_pool, c
     p.q_len = q_len;
     p.vmap = vmap;
     p.vcount = vcount;
-    const cudaError_t e = pkv::launch_decode_attn_tokens(p, *mk, *mv, ctx->cfg.head_dim, fp8, ctx->attn_tok, stream);
+    const cudaError_t e = pkv::launch_decode_attn_tokens(p, *mk, *mv, ctx->cfg.head_dim, fp8, ctx->attn_tok, stream,
+                                                         pdl);
     return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
@@ -440,6 +460,29 @@ pkv_status pkv_decode_attn_tokens(pkv_ctx* ctx, const void* q, const void* k_poo
     if (!q || !out || !aligned16(q) || !aligned16(out)) return PKV_ERR_INVALID_ARG;
     return attn_tokens_launch(ctx, q, k_pool, v_pool, k_scale, v_scale, block_tables, bt_stride, seq_lens, batch,
                               q_len, nullptr, nullptr, out, stream);
+}
+
+pkv_status pkv_decode_step(pkv_ctx* ctx, void* q, const void* k_new, const void* v_new, void* k_pool,
+                           void* v_pool, const float* k_scale, const float* v_scale, const int32_t* block_tables,
+                           int bt_stride, const int32_t* seq_lens, int batch, int q_len, void* out,
+                           cudaStream_t stream)
+{
+    pkv_status st = check_call(ctx, batch, bt_stride, k_pool, v_pool, k_scale, v_scale, block_tables, seq_lens);
+    if (st != PKV_OK || batch == 0) return st;
+    if (q_len < 1 || (long long)batch * q_len > (1LL << 31) - 1) return PKV_ERR_INVALID_ARG;
+    if (q_len > 1 && (long long)ctx->G * q_len > pkv::kMaxTokenRows) return PKV_ERR_UNSUPPORTED;
+    if (!q || !k_new || !v_new || !out || !aligned16(q) || !aligned16(k_new) || !aligned16(v_new) ||
+        !aligned16(out))
+        return PKV_ERR_INVALID_ARG;
+    st = pkv_rope_append_tokens(ctx, q, k_new, v_new, k_pool, v_pool, k_scale, v_scale, block_tables, bt_stride,
+                                seq_lens, batch, q_len, stream);
+    if (st != PKV_OK) return st;
+    // the attention starts its prologue while the RoPE + append kernel runs
+    if (q_len == 1)
+        return decode_attn_launch(ctx, q, k_pool, v_pool, k_scale, v_scale, block_tables, bt_stride, seq_lens,
+                                  batch, out, stream, true);
+    return attn_tokens_launch(ctx, q, k_pool, v_pool, k_scale, v_scale, block_tables, bt_stride, seq_lens, batch,
+                              q_len, nullptr, nullptr, out, stream, true);
 }
 
 pkv_status pkv_rope_append_varlen(pkv_ctx* ctx, void* q, const void* k_new, const void* v_new, void* k_pool,

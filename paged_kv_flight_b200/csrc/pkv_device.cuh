@@ -81,6 +81,23 @@ __device__ __forceinline__ void fence_proxy_async_smem()
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// ---- programmatic dependent launch ---------------------------------------------
+
+// Lets the grid launched after this one on the stream as a programmatic
+// dependent start once every CTA of this grid has executed this (or exited).
+__device__ __forceinline__ void grid_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Waits until the grid this one depends on programmatically has completed and
+// its memory operations are visible; returns at once in a grid launched
+// without that dependency.
+__device__ __forceinline__ void grid_dependency_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ---- TMA --------------------------------------------------------------------
 
 // 2-D tiled bulk tensor load global -> shared, completion counted in bytes on

@@ -114,8 +114,13 @@ struct AttnLaunch {
     int tile;             // tokens per tile (attn_tile)
 };
 cudaError_t attn_prepare(int head_dim, bool fp8, int page_size, int num_sms, int max_batch, AttnLaunch* out);
+// pdl: launch the attention as a programmatic dependent of the kernel before
+// it on the stream (only where that kernel is this library's RoPE + append,
+// which triggers its dependents at once and writes nothing the attention's
+// prologue reads).
 cudaError_t launch_decode_attn(const AttnParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
-                               int head_dim, bool fp8, const AttnLaunch& L, cudaStream_t stream);
+                               int head_dim, bool fp8, const AttnLaunch& L, cudaStream_t stream,
+                               bool pdl = false);
 
 // Attention of several new tokens per request (decode_attn_tokens.cu, bf16
 // or E4M3 pools with 16-token tiles, G x q_len <= 16): shape of its launch
@@ -127,7 +132,8 @@ cudaError_t attn_tokens_prepare(int head_dim, bool fp8, int num_sms, int max_bat
 cudaError_t launch_varlen_plan(const int32_t* cu_q, const int32_t* seq_lens, int batch, int block, int vmax,
                                int4* vmap, int* vcount, int* err, cudaStream_t stream);
 cudaError_t launch_decode_attn_tokens(const AttnParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
-                                      int head_dim, bool fp8, const AttnLaunch& L, cudaStream_t stream);
+                                      int head_dim, bool fp8, const AttnLaunch& L, cudaStream_t stream,
+                                      bool pdl = false);
 
 // QKV projection of the new tokens on tcgen05, fused with RoPE and the append
 // (qkv_rope_append.cu).

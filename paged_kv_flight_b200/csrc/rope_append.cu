@@ -55,6 +55,10 @@ __global__ void __launch_bounds__(kRopeThreads) rope_append_kernel(const RopePar
     constexpr int PIECES = HALF / 8;  // 8 pairs per work item
     __shared__ double s_cos[HALF], s_sin[HALF];
 
+    // a decode attention launched as this grid's programmatic dependent may
+    // start its prologue now; it reads q and the pools only once this grid
+    // has finished
+    dev::grid_launch_dependents();
     const int bt = blockIdx.x;               // (request, new token) row of q, k_new, v_new
     int b, t;
     if (p.cu_q) {

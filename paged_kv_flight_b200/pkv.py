@@ -49,7 +49,7 @@ EXPORTS = ("pkv_create", "pkv_rope_append", "pkv_decode_attn", "pkv_destroy", "p
            "pkv_pages_release", "pkv_pages_block_table", "pkv_pages_seq_lens", "pkv_pages_active",
            "pkv_pages_refcount", "pkv_pages_free_count", "pkv_pages_take_changes", "pkv_qkv_rope_append",
            "pkv_qkv_pack_weight", "pkv_set_qkv_split", "pkv_qkv_launch_shape",
-           "pkv_table_sync", "pkv_rope_append_varlen", "pkv_decode_attn_varlen")
+           "pkv_table_sync", "pkv_rope_append_varlen", "pkv_decode_attn_varlen", "pkv_decode_step")
 
 
 class pkv_config(C.Structure):
@@ -115,6 +115,8 @@ lib.pkv_workspace_bytes.restype = C.c_size_t
 lib.pkv_decode_attn_noalloc.argtypes = [C.POINTER(pkv_config), _V, _V, _V, _V, _V, _V, C.c_int, _V, C.c_int,
                                         _V, _V]
 lib.pkv_decode_attn_noalloc.restype = C.c_int
+lib.pkv_decode_step.argtypes = [_V, _V, _V, _V, _V, _V, _V, _V, _V, C.c_int, _V, C.c_int, C.c_int, _V, _V]
+lib.pkv_decode_step.restype = C.c_int
 
 
 class PkvError(RuntimeError):
@@ -314,6 +316,24 @@ def pkv_decode_attn_tokens(ctx, q, k_pool, v_pool, k_scale, v_scale, block_table
                                     _ptr(seq_lens, _I32, "seq_lens"), int(batch), int(q_len),
                                     _ptr(out, _ACT, "out"), _stream(stream))
     return _done(st, "pkv_decode_attn_tokens", check)
+
+
+def pkv_decode_step(ctx, q, k_new, v_new, k_pool, v_pool, k_scale, v_scale, block_tables, seq_lens, out,
+                    batch: int | None = None, q_len: int = 1, bt_stride: int | None = None, stream=None,
+                    check: bool = True) -> int:
+    """The whole step in one call: pkv_rope_append(_tokens) then
+    pkv_decode_attn(_tokens), the attention overlapping the RoPE kernel's end.
+    q / out [batch, (q_len,) Hq, d], k_new / v_new [batch, (q_len,) Hkv, d]."""
+    if batch is None:
+        batch = int(seq_lens.shape[0])
+    if bt_stride is None:
+        bt_stride = int(block_tables.shape[1])
+    st = lib.pkv_decode_step(ctx, _ptr(q, _ACT, "q"), _ptr(k_new, _ACT, "k_new"), _ptr(v_new, _ACT, "v_new"),
+                             *_kv(k_pool, v_pool, k_scale, v_scale),
+                             _ptr(block_tables, _I32, "block_tables"), int(bt_stride),
+                             _ptr(seq_lens, _I32, "seq_lens"), int(batch), int(q_len), _ptr(out, _ACT, "out"),
+                             _stream(stream))
+    return _done(st, "pkv_decode_step", check)
 
 
 class Pages:

@@ -38,11 +38,17 @@ def make_ctx(pkv, w: Workload, max_batch=None, max_blocks=None):
     return pkv.pkv_create(cfg)
 
 
-def gpu_step(pkv, ctx, dv: dict, out=None, check=True):
+def gpu_step(pkv, ctx, dv: dict, out=None, check=True, fused=False):
+    """The step through the C ABI: pkv_rope_append then pkv_decode_attn, or
+    with fused=True the one call pkv_decode_step."""
     B = dv["seq_lens"].shape[0]
     Hq, d = dv["q"].shape[1], dv["q"].shape[2]
     if out is None:
         out = torch.empty(B, Hq, d, dtype=torch.bfloat16, device=dv["q"].device)
+    if fused:
+        pkv.pkv_decode_step(ctx, dv["q"], dv["k_new"], dv["v_new"], dv["k_pool"], dv["v_pool"], dv["k_scale"],
+                            dv["v_scale"], dv["block_tables"], dv["seq_lens"], out, check=check)
+        return out
     pkv.pkv_rope_append(ctx, dv["q"], dv["k_new"], dv["v_new"], dv["k_pool"], dv["v_pool"],
                         dv["k_scale"], dv["v_scale"], dv["block_tables"], dv["seq_lens"], check=check)
     pkv.pkv_decode_attn(ctx, dv["q"], dv["k_pool"], dv["v_pool"], dv["k_scale"], dv["v_scale"],

@@ -112,6 +112,38 @@ def test_full_size_whole_batch_matches_oracle(pkv, name):
     assert mx <= t["max"] and mean <= t["mean"], (mx, mean)
 
 
+@pytest.mark.parametrize("case", SMALL + [("llama8b",), ("hetero70b",), ("fp8",), ("longctx",)],
+                         ids=lambda c: c[0])
+def test_decode_step_equals_the_two_calls(pkv, case):
+    """pkv_decode_step runs the same kernels as pkv_rope_append followed by
+    pkv_decode_attn, the attention launched as a programmatic dependent of
+    the append: q, both pools and the output must be bit-identical to the two
+    calls' on the same inputs, small cases and full-size workloads alike."""
+    w = workloads.make(case[0], device="cuda") if len(case) == 1 else _small(case)
+    results = []
+    for fused in (False, True):
+        dv = _gpu.to_device(w)
+        ctx = _gpu.make_ctx(pkv, w)
+        try:
+            out = _gpu.gpu_step(pkv, ctx, dv, fused=fused)
+            assert pkv.pkv_check_device_error(ctx)[0] == pkv.PKV_OK
+        finally:
+            pkv.pkv_destroy(ctx)
+        results.append((out, dv))
+        del dv
+    (o0, d0), (o1, d1) = results
+    assert torch.equal(o0.view(torch.int16), o1.view(torch.int16))
+    for k in ("q", "k_pool", "v_pool"):
+        a, b = d0[k], d1[k]
+        if a.dtype == torch.bfloat16:
+            a, b = a.view(torch.int16), b.view(torch.int16)        # NaN sentinels: compare bits
+        assert torch.equal(a, b), k
+    if len(case) > 1:
+        _, ref, _ = oracle_step(w)
+        mx, mean, finite = _gpu.errors(o1, ref)
+        assert finite and mx <= _gpu.tol(w)["max"] and mean <= _gpu.tol(w)["mean"], (mx, mean)
+
+
 @pytest.mark.parametrize("case_name", ["g4_d128_p32_bf16", "g4_d128_p32_fp8", "llama8b"])
 def test_split_count_invariance(pkv, case_name):
     if case_name == "llama8b":

@@ -148,6 +148,33 @@ def test_full_size_spec4_whole_batch_matches_oracle(pkv):
     assert finite and mx <= _gpu.TOL_BF16["max"] and mean <= _gpu.TOL_BF16["mean"], (mx, mean)
 
 
+@pytest.mark.parametrize("case", [CASES[0], CASES[1], ("spec4",)], ids=lambda c: c[0])
+def test_decode_step_with_several_tokens_equals_the_two_calls(pkv, case):
+    """pkv_decode_step with q_len > 1 against pkv_rope_append_tokens followed
+    by pkv_decode_attn_tokens on the same inputs: bit-identical q, pools and
+    output (the same kernels; the attention is a programmatic dependent of
+    the append in the one call)."""
+    w = workloads.make("spec4", device="cuda") if len(case) == 1 else _build(case)
+    results = []
+    for fused in (False, True):
+        dv = _gpu.to_device(w)
+        ctx = _gpu.make_ctx(pkv, w)
+        try:
+            if fused:
+                q, kn, vn = (_q3(dv[k], w).contiguous() for k in ("q", "k_new", "v_new"))
+                out = torch.empty(w.batch, w.q_len, w.Hq, w.d, dtype=torch.bfloat16, device="cuda")
+                pkv.pkv_decode_step(ctx, q, kn, vn, dv["k_pool"], dv["v_pool"], None, None, dv["block_tables"],
+                                    dv["seq_lens"], out, q_len=w.q_len)
+            else:
+                q, out = _gpu_tokens(pkv, ctx, w, dv)
+            assert pkv.pkv_check_device_error(ctx)[0] == pkv.PKV_OK
+        finally:
+            pkv.pkv_destroy(ctx)
+        results.append((q, out, dv["k_pool"], dv["v_pool"]))
+    for a, b in zip(*results):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
 def test_tokens_host_side_rejections(pkv):
     w = _build(CASES[0])                     # G = 4
     dv = _gpu.to_device(w)
