@@ -342,7 +342,8 @@ def workload_config(w, name, world) -> dict:
             "new_tokens_per_request": w.q_len,
             "metric_bytes_per_step": workload_bytes(w),
             "full_step_bytes": full_step_bytes(w.seq_lens, w.Hq, w.Hkv, w.d, w.P, w.kv_fp8, w.q_len),
-            "l2": L2_NOTE, "replicas": world}
+            "l2": L2_NOTE, "replicas": world,
+            **({"requests_kept": w.batch} if w.extra.get("requests") else {})}
 
 
 # ---------------------------------------------------------------- GPU leg
@@ -364,7 +365,7 @@ def run_ours(args, name, rank, world, local_rank, cpu_budget=None):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    w = workloads.make(name, device=dev, offset=rank)
+    w = workloads.make(name, device=dev, offset=rank, requests=args.requests)
     dv = _device_inputs(w, dev)
     B = w.batch
     cfg = pkv.make_config(w.Hq, w.Hkv, w.d, w.P, "fp8" if w.kv_fp8 else "bf16", w.rope_base, B,
@@ -968,6 +969,8 @@ def main(argv=None):
     ap.add_argument("--tail-chunks", type=int, default=None,
                     help="cap on dynamic tail chunks per warp range (library default if omitted; 0: static split)")
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--requests", type=int, default=None,
+                    help="keep only the first N requests of the workload (a smaller case for profiler captures)")
     ap.add_argument("--ref-budget", type=int, default=1_200_000,
                     help="attended token-heads per reference step")
     args = ap.parse_args(argv)

@@ -228,13 +228,21 @@ def build(name: str, Hq: int, Hkv: int, d: int, P: int, kv_fp8: bool, rope_base:
                     q_len=q_len)
 
 
-def make(name: str, device="cpu", offset: int = 0) -> Workload:
-    """One of the five named workloads; ``offset`` draws an independent replica."""
+def make(name: str, device="cpu", offset: int = 0, requests: Optional[int] = None) -> Workload:
+    """One of the five named workloads; ``offset`` draws an independent replica.
+    ``requests`` keeps only the first that many requests of the batch (same
+    shapes and lengths, a pool sized for them): a smaller case of the same
+    workload, for profiler captures."""
     s = _SHAPES[name]
     seed = config_seed(name, offset)
     lengths = draw_lengths(name, np.random.default_rng(seed))
-    return build(name, s["Hq"], s["Hkv"], s["d"], s["P"], s["kv_fp8"], s["base"], lengths,
-                 seed, device=device, num_pages=64 if name == "tiny" else None, q_len=s.get("q_len", 1))
+    if requests is not None:
+        lengths = lengths[:max(1, int(requests))]
+    w = build(name, s["Hq"], s["Hkv"], s["d"], s["P"], s["kv_fp8"], s["base"], lengths,
+              seed, device=device, num_pages=64 if name == "tiny" else None, q_len=s.get("q_len", 1))
+    if requests is not None:
+        w.extra["requests"] = w.batch
+    return w
 
 
 def make_mixed(device="cpu", offset: int = 0, chunk: int = 64, prefills: int = 8):
