@@ -300,6 +300,11 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
     float o[NTD][2];
     uint32_t qa[KSTEPS][2], qn[KSTEPS][2];
     float m_run = -INFINITY, l_run = 0.f;
+    // E4M3: o holds the pair's P V sum over the V codes in units of the V
+    // scale vs_cur (the true sum is o x vs_cur); a tile of another scale
+    // rescales o by vs_cur / vs together with the softmax rescale, so the
+    // P V mma accumulates into o directly
+    float vs_cur = 1.f;
     int n_cur = 0, n_next = 0;
     bool dead = false;
     int k_dead = 0;
@@ -358,6 +363,7 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
             for (int nt = 0; nt < NTD; ++nt) o[nt][0] = o[nt][1] = 0.f;
             m_run = -INFINITY;
             l_run = 0.f;
+            vs_cur = 1.f;
             unit_first = false;
         }
         if (pair_end && k + 1 < issued) {
@@ -468,11 +474,16 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
             }
             l_run = l_run * alpha + psum;
             m_run = m_new;
-            if (__any_sync(kFull, alpha != 1.f)) {
+            float rescale = alpha;
+            if constexpr (FP8) {
+                rescale = alpha * (vs_cur / si.vs);
+                vs_cur = si.vs;
+            }
+            if (__any_sync(kFull, rescale != 1.f)) {
 #pragma unroll
                 for (int nt = 0; nt < NTD; ++nt) {
-                    o[nt][0] *= alpha;
-                    o[nt][1] *= alpha;
+                    o[nt][0] *= rescale;
+                    o[nt][1] *= rescale;
                 }
             }
 
@@ -491,7 +502,6 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
                 // d, and the mma n-index j of n-tile nt stands for d = DV*j + nt.
                 constexpr int DV = D / 8;
                 constexpr int WORDS = DV / 4;
-                const float vs = si.vs;
                 // one 16-token half at a time (not unrolled: the second half's
                 // loads are not hoisted over the first's mma, which keeps the
                 // 32-token tile within the register file)
@@ -527,16 +537,10 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
                         const uint32_t x1 = __byte_perm(wa[kw], wb[kw], 0x7362);
                         const uint32_t y0 = __byte_perm(wc[kw], wd[kw], 0x5140);
                         const uint32_t y1 = __byte_perm(wc[kw], wd[kw], 0x7362);
-                        float t[4][2] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
-                        mma_f16_r8(t[0][0], t[0][1], pl, ph, cvt_lo(x0), cvt_lo(y0));
-                        mma_f16_r8(t[1][0], t[1][1], pl, ph, cvt_hi(x0), cvt_hi(y0));
-                        mma_f16_r8(t[2][0], t[2][1], pl, ph, cvt_lo(x1), cvt_lo(y1));
-                        mma_f16_r8(t[3][0], t[3][1], pl, ph, cvt_hi(x1), cvt_hi(y1));
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            o[4 * kw + e][0] = fmaf(t[e][0], vs, o[4 * kw + e][0]);
-                            o[4 * kw + e][1] = fmaf(t[e][1], vs, o[4 * kw + e][1]);
-                        }
+                        mma_f16_r8(o[4 * kw][0], o[4 * kw][1], pl, ph, cvt_lo(x0), cvt_lo(y0));
+                        mma_f16_r8(o[4 * kw + 1][0], o[4 * kw + 1][1], pl, ph, cvt_hi(x0), cvt_hi(y0));
+                        mma_f16_r8(o[4 * kw + 2][0], o[4 * kw + 2][1], pl, ph, cvt_lo(x1), cvt_lo(y1));
+                        mma_f16_r8(o[4 * kw + 3][0], o[4 * kw + 3][1], pl, ph, cvt_hi(x1), cvt_hi(y1));
                     }
                 }
             }
@@ -557,7 +561,7 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
             const size_t orow = ((size_t)cb * p.Hq + (size_t)ckvh * G + g) * D;
             if (cu0 <= ts && te <= cu1) {
                 if (g < G) {
-                    const float inv = 1.f / lsum;
+                    const float inv = (FP8 ? vs_cur : 1.f) / lsum;
                     uint32_t* dst = reinterpret_cast<uint32_t*>(p.out + orow);
                     if constexpr (!FP8) {
 #pragma unroll
@@ -584,13 +588,14 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
                         for (int nt = 0; nt < NTD; ++nt)
                             *reinterpret_cast<float2*>(dst + 8 * nt + 2 * c4) = make_float2(o[nt][0], o[nt][1]);
                     } else {
+                        // the partial is the true sum: o in units of vs_cur
                         constexpr int DV = D / 8;
 #pragma unroll
                         for (int e = 0; e < 2; ++e)
 #pragma unroll
                             for (int u = 0; u < DV / 2; ++u)
                                 *reinterpret_cast<float2*>(dst + DV * (2 * c4 + e) + 2 * u) =
-                                    make_float2(o[2 * u][e], o[2 * u + 1][e]);
+                                    make_float2(o[2 * u][e] * vs_cur, o[2 * u + 1][e] * vs_cur);
                     }
                     if (c4 == 0)
                         *reinterpret_cast<float2*>(p.part_ml + ((size_t)slot * G + g) * 2) =
