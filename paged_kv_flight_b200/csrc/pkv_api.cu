@@ -545,7 +545,11 @@ pkv_status pkv_decode_attn_varlen(pkv_ctx* ctx, const void* q, const void* k_poo
     // go to the prefill kernel, in blocks of pblock tokens (at most
     // ceil(q / pblock) <= 3 q / pblock blocks for a request of q >= pblock / 2)
     const bool fp8 = ctx->cfg.kv_dtype == PKV_KV_FP8_E4M3;
-    const int pblock = fp8 ? 0 : pkv::prefill_block_tokens(ctx->G), pmin = std::max(1, pblock / 2);
+#ifndef PKV_PREFILL_ROUTE
+#define PKV_PREFILL_ROUTE 1
+#endif
+    const int pblock = (fp8 || !PKV_PREFILL_ROUTE) ? 0 : pkv::prefill_block_tokens(ctx->G),
+              pmin = std::max(1, pblock / 2);
     if (pkv::launch_varlen_plan(cu_q, seq_lens, batch, block, ctx->vmax, ctx->d_vmap, ctx->d_vcount, pblock, pmin,
                                 ctx->vmax, ctx->d_pmap, ctx->d_pcount, ctx->d_err, stream) != cudaSuccess)
         return PKV_ERR_CUDA;

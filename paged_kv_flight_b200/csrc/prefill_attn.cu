@@ -38,7 +38,12 @@ using namespace attn;
 
 constexpr int kTeamWarps = 8;                           // consumer warps of a block
 constexpr int kTeamThreads = (kTeamWarps + 1) * 32;     // and one producer warp
-constexpr int kTeamStages = 6;
+// The eight warps consume a tile in a fraction of the TMA latency, so the
+// ring holds many tiles (the CTA is alone on its SM: registers bound it).
+#ifndef PKV_TEAM_STAGES
+#define PKV_TEAM_STAGES 16
+#endif
+constexpr int kTeamStages = PKV_TEAM_STAGES;
 
 // m16n8k16, bf16 A and B, all 16 rows, fp32 accumulation in place.
 __device__ __forceinline__ void mma16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
