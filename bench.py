@@ -50,7 +50,6 @@ DEFAULT_CONFIG = "suite"
 # attention kernels for the attention workloads, the fused projection for qkv8b
 KERNEL_SOURCES = {
     "attn": ("paged_kv_flight_b200/csrc/decode_attn.cu", "paged_kv_flight_b200/csrc/decode_attn_tokens.cu",
-             "paged_kv_flight_b200/csrc/prefill_attn.cu",
              "paged_kv_flight_b200/csrc/attn_common.cuh", "paged_kv_flight_b200/csrc/combine.cu",
              "paged_kv_flight_b200/csrc/pkv_device.cuh", "paged_kv_flight_b200/csrc/pkv_internal.h"),
     "qkv": ("paged_kv_flight_b200/csrc/qkv_rope_append.cu", "paged_kv_flight_b200/csrc/pkv_device.cuh",
@@ -894,17 +893,10 @@ def run_mixed(args, rank, world, local_rank):
     row = 2 * w.Hkv * w.d * 2                      # K + V bytes of one token
     # metric bytes: each request's cache (its new tokens included) once, q and out of every new token
     by = int((row * (L + q_lens)).sum()) + 2 * n_tok * w.Hq * w.d * 2
-    # streamed: every block of new tokens reads its own prefix; a request of
-    # at least half a prefill block (8 x 16 / G tokens) goes to the prefill
-    # kernel in blocks of that length, any other in blocks of 16 / G
-    G = w.Hq // w.Hkv
-    blk, pblk = 16 // G, 8 * (16 // G)
-
-    def blocks(qb):
-        return pblk if qb >= pblk // 2 else blk
-    streamed = sum(row * (int(Lb) + min(j + blocks(int(qb)), int(qb)))
-                   for Lb, qb in zip(L, q_lens) for j in range(0, int(qb), blocks(int(qb)))) \
-        + 2 * n_tok * w.Hq * w.d * 2
+    # streamed: every block of 16 / G new tokens reads its own prefix
+    blk = 16 // (w.Hq // w.Hkv)
+    streamed = sum(row * (int(Lb) + min(j + blk, int(qb)))
+                   for Lb, qb in zip(L, q_lens) for j in range(0, int(qb), blk)) + 2 * n_tok * w.Hq * w.d * 2
     peak, peak_src = measured_peak()
     gbs = by / (attn_ms * 1e-3) / 1e9
     return {"metric": METRIC, "value": sum_over_ranks(float(by)) / (step_ms * 1e-3) / 1e9, "unit": "GB/s",
@@ -919,11 +911,11 @@ def run_mixed(args, rank, world, local_rank):
             "new_tokens_per_s": sum_over_ranks(float(n_tok)) / (step_ms * 1e-3),
             "streamed_bytes_per_launch": streamed,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
-                         "traffic": recorded_traffic("mixed"), "kernel": "decode_attn_tokens_kernel<128> + prefill_attn_kernel<128> (varlen)",
+                         "traffic": recorded_traffic("mixed"), "kernel": "decode_attn_tokens_kernel<128> (varlen)",
                          "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)", "bytes_per_launch": by,
                          "note": "bytes = each request's cache once (the metric); a prefill chunk's blocks "
                                  "re-read their prefix, see streamed_bytes_per_launch"},
-            "gpu_launches": 9 * K, "clocks": clock_info}   # step: rope, plan, attention, combine, prefill; alone: 4
+            "gpu_launches": 7 * K, "clocks": clock_info}   # step: rope, plan, attention, combine; alone: 3
 
 
 def run_loop(args, rank, world, local_rank):

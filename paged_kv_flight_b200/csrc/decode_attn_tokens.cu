@@ -616,49 +616,35 @@ cudaError_t prepare_tokens_t(int num_sms, int max_batch, AttnLaunch* out)
 
 namespace {
 
-// One CTA: request b's new tokens (q = cu_q[b + 1] - cu_q[b] of them) cut
-// into blocks.  A request with q >= pmin (pblock > 0) is cut into blocks of
-// pblock tokens for the prefill kernel (pmap), any other into blocks of
-// `block` tokens for the several-new-tokens kernel (vmap); entry = {b, first
-// q row, tokens, L_b + offset of the block}, counted in request order (an
-// exclusive scan of the blocks per request and list).  More than vmax (pmax)
-// blocks, or a negative token count, set kErrLength (the surplus is dropped).
+// One CTA: request b's new tokens (cu_q[b + 1] - cu_q[b] of them) cut into
+// blocks of `block`; vmap[v] = {b, first q row, tokens, L_b + offset of the
+// block}, v counted in request order (an exclusive scan of the blocks per
+// request).  More than vmax blocks, or a negative token count, set kErrLength
+// (the surplus is dropped).
 __global__ void __launch_bounds__(1024) varlen_plan_kernel(const int32_t* __restrict__ cu_q,
                                                            const int32_t* __restrict__ seq_lens, int batch,
                                                            int block, int vmax, int4* __restrict__ vmap,
-                                                           int* __restrict__ vcount, int pblock, int pmin, int pmax,
-                                                           int4* __restrict__ pmap, int* __restrict__ pcount,
-                                                           int* __restrict__ err)
+                                                           int* __restrict__ vcount, int* __restrict__ err)
 {
-    __shared__ int s_warp[2][32];
+    __shared__ int s_warp[32];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
     const int per = (batch + (int)blockDim.x - 1) / (int)blockDim.x;
     const int lo = min(batch, tid * per), hi = min(batch, lo + per);
-    auto prefill = [&](int q) { return pblock > 0 && q >= pmin; };
-    int local[2] = {0, 0};
+    int local = 0;
     for (int b = lo; b < hi; ++b) {
         const int q = cu_q[b + 1] - cu_q[b];
-        if (q <= 0) continue;
-        if (prefill(q)) local[1] += (q + pblock - 1) / pblock;
-        else local[0] += (q + block - 1) / block;
+        local += q > 0 ? (q + block - 1) / block : 0;
     }
-    int run[2];
+    int incl = local;
 #pragma unroll
-    for (int l = 0; l < 2; ++l) {
-        int incl = local[l];
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(kFull, incl, o);
-            if (lane >= o) incl += v;
-        }
-        if (lane == 31) s_warp[l][warp] = incl;
-        run[l] = incl - local[l];
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += v;
     }
+    if (lane == 31) s_warp[warp] = incl;
     __syncthreads();
-    for (int w2 = 0; w2 < warp; ++w2) {
-        run[0] += s_warp[0][w2];
-        run[1] += s_warp[1][w2];
-    }
+    int run = incl - local;
+    for (int w2 = 0; w2 < warp; ++w2) run += s_warp[w2];
     for (int b = lo; b < hi; ++b) {
         const int a = cu_q[b], q = cu_q[b + 1] - a;
         if (q < 0) {
@@ -666,37 +652,31 @@ __global__ void __launch_bounds__(1024) varlen_plan_kernel(const int32_t* __rest
             continue;
         }
         const long long L = seq_lens[b];
-        const bool pf = prefill(q);
-        const int bl = pf ? pblock : block, cap = pf ? pmax : vmax;
-        int4* const map = pf ? pmap : vmap;
-        int& r = run[pf ? 1 : 0];
-        for (int j = 0; (long long)j * bl < q; ++j) {
-            const long long pos = L + (long long)j * bl;
-            if (r < cap)
-                map[r] = make_int4(b, a + j * bl, min(bl, q - j * bl), (L < 0 || pos > 0x7fffffffll) ? -1 : (int)pos);
-            ++r;
+        for (int j = 0; (long long)j * block < q; ++j) {
+            const long long pos = L + (long long)j * block;
+            if (run < vmax)
+                vmap[run] = make_int4(b, a + j * block, min(block, q - j * block),
+                                      (L < 0 || pos > 0x7fffffffll) ? -1 : (int)pos);
+            ++run;
         }
     }
     if (tid == 0) {
-        int total[2] = {0, 0};
-        for (int w2 = 0; w2 < nwarps; ++w2) {
-            total[0] += s_warp[0][w2];
-            total[1] += s_warp[1][w2];
+        int total = 0;
+        for (int w2 = 0; w2 < nwarps; ++w2) total += s_warp[w2];
+        if (total > vmax) {
+            atomicOr(err, kErrLength);
+            total = vmax;
         }
-        if (total[0] > vmax || total[1] > pmax) atomicOr(err, kErrLength);
-        *vcount = min(total[0], vmax);
-        if (pcount) *pcount = min(total[1], pmax);
+        *vcount = total;
     }
 }
 
 }  // namespace
 
 cudaError_t launch_varlen_plan(const int32_t* cu_q, const int32_t* seq_lens, int batch, int block, int vmax,
-                               int4* vmap, int* vcount, int pblock, int pmin, int pmax, int4* pmap, int* pcount,
-                               int* err, cudaStream_t stream)
+                               int4* vmap, int* vcount, int* err, cudaStream_t stream)
 {
-    varlen_plan_kernel<<<1, 1024, 0, stream>>>(cu_q, seq_lens, batch, block, vmax, vmap, vcount, pblock, pmin, pmax,
-                                               pmap, pcount, err);
+    varlen_plan_kernel<<<1, 1024, 0, stream>>>(cu_q, seq_lens, batch, block, vmax, vmap, vcount, err);
     return cudaGetLastError();
 }
 

@@ -32,8 +32,6 @@ struct pkv_ctx {
     int vmax;             // virtual requests a varlen attention call may have (bf16 pools)
     int4* d_vmap;         // [vmax] the varlen plan
     int* d_vcount;
-    int4* d_pmap;         // [vmax] the varlen plan's prefill blocks (bf16 pools)
-    int* d_pcount;
     float* d_part_o;
     float* d_part_ml;
     const void* tm_k_ptr;
@@ -202,7 +200,7 @@ pkv_status pkv_create(const pkv_config* cfg, pkv_ctx** out)
         free(ctx);
         return PKV_ERR_CUDA;
     }
-    if (pkv::qkv_prepare() != cudaSuccess || pkv::prefill_prepare(cfg->head_dim) != cudaSuccess) {
+    if (pkv::qkv_prepare() != cudaSuccess) {
         free(ctx);
         return PKV_ERR_CUDA;
     }
@@ -218,7 +216,7 @@ pkv_status pkv_create(const pkv_config* cfg, pkv_ctx** out)
     const size_t b_po = 2 * rows_units * cfg->head_dim * sizeof(float);
     const size_t b_pml = 2 * rows_units * 2 * sizeof(float);
     const size_t b_vm = (size_t)ctx->vmax * sizeof(int4) + 256;   // varlen plan + its count
-    ctx->ws_bytes = b_err + b_cnt + b_po + b_pml + 2 * b_vm;         // two lists: decode blocks, prefill blocks
+    ctx->ws_bytes = b_err + b_cnt + b_po + b_pml + b_vm;
     if (cudaMalloc(&ctx->ws, ctx->ws_bytes) != cudaSuccess) {
         cudaGetLastError();
         free(ctx);
@@ -233,8 +231,6 @@ pkv_status pkv_create(const pkv_config* cfg, pkv_ctx** out)
     ctx->d_part_ml = reinterpret_cast<float*>(base + b_err + b_cnt + b_po);
     ctx->d_vcount = reinterpret_cast<int*>(base + b_err + b_cnt + b_po + b_pml);
     ctx->d_vmap = reinterpret_cast<int4*>(base + b_err + b_cnt + b_po + b_pml + 256);
-    ctx->d_pcount = reinterpret_cast<int*>(base + b_err + b_cnt + b_po + b_pml + b_vm);
-    ctx->d_pmap = reinterpret_cast<int4*>(base + b_err + b_cnt + b_po + b_pml + b_vm + 256);
     if (cudaMemset(ctx->ws, 0, b_err + b_cnt) != cudaSuccess) {
         cudaFree(ctx->ws);
         free(ctx);
@@ -541,50 +537,11 @@ pkv_status pkv_decode_attn_varlen(pkv_ctx* ctx, const void* q, const void* k_poo
     // blocks of `block` new tokens: G x block <= 16 query rows per (block, kv head)
     const int block = pkv::kMaxTokenRows / ctx->G;
     if ((long long)batch + (n_tokens + block - 1) / block > ctx->vmax) return PKV_ERR_UNSUPPORTED;
-    // bf16 pools: requests with at least half a prefill block of new tokens
-    // go to the prefill kernel, in blocks of pblock tokens (at most
-    // ceil(q / pblock) <= 3 q / pblock blocks for a request of q >= pblock / 2)
-    const bool fp8 = ctx->cfg.kv_dtype == PKV_KV_FP8_E4M3;
-#ifndef PKV_PREFILL_ROUTE
-#define PKV_PREFILL_ROUTE 1
-#endif
-    const int pblock = (fp8 || !PKV_PREFILL_ROUTE) ? 0 : pkv::prefill_block_tokens(ctx->G),
-              pmin = std::max(1, pblock / 2);
-    if (pkv::launch_varlen_plan(cu_q, seq_lens, batch, block, ctx->vmax, ctx->d_vmap, ctx->d_vcount, pblock, pmin,
-                                ctx->vmax, ctx->d_pmap, ctx->d_pcount, ctx->d_err, stream) != cudaSuccess)
+    if (pkv::launch_varlen_plan(cu_q, seq_lens, batch, block, ctx->vmax, ctx->d_vmap, ctx->d_vcount, ctx->d_err,
+                                stream) != cudaSuccess)
         return PKV_ERR_CUDA;
-    pkv_status st2 = attn_tokens_launch(ctx, q, k_pool, v_pool, k_scale, v_scale, block_tables, bt_stride, seq_lens,
-                                        ctx->vmax, block, ctx->d_vmap, ctx->d_vcount, out, stream);
-    if (st2 != PKV_OK || pblock == 0) return st2;
-    // the prefill blocks (the tensor maps were set up by the launch above)
-    pkv::AttnParams p;
-    p.q = static_cast<const __nv_bfloat16*>(q);
-    p.out = static_cast<__nv_bfloat16*>(out);
-    p.k_scale = p.v_scale = nullptr;
-    p.block_tables = block_tables;
-    p.seq_lens = seq_lens;
-    p.part_o = p.part_ml = nullptr;
-    p.meta = nullptr;
-    p.err = ctx->d_err;
-    p.claim = nullptr;
-    p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)ctx->cfg.head_dim));
-    p.batch = ctx->vmax;
-    p.bt_stride = bt_stride;
-    p.Hq = ctx->cfg.num_q_heads;
-    p.Hkv = ctx->cfg.num_kv_heads;
-    p.G = ctx->G;
-    p.P = ctx->cfg.page_size;
-    p.num_pages = ctx->cfg.num_pages;
-    p.stages = 0;
-    p.workers = 0;
-    p.tail_chunks = 0;
-    p.q_len = pblock;
-    p.vmap = ctx->d_pmap;
-    p.vcount = ctx->d_pcount;
-    const int grid_blocks = (int)std::min<long long>(ctx->vmax, 3LL * n_tokens / pblock + 1);
-    return pkv::launch_prefill_attn(p, ctx->tmk, ctx->tmv, ctx->cfg.head_dim, grid_blocks, stream) == cudaSuccess
-               ? PKV_OK
-               : PKV_ERR_CUDA;
+    return attn_tokens_launch(ctx, q, k_pool, v_pool, k_scale, v_scale, block_tables, bt_stride, seq_lens,
+                              ctx->vmax, block, ctx->d_vmap, ctx->d_vcount, out, stream);
 }
 
 pkv_status pkv_qkv_pack_weight(pkv_ctx* ctx, const void* w_qkv, int hidden, void* w_tiled, cudaStream_t stream)

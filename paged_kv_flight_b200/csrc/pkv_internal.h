@@ -128,21 +128,9 @@ cudaError_t launch_decode_attn(const AttnParams& p, const CUtensorMap& tmk, cons
 cudaError_t attn_tokens_prepare(int head_dim, bool fp8, int num_sms, int max_batch, AttnLaunch* out);
 // The virtual requests of a varlen call: blocks of `block` new tokens (the
 // last of a request may be shorter) of requests with cu_q[b + 1] > cu_q[b];
-// writes vmap and the count (capped at vmax; more sets kErrLength).  With
-// pblock > 0, requests of at least pmin new tokens are cut into blocks of
-// pblock tokens for the prefill kernel instead (pmap, pcount, capped at pmax).
+// writes vmap and the count (capped at vmax; more sets kErrLength).
 cudaError_t launch_varlen_plan(const int32_t* cu_q, const int32_t* seq_lens, int batch, int block, int vmax,
-                               int4* vmap, int* vcount, int pblock, int pmin, int pmax, int4* pmap, int* pcount,
-                               int* err, cudaStream_t stream);
-
-// The prefill kernel (prefill_attn.cu, bf16 pools): tokens per block for a
-// group size G, its kernel attribute, and its launch over the plan's blocks
-// (p.vmap / p.vcount = the prefill list, p.batch = its capacity; grid_blocks
-// CTAs per kv head, those past the count exit at once).
-int prefill_block_tokens(int G);
-cudaError_t prefill_prepare(int head_dim);
-cudaError_t launch_prefill_attn(const AttnParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv, int head_dim,
-                                int grid_blocks, cudaStream_t stream);
+                               int4* vmap, int* vcount, int* err, cudaStream_t stream);
 cudaError_t launch_decode_attn_tokens(const AttnParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
                                       int head_dim, bool fp8, const AttnLaunch& L, cudaStream_t stream,
                                       bool pdl = false);

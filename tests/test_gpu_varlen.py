@@ -23,8 +23,8 @@ CASES = [
     ("g8_d128_p16", 64, 8, 128, 16, [5, 300, 1000], [7, 1, 33]),
     ("g2_d64_p64", 8, 4, 64, 64, [0, 63, 64, 200], [16, 1, 9, 65]),
     ("g1_d64_p16", 4, 4, 64, 16, [10, 40, 0], [50, 1, 1]),
-    # chunks long enough for the prefill kernel (blocks of 8 x 16 / G tokens
-    # shared by a team of warps), long prefixes (many ring wraps), ragged ends
+    # longer chunks (up to 130 new tokens), prefixes of up to 3000 tokens,
+    # ragged last blocks
     ("g1_d64_p16_prefill", 4, 4, 64, 16, [10, 700, 0], [100, 1, 130]),
     ("g8_d128_p16_prefill", 64, 8, 128, 16, [3000, 20, 511], [48, 1, 9]),
     ("g4_d128_p64_prefill", 32, 8, 128, 64, [2049, 0, 77, 1000], [64, 16, 1, 15]),
