@@ -373,11 +373,6 @@ def run_ours(args, name, rank, world, local_rank, cpu_budget=None):
     ctx = pkv.pkv_create(cfg)
     if args.tail_chunks is not None:
         pkv.pkv_set_tail_chunks(ctx, args.tail_chunks)
-    # per-SM weights of the attention split, measured once for this context
-    # (a setup call, outside every timed region)
-    if not args.no_calibrate:
-        pkv.pkv_calibrate(ctx, dv["k_pool"], dv["v_pool"], dv["k_scale"], dv["v_scale"], rounds=5)
-    sm_weights = pkv.pkv_get_sm_weights(ctx)
     tok = w.q_len > 1          # several new tokens per request: the *_tokens entry points
     out = torch.empty(B, *((w.q_len,) if tok else ()), w.Hq, w.d, dtype=torch.bfloat16, device=dev)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
@@ -623,9 +618,6 @@ def run_ours(args, name, rank, world, local_rank, cpu_budget=None):
                      else "fallback 6650 GB/s",
                      "bytes_per_launch": by},
         "e2e": e2e,
-        "sm_weights": {"calibrated": not args.no_calibrate, "min": min(sm_weights), "max": max(sm_weights),
-                       "note": "per-SM weights of the attention split (1024 = 1.0), measured by pkv_calibrate "
-                               "before timing"},
         "gpu_launches": 3 * K,
         "clocks": clock_info,
         "when": datetime.datetime.utcnow().isoformat() + "Z",
@@ -972,8 +964,6 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay timing")
-    ap.add_argument("--no-calibrate", action="store_true",
-                    help="equal split ranges (skip pkv_calibrate's per-SM weights)")
     ap.add_argument("--two-calls", action="store_true",
                     help="time the step as pkv_rope_append + pkv_decode_attn instead of pkv_decode_step")
     ap.add_argument("--tail-chunks", type=int, default=None,

@@ -63,11 +63,8 @@
  *       host page allocator of pkv_pages.h;
  *   pkv_decode_attn_noalloc                          the attention without a
  *       context (no allocation);
- *   pkv_calibrate, pkv_set_sm_weights                per-SM weights of the
- *       attention split, measured once per context;
  *   pkv_set_workers, pkv_set_tail_chunks, pkv_set_qkv_split,
- *   pkv_qkv_launch_shape, pkv_workspace_bytes,
- *   pkv_get_sm_weights                               tuning and inspection.
+ *   pkv_qkv_launch_shape, pkv_workspace_bytes        tuning and inspection.
  *
  * Errors: host-side checks return PKV_ERR_INVALID_ARG / PKV_ERR_UNSUPPORTED
  * and launch nothing.  A failed launch returns PKV_ERR_CUDA.  Range errors
@@ -339,35 +336,6 @@ pkv_status pkv_qkv_launch_shape(pkv_ctx* ctx, int batch, int hidden, int* shape)
 
 /* Bytes of device workspace the context holds. */
 size_t pkv_workspace_bytes(const pkv_ctx* ctx);
-
-/* Per-SM weights of the attention split.  The attention cuts the flattened
- * (request, kv head, tile) sequence into one contiguous range per warp
- * worker; by default the ranges are equal.  Some SMs stream measurably slower
- * than others, and the same ones on every launch, so equal ranges end on the
- * slowest SM.  With weights, worker v (on CTA v % ctas, one CTA per SM) gets
- * a range proportional to its CTA's weight (fixed point, 1024 = 1.0, each in
- * [512, 2048]; applied when the batch has at least 8 tiles per worker, and
- * then without a dynamic tail).  Results do not depend on the weights beyond
- * rounding; a context's calls are deterministic while its weights stay put.
- *
- * pkv_calibrate measures them: it runs the attention `rounds` times (>= 2; the
- * first warms up) on a synthetic batch whose pages are drawn at random from
- * the given pools (read only; the pools' contents do not matter) and after
- * each launch moves every CTA's weight by the ratio of the mean CTA time to
- * its own.  It allocates and frees a small scratch, synchronises `stream`,
- * and keeps the weights in the context.  Make the call before any stream
- * capture and not while another call of this context runs.  On an error the
- * weights return to equal.  k_scale / v_scale as for pkv_decode_attn.
- *
- * pkv_set_sm_weights sets them (host array of *count entries as
- * pkv_get_sm_weights reports; NULL: equal ranges again), synchronously;
- * PKV_ERR_INVALID_ARG for a weight outside [512, 2048].  pkv_get_sm_weights
- * writes the count of CTAs to *count and, if weights is not NULL, the
- * current weights (1024 each when none are set). */
-pkv_status pkv_calibrate(pkv_ctx* ctx, const void* k_pool, const void* v_pool, const float* k_scale,
-                         const float* v_scale, int rounds, cudaStream_t stream);
-pkv_status pkv_set_sm_weights(pkv_ctx* ctx, const int* weights);
-pkv_status pkv_get_sm_weights(const pkv_ctx* ctx, int* weights, int* count);
 
 /* pkv_decode_attn for callers that cannot allocate device memory.  The pages
  * describe no such entry point; it exists for callers such as a serving

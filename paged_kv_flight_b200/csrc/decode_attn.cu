@@ -107,7 +107,6 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
         s_bad = 0;
         prefetch_tensormap(&tmk);
         prefetch_tensormap(&tmv);
-        if (p.ctimes) p.ctimes[(size_t)blockIdx.x * (1 + WARPS)] = global_timer_ns();
     }
     __syncthreads();
 
@@ -160,7 +159,7 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
     else Wl = min(Wl, (T + kMinTilesPerWorker - 1) / kMinTilesPerWorker);
     Wl = max(1LL, min(Wl, max(T, 1LL)));
     const int W = (int)Wl;
-    const Split sp = make_split(max(T, 1LL), W, p.tail_chunks, p.wpre, p.ctas);
+    const Split sp = make_split(max(T, 1LL), W, p.tail_chunks);
     if (blockIdx.x == 0) {
         // the combine kernel that follows needs the same split geometry
         if (tid == 0) {
@@ -632,8 +631,6 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
         }
     }
 
-    if (p.ctimes && lane == 0) p.ctimes[(size_t)blockIdx.x * (1 + WARPS) + 1 + warp] = global_timer_ns();
-
     // a worker that timed out still owns the loads it issued for tiles
     // k_dead .. issued-1 (one per stage): wait for them, bounded
     if (dead && lane == 0) {
@@ -702,7 +699,6 @@ cudaError_t launch_decode_attn(const AttnParams& p, const CUtensorMap& tmk, cons
     const dim3 grid(L.ctas), block(kAttnWarps * 32);
     AttnParams q = p;
     q.stages = L.stages;
-    q.ctas = L.ctas;           // the weighted split maps worker v to CTA v % ctas
     const bool wide = L.tile == kTileWide;
     cudaError_t e;
     if (head_dim == 128) {

@@ -28,9 +28,6 @@ struct pkv_ctx {
     size_t ws_bytes;
     int* d_err;
     int* d_claim;         // chunk counter of the attention's dynamic tail
-    int* d_wpre;          // [attn.ctas + 1] prefix of the per-CTA split weights
-    int weighted;         // 1: the attention splits by d_wpre (pkv_set_sm_weights / pkv_calibrate)
-    int* h_weights;       // [attn.ctas] the weights on the host
     int* d_meta;
     int vmax;             // virtual requests a varlen attention call may have (bf16 pools)
     int4* d_vmap;         // [vmax] the varlen plan
@@ -219,8 +216,7 @@ pkv_status pkv_create(const pkv_config* cfg, pkv_ctx** out)
     const size_t b_po = 2 * rows_units * cfg->head_dim * sizeof(float);
     const size_t b_pml = 2 * rows_units * 2 * sizeof(float);
     const size_t b_vm = (size_t)ctx->vmax * sizeof(int4) + 256;   // varlen plan + its count
-    const size_t b_w = ((size_t)(ctx->attn.ctas + 1) * sizeof(int) + 255) & ~(size_t)255;   // split weights
-    ctx->ws_bytes = b_err + b_cnt + b_po + b_pml + b_vm + b_w;
+    ctx->ws_bytes = b_err + b_cnt + b_po + b_pml + b_vm;
     if (cudaMalloc(&ctx->ws, ctx->ws_bytes) != cudaSuccess) {
         cudaGetLastError();
         free(ctx);
@@ -229,14 +225,6 @@ pkv_status pkv_create(const pkv_config* cfg, pkv_ctx** out)
     uint8_t* base = static_cast<uint8_t*>(ctx->ws);
     ctx->d_err = reinterpret_cast<int*>(base);
     ctx->d_claim = reinterpret_cast<int*>(base + 128);
-    ctx->d_wpre = reinterpret_cast<int*>(base + b_err + b_cnt + b_po + b_pml + b_vm);
-    ctx->h_weights = static_cast<int*>(malloc(sizeof(int) * (size_t)ctx->attn.ctas));
-    if (!ctx->h_weights) {
-        cudaFree(ctx->ws);
-        free(ctx);
-        return PKV_ERR_OOM;
-    }
-    for (int c = 0; c < ctx->attn.ctas; ++c) ctx->h_weights[c] = pkv::kWeightOne;
     ctx->tail_chunks = pkv::kDefaultTailChunks;
     ctx->d_meta = reinterpret_cast<int*>(base + b_err);
     ctx->d_part_o = reinterpret_cast<float*>(base + b_err + b_cnt);
@@ -330,7 +318,6 @@ pkv_status decode_attn_launch(pkv_ctx* ctx, const void* q, const void* k_pool, c
     p.stages = ctx->attn.stages;
     p.workers = ctx->workers;
     p.tail_chunks = ctx->tail_chunks;
-    p.wpre = ctx->weighted ? ctx->d_wpre : nullptr;
     p.q_len = 1;
     const cudaError_t e = pkv::launch_decode_attn(p, ctx->tmk, ctx->tmv, ctx->cfg.head_dim,
                                                   ctx->cfg.kv_dtype == PKV_KV_FP8_E4M3, ctx->attn, stream, pdl);
@@ -452,7 +439,6 @@ pkv_status attn_tokens_launch(pkv_ctx* ctx, const void* q, const void* k_pool, c
     p.q_len = q_len;
     p.vmap = vmap;
     p.vcount = vcount;
-    p.wpre = ctx->weighted ? ctx->d_wpre : nullptr;
     const cudaError_t e = pkv::launch_decode_attn_tokens(p, *mk, *mv, ctx->cfg.head_dim, fp8, ctx->attn_tok, stream,
                                                          pdl);
     return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
@@ -634,7 +620,6 @@ pkv_status pkv_destroy(pkv_ctx* ctx)
     pkv_status st = PKV_OK;
     if (cudaDeviceSynchronize() != cudaSuccess) st = PKV_ERR_CUDA;
     if (ctx->ws && cudaFree(ctx->ws) != cudaSuccess) st = PKV_ERR_CUDA;
-    free(ctx->h_weights);
     free(ctx);
     return st;
 }
@@ -700,193 +685,5 @@ pkv_status pkv_set_tail_chunks(pkv_ctx* ctx, int max_chunks)
 }
 
 size_t pkv_workspace_bytes(const pkv_ctx* ctx) { return ctx ? ctx->ws_bytes : 0; }
-
-}  // extern "C"
-
-namespace {
-
-// Uploads the prefix of the context's host weights; synchronous.
-pkv_status upload_weights(pkv_ctx* ctx, bool weighted)
-{
-    const int n = ctx->attn.ctas;
-    int* pre = static_cast<int*>(malloc(sizeof(int) * (size_t)(n + 1)));
-    if (!pre) return PKV_ERR_OOM;
-    pre[0] = 0;
-    for (int c = 0; c < n; ++c) pre[c + 1] = pre[c] + ctx->h_weights[c];
-    const cudaError_t e = cudaMemcpy(ctx->d_wpre, pre, sizeof(int) * (size_t)(n + 1), cudaMemcpyHostToDevice);
-    free(pre);
-    if (e != cudaSuccess) return PKV_ERR_CUDA;
-    ctx->weighted = weighted ? 1 : 0;
-    return PKV_OK;
-}
-
-// Scales w so that its mean is kWeightOne, within [kWeightMin, kWeightMax].
-void normalise_weights(double* w, int n, int* out)
-{
-    for (int pass = 0; pass < 3; ++pass) {
-        double mean = 0.0;
-        for (int c = 0; c < n; ++c) mean += w[c];
-        mean /= n;
-        for (int c = 0; c < n; ++c) {
-            w[c] *= pkv::kWeightOne / mean;
-            w[c] = std::min<double>(pkv::kWeightMax, std::max<double>(pkv::kWeightMin, w[c]));
-        }
-    }
-    for (int c = 0; c < n; ++c) out[c] = (int)lrint(w[c]);
-}
-
-}  // namespace
-
-extern "C" {
-
-pkv_status pkv_set_sm_weights(pkv_ctx* ctx, const int* weights)
-{
-    if (!ctx) return PKV_ERR_INVALID_ARG;
-    const int n = ctx->attn.ctas;
-    if (!weights) {
-        for (int c = 0; c < n; ++c) ctx->h_weights[c] = pkv::kWeightOne;
-        return upload_weights(ctx, false);
-    }
-    for (int c = 0; c < n; ++c)
-        if (weights[c] < pkv::kWeightMin || weights[c] > pkv::kWeightMax) return PKV_ERR_INVALID_ARG;
-    for (int c = 0; c < n; ++c) ctx->h_weights[c] = weights[c];
-    return upload_weights(ctx, true);
-}
-
-pkv_status pkv_get_sm_weights(const pkv_ctx* ctx, int* weights, int* count)
-{
-    if (!ctx || !count) return PKV_ERR_INVALID_ARG;
-    *count = ctx->attn.ctas;
-    if (weights)
-        for (int c = 0; c < ctx->attn.ctas; ++c) weights[c] = ctx->h_weights[c];
-    return PKV_OK;
-}
-
-pkv_status pkv_calibrate(pkv_ctx* ctx, const void* k_pool, const void* v_pool, const float* k_scale,
-                         const float* v_scale, int rounds, cudaStream_t stream)
-{
-    if (!ctx || !k_pool || !v_pool || !aligned16(k_pool) || !aligned16(v_pool) || rounds < 2 || rounds > 64)
-        return PKV_ERR_INVALID_ARG;
-    const bool fp8 = ctx->cfg.kv_dtype == PKV_KV_FP8_E4M3;
-    if (fp8 && (!k_scale || !v_scale || !aligned16(k_scale) || !aligned16(v_scale))) return PKV_ERR_INVALID_ARG;
-    const int ctas = ctx->attn.ctas, W = ctas * pkv::kAttnWarps, Hkv = ctx->cfg.num_kv_heads;
-    const int Hq = ctx->cfg.num_q_heads, d = ctx->cfg.head_dim, P = ctx->cfg.page_size;
-    // a synthetic batch over the whole pool: nb requests of equal length,
-    // pages drawn at random, about 96 tiles per warp; q is zero
-    const int nb = 16;
-    const long long tiles = 96LL * W;
-    const int n_tok = (int)std::max<long long>(P, tiles / ((long long)Hkv * nb) * ctx->attn.tile);
-    const int bt_stride = (n_tok + P - 1) / P;
-    const size_t q_bytes = (size_t)nb * Hq * d * 2, bt_bytes = (size_t)nb * bt_stride * 4;
-    const size_t t_bytes = (size_t)ctas * (1 + pkv::kAttnWarps) * sizeof(unsigned long long);
-    const size_t off_out = (q_bytes + 255) & ~(size_t)255, off_bt = off_out + ((q_bytes + 255) & ~(size_t)255);
-    const size_t off_len = off_bt + ((bt_bytes + 255) & ~(size_t)255), off_t = off_len + 256;
-    void* scratch = nullptr;
-    if (cudaMalloc(&scratch, off_t + t_bytes) != cudaSuccess) {
-        cudaGetLastError();
-        return PKV_ERR_OOM;
-    }
-    uint8_t* base = static_cast<uint8_t*>(scratch);
-    int32_t* h_bt = static_cast<int32_t*>(malloc(bt_bytes));
-    unsigned long long* h_t = static_cast<unsigned long long*>(malloc(t_bytes));
-    double* w = static_cast<double*>(malloc(sizeof(double) * (size_t)ctas));
-    pkv_status st = (h_bt && h_t && w) ? PKV_OK : PKV_ERR_OOM;
-    if (st == PKV_OK) {
-        uint64_t x = 0x9E3779B97F4A7C15ull;   // a fixed sequence: the same batch every time
-        for (size_t i = 0; i < (size_t)nb * bt_stride; ++i) {
-            x = x * 6364136223846793005ull + 1442695040888963407ull;
-            h_bt[i] = (int32_t)((x >> 33) % (uint64_t)ctx->cfg.num_pages);
-        }
-        int32_t h_len[nb];
-        for (int b = 0; b < nb; ++b) h_len[b] = n_tok - 1;
-        if (cudaMemsetAsync(base, 0, q_bytes, stream) != cudaSuccess ||
-            cudaMemcpyAsync(base + off_bt, h_bt, bt_bytes, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
-            cudaMemcpyAsync(base + off_len, h_len, sizeof(h_len), cudaMemcpyHostToDevice, stream) != cudaSuccess)
-            st = PKV_ERR_CUDA;
-        for (int c = 0; c < ctas; ++c) w[c] = ctx->h_weights[c];
-    }
-    if (st == PKV_OK && ctx->tm_k_ptr != k_pool) {
-        if (!encode_pool(ctx, k_pool, &ctx->tmk)) st = PKV_ERR_CUDA;
-        else ctx->tm_k_ptr = k_pool;
-    }
-    if (st == PKV_OK && ctx->tm_v_ptr != v_pool) {
-        if (!encode_pool(ctx, v_pool, &ctx->tmv)) st = PKV_ERR_CUDA;
-        else ctx->tm_v_ptr = v_pool;
-    }
-    for (int it = 0; it < rounds && st == PKV_OK; ++it) {
-        // the first launch only warms up; each later one moves every CTA's
-        // weight by the ratio of the mean CTA time to its own
-        if ((st = upload_weights(ctx, true)) != PKV_OK) break;
-        pkv::AttnParams p;
-        p.q = reinterpret_cast<const __nv_bfloat16*>(base);
-        p.out = reinterpret_cast<__nv_bfloat16*>(base + off_out);
-        p.k_scale = fp8 ? k_scale : nullptr;
-        p.v_scale = fp8 ? v_scale : nullptr;
-        p.block_tables = reinterpret_cast<const int32_t*>(base + off_bt);
-        p.seq_lens = reinterpret_cast<const int32_t*>(base + off_len);
-        p.part_o = ctx->d_part_o;
-        p.part_ml = ctx->d_part_ml;
-        p.meta = ctx->d_meta;
-        p.err = ctx->d_err;
-        p.claim = ctx->d_claim;
-        p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)d));
-        p.batch = nb;
-        p.bt_stride = bt_stride;
-        p.Hq = Hq;
-        p.Hkv = Hkv;
-        p.G = ctx->G;
-        p.P = P;
-        p.num_pages = ctx->cfg.num_pages;
-        p.stages = ctx->attn.stages;
-        p.workers = W;
-        p.tail_chunks = 0;
-        p.q_len = 1;
-        p.wpre = ctx->d_wpre;
-        p.ctimes = reinterpret_cast<unsigned long long*>(base + off_t);
-        if (cudaMemsetAsync(p.ctimes, 0, t_bytes, stream) != cudaSuccess ||
-            pkv::launch_decode_attn(p, ctx->tmk, ctx->tmv, d, fp8, ctx->attn, stream) != cudaSuccess ||
-            cudaMemcpyAsync(h_t, p.ctimes, t_bytes, cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
-            cudaStreamSynchronize(stream) != cudaSuccess) {
-            st = PKV_ERR_CUDA;
-            break;
-        }
-        if (it == 0) continue;
-        double mean = 0.0;
-        int counted = 0;
-        double* el = static_cast<double*>(malloc(sizeof(double) * (size_t)ctas));
-        if (!el) {
-            st = PKV_ERR_OOM;
-            break;
-        }
-        for (int c = 0; c < ctas; ++c) {
-            const unsigned long long* t = h_t + (size_t)c * (1 + pkv::kAttnWarps);
-            unsigned long long end = 0;
-            for (int j = 1; j <= pkv::kAttnWarps; ++j) end = std::max(end, t[j]);
-            el[c] = (end > t[0] && t[0] != 0) ? (double)(end - t[0]) : 0.0;
-            if (el[c] > 0.0) {
-                mean += el[c];
-                ++counted;
-            }
-        }
-        if (counted == ctas) {
-            mean /= counted;
-            for (int c = 0; c < ctas; ++c) w[c] *= mean / el[c];
-            normalise_weights(w, ctas, ctx->h_weights);
-        }
-        free(el);
-    }
-    // the synthetic batch may have read NaN sentinels: nothing it produced is kept
-    int word = 0;
-    if (st == PKV_OK && cudaMemcpy(&word, ctx->d_err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
-        st = PKV_ERR_CUDA;
-    if (st == PKV_OK && (word & pkv::kErrTimeout)) st = PKV_ERR_DEVICE_TIMEOUT;
-    if (st == PKV_OK) st = upload_weights(ctx, true);
-    else (void)pkv_set_sm_weights(ctx, nullptr);
-    cudaFree(scratch);
-    free(h_bt);
-    free(h_t);
-    free(w);
-    return st;
-}
 
 }  // extern "C"

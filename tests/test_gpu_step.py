@@ -210,85 +210,6 @@ def test_a_later_context_with_a_smaller_batch_leaves_an_earlier_one_usable(pkv):
         assert finite and mx <= _gpu.TOL_BF16["max"] and mean <= _gpu.TOL_BF16["mean"], (mx, mean)
 
 
-@pytest.mark.parametrize("case_name", ["g4_d128_p32_bf16", "g8_d128_p16_bf16", "g4_d64_p32_fp8", "llama8b",
-                                       "hetero70b"])
-def test_weighted_split_matches_oracle(pkv, case_name):
-    """Per-SM weights of the split (seeded, spread over the whole allowed
-    range [512, 2048]) move every range boundary; the output must still match
-    the oracle, also with forced worker counts, and two calls must agree bit
-    for bit."""
-    if case_name in ("llama8b", "hetero70b"):
-        w = workloads.make(case_name, device="cuda")
-    else:
-        w = _small(next(c for c in SMALL if c[0] == case_name))
-    _, ref, _ = oracle_step(w)
-    dv = _gpu.to_device(w)
-    ctx = _gpu.make_ctx(pkv, w)
-    outs = []
-    try:
-        n = len(pkv.pkv_get_sm_weights(ctx))
-        weights = np.random.default_rng(7).integers(512, 2048, size=n, endpoint=True)
-        pkv.pkv_set_sm_weights(ctx, weights)
-        assert pkv.pkv_get_sm_weights(ctx) == [int(x) for x in weights]
-        pkv.pkv_rope_append(ctx, dv["q"], dv["k_new"], dv["v_new"], dv["k_pool"], dv["v_pool"], dv["k_scale"],
-                            dv["v_scale"], dv["block_tables"], dv["seq_lens"])
-        for workers in (0, 0, 7, 100):
-            pkv.pkv_set_workers(ctx, workers)
-            out = torch.empty(w.batch, w.Hq, w.d, dtype=torch.bfloat16, device="cuda")
-            pkv.pkv_decode_attn(ctx, dv["q"], dv["k_pool"], dv["v_pool"], dv["k_scale"], dv["v_scale"],
-                                dv["block_tables"], dv["seq_lens"], out)
-            outs.append(out)
-        assert pkv.pkv_check_device_error(ctx)[0] == pkv.PKV_OK
-    finally:
-        pkv.pkv_destroy(ctx)
-    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))   # deterministic
-    for o in outs:
-        mx, mean, finite = _gpu.errors(o, ref)
-        assert finite and mx <= _gpu.tol(w)["max"] and mean <= _gpu.tol(w)["mean"], (mx, mean)
-
-
-@pytest.mark.parametrize("fp8", [False, True])
-def test_calibrated_weights_are_bounded_and_keep_parity(pkv, fp8):
-    name = "fp8" if fp8 else "llama8b"
-    w = workloads.make(name, device="cuda")
-    _, ref, _ = oracle_step(w)
-    dv = _gpu.to_device(w)
-    ctx = _gpu.make_ctx(pkv, w)
-    try:
-        pkv.pkv_calibrate(ctx, dv["k_pool"], dv["v_pool"], dv["k_scale"], dv["v_scale"], rounds=4)
-        weights = pkv.pkv_get_sm_weights(ctx)
-        assert all(512 <= x <= 2048 for x in weights)
-        assert abs(np.mean(weights) - 1024) <= 16
-        out = _gpu.gpu_step(pkv, ctx, dv)
-        out2 = torch.empty_like(out)
-        pkv.pkv_decode_attn(ctx, dv["q"], dv["k_pool"], dv["v_pool"], dv["k_scale"], dv["v_scale"],
-                            dv["block_tables"], dv["seq_lens"], out2)
-        assert pkv.pkv_check_device_error(ctx)[0] == pkv.PKV_OK
-    finally:
-        pkv.pkv_destroy(ctx)
-    assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
-    mx, mean, finite = _gpu.errors(out, ref)
-    assert finite and mx <= _gpu.tol(w)["max"] and mean <= _gpu.tol(w)["mean"], (mx, mean)
-
-
-def test_sm_weight_rejections(pkv):
-    w = _small(SMALL[0])
-    dv = _gpu.to_device(w)
-    ctx = _gpu.make_ctx(pkv, w)
-    try:
-        n = len(pkv.pkv_get_sm_weights(ctx))
-        assert pkv.pkv_get_sm_weights(ctx) == [1024] * n
-        assert pkv.pkv_set_sm_weights(ctx, [1024] * (n - 1) + [511], check=False) == pkv.PKV_ERR_INVALID_ARG
-        assert pkv.pkv_set_sm_weights(ctx, [2049] + [1024] * (n - 1), check=False) == pkv.PKV_ERR_INVALID_ARG
-        with pytest.raises(ValueError):
-            pkv.pkv_set_sm_weights(ctx, [1024] * (n + 1))
-        assert pkv.pkv_calibrate(ctx, dv["k_pool"], dv["v_pool"], rounds=1, check=False) == pkv.PKV_ERR_INVALID_ARG
-        assert pkv.pkv_set_sm_weights(ctx, None) == pkv.PKV_OK
-        assert pkv.pkv_get_sm_weights(ctx) == [1024] * n
-    finally:
-        pkv.pkv_destroy(ctx)
-
-
 def test_combine_merges_more_contributors_than_one_staging_block(pkv):
     # one (request, kv head) pair of 270,001 tokens over 128 warps: 16,876
     # tiles, 131 per warp range, a tail of 8 chunks per range -> 1,152 units
