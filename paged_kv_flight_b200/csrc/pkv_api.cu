@@ -28,6 +28,7 @@ struct pkv_ctx {
     size_t ws_bytes;
     int* d_err;
     int* d_claim;         // chunk counter of the attention's dynamic tail
+    double* d_theta;      // [head_dim / 2] rope_base^(-2i/d), fp64
     int* d_meta;
     int vmax;             // virtual requests a varlen attention call may have (bf16 pools)
     int4* d_vmap;         // [vmax] the varlen plan
@@ -216,7 +217,8 @@ pkv_status pkv_create(const pkv_config* cfg, pkv_ctx** out)
     const size_t b_po = 2 * rows_units * cfg->head_dim * sizeof(float);
     const size_t b_pml = 2 * rows_units * 2 * sizeof(float);
     const size_t b_vm = (size_t)ctx->vmax * sizeof(int4) + 256;   // varlen plan + its count
-    ctx->ws_bytes = b_err + b_cnt + b_po + b_pml + b_vm;
+    const size_t b_th = ((size_t)cfg->head_dim / 2 * sizeof(double) + 255) & ~(size_t)255;   // RoPE frequencies
+    ctx->ws_bytes = b_err + b_cnt + b_po + b_pml + b_vm + b_th;
     if (cudaMalloc(&ctx->ws, ctx->ws_bytes) != cudaSuccess) {
         cudaGetLastError();
         free(ctx);
@@ -231,7 +233,13 @@ pkv_status pkv_create(const pkv_config* cfg, pkv_ctx** out)
     ctx->d_part_ml = reinterpret_cast<float*>(base + b_err + b_cnt + b_po);
     ctx->d_vcount = reinterpret_cast<int*>(base + b_err + b_cnt + b_po + b_pml);
     ctx->d_vmap = reinterpret_cast<int4*>(base + b_err + b_cnt + b_po + b_pml + 256);
-    if (cudaMemset(ctx->ws, 0, b_err + b_cnt) != cudaSuccess) {
+    ctx->d_theta = reinterpret_cast<double*>(base + b_err + b_cnt + b_po + b_pml + b_vm);
+    // theta_i = rope_base^(-2i/d) once, in fp64 on the host
+    double theta[64];
+    for (int i = 0; i < cfg->head_dim / 2; ++i) theta[i] = pow(cfg->rope_base, (-2.0 * i) / cfg->head_dim);
+    if (cudaMemset(ctx->ws, 0, b_err + b_cnt) != cudaSuccess ||
+        cudaMemcpy(ctx->d_theta, theta, sizeof(double) * (size_t)(cfg->head_dim / 2), cudaMemcpyHostToDevice) !=
+            cudaSuccess) {
         cudaFree(ctx->ws);
         free(ctx);
         return PKV_ERR_CUDA;
@@ -262,6 +270,8 @@ pkv_status pkv_rope_append(pkv_ctx* ctx, void* q, const void* k_new, const void*
     p.seq_lens = seq_lens;
     p.err = ctx->d_err;
     p.rope_base = ctx->cfg.rope_base;
+    p.theta = ctx->d_theta;
+    p.prefetch_tables = 1;
     p.batch = batch;
     p.bt_stride = bt_stride;
     p.Hq = ctx->cfg.num_q_heads;
@@ -363,6 +373,8 @@ pkv_status pkv_rope_append_tokens(pkv_ctx* ctx, void* q, const void* k_new, cons
     p.seq_lens = seq_lens;
     p.err = ctx->d_err;
     p.rope_base = ctx->cfg.rope_base;
+    p.theta = ctx->d_theta;
+    p.prefetch_tables = 1;
     p.batch = batch;
     p.bt_stride = bt_stride;
     p.Hq = ctx->cfg.num_q_heads;
@@ -510,6 +522,8 @@ pkv_status pkv_rope_append_varlen(pkv_ctx* ctx, void* q, const void* k_new, cons
     p.seq_lens = seq_lens;
     p.err = ctx->d_err;
     p.rope_base = ctx->cfg.rope_base;
+    p.theta = ctx->d_theta;
+    p.prefetch_tables = 1;
     p.batch = batch;
     p.bt_stride = bt_stride;
     p.Hq = ctx->cfg.num_q_heads;
@@ -598,6 +612,7 @@ pkv_status pkv_qkv_rope_append(pkv_ctx* ctx, const void* x, const void* w_qkv, i
     p.v_scale = v_scale;
     p.err = ctx->d_err;
     p.rope_base = ctx->cfg.rope_base;
+    p.theta = ctx->d_theta;
     p.batch = batch;
     p.hidden = hidden;
     p.bt_stride = bt_stride;

@@ -75,6 +75,8 @@ struct RopeParams {
     // position L_b + i - cu_q[b]; the grid covers n_tokens rows; q_len unused
     const int32_t* cu_q = nullptr;
     int n_tokens = 0;
+    const double* theta = nullptr;   // [D / 2] rope_base^(-2i/D) in fp64, from the context
+    int prefetch_tables = 0;         // 1: prefetch each request's block-table row into L2
 };
 
 struct AttnParams {
@@ -149,6 +151,7 @@ struct QkvParams {
     const float* v_scale;
     int* err;
     double rope_base;
+    const double* theta;      // [D / 2] rope_base^(-2i/D) in fp64, from the context
     int batch, hidden, bt_stride, Hq, Hkv, D, P, num_pages, fp8;
     int x_rows;               // token rows per x TMA box: min(128, batch rounded up to 16)
     int w_tiled;              // 1: weights in the tiled layout of pkv_qkv_pack_weight

@@ -296,7 +296,7 @@ qkv_rope_append_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_con
         }
         if (kind < 2) {
             const int np = 8 * ng;
-            for (int i = u; i < np; i += kTabThreads) s_theta[i] = pow(p.rope_base, (-2.0 * (8 * g0 + i)) / D);
+            for (int i = u; i < np; i += kTabThreads) s_theta[i] = p.theta[8 * g0 + i];
             asm volatile("bar.sync 1, %0;" ::"n"(kTabThreads) : "memory");   // s_L and s_theta complete
             for (int it = u; it < rows * np; it += kTabThreads) {
                 const int r = it / np, i = it - r * np;

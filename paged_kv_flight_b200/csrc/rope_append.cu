@@ -48,8 +48,11 @@ __device__ __forceinline__ void sincos_reduced(double phi, double* s, double* c)
     sincos(r, s, c);
 }
 
+// bf16 pools: nine CTAs per SM (at most 56 registers) keep the largest
+// batches' grids to one wave (256 requests x 5 CTAs for 64 + 8 heads of
+// d = 128); the E4M3 stores need more registers and are left unbounded.
 template <int D, bool FP8>
-__global__ void __launch_bounds__(kRopeThreads) rope_append_kernel(const RopeParams p)
+__global__ void __launch_bounds__(kRopeThreads, FP8 ? 1 : 9) rope_append_kernel(const RopeParams p)
 {
     constexpr int HALF = D / 2;
     constexpr int PIECES = HALF / 8;  // 8 pairs per work item
@@ -112,9 +115,17 @@ __global__ void __launch_bounds__(kRopeThreads) rope_append_kernel(const RopePar
         return;
     }
     const int slot = L % p.P;
+    if (blockIdx.y == 0 && t == 0 && p.prefetch_tables) {
+        // the attention that follows walks this request's block-table row:
+        // bring it into L2 now (one 128-byte line per thread)
+        const int lines = (p.bt_stride * 4 + 127) / 128;
+        const char* row = reinterpret_cast<const char*>(p.block_tables + (size_t)b * p.bt_stride);
+        for (int i = threadIdx.x; i < lines; i += blockDim.x)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(row + 128 * i));
+    }
 
     for (int i = threadIdx.x; i < HALF; i += blockDim.x) {
-        const double theta = pow(p.rope_base, (-2.0 * i) / D);
+        const double theta = p.theta[i];    // rope_base^(-2i/d), computed once per context
         double s, c;
         sincos_reduced((double)L * theta, &s, &c);
         s_cos[i] = c;
