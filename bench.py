@@ -620,7 +620,7 @@ def run_ours(args, name, rank, world, local_rank, cpu_budget=None):
         "e2e": e2e,
         "gpu_launches": 3 * K,
         "clocks": clock_info,
-        "when": datetime.datetime.utcnow().isoformat() + "Z",
+        "when": datetime.datetime.now(datetime.timezone.utc).isoformat(),
     }
     if cpu is not None:
         line["cpu_baseline"] = cpu
@@ -953,6 +953,36 @@ def run_loop(args, rank, world, local_rank):
             "loop_stats": r["stats"], "gpu_launches": int(r["stats"].get("pkv_launches", 0)), "clocks": clock_info}
 
 
+def run_each_in_own_process(args, names) -> int:
+    """One GPU, several workloads: each runs in a fresh process of this script
+    (its own CUDA context and allocator), and its JSON line is passed on.
+    Measured on one box: the 70B-shaped workload's step ran 5% slower right
+    after the llama8b workload in the same process than alone, with the same
+    flags."""
+    import subprocess
+    flags = ["--steps", str(args.steps), "--warmup", str(args.warmup), "--gpus", "1"]
+    for opt in ("no_e2e", "no_cpu_baseline", "no_graph", "two_calls"):
+        if getattr(args, opt):
+            flags.append("--" + opt.replace("_", "-"))
+    if args.tail_chunks is not None:
+        flags += ["--tail-chunks", str(args.tail_chunks)]
+    if args.requests is not None:
+        flags += ["--requests", str(args.requests)]
+    for i, name in enumerate(names):
+        last = i == len(names) - 1
+        # the full CPU-baseline budget on the last line printed, a short one before it
+        budget = args.cpu_budget if last else min(5.0, args.cpu_budget)
+        cmd = [sys.executable, os.path.abspath(__file__), "--config", name, "--cpu-budget", str(budget), *flags]
+        r = subprocess.run(cmd, stdout=subprocess.PIPE, text=True)
+        for ln in r.stdout.splitlines():
+            if ln.startswith("{"):
+                print(ln, flush=True)
+        if r.returncode != 0:
+            print(f"bench: workload {name} failed (exit {r.returncode})", file=sys.stderr)
+            return r.returncode
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -973,6 +1003,8 @@ def main(argv=None):
                     help="keep only the first N requests of the workload (a smaller case for profiler captures)")
     ap.add_argument("--ref-budget", type=int, default=1_200_000,
                     help="attended token-heads per reference step")
+    ap.add_argument("--in-process", action="store_true",
+                    help="on one GPU, run several workloads in this process instead of one process each")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -993,6 +1025,9 @@ def main(argv=None):
             last = i == len(names) - 1
             print(json.dumps(run_reference(args, name, world, time_budget_s=45.0 if last else 12.0)), flush=True)
         return 0
+
+    if world == 1 and len(names) > 1 and not args.in_process:
+        return run_each_in_own_process(args, names)
 
     import torch
     if world > 1:

@@ -55,7 +55,10 @@ constexpr int kQkvThreads = 192;            // 6 warps: producer, MMA, 4 for the
 constexpr int kQkvM = 128;                     // tokens per tile (TMEM lanes, rows of A)
 constexpr int kQkvBK = 64;                     // hidden elements per stage: one 128-byte row
 constexpr int kQkvMaxStages = 8;
-constexpr int kQkvBudgetWide = 200 * 1024;     // ring + table: one CTA per SM
+#ifndef PKV_QKV_BUDGET_KB
+#define PKV_QKV_BUDGET_KB 200
+#endif
+constexpr int kQkvBudgetWide = PKV_QKV_BUDGET_KB * 1024;   // ring + table: one CTA per SM
 constexpr int kQkvBudgetNarrow = 104 * 1024;   // two CTAs per SM
 constexpr int kQkvSmemLimit = 1024 + 220 * 1024;
 constexpr int kQkvRecvRow = 80;                // bytes per row of received partials (64 + 16: no bank conflicts)

@@ -147,3 +147,30 @@ def test_reference_arm_under_torchrun_prints_once_from_rank_zero():
     assert len(lines) == 1
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
+
+
+def test_one_gpu_suite_runs_each_workload_in_its_own_process(monkeypatch, capsys):
+    # the children's command lines carry the parent's flags, each workload's
+    # name and its CPU-baseline budget (short before the last line); their
+    # JSON lines are passed on in order
+    import subprocess
+    calls = []
+
+    class Done:
+        def __init__(self, cmd):
+            self.returncode = 0
+            self.stdout = "noise\n" + json.dumps({"workload": cmd[cmd.index("--config") + 1]}) + "\n"
+
+    def fake_run(cmd, stdout=None, text=None):
+        calls.append(cmd)
+        return Done(cmd)
+
+    monkeypatch.setattr(subprocess, "run", fake_run)
+    assert bench.main(["--steps", "7", "--warmup", "4", "--no-e2e"]) == 0
+    assert [c[c.index("--config") + 1] for c in calls] == list(bench.SUITE)
+    budgets = [float(c[c.index("--cpu-budget") + 1]) for c in calls]
+    assert budgets[:-1] == [5.0] * (len(calls) - 1) and budgets[-1] == 20.0
+    for c in calls:
+        assert c[c.index("--steps") + 1] == "7" and c[c.index("--warmup") + 1] == "4" and "--no-e2e" in c
+    out = [json.loads(ln)["workload"] for ln in capsys.readouterr().out.splitlines() if ln.startswith("{")]
+    assert out == list(bench.SUITE)
