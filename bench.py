@@ -488,6 +488,38 @@ def run_ours(args, name, rank, world, local_rank, cpu_budget=None):
     torch.cuda.synchronize()
     barrier()
     step_call_ms = [a.elapsed_time(b) for a, b in sev]
+
+    # the kernels' own time inside a replayed step: the two calls captured
+    # in a graph with timing events recorded as graph nodes before the
+    # append, between the calls and after the combine; each replay is read
+    # back before the next (L2 flushed before each, outside the events)
+    rope_g_ms, attn_g_ms = [], []
+    if not args.no_graph:
+        try:
+            te = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)]
+            side = torch.cuda.Stream(dev)
+            torch.cuda.synchronize()
+            tgraph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(tgraph, stream=side):
+                te[0].record()
+                rope_call(dv)
+                te[1].record()
+                attn_call(dv, out)
+                te[2].record()
+            for k in range(args.warmup + K):
+                flush.zero_()
+                tgraph.replay()
+                torch.cuda.synchronize()
+                if k >= args.warmup:
+                    rope_g_ms.append(te[0].elapsed_time(te[1]))
+                    attn_g_ms.append(te[1].elapsed_time(te[2]))
+            del tgraph
+        except RuntimeError as e:          # timing events inside graphs unavailable: eager figures only
+            print(f"bench: in-graph kernel timing unavailable ({e})", file=sys.stderr)
+            rope_g_ms, attn_g_ms = [], []
+            torch.cuda.synchronize()
+        clocks.sample()
+        barrier()
     clock_info = clocks.stop()
     step_ms = [a.elapsed_time(c) for a, _, c in ev]
     rope_ms = [a.elapsed_time(b) for a, b, _ in ev]
@@ -501,6 +533,11 @@ def run_ours(args, name, rank, world, local_rank, cpu_budget=None):
     attn_max = max_over_ranks(med(attn_ms))
     step_max = max_over_ranks(med(graph_ms)) if graph_ms is not None else eager_max
     step_mean = max_over_ranks(sum(graph_ms if graph_ms is not None else step_ms) / K)
+    # the attention's own time: inside the replayed graph when measured,
+    # else the eager events (which include the launch gap)
+    attn_graph_max = max_over_ranks(med(attn_g_ms)) if attn_g_ms else None
+    rope_graph_max = max_over_ranks(med(rope_g_ms)) if rope_g_ms else None
+    attn_for_roofline = attn_graph_max if attn_graph_max is not None else attn_max
     by = workload_bytes(w)
     total_bytes = sum_over_ranks(float(by))
     total_reqs = sum_over_ranks(float(B))
@@ -588,7 +625,7 @@ def run_ours(args, name, rank, world, local_rank, cpu_budget=None):
 
     peak, peak_src = measured_peak()
     value = total_bytes / (step_max * 1e-3) / 1e9
-    attn_gbs = by / (attn_max * 1e-3) / 1e9
+    attn_gbs = by / (attn_for_roofline * 1e-3) / 1e9
     traffic = recorded_traffic(name)
     kernel = (f"decode_attn_tokens_kernel<{w.d},bf16>" if tok
               else f"decode_attn_kernel<{w.d},{'e4m3' if w.kv_fp8 else 'bf16'}>")
@@ -607,6 +644,8 @@ def run_ours(args, name, rank, world, local_rank, cpu_budget=None):
         "request_tokens_per_s": total_reqs / (step_max * 1e-3),
         "step_us": step_max * 1e3, "step_us_eager_one_call": max_over_ranks(med(step_call_ms)) * 1e3,
         "step_us_eager": eager_max * 1e3, "attn_us": attn_max * 1e3,
+        "attn_us_in_graph": None if attn_graph_max is None else attn_graph_max * 1e3,
+        "rope_append_us_in_graph": None if rope_graph_max is None else rope_graph_max * 1e3,
         "rope_append_us": max_over_ranks(med(rope_ms)) * 1e3,
         "ms_per_step_mean": step_mean,
         "step_us_hot_l2": hot_ms * 1e3,
@@ -616,7 +655,10 @@ def run_ours(args, name, rank, world, local_rank, cpu_budget=None):
                      "frac": attn_gbs / peak, "traffic": traffic, "kernel": kernel,
                      "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
                      else "fallback 6650 GB/s",
-                     "bytes_per_launch": by},
+                     "bytes_per_launch": by,
+                     "duration": ("attention + combine inside a replayed CUDA graph (timing events as graph "
+                                  "nodes), median" if attn_graph_max is not None
+                                  else "attention + combine, eager events (launch gap included), median")},
         "e2e": e2e,
         "gpu_launches": 3 * K,
         "clocks": clock_info,
@@ -706,6 +748,8 @@ def run_qkv(args, rank, world, local_rank):
         flush_w.zero_()
         torch.sum(flush_r, dim=0, out=sink)
 
+    if args.qkv_split is not None:
+        pkv.pkv_set_qkv_split(ctx, args.qkv_split)
     # the weight is static: packed once into the tiled layout at load time
     Wt = torch.empty_like(W)
     pkv.pkv_qkv_pack_weight(ctx, W, Wt)
@@ -761,12 +805,36 @@ def run_qkv(args, rank, world, local_rank):
     clocks.sample()
     torch.cuda.synchronize()
     barrier()
+    # the projection's own time inside a replayed step: timing events
+    # recorded as graph nodes around it, each replay read back before the next
+    proj_g = []
+    try:
+        te = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+        tgraph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(tgraph, stream=side):
+            te[0].record()
+            proj()
+            te[1].record()
+            pkv.pkv_decode_attn(ctx, q, dv["k_pool"], dv["v_pool"], None, None, dv["block_tables"], dv["seq_lens"],
+                                out)
+        for k in range(args.warmup + K):
+            flush()
+            tgraph.replay()
+            torch.cuda.synchronize()
+            if k >= args.warmup:
+                proj_g.append(te[0].elapsed_time(te[1]))
+        del tgraph
+    except RuntimeError as e:
+        print(f"bench: in-graph kernel timing unavailable ({e})", file=sys.stderr)
+        proj_g = []
+        torch.cuda.synchronize()
     clock_info = clocks.stop()
     st, bits = pkv.pkv_check_device_error(ctx)
     if st != pkv.PKV_OK:
         raise RuntimeError(f"device error: {pkv.pkv_status_str(st)} bits={bits}")
     del graph
     pkv.pkv_destroy(ctx)
+    proj_graph_ms = max_over_ranks(statistics.median(proj_g)) if proj_g else None
     proj_ms = max_over_ranks(statistics.median(a.elapsed_time(b) for a, b in ev))
     rows_ms = max_over_ranks(statistics.median(a.elapsed_time(b) for a, b in rev))
     step_ms = max_over_ranks(statistics.median(a.elapsed_time(b) for a, b in gev))
@@ -777,7 +845,8 @@ def run_qkv(args, rank, world, local_rank):
     attn_bytes = workload_bytes(w)
     by = sum_over_ranks(float(proj_bytes + attn_bytes))
     peak, peak_src = measured_peak()
-    gbs = proj_bytes / (proj_ms * 1e-3) / 1e9
+    proj_roof_ms = proj_graph_ms if proj_graph_ms is not None else proj_ms
+    gbs = proj_bytes / (proj_roof_ms * 1e-3) / 1e9
     tflops_peak = None
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -790,16 +859,20 @@ def run_qkv(args, rank, world, local_rank):
             "config": {"workload": "qkv8b", "description": "llama8b batch (64 tokens) from the layer input: "
                        "QKV projection 4096 -> 6144 on tcgen05 fused with RoPE + append, then decode attention",
                        "l2": "flushed before every step, outside the event window",
-                       "timing": "projection alone: eager events; step: CUDA-graph replay of projection + attention",
+                       "timing": "projection: eager events and inside a replayed graph; step: CUDA-graph replay "
+                                 "of projection + attention",
                        "weights": "packed once into the tiled layout (pkv_qkv_pack_weight) before timing"},
             "step_us": step_ms * 1e3, "projection_us": proj_ms * 1e3,
+            "projection_us_in_graph": None if proj_graph_ms is None else proj_graph_ms * 1e3,
             "projection_rows_layout_us": rows_ms * 1e3,
             "projection_launch": dict(shape, clusters=w.Hq + 2 * w.Hkv),
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
                          "traffic": recorded_traffic("qkv8b"), "kernel": "qkv_rope_append_kernel<128>",
-                         "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)", "bytes_per_launch": proj_bytes},
-            "projection_tflops": proj_flop / (proj_ms * 1e-3) / 1e12,
-            "projection_tflops_frac_of_bf16_peak": proj_flop / (proj_ms * 1e-3) / 1e12 / tflops_peak,
+                         "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)", "bytes_per_launch": proj_bytes,
+                         "duration": ("the projection inside a replayed CUDA graph (timing events as graph nodes), "
+                                      "median" if proj_graph_ms is not None else "the projection, eager events, median")},
+            "projection_tflops": proj_flop / (proj_roof_ms * 1e-3) / 1e12,
+            "projection_tflops_frac_of_bf16_peak": proj_flop / (proj_roof_ms * 1e-3) / 1e12 / tflops_peak,
             "gpu_launches": 5 * K, "clocks": clock_info}
 
 
@@ -1003,6 +1076,8 @@ def main(argv=None):
                     help="keep only the first N requests of the workload (a smaller case for profiler captures)")
     ap.add_argument("--ref-budget", type=int, default=1_200_000,
                     help="attended token-heads per reference step")
+    ap.add_argument("--qkv-split", type=int, default=None,
+                    help="qkv8b: CTAs per head for the projection (1..4; library choice if omitted)")
     ap.add_argument("--in-process", action="store_true",
                     help="on one GPU, run several workloads in this process instead of one process each")
     args = ap.parse_args(argv)
