@@ -373,7 +373,6 @@ def run_ours(args, name, rank, world, local_rank, cpu_budget=None):
     ctx = pkv.pkv_create(cfg)
     if args.tail_chunks is not None:
         pkv.pkv_set_tail_chunks(ctx, args.tail_chunks)
-
     tok = w.q_len > 1          # several new tokens per request: the *_tokens entry points
     out = torch.empty(B, *((w.q_len,) if tok else ()), w.Hq, w.d, dtype=torch.bfloat16, device=dev)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
@@ -416,21 +415,6 @@ def run_ours(args, name, rank, world, local_rank, cpu_budget=None):
         else:
             pkv.pkv_decode_step(ctx, x["q"], x["k_new"], x["v_new"], dv["k_pool"], dv["v_pool"], dv["k_scale"],
                                 dv["v_scale"], x["block_tables"], x["seq_lens"], o, q_len=w.q_len, stream=stream)
-
-    # per-warp weights of the attention split, measured on this batch once
-    # (a setup call, outside every timed region; one-token batches only)
-    # (several new tokens per request: measured with the one-token attention
-    # over the same cache, the first new token's query)
-    calibrated = False
-    if not args.no_calibrate:
-        rope_call(dv)
-        q1 = dv["q"][:, 0].contiguous() if tok else dv["q"]
-        o1 = torch.empty(B, w.Hq, w.d, dtype=torch.bfloat16, device=dev)
-        calibrated = pkv.pkv_calibrate(ctx, q1, dv["k_pool"], dv["v_pool"], dv["k_scale"], dv["v_scale"],
-                                       dv["block_tables"], dv["seq_lens"], o1, rounds=6,
-                                       check=False) == pkv.PKV_OK
-        del q1, o1
-    split_weights = pkv.pkv_get_split_weights(ctx)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -676,9 +660,6 @@ def run_ours(args, name, rank, world, local_rank, cpu_budget=None):
                                   "nodes), median" if attn_graph_max is not None
                                   else "attention + combine, eager events (launch gap included), median")},
         "e2e": e2e,
-        "split_weights": {"calibrated": calibrated, "min": min(split_weights), "max": max(split_weights),
-                          "note": "per-warp weights of the attention split (1024 = 1.0), measured by pkv_calibrate "
-                                  "on this batch before timing"},
         "gpu_launches": 3 * K,
         "clocks": clock_info,
         "when": datetime.datetime.now(datetime.timezone.utc).isoformat(),
@@ -1086,8 +1067,6 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay timing")
-    ap.add_argument("--no-calibrate", action="store_true",
-                    help="equal split ranges (skip pkv_calibrate's per-warp weights)")
     ap.add_argument("--two-calls", action="store_true",
                     help="time the step as pkv_rope_append + pkv_decode_attn instead of pkv_decode_step")
     ap.add_argument("--tail-chunks", type=int, default=None,

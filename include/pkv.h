@@ -63,11 +63,8 @@
  *       host page allocator of pkv_pages.h;
  *   pkv_decode_attn_noalloc                          the attention without a
  *       context (no allocation);
- *   pkv_calibrate, pkv_set_split_weights             per-warp weights of the
- *       attention split, measured on a representative batch;
  *   pkv_set_workers, pkv_set_tail_chunks, pkv_set_qkv_split,
- *   pkv_qkv_launch_shape, pkv_workspace_bytes,
- *   pkv_get_split_weights                            tuning and inspection.
+ *   pkv_qkv_launch_shape, pkv_workspace_bytes        tuning and inspection.
  *
  * Errors: host-side checks return PKV_ERR_INVALID_ARG / PKV_ERR_UNSUPPORTED
  * and launch nothing.  A failed launch returns PKV_ERR_CUDA.  Range errors
@@ -339,43 +336,6 @@ pkv_status pkv_qkv_launch_shape(pkv_ctx* ctx, int batch, int hidden, int* shape)
 
 /* Bytes of device workspace the context holds. */
 size_t pkv_workspace_bytes(const pkv_ctx* ctx);
-
-/* Per-warp weights of the attention split.  The attention cuts the
- * flattened (request, kv head, tile) sequence into one contiguous range per
- * warp worker (8 per SM); by default the ranges are equal.  Warps stream at
- * measurably different speeds (up to ~15% apart on one GPU), the same warps
- * on every launch of a given kind of batch, so equal ranges end on the
- * slowest ones.  With weights, worker v gets a range proportional to its
- * weight (fixed point, 1024 = 1.0, each in [512, 2048]); they apply when
- * every warp of the grid is a worker (the automatic worker count of a batch
- * of at least 8 tiles per warp) and the batch has at least 8 tiles per
- * worker, and then without a dynamic tail.  Results do not depend on the
- * weights beyond rounding; a context's calls are deterministic while its
- * weights stay put.
- *
- * pkv_calibrate measures them on a representative batch: the arguments and
- * effect of pkv_decode_attn (out receives the batch's attention), run
- * `rounds` times (2 .. 64; the first warms up); after each later launch
- * every warp's streaming speed (its tiles over the time from its first
- * tile's data to its end, read from the device clock) is folded into a
- * running mean and the weights are set proportional to it.  Synchronous:
- * it allocates and frees a small scratch and synchronises `stream`; make it
- * before any stream capture and not while another call of this context
- * runs.  PKV_ERR_UNSUPPORTED (weights back to equal) when the batch is too
- * small to give every warp work; other errors as for pkv_decode_attn, with
- * the weights back to equal.
- *
- * pkv_set_split_weights sets them (host array of *count entries as
- * pkv_get_split_weights reports; NULL: equal ranges again), synchronously;
- * PKV_ERR_INVALID_ARG for a weight outside [512, 2048].
- * pkv_get_split_weights writes the count of workers to *count and, if
- * weights is not NULL, the current weights (1024 each when none are set). */
-pkv_status pkv_calibrate(pkv_ctx* ctx, const void* q, const void* k_pool, const void* v_pool,
-                         const float* k_scale, const float* v_scale, const int32_t* block_tables,
-                         int bt_stride, const int32_t* seq_lens, int batch, void* out, int rounds,
-                         cudaStream_t stream);
-pkv_status pkv_set_split_weights(pkv_ctx* ctx, const int* weights);
-pkv_status pkv_get_split_weights(const pkv_ctx* ctx, int* weights, int* count);
 
 /* pkv_decode_attn for callers that cannot allocate device memory.  The pages
  * describe no such entry point; it exists for callers such as a serving

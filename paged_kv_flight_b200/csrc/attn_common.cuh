@@ -46,28 +46,19 @@ struct StageInfo {
     int pad;
 };
 
-// Units of the split.  Warp range v is [r(v), r(v+1)).  Equal ranges:
-// r(v) = v T / W.  Weighted ranges (wpre set, every warp of the grid a
-// worker): worker v has weight wpre[v + 1] - wpre[v] (fixed-point integers,
-// wpre their prefix) and r(v) = T wpre[v] / wpre[W]; the weights follow the
-// per-warp streaming speed measured on the caller's batch (pkv_calibrate),
-// so that warps on slower SMs get fewer tiles.  With K = 0 a range is one
-// unit.  With K > 0 (equal ranges only) unit v (K+1) is the head
-// [r(v), s(v)) and units v (K+1) + 1 + j, j < K, cut the tail
-// [s(v), r(v+1)) of tl = min(range / kTailDen, kTailMaxTiles) tiles at
-// s(v) + j tl / K.  Units are numbered in the order of the tiles they hold
-// and together cover [0, T) once, none empty.  W < 2^16, so an equal r(v)
-// needs one 32-bit division (T = qT W + rT), and tl is small.
+// Units of the split.  Warp range v is [r(v), r(v+1)), r(v) = v T / W.  With
+// K = 0 a range is one unit.  With K > 0 unit v (K+1) is the head
+// [r(v), s(v)) and units v (K+1) + 1 + j, j < K, cut the tail [s(v), r(v+1))
+// of tl = min(range / kTailDen, kTailMaxTiles) tiles at s(v) + j tl / K.
+// Units are numbered in the order of the tiles they hold, none is empty, and
+// together they cover [0, T) once.  W < 2^16, so r(v) needs one 32-bit
+// division (T = qT W + rT), and tl is small.
 struct Split {
     long long T, qT;
     int W, K, rT;
-    const int* wpre;     // [W + 1] prefix of per-worker weights, or null (equal ranges)
-    int ctas;
-    long long cumW;      // wpre[W]
 
     __device__ __forceinline__ long long r(int v) const
     {
-        if (wpre) return (T * (long long)__ldg(&wpre[v])) / cumW;
         return (long long)v * qT + (long long)(((unsigned)v * (unsigned)rT) / (unsigned)W);
     }
     __device__ __forceinline__ static int tail_of(long long range)
@@ -88,17 +79,6 @@ struct Split {
     // index of the unit holding tile x, 0 <= x < T
     __device__ __forceinline__ int unit_of(long long x) const
     {
-        if (wpre) {
-            // the largest v with r(v) <= x (K = 0 here); empty ranges before it
-            // have the same start and a smaller index
-            int lo = 0, hi = W;
-            while (hi - lo > 1) {
-                const int mid = (lo + hi) >> 1;
-                if (r(mid) <= x) lo = mid;
-                else hi = mid;
-            }
-            return lo;
-        }
         const int v = (int)(((x + 1) * W - 1) / T);
         if (K == 0) return v;
         const long long rv = r(v), range = r(v + 1) - rv;
@@ -110,16 +90,10 @@ struct Split {
     }
 };
 
-// The split of T tiles over W warps: weighted ranges when wpre is set, every
-// warp of the grid is a worker (W = ctas x kAttnWarps) and T >= 8 W (then no
-// dynamic tail; with every weight within a factor 4 of every other, each
-// range then holds at least one tile, so every unit of a pair cut between
-// units leaves its partial), else equal ranges with K tail chunks, K at most
-// `max_chunks`: chunks of at least kTailChunkTiles tiles, none when the
-// shortest range is under kTailMinTiles tiles (its tail then holds at least 8
-// tiles, and the head at least 24).
-__device__ __forceinline__ Split make_split(long long T, int W, int max_chunks, const int* wpre = nullptr,
-                                            int ctas = 1)
+// K for T tiles over W warps, at most `max_chunks`: chunks of at least
+// kTailChunkTiles tiles, none when the shortest range is under kTailMinTiles
+// tiles (its tail then holds at least 8 tiles, and the head at least 24).
+__device__ __forceinline__ Split make_split(long long T, int W, int max_chunks)
 {
     Split sp;
     sp.T = T;
@@ -127,14 +101,6 @@ __device__ __forceinline__ Split make_split(long long T, int W, int max_chunks, 
     sp.qT = T / W;
     sp.rT = (int)(T - sp.qT * W);
     sp.K = 0;
-    sp.wpre = nullptr;
-    sp.ctas = ctas;
-    sp.cumW = 1;
-    if (wpre && W == ctas * kAttnWarps && T >= 8LL * W) {
-        sp.wpre = wpre;
-        sp.cumW = max((long long)__ldg(&wpre[W]), 1LL);
-        return sp;
-    }
     if (max_chunks > 0 && sp.qT >= kTailMinTiles)
         sp.K = min(max_chunks, max(1, Split::tail_of(sp.qT) / kTailChunkTiles));
     return sp;

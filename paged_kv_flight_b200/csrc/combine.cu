@@ -65,8 +65,8 @@ __global__ void __launch_bounds__(kCombineThreads, 2) combine_kernel(const AttnP
     const int* prefix = p.meta + 4;
     const int nt = __ldg(&prefix[b + 1]) - __ldg(&prefix[b]);
     if (nt == 0) return;
-    Split sp = make_split(T, W, 0, p.wpre, p.ctas);   // the attention launch's split
-    sp.K = __ldg(&p.meta[3]);   // as the attention launch chose it (0 when weighted)
+    Split sp = make_split(T, W, 0);
+    sp.K = __ldg(&p.meta[3]);   // as the attention launch chose it
     const long long ts = (long long)__ldg(&prefix[b]) * p.Hkv + (long long)kvh * nt;
     const int U0 = sp.unit_of(ts), U1 = sp.unit_of(ts + nt - 1);
     if (U0 == U1) return;
@@ -230,8 +230,8 @@ __global__ void __launch_bounds__(kCombineWarpThreads, 2) combine_warp_kernel(co
     const int pb = __ldg(&prefix[b]);
     const int nt = __ldg(&prefix[b + 1]) - pb;
     if (T == 0 || nt == 0) return;
-    Split sp = make_split(T, W, 0, p.wpre, p.ctas);   // the attention launch's split
-    sp.K = __ldg(&p.meta[3]);   // as the attention launch chose it (0 when weighted)
+    Split sp = make_split(T, W, 0);
+    sp.K = __ldg(&p.meta[3]);   // as the attention launch chose it
     const long long ts = (long long)pb * p.Hkv + (long long)kvh * nt;
     const int U0 = sp.unit_of(ts), U1 = sp.unit_of(ts + nt - 1);
     if (U0 == U1) return;

@@ -159,7 +159,7 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
     else Wl = min(Wl, (T + kMinTilesPerWorker - 1) / kMinTilesPerWorker);
     Wl = max(1LL, min(Wl, max(T, 1LL)));
     const int W = (int)Wl;
-    const Split sp = make_split(max(T, 1LL), W, p.tail_chunks, p.wpre, p.ctas);
+    const Split sp = make_split(max(T, 1LL), W, p.tail_chunks);
     if (blockIdx.x == 0) {
         // the combine kernel that follows needs the same split geometry
         if (tid == 0) {
@@ -325,7 +325,6 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
     load_q<D, FP8>(p, cb, ckvh, g, c4, qn);
     n_next = p.seq_lens[cb] + 1;
 
-    unsigned long long t_first = 0;   // calibration only
     for (int k = 0; k < issued; ++k) {
         if (!dead) {
             const bool ok = __all_sync(kFull, mbar_wait_bounded(my_bar0 + 8u * s, parity, kWaitLimitNs));
@@ -334,7 +333,6 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
                 k_dead = k;
                 if (lane == 0) atomicOr(p.err, kErrTimeout);
             }
-            if (k == 0 && p.ctimes) t_first = global_timer_ns();
         }
         if (dead) {
             // control flow only: no data, no writes
@@ -633,15 +631,6 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
         }
     }
 
-    if (p.ctimes && lane == 0) {
-        // calibration: this worker's loop time (first tile's data to the
-        // end) and its tiles
-        unsigned long long* t = p.ctimes + (size_t)w * 4;
-        t[0] = t_first;
-        t[1] = global_timer_ns();
-        t[2] = (unsigned long long)issued;
-    }
-
     // a worker that timed out still owns the loads it issued for tiles
     // k_dead .. issued-1 (one per stage): wait for them, bounded
     if (dead && lane == 0) {
@@ -710,7 +699,6 @@ cudaError_t launch_decode_attn(const AttnParams& p, const CUtensorMap& tmk, cons
     const dim3 grid(L.ctas), block(kAttnWarps * 32);
     AttnParams q = p;
     q.stages = L.stages;
-    q.ctas = L.ctas;           // the weighted split needs the grid size (every warp a worker)
     const bool wide = L.tile == kTileWide;
     cudaError_t e;
     if (head_dim == 128) {

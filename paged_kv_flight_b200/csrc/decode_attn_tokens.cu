@@ -190,7 +190,7 @@ decode_attn_tokens_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_
     else Wl = min(Wl, (T + kMinTilesPerWorker - 1) / kMinTilesPerWorker);
     Wl = max(1LL, min(Wl, max(T, 1LL)));
     const int W = (int)Wl;
-    const Split sp = make_split(max(T, 1LL), W, 0, p.wpre, p.ctas);
+    const Split sp = make_split(max(T, 1LL), W, 0);
     if (blockIdx.x == 0) {
         // the combine kernel that follows needs the same split geometry
         if (tid == 0) {
@@ -695,7 +695,6 @@ cudaError_t launch_decode_attn_tokens(const AttnParams& p, const CUtensorMap& tm
     AttnParams q = p;
     q.stages = L.stages;
     q.tail_chunks = 0;
-    q.ctas = L.ctas;           // the weighted split needs the grid size (every warp a worker)
     cudaError_t e;
     if (head_dim == 128) {
         if (fp8) e = launch_attn_kernel(decode_attn_tokens_kernel<128, true, kAttnWarps>, grid, block, L.smem_bytes, stream, pdl, tmk, tmv, q);

@@ -29,9 +29,6 @@ struct pkv_ctx {
     int* d_err;
     int* d_claim;         // chunk counter of the attention's dynamic tail
     double* d_theta;      // [head_dim / 2] rope_base^(-2i/d), fp64
-    int* d_wpre;          // [workers + 1] prefix of the per-worker split weights
-    int weighted;         // 1: the attention splits by d_wpre (pkv_set_split_weights / pkv_calibrate)
-    int* h_weights;       // [workers] the weights on the host
     int* d_meta;
     int vmax;             // virtual requests a varlen attention call may have (bf16 pools)
     int4* d_vmap;         // [vmax] the varlen plan
@@ -221,9 +218,7 @@ pkv_status pkv_create(const pkv_config* cfg, pkv_ctx** out)
     const size_t b_pml = 2 * rows_units * 2 * sizeof(float);
     const size_t b_vm = (size_t)ctx->vmax * sizeof(int4) + 256;   // varlen plan + its count
     const size_t b_th = ((size_t)cfg->head_dim / 2 * sizeof(double) + 255) & ~(size_t)255;   // RoPE frequencies
-    const int nw = ctx->attn.ctas * pkv::kAttnWarps;                                        // warp workers
-    const size_t b_w = ((size_t)(nw + 1) * sizeof(int) + 255) & ~(size_t)255;              // split weights
-    ctx->ws_bytes = b_err + b_cnt + b_po + b_pml + b_vm + b_th + b_w;
+    ctx->ws_bytes = b_err + b_cnt + b_po + b_pml + b_vm + b_th;
     if (cudaMalloc(&ctx->ws, ctx->ws_bytes) != cudaSuccess) {
         cudaGetLastError();
         free(ctx);
@@ -232,14 +227,6 @@ pkv_status pkv_create(const pkv_config* cfg, pkv_ctx** out)
     uint8_t* base = static_cast<uint8_t*>(ctx->ws);
     ctx->d_err = reinterpret_cast<int*>(base);
     ctx->d_claim = reinterpret_cast<int*>(base + 128);
-    ctx->d_wpre = reinterpret_cast<int*>(base + b_err + b_cnt + b_po + b_pml + b_vm + b_th);
-    ctx->h_weights = static_cast<int*>(malloc(sizeof(int) * (size_t)nw));
-    if (!ctx->h_weights) {
-        cudaFree(ctx->ws);
-        free(ctx);
-        return PKV_ERR_OOM;
-    }
-    for (int v = 0; v < nw; ++v) ctx->h_weights[v] = pkv::kWeightOne;
     ctx->tail_chunks = pkv::kDefaultTailChunks;
     ctx->d_meta = reinterpret_cast<int*>(base + b_err);
     ctx->d_part_o = reinterpret_cast<float*>(base + b_err + b_cnt);
@@ -341,7 +328,6 @@ pkv_status decode_attn_launch(pkv_ctx* ctx, const void* q, const void* k_pool, c
     p.stages = ctx->attn.stages;
     p.workers = ctx->workers;
     p.tail_chunks = ctx->tail_chunks;
-    p.wpre = ctx->weighted ? ctx->d_wpre : nullptr;
     p.q_len = 1;
     const cudaError_t e = pkv::launch_decode_attn(p, ctx->tmk, ctx->tmv, ctx->cfg.head_dim,
                                                   ctx->cfg.kv_dtype == PKV_KV_FP8_E4M3, ctx->attn, stream, pdl);
@@ -465,7 +451,6 @@ pkv_status attn_tokens_launch(pkv_ctx* ctx, const void* q, const void* k_pool, c
     p.q_len = q_len;
     p.vmap = vmap;
     p.vcount = vcount;
-    p.wpre = ctx->weighted ? ctx->d_wpre : nullptr;
     const cudaError_t e = pkv::launch_decode_attn_tokens(p, *mk, *mv, ctx->cfg.head_dim, fp8, ctx->attn_tok, stream,
                                                          pdl);
     return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
@@ -650,7 +635,6 @@ pkv_status pkv_destroy(pkv_ctx* ctx)
     pkv_status st = PKV_OK;
     if (cudaDeviceSynchronize() != cudaSuccess) st = PKV_ERR_CUDA;
     if (ctx->ws && cudaFree(ctx->ws) != cudaSuccess) st = PKV_ERR_CUDA;
-    free(ctx->h_weights);
     free(ctx);
     return st;
 }
@@ -716,167 +700,5 @@ pkv_status pkv_set_tail_chunks(pkv_ctx* ctx, int max_chunks)
 }
 
 size_t pkv_workspace_bytes(const pkv_ctx* ctx) { return ctx ? ctx->ws_bytes : 0; }
-
-}  // extern "C"
-
-namespace {
-
-// Uploads the prefix of the context's host weights (one per warp worker);
-// synchronous.
-pkv_status upload_weights(pkv_ctx* ctx, bool weighted)
-{
-    const int n = ctx->attn.ctas * pkv::kAttnWarps;
-    int* pre = static_cast<int*>(malloc(sizeof(int) * (size_t)(n + 1)));
-    if (!pre) return PKV_ERR_OOM;
-    pre[0] = 0;
-    for (int v = 0; v < n; ++v) pre[v + 1] = pre[v] + ctx->h_weights[v];
-    const cudaError_t e = cudaMemcpy(ctx->d_wpre, pre, sizeof(int) * (size_t)(n + 1), cudaMemcpyHostToDevice);
-    free(pre);
-    if (e != cudaSuccess) return PKV_ERR_CUDA;
-    ctx->weighted = weighted ? 1 : 0;
-    return PKV_OK;
-}
-
-// Scales w so that its mean is kWeightOne, within [kWeightMin, kWeightMax].
-void normalise_weights(double* w, int n, int* out)
-{
-    for (int pass = 0; pass < 3; ++pass) {
-        double mean = 0.0;
-        for (int c = 0; c < n; ++c) mean += w[c];
-        mean /= n;
-        for (int c = 0; c < n; ++c) {
-            w[c] *= pkv::kWeightOne / mean;
-            w[c] = std::min<double>(pkv::kWeightMax, std::max<double>(pkv::kWeightMin, w[c]));
-        }
-    }
-    for (int c = 0; c < n; ++c) out[c] = (int)lrint(w[c]);
-}
-
-}  // namespace
-
-extern "C" {
-
-pkv_status pkv_set_split_weights(pkv_ctx* ctx, const int* weights)
-{
-    if (!ctx) return PKV_ERR_INVALID_ARG;
-    const int n = ctx->attn.ctas * pkv::kAttnWarps;
-    if (!weights) {
-        for (int v = 0; v < n; ++v) ctx->h_weights[v] = pkv::kWeightOne;
-        return upload_weights(ctx, false);
-    }
-    for (int v = 0; v < n; ++v)
-        if (weights[v] < pkv::kWeightMin || weights[v] > pkv::kWeightMax) return PKV_ERR_INVALID_ARG;
-    for (int v = 0; v < n; ++v) ctx->h_weights[v] = weights[v];
-    return upload_weights(ctx, true);
-}
-
-pkv_status pkv_get_split_weights(const pkv_ctx* ctx, int* weights, int* count)
-{
-    if (!ctx || !count) return PKV_ERR_INVALID_ARG;
-    const int n = ctx->attn.ctas * pkv::kAttnWarps;
-    *count = n;
-    if (weights)
-        for (int v = 0; v < n; ++v) weights[v] = ctx->h_weights[v];
-    return PKV_OK;
-}
-
-pkv_status pkv_calibrate(pkv_ctx* ctx, const void* q, const void* k_pool, const void* v_pool, const float* k_scale,
-                         const float* v_scale, const int32_t* block_tables, int bt_stride, const int32_t* seq_lens,
-                         int batch, void* out, int rounds, cudaStream_t stream)
-{
-    pkv_status st = check_call(ctx, batch, bt_stride, k_pool, v_pool, k_scale, v_scale, block_tables, seq_lens);
-    if (st != PKV_OK) return st;
-    if (batch == 0 || rounds < 2 || rounds > 64 || !q || !out || !aligned16(q) || !aligned16(out))
-        return PKV_ERR_INVALID_ARG;
-    const bool fp8 = ctx->cfg.kv_dtype == PKV_KV_FP8_E4M3;
-    const int nw = ctx->attn.ctas * pkv::kAttnWarps;
-    const size_t t_bytes = (size_t)nw * 4 * sizeof(unsigned long long);
-    void* d_t = nullptr;
-    if (cudaMalloc(&d_t, t_bytes) != cudaSuccess) {
-        cudaGetLastError();
-        return PKV_ERR_OOM;
-    }
-    unsigned long long* h_t = static_cast<unsigned long long*>(malloc(t_bytes));
-    double* w = static_cast<double*>(malloc(sizeof(double) * (size_t)nw));
-    double* speed = static_cast<double*>(calloc((size_t)nw, sizeof(double)));
-    if (!h_t || !w || !speed) st = PKV_ERR_OOM;
-    if (st == PKV_OK && ctx->tm_k_ptr != k_pool) {
-        if (!encode_pool(ctx, k_pool, &ctx->tmk)) st = PKV_ERR_CUDA;
-        else ctx->tm_k_ptr = k_pool;
-    }
-    if (st == PKV_OK && ctx->tm_v_ptr != v_pool) {
-        if (!encode_pool(ctx, v_pool, &ctx->tmv)) st = PKV_ERR_CUDA;
-        else ctx->tm_v_ptr = v_pool;
-    }
-    for (int v = 0; st == PKV_OK && v < nw; ++v) w[v] = ctx->h_weights[v];
-    int measured = 0;
-    for (int it = 0; it < rounds && st == PKV_OK; ++it) {
-        // the first launch warms up; after each later one every worker's
-        // streaming speed (tiles per unit of loop time) is folded into a
-        // running mean, and the weights follow that mean
-        if ((st = upload_weights(ctx, true)) != PKV_OK) break;
-        pkv::AttnParams p;
-        p.q = static_cast<const __nv_bfloat16*>(q);
-        p.out = static_cast<__nv_bfloat16*>(out);
-        p.k_scale = fp8 ? k_scale : nullptr;
-        p.v_scale = fp8 ? v_scale : nullptr;
-        p.block_tables = block_tables;
-        p.seq_lens = seq_lens;
-        p.part_o = ctx->d_part_o;
-        p.part_ml = ctx->d_part_ml;
-        p.meta = ctx->d_meta;
-        p.err = ctx->d_err;
-        p.claim = ctx->d_claim;
-        p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)ctx->cfg.head_dim));
-        p.batch = batch;
-        p.bt_stride = bt_stride;
-        p.Hq = ctx->cfg.num_q_heads;
-        p.Hkv = ctx->cfg.num_kv_heads;
-        p.G = ctx->G;
-        p.P = ctx->cfg.page_size;
-        p.num_pages = ctx->cfg.num_pages;
-        p.stages = ctx->attn.stages;
-        p.workers = 0;
-        p.tail_chunks = 0;
-        p.q_len = 1;
-        p.wpre = ctx->d_wpre;
-        p.ctimes = static_cast<unsigned long long*>(d_t);
-        if (cudaMemsetAsync(d_t, 0, t_bytes, stream) != cudaSuccess ||
-            pkv::launch_decode_attn(p, ctx->tmk, ctx->tmv, ctx->cfg.head_dim, fp8, ctx->attn, stream) != cudaSuccess ||
-            cudaMemcpyAsync(h_t, d_t, t_bytes, cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
-            cudaStreamSynchronize(stream) != cudaSuccess) {
-            st = PKV_ERR_CUDA;
-            break;
-        }
-        if (it == 0) continue;
-        bool all = true;
-        for (int v = 0; v < nw && all; ++v) {
-            const unsigned long long* t = h_t + (size_t)v * 4;
-            all = t[1] > t[0] && t[0] != 0 && t[2] > 0;
-        }
-        if (!all) continue;    // a batch too small for every warp: the weights stay as they are
-        ++measured;
-        for (int v = 0; v < nw; ++v) {
-            const unsigned long long* t = h_t + (size_t)v * 4;
-            const double sp = (double)t[2] / (double)(t[1] - t[0]);
-            speed[v] += (sp - speed[v]) / measured;
-            w[v] = speed[v];
-        }
-        normalise_weights(w, nw, ctx->h_weights);
-        for (int v = 0; v < nw; ++v) w[v] = ctx->h_weights[v];
-    }
-    int word = 0;
-    if (st == PKV_OK && cudaMemcpy(&word, ctx->d_err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
-        st = PKV_ERR_CUDA;
-    if (st == PKV_OK && (word & pkv::kErrTimeout)) st = PKV_ERR_DEVICE_TIMEOUT;
-    if (st == PKV_OK && measured == 0) st = PKV_ERR_UNSUPPORTED;
-    if (st == PKV_OK) st = upload_weights(ctx, true);
-    else (void)pkv_set_split_weights(ctx, nullptr);
-    cudaFree(d_t);
-    free(h_t);
-    free(w);
-    free(speed);
-    return st;
-}
 
 }  // extern "C"

@@ -51,10 +51,6 @@ constexpr int kMaxTailChunks = 8;
 static_assert(kTailChunkTiles > PKV_ATTN_MAX_STAGES, "tail chunks must be longer than the TMA ring");
 constexpr int kDefaultTailChunks = 0;
 
-// Per-CTA weights of the attention split (fixed point, kWeightOne = 1.0),
-// kept within a factor 4 of each other so every weighted range holds a tile.
-constexpr int kWeightOne = 1024, kWeightMin = 512, kWeightMax = 2048;
-
 // Units the split may cut the tiles into (two partial slots each).
 inline size_t max_units(int max_workers, int tail_chunks)
 {
@@ -108,13 +104,6 @@ struct AttnParams {
     // the varlen plan; null for the other calls
     const int4* vmap = nullptr;
     const int* vcount = nullptr;
-    // weighted split (see attn_common.cuh): prefix of the per-CTA weights
-    // [ctas + 1], null for equal ranges; ctas = the attention launch's CTAs
-    const int* wpre = nullptr;
-    int ctas = 0;
-    // calibration only: per worker w, [w][0] its first tile's data and [w][1]
-    // its end (globaltimer ns), [w][2] its tiles; null otherwise
-    unsigned long long* ctimes = nullptr;
 };
 
 cudaError_t launch_rope_append(const RopeParams& p, cudaStream_t stream);

@@ -49,8 +49,7 @@ EXPORTS = ("pkv_create", "pkv_rope_append", "pkv_decode_attn", "pkv_destroy", "p
            "pkv_pages_release", "pkv_pages_block_table", "pkv_pages_seq_lens", "pkv_pages_active",
            "pkv_pages_refcount", "pkv_pages_free_count", "pkv_pages_take_changes", "pkv_qkv_rope_append",
            "pkv_qkv_pack_weight", "pkv_set_qkv_split", "pkv_qkv_launch_shape",
-           "pkv_table_sync", "pkv_rope_append_varlen", "pkv_decode_attn_varlen", "pkv_decode_step",
-           "pkv_calibrate", "pkv_set_split_weights", "pkv_get_split_weights")
+           "pkv_table_sync", "pkv_rope_append_varlen", "pkv_decode_attn_varlen", "pkv_decode_step")
 
 
 class pkv_config(C.Structure):
@@ -118,12 +117,6 @@ lib.pkv_decode_attn_noalloc.argtypes = [C.POINTER(pkv_config), _V, _V, _V, _V, _
 lib.pkv_decode_attn_noalloc.restype = C.c_int
 lib.pkv_decode_step.argtypes = [_V, _V, _V, _V, _V, _V, _V, _V, _V, C.c_int, _V, C.c_int, C.c_int, _V, _V]
 lib.pkv_decode_step.restype = C.c_int
-lib.pkv_calibrate.argtypes = [_V, _V, _V, _V, _V, _V, _V, C.c_int, _V, C.c_int, _V, C.c_int, _V]
-lib.pkv_calibrate.restype = C.c_int
-lib.pkv_set_split_weights.argtypes = [_V, _V]
-lib.pkv_set_split_weights.restype = C.c_int
-lib.pkv_get_split_weights.argtypes = [_V, _V, C.POINTER(C.c_int)]
-lib.pkv_get_split_weights.restype = C.c_int
 
 
 class PkvError(RuntimeError):
@@ -341,42 +334,6 @@ def pkv_decode_step(ctx, q, k_new, v_new, k_pool, v_pool, k_scale, v_scale, bloc
                              _ptr(seq_lens, _I32, "seq_lens"), int(batch), int(q_len), _ptr(out, _ACT, "out"),
                              _stream(stream))
     return _done(st, "pkv_decode_step", check)
-
-
-def pkv_calibrate(ctx, q, k_pool, v_pool, k_scale, v_scale, block_tables, seq_lens, out, rounds: int = 5,
-                  batch: int | None = None, bt_stride: int | None = None, stream=None, check: bool = True) -> int:
-    """Measures the per-warp weights of the attention split on this batch
-    (the arguments of pkv_decode_attn; synchronous; see include/pkv.h)."""
-    if batch is None:
-        batch = int(seq_lens.shape[0])
-    if bt_stride is None:
-        bt_stride = int(block_tables.shape[1])
-    st = lib.pkv_calibrate(ctx, _ptr(q, _ACT, "q"), *_kv(k_pool, v_pool, k_scale, v_scale),
-                           _ptr(block_tables, _I32, "block_tables"), int(bt_stride), _ptr(seq_lens, _I32, "seq_lens"),
-                           int(batch), _ptr(out, _ACT, "out"), int(rounds), _stream(stream))
-    return _done(st, "pkv_calibrate", check)
-
-
-def pkv_get_split_weights(ctx) -> list:
-    n = C.c_int(0)
-    _done(lib.pkv_get_split_weights(ctx, None, C.byref(n)), "pkv_get_split_weights", True)
-    arr = (C.c_int * n.value)()
-    _done(lib.pkv_get_split_weights(ctx, arr, C.byref(n)), "pkv_get_split_weights", True)
-    return list(arr)
-
-
-def pkv_set_split_weights(ctx, weights, check: bool = True) -> int:
-    """weights: a sequence of one int per warp worker (see
-    pkv_get_split_weights), or None for equal ranges."""
-    if weights is None:
-        st = lib.pkv_set_split_weights(ctx, None)
-    else:
-        n = len(pkv_get_split_weights(ctx))
-        if len(weights) != n:
-            raise ValueError(f"pkv_set_split_weights: expected {n} weights, got {len(weights)}")
-        arr = (C.c_int * n)(*[int(x) for x in weights])
-        st = lib.pkv_set_split_weights(ctx, arr)
-    return _done(st, "pkv_set_split_weights", check)
 
 
 class Pages:

@@ -211,105 +211,6 @@ def test_a_later_context_with_a_smaller_batch_leaves_an_earlier_one_usable(pkv):
         assert finite and mx <= _gpu.TOL_BF16["max"] and mean <= _gpu.TOL_BF16["mean"], (mx, mean)
 
 
-@pytest.mark.parametrize("case_name", ["llama8b", "hetero70b", "fp8", "spec4"])
-def test_weighted_split_matches_oracle(pkv, case_name):
-    """Per-warp weights of the split (seeded, spread over the whole allowed
-    range [512, 2048]) move every range boundary of these batches (each has
-    at least 8 tiles per warp); the output must still match the oracle, two
-    calls must agree bit for bit, and forced worker counts (which use equal
-    ranges) still match."""
-    w = workloads.make(case_name, device="cuda")
-    h = host_inputs(w)
-    dv = _gpu.to_device(w)
-    w.k_pool = w.v_pool = None
-    ctx = _gpu.make_ctx(pkv, w)
-    tok = w.q_len > 1
-    outs = []
-    try:
-        n = len(pkv.pkv_get_split_weights(ctx))
-        weights = np.random.default_rng(7).integers(512, 2048, size=n, endpoint=True)
-        pkv.pkv_set_split_weights(ctx, weights)
-        assert pkv.pkv_get_split_weights(ctx) == [int(x) for x in weights]
-        (pkv.pkv_rope_append_tokens if tok else pkv.pkv_rope_append)(
-            ctx, dv["q"], dv["k_new"], dv["v_new"], dv["k_pool"], dv["v_pool"], dv["k_scale"], dv["v_scale"],
-            dv["block_tables"], dv["seq_lens"])
-        for workers in (0, 0, 7, 1000):
-            pkv.pkv_set_workers(ctx, workers)
-            out = torch.empty(dv["q"].shape, dtype=torch.bfloat16, device="cuda")
-            (pkv.pkv_decode_attn_tokens if tok else pkv.pkv_decode_attn)(
-                ctx, dv["q"], dv["k_pool"], dv["v_pool"], dv["k_scale"], dv["v_scale"], dv["block_tables"],
-                dv["seq_lens"], out)
-            outs.append(out)
-        assert pkv.pkv_check_device_error(ctx)[0] == pkv.PKV_OK
-    finally:
-        pkv.pkv_destroy(ctx)
-    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))   # deterministic
-    cfg = oracle_cfg(w)
-    if tok:
-        assert oracle.rope_append_tokens(cfg, h["q"], h["k_new"], h["v_new"], h["k_pool"], h["v_pool"],
-                                         h["k_scale"], h["v_scale"], h["block_tables"], h["seq_lens"]) == 0
-    else:
-        assert oracle.rope_append(cfg, h["q"], h["k_new"], h["v_new"], h["k_pool"], h["v_pool"], h["k_scale"],
-                                  h["v_scale"], h["block_tables"], h["seq_lens"]) == 0
-    ref, st = oracle_attn_threaded(w, h)
-    assert st == 0
-    for o in outs:
-        mx, mean, finite = _gpu.errors(o, ref)
-        assert finite and mx <= _gpu.tol(w)["max"] and mean <= _gpu.tol(w)["mean"], (mx, mean)
-
-
-@pytest.mark.parametrize("name", ["llama8b", "fp8"])
-def test_calibrated_weights_are_bounded_and_keep_parity(pkv, name):
-    w = workloads.make(name, device="cuda")
-    _, ref, _ = oracle_step(w)
-    dv = _gpu.to_device(w)
-    ctx = _gpu.make_ctx(pkv, w)
-    try:
-        pkv.pkv_rope_append(ctx, dv["q"], dv["k_new"], dv["v_new"], dv["k_pool"], dv["v_pool"], dv["k_scale"],
-                            dv["v_scale"], dv["block_tables"], dv["seq_lens"])
-        out0 = torch.empty(w.batch, w.Hq, w.d, dtype=torch.bfloat16, device="cuda")
-        pkv.pkv_calibrate(ctx, dv["q"], dv["k_pool"], dv["v_pool"], dv["k_scale"], dv["v_scale"],
-                          dv["block_tables"], dv["seq_lens"], out0, rounds=4)
-        weights = pkv.pkv_get_split_weights(ctx)
-        assert all(512 <= x <= 2048 for x in weights)
-        assert abs(np.mean(weights) - 1024) <= 16
-        out, out2 = torch.empty_like(out0), torch.empty_like(out0)
-        for o in (out, out2):
-            pkv.pkv_decode_attn(ctx, dv["q"], dv["k_pool"], dv["v_pool"], dv["k_scale"], dv["v_scale"],
-                                dv["block_tables"], dv["seq_lens"], o)
-        assert pkv.pkv_check_device_error(ctx)[0] == pkv.PKV_OK
-    finally:
-        pkv.pkv_destroy(ctx)
-    assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
-    for o in (out0, out):
-        mx, mean, finite = _gpu.errors(o, ref)
-        assert finite and mx <= _gpu.tol(w)["max"] and mean <= _gpu.tol(w)["mean"], (mx, mean)
-
-
-def test_split_weight_rejections(pkv):
-    w = _small(SMALL[0])
-    dv = _gpu.to_device(w)
-    ctx = _gpu.make_ctx(pkv, w)
-    out = torch.empty(w.batch, w.Hq, w.d, dtype=torch.bfloat16, device="cuda")
-    try:
-        n = len(pkv.pkv_get_split_weights(ctx))
-        assert pkv.pkv_get_split_weights(ctx) == [1024] * n
-        assert pkv.pkv_set_split_weights(ctx, [1024] * (n - 1) + [511], check=False) == pkv.PKV_ERR_INVALID_ARG
-        assert pkv.pkv_set_split_weights(ctx, [2049] + [1024] * (n - 1), check=False) == pkv.PKV_ERR_INVALID_ARG
-        with pytest.raises(ValueError):
-            pkv.pkv_set_split_weights(ctx, [1024] * (n + 1))
-        args = (dv["q"], dv["k_pool"], dv["v_pool"], None, None, dv["block_tables"], dv["seq_lens"], out)
-        assert pkv.pkv_calibrate(ctx, *args, rounds=1, check=False) == pkv.PKV_ERR_INVALID_ARG
-        # a batch too small to give every warp work cannot be measured: equal ranges stay
-        assert pkv.pkv_calibrate(ctx, *args, rounds=3, check=False) == pkv.PKV_ERR_UNSUPPORTED
-        assert pkv.pkv_get_split_weights(ctx) == [1024] * n
-        assert pkv.pkv_set_split_weights(ctx, [700] * n) == pkv.PKV_OK
-        assert pkv.pkv_set_split_weights(ctx, None) == pkv.PKV_OK
-        assert pkv.pkv_get_split_weights(ctx) == [1024] * n
-    finally:
-        pkv.pkv_destroy(ctx)
-
-
 def test_combine_merges_more_contributors_than_one_staging_block(pkv):
     # one (request, kv head) pair of 270,001 tokens over 128 warps: 16,876
     # tiles, 131 per warp range, a tail of 8 chunks per range -> 1,152 units
