@@ -246,5 +246,30 @@ __device__ __forceinline__ uint8_t e4m3_satfinite(float x)
     return (uint8_t)__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3);
 }
 
+// ---- rotary embedding arithmetic (every kernel that rotates uses these) -----
+
+// sin and cos of the angle pos * theta_i: the product rounded once in fp64,
+// reduced to [-pi, pi] with a two-part 2*pi (Cody & Waite; the high part is
+// the double nearest 2*pi), then sincos.
+__device__ __forceinline__ void rope_sincos(double phi, double* s, double* c)
+{
+    constexpr double kTwoPiHi = 6.283185307179586;
+    constexpr double kTwoPiLo = 2.4492935982947064e-16;
+    constexpr double kInvTwoPi = 0.15915494309189535;
+    const double k = rint(phi * kInvTwoPi);
+    double r = fma(-k, kTwoPiHi, phi);
+    r = fma(-k, kTwoPiLo, r);
+    sincos(r, s, c);
+}
+
+// One rotation pair (x_i, x_{i+d/2}) = (a, b) by the angle of cosine c and
+// sine s: (a c - b s, b c + a s) in fp64, every product and sum rounded on
+// its own (no fused multiply-add).
+__device__ __forceinline__ void rope_rotate(double a, double b, double c, double s, double* ya, double* yb)
+{
+    *ya = __dsub_rn(__dmul_rn(a, c), __dmul_rn(b, s));
+    *yb = __dadd_rn(__dmul_rn(b, c), __dmul_rn(a, s));
+}
+
 }  // namespace dev
 }  // namespace pkv

@@ -64,10 +64,6 @@ constexpr int kQkvSmemLimit = 1024 + 220 * 1024;
 constexpr int kQkvRecvRow = 80;                // bytes per row of received partials (64 + 16: no bank conflicts)
 constexpr uint64_t kQkvWaitNs = 500ull * 1000ull * 1000ull;
 
-constexpr double kTwoPiHi = 6.283185307179586;
-constexpr double kTwoPiLo = 2.4492935982947064e-16;
-constexpr double kInvTwoPi = 0.15915494309189535;
-
 // Shared-memory matrix descriptor of a K-major tile with 128-byte rows and
 // the 128-byte swizzle (the layout the TMA loads write): start address >> 4,
 // leading byte offset 1 (unused by this layout), stride byte offset 1024 B
@@ -141,14 +137,6 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint32_t a, uint32_
 {
     asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
                  : "memory");
-}
-
-__device__ __forceinline__ void sincos_reduced(double phi, double* s, double* c)
-{
-    const double k = rint(phi * kInvTwoPi);
-    double r = fma(-k, kTwoPiHi, phi);
-    r = fma(-k, kTwoPiLo, r);
-    sincos(r, s, c);
 }
 
 // Bytes of one ring stage's x area: at least the part of the 128-row A
@@ -305,7 +293,7 @@ qkv_rope_append_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_con
                 const int r = it / np, i = it - r * np;
                 const int L = s_L[r];
                 double sn = 0.0, cs = 1.0;
-                if (L >= 0) sincos_reduced((double)L * s_theta[i], &sn, &cs);
+                if (L >= 0) dev::rope_sincos((double)L * s_theta[i], &sn, &cs);
                 tab[r * TP + i] = make_double2(cs, sn);
             }
         }
@@ -399,8 +387,8 @@ qkv_rope_append_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_con
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
                 const double2 cssn = tr[c];
-                const double ylo = __dsub_rn(__dmul_rn(lo[c], cssn.x), __dmul_rn(hi[c], cssn.y));
-                const double yhi = __dadd_rn(__dmul_rn(hi[c], cssn.x), __dmul_rn(lo[c], cssn.y));
+                double ylo, yhi;
+                dev::rope_rotate(lo[c], hi[c], cssn.x, cssn.y, &ylo, &yhi);
                 lo[c] = ylo;
                 hi[c] = yhi;
             }

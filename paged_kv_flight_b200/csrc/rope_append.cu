@@ -29,24 +29,12 @@
 // one final rounding to the storage type.
 #include "pkv_internal.h"
 #include "pkv_device.cuh"
+#include "rope_common.cuh"
 
 namespace pkv {
 namespace {
 
 constexpr int kRopeThreads = 128;
-
-// 2*pi = kTwoPiHi + kTwoPiLo; kTwoPiHi is the double nearest 2*pi.
-constexpr double kTwoPiHi = 6.283185307179586;
-constexpr double kTwoPiLo = 2.4492935982947064e-16;
-constexpr double kInvTwoPi = 0.15915494309189535;
-
-__device__ __forceinline__ void sincos_reduced(double phi, double* s, double* c)
-{
-    const double k = rint(phi * kInvTwoPi);
-    double r = fma(-k, kTwoPiHi, phi);
-    r = fma(-k, kTwoPiLo, r);
-    sincos(r, s, c);
-}
 
 // bf16 pools: nine CTAs per SM (at most 56 registers) keep the largest
 // batches' grids to one wave (256 requests x 5 CTAs for 64 + 8 heads of
@@ -84,22 +72,10 @@ __global__ void __launch_bounds__(kRopeThreads, FP8 ? 1 : 9) rope_append_kernel(
     const bool active = it < rows * PIECES;
     const int r = it / PIECES;
     const int i0 = (it % PIECES) * 8;
-    const bool is_q = r < p.Hq;
-    const int kvh = r - p.Hq;
 
     // loads that do not depend on the position go out first
-    uint4 xa = make_uint4(0, 0, 0, 0), xb = xa, va = xa, vb = xa;
-    if (active) {
-        const __nv_bfloat16* src = is_q ? p.q + ((size_t)bt * p.Hq + r) * D
-                                        : p.k_new + ((size_t)bt * p.Hkv + kvh) * D;
-        xa = *reinterpret_cast<const uint4*>(src + i0);          // x_i
-        xb = *reinterpret_cast<const uint4*>(src + i0 + HALF);   // x_{i+d/2}
-        if (!is_q) {
-            const __nv_bfloat16* vsrc = p.v_new + ((size_t)bt * p.Hkv + kvh) * D;
-            va = *reinterpret_cast<const uint4*>(vsrc + i0);
-            vb = *reinterpret_cast<const uint4*>(vsrc + i0 + HALF);
-        }
-    }
+    rope::Item item{};
+    if (active) item = rope::load_item<D>(p.q, p.k_new, p.v_new, p.Hq, p.Hkv, bt, r, i0);
 
     const int L0 = p.seq_lens[b];
     const long long Lt = (long long)L0 + t;  // position of this new token
@@ -114,7 +90,6 @@ __global__ void __launch_bounds__(kRopeThreads, FP8 ? 1 : 9) rope_append_kernel(
         if (threadIdx.x == 0 && blockIdx.y == 0) atomicOr(p.err, kErrPage);
         return;
     }
-    const int slot = L % p.P;
     if (blockIdx.y == 0 && t == 0 && p.prefetch_tables) {
         // the attention that follows walks this request's block-table row:
         // bring it into L2 now (one 128-byte line per thread)
@@ -127,72 +102,14 @@ __global__ void __launch_bounds__(kRopeThreads, FP8 ? 1 : 9) rope_append_kernel(
     for (int i = threadIdx.x; i < HALF; i += blockDim.x) {
         const double theta = p.theta[i];    // rope_base^(-2i/d), computed once per context
         double s, c;
-        sincos_reduced((double)L * theta, &s, &c);
+        dev::rope_sincos((double)L * theta, &s, &c);
         s_cos[i] = c;
         s_sin[i] = s;
     }
     __syncthreads();
     if (!active) return;
-
-    const uint32_t wa[4] = {xa.x, xa.y, xa.z, xa.w};
-    const uint32_t wb[4] = {xb.x, xb.y, xb.z, xb.w};
-    double ya[8], yb[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        const double a = (double)((k & 1) ? dev::bf16_hi(wa[k >> 1]) : dev::bf16_lo(wa[k >> 1]));
-        const double bb = (double)((k & 1) ? dev::bf16_hi(wb[k >> 1]) : dev::bf16_lo(wb[k >> 1]));
-        const double c = s_cos[i0 + k], s = s_sin[i0 + k];
-        // separate roundings, no fused multiply-add
-        ya[k] = __dsub_rn(__dmul_rn(a, c), __dmul_rn(bb, s));
-        yb[k] = __dadd_rn(__dmul_rn(bb, c), __dmul_rn(a, s));
-    }
-
-    const size_t prow = ((size_t)page * p.Hkv + kvh) * p.P + slot;   // pool row (k rows only)
-    if (is_q || !FP8) {
-        uint32_t oa[4], ob[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            oa[k] = (uint32_t)__bfloat16_as_ushort(dev::bf16_from_f64(ya[2 * k])) |
-                    ((uint32_t)__bfloat16_as_ushort(dev::bf16_from_f64(ya[2 * k + 1])) << 16);
-            ob[k] = (uint32_t)__bfloat16_as_ushort(dev::bf16_from_f64(yb[2 * k])) |
-                    ((uint32_t)__bfloat16_as_ushort(dev::bf16_from_f64(yb[2 * k + 1])) << 16);
-        }
-        __nv_bfloat16* dst = is_q ? p.q + ((size_t)bt * p.Hq + r) * D
-                                  : reinterpret_cast<__nv_bfloat16*>(p.k_pool) + prow * D;
-        *reinterpret_cast<uint4*>(dst + i0) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
-        *reinterpret_cast<uint4*>(dst + i0 + HALF) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
-    }
-    if (is_q) return;
-
-    if (!FP8) {
-        __nv_bfloat16* vdst = reinterpret_cast<__nv_bfloat16*>(p.v_pool) + prow * D;
-        *reinterpret_cast<uint4*>(vdst + i0) = va;
-        *reinterpret_cast<uint4*>(vdst + i0 + HALF) = vb;
-    } else {
-        const size_t si = (size_t)page * p.Hkv + kvh;
-        const double sk = (double)p.k_scale[si];
-        const float sv = p.v_scale[si];
-        const uint32_t vwa[4] = {va.x, va.y, va.z, va.w};
-        const uint32_t vwb[4] = {vb.x, vb.y, vb.z, vb.w};
-        uint8_t ka[8], kb[8], qa8[8], qb8[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            // k: fp64 quotient rounded once to fp32, then E4M3 RNE satfinite
-            ka[k] = dev::e4m3_satfinite(__double2float_rn(__ddiv_rn(ya[k], sk)));
-            kb[k] = dev::e4m3_satfinite(__double2float_rn(__ddiv_rn(yb[k], sk)));
-            // v: exact bf16 value, IEEE fp32 quotient
-            const float a = (k & 1) ? dev::bf16_hi(vwa[k >> 1]) : dev::bf16_lo(vwa[k >> 1]);
-            const float bb = (k & 1) ? dev::bf16_hi(vwb[k >> 1]) : dev::bf16_lo(vwb[k >> 1]);
-            qa8[k] = dev::e4m3_satfinite(__fdiv_rn(a, sv));
-            qb8[k] = dev::e4m3_satfinite(__fdiv_rn(bb, sv));
-        }
-        uint8_t* kdst = reinterpret_cast<uint8_t*>(p.k_pool) + prow * D;
-        uint8_t* vdst = reinterpret_cast<uint8_t*>(p.v_pool) + prow * D;
-        *reinterpret_cast<uint2*>(kdst + i0) = *reinterpret_cast<const uint2*>(ka);
-        *reinterpret_cast<uint2*>(kdst + i0 + HALF) = *reinterpret_cast<const uint2*>(kb);
-        *reinterpret_cast<uint2*>(vdst + i0) = *reinterpret_cast<const uint2*>(qa8);
-        *reinterpret_cast<uint2*>(vdst + i0 + HALF) = *reinterpret_cast<const uint2*>(qb8);
-    }
+    rope::store_item<D, FP8>(item, p.q, p.k_pool, p.v_pool, p.k_scale, p.v_scale, p.Hq, p.Hkv, p.P, bt, r, i0,
+                             page, L % p.P, s_cos, s_sin);
 }
 
 }  // namespace

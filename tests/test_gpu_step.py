@@ -6,6 +6,9 @@ whole pools.  The four full-size workloads run in the benchmark's launch
 configuration and are compared the same way: the oracle recomputes the whole
 batch from the generator's original inputs.
 
+Both forms of the one-token step are checked: pkv_rope_append followed by
+pkv_decode_attn, and pkv_decode_step (bit-identical to the two calls).
+
 Bars: appended V bit-exact, appended K (and rotated q) within 1 bf16 ulp /
 1 E4M3 code step, every other pool byte untouched; attention max abs error
 <= 1e-2 and mean <= 1e-3 for bf16 KV, <= 6e-2 / 6e-3 for E4M3 KV."""
@@ -66,15 +69,16 @@ def _check_append(w, h_oracle, dv):
             assert np.abs(bf16_ordinal(gk[diff]) - bf16_ordinal(h_oracle["k_pool"][diff])).max() <= 1
 
 
+@pytest.mark.parametrize("fused", [False, True], ids=["two_calls", "decode_step"])
 @pytest.mark.parametrize("case", SMALL + [("tiny",)], ids=lambda c: c[0])
-def test_small_step_matches_oracle(pkv, case):
+def test_small_step_matches_oracle(pkv, case, fused):
     w = workloads.make("tiny") if case[0] == "tiny" else _small(case)
     h, ref, st = oracle_step(w)
     assert st == 0
     dv = _gpu.to_device(w)
     ctx = _gpu.make_ctx(pkv, w)
     try:
-        out = _gpu.gpu_step(pkv, ctx, dv)
+        out = _gpu.gpu_step(pkv, ctx, dv, fused=fused)
         assert pkv.pkv_check_device_error(ctx)[0] == pkv.PKV_OK
     finally:
         pkv.pkv_destroy(ctx)
@@ -91,14 +95,16 @@ def test_full_size_whole_batch_matches_oracle(pkv, name):
     """The full-size workloads in the benchmark's launch configuration: the
     oracle recomputes the whole step (append over the whole pools, attention
     of every request and kv head) from the generator's original inputs, and
-    every output element, the rotated q and both whole pools are compared."""
+    every output element, the rotated q and both whole pools are compared.
+    The step is pkv_decode_step, as the benchmark times it (the two-call form
+    is held to the same bits by test_decode_step_equals_the_two_calls)."""
     w = workloads.make(name, device="cuda")
     h = host_inputs(w)                                   # original inputs, before the step
     dv = _gpu.to_device(w)
     w.k_pool = w.v_pool = None                           # the device keeps one copy of the pools
     ctx = _gpu.make_ctx(pkv, w)
     try:
-        out = _gpu.gpu_step(pkv, ctx, dv)
+        out = _gpu.gpu_step(pkv, ctx, dv, fused=True)
         assert pkv.pkv_check_device_error(ctx)[0] == pkv.PKV_OK
     finally:
         pkv.pkv_destroy(ctx)
@@ -117,10 +123,10 @@ def test_full_size_whole_batch_matches_oracle(pkv, name):
 @pytest.mark.parametrize("case", SMALL + [("llama8b",), ("hetero70b",), ("fp8",), ("longctx",)],
                          ids=lambda c: c[0])
 def test_decode_step_equals_the_two_calls(pkv, case):
-    """pkv_decode_step runs the same kernels as pkv_rope_append followed by
-    pkv_decode_attn, the attention launched as a programmatic dependent of
-    the append: q, both pools and the output must be bit-identical to the two
-    calls' on the same inputs, small cases and full-size workloads alike."""
+    """pkv_decode_step (the attention launched as a programmatic dependent of
+    the RoPE + append kernel): q, both pools and the output must be
+    bit-identical to those of pkv_rope_append followed by pkv_decode_attn on
+    the same inputs, small cases and full-size workloads alike."""
     w = workloads.make(case[0], device="cuda") if len(case) == 1 else _small(case)
     results = []
     for fused in (False, True):
@@ -185,6 +191,37 @@ def test_split_count_invariance(pkv, case_name):
     for o in outs:
         mx, mean, _ = _gpu.errors(o, ref)
         assert mx <= _gpu.tol(w)["max"] and mean <= _gpu.tol(w)["mean"]
+
+
+@pytest.mark.parametrize("case_name", ["g4_d128_p32_bf16", "g2_d64_p32_bf16", "g4_d128_p32_fp8",
+                                       "g4_d64_p32_fp8", "llama8b"])
+def test_decode_step_under_every_split_equals_the_two_calls(pkv, case_name):
+    """pkv_decode_step under static and dynamic splits of every size (fewer
+    warp workers than warps included) against pkv_rope_append +
+    pkv_decode_attn under the same split, on fresh inputs each time:
+    bit-identical q, pools and output."""
+    if case_name == "llama8b":
+        w = workloads.make("llama8b", device="cuda")
+    else:
+        w = _small(next(c for c in SMALL if c[0] == case_name))
+    ctx = _gpu.make_ctx(pkv, w)
+    try:
+        for tail, workers in [(0, 1), (0, 2), (0, 7), (0, 100), (0, 0), (1, 2), (8, 1), (8, 7), (8, 100), (8, 0)]:
+            pkv.pkv_set_tail_chunks(ctx, tail)
+            pkv.pkv_set_workers(ctx, workers)
+            two, one = _gpu.to_device(w), _gpu.to_device(w)
+            o2 = _gpu.gpu_step(pkv, ctx, two)
+            o1 = _gpu.gpu_step(pkv, ctx, one, fused=True)
+            assert torch.equal(o1.view(torch.int16), o2.view(torch.int16)), (tail, workers)
+            for k in ("q", "k_pool", "v_pool"):
+                a, b = two[k], one[k]
+                if a.dtype == torch.bfloat16:
+                    a, b = a.view(torch.int16), b.view(torch.int16)
+                assert torch.equal(a, b), (k, tail, workers)
+            del two, one
+        assert pkv.pkv_check_device_error(ctx)[0] == pkv.PKV_OK
+    finally:
+        pkv.pkv_destroy(ctx)
 
 
 def test_a_later_context_with_a_smaller_batch_leaves_an_earlier_one_usable(pkv):
@@ -361,8 +398,9 @@ def test_host_side_rejections(pkv):
         pkv.pkv_destroy(ctx)
 
 
+@pytest.mark.parametrize("fused", [False, True], ids=["two_calls", "decode_step"])
 @pytest.mark.parametrize("fp8", [False, True])
-def test_device_range_errors_are_reported_not_trapped(pkv, fp8):
+def test_device_range_errors_are_reported_not_trapped(pkv, fp8, fused):
     case = SMALL[5] if fp8 else SMALL[0]
     w = _small(case, seed=5)
     h, ref, _ = oracle_step(w)
@@ -373,7 +411,7 @@ def test_device_range_errors_are_reported_not_trapped(pkv, fp8):
     dv["seq_lens"][bad_len_req] = w.bt_stride * w.P
     ctx = _gpu.make_ctx(pkv, w)
     try:
-        out = _gpu.gpu_step(pkv, ctx, dv)
+        out = _gpu.gpu_step(pkv, ctx, dv, fused=fused)
         st, bits = pkv.pkv_check_device_error(ctx)
         assert st == pkv.PKV_ERR_DEVICE_BOUNDS and bits & 1 and bits & 2
         assert pkv.pkv_check_device_error(ctx) == (pkv.PKV_OK, 0)    # cleared after reading
@@ -384,7 +422,7 @@ def test_device_range_errors_are_reported_not_trapped(pkv, fp8):
         assert finite and mx <= t["max"] and mean <= t["mean"]
         # the context still works afterwards
         dv2 = _gpu.to_device(w)
-        out2 = _gpu.gpu_step(pkv, ctx, dv2)
+        out2 = _gpu.gpu_step(pkv, ctx, dv2, fused=fused)
         assert pkv.pkv_check_device_error(ctx)[0] == pkv.PKV_OK
         mx, mean, finite = _gpu.errors(out2, ref)
         assert finite and mx <= t["max"]
