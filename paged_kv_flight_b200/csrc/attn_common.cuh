@@ -106,6 +106,45 @@ __device__ __forceinline__ Split make_split(long long T, int W, int max_chunks)
     return sp;
 }
 
+// Warp workers of the split of T tiles when the grid has `grid_warps`
+// warps: all of them, at most `workers` when that is set, else one per
+// kMinTilesPerWorker tiles; at least one and at most T.  The attention and
+// the combine that derives the split itself both use this.
+__device__ __forceinline__ int split_workers(long long T, long long grid_warps, int workers)
+{
+    long long Wl = grid_warps;
+    if (workers > 0) Wl = min(Wl, (long long)workers);
+    else Wl = min(Wl, (T + kMinTilesPerWorker - 1) / kMinTilesPerWorker);
+    return (int)max(1LL, min(Wl, max(T, 1LL)));
+}
+
+// One warp: request b's tile count, the tiles of the requests before it and
+// of all requests, from seq_lens with the attention's rule (ceil((L + 1) /
+// tile) tiles, none for a length out of range).  seq_lens is read-only in a
+// step, so this may run before the wait for the attention grid.
+__device__ __forceinline__ void warp_request_span(const AttnParams& p, int b, int lane, int& before, int& mine,
+                                                  int& all)
+{
+    const long long cap = (long long)p.bt_stride * p.P;
+    int bf = 0, mn = 0, al = 0;
+    for (int c = lane; c < p.batch; c += 32) {
+        const int L = __ldg(&p.seq_lens[c]);
+        const int n = (L >= 0 && (long long)L < cap) ? (L + p.tile) / p.tile : 0;
+        al += n;
+        if (c < b) bf += n;
+        if (c == b) mn = n;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        bf += __shfl_xor_sync(kFull, bf, o);
+        mn += __shfl_xor_sync(kFull, mn, o);
+        al += __shfl_xor_sync(kFull, al, o);
+    }
+    before = bf;
+    mine = mn;
+    all = al;
+}
+
 // Largest b with prefix[b] * Hkv <= x, for 0 <= x < prefix[B] * Hkv.
 __device__ __forceinline__ int seek_request(const int* prefix, int B, int Hkv, long long x)
 {

@@ -55,19 +55,34 @@ __global__ void __launch_bounds__(kCombineThreads, 2) combine_kernel(const AttnP
     float* const s_dyn = reinterpret_cast<float*>(s_dyn4);
     __shared__ float s_m[MAXR], s_l[MAXR];
 
-    if (blockIdx.x == 0 && threadIdx.x == 0) *p.claim = 0;   // the attention launch has ended
     const int pair = blockIdx.x;
     const int b = pair / p.Hkv, kvh = pair - b * p.Hkv;
-    const int W = __ldg(&p.meta[0]);
-    const long long T = (long long)(unsigned)__ldg(&p.meta[1]) | ((long long)__ldg(&p.meta[2]) << 32);
-    const int B = p.vmap ? min(__ldg(p.vcount), p.batch) : p.batch;   // requests, or virtual requests
-    if (T == 0 || b >= B) return;
-    const int* prefix = p.meta + 4;
-    const int nt = __ldg(&prefix[b + 1]) - __ldg(&prefix[b]);
-    if (nt == 0) return;
+    int pb, nt, W, K;
+    long long T;
+    if (p.own_split) {
+        // one new token per request: the attention's split from seq_lens
+        // (every warp alike), then wait for that grid
+        int all;
+        warp_request_span(p, b, threadIdx.x & 31, pb, nt, all);
+        T = (long long)all * p.Hkv;
+        W = split_workers(T, p.grid_warps, p.workers);
+        K = make_split(max(T, 1LL), W, p.tail_chunks).K;
+        grid_dependency_wait();
+    }
+    if (blockIdx.x == 0 && threadIdx.x == 0) *p.claim = 0;   // the attention launch has ended
+    if (!p.own_split) {
+        W = __ldg(&p.meta[0]);
+        T = (long long)(unsigned)__ldg(&p.meta[1]) | ((long long)__ldg(&p.meta[2]) << 32);
+        K = __ldg(&p.meta[3]);
+        const int B = p.vmap ? min(__ldg(p.vcount), p.batch) : p.batch;   // requests, or virtual requests
+        if (T == 0 || b >= B) return;
+        pb = __ldg(&p.meta[4 + b]);
+        nt = __ldg(&p.meta[4 + b + 1]) - pb;
+    }
+    if (T == 0 || nt == 0) return;
     Split sp = make_split(T, W, 0);
-    sp.K = __ldg(&p.meta[3]);   // as the attention launch chose it
-    const long long ts = (long long)__ldg(&prefix[b]) * p.Hkv + (long long)kvh * nt;
+    sp.K = K;   // as the attention launch chose it
+    const long long ts = (long long)pb * p.Hkv + (long long)kvh * nt;
     const int U0 = sp.unit_of(ts), U1 = sp.unit_of(ts + nt - 1);
     if (U0 == U1) return;
     const int G = p.G, R = G * p.q_len;            // partial rows: new token t, head h at row t G + h
@@ -205,131 +220,118 @@ __global__ void __launch_bounds__(kCombineThreads, 2) combine_kernel(const AttnP
 
 // The same merge with one warp per pair, for batches with many pairs: all
 // pairs then fit in about one wave and no shared memory or CTA barrier is
-// needed.  Lanes take contributors 32 at a time for m* and l* (online, then a
-// butterfly over the lanes) and for the weights; the weighted sum walks the
-// contributors with every lane on its own 16-byte pieces of the G x D
-// values, a piece of D = 128 belonging to head t for the t-th piece of the
-// lane and a piece of D = 64 to head 2t or 2t + 1 by lane half.
+// needed.  One pass over the contributors with a running log-sum-exp per
+// head (the online form of the merge: o* = sum_i 2^(m_i - m*) o_i / l*): lane
+// piece t is float4 f = lane + 32 t of the G x D values, of head f / (d/4),
+// and each contributor's (m, l) and values are read together.  With at most
+// 4 pieces a lane (GMAX d <= 512) the next contributor's loads are in flight
+// while one merges; with 8 the registers hold one contributor at a time.
 constexpr int kCombineWarpThreads = 256;
 
-template <int D>
+template <int D, int GMAX>
 __global__ void __launch_bounds__(kCombineWarpThreads, 2) combine_warp_kernel(const AttnParams p)
 {
-    constexpr unsigned kFullMask = 0xFFFFFFFFu;
-    constexpr int F4 = kMaxGroup * D / 4 / 32;   // 16-byte pieces per lane, at most
+    constexpr int F4 = GMAX * D / 4 / 32;   // 16-byte pieces per lane
+    constexpr bool kAhead = F4 <= 4;
     static_assert(D == 128 || D == 64, "head_dim");
 
-    if (blockIdx.x == 0 && threadIdx.x == 0) *p.claim = 0;   // the attention launch has ended
     const int lane = threadIdx.x & 31;
     const int pair = blockIdx.x * (kCombineWarpThreads / 32) + (threadIdx.x >> 5);
     if (pair >= p.batch * p.Hkv) return;
     const int b = pair / p.Hkv, kvh = pair - b * p.Hkv;
-    const int W = __ldg(&p.meta[0]);
-    const long long T = (long long)(unsigned)__ldg(&p.meta[1]) | ((long long)__ldg(&p.meta[2]) << 32);
-    const int* prefix = p.meta + 4;
-    const int pb = __ldg(&prefix[b]);
-    const int nt = __ldg(&prefix[b + 1]) - pb;
+    int pb, nt, W, K;
+    long long T;
+    if (p.own_split) {
+        // the attention's split from seq_lens, then wait for that grid
+        int all;
+        warp_request_span(p, b, lane, pb, nt, all);
+        T = (long long)all * p.Hkv;
+        W = split_workers(T, p.grid_warps, p.workers);
+        K = make_split(max(T, 1LL), W, p.tail_chunks).K;
+        grid_dependency_wait();
+    } else {
+        W = __ldg(&p.meta[0]);
+        T = (long long)(unsigned)__ldg(&p.meta[1]) | ((long long)__ldg(&p.meta[2]) << 32);
+        K = __ldg(&p.meta[3]);
+        pb = __ldg(&p.meta[4 + b]);
+        nt = __ldg(&p.meta[4 + b + 1]) - pb;
+    }
+    if (blockIdx.x == 0 && threadIdx.x == 0) *p.claim = 0;   // the attention launch has ended
     if (T == 0 || nt == 0) return;
     Split sp = make_split(T, W, 0);
-    sp.K = __ldg(&p.meta[3]);   // as the attention launch chose it
+    sp.K = K;   // as the attention launch chose it
     const long long ts = (long long)pb * p.Hkv + (long long)kvh * nt;
     const int U0 = sp.unit_of(ts), U1 = sp.unit_of(ts + nt - 1);
     if (U0 == U1) return;
     const int k = U1 - U0 + 1, G = p.G, GD4 = G * D / 4;
     const int side0 = sp.ustart(U0) < ts ? 1 : 0;
 
-    // pass 1: m* and l* per head; lane j keeps the m of its first contributor
-    // (j) so that the weights of the first 32 need no second load
-    float M[kMaxGroup], L[kMaxGroup], m_own[kMaxGroup];
-#pragma unroll
-    for (int g = 0; g < kMaxGroup; ++g) {
-        M[g] = -INFINITY;
-        L[g] = 0.f;
-        m_own[g] = -INFINITY;
-    }
-    for (int i = lane; i < k; i += 32) {
-        const int slot = 2 * (U0 + i) + (i == 0 ? side0 : 0);
-#pragma unroll
-        for (int g = 0; g < kMaxGroup; ++g) {
-            if (g < G) {
-                const float2 ml = __ldg(reinterpret_cast<const float2*>(p.part_ml + ((size_t)slot * G + g) * 2));
-                if (i == lane) m_own[g] = ml.x;
-                const float m_new = fmaxf(M[g], ml.x);
-                const float ref = (m_new == -INFINITY) ? 0.f : m_new;
-                L[g] = L[g] * ex2(M[g] - ref) + ml.y * ex2(ml.x - ref);
-                M[g] = m_new;
-            }
-        }
-    }
-#pragma unroll
-    for (int g = 0; g < kMaxGroup; ++g) {
-        if (g < G) {
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const float m2 = __shfl_xor_sync(kFullMask, M[g], o), l2 = __shfl_xor_sync(kFullMask, L[g], o);
-                const float m_new = fmaxf(M[g], m2);
-                const float ref = (m_new == -INFINITY) ? 0.f : m_new;
-                L[g] = L[g] * ex2(M[g] - ref) + l2 * ex2(m2 - ref);
-                M[g] = m_new;
-            }
-            if (M[g] == -INFINITY) M[g] = 0.f;
-        }
-    }
-
-    // pass 2: weighted sum, contributors in batches of 32 (lane j holds the
-    // slot and the weights of contributor i0 + j)
     float4 acc[F4];
+    float Mr[F4], Lr[F4];
 #pragma unroll
-    for (int t = 0; t < F4; ++t) acc[t] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int i0 = 0; i0 < k; i0 += 32) {
-        const int i = i0 + lane;
-        int slot_l = 0;
-        float wl[kMaxGroup];
+    for (int t = 0; t < F4; ++t) {
+        acc[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+        Mr[t] = -INFINITY;
+        Lr[t] = 0.f;
+    }
+    auto load = [&](int i, float4 (&v)[F4], float2 (&ml)[F4]) {
+        const int slot = 2 * (U0 + i) + (i == 0 ? side0 : 0);
+        const float4* src = reinterpret_cast<const float4*>(p.part_o + (size_t)slot * G * D);
 #pragma unroll
-        for (int g = 0; g < kMaxGroup; ++g) wl[g] = 0.f;
-        if (i < k) {
-            slot_l = 2 * (U0 + i) + (i == 0 ? side0 : 0);
-#pragma unroll
-            for (int g = 0; g < kMaxGroup; ++g) {
-                if (g < G) {
-                    const float m = (i0 == 0) ? m_own[g] : __ldg(p.part_ml + ((size_t)slot_l * G + g) * 2);
-                    wl[g] = ex2(m - M[g]) / L[g];
-                }
+        for (int t = 0; t < F4; ++t) {
+            const int f = lane + 32 * t;
+            if (f < GD4) {
+                ml[t] = __ldg(reinterpret_cast<const float2*>(p.part_ml + ((size_t)slot * G + f / (D / 4)) * 2));
+                v[t] = __ldg(src + f);
             }
         }
-        const int n = min(32, k - i0);
-        for (int j = 0; j < n; ++j) {
-            const int slot = __shfl_sync(kFullMask, slot_l, j);
-            const float4* src = reinterpret_cast<const float4*>(p.part_o + (size_t)slot * G * D);
+    };
+    auto merge = [&](const float4 (&v)[F4], const float2 (&ml)[F4]) {
 #pragma unroll
-            for (int t = 0; t < F4; ++t) {
-                float w;
-                if constexpr (D == 128) {
-                    w = __shfl_sync(kFullMask, wl[t], j);
-                } else {
-                    const float wa = __shfl_sync(kFullMask, wl[2 * t], j);
-                    const float wb = __shfl_sync(kFullMask, wl[2 * t + 1], j);
-                    w = lane < 16 ? wa : wb;
-                }
-                const int f = lane + 32 * t;
-                if (f < GD4) {
-                    const float4 v = __ldg(src + f);
-                    acc[t].x += w * v.x;
-                    acc[t].y += w * v.y;
-                    acc[t].z += w * v.z;
-                    acc[t].w += w * v.w;
-                }
+        for (int t = 0; t < F4; ++t) {
+            if (lane + 32 * t < GD4) {
+                const float m_new = fmaxf(Mr[t], ml[t].x);
+                const float ref = (m_new == -INFINITY) ? 0.f : m_new;
+                const float a = ex2(Mr[t] - ref), w = ex2(ml[t].x - ref);
+                acc[t].x = acc[t].x * a + w * v[t].x;
+                acc[t].y = acc[t].y * a + w * v[t].y;
+                acc[t].z = acc[t].z * a + w * v[t].z;
+                acc[t].w = acc[t].w * a + w * v[t].w;
+                Lr[t] = Lr[t] * a + w * ml[t].y;
+                Mr[t] = m_new;
             }
+        }
+    };
+    if constexpr (kAhead) {
+        float4 va[F4], vb[F4];
+        float2 ma[F4], mb[F4];
+        load(0, va, ma);
+        for (int i = 0; i < k; i += 2) {
+            if (i + 1 < k) load(i + 1, vb, mb);
+            merge(va, ma);
+            if (i + 1 < k) {
+                if (i + 2 < k) load(i + 2, va, ma);
+                merge(vb, mb);
+            }
+        }
+    } else {
+        float4 va[F4];
+        float2 ma[F4];
+        for (int i = 0; i < k; ++i) {
+            load(i, va, ma);
+            merge(va, ma);
         }
     }
     uint2* const dst = reinterpret_cast<uint2*>(p.out + ((size_t)b * p.Hq + (size_t)kvh * G) * D);
 #pragma unroll
     for (int t = 0; t < F4; ++t) {
         const int f = lane + 32 * t;
-        if (f < GD4) dst[f] = make_uint2(pack_bf16(acc[t].x, acc[t].y), pack_bf16(acc[t].z, acc[t].w));
+        if (f < GD4) {
+            const float inv = 1.f / Lr[t];
+            dst[f] = make_uint2(pack_bf16(acc[t].x * inv, acc[t].y * inv), pack_bf16(acc[t].z * inv, acc[t].w * inv));
+        }
     }
 }
-
 
 template <int D>
 cudaError_t prepare_d()
@@ -341,22 +343,38 @@ cudaError_t prepare_d()
                                 (int)combine_smem_bytes(kCombineBlock, 16, D));
 }
 
+template <typename Kern>
+cudaError_t launch_one(Kern kern, int grid, int threads, size_t smem, cudaStream_t stream, bool pdl,
+                       const AttnParams& p)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
 template <int D>
-cudaError_t launch_d(const AttnParams& p, int max_units_n, int ctas, cudaStream_t stream)
+cudaError_t launch_d(const AttnParams& p, int max_units_n, int ctas, cudaStream_t stream, bool pdl)
 {
     const int pairs = p.batch * p.Hkv, R = p.G * p.q_len;
     // a warp per pair when there are at least two pairs per attention CTA
     // (many pairs, each with few contributors) and at most 8 rows; else a
     // CTA per pair
     if (p.q_len == 1 && pairs >= 2 * ctas) {
-        const int wpc = kCombineWarpThreads / 32;
-        combine_warp_kernel<D><<<(pairs + wpc - 1) / wpc, kCombineWarpThreads, 0, stream>>>(p);
-    } else {
-        const size_t smem = combine_smem_bytes(max_units_n, R, D);
-        if (R <= 8) combine_kernel<D, 8><<<pairs, kCombineThreads, smem, stream>>>(p);
-        else combine_kernel<D, 16><<<pairs, kCombineThreads, smem, stream>>>(p);
+        const int wpc = kCombineWarpThreads / 32, grid = (pairs + wpc - 1) / wpc;
+        if (p.G <= 4) return launch_one(combine_warp_kernel<D, 4>, grid, kCombineWarpThreads, 0, stream, pdl, p);
+        return launch_one(combine_warp_kernel<D, 8>, grid, kCombineWarpThreads, 0, stream, pdl, p);
     }
-    return cudaGetLastError();
+    const size_t smem = combine_smem_bytes(max_units_n, R, D);
+    if (R <= 8) return launch_one(combine_kernel<D, 8>, pairs, kCombineThreads, smem, stream, pdl, p);
+    return launch_one(combine_kernel<D, 16>, pairs, kCombineThreads, smem, stream, pdl, p);
 }
 
 }  // namespace
@@ -366,9 +384,13 @@ cudaError_t combine_prepare(int head_dim)
     return head_dim == 128 ? prepare_d<128>() : prepare_d<64>();
 }
 
-cudaError_t launch_combine(const AttnParams& p, int head_dim, int max_units_n, int ctas, cudaStream_t stream)
+cudaError_t launch_combine(const AttnParams& p, int head_dim, int max_units_n, int ctas, cudaStream_t stream,
+                           bool dependent)
 {
-    return head_dim == 128 ? launch_d<128>(p, max_units_n, ctas, stream) : launch_d<64>(p, max_units_n, ctas, stream);
+    AttnParams q = p;
+    q.own_split = dependent ? 1 : 0;
+    return head_dim == 128 ? launch_d<128>(q, max_units_n, ctas, stream, dependent)
+                           : launch_d<64>(q, max_units_n, ctas, stream, dependent);
 }
 
 }  // namespace pkv

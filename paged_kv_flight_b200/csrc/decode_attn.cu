@@ -108,6 +108,10 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
         prefetch_tensormap(&tmk);
         prefetch_tensormap(&tmv);
     }
+    // the combine launched after this grid as its programmatic dependent may
+    // take SMs as they free up: it derives the split and then waits for this
+    // grid to finish before it reads anything this grid writes
+    grid_launch_dependents();
     __syncthreads();
 
     // ---- 1. tiles per request and their exclusive prefix ----------------------
@@ -154,11 +158,7 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
 
     // ---- 2. split geometry and this warp's head unit ------------------------------
     const long long T = (long long)prefix[B] * Hkv;
-    long long Wl = (long long)gridDim.x * WARPS;
-    if (p.workers > 0) Wl = min(Wl, (long long)p.workers);
-    else Wl = min(Wl, (T + kMinTilesPerWorker - 1) / kMinTilesPerWorker);
-    Wl = max(1LL, min(Wl, max(T, 1LL)));
-    const int W = (int)Wl;
+    const int W = split_workers(T, (long long)gridDim.x * WARPS, p.workers);
     const Split sp = make_split(max(T, 1LL), W, p.tail_chunks);
     if (blockIdx.x == 0) {
         // the combine kernel that follows needs the same split geometry
@@ -713,7 +713,9 @@ cudaError_t launch_decode_attn(const AttnParams& p, const CUtensorMap& tmk, cons
         else e = launch_attn_kernel(decode_attn_kernel<64, true, kAttnWarps, kTile>, grid, block, L.smem_bytes, stream, pdl, tmk, tmv, q);
     }
     if (e != cudaSuccess) return e;
-    return launch_combine(q, head_dim, (int)max_units(L.ctas * kAttnWarps, p.tail_chunks), L.ctas, stream);
+    q.tile = L.tile;
+    q.grid_warps = L.ctas * kAttnWarps;
+    return launch_combine(q, head_dim, (int)max_units(L.ctas * kAttnWarps, p.tail_chunks), L.ctas, stream, true);
 }
 
 }  // namespace pkv

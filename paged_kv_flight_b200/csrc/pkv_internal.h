@@ -104,6 +104,13 @@ struct AttnParams {
     // the varlen plan; null for the other calls
     const int4* vmap = nullptr;
     const int* vcount = nullptr;
+    // the combine of the one-token attention runs as its programmatic
+    // dependent (own_split = 1): it derives the split itself from seq_lens
+    // (tiles of `tile` tokens over `grid_warps` warps, as the attention did)
+    // before it waits for the attention grid, instead of reading meta after
+    int own_split = 0;
+    int tile = 0;
+    int grid_warps = 0;
 };
 
 cudaError_t launch_rope_append(const RopeParams& p, cudaStream_t stream);
@@ -179,7 +186,11 @@ cudaError_t launch_qkv_pack_weight(const __nv_bfloat16* w, __nv_bfloat16* out, i
 // The split combine (combine.cu), run after either attention kernel: sets its
 // shared-memory limits once per head_dim, and launches it for p (max_units_n:
 // units the split may use; ctas: attention CTAs, for the choice of mode).
+// dependent (one new token per request, p.tile and p.grid_warps set): the
+// combine is the attention's programmatic dependent and derives the split
+// from seq_lens while that grid runs; otherwise it reads the split from meta.
 cudaError_t combine_prepare(int head_dim);
-cudaError_t launch_combine(const AttnParams& p, int head_dim, int max_units_n, int ctas, cudaStream_t stream);
+cudaError_t launch_combine(const AttnParams& p, int head_dim, int max_units_n, int ctas, cudaStream_t stream,
+                           bool dependent = false);
 
 }  // namespace pkv
