@@ -252,10 +252,12 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- oracle leg
 
-def _request_pages(w, b, src):
-    """Host copies (oracle form) of request b's pages, block table renumbered."""
+def _request_pages(w, b, src, cached=None):
+    """Host copies (oracle form) of request b's pages, block table renumbered;
+    with `cached`, the request cut to its first `cached` cached tokens (the new
+    tokens then land right after them)."""
     import torch
-    L = int(w.seq_lens[b])
+    L = int(w.seq_lens[b]) if cached is None else min(int(cached), int(w.seq_lens[b]))
     npg = (L + w.q_len + w.P - 1) // w.P
     idx = torch.from_numpy(w.block_tables[b, :npg].astype(np.int64)).to(src["k_pool"].device)
 
@@ -687,8 +689,14 @@ def run_reference(args, name, world=1, time_budget_s=45.0):
     rate = (int(w.seq_lens[0]) + w.q_len) * w.Hkv / max(time.perf_counter() - t0, 1e-6)   # token-heads / s
     budget = int(min(args.ref_budget, rate * time_budget_s / (args.steps + args.warmup)))
     picks = sample_requests(w, budget)
-    views = [_request_pages(w, b, src) for b in picks]
-    by = metric_bytes(w.seq_lens[picks], w.Hq, w.Hkv, w.d, w.P, w.kv_fp8, w.q_len)
+    lens = w.seq_lens[picks].astype(np.int64)
+    if (int(lens[0]) + w.q_len) * w.Hkv > budget:
+        # even the first request is over the step's budget (long contexts):
+        # the sample is that request cut to the cached tokens that fit (at
+        # least one page), so that the warm-up and timed steps stay bounded
+        lens = np.array([max(w.P, min(int(lens[0]), budget // w.Hkv - w.q_len))], np.int64)
+    views = [_request_pages(w, b, src, int(L)) for b, L in zip(picks, lens)]
+    by = metric_bytes(lens, w.Hq, w.Hkv, w.d, w.P, w.kv_fp8, w.q_len)
     for _ in range(args.warmup):
         oracle_step_requests(w, views)
     ts = []
@@ -698,8 +706,9 @@ def run_reference(args, name, world=1, time_budget_s=45.0):
         ts.append(time.perf_counter() - t0)
     sec = statistics.median(ts)
     value = by / sec / 1e9
-    toks = int((w.seq_lens[picks].astype(np.int64) + w.q_len).sum())
-    sample = (f"requests 0..{len(picks) - 1} of {w.batch} ({toks} attended tokens, "
+    toks = int((lens + w.q_len).sum())
+    cut = "" if int(lens[0]) == int(w.seq_lens[picks[0]]) else f", cut to its first {int(lens[0])} cached tokens"
+    sample = (f"requests 0..{len(picks) - 1} of {w.batch}{cut} ({toks} attended tokens, "
               f"{100.0 * by / workload_bytes(w):.1f}% of the step's bytes) per step; plain fp64 C oracle, "
               f"single thread, append + attention")
     return {

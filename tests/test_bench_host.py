@@ -98,6 +98,20 @@ def test_reference_arm_prints_one_json_line_on_cpu():
     assert d["config"] == bench.workload_config(workloads.make("tiny"), "tiny", 1)
 
 
+def test_reference_sample_cuts_a_request_that_exceeds_the_step_budget():
+    """A step budget below one request (long contexts: one request of 32k-128k
+    tokens x 8 kv heads times 1000 steps would run for an hour) cuts the
+    sampled request to the cached tokens that fit, at least one page."""
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config",
+                        "tiny", "--steps", "3", "--warmup", "3", "--ref-budget", "8"], capture_output=True,
+                       text=True, env=env, timeout=600, check=True)
+    d = json.loads([ln for ln in r.stdout.splitlines() if ln.startswith("{")][0])
+    w = workloads.make("tiny")                     # first request: 17 cached tokens, page 16, Hkv 2
+    assert "cut to its first 16 cached tokens" in d["cpu_baseline"]["sample"]
+    assert d["metric_bytes_per_step_sampled"] == bench.metric_bytes([16], w.Hq, w.Hkv, w.d, w.P, w.kv_fp8)
+
+
 def test_default_suite_ends_on_the_largest_workload():
     assert bench.DEFAULT_CONFIG == "suite"
     sizes = {n: bench.workload_bytes(workloads.make(n)) for n in bench.SUITE}
