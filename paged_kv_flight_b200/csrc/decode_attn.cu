@@ -502,10 +502,10 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constan
                 // d, and the mma n-index j of n-tile nt stands for d = DV*j + nt.
                 constexpr int DV = D / 8;
                 constexpr int WORDS = DV / 4;
-                // one 16-token half at a time (not unrolled: the second half's
-                // loads are not hoisted over the first's mma, which keeps the
-                // 32-token tile within the register file)
-#pragma unroll 1
+                // the 16-token halves unrolled: the second half's shared-memory
+                // loads may issue while the first half's mma run (the tile
+                // still fits the register file: 234 registers, no spills)
+#pragma unroll
                 for (int h16 = 0; h16 < TT / 16; ++h16) {
                     const uint32_t pl = (TT == 16 || h16 == 0) ? pa0[0] : pa0[TT / 16 - 1];
                     const uint32_t ph = (TT == 16 || h16 == 0) ? pa2[0] : pa2[TT / 16 - 1];
