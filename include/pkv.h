@@ -313,11 +313,13 @@ pkv_status pkv_check_device_error(pkv_ctx* ctx, cudaStream_t stream, int* bits);
 pkv_status pkv_set_workers(pkv_ctx* ctx, int workers);
 
 /* Caps the number of dynamic chunks each warp range's tail is cut into
- * (0 .. 8; 0, the default, gives a static split).  With a cap above 0 the
- * last quarter of every range (at most 48 tiles of 16 tokens) is cut into
- * chunks of at least 4 tiles that warps which finish their own share early
- * claim; ranges under 32 tiles get no tail.  Results do not depend on it
- * beyond rounding. */
+ * (0 .. 8; 0 gives a static split; -1, the default, is automatic: 4 chunks
+ * when every range holds at least 192 tiles, as long contexts do, else a
+ * static split).  With a cap above 0 the last quarter of every range (at
+ * most 48 tiles of 16 tokens) is cut into chunks of at least 4 tiles that
+ * warps which finish their own share early claim; ranges under 32 tiles get
+ * no tail.  Results do not depend on it beyond rounding, and each chunk's
+ * partial has a fixed slot, so they repeat bit for bit. */
 pkv_status pkv_set_tail_chunks(pkv_ctx* ctx, int max_chunks);
 
 /* Sets how many CTAs (one thread-block cluster) share each head's hidden

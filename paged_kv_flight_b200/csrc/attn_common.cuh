@@ -101,6 +101,7 @@ __device__ __forceinline__ Split make_split(long long T, int W, int max_chunks)
     sp.qT = T / W;
     sp.rT = (int)(T - sp.qT * W);
     sp.K = 0;
+    if (max_chunks == kTailAuto) max_chunks = sp.qT >= kAutoTailTiles ? kAutoTailChunks : 0;
     if (max_chunks > 0 && sp.qT >= kTailMinTiles)
         sp.K = min(max_chunks, max(1, Split::tail_of(sp.qT) / kTailChunkTiles));
     return sp;

@@ -715,7 +715,8 @@ cudaError_t launch_decode_attn(const AttnParams& p, const CUtensorMap& tmk, cons
     if (e != cudaSuccess) return e;
     q.tile = L.tile;
     q.grid_warps = L.ctas * kAttnWarps;
-    return launch_combine(q, head_dim, (int)max_units(L.ctas * kAttnWarps, p.tail_chunks), L.ctas, stream, true);
+    const int tail_cap = p.tail_chunks == kTailAuto ? kAutoTailChunks : p.tail_chunks;
+    return launch_combine(q, head_dim, (int)max_units(L.ctas * kAttnWarps, tail_cap), L.ctas, stream, true);
 }
 
 }  // namespace pkv

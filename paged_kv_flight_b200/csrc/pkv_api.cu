@@ -694,7 +694,7 @@ pkv_status pkv_set_qkv_split(pkv_ctx* ctx, int split)
 
 pkv_status pkv_set_tail_chunks(pkv_ctx* ctx, int max_chunks)
 {
-    if (!ctx || max_chunks < 0 || max_chunks > pkv::kMaxTailChunks) return PKV_ERR_INVALID_ARG;
+    if (!ctx || max_chunks < pkv::kTailAuto || max_chunks > pkv::kMaxTailChunks) return PKV_ERR_INVALID_ARG;
     ctx->tail_chunks = max_chunks;
     return PKV_OK;
 }

@@ -49,7 +49,13 @@ constexpr int kTailMinTiles = 32;
 constexpr int kMaxTailChunks = 8;
 // a chunk must outlast the producer's lead over the consumer (see decode_attn.cu)
 static_assert(kTailChunkTiles > PKV_ATTN_MAX_STAGES, "tail chunks must be longer than the TMA ring");
-constexpr int kDefaultTailChunks = 0;
+// -1 (the default): automatic, kAutoTailChunks chunks when every warp range
+// holds at least kAutoTailTiles tiles (long contexts, where a chunk's fresh
+// page lookahead and query load are amortised), a static split otherwise
+constexpr int kTailAuto = -1;
+constexpr int kAutoTailChunks = 4;
+constexpr int kAutoTailTiles = 192;
+constexpr int kDefaultTailChunks = kTailAuto;
 
 // Units the split may cut the tiles into (two partial slots each).
 inline size_t max_units(int max_workers, int tail_chunks)
@@ -95,7 +101,7 @@ struct AttnParams {
     int batch, bt_stride, Hq, Hkv, G, P, num_pages;
     int stages;           // pipeline depth per warp
     int workers;          // 0: automatic
-    int tail_chunks;      // largest K (chunks per warp tail); 0: static split only
+    int tail_chunks;      // largest K (chunks per warp tail); 0: static split only; kTailAuto: automatic
     int q_len;            // new tokens per request (1: one new token); partial rows = G x q_len
     // varlen (several new tokens, a different count per request): the kernel
     // works on virtual requests, blocks of at most q_len new tokens of one

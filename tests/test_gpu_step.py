@@ -224,6 +224,20 @@ def test_decode_step_under_every_split_equals_the_two_calls(pkv, case_name):
         pkv.pkv_destroy(ctx)
 
 
+def test_tail_chunk_setting_accepts_automatic_and_rejects_out_of_range(pkv):
+    """-1 (the default) is the automatic tail, 0 .. 8 a cap; anything else
+    is rejected without changing the setting."""
+    w = _small(SMALL[0])
+    ctx = _gpu.make_ctx(pkv, w)
+    try:
+        for ok in (-1, 0, 1, 8):
+            assert pkv.pkv_set_tail_chunks(ctx, ok, check=False) == pkv.PKV_OK, ok
+        for bad in (-2, 9):
+            assert pkv.pkv_set_tail_chunks(ctx, bad, check=False) == pkv.PKV_ERR_INVALID_ARG, bad
+    finally:
+        pkv.pkv_destroy(ctx)
+
+
 def test_a_later_context_with_a_smaller_batch_leaves_an_earlier_one_usable(pkv):
     # the attention kernels' shared-memory limit is one process-wide setting;
     # a context created later with a smaller max_batch must not lower it
