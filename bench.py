@@ -910,6 +910,9 @@ def run_mixed(args, rank, world, local_rank):
     cu_d = torch.from_numpy(cu).to(dev)
     cfg = pkv.make_config(w.Hq, w.Hkv, w.d, w.P, "bf16", w.rope_base, B, w.bt_stride, w.num_pages)
     ctx = pkv.pkv_create(cfg)
+    G = w.Hq // w.Hkv
+    prefill_rows = 64 if args.prefill_rows is None else args.prefill_rows
+    pkv.pkv_set_prefill_rows(ctx, prefill_rows)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush_w = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
     flush_r = torch.ones(2 * l2 // 8, dtype=torch.int64, device=dev)
@@ -975,10 +978,16 @@ def run_mixed(args, rank, world, local_rank):
     row = 2 * w.Hkv * w.d * 2                      # K + V bytes of one token
     # metric bytes: each request's cache (its new tokens included) once, q and out of every new token
     by = int((row * (L + q_lens)).sum()) + 2 * n_tok * w.Hq * w.d * 2
-    # streamed: every block of 16 / G new tokens reads its own prefix
-    blk = 16 // (w.Hq // w.Hkv)
+    # streamed: every block reads its own prefix — blocks of 128 / G new tokens
+    # for requests with G x new tokens >= prefill_rows (the tensor-core
+    # prefill blocks), of 16 / G for the others
+    cmin = -(-prefill_rows // G) if prefill_rows > 0 else None
+    chunked = [cmin is not None and int(qb) >= cmin for qb in q_lens]
+    n_chunked = sum(chunked)
     streamed = sum(row * (int(Lb) + min(j + blk, int(qb)))
-                   for Lb, qb in zip(L, q_lens) for j in range(0, int(qb), blk)) + 2 * n_tok * w.Hq * w.d * 2
+                   for Lb, qb, ch in zip(L, q_lens, chunked)
+                   for blk in [128 // G if ch else 16 // G]
+                   for j in range(0, int(qb), blk)) + 2 * n_tok * w.Hq * w.d * 2
     peak, peak_src = measured_peak()
     gbs = by / (attn_ms * 1e-3) / 1e9
     return {"metric": METRIC, "value": sum_over_ranks(float(by)) / (step_ms * 1e-3) / 1e9, "unit": "GB/s",
@@ -988,16 +997,19 @@ def run_mixed(args, rank, world, local_rank):
                        "description": "llama8b batch, 56 requests decode one token, 8 prefill a 64-token "
                                       "chunk (568 new tokens): varlen RoPE + append, then varlen attention",
                        "l2": "flushed before every step, outside the event window",
-                       "timing": "step: CUDA-graph replay; attention alone: eager events"},
+                       "timing": "step: CUDA-graph replay; attention alone: eager events",
+                       "prefill_rows": prefill_rows, "prefill_requests": n_chunked},
             "step_us": step_ms * 1e3, "attn_us": attn_ms * 1e3, "new_tokens": n_tok,
             "new_tokens_per_s": sum_over_ranks(float(n_tok)) / (step_ms * 1e-3),
             "streamed_bytes_per_launch": streamed,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
-                         "traffic": recorded_traffic("mixed"), "kernel": "decode_attn_tokens_kernel<128> (varlen)",
+                         "traffic": recorded_traffic("mixed"),
+                         "kernel": ("chunk_attn_kernel<128> + " if n_chunked else "") + "decode_attn_tokens_kernel<128> (varlen)",
                          "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)", "bytes_per_launch": by,
                          "note": "bytes = each request's cache once (the metric); a prefill chunk's blocks "
                                  "re-read their prefix, see streamed_bytes_per_launch"},
-            "gpu_launches": 7 * K, "clocks": clock_info}   # step: rope, plan, attention, combine; alone: 3
+            # step: rope, plan, (prefill blocks,) attention, combine; alone: the same without rope
+            "gpu_launches": (9 if n_chunked else 7) * K, "clocks": clock_info}
 
 
 def run_loop(args, rank, world, local_rank):
@@ -1048,6 +1060,8 @@ def run_each_in_own_process(args, names) -> int:
             flags.append("--" + opt.replace("_", "-"))
     if args.tail_chunks is not None:
         flags += ["--tail-chunks", str(args.tail_chunks)]
+    if args.prefill_rows is not None:
+        flags += ["--prefill-rows", str(args.prefill_rows)]
     if args.requests is not None:
         flags += ["--requests", str(args.requests)]
     for i, name in enumerate(names):
@@ -1080,6 +1094,9 @@ def main(argv=None):
                     help="time the step as pkv_rope_append + pkv_decode_attn instead of pkv_decode_step")
     ap.add_argument("--tail-chunks", type=int, default=None,
                     help="cap on dynamic tail chunks per warp range (library default if omitted; 0: static split)")
+    ap.add_argument("--prefill-rows", type=int, default=None,
+                    help="mixed: G x new tokens from which a request takes the tensor-core prefill blocks "
+                         "(library default 64 if omitted; 0: none)")
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--requests", type=int, default=None,
                     help="keep only the first N requests of the workload (a smaller case for profiler captures)")

@@ -63,7 +63,7 @@
  *       host page allocator of pkv_pages.h;
  *   pkv_decode_attn_noalloc                          the attention without a
  *       context (no allocation);
- *   pkv_set_workers, pkv_set_tail_chunks, pkv_set_qkv_split,
+ *   pkv_set_workers, pkv_set_tail_chunks, pkv_set_qkv_split, pkv_set_prefill_rows,
  *   pkv_qkv_launch_shape, pkv_workspace_bytes        tuning and inspection.
  *
  * Errors: host-side checks return PKV_ERR_INVALID_ARG / PKV_ERR_UNSUPPORTED
@@ -225,7 +225,10 @@ pkv_status pkv_rope_append_varlen(pkv_ctx* ctx, void* q, const void* k_new, cons
  * pkv_decode_attn).  A plan
  * kernel cuts each request's new tokens into blocks of 16 / G tokens (the G x
  * 16/G query rows of a block and kv head are one 16-row mma), each block
- * streams its prefix of the cache once for its tokens.  The context holds
+ * streams its prefix of the cache once for its tokens; with bf16 pools a
+ * request of at least 64 / G new tokens (pkv_set_prefill_rows) is cut
+ * instead into blocks of 128 / G tokens for the tensor cores (one 128-row
+ * MMA block per kv head).  The context holds
  * room for 4 x max_batch blocks (at most 8192): a call with batch +
  * ceil(n_tokens / (16 / G)) above that returns PKV_ERR_UNSUPPORTED without
  * launching; lengths past the block table zero the affected tokens' output
@@ -321,6 +324,17 @@ pkv_status pkv_set_workers(pkv_ctx* ctx, int workers);
  * no tail.  Results do not depend on it beyond rounding, and each chunk's
  * partial has a fixed slot, so they repeat bit for bit. */
 pkv_status pkv_set_tail_chunks(pkv_ctx* ctx, int max_chunks);
+
+/* Which requests of a pkv_decode_attn_varlen call (bf16 pools) take the
+ * tensor-core prefill-chunk path: those with G x new tokens >= rows (1 ..
+ * 128; 64, the default, is half a block); 0 sends every request to the
+ * several-new-tokens kernel.  That path cuts a request's new tokens into
+ * blocks of 128 / G, whose 128 query rows (G heads of each token) share one
+ * pass over the request's cache per kv head: S = q K^T and P V on tcgen05
+ * with fp32 accumulators in tensor memory, P carried as two bf16 terms
+ * (about 16 significant bits).  Results agree with the other path within
+ * rounding. */
+pkv_status pkv_set_prefill_rows(pkv_ctx* ctx, int rows);
 
 /* Sets how many CTAs (one thread-block cluster) share each head's hidden
  * dimension in pkv_qkv_rope_append: 1 .. 4, or 0 (the default) for the

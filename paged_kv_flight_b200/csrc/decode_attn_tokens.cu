@@ -619,32 +619,48 @@ namespace {
 // One CTA: request b's new tokens (cu_q[b + 1] - cu_q[b] of them) cut into
 // blocks of `block`; vmap[v] = {b, first q row, tokens, L_b + offset of the
 // block}, v counted in request order (an exclusive scan of the blocks per
-// request).  More than vmax blocks, or a negative token count, set kErrLength
-// (the surplus is dropped).
+// request).  With cmin > 0, a request of at least cmin new tokens is cut
+// instead into blocks of cblock tokens listed the same way in cmap (the
+// prefill-chunk kernel's work).  More blocks than a map holds, or a negative
+// token count, set kErrLength (the surplus is dropped).
 __global__ void __launch_bounds__(1024) varlen_plan_kernel(const int32_t* __restrict__ cu_q,
                                                            const int32_t* __restrict__ seq_lens, int batch,
                                                            int block, int vmax, int4* __restrict__ vmap,
-                                                           int* __restrict__ vcount, int* __restrict__ err)
+                                                           int* __restrict__ vcount, int cmin, int cblock, int cmax,
+                                                           int4* __restrict__ cmap, int* __restrict__ ccount,
+                                                           int* __restrict__ err)
 {
-    __shared__ int s_warp[32];
+    __shared__ int s_warp[2][32];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
     const int per = (batch + (int)blockDim.x - 1) / (int)blockDim.x;
     const int lo = min(batch, tid * per), hi = min(batch, lo + per);
-    int local = 0;
+    auto chunked = [&](int q) { return cmin > 0 && q >= cmin; };
+    int lv = 0, lc = 0;   // this thread's virtual and chunk blocks
     for (int b = lo; b < hi; ++b) {
         const int q = cu_q[b + 1] - cu_q[b];
-        local += q > 0 ? (q + block - 1) / block : 0;
+        if (q <= 0) continue;
+        if (chunked(q)) lc += (q + cblock - 1) / cblock;
+        else lv += (q + block - 1) / block;
     }
-    int incl = local;
+    int iv = lv, ic = lc;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(kFull, incl, o);
-        if (lane >= o) incl += v;
+        const int v = __shfl_up_sync(kFull, iv, o), c = __shfl_up_sync(kFull, ic, o);
+        if (lane >= o) {
+            iv += v;
+            ic += c;
+        }
     }
-    if (lane == 31) s_warp[warp] = incl;
+    if (lane == 31) {
+        s_warp[0][warp] = iv;
+        s_warp[1][warp] = ic;
+    }
     __syncthreads();
-    int run = incl - local;
-    for (int w2 = 0; w2 < warp; ++w2) run += s_warp[w2];
+    int rv = iv - lv, rc = ic - lc;
+    for (int w2 = 0; w2 < warp; ++w2) {
+        rv += s_warp[0][w2];
+        rc += s_warp[1][w2];
+    }
     for (int b = lo; b < hi; ++b) {
         const int a = cu_q[b], q = cu_q[b + 1] - a;
         if (q < 0) {
@@ -652,31 +668,40 @@ __global__ void __launch_bounds__(1024) varlen_plan_kernel(const int32_t* __rest
             continue;
         }
         const long long L = seq_lens[b];
-        for (int j = 0; (long long)j * block < q; ++j) {
-            const long long pos = L + (long long)j * block;
-            if (run < vmax)
-                vmap[run] = make_int4(b, a + j * block, min(block, q - j * block),
-                                      (L < 0 || pos > 0x7fffffffll) ? -1 : (int)pos);
-            ++run;
+        const bool ch = chunked(q);
+        const int blk = ch ? cblock : block;
+        for (int j = 0; (long long)j * blk < q; ++j) {
+            const long long pos = L + (long long)j * blk;
+            const int4 e = make_int4(b, a + j * blk, min(blk, q - j * blk), (L < 0 || pos > 0x7fffffffll) ? -1 : (int)pos);
+            if (ch) {
+                if (rc < cmax) cmap[rc] = e;
+                ++rc;
+            } else {
+                if (rv < vmax) vmap[rv] = e;
+                ++rv;
+            }
         }
     }
     if (tid == 0) {
-        int total = 0;
-        for (int w2 = 0; w2 < nwarps; ++w2) total += s_warp[w2];
-        if (total > vmax) {
-            atomicOr(err, kErrLength);
-            total = vmax;
+        int tv = 0, tc = 0;
+        for (int w2 = 0; w2 < nwarps; ++w2) {
+            tv += s_warp[0][w2];
+            tc += s_warp[1][w2];
         }
-        *vcount = total;
+        if (tv > vmax || tc > cmax) atomicOr(err, kErrLength);
+        *vcount = min(tv, vmax);
+        if (ccount) *ccount = min(tc, cmax);
     }
 }
 
 }  // namespace
 
 cudaError_t launch_varlen_plan(const int32_t* cu_q, const int32_t* seq_lens, int batch, int block, int vmax,
-                               int4* vmap, int* vcount, int* err, cudaStream_t stream)
+                               int4* vmap, int* vcount, int cmin, int cblock, int cmax, int4* cmap, int* ccount,
+                               int* err, cudaStream_t stream)
 {
-    varlen_plan_kernel<<<1, 1024, 0, stream>>>(cu_q, seq_lens, batch, block, vmax, vmap, vcount, err);
+    varlen_plan_kernel<<<1, 1024, 0, stream>>>(cu_q, seq_lens, batch, block, vmax, vmap, vcount,
+                                               cmap ? cmin : 0, cblock > 0 ? cblock : 1, cmax, cmap, ccount, err);
     return cudaGetLastError();
 }
 

@@ -33,6 +33,9 @@ struct pkv_ctx {
     int vmax;             // virtual requests a varlen attention call may have (bf16 pools)
     int4* d_vmap;         // [vmax] the varlen plan
     int* d_vcount;
+    int prefill_rows;     // varlen requests with G x new tokens >= this go to the prefill-chunk kernel (0: none)
+    int4* d_cmap;         // [vmax] its blocks
+    int* d_ccount;
     float* d_part_o;
     float* d_part_ml;
     const void* tm_k_ptr;
@@ -43,6 +46,10 @@ struct pkv_ctx {
     const void* t16_k_ptr;
     const void* t16_v_ptr;
     CUtensorMap t16k, t16v;
+    // page-high boxes (P rows) for the prefill-chunk kernel (bf16 pools)
+    const void* tp_k_ptr;
+    const void* tp_v_ptr;
+    CUtensorMap tpk, tpv;
     const void* tm_w_ptr;        // QKV weight and input maps of pkv_qkv_rope_append
     int tm_w_hidden, tm_w_layout;
     int qkv_split;               // 0: automatic
@@ -201,7 +208,7 @@ pkv_status pkv_create(const pkv_config* cfg, pkv_ctx** out)
         free(ctx);
         return PKV_ERR_CUDA;
     }
-    if (pkv::qkv_prepare() != cudaSuccess) {
+    if (pkv::qkv_prepare() != cudaSuccess || pkv::chunk_attn_prepare(cfg->head_dim) != cudaSuccess) {
         free(ctx);
         return PKV_ERR_CUDA;
     }
@@ -216,7 +223,7 @@ pkv_status pkv_create(const pkv_config* cfg, pkv_ctx** out)
     const size_t b_cnt = ((size_t)(std::max(cfg->max_batch, ctx->vmax) + 8) * sizeof(int) + 255) & ~(size_t)255;
     const size_t b_po = 2 * rows_units * cfg->head_dim * sizeof(float);
     const size_t b_pml = 2 * rows_units * 2 * sizeof(float);
-    const size_t b_vm = (size_t)ctx->vmax * sizeof(int4) + 256;   // varlen plan + its count
+    const size_t b_vm = 2 * ((size_t)ctx->vmax * sizeof(int4) + 256);   // varlen plans (virtual, chunk) + counts
     const size_t b_th = ((size_t)cfg->head_dim / 2 * sizeof(double) + 255) & ~(size_t)255;   // RoPE frequencies
     ctx->ws_bytes = b_err + b_cnt + b_po + b_pml + b_vm + b_th;
     if (cudaMalloc(&ctx->ws, ctx->ws_bytes) != cudaSuccess) {
@@ -233,6 +240,9 @@ pkv_status pkv_create(const pkv_config* cfg, pkv_ctx** out)
     ctx->d_part_ml = reinterpret_cast<float*>(base + b_err + b_cnt + b_po);
     ctx->d_vcount = reinterpret_cast<int*>(base + b_err + b_cnt + b_po + b_pml);
     ctx->d_vmap = reinterpret_cast<int4*>(base + b_err + b_cnt + b_po + b_pml + 256);
+    ctx->d_ccount = reinterpret_cast<int*>(base + b_err + b_cnt + b_po + b_pml + b_vm / 2);
+    ctx->d_cmap = reinterpret_cast<int4*>(base + b_err + b_cnt + b_po + b_pml + b_vm / 2 + 256);
+    ctx->prefill_rows = pkv::kDefaultPrefillRows;
     ctx->d_theta = reinterpret_cast<double*>(base + b_err + b_cnt + b_po + b_pml + b_vm);
     // theta_i = rope_base^(-2i/d) once, in fp64 on the host
     double theta[64];
@@ -551,9 +561,57 @@ pkv_status pkv_decode_attn_varlen(pkv_ctx* ctx, const void* q, const void* k_poo
     // blocks of `block` new tokens: G x block <= 16 query rows per (block, kv head)
     const int block = pkv::kMaxTokenRows / ctx->G;
     if ((long long)batch + (n_tokens + block - 1) / block > ctx->vmax) return PKV_ERR_UNSUPPORTED;
-    if (pkv::launch_varlen_plan(cu_q, seq_lens, batch, block, ctx->vmax, ctx->d_vmap, ctx->d_vcount, ctx->d_err,
+    // requests with at least cmin new tokens: blocks of cblock on the tensor
+    // cores (bf16 pools).  At most min(batch, n_tokens / cmin) requests take
+    // that path, so it has at most n_tokens / cblock + that many blocks: within
+    // vmax (>= batch + n_tokens / block) by the check above
+    const bool fp8 = ctx->cfg.kv_dtype == PKV_KV_FP8_E4M3;
+    const int cblock = pkv::kChunkRows / ctx->G;
+    const int cmin = (!fp8 && ctx->prefill_rows > 0) ? std::max(1, (ctx->prefill_rows + ctx->G - 1) / ctx->G) : 0;
+    const long long creq = cmin > 0 ? std::min<long long>(batch, n_tokens / cmin) : 0;
+    const int citems = creq > 0 ? (int)std::min<long long>(ctx->vmax, (long long)n_tokens / cblock + creq) : 0;
+    if (pkv::launch_varlen_plan(cu_q, seq_lens, batch, block, ctx->vmax, ctx->d_vmap, ctx->d_vcount, cmin, cblock,
+                                ctx->vmax, cmin > 0 ? ctx->d_cmap : nullptr, ctx->d_ccount, ctx->d_err,
                                 stream) != cudaSuccess)
         return PKV_ERR_CUDA;
+    if (citems > 0) {
+        if (ctx->tp_k_ptr != k_pool) {
+            if (!encode_pool_rows(ctx, k_pool, ctx->cfg.page_size, &ctx->tpk)) return PKV_ERR_CUDA;
+            ctx->tp_k_ptr = k_pool;
+        }
+        if (ctx->tp_v_ptr != v_pool) {
+            if (!encode_pool_rows(ctx, v_pool, ctx->cfg.page_size, &ctx->tpv)) return PKV_ERR_CUDA;
+            ctx->tp_v_ptr = v_pool;
+        }
+        pkv::AttnParams cp;
+        cp.q = static_cast<const __nv_bfloat16*>(q);
+        cp.out = static_cast<__nv_bfloat16*>(out);
+        cp.k_scale = nullptr;
+        cp.v_scale = nullptr;
+        cp.block_tables = block_tables;
+        cp.seq_lens = seq_lens;
+        cp.part_o = nullptr;
+        cp.part_ml = nullptr;
+        cp.meta = nullptr;
+        cp.err = ctx->d_err;
+        cp.claim = nullptr;
+        cp.scale_log2 = (float)(1.4426950408889634 / sqrt((double)ctx->cfg.head_dim));
+        cp.batch = batch;
+        cp.bt_stride = bt_stride;
+        cp.Hq = ctx->cfg.num_q_heads;
+        cp.Hkv = ctx->cfg.num_kv_heads;
+        cp.G = ctx->G;
+        cp.P = ctx->cfg.page_size;
+        cp.num_pages = ctx->cfg.num_pages;
+        cp.stages = 0;
+        cp.workers = 0;
+        cp.tail_chunks = 0;
+        cp.q_len = cblock;
+        cp.cmap = ctx->d_cmap;
+        cp.ccount = ctx->d_ccount;
+        if (pkv::launch_chunk_attn(cp, ctx->tpk, ctx->tpv, ctx->cfg.head_dim, citems, stream) != cudaSuccess)
+            return PKV_ERR_CUDA;
+    }
     return attn_tokens_launch(ctx, q, k_pool, v_pool, k_scale, v_scale, block_tables, bt_stride, seq_lens,
                               ctx->vmax, block, ctx->d_vmap, ctx->d_vcount, out, stream);
 }
@@ -696,6 +754,13 @@ pkv_status pkv_set_tail_chunks(pkv_ctx* ctx, int max_chunks)
 {
     if (!ctx || max_chunks < pkv::kTailAuto || max_chunks > pkv::kMaxTailChunks) return PKV_ERR_INVALID_ARG;
     ctx->tail_chunks = max_chunks;
+    return PKV_OK;
+}
+
+pkv_status pkv_set_prefill_rows(pkv_ctx* ctx, int rows)
+{
+    if (!ctx || rows < 0 || rows > pkv::kChunkRows) return PKV_ERR_INVALID_ARG;
+    ctx->prefill_rows = rows;
     return PKV_OK;
 }
 

@@ -32,6 +32,13 @@ constexpr int kTileWide = 32;      // E4M3 tiles when pages hold at least 32 tok
 inline int attn_tile(bool fp8, int page_size) { return (fp8 && page_size >= kTileWide) ? kTileWide : kTile; }
 constexpr int kMaxGroup = 8;       // query heads per kv head handled by one mma row block
 constexpr int kMaxTokenRows = 16;  // G x q_len rows of the several-new-tokens attention
+// Prefill chunks of a varlen call on the tensor cores (chunk_attn.cu): blocks
+// of kChunkRows / G new tokens (G x that query rows), tiles of kChunkKeys
+// keys; a request takes that path when it has at least kDefaultPrefillRows / G
+// new tokens (pkv_set_prefill_rows; 0: never).
+constexpr int kChunkRows = 128;
+constexpr int kChunkKeys = 128;
+constexpr int kDefaultPrefillRows = 64;
 constexpr int kAttnWarps = PKV_ATTN_WARPS;
 constexpr int kAttnMaxStages = PKV_ATTN_MAX_STAGES;
 constexpr int kMinTilesPerWorker = 8;
@@ -110,6 +117,10 @@ struct AttnParams {
     // the varlen plan; null for the other calls
     const int4* vmap = nullptr;
     const int* vcount = nullptr;
+    // varlen prefill blocks for chunk_attn (same entries as vmap, blocks of
+    // kChunkRows / G tokens), *ccount of them
+    const int4* cmap = nullptr;
+    const int* ccount = nullptr;
     // the combine of the one-token attention runs as its programmatic
     // dependent (own_split = 1): it derives the split itself from seq_lens
     // (tiles of `tile` tokens over `grid_warps` warps, as the attention did)
@@ -143,9 +154,18 @@ cudaError_t launch_decode_attn(const AttnParams& p, const CUtensorMap& tmk, cons
 cudaError_t attn_tokens_prepare(int head_dim, bool fp8, int num_sms, int max_batch, AttnLaunch* out);
 // The virtual requests of a varlen call: blocks of `block` new tokens (the
 // last of a request may be shorter) of requests with cu_q[b + 1] > cu_q[b];
-// writes vmap and the count (capped at vmax; more sets kErrLength).
+// writes vmap and the count (capped at vmax; more sets kErrLength).  With
+// cmin > 0 a request of at least cmin new tokens goes instead to cmap in
+// blocks of cblock tokens (capped at cmax), for the prefill-chunk kernel.
 cudaError_t launch_varlen_plan(const int32_t* cu_q, const int32_t* seq_lens, int batch, int block, int vmax,
-                               int4* vmap, int* vcount, int* err, cudaStream_t stream);
+                               int4* vmap, int* vcount, int cmin, int cblock, int cmax, int4* cmap,
+                               int* ccount, int* err, cudaStream_t stream);
+// The prefill-chunk attention (chunk_attn.cu, bf16 pools): sets its shared-
+// memory limit once, and launches max_items x Hkv CTAs for p.cmap (the CTAs
+// past *p.ccount return at once).  It writes its rows of p.out directly.
+cudaError_t chunk_attn_prepare(int head_dim);
+cudaError_t launch_chunk_attn(const AttnParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv, int head_dim,
+                              int max_items, cudaStream_t stream);
 cudaError_t launch_decode_attn_tokens(const AttnParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
                                       int head_dim, bool fp8, const AttnLaunch& L, cudaStream_t stream,
                                       bool pdl = false);

@@ -45,6 +45,7 @@
 // its stores.
 #include "pkv_internal.h"
 #include "pkv_device.cuh"
+#include "umma.cuh"
 
 namespace pkv {
 namespace {
@@ -64,59 +65,12 @@ constexpr int kQkvSmemLimit = 1024 + 220 * 1024;
 constexpr int kQkvRecvRow = 80;                // bytes per row of received partials (64 + 16: no bank conflicts)
 constexpr uint64_t kQkvWaitNs = 500ull * 1000ull * 1000ull;
 
-// Shared-memory matrix descriptor of a K-major tile with 128-byte rows and
-// the 128-byte swizzle (the layout the TMA loads write): start address >> 4,
-// leading byte offset 1 (unused by this layout), stride byte offset 1024 B
-// (8 rows), descriptor version 1, layout type 2 (128-byte swizzle).  The tile
-// base is 1024-byte aligned; a K step of 16 elements adds 32 bytes to the
-// start address.
-__device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr)
-{
-    uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
-    d |= (uint64_t)1u << 16;
-    d |= (uint64_t)(1024u >> 4) << 32;
-    d |= (uint64_t)1u << 46;
-    d |= (uint64_t)2u << 61;
-    return d;
-}
-
-// Instruction descriptor of kind::f16: fp32 accumulator, bf16 A and B, both
-// K-major, N >> 3 at bit 17, M >> 4 at bit 24.
+// Instruction descriptor of the projection's MMA: M = 128 token rows, N = d.
 template <int N>
 __host__ __device__ constexpr uint32_t qkv_idesc()
 {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(kQkvM >> 4) << 24);
+    return umma_idesc_bf16<kQkvM, N>();
 }
-
-template <int N>
-__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t"
-        ".reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t"
-        "}\n" ::"r"(tmem_d),
-        "l"(adesc), "l"(bdesc), "r"(qkv_idesc<N>()), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
-}
-
-__device__ __forceinline__ void umma_commit(uint32_t bar)
-{
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-                 : "memory");
-}
-
-__device__ __forceinline__ void tmem_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tmem_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-// 8 consecutive fp32 columns of this thread's TMEM lane (completion: tmem_wait_ld).
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8])
-{
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
-                 : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // The shared-memory address of the same variable in CTA `rank` of the cluster.
 __device__ __forceinline__ uint32_t cluster_map(uint32_t local, uint32_t rank)
@@ -213,9 +167,7 @@ qkv_rope_append_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_con
     }
     if (warp == 0) {
         __syncwarp();   // converged for the aligned allocation
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s_tmem)),
-                     "r"(kCols));
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+        tmem_alloc(smem_u32(&s_tmem), kCols);
     }
     tmem_fence_before();
     __syncthreads();
@@ -249,8 +201,8 @@ qkv_rope_append_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_con
                 const uint32_t a = stage0 + (uint32_t)(s * STB), b = a + (uint32_t)XA;
 #pragma unroll
                 for (int kk = 0; kk < kQkvBK / 16; ++kk)
-                    umma_bf16<D>(tmem, sw128_kmajor_desc(a + 32u * kk), sw128_kmajor_desc(b + 32u * kk),
-                                 (i | kk) != 0 ? 1u : 0u);
+                    umma_bf16(tmem, sw128_kmajor_desc(a + 32u * kk), sw128_kmajor_desc(b + 32u * kk), qkv_idesc<D>(),
+                              (i | kk) != 0 ? 1u : 0u);
                 umma_commit(empty0 + 8u * s);
             }
             umma_commit(done);   // arrives once every MMA issued above has completed
@@ -352,7 +304,7 @@ qkv_rope_append_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_con
     cluster_sync_all();                      // every partial delivered; no cluster access after this
     if (warp == 0) {
         tmem_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kCols));
+        tmem_dealloc(tmem, kCols);
     }
 
     // ---- epilogue: (own group, token row) items over all threads, rows

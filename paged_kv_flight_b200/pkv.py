@@ -44,7 +44,7 @@ PKV_KV_FP8_E4M3 = 1
 # names of every symbol include/pkv.h declares
 EXPORTS = ("pkv_create", "pkv_rope_append", "pkv_decode_attn", "pkv_destroy", "pkv_status_str",
            "pkv_check_device_error", "pkv_set_workers", "pkv_workspace_bytes", "pkv_decode_attn_noalloc",
-           "pkv_set_tail_chunks", "pkv_rope_append_tokens", "pkv_decode_attn_tokens",
+           "pkv_set_tail_chunks", "pkv_set_prefill_rows", "pkv_rope_append_tokens", "pkv_decode_attn_tokens",
            "pkv_pages_create", "pkv_pages_destroy", "pkv_pages_admit", "pkv_pages_reserve", "pkv_pages_advance",
            "pkv_pages_release", "pkv_pages_block_table", "pkv_pages_seq_lens", "pkv_pages_active",
            "pkv_pages_refcount", "pkv_pages_free_count", "pkv_pages_take_changes", "pkv_qkv_rope_append",
@@ -110,6 +110,8 @@ lib.pkv_decode_attn_varlen.argtypes = [_V, _V, _V, _V, _V, _V, _V, C.c_int, _V, 
 lib.pkv_decode_attn_varlen.restype = C.c_int
 lib.pkv_set_tail_chunks.argtypes = [_V, C.c_int]
 lib.pkv_set_tail_chunks.restype = C.c_int
+lib.pkv_set_prefill_rows.argtypes = [_V, C.c_int]
+lib.pkv_set_prefill_rows.restype = C.c_int
 lib.pkv_workspace_bytes.argtypes = [_V]
 lib.pkv_workspace_bytes.restype = C.c_size_t
 lib.pkv_decode_attn_noalloc.argtypes = [C.POINTER(pkv_config), _V, _V, _V, _V, _V, _V, C.c_int, _V, C.c_int,
@@ -261,6 +263,10 @@ def pkv_set_workers(ctx, workers: int, check: bool = True) -> int:
 
 def pkv_set_tail_chunks(ctx, max_chunks: int, check: bool = True) -> int:
     return _done(lib.pkv_set_tail_chunks(ctx, int(max_chunks)), "pkv_set_tail_chunks", check)
+
+
+def pkv_set_prefill_rows(ctx, rows: int, check: bool = True) -> int:
+    return _done(lib.pkv_set_prefill_rows(ctx, int(rows)), "pkv_set_prefill_rows", check)
 
 
 def pkv_workspace_bytes(ctx) -> int:

@@ -28,6 +28,9 @@ CASES = [
     ("g1_d64_p16_prefill", 4, 4, 64, 16, [10, 700, 0], [100, 1, 130]),
     ("g8_d128_p16_prefill", 64, 8, 128, 16, [3000, 20, 511], [48, 1, 9]),
     ("g4_d128_p64_prefill", 32, 8, 128, 64, [2049, 0, 77, 1000], [64, 16, 1, 15]),
+    # key counts that end exactly on 128-key tiles (no rows past the keys)
+    # next to ragged ones, for the tensor-core prefill blocks
+    ("g4_d128_p16_aligned", 32, 8, 128, 16, [100, 1000, 4064, 7], [28, 24, 32, 40]),
 ]
 
 
@@ -77,13 +80,17 @@ def _step(pkv, ctx, dv):
     return out
 
 
+@pytest.mark.parametrize("prefill_rows", [64, 0], ids=["prefill_blocks", "token_blocks_only"])
 @pytest.mark.parametrize("case", CASES, ids=lambda c: c[0])
-def test_varlen_step_matches_oracle(pkv, case):
+def test_varlen_step_matches_oracle(pkv, case, prefill_rows):
+    """Default: requests of >= 64 / G new tokens on the tensor-core prefill
+    blocks, the rest on the several-new-tokens kernel; 0: all on the latter."""
     w, h, q_lens = _setup(case)
     ho, ref = _oracle(w, h)
     dv = _device(h)
     ctx = _gpu.make_ctx(pkv, w, max_batch=64)
     try:
+        pkv.pkv_set_prefill_rows(ctx, prefill_rows)
         out = _step(pkv, ctx, dv)
         assert pkv.pkv_check_device_error(ctx)[0] == pkv.PKV_OK
     finally:
@@ -139,6 +146,91 @@ def test_varlen_rejections_and_range_errors(pkv):
     finally:
         pkv.pkv_destroy(ctx)
 
+
+
+def test_varlen_every_request_on_prefill_blocks(pkv):
+    """prefill rows 1: every request with a new token takes the tensor-core
+    blocks (the several-new-tokens kernel gets no work) — single decode tokens,
+    a request with none, ragged blocks."""
+    case = CASES[0]
+    w, h, _ = _setup(case, seed=53)
+    _, ref = _oracle(w, h)
+    ctx = _gpu.make_ctx(pkv, w, max_batch=64)
+    try:
+        pkv.pkv_set_prefill_rows(ctx, 1)
+        out = _step(pkv, ctx, _device(h))
+        assert pkv.pkv_check_device_error(ctx)[0] == pkv.PKV_OK
+    finally:
+        pkv.pkv_destroy(ctx)
+    mx, mean, finite = _gpu.errors(out, ref)
+    assert finite and mx <= _gpu.TOL_BF16["max"] and mean <= _gpu.TOL_BF16["mean"], (mx, mean)
+
+
+def test_prefill_rows_setting_range(pkv):
+    w, _, _ = _setup(CASES[0])
+    ctx = _gpu.make_ctx(pkv, w, max_batch=8)
+    try:
+        for ok in (0, 1, 64, 128):
+            assert pkv.pkv_set_prefill_rows(ctx, ok, check=False) == pkv.PKV_OK, ok
+        for bad in (-1, 129):
+            assert pkv.pkv_set_prefill_rows(ctx, bad, check=False) == pkv.PKV_ERR_INVALID_ARG, bad
+    finally:
+        pkv.pkv_destroy(ctx)
+
+
+@pytest.mark.parametrize("fault", ["length", "page"])
+def test_varlen_prefill_block_range_errors(pkv, fault):
+    """A prefill request whose last token lies past its block table, or
+    whose table names a page outside the pool: its rows come out zero, the
+    error word says which, the other requests are still right."""
+    case = CASES[0]                       # request 3 prefills 64 tokens (G = 4: on the prefill blocks)
+    w, h, q_lens = _setup(case, seed=55)
+    _, ref = _oracle(w, h)
+    dv = _device(h)
+    bt, sl = dv["block_tables"].clone(), dv["seq_lens"].clone()
+    if fault == "length":
+        sl[3] = w.bt_stride * w.P - 10    # its 64 tokens run past the table
+    else:
+        bt[3, 0] = w.num_pages + 3        # its first page is outside the pool
+    out = torch.full_like(dv["q"], 1.0)
+    ctx = _gpu.make_ctx(pkv, w, max_batch=64)
+    try:
+        # the append with the good tables, the attention with the bad ones
+        pkv.pkv_rope_append_varlen(ctx, dv["q"], dv["k_new"], dv["v_new"], dv["k_pool"], dv["v_pool"], None, None,
+                                   dv["block_tables"], dv["seq_lens"], dv["cu_q"])
+        assert pkv.pkv_check_device_error(ctx)[0] == pkv.PKV_OK
+        pkv.pkv_decode_attn_varlen(ctx, dv["q"], dv["k_pool"], dv["v_pool"], None, None, bt, sl, dv["cu_q"], out)
+        st, bits = pkv.pkv_check_device_error(ctx)
+    finally:
+        pkv.pkv_destroy(ctx)
+    assert st == pkv.PKV_ERR_DEVICE_BOUNDS and bits & (1 if fault == "length" else 2), bits
+    cu = h["cu_q"]
+    rows = slice(int(cu[3]), int(cu[4]))
+    assert torch.count_nonzero(out[rows].float()) == 0
+    other = np.ones(int(cu[-1]), bool)
+    other[rows] = False
+    o = out.float().cpu().numpy()[other]
+    assert np.abs(o - ref[other]).max() <= _gpu.TOL_BF16["max"]
+
+
+def test_full_size_mixed_batch_matches_oracle(pkv):
+    """The benchmark's mixed batch (llama8b lengths, 8 requests prefill a
+    64-token chunk, 56 decode one token), as the benchmark runs it: RoPE +
+    append, then the attention, every output row against the oracle."""
+    w, q_lens = workloads.make_mixed(device="cpu")
+    h = varlen_host(w, q_lens)
+    ho, ref = _oracle(w, h)
+    dv = _device(h)
+    ctx = _gpu.make_ctx(pkv, w, max_batch=w.batch)
+    try:
+        out = _step(pkv, ctx, dv)
+        assert pkv.pkv_check_device_error(ctx)[0] == pkv.PKV_OK
+    finally:
+        pkv.pkv_destroy(ctx)
+    assert np.array_equal(bits16(dv["v_pool"]), ho["v_pool"])
+    mx, mean, finite = _gpu.errors(out, ref)
+    print(f"mixed: attention output vs the oracle over the whole batch: max abs {mx:.3e}, mean abs {mean:.3e}")
+    assert finite and mx <= _gpu.TOL_BF16["max"] and mean <= _gpu.TOL_BF16["mean"], (mx, mean)
 
 
 @pytest.mark.parametrize("P", [16, 32])
