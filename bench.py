@@ -53,7 +53,7 @@ KERNEL_SOURCES = {
              "paged_kv_flight_b200/csrc/attn_common.cuh", "paged_kv_flight_b200/csrc/combine.cu",
              "paged_kv_flight_b200/csrc/pkv_device.cuh", "paged_kv_flight_b200/csrc/pkv_internal.h"),
     "qkv": ("paged_kv_flight_b200/csrc/qkv_rope_append.cu", "paged_kv_flight_b200/csrc/pkv_device.cuh",
-            "paged_kv_flight_b200/csrc/pkv_internal.h"),
+            "paged_kv_flight_b200/csrc/umma.cuh", "paged_kv_flight_b200/csrc/pkv_internal.h"),
 }
 
 

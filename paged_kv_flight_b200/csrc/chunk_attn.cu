@@ -24,11 +24,13 @@
 //                   significant bits, so the weights of a row with few keys
 //                   carry no bf16-sized error), written over the warp's own S
 //                   columns; each half keeps its own running sum (same max)
-//   O_j = P V       tcgen05, A = P from TMEM, B = V (MN-major); M 128, N d,
-//                   K 2 x 128: P_hi V then P_lo V over the same V tile
-//   acc = acc 2^(m_old - m_new) + O_j, in registers (each warp half of d)
-// With S / P in two buffers, the softmax of tile j + 1 runs while P V of
-// tile j is on the tensor pipe; only the fold of O_j waits for it.  Roles:
+//   O += P V        tcgen05, A = P from TMEM, B = V (MN-major); M 128, N d,
+//                   K 2 x 128: P_hi V then P_lo V over the same V tile; O
+//                   stays in TMEM over all tiles
+// The reference max m of a row moves only when the row's max passes it by
+// more than 2^8 (P <= 2^8 meanwhile); then O and l are rescaled in place.
+// With S / P in two buffers and no per-tile fold of O, the softmax of tile
+// j + 1 runs while P V of tile j is on the tensor pipe.  Roles:
 // warp 0 lane 0 issues the K / V page loads, warp 1 lane 0 the MMAs (S and P
 // V each as soon as its inputs are ready), warps 2 .. 9 the softmax and the
 // output rows.  Every wait is bounded.
@@ -76,7 +78,7 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     using Gm = ChunkGeo<D>;
     constexpr int KB = Gm::KB, HD = D / 2;
     extern __shared__ uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t s_full[kCStages], s_empty[kCStages], s_sfull[2], s_pfull, s_ofull, s_drain;
+    __shared__ __align__(8) uint64_t s_full[kCStages], s_empty[kCStages], s_sfull[2], s_pfull, s_ofull, s_ofin, s_drain;
     __shared__ uint32_t s_tmem;
     __shared__ int s_bad, s_fail;
     __shared__ int s_issued, s_landed;         // tiles whose copies went out / were consumed by the MMA
@@ -146,6 +148,7 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
         mbar_init(sfull0 + 8u, 1u);
         mbar_init(pfull, (uint32_t)kCSoftWarps);
         mbar_init(ofull, 1u);
+        mbar_init(smem_u32(&s_ofin), 1u);
         mbar_init(smem_u32(&s_drain), 1u);
         fence_mbar_init();
         s_issued = min(kCStages, NT);
@@ -209,7 +212,7 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
             constexpr uint32_t idO = umma_idesc_bf16<kChunkRows, D, true>();
             int js = 0, jp = 0;
             bool ok = true;
-            uint64_t t0 = global_timer_ns();   // the last progress
+            uint64_t t_prog = global_timer_ns();   // the last progress
             for (uint32_t it = 0; jp < NT; ++it) {
                 bool moved = false;
                 if (js < NT && js <= jp + 1 &&
@@ -245,16 +248,17 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                         // along K, 8 key rows (1024 B) per swizzle atom
                         umma_bf16_ts(tmem + kCOcol, pcol + acol,
                                      sw128_mnmajor_desc(vd + (uint32_t)(k8 * 2048), (uint32_t)kCBlk, 1024u), idO,
-                                     kk ? 1u : 0u);
+                                     (jp | kk) ? 1u : 0u);
                     }
                     umma_commit(ofull);
+                    if (jp == NT - 1) umma_commit(smem_u32(&s_ofin));
                     umma_commit(empty0 + 8u * s);   // K and V of the stage are no longer read
                     ++jp;
                     moved = true;
                 }
                 if (moved) {
-                    t0 = global_timer_ns();
-                } else if ((it & 63u) == 63u && global_timer_ns() - t0 > kCWaitNs) {
+                    t_prog = global_timer_ns();
+                } else if ((it & 63u) == 63u && global_timer_ns() - t_prog > kCWaitNs) {
                     ok = false;
                     break;
                 }
@@ -269,24 +273,11 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     } else {
         // ---- softmax and output: row r, half h of the keys and of d
         const int pos = posb + (row_ok ? t : 0);   // row r attends keys 0 .. pos
-        float acc[HD];
-#pragma unroll
-        for (int c = 0; c < HD; ++c) acc[c] = 0.f;
-        float m_run = -INFINITY, l_run = 0.f, alpha_prev = 1.f;
-        // acc = acc alpha + this half of the P V tile in TMEM
-        auto add_o = [&](float alpha) {
-#pragma unroll
-            for (int c0 = 0; c0 < HD; c0 += 32) {
-                uint32_t o[32];
-                tmem_ld32(lane_base + kCOcol + (uint32_t)(h * HD + c0), o);
-                tmem_wait_ld();
-#pragma unroll
-                for (int c = 0; c < 32; ++c) acc[c0 + c] = fmaf(acc[c0 + c], alpha, __uint_as_float(o[c]));
-            }
-        };
+        const uint32_t ocol = lane_base + kCOcol + (uint32_t)(h * HD);
+        float m_run = -INFINITY, l_run = 0.f;
         // a wait's result is made warp-uniform (the TMEM accesses are
         // .aligned); after a timeout the warp does no more TMEM or shared-
-        // memory work but still takes the named barrier once per tile
+        // memory work but still takes its pair barrier once per tile
         auto wait_warp = [&](uint32_t bar, uint32_t parity) {
             return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity, kCWaitNs)) != 0;
         };
@@ -296,28 +287,65 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
             tmem_fence_after();
             const uint32_t scol = lane_base + (uint32_t)((j & 1) * kChunkKeys + 64 * h);
             const int lim = pos - (j * kChunkKeys + 64 * h);   // keys c <= lim of this half are attended
-            // the max of this half of the row's S (read again for P below:
-            // TMEM reads are cheap, registers are not); masked keys are -inf
-            // (the select ignores what unloaded rows hold)
+            // no key of this half is masked for any row of the warp (every
+            // tile but the last one or two): no selects
+            const bool whole = __all_sync(0xffffffffu, lim >= 63) != 0;
+            // the max of this half of the row's S; masked keys are -inf (the
+            // select ignores what unloaded rows hold)
             float mx = -INFINITY;
             if (ok) {
+                uint32_t sa[32], sb[32];
+                tmem_ld32(scol, sa);
+                tmem_ld32(scol + 32u, sb);
+                tmem_wait_ld();
+                if (whole) {
 #pragma unroll
-                for (int c0 = 0; c0 < 64; c0 += 32) {
-                    uint32_t sv[32];
-                    tmem_ld32(scol + (uint32_t)c0, sv);
-                    tmem_wait_ld();
+                    for (int c = 0; c < 32; ++c) mx = fmaxf(mx, fmaxf(__uint_as_float(sa[c]), __uint_as_float(sb[c])));
+                } else {
 #pragma unroll
-                    for (int c = 0; c < 32; ++c)
-                        if (c0 + c <= lim) mx = fmaxf(mx, __uint_as_float(sv[c]));
+                    for (int c = 0; c < 32; ++c) {
+                        if (c <= lim) mx = fmaxf(mx, __uint_as_float(sa[c]));
+                        if (c + 32 <= lim) mx = fmaxf(mx, __uint_as_float(sb[c]));
+                    }
                 }
             }
             mx *= p.scale_log2;   // scale_log2 > 0: the max commutes with it
+            // the two warps of this lane quarter (both halves of the rows) swap maxima
             s_mx[j & 1][h][r] = mx;
-            asm volatile("bar.sync 1, %0;" ::"n"(32 * kCSoftWarps) : "memory");
+            asm volatile("bar.sync %0, 64;" ::"r"(1 + quarter) : "memory");
             mx = fmaxf(mx, s_mx[j & 1][h ^ 1][r]);
             if (!ok) continue;
-            const float m_new = fmaxf(m_run, mx);   // finite: tile 0 holds key 0 for every row
-            const float alpha = ex2(m_run - m_new);
+            // The reference max moves only when a row's max passes it by more
+            // than 2^8 (P stays <= 2^8: exact in the sums, fine for bf16);
+            // then O (this half of d) and l are rescaled in place, once the
+            // P V already issued has landed.  Both warps of the quarter see
+            // the same maxima, so they take the same decision.
+            if (j == 0) {
+                m_run = mx;   // finite: tile 0 holds key 0 for every row
+            } else if (__any_sync(0xffffffffu, mx > m_run + 8.f)) {
+                const float m_new = fmaxf(m_run, mx);
+                const float alpha = ex2(m_run - m_new);
+                // completions of the P V barrier here are j - 1 or j (S_j's
+                // commit covered P V of tile j - 2), so the parity of j - 1
+                // names the one this waits for
+                ok = wait_warp(ofull, (uint32_t)((j - 1) & 1));
+                if (!ok) continue;
+                tmem_fence_after();
+#pragma unroll
+                for (int c0 = 0; c0 < HD; c0 += 32) {
+                    uint32_t o[32];
+                    tmem_ld32(ocol + (uint32_t)c0, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+                    tmem_st8(ocol + (uint32_t)c0, *reinterpret_cast<const uint32_t(*)[8]>(&o[0]));
+                    tmem_st8(ocol + (uint32_t)c0 + 8u, *reinterpret_cast<const uint32_t(*)[8]>(&o[8]));
+                    tmem_st8(ocol + (uint32_t)c0 + 16u, *reinterpret_cast<const uint32_t(*)[8]>(&o[16]));
+                    tmem_st8(ocol + (uint32_t)c0 + 24u, *reinterpret_cast<const uint32_t(*)[8]>(&o[24]));
+                }
+                l_run *= alpha;
+                m_run = m_new;
+            }
             // P = 2^(s scale - m) as P_hi + P_lo over this half's S columns,
             // 32 keys per pass over the 32 columns that pass has just read:
             // keys c0 + 2i, + 1 in column c0 + i (P_hi) and c0 + 16 + i (P_lo)
@@ -333,30 +361,22 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
 #pragma unroll
                     for (int k2 = 0; k2 < 8; ++k2) {
                         const int i = 8 * k8 + k2, c = c0 + 2 * i;
-                        const float p0 = (c <= lim) ? ex2(__uint_as_float(sv[2 * i]) * p.scale_log2 - m_new) : 0.f;
-                        const float p1 =
-                            (c + 1 <= lim) ? ex2(__uint_as_float(sv[2 * i + 1]) * p.scale_log2 - m_new) : 0.f;
+                        float p0 = ex2(__uint_as_float(sv[2 * i]) * p.scale_log2 - m_run);
+                        float p1 = ex2(__uint_as_float(sv[2 * i + 1]) * p.scale_log2 - m_run);
+                        if (!whole) {
+                            p0 = c <= lim ? p0 : 0.f;
+                            p1 = c + 1 <= lim ? p1 : 0.f;
+                        }
                         whi[k2] = pack_bf16(p0, p1);
-                        const float h0 = bf16_lo(whi[k2]), h1 = bf16_hi(whi[k2]);
-                        wlo[k2] = pack_bf16(p0 - h0, p1 - h1);   // exact differences, rounded once
-                        psum += (h0 + bf16_lo(wlo[k2])) + (h1 + bf16_hi(wlo[k2]));
+                        wlo[k2] = pack_bf16(p0 - bf16_lo(whi[k2]), p1 - bf16_hi(whi[k2]));   // exact differences
+                        psum += p0 + p1;   // P_hi + P_lo equals p to about 2^-17
                     }
                     tmem_st8(scol + (uint32_t)(c0 + 8 * k8), whi);
                     tmem_st8(scol + (uint32_t)(c0 + 16 + 8 * k8), wlo);
                 }
             }
             tmem_wait_st();
-            l_run = l_run * alpha + psum;
-            m_run = m_new;
-            // the previous tile's P V has landed: fold it in (the P V of this
-            // tile overwrites it once P is released below)
-            if (j > 0) {
-                ok = wait_warp(ofull, (uint32_t)((j - 1) & 1));
-                if (!ok) continue;
-                tmem_fence_after();
-                add_o(alpha_prev);
-            }
-            alpha_prev = alpha;
+            l_run += psum;
             if ((j + 1) * kChunkKeys > n_keys) {
                 // the last tile: V rows of keys >= n_keys hold unloaded or
                 // foreign data; zero them so that 0 x V stays 0, after the
@@ -371,37 +391,44 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
                 }
                 fence_proxy_async_smem();   // the zeroed V rows are read by the async proxy
             }
-            tmem_fence_before();   // P written, the P V tile read, before the MMA goes on
+            tmem_fence_before();   // P and any rescaled O written before the MMA goes on
             __syncwarp();
             if (lane == 0) mbar_arrive(pfull);
         }
-        if (ok) {
-            ok = wait_warp(ofull, (uint32_t)((NT - 1) & 1));
-            if (ok) {
-                tmem_fence_after();
-                add_o(alpha_prev);
-            }
-        }
+        // the last P V (its own barrier: the P V barrier may be two phases on)
+        if (ok) ok = wait_warp(smem_u32(&s_ofin), 0u);
         if (!ok) s_fail = 1;
         s_l[h][r] = l_run;
-        tmem_fence_before();
-        __syncthreads();   // (A) every TMEM access done; s_l, s_bad and s_fail settled
+        tmem_fence_after();
+        __syncthreads();   // (A) s_l, s_bad and s_fail settled
         const bool zero = s_bad != 0 || s_fail != 0;
-        if (row_ok) {
-            const float inv = 1.f / (l_run + s_l[h ^ 1][r]);
-            uint4* dst = reinterpret_cast<uint4*>(out_row(t, g) + h * HD);
+        const float inv = 1.f / (l_run + s_l[h ^ 1][r]);
+        uint4* dst = reinterpret_cast<uint4*>(out_row(t, g) + h * HD);
 #pragma unroll
-            for (int c = 0; c < HD / 8; ++c)
-                dst[c] = zero ? make_uint4(0u, 0u, 0u, 0u)
-                              : make_uint4(pack_bf16(acc[8 * c] * inv, acc[8 * c + 1] * inv),
-                                           pack_bf16(acc[8 * c + 2] * inv, acc[8 * c + 3] * inv),
-                                           pack_bf16(acc[8 * c + 4] * inv, acc[8 * c + 5] * inv),
-                                           pack_bf16(acc[8 * c + 6] * inv, acc[8 * c + 7] * inv));
+        for (int c0 = 0; c0 < HD; c0 += 32) {
+            uint32_t o[32];
+            if (!zero) {
+                tmem_ld32(ocol + (uint32_t)c0, o);
+                tmem_wait_ld();
+            }
+#pragma unroll
+            for (int c = 0; c < 32; c += 8) {
+                const float* f = reinterpret_cast<const float*>(&o[c]);
+                if (row_ok)
+                    dst[(c0 + c) / 8] = zero ? make_uint4(0u, 0u, 0u, 0u)
+                                             : make_uint4(pack_bf16(f[0] * inv, f[1] * inv),
+                                                          pack_bf16(f[2] * inv, f[3] * inv),
+                                                          pack_bf16(f[4] * inv, f[5] * inv),
+                                                          pack_bf16(f[6] * inv, f[7] * inv));
+            }
         }
+        tmem_fence_before();
+        __syncthreads();   // (B) every TMEM read done: the allocation may go
         return;
     }
-    // warps 0 and 1 (all lanes) meet the softmax warps at (A)
+    // warps 0 and 1 (all lanes) meet the softmax warps at (A) and (B)
     __syncwarp();
+    __syncthreads();
     tmem_fence_before();
     __syncthreads();
     if (warp == 0) {
