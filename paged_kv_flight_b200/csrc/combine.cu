@@ -86,7 +86,10 @@ __global__ void __launch_bounds__(kCombineThreads, 2) combine_kernel(const AttnP
     const int U0 = sp.unit_of(ts), U1 = sp.unit_of(ts + nt - 1);
     if (U0 == U1) return;
     const int G = p.G, R = G * p.q_len;            // partial rows: new token t, head h at row t G + h
-    const int k = U1 - U0 + 1, RD4 = R * D / 4;
+    // rows that hold partials: a virtual request of e.z < q_len tokens
+    // leaves only its G e.z rows (the rest of its slot is stale)
+    const int Rv = p.vmap ? G * min(max(__ldg(&p.vmap[b].z), 0), p.q_len) : R;
+    const int k = U1 - U0 + 1, RD4 = Rv * D / 4;
     const int side0 = sp.ustart(U0) < ts ? 1 : 0;   // slot side of the first unit
     const int kb = min(k, kCombineBlock);              // the dynamic shared memory holds kb contributors
     const int nblk = (k + kCombineBlock - 1) / kCombineBlock;
@@ -102,11 +105,11 @@ __global__ void __launch_bounds__(kCombineThreads, 2) combine_kernel(const AttnP
         for (int i = tid; i < n; i += kCombineThreads)
             s_slot[i] = 2 * (U0 + i0 + i) + (i0 + i == 0 ? side0 : 0);
         __syncthreads();
-        for (int e = tid; e < n * R; e += kCombineThreads) {
-            const int i = e / R, rr = e - i * R;
+        for (int e = tid; e < n * Rv; e += kCombineThreads) {
+            const int i = e / Rv, rr = e - i * Rv;
             const float2 ml = __ldg(reinterpret_cast<const float2*>(p.part_ml + ((size_t)s_slot[i] * R + rr) * 2));
-            s_mv[e] = ml.x;
-            s_lv[e] = ml.y;
+            s_mv[i * R + rr] = ml.x;
+            s_lv[i * R + rr] = ml.y;
         }
         __syncthreads();
         return n;
@@ -127,7 +130,7 @@ __global__ void __launch_bounds__(kCombineThreads, 2) combine_kernel(const AttnP
 #pragma unroll
         for (int j = 0; j < RPW; ++j) {
             const int row = warp + kCombineWarps * j;
-            if (row < R) {
+            if (row < Rv) {
                 float m = -INFINITY;
                 for (int i = lane; i < n; i += 32) m = fmaxf(m, s_mv[i * R + row]);
 #pragma unroll
@@ -146,7 +149,7 @@ __global__ void __launch_bounds__(kCombineThreads, 2) combine_kernel(const AttnP
 #pragma unroll
     for (int j = 0; j < RPW; ++j) {
         const int row = warp + kCombineWarps * j;
-        if (row < R && lane == 0) {
+        if (row < Rv && lane == 0) {
             s_m[row] = (Mg[j] == -INFINITY) ? 0.f : Mg[j];
             s_l[row] = Lg[j];
         }
@@ -163,9 +166,9 @@ __global__ void __launch_bounds__(kCombineThreads, 2) combine_kernel(const AttnP
             __syncthreads();
             n = stage(blk);
         }
-        for (int e = tid; e < n * R; e += kCombineThreads) {
-            const int rr = e % R;
-            s_mv[e] = ex2(s_mv[e] - s_m[rr]) / s_l[rr];   // now the weight
+        for (int e = tid; e < n * Rv; e += kCombineThreads) {
+            const int i = e / Rv, rr = e - i * Rv;
+            s_mv[i * R + rr] = ex2(s_mv[i * R + rr] - s_m[rr]) / s_l[rr];   // now the weight
         }
         __syncthreads();
 #pragma unroll 2
