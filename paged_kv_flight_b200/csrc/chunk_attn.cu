@@ -1,6 +1,6 @@
 // chunk_attn.cu -- attention of the prefill chunks of a varlen call on the
-// Blackwell tensor cores: S and each tile's P V in tensor memory (tcgen05),
-// K / V pages by TMA, P staged through shared memory.
+// Blackwell tensor cores: Q, S, P and O in tensor memory (tcgen05), K / V
+// pages by TMA into shared memory.
 //
 // "Scaling TensorRT-LLM: Kernel Fusion and Inflight Batching in Production",
 // section "What the Scheduler Actually Does" (chunked prefill mixed with
@@ -13,9 +13,9 @@
 // Work item: a block of up to 128 / G new tokens of one request and one kv
 // head.  Its 128 query rows r = t G + g (token t of the block, head g of the
 // group) are the M = 128 rows of both MMAs, so the block reads its request's
-// cache once for all of them.  Q, S, P and the P V tile live in tensor
-// memory; shared memory holds only a ring of K / V tiles (three stages of 128
-// keys, as TMA lands them with the 128-byte swizzle).  Per tile j:
+// cache once for all of them.  Q, S, P and O live in tensor memory; shared
+// memory holds only a ring of K / V tiles (three stages of 128 keys, as TMA
+// lands them with the 128-byte swizzle).  Per tile j:
 //   S_j = Q K^T     tcgen05, A = Q from TMEM, B = K (K-major); M 128, N 128
 //                   keys, K d; fp32 into TMEM buffer j % 2
 //   softmax         eight warps, two per TMEM lane quarter, one per half of the
@@ -46,8 +46,8 @@ using namespace dev;
 constexpr int kCStages = 3;
 constexpr int kCSoftWarps = 8;
 constexpr int kCThreads = 64 + 32 * kCSoftWarps;
-// tensor memory: S / P buffers (2 x 128 columns), the P V tile (d), Q (d / 2:
-// two bf16 per column)
+// tensor memory: S / P buffers (2 x 128 columns), O (d), Q (d / 2: two bf16
+// per column)
 constexpr uint32_t kCCols = 512;
 constexpr uint32_t kCOcol = 2 * kChunkKeys;
 constexpr uint32_t kCQcol = kCOcol + 128;
