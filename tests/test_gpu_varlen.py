@@ -166,6 +166,39 @@ def test_varlen_every_request_on_prefill_blocks(pkv):
     assert finite and mx <= _gpu.TOL_BF16["max"] and mean <= _gpu.TOL_BF16["mean"], (mx, mean)
 
 
+def test_varlen_prefill_blocks_rescale_when_later_keys_dominate(pkv):
+    """Keys from position 256 on are scaled by 4 (exact in bf16), so a row's
+    max grows by far more than 2^8 after the first 128-key tiles: the
+    prefill blocks' reference max moves and O and l are rescaled in tensor
+    memory.  Against the oracle on the same inputs.  The softmax is then
+    sharp and an output is close to one V row, so V is scaled by 1/4 too:
+    outputs stay below about 1.2, where bf16 rounding (half an ulp, <= 2^-8)
+    leaves room inside the 1e-2 bar."""
+    Hq, Hkv, d, P = 32, 8, 128, 16
+    lengths, q_lens = [600, 300, 1000], [40, 20, 1]
+    w = workloads.build("rescale", Hq, Hkv, d, P, False, 5e5, lengths, 57, device="cpu", q_len=max(q_lens))
+    h = varlen_host(w, q_lens)
+    kp = h["k_pool"]
+    for b, L in enumerate(lengths):
+        for pos in range(256, L):
+            page, slot = int(h["block_tables"][b][pos // P]), pos % P
+            f = (kp[page, :, slot, :].astype(np.uint16).astype(np.uint32) << 16).view(np.float32) * np.float32(4)
+            kp[page, :, slot, :] = (f.view(np.uint32) >> 16).astype(kp.dtype)
+    for key in ("v_pool", "v_new"):
+        a = h[key]
+        f = (a.astype(np.uint16).astype(np.uint32) << 16).view(np.float32) * np.float32(0.25)
+        h[key] = (f.view(np.uint32) >> 16).astype(a.dtype)
+    _, ref = _oracle(w, h)
+    ctx = _gpu.make_ctx(pkv, w, max_batch=8)
+    try:
+        out = _step(pkv, ctx, _device(h))
+        assert pkv.pkv_check_device_error(ctx)[0] == pkv.PKV_OK
+    finally:
+        pkv.pkv_destroy(ctx)
+    mx, mean, finite = _gpu.errors(out, ref)
+    assert finite and mx <= _gpu.TOL_BF16["max"] and mean <= _gpu.TOL_BF16["mean"], (mx, mean)
+
+
 def test_prefill_rows_setting_range(pkv):
     w, _, _ = _setup(CASES[0])
     ctx = _gpu.make_ctx(pkv, w, max_batch=8)
