@@ -86,6 +86,10 @@ chunk_attn_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     __shared__ float s_l[2][kChunkRows];       // [half][row] running sums
 
     const int item = blockIdx.y;
+    // the host sizes the grid from the call's token counts; a plan with more
+    // blocks than that would leave rows unwritten, so it is reported
+    if (blockIdx.x == 0 && item == 0 && threadIdx.x == 0 && __ldg(p.ccount) > (int)gridDim.y)
+        atomicOr(p.err, kErrLength);
     if (item >= __ldg(p.ccount)) return;       // CTA-uniform, before any barrier
     const int kvh = blockIdx.x, G = p.G;
     const int4 e = p.cmap[item];
