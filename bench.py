@@ -55,6 +55,10 @@ KERNEL_SOURCES = {
     "qkv": ("paged_kv_flight_b200/csrc/qkv_rope_append.cu", "paged_kv_flight_b200/csrc/pkv_device.cuh",
             "paged_kv_flight_b200/csrc/umma.cuh", "paged_kv_flight_b200/csrc/pkv_internal.h"),
 }
+# the mixed leg's attention: the several-new-tokens kernels, the combine and
+# the prefill blocks on tcgen05 (its traffic line is the three kernels' sum)
+KERNEL_SOURCES["mixed"] = KERNEL_SOURCES["attn"] + ("paged_kv_flight_b200/csrc/chunk_attn.cu",
+                                                    "paged_kv_flight_b200/csrc/umma.cuh")
 
 
 # ---------------------------------------------------------------- accounting
@@ -128,7 +132,7 @@ def recorded_traffic(workload: str):
     """DRAM bytes per launch of the workload's dominant kernel from a
     committed ncu summary, if it was taken on that kernel's current sources;
     otherwise None."""
-    sha = source_sha("qkv" if workload == "qkv8b" else "attn")
+    sha = source_sha({"qkv8b": "qkv", "mixed": "mixed"}.get(workload, "attn"))
     pat = re.compile(r"traffic-per-launch:\s+(\S+)\s+(\d+)\s+src=([0-9a-f]+)")
     pdir = os.path.join(ROOT, "profiles")
     if not os.path.isdir(pdir):
